@@ -1,0 +1,178 @@
+/*
+ * gdr.h -- C ABI of libgdr: the generalized delta-rule matrix memory on B200.
+ *
+ * The recurrence (spec column form; the state S is d_v x d_k):
+ *
+ *     e_t = S_{t-1} u_t
+ *     S_t = S_{t-1} Diag(w_t) - e_t z_t^T + v_t k_t^T  = S_{t-1}(Diag(w_t) - u_t z_t^T) + v_t k_t^T
+ *     o_t = S_t q_t                                      (readout after the update)
+ *
+ * Sources:
+ *  - "Exponential gates and matrix memory: xLSTM and RWKV-7", section 13.3
+ *    (the generalized delta rule S_t = S_{t-1}(Diag(w_t) - c_t a_t a_t^T) + u_t b_t^T,
+ *    retrieval by S q with the transition acting on the right), section 13.1
+ *    (the generalized transition Diag(w) - c a a^T with a unit a).
+ *  - "Muir: Linear Attention with Sensitivity-Allocated Gating and Matched-Filter
+ *    Readout", section 2.1 eq. (1) (GDN-2 update with channel-wise decay alpha,
+ *    erase gate b, write gate w) and section 4.2 eq. (8) (Muir readout with the
+ *    gain-modulated query); section 2.2 and section 4.2 eq. (10) give the chunkwise
+ *    form that gdr_forward_chunked evaluates.
+ *
+ * Storage orientation.  Every state buffer is stored as [B][H][d_k][d_v] fp32,
+ * row-major: element (j, c) is key channel j, value channel c.  That is the Muir
+ * page's orientation (S in R^{d_k x d_v}, row vectors, o = q S), i.e. the transpose
+ * of the column form above.  Both describe the same numbers.
+ *
+ * Forms (how u_t and z_t are built from the arguments e1, e2; w_t = exp(log_w_t)):
+ *   GDR_FORM_GENERAL : e1 = u [.., d_k], e2 = z [.., d_k]; write (v, k).
+ *   GDR_FORM_GDN2    : e1 = b erase gate [.., d_k]; e2 = write gate wg [.., d_v] or NULL (= 1).
+ *                      u = alpha (.) b (.) k, z = k; written value wg (.) v with key k.
+ *                      (Muir eq. (1)/(8) transposed: the erase acts on the decayed state
+ *                      Diag(alpha) S_{t-1}, which is why alpha is folded into u.)
+ *                      For Muir pass q_hat = gamma (.) q as q.
+ *   GDR_FORM_RWKV7   : e1 = a unit removal direction [.., d_k]; e2 = c removal coefficient,
+ *                      one scalar per (b, t, h), i.e. [B][T][H]; u = c a, z = a; write (v, k).
+ *                      (the chapter's u_t b_t^T write is passed here as v = u_t, k = b_t.)
+ *   GDR_FORM_GLA     : u = 0 (gated linear attention); e1 = e2 = NULL.
+ *
+ * Memory and ownership.  The caller owns every buffer; pointers are device
+ * pointers unless stated otherwise.  libgdr allocates no device memory, keeps no
+ * global state between calls, and never synchronizes the stream except where a
+ * function says so.  Everything is enqueued asynchronously on the given stream
+ * (a cudaStream_t passed as void*, NULL = legacy default stream).
+ *
+ * Errors.  Every function returns a gdr_status.  Invalid arguments are rejected on
+ * the host before any launch.  Launch failures come back as GDR_ERR_CUDA.  Faults
+ * that happen later on the device surface at the caller's next synchronization.
+ * Kernels that wait on an mbarrier bound each wait; a wait that runs out writes
+ * GDR_ERR_TIMEOUT into the caller's workspace status word, which
+ * gdr_read_status() returns.  No function aborts, exits or traps.
+ */
+#ifndef GDR_H_
+#define GDR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GDR_OK = 0,
+  GDR_ERR_INVALID_ARG = 1,   /* null pointer where one is required, negative size, bad enum */
+  GDR_ERR_UNSUPPORTED = 2,   /* a size or form this build has no kernel for (see each call) */
+  GDR_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned                            */
+  GDR_ERR_CUDA = 4,          /* a CUDA runtime call or a launch failed                       */
+  GDR_ERR_DEVICE_CHECK = 5,  /* a device-side argument check failed (read via gdr_read_status) */
+  GDR_ERR_TIMEOUT = 6,       /* a bounded device wait ran out (read via gdr_read_status)       */
+  GDR_ERR_WORKSPACE = 7      /* workspace missing or smaller than gdr_forward_workspace_size   */
+} gdr_status;
+
+typedef enum { GDR_F32 = 0, GDR_BF16 = 1 } gdr_dtype;
+
+typedef enum {
+  GDR_FORM_GENERAL = 0,
+  GDR_FORM_GDN2 = 1,
+  GDR_FORM_RWKV7 = 2,
+  GDR_FORM_GLA = 3
+} gdr_form;
+
+/* Kernel selection for gdr_forward_chunked. */
+typedef enum {
+  GDR_ALGO_AUTO = 0,   /* tensor-core kernel where it applies, else the fp32 kernel        */
+  GDR_ALGO_FP32 = 1,   /* fp32 CUDA-core kernel: every product in fp32 (all forms, all dtypes) */
+  GDR_ALGO_TC = 2      /* tcgen05/TMEM kernel: bf16 operands, fp32 accumulate and state;
+                          GDR_ERR_UNSUPPORTED where it does not apply                       */
+} gdr_algo;
+
+/*
+ * Arguments of gdr_forward_chunked.  Shapes are token-major and contiguous:
+ *   q, k, log_w, and e1 for GENERAL/GDN2/RWKV7 : [B][T][H][dk]
+ *   v, o, and e2 for GDN2                      : [B][T][H][dv]
+ *   e2 for GENERAL                             : [B][T][H][dk]
+ *   e2 for RWKV7                               : [B][T][H]
+ *   S0, S_T                                    : [B][H][dk][dv]
+ * q, k, v, e1, e2 have element type `dtype`; log_w, S0, S_T, o are fp32.
+ */
+typedef struct {
+  gdr_form form;
+  gdr_dtype dtype;
+  int B, H, T, dk, dv;  /* B, H, T >= 0 (zero sizes are a no-op apart from S_T = S0);
+                           dk, dv in {16, 32, 64, 128}                                  */
+  int chunk;            /* chunk length C of the chunkwise form: 16, 32, 64 or 128.
+                           T need not be a multiple of C (the last chunk is partial).   */
+  gdr_algo algo;
+  const void *q, *k, *v;
+  const float *log_w;   /* log of the decay, must be <= 0 (decay w = exp(log_w) in (0,1]) */
+  const void *e1, *e2;  /* per form, above                                             */
+  const float *S0;      /* initial state, or NULL for S0 = 0                           */
+  float *o;             /* outputs o_t, required                                       */
+  float *S_T;           /* final state, or NULL; may alias S0 (read before written)    */
+  void *workspace;      /* device scratch of gdr_forward_workspace_size bytes, 256-B aligned */
+  size_t workspace_bytes;
+} gdr_fwd_args;
+
+/* Workspace bytes gdr_forward_chunked needs for these arguments (host-only, no CUDA call). */
+gdr_status gdr_forward_workspace_size(const gdr_fwd_args *args, size_t *bytes);
+
+/*
+ * Chunkwise-parallel forward over whole sequences: for every (b, h) runs the
+ * recurrence over t = 1..T from S0 and writes every o_t and, if S_T != NULL, the
+ * final state.  Chunkwise algorithm: "Muir ...", section 2.2 (effective write,
+ * the unit lower-triangular system T V~ = V^ - K^_pi S0, S_C and O as matrix
+ * products) and section 4.2 eq. (10) (outputs and end state affine in S0),
+ * generalized to a separate erase key z (e_t and v_t carried as two write streams).
+ * Cumulative decays are formed in log space and only exponentiated at non-positive
+ * arguments (section 4.2, boundary-pivoted splitting), so nothing overflows.
+ */
+gdr_status gdr_forward_chunked(const gdr_fwd_args *args, void *stream);
+
+/*
+ * Arguments of gdr_decode_step: one token for each (b, h).
+ *   q, k, log_w, e1 (GENERAL/GDN2/RWKV7) : [B][H][dk]
+ *   v, o, e2 (GDN2)                      : [B][H][dv]
+ *   e2 (GENERAL)                         : [B][H][dk]
+ *   e2 (RWKV7)                           : [B][H]
+ *   S                                    : [B][H][dk][dv] fp32, updated in place
+ */
+typedef struct {
+  gdr_form form;
+  gdr_dtype dtype;
+  int B, H, dk, dv;     /* dk, dv in {16, 32, 64, 128}; B, H >= 0 */
+  const void *q, *k, *v;
+  const float *log_w;
+  const void *e1, *e2;
+  float *S;
+  float *o;             /* [B][H][dv] fp32, required */
+} gdr_step_args;
+
+/*
+ * One recurrent step (decode).  "Muir ...", section 2.1 eq. (1) and section 4.2
+ * eq. (8); "Exponential gates and matrix memory ...", section 13.3.  Reads S once:
+ * e = S u and S (w (.) q) come from the old state in the same pass, then
+ * o = S(w (.) q) - e <z, q> + v <k, q> and S <- S Diag(w) - e z^T + v k^T in place.
+ */
+gdr_status gdr_decode_step(const gdr_step_args *args, void *stream);
+
+/* S[B][H][dk][dv] = src (device pointer, same layout) or 0 when src == NULL. */
+gdr_status gdr_state_init(float *S, int B, int H, int dk, int dv, const float *src, void *stream);
+
+/*
+ * Synchronizes `stream`, then reads and clears the status word the kernels keep
+ * at the start of `workspace` (GDR_OK if no device check or bounded wait failed).
+ * The only call here that synchronizes.
+ */
+gdr_status gdr_read_status(void *workspace, void *stream, gdr_status *device_status);
+
+/* Static text for a status code; never NULL. */
+const char *gdr_status_string(gdr_status s);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int gdr_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR_H_ */

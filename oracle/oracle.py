@@ -1,0 +1,111 @@
+"""ctypes front end of the fp64 oracle in ``gdr_oracle.c``.
+
+TEST INFRASTRUCTURE (see the package docstring).  Everything here is argument
+marshalling: the recurrence itself is the C loop in ``gdr_oracle.c``, which
+follows "Exponential gates and matrix memory: xLSTM and RWKV-7", section 13.3,
+and "Muir: Linear Attention with Sensitivity-Allocated Gating and
+Matched-Filter Readout", section 2.1 eq. (1) / section 4.2 eq. (8).
+
+Inputs are float64 numpy arrays holding the values the GPU receives (bf16 or
+fp32 values widened exactly to float64); ``log_w`` likewise (fp32 widened).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+FORMS = {"general": 0, "gdn2": 1, "rwkv7": 2, "gla": 3}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _LIB
+
+
+def build(force: bool = False) -> str:
+    """Compiles ``gdr_oracle.c`` with gcc and OpenMP into ``liboracle.so``."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def load_library(path: str):
+    """Opens a compiled oracle (the real one, or a test's planted-mistake copy)."""
+    lib = ctypes.CDLL(path)
+    dp = ctypes.POINTER(ctypes.c_double)
+    lib.oracle_forward.restype = ctypes.c_int
+    lib.oracle_forward.argtypes = [ctypes.c_int] * 6 + [dp] * 9 + [ctypes.c_int]
+    lib.oracle_max_threads.restype = ctypes.c_int
+    return lib
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            _lib = load_library(_LIB)
+    return _lib
+
+
+def max_threads() -> int:
+    return int(_load().oracle_max_threads())
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _f64(a):
+    if a is None:
+        return None
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def forward(form: str, q, k, v, log_w, e1=None, e2=None, S0=None, n_threads: int = 0,
+            lib=None):
+    """Token-by-token recurrence over [B, T, H, d] inputs.
+
+    Returns ``(o, S_T)``: o is [B, T, H, dv]; S_T is [B, H, dk, dv] (key channel
+    first, the library's storage layout).  ``lib`` selects another compiled copy
+    (tests only); default is the oracle built from ``gdr_oracle.c``.
+    """
+    lib = _load() if lib is None else lib
+    q, k, v, log_w, e1, e2, S0 = map(_f64, (q, k, v, log_w, e1, e2, S0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, T, H, dk) and log_w.shape == (B, T, H, dk)
+    assert v.shape == (B, T, H, dv)
+    if S0 is not None:
+        assert S0.shape == (B, H, dk, dv)
+    o = np.zeros((B, T, H, dv), dtype=np.float64)
+    S_T = np.zeros((B, H, dk, dv), dtype=np.float64)
+    rc = lib.oracle_forward(FORMS[form], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                            _ptr(log_w), _ptr(e1), _ptr(e2), _ptr(S0), _ptr(o), _ptr(S_T),
+                            int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_forward failed with code {rc}")
+    return o, S_T
+
+
+def decode_step(form: str, q, k, v, log_w, e1, e2, S, n_threads: int = 0):
+    """One token per (b, h): inputs [B, H, d], state [B, H, dk, dv].  Returns (o, S_new)."""
+    def tok(a):
+        return None if a is None else _f64(a)[:, None]
+    o, S_new = forward(form, tok(q), tok(k), tok(v), tok(log_w), tok(e1), tok(e2), S,
+                       n_threads=n_threads)
+    return o[:, 0], S_new
