@@ -1,0 +1,142 @@
+// gdr_api.cu -- the extern "C" entry points of libgdr: argument validation,
+// kernel selection and launch.  Declarations and the contract: include/gdr.h.
+#include <cstdint>
+#include <cstring>
+
+#include "gdr_internal.cuh"
+
+namespace {
+
+bool dim_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64 || c == 128; }
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool form_ok(gdr_form f) { return f >= GDR_FORM_GENERAL && f <= GDR_FORM_GLA; }
+bool dtype_ok(gdr_dtype d) { return d == GDR_F32 || d == GDR_BF16; }
+
+// Which of e1 / e2 a form needs (e2 is optional for GDN-2: the write gate).
+bool needs_e1(gdr_form f) { return f != GDR_FORM_GLA; }
+bool needs_e2(gdr_form f) { return f == GDR_FORM_GENERAL || f == GDR_FORM_RWKV7; }
+
+gdr_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GDR_OK : GDR_ERR_CUDA; }
+
+// Common pointer checks of the token inputs.  `tokens` = B*T*H (or B*H).
+gdr_status check_token_ptrs(gdr_form form, size_t tokens, const void *q, const void *k,
+                            const void *v, const float *log_w, const void *e1, const void *e2,
+                            const float *o) {
+  if (tokens == 0) return GDR_OK;
+  if (!q || !k || !v || !log_w || !o) return GDR_ERR_INVALID_ARG;
+  if (needs_e1(form) && !e1) return GDR_ERR_INVALID_ARG;
+  if (needs_e2(form) && !e2) return GDR_ERR_INVALID_ARG;
+  const void *ptrs[] = {q, k, v, log_w, o, e1, e2};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return GDR_ERR_MISALIGNED;
+  return GDR_OK;
+}
+
+constexpr size_t kStatusBytes = 256;  // status word, padded to the workspace alignment
+
+}  // namespace
+
+extern "C" {
+
+const char *gdr_status_string(gdr_status s) {
+  switch (s) {
+    case GDR_OK: return "ok";
+    case GDR_ERR_INVALID_ARG: return "invalid argument";
+    case GDR_ERR_UNSUPPORTED: return "unsupported size or form";
+    case GDR_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case GDR_ERR_CUDA: return "CUDA runtime or launch error";
+    case GDR_ERR_DEVICE_CHECK: return "device-side check failed";
+    case GDR_ERR_TIMEOUT: return "bounded device wait ran out";
+    case GDR_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+int gdr_version(void) { return 100; }
+
+gdr_status gdr_forward_workspace_size(const gdr_fwd_args *a, size_t *bytes) {
+  if (!a || !bytes) return GDR_ERR_INVALID_ARG;
+  *bytes = kStatusBytes;
+  return GDR_OK;
+}
+
+gdr_status gdr_state_init(float *S, int B, int H, int dk, int dv, const float *src,
+                          void *stream) {
+  if (B < 0 || H < 0 || !dim_ok(dk) || !dim_ok(dv)) return GDR_ERR_INVALID_ARG;
+  const size_t n = (size_t)B * H * dk * dv;
+  if (n == 0) return GDR_OK;
+  if (!S) return GDR_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (src) {
+    if (src == S) return GDR_OK;
+    return cuda_status(cudaMemcpyAsync(S, src, n * sizeof(float), cudaMemcpyDeviceToDevice, st));
+  }
+  return cuda_status(cudaMemsetAsync(S, 0, n * sizeof(float), st));
+}
+
+gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
+  if (!a) return GDR_ERR_INVALID_ARG;
+  if (!form_ok(a->form) || !dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 0 || a->T < 0) return GDR_ERR_INVALID_ARG;
+  if (!dim_ok(a->dk) || !dim_ok(a->dv) || !chunk_ok(a->chunk)) return GDR_ERR_UNSUPPORTED;
+  if (a->algo < GDR_ALGO_AUTO || a->algo > GDR_ALGO_TC) return GDR_ERR_INVALID_ARG;
+  const size_t tokens = (size_t)a->B * a->T * a->H;
+  gdr_status st = check_token_ptrs(a->form, tokens, a->q, a->k, a->v, a->log_w, a->e1, a->e2,
+                                   a->o);
+  if (st != GDR_OK) return st;
+  if ((a->S0 && !aligned16(a->S0)) || (a->S_T && !aligned16(a->S_T))) return GDR_ERR_MISALIGNED;
+  if (a->workspace && (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
+    return GDR_ERR_MISALIGNED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  if (a->B == 0 || a->H == 0) return GDR_OK;
+  if (a->T == 0) {  // no tokens: S_T = S0
+    if (!a->S_T) return GDR_OK;
+    return gdr_state_init(a->S_T, a->B, a->H, a->dk, a->dv, a->S0, stream);
+  }
+
+  gdr::FwdParams p;
+  p.form = a->form;
+  p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv; p.chunk = a->chunk;
+  p.q = a->q; p.k = a->k; p.v = a->v; p.e1 = a->e1;
+  p.e2 = a->e2;
+  p.log_w = a->log_w;
+  p.S0 = a->S0;
+  p.o = a->o;
+  p.S_T = a->S_T;
+  p.status = static_cast<uint32_t *>(a->workspace);
+
+  if (a->algo == GDR_ALGO_TC) return GDR_ERR_UNSUPPORTED;
+  if (!gdr::forward_fp32_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
+  return cuda_status(gdr::launch_forward_fp32(p, a->dtype, s));
+}
+
+gdr_status gdr_decode_step(const gdr_step_args *a, void *stream) {
+  if (!a) return GDR_ERR_INVALID_ARG;
+  if (!form_ok(a->form) || !dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 0) return GDR_ERR_INVALID_ARG;
+  if (!dim_ok(a->dk) || !dim_ok(a->dv)) return GDR_ERR_UNSUPPORTED;
+  const size_t tokens = (size_t)a->B * a->H;
+  gdr_status st = check_token_ptrs(a->form, tokens, a->q, a->k, a->v, a->log_w, a->e1, a->e2,
+                                   a->o);
+  if (st != GDR_OK) return st;
+  if (tokens == 0) return GDR_OK;
+  if (!a->S) return GDR_ERR_INVALID_ARG;
+  if (!aligned16(a->S)) return GDR_ERR_MISALIGNED;
+  return cuda_status(gdr::launch_decode(*a, static_cast<cudaStream_t>(stream)));
+}
+
+gdr_status gdr_read_status(void *workspace, void *stream, gdr_status *device_status) {
+  if (!workspace || !device_status) return GDR_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return GDR_ERR_CUDA;
+  uint32_t word = 0;
+  if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return GDR_ERR_CUDA;
+  if (cudaMemset(workspace, 0, sizeof(word)) != cudaSuccess) return GDR_ERR_CUDA;
+  *device_status = static_cast<gdr_status>(word);
+  return GDR_OK;
+}
+
+}  // extern "C"

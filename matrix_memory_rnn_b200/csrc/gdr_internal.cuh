@@ -1,0 +1,67 @@
+// gdr_internal.cuh -- device helpers and launcher declarations shared by the
+// libgdr kernels (not part of the public ABI; see include/gdr.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "gdr.h"
+
+namespace gdr {
+
+// Widening loads of the two input element types.
+__device__ __forceinline__ float ld_in(const float *p, size_t i) { return __ldg(p + i); }
+__device__ __forceinline__ float ld_in(const __nv_bfloat16 *p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+
+// The form's erase vector u_j and erase key z_j for one token, from the raw
+// arguments (include/gdr.h): general u = e1, z = e2; GDN-2 u = alpha b k, z = k;
+// RWKV-7 u = c a, z = a; GLA u = z = 0.  `wj` is the decay exp(log_w_j).
+template <typename Tin>
+__device__ __forceinline__ void erase_pair(gdr_form form, const Tin *k, const Tin *e1,
+                                           const Tin *e2, size_t idx_k, size_t idx_s,
+                                           float wj, float &u, float &z) {
+  switch (form) {
+    case GDR_FORM_GENERAL:
+      u = ld_in(e1, idx_k);
+      z = ld_in(e2, idx_k);
+      break;
+    case GDR_FORM_GDN2: {
+      const float kj = ld_in(k, idx_k);
+      u = wj * ld_in(e1, idx_k) * kj;
+      z = kj;
+      break;
+    }
+    case GDR_FORM_RWKV7: {
+      const float a = ld_in(e1, idx_k);
+      u = ld_in(e2, idx_s) * a;
+      z = a;
+      break;
+    }
+    default:
+      u = 0.f;
+      z = 0.f;
+      break;
+  }
+}
+
+struct FwdParams {
+  gdr_form form;
+  int B, H, T, dk, dv, chunk;
+  const void *q, *k, *v, *e1, *e2;
+  const float *log_w;
+  const float *S0;
+  float *o;
+  float *S_T;
+  uint32_t *status;  // device status word (workspace), may be null
+};
+
+// Launchers (host).  Return cudaSuccess or the launch error.
+cudaError_t launch_decode(const gdr_step_args &a, cudaStream_t stream);
+cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_t stream);
+bool forward_fp32_supported(int dk, int dv);
+size_t forward_fp32_smem_bytes(int dk, int dv, int chunk);
+
+}  // namespace gdr

@@ -1,0 +1,257 @@
+"""Python binding of libgdr (include/gdr.h): argument marshalling only.
+
+Every function here validates tensor dtypes/devices, passes raw device pointers
+and the current CUDA stream to the C ABI, and raises ``GdrError`` on a non-OK
+status.  All arithmetic runs in libgdr's CUDA kernels; there is no fallback.
+If ``libgdr.so`` is missing and cannot be built, importing the library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgdr.so")
+
+FORMS = {"general": 0, "gdn2": 1, "rwkv7": 2, "gla": 3}
+DTYPES = {"f32": 0, "bf16": 1}
+ALGOS = {"auto": 0, "fp32": 1, "tc": 2}
+STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED",
+          3: "GDR_ERR_MISALIGNED", 4: "GDR_ERR_CUDA", 5: "GDR_ERR_DEVICE_CHECK",
+          6: "GDR_ERR_TIMEOUT", 7: "GDR_ERR_WORKSPACE"}
+
+_c_int, _vp, _fp = ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p
+
+
+class gdr_fwd_args(ctypes.Structure):
+    _fields_ = [("form", _c_int), ("dtype", _c_int), ("B", _c_int), ("H", _c_int),
+                ("T", _c_int), ("dk", _c_int), ("dv", _c_int), ("chunk", _c_int),
+                ("algo", _c_int), ("q", _vp), ("k", _vp), ("v", _vp), ("log_w", _fp),
+                ("e1", _vp), ("e2", _vp), ("S0", _fp), ("o", _fp), ("S_T", _fp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
+class gdr_step_args(ctypes.Structure):
+    _fields_ = [("form", _c_int), ("dtype", _c_int), ("B", _c_int), ("H", _c_int),
+                ("dk", _c_int), ("dv", _c_int), ("q", _vp), ("k", _vp), ("v", _vp),
+                ("log_w", _fp), ("e1", _vp), ("e2", _vp), ("S", _fp), ("o", _fp)]
+
+
+class GdrError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = int(code)
+        super().__init__(f"{fn} failed: {STATUS.get(self.code, self.code)}")
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                from . import build as _build   # nvcc is required; raises if absent
+                _build.build()
+            lib = ctypes.CDLL(LIB_PATH)
+            lib.gdr_forward_chunked.argtypes = [ctypes.POINTER(gdr_fwd_args), _vp]
+            lib.gdr_forward_workspace_size.argtypes = [ctypes.POINTER(gdr_fwd_args),
+                                                       ctypes.POINTER(ctypes.c_size_t)]
+            lib.gdr_decode_step.argtypes = [ctypes.POINTER(gdr_step_args), _vp]
+            lib.gdr_state_init.argtypes = [_fp, _c_int, _c_int, _c_int, _c_int, _fp, _vp]
+            lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
+            lib.gdr_status_string.restype = ctypes.c_char_p
+            lib.gdr_status_string.argtypes = [_c_int]
+            for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size", "gdr_decode_step",
+                       "gdr_state_init", "gdr_read_status", "gdr_version"):
+                getattr(lib, fn).restype = _c_int
+            _lib = lib
+    return _lib
+
+
+def library():
+    """The loaded ``ctypes.CDLL`` (loads it on first use)."""
+    return _load()
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise GdrError(fn, rc)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype, shape):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _dtype_of(q):
+    if q.dtype == torch.bfloat16:
+        return "bf16", torch.bfloat16
+    if q.dtype == torch.float32:
+        return "f32", torch.float32
+    raise ValueError(f"inputs must be bf16 or fp32, got {q.dtype}")
+
+
+def _e_shapes(form, lead, dk, dv):
+    if form == "general":
+        return lead + (dk,), lead + (dk,)
+    if form == "gdn2":
+        return lead + (dk,), lead + (dv,)
+    if form == "rwkv7":
+        return lead + (dk,), lead
+    return None, None
+
+
+def _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, workspace):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dname, tdt = _dtype_of(q)
+    _need(q, "q", tdt, (B, T, H, dk))
+    _need(k, "k", tdt, (B, T, H, dk))
+    _need(v, "v", tdt, (B, T, H, dv))
+    _need(log_w, "log_w", torch.float32, (B, T, H, dk))
+    s1, s2 = _e_shapes(form, (B, T, H), dk, dv)
+    if s1 is not None:
+        _need(e1, "e1", tdt, s1)
+    if e2 is not None or form in ("general", "rwkv7"):
+        _need(e2, "e2", tdt, s2)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv))
+    _need(o, "o", torch.float32, (B, T, H, dv))
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dk, dv))
+    a = gdr_fwd_args()
+    a.form, a.dtype, a.algo = FORMS[form], DTYPES[dname], ALGOS[algo]
+    a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, dv, chunk
+    a.q, a.k, a.v, a.log_w = _ptr(q), _ptr(k), _ptr(v), _ptr(log_w)
+    a.e1, a.e2, a.S0, a.o, a.S_T = _ptr(e1), _ptr(e2), _ptr(S0), _ptr(o), _ptr(S_T)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    return a
+
+
+def gdr_forward_workspace_size(form, q, k, v, log_w, e1=None, e2=None, chunk=64, algo="auto"):
+    """Bytes of device workspace ``gdr_forward_chunked`` needs for these inputs."""
+    B, T, H, dk = q.shape
+    a = gdr_fwd_args()
+    a.form, a.dtype, a.algo = FORMS[form], DTYPES[_dtype_of(q)[0]], ALGOS[algo]
+    a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, v.shape[-1], chunk
+    n = ctypes.c_size_t(0)
+    _check("gdr_forward_workspace_size",
+           _load().gdr_forward_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    return int(n.value)
+
+
+def new_workspace(nbytes, device):
+    """A zeroed, 256-byte aligned device workspace of at least ``nbytes`` bytes."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def gdr_forward_chunked(form, q, k, v, log_w, e1=None, e2=None, S0=None, *, chunk=64,
+                        algo="auto", o=None, S_T=None, want_state=True, workspace=None,
+                        stream=None):
+    """Chunkwise forward.  Tensors [B, T, H, d] (q, k, v, e1, e2 bf16 or fp32; log_w fp32).
+
+    Returns ``(o, S_T)`` with o [B, T, H, dv] fp32 and S_T [B, H, dk, dv] fp32
+    (None when ``want_state`` is False and no ``S_T`` buffer is given).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(gdr_forward_workspace_size(form, q, k, v, log_w, e1, e2,
+                                                             chunk, algo), q.device)
+    a = _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, workspace)
+    _check("gdr_forward_chunked", _load().gdr_forward_chunked(ctypes.byref(a), _stream(stream)))
+    return o, S_T
+
+
+def gdr_decode_step(form, q, k, v, log_w, e1, e2, S, *, o=None, stream=None):
+    """One token per (b, h): inputs [B, H, d]; S [B, H, dk, dv] fp32 updated in place.  Returns o."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dname, tdt = _dtype_of(q)
+    _need(q, "q", tdt, (B, H, dk))
+    _need(k, "k", tdt, (B, H, dk))
+    _need(v, "v", tdt, (B, H, dv))
+    _need(log_w, "log_w", torch.float32, (B, H, dk))
+    s1, s2 = _e_shapes(form, (B, H), dk, dv)
+    if s1 is not None:
+        _need(e1, "e1", tdt, s1)
+    if e2 is not None or form in ("general", "rwkv7"):
+        _need(e2, "e2", tdt, s2)
+    _need(S, "S", torch.float32, (B, H, dk, dv))
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=torch.float32, device=q.device)
+    _need(o, "o", torch.float32, (B, H, dv))
+    a = gdr_step_args()
+    a.form, a.dtype = FORMS[form], DTYPES[dname]
+    a.B, a.H, a.dk, a.dv = B, H, dk, dv
+    a.q, a.k, a.v, a.log_w = _ptr(q), _ptr(k), _ptr(v), _ptr(log_w)
+    a.e1, a.e2, a.S, a.o = _ptr(e1), _ptr(e2), _ptr(S), _ptr(o)
+    _check("gdr_decode_step", _load().gdr_decode_step(ctypes.byref(a), _stream(stream)))
+    return o
+
+
+def gdr_state_init(S, src=None, *, stream=None):
+    """S [B, H, dk, dv] fp32 = src (same shape) or zeros."""
+    B, H, dk, dv = S.shape
+    _need(S, "S", torch.float32, (B, H, dk, dv))
+    if src is not None:
+        _need(src, "src", torch.float32, (B, H, dk, dv))
+    _check("gdr_state_init",
+           _load().gdr_state_init(_ptr(S), B, H, dk, dv, _ptr(src), _stream(stream)))
+    return S
+
+
+def gdr_read_status(workspace, *, stream=None):
+    """Synchronizes and returns (and clears) the device status word of ``workspace``."""
+    st = ctypes.c_int(0)
+    _check("gdr_read_status", _load().gdr_read_status(_ptr(workspace), _stream(stream),
+                                                      ctypes.byref(st)))
+    return STATUS.get(st.value, st.value)
+
+
+def gdr_version():
+    return int(_load().gdr_version())
+
+
+def to_device(arrays: dict, dtype: str, device="cuda") -> dict:
+    """Moves the float32 numpy arrays of ``synth`` to the device: ``log_w``/``S0`` stay
+    fp32, the token inputs become ``dtype`` ("bf16" or "f32"; exact, the values are
+    already rounded to it)."""
+    import numpy as np
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    out = {}
+    for name, a in arrays.items():
+        if a is None:
+            out[name] = None
+            continue
+        t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32))
+        t = t.to(device=device, dtype=torch.float32 if name in ("log_w", "S0") else tdt)
+        out[name] = t.contiguous()
+    return out

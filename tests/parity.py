@@ -1,0 +1,61 @@
+"""Shared helpers of the GPU parity tests: run libgdr and the oracle on the same
+seeded inputs and measure the per-head relative error.
+
+Error norm (per (b, h) head, max over heads): ||X_gpu - X_ref||_F / max(||X_ref||_F, 1e-30),
+with X the head's T x dv output block, and separately its final d_k x d_v state.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from matrix_memory_rnn_b200 import gdr, synth
+
+# Bars: fp32 inputs 1e-4, bf16 inputs 2e-2 (fp32 state and accumulation).  The fp32
+# kernel is held to 1e-4 on either input dtype (it computes every product in fp32).
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+TOL_FP32_KERNEL = 1e-4
+
+
+def head_rel_err(x, ref, head_axes):
+    """Max over heads of the Frobenius relative error; `head_axes` index the head in x."""
+    x = np.asarray(x, np.float64)
+    ref = np.asarray(ref, np.float64)
+    other = tuple(i for i in range(x.ndim) if i not in head_axes)
+    num = np.sqrt(np.sum((x - ref) ** 2, axis=other))
+    den = np.maximum(np.sqrt(np.sum(ref ** 2, axis=other)), 1e-30)
+    return float(np.max(num / den)) if num.size else 0.0
+
+
+def oracle_forward(w, inp, S0=None, heads=None):
+    """Oracle on the synth inputs; `heads` = optional list of (b, h) to restrict to."""
+    S0 = inp.get("S0") if S0 is None else S0
+    args = [inp["q"], inp["k"], inp["v"], inp["log_w"], inp["e1"], inp["e2"], S0]
+    if heads is None:
+        return oracle.forward(w.form, *args)
+    outs = []
+    for b, h in heads:
+        sub = [None if a is None else (a[b:b + 1, h:h + 1] if a.ndim == 4 and a is S0 else
+                                       (a[b:b + 1, :, h:h + 1] if a.ndim >= 3 else a))
+               for a in args]
+        outs.append(oracle.forward(w.form, *sub))
+    return outs
+
+
+def gpu_forward(w, inp, algo="auto", chunk=None, S0=None, device="cuda"):
+    d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, w.dtype,
+                      device)
+    s0 = inp.get("S0") if S0 is None else S0
+    s0 = None if s0 is None else torch.from_numpy(np.ascontiguousarray(s0, np.float32)).to(device)
+    o, S_T = gdr.gdr_forward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
+                                     d["e2"], s0, chunk=chunk or w.chunk, algo=algo)
+    torch.cuda.synchronize()
+    return o.cpu().numpy(), S_T.cpu().numpy()
+
+
+def small(form, dtype, dk=64, dv=64, T=100, B=2, H=3, chunk=32, seed=11, **kw):
+    base = dict(gdn2=synth.PRESETS["gdn2_bf16"], rwkv7=synth.PRESETS["rwkv7_bf16"],
+                general=synth.PRESETS["rwkv7_bf16"], gla=synth.PRESETS["gdn2_bf16"])[form]
+    return base.with_(name=f"{form}_{dtype}_small", form=form, dtype=dtype, B=B, H=H, T=T,
+                      dk=dk, dv=dv, chunk=chunk, seed=seed, **kw)

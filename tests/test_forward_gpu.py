@@ -1,0 +1,125 @@
+"""GPU parity of gdr_forward_chunked against the fp64 oracle, plus internal
+consistency (chunk-size invariance, split-sequence resume, decode x T)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from matrix_memory_rnn_b200 import gdr, synth
+from parity import TOL, TOL_FP32_KERNEL, gpu_forward, head_rel_err, oracle_forward, small
+
+pytestmark = pytest.mark.gpu
+
+FORMS = ["gdn2", "rwkv7", "general", "gla"]
+
+
+@pytest.mark.parametrize("form", FORMS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dk,dv,chunk,T", [(64, 64, 32, 100), (128, 128, 64, 77),
+                                           (32, 128, 16, 50), (128, 16, 128, 300),
+                                           (16, 32, 64, 1)])
+def test_fp32_kernel_small(form, dtype, dk, dv, chunk, T):
+    w = small(form, dtype, dk=dk, dv=dv, T=T, chunk=chunk)
+    inp = synth.forward_inputs(w)
+    inp["S0"] = synth.round_f32(np.random.default_rng(5).normal(0, 0.3, (w.B, w.H, dk, dv)))
+    o, S = gpu_forward(w, inp, algo="fp32")
+    o_ref, S_ref = oracle_forward(w, inp)
+    assert head_rel_err(o, o_ref, (0, 2)) < TOL_FP32_KERNEL
+    assert head_rel_err(S, S_ref, (0, 1)) < TOL_FP32_KERNEL
+
+
+@pytest.mark.parametrize("name", ["rwkv7_f32", "gdn2_bf16", "rwkv7_bf16", "gdn2_long"])
+def test_preset_full_size(name):
+    w = synth.PRESETS[name]
+    inp = synth.forward_inputs(w)
+    o, S = gpu_forward(w, inp, algo="auto")
+    o_ref, S_ref = oracle_forward(w, inp)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    print(f"{name}: max head rel err o {eo:.3e} S {es:.3e}")
+    assert eo < TOL[w.dtype] and es < TOL[w.dtype]
+
+
+def test_zero_tokens_copies_state():
+    w = small("gdn2", "bf16", T=0)
+    inp = synth.forward_inputs(w.with_(T=1))
+    S0 = np.random.default_rng(3).normal(0, 1, (w.B, w.H, w.dk, w.dv)).astype(np.float32)
+    d = gdr.to_device({k: inp[k][:, :0] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "bf16")
+    s0 = torch.from_numpy(S0).cuda()
+    o, S_T = gdr.gdr_forward_chunked("gdn2", d["q"], d["k"], d["v"], d["log_w"], d["e1"],
+                                     d["e2"], s0, chunk=64)
+    torch.cuda.synchronize()
+    assert o.numel() == 0 and np.array_equal(S_T.cpu().numpy(), S0)
+
+
+@pytest.mark.parametrize("algo", ["fp32", "auto"])
+def test_state_alias_and_resume(algo):
+    """S_T may alias S0; running [0, T1) then [T1, T) from its state equals [0, T)."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=192, chunk=64)
+    inp = synth.forward_inputs(w)
+    o_full, S_full = gpu_forward(w, inp, algo=algo)
+    d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "bf16")
+    S = torch.zeros((w.B, w.H, w.dk, w.dv), device="cuda")
+    outs = []
+    for lo, hi in ((0, 70), (70, 192)):
+        part = {k: None if d[k] is None else d[k][:, lo:hi].contiguous() for k in d}
+        o, _ = gdr.gdr_forward_chunked("gdn2", part["q"], part["k"], part["v"], part["log_w"],
+                                       part["e1"], part["e2"], S, S_T=S, chunk=64, algo=algo)
+        outs.append(o)
+    torch.cuda.synchronize()
+    o_split = torch.cat(outs, dim=1).cpu().numpy()
+    tol = TOL_FP32_KERNEL if algo == "fp32" else 1e-2
+    assert head_rel_err(o_split, o_full, (0, 2)) < tol
+    assert head_rel_err(S.cpu().numpy(), S_full, (0, 1)) < tol
+
+
+@pytest.mark.parametrize("algo", ["fp32", "auto"])
+def test_chunk_size_invariance(algo):
+    w = small("rwkv7", "bf16", dk=64, dv=64, T=256)
+    inp = synth.forward_inputs(w)
+    res = [gpu_forward(w, inp, algo=algo, chunk=c) for c in (16, 32, 64, 128)]
+    tol = TOL_FP32_KERNEL if algo == "fp32" else 1e-2
+    for o, S in res[1:]:
+        assert head_rel_err(o, res[0][0], (0, 2)) < tol
+        assert head_rel_err(S, res[0][1], (0, 1)) < tol
+
+
+def test_decode_steps_equal_chunked_forward():
+    w = small("rwkv7", "f32", dk=64, dv=64, T=40, chunk=16)
+    inp = synth.forward_inputs(w)
+    o_ref, S_ref = gpu_forward(w, inp, algo="fp32")
+    d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "f32")
+    S = torch.zeros((w.B, w.H, w.dk, w.dv), device="cuda")
+    outs = []
+    for t in range(w.T):
+        tok = {k: d[k][:, t].contiguous() for k in d}
+        outs.append(gdr.gdr_decode_step("rwkv7", tok["q"], tok["k"], tok["v"], tok["log_w"],
+                                        tok["e1"], tok["e2"], S).clone())
+    torch.cuda.synchronize()
+    o_dec = torch.stack(outs, dim=1).cpu().numpy()
+    assert head_rel_err(o_dec, o_ref, (0, 2)) < 1e-4
+    assert head_rel_err(S.cpu().numpy(), S_ref, (0, 1)) < 1e-4
+
+
+def test_eviction_on_gpu():
+    """Targeted removal evicts (k_A, v_A) as (1 - c)^T ("Exponential gates ...", 13.3)."""
+    d, T, c = 64, 30, 0.1
+    rng = np.random.default_rng(4)
+    kA = rng.standard_normal(d); kA /= np.linalg.norm(kA)
+    vA = rng.standard_normal(d)
+    P = np.eye(d) - np.outer(kA, kA)
+    n = T + 1
+    q = np.ones((1, n, 1, d)); k = np.zeros((1, n, 1, d)); v = np.zeros((1, n, 1, d))
+    a = np.zeros((1, n, 1, d)); cc = np.zeros((1, n, 1))
+    k[0, 0, 0], v[0, 0, 0], a[0, 0, 0] = kA, vA, kA
+    for t in range(1, n):
+        b = P @ rng.standard_normal(d); b /= np.linalg.norm(b)
+        k[0, t, 0], v[0, t, 0], a[0, t, 0], cc[0, t, 0] = b, rng.standard_normal(d), kA, c
+    f = lambda x: torch.tensor(x, dtype=torch.float32, device="cuda").contiguous()
+    _, S_T = gdr.gdr_forward_chunked("rwkv7", f(q), f(k), f(v), f(np.zeros((1, n, 1, d))),
+                                     f(a), f(cc), None, chunk=16, algo="fp32")
+    torch.cuda.synchronize()
+    St = S_T[0, 0].double().cpu().numpy()
+    kA32 = np.asarray(f(kA).cpu().numpy(), np.float64)
+    vA32 = np.asarray(f(vA).cpu().numpy(), np.float64)
+    ratio = np.linalg.norm(St.T @ kA32) / np.linalg.norm(vA32)
+    assert abs(ratio - (1 - c) ** T) < 1e-5
