@@ -75,57 +75,95 @@ def load_peaks():
 
 
 class ClockSampler:
-    """Samples nvidia-smi clocks and throttle reasons during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clocks and clock-event (throttle) reasons during a timed region.
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+    Uses NVML from a background thread (about every 2 ms, so even a region of a
+    few milliseconds gets samples); falls back to ``nvidia-smi -lms 20``.  Reads
+    settings only; changes nothing on the GPU.
+    """
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.samples = []
+        self.max_mhz = None
+        self._stop = None
+        self._thread = None
+        self._proc = None
+        self._path = None
+
+    def _nvml_loop(self, nv, handle):
+        import time as _t
+        masks = [(n, getattr(nv, c, 0)) for n, c in self.REASONS]
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                bits = get_reasons(handle)
+                self.samples.append((float(mhz), [n for n, m in masks if bits & m]))
+            except Exception:
+                pass
+            _t.sleep(0.002)
 
     def __enter__(self):
         try:
-            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            import threading
+            import pynvml as nv
+            nv.nvmlInit()
+            handle = nv.nvmlDeviceGetHandleByUUID(self.uuid)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM))
+            self._stop = threading.Event()
+            self._thread = threading.Thread(target=self._nvml_loop, args=(nv, handle), daemon=True)
+            self._thread.start()
+            return self
+        except Exception:
+            self._thread = None
+        try:
+            fd, self._path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.uuid}",
+                 "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                 "clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap",
+                 "--format=csv,noheader,nounits", "-lms", "20"],
+                stdout=open(self._path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
-            self.proc = None
+            self._proc = None
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+        if self._proc is not None:
+            self._proc.terminate()
             try:
-                self.proc.wait(timeout=5)
+                self._proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._proc.kill()
+            for line in open(self._path):
+                parts = [x.strip() for x in line.split(",")]
+                try:
+                    self.max_mhz = float(parts[1])
+                    self.samples.append((float(parts[0]), [n for (n, _), x in
+                                                          zip(self.REASONS, parts[2:6])
+                                                          if x.lower() == "active"]))
+                except (ValueError, IndexError):
+                    continue
+            os.unlink(self._path)
 
     def summary(self):
-        if self.proc is None or not self.path or not os.path.exists(self.path):
+        if not self.samples:
             return None
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-            except ValueError:
-                continue
-        os.unlink(self.path)
-        if not rows:
-            return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, x in enumerate(r)
-                          if x.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows),
-                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
 
 
 # ----------------------------------------------------------------------------
@@ -186,6 +224,161 @@ def run_reference(args):
 # ----------------------------------------------------------------------------
 # GPU side
 # ----------------------------------------------------------------------------
+class Ctx:
+    """Device, stream and the rank plumbing (barrier, max over ranks)."""
+
+    def __init__(self, torch, dist, world, rank, local):
+        self.torch, self.dist = torch, dist
+        self.world, self.rank, self.local = world, rank, local
+        self.dev = torch.device("cuda", local)
+        self.stream = torch.cuda.current_stream()
+        self.peaks = load_peaks()
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+        except Exception:
+            self.uuid = str(local)
+
+    def barrier(self):
+        if self.world > 1:
+            self.dist.barrier()
+
+    def max_over_ranks(self, x):
+        if self.world == 1:
+            return x
+        t = self.torch.tensor([x], dtype=self.torch.float64, device=self.dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def event(self):
+        return self.torch.cuda.Event(enable_timing=True)
+
+
+def bench_forward(ctx, args, gdr):
+    """Device-resident chunked forward: K timed steps, kernel time per launch."""
+    torch = ctx.torch
+    w = FWD
+    inp = synth.forward_inputs(w, seed=w.seed + 1000 * ctx.rank)
+    names = ("q", "k", "v", "log_w", "e1", "e2")
+    d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=ctx.dev)
+    S_T = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=ctx.dev)
+    ws = gdr.new_workspace(gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"],
+                                                          d["log_w"], d["e1"], d["e2"],
+                                                          w.chunk, args.algo), ctx.dev)
+
+    def step(bufs):
+        gdr.gdr_forward_chunked(w.form, bufs["q"], bufs["k"], bufs["v"], bufs["log_w"],
+                                bufs["e1"], bufs["e2"], None, chunk=w.chunk, algo=args.algo,
+                                o=o, S_T=S_T, workspace=ws)
+
+    evs = [(ctx.event(), ctx.event()) for _ in range(args.steps)]
+    t0, t1 = ctx.event(), ctx.event()
+    # The clock sampler runs from the warm-up through the timed region: a timed
+    # region of a few milliseconds is shorter than nvidia-smi's sampling period.
+    with ClockSampler(ctx.uuid) as clk:
+        for _ in range(max(args.warmup, 1)):
+            step(d)
+        torch.cuda.synchronize()
+        status = gdr.gdr_read_status(ws)
+        if status != "GDR_OK":
+            raise RuntimeError(f"device status after warm-up: {status}")
+        ctx.barrier()
+        torch.cuda.synchronize()
+        t0.record(ctx.stream)
+        for i in range(args.steps):
+            evs[i][0].record(ctx.stream)
+            step(d)
+            evs[i][1].record(ctx.stream)
+        t1.record(ctx.stream)
+        torch.cuda.synchronize()
+        ctx.barrier()
+    status = gdr.gdr_read_status(ws)
+    if status != "GDR_OK":
+        raise RuntimeError(f"device status after the timed steps: {status}")
+    ms_total = ctx.max_over_ranks(t0.elapsed_time(t1))
+    ms_kernel = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    res = {"w": w, "ms_per_step": ms_total / args.steps, "ms_kernel": ms_kernel,
+           "clocks": clk.summary(), "launches": args.steps}
+    if args.only == "all":
+        res["e2e"] = bench_e2e(ctx, args, gdr, w, inp, names, step, o)
+    return res
+
+
+def bench_e2e(ctx, args, gdr, w, inp, names, step, o):
+    """Same call with host inputs: pinned H2D copies, the forward, D2H of o, all timed."""
+    torch = ctx.torch
+    host = {k: None if inp[k] is None else torch.from_numpy(inp[k]) for k in names}
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    pinned = {k: None if t is None else
+              t.to(torch.float32 if k == "log_w" else tdt).pin_memory() for k, t in host.items()}
+    dev_bufs = {k: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=ctx.dev)
+                for k, t in pinned.items()}
+    o_host = torch.empty(o.shape, dtype=torch.float32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
+    d2h = o.numel() * 4
+
+    def e2e_step():
+        for k, t in pinned.items():
+            if t is not None:
+                dev_bufs[k].copy_(t, non_blocking=True)
+        step(dev_bufs)
+        o_host.copy_(o, non_blocking=True)
+
+    n = max(3, min(args.steps, 10))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ctx.barrier()
+    e0, e1 = ctx.event(), ctx.event()
+    e0.record(ctx.stream)
+    for _ in range(n):
+        e2e_step()
+    e1.record(ctx.stream)
+    torch.cuda.synchronize()
+    ms = ctx.max_over_ranks(e0.elapsed_time(e1)) / n
+    return {"value": w.tokens * ctx.world / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+def bench_decode(ctx, args, gdr):
+    """Decode step on the resident 1 GiB state, inputs cycled from 8 seeded steps."""
+    torch = ctx.torch
+    dw = DEC
+    S = torch.from_numpy(synth.decode_state(dw, seed=dw.seed + 1000 * ctx.rank)).to(ctx.dev)
+    names = ("q", "k", "v", "log_w", "e1", "e2")
+    pool = [gdr.to_device({k: p[k] for k in names}, "bf16", ctx.dev)
+            for p in (synth.decode_step_inputs(dw, s, seed=dw.seed + 1000 * ctx.rank)
+                      for s in range(8))]
+    o_dec = torch.empty((dw.B, dw.H, dw.dv), dtype=torch.float32, device=ctx.dev)
+
+    def step(i):
+        p = pool[i % len(pool)]
+        gdr.gdr_decode_step(dw.form, p["q"], p["k"], p["v"], p["log_w"], p["e1"], p["e2"], S,
+                            o=o_dec)
+
+    d0, d1 = ctx.event(), ctx.event()
+    with ClockSampler(ctx.uuid) as clk:
+        for i in range(args.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        ctx.barrier()
+        d0.record(ctx.stream)
+        for i in range(args.decode_steps):
+            step(i)
+        d1.record(ctx.stream)
+        torch.cuda.synchronize()
+    ms = ctx.max_over_ranks(d0.elapsed_time(d1)) / args.decode_steps
+    nbytes = dec_algorithmic_bytes(dw)
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": dw.name, "form": dw.form, "B": dw.B, "H": dw.H, "dk": dw.dk,
+            "dv": dw.dv, "steps": args.decode_steps, "steps_per_s": 1e3 / ms,
+            "ms_per_step": ms,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"], "traffic": None,
+                         "bytes_per_launch": nbytes, "peak_source": ctx.peaks["source"]},
+            "gpu_launches": args.decode_steps, "clocks": clk.summary()}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -196,6 +389,8 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=15.0)
+    ap.add_argument("--only", default="all", choices=["all", "forward", "decode"],
+                    help="time one part only (profiling runs); the default line needs 'all'")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -209,170 +404,51 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
     if world > 1:
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+                                device_id=torch.device("cuda", local))
+    ctx = Ctx(torch, dist, world, rank, local)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    peaks = load_peaks()
-    stream = torch.cuda.current_stream()
-
-    # ---------------- chunked forward (the headline) ----------------
-    w = FWD
-    inp = synth.forward_inputs(w, seed=w.seed + 1000 * rank)
-    host = {k: None if inp[k] is None else torch.from_numpy(inp[k]) for k in
-            ("q", "k", "v", "log_w", "e1", "e2")}
-    d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, w.dtype, dev)
-    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=dev)
-    S_T = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
-    ws = gdr.new_workspace(gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"],
-                                                          d["log_w"], d["e1"], d["e2"],
-                                                          w.chunk, args.algo), dev)
-
-    def fwd_step():
-        gdr.gdr_forward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"], d["e2"],
-                                None, chunk=w.chunk, algo=args.algo, o=o, S_T=S_T,
-                                workspace=ws)
-
-    for _ in range(args.warmup):
-        fwd_step()
-    torch.cuda.synchronize()
-    status = gdr.gdr_read_status(ws)
-    if status != "GDR_OK":
-        raise RuntimeError(f"device status after warm-up: {status}")
-
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
-    t_all0, t_all1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t_all0.record(stream)
-        for i in range(args.steps):
-            evs[i][0].record(stream)
-            fwd_step()
-            evs[i][1].record(stream)
-        t_all1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-    clocks = clk.summary()
-    ms_total = max_over_ranks(t_all0.elapsed_time(t_all1))
-    ms_kernel = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    ms_per_step = ms_total / args.steps
-    tokens = w.tokens * world
-    value = tokens / (ms_per_step * 1e-3)
-    nbytes = fwd_algorithmic_bytes(w)
-    nflops = fwd_flops(w)
-    achieved = nbytes / (ms_kernel * 1e-3) / 1e9
-
-    # ---------------- e2e through the C-ABI call with host buffers ----------------
-    pinned = {k: None if t is None else t.to(d[k].dtype).pin_memory() for k, t in host.items()}
-    dev_bufs = {k: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev)
-                for k, t in pinned.items()}
-    o_host = torch.empty(o.shape, dtype=torch.float32, pin_memory=True)
-    h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
-    d2h = o.numel() * 4
-
-    def e2e_step():
-        for k, t in pinned.items():
-            if t is not None:
-                dev_bufs[k].copy_(t, non_blocking=True)
-        gdr.gdr_forward_chunked(w.form, dev_bufs["q"], dev_bufs["k"], dev_bufs["v"],
-                                dev_bufs["log_w"], dev_bufs["e1"], dev_bufs["e2"], None,
-                                chunk=w.chunk, algo=args.algo, o=o, S_T=S_T, workspace=ws)
-        o_host.copy_(o, non_blocking=True)
-
-    e2e_steps = max(3, min(args.steps, 10))
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier()
-    e0, e1_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    e1_.record(stream)
-    torch.cuda.synchronize()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1_)) / e2e_steps
-    e2e_value = tokens / (ms_e2e * 1e-3)
-
-    # ---------------- decode step ----------------
-    dw = DEC
-    S = torch.from_numpy(synth.decode_state(dw, seed=dw.seed + 1000 * rank)).to(dev)
-    pool = [gdr.to_device({k: p[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "bf16", dev)
-            for p in (synth.decode_step_inputs(dw, s, seed=dw.seed + 1000 * rank)
-                      for s in range(8))]
-    o_dec = torch.empty((dw.B, dw.H, dw.dv), dtype=torch.float32, device=dev)
-
-    def dec_step(i):
-        p = pool[i % len(pool)]
-        gdr.gdr_decode_step(dw.form, p["q"], p["k"], p["v"], p["log_w"], p["e1"], p["e2"], S,
-                            o=o_dec)
-
-    for i in range(args.warmup):
-        dec_step(i)
-    torch.cuda.synchronize()
-    barrier()
-    dev0, dev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dev0.record(stream)
-    for i in range(args.decode_steps):
-        dec_step(i)
-    dev1.record(stream)
-    torch.cuda.synchronize()
-    ms_dec = max_over_ranks(dev0.elapsed_time(dev1)) / args.decode_steps
-    dec_bytes = dec_algorithmic_bytes(dw)
-    dec_gbs = dec_bytes / (ms_dec * 1e-3) / 1e9
-
+    fwd = bench_forward(ctx, args, gdr) if args.only in ("all", "forward") else None
+    dec = bench_decode(ctx, args, gdr) if args.only in ("all", "decode") else None
+    ctx.barrier()
     if world > 1:
-        barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    cpu = None
-    if not args.no_cpu_baseline and world == 1:
-        v_cpu, cores, sample = oracle_sample_rate(w, budget_s=15.0)
-        cpu = {"value": v_cpu, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "form": w.form, "B": w.B, "H": w.H, "T": w.T,
-                   "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "algo": args.algo,
-                   "parallelism": f"dp{world} (independent sequences, no collective)",
-                   "l2": f"inputs larger than L2 ({nbytes / 2**20:.0f} MiB per step > 126 MiB)"},
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                     "peak_source": peaks["source"], "bytes_per_launch": nbytes,
-                     "kernel_ms": ms_kernel},
-        "tensor": {"flops_per_launch": nflops, "achieved_tflops": nflops / (ms_kernel * 1e-3) / 1e12,
-                   "peak_tflops": peaks["bf16_tflops"],
-                   "frac": nflops / (ms_kernel * 1e-3) / 1e12 / peaks["bf16_tflops"]},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
-        "gpu_launches": args.steps,
-        "clocks": clocks,
-        "cpu_baseline": cpu,
-        "decode": {"workload": dw.name, "B": dw.B, "H": dw.H, "dk": dw.dk, "dv": dw.dv,
-                   "steps": args.decode_steps, "steps_per_s": 1e3 / ms_dec, "ms_per_step": ms_dec,
-                   "roofline": {"bound": "hbm", "achieved": dec_gbs, "peak": peaks["hbm_gbs"],
-                                "unit": "GB/s", "frac": dec_gbs / peaks["hbm_gbs"],
-                                "traffic": None, "bytes_per_launch": dec_bytes},
-                   "gpu_launches": args.decode_steps},
-    }
+    line = {"metric": METRIC, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic"}
+    if fwd is not None:
+        w = fwd["w"]
+        nbytes, nflops = fwd_algorithmic_bytes(w), fwd_flops(w)
+        achieved = nbytes / (fwd["ms_kernel"] * 1e-3) / 1e9
+        tflops = nflops / (fwd["ms_kernel"] * 1e-3) / 1e12
+        line.update({
+            "value": w.tokens * world / (fwd["ms_per_step"] * 1e-3),
+            "ms_per_step": fwd["ms_per_step"],
+            "config": {"workload": w.name, "form": w.form, "B": w.B, "H": w.H, "T": w.T,
+                       "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "algo": args.algo,
+                       "parallelism": f"dp{world} (independent sequences, no collective)",
+                       "l2": f"inputs larger than L2 ({nbytes / 2**20:.0f} MiB per step > 126 MiB)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": ctx.peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / ctx.peaks["hbm_gbs"],
+                         "traffic": None, "peak_source": ctx.peaks["source"],
+                         "bytes_per_launch": nbytes, "kernel_ms": fwd["ms_kernel"]},
+            "tensor": {"flops_per_launch": nflops, "achieved_tflops": tflops,
+                       "peak_tflops": ctx.peaks["bf16_tflops"],
+                       "frac": tflops / ctx.peaks["bf16_tflops"]},
+            "gpu_launches": fwd["launches"], "clocks": fwd["clocks"]})
+        if "e2e" in fwd:
+            line["e2e"] = fwd["e2e"]
+        if not args.no_cpu_baseline and world == 1:
+            v_cpu, cores, sample = oracle_sample_rate(w, budget_s=15.0)
+            line["cpu_baseline"] = {"value": v_cpu, "unit": UNIT, "cores": cores,
+                                    "kind": "oracle", "sample": sample}
+    if dec is not None:
+        line["decode"] = dec
     print(json.dumps(line), flush=True)
     return 0
 

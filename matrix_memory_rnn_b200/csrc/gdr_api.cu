@@ -107,7 +107,12 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
   p.S_T = a->S_T;
   p.status = static_cast<uint32_t *>(a->workspace);
 
-  if (a->algo == GDR_ALGO_TC) return GDR_ERR_UNSUPPORTED;
+  const bool tc_ok = gdr::forward_tc_supported(p, a->dtype);
+  if (a->algo == GDR_ALGO_TC || (a->algo == GDR_ALGO_AUTO && tc_ok)) {
+    if (!tc_ok) return GDR_ERR_UNSUPPORTED;
+    if (!a->workspace || a->workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
+    return cuda_status(gdr::launch_forward_tc(p, s));
+  }
   if (!gdr::forward_fp32_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
   return cuda_status(gdr::launch_forward_fp32(p, a->dtype, s));
 }

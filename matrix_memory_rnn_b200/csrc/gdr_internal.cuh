@@ -62,6 +62,8 @@ struct FwdParams {
 cudaError_t launch_decode(const gdr_step_args &a, cudaStream_t stream);
 cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_t stream);
 bool forward_fp32_supported(int dk, int dv);
+cudaError_t launch_forward_tc(const FwdParams &p, cudaStream_t stream);
+bool forward_tc_supported(const FwdParams &p, gdr_dtype dtype);
 size_t forward_fp32_smem_bytes(int dk, int dv, int chunk);
 
 }  // namespace gdr

@@ -123,3 +123,42 @@ def test_eviction_on_gpu():
     vA32 = np.asarray(f(vA).cpu().numpy(), np.float64)
     ratio = np.linalg.norm(St.T @ kA32) / np.linalg.norm(vA32)
     assert abs(ratio - (1 - c) ** T) < 1e-5
+
+
+@pytest.mark.parametrize("T", [1, 64, 100, 257])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_tc_kernel_gdn2(T, with_state):
+    """Tensor-core kernel (GDN-2, bf16, d = 128, C = 64) against the oracle, with a ragged tail."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=T, B=2, H=3, chunk=64)
+    inp = synth.forward_inputs(w)
+    if with_state:
+        inp["S0"] = synth.round_f32(np.random.default_rng(7).normal(0, 0.5, (w.B, w.H, 128, 128)))
+    o, S = gpu_forward(w, inp, algo="tc")
+    o_ref, S_ref = oracle_forward(w, inp)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    print(f"tc T={T} S0={with_state}: o {eo:.3e} S {es:.3e}")
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
+def test_tc_kernel_strong_decay_uses_exact_path():
+    """Channels whose decay over a chunk exceeds e^-80 take the exact pairwise path."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=200, B=1, H=2, chunk=64)
+    inp = synth.forward_inputs(w)
+    lw = inp["log_w"].copy()
+    lw[:, :, :, ::7] = -3.0          # 64 tokens x 3 nats = 192 nats per chunk on these channels
+    lw[:, 70:80, 1, 5] = -60.0       # a burst of very strong decay on one head
+    inp["log_w"] = lw.astype(np.float32)
+    o, S = gpu_forward(w, inp, algo="tc")
+    o_ref, S_ref = oracle_forward(w, inp)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    print(f"tc strong decay: o {eo:.3e} S {es:.3e}")
+    assert np.isfinite(o).all() and np.isfinite(S).all()
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
+def test_tc_rejects_what_it_does_not_cover():
+    w = small("rwkv7", "bf16", dk=64, dv=64, T=64, B=1, H=1)
+    inp = synth.forward_inputs(w)
+    with pytest.raises(gdr.GdrError) as ei:
+        gpu_forward(w, inp, algo="tc")
+    assert ei.value.code == 2
