@@ -129,6 +129,33 @@ gdr_status gdr_forward_workspace_size(const gdr_fwd_args *args, size_t *bytes);
 gdr_status gdr_forward_chunked(const gdr_fwd_args *args, void *stream);
 
 /*
+ * gdr_forward_chunked for callers that cannot allocate device memory.  (No
+ * counterpart in the papers: this is a deployment convenience.)
+ *
+ * Some callers are not allowed to allocate: a plugin whose host application owns
+ * every device allocation, a serving loop that forbids allocation once its memory
+ * plan is fixed, code where cudaMalloc is unavailable or would synchronize.  This
+ * call computes exactly what gdr_forward_chunked computes, but ignores
+ * args->workspace / workspace_bytes and uses a fixed scratch array compiled into
+ * libgdr instead (a static __device__ array of 4096 bytes that every GPU loading
+ * the library holds until process exit).  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture.
+ *   - All calls share the one array; calls that overlap on the GPU (different
+ *     streams, or different host threads on the same device) race on it.
+ *     Serialize them.
+ *   - The array keeps the last call's contents; each call clears the status word
+ *     it uses on `stream` before the launch.
+ *   - A call that would need more scratch than the array holds returns
+ *     GDR_ERR_WORKSPACE.  The device status word lives in the library's array,
+ *     so gdr_read_status cannot report this variant's device-side failures.
+ * Errors and all other arguments: as gdr_forward_chunked.
+ */
+gdr_status gdr_forward_chunked_noalloc(const gdr_fwd_args *args, void *stream);
+
+/*
  * Arguments of gdr_decode_step: one token for each (b, h).
  *   q, k, log_w, e1 (GENERAL/GDN2/RWKV7) : [B][H][dk]
  *   v, o, e2 (GDN2)                      : [B][H][dv]

@@ -255,3 +255,22 @@ def to_device(arrays: dict, dtype: str, device="cuda") -> dict:
         t = t.to(device=device, dtype=torch.float32 if name in ("log_w", "S0") else tdt)
         out[name] = t.contiguous()
     return out
+
+
+def gdr_forward_chunked_noalloc(form, q, k, v, log_w, e1=None, e2=None, S0=None, *, chunk=64,
+                                algo="auto", o=None, S_T=None, stream=None):
+    """``gdr_forward_chunked`` through the entry point that allocates nothing.
+
+    For callers that may not allocate device memory: libgdr supplies the scratch
+    from a fixed array of its own (see include/gdr.h).  ``o`` and ``S_T`` must be
+    given by the caller (this function allocates nothing either).
+    """
+    lib = _load()
+    fn = lib.gdr_forward_chunked_noalloc
+    fn.argtypes = [ctypes.POINTER(gdr_fwd_args), _vp]
+    fn.restype = _c_int
+    if o is None:
+        raise ValueError("o is required (the no-alloc path allocates nothing)")
+    a = _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, None)
+    _check("gdr_forward_chunked_noalloc", fn(ctypes.byref(a), _stream(stream)))
+    return o, S_T
