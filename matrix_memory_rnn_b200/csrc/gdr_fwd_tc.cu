@@ -41,6 +41,11 @@
 #include "gdr_internal.cuh"
 #include "gdr_sm100.cuh"
 
+// Phase hooks for an external timing harness; empty in the library build.
+#ifndef GDR_PHASE
+#define GDR_PHASE(i)
+#endif
+
 namespace gdr {
 namespace {
 
@@ -286,6 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     __syncthreads();
     const bool exact = sflag[0] != 0;
 
+    GDR_PHASE(0);
     // ---- P1: operand tiles [K^ f; Q f], K g, K~, Q_pi
     for (int it = tid; it < kC * (kDK / 8); it += kThreads) {
       const int t = it >> 4, g = it & 15, j0 = 8 * g;
@@ -330,6 +336,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     fence_proxy_async_smem();
     __syncthreads();
 
+    GDR_PHASE(1);
     // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK
     if (tid == 0) {
       tc_fence_after();
@@ -344,6 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     }
     if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
 
+    GDR_PHASE(2);
     // ---- L (fp32, strictly lower) and M (bf16, lower incl. diagonal) out of TMEM
     if (!exact) {
       float x[32];
@@ -387,6 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     }
     __syncthreads();
 
+    GDR_PHASE(3);
     // ---- T^-1 (fp32), then bf16 copy as the A operand of MMA2
     invert_unit_lower(sL, sTi, tid);
     for (int it = tid; it < kC * (kC / 8); it += kThreads) {
@@ -403,6 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     tc_fence_before();
     __syncthreads();
 
+    GDR_PHASE(4);
     // ---- MMA2: U = T^-1 V^ (N = NV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
     if (tid == 0) {
       tc_fence_after();
@@ -420,6 +430,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     }
     if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
 
+    GDR_PHASE(5);
     // ---- Y = (T^-1 (K^ f)) Diag(alpha_1) -> bf16 (K-major, rows = tokens);
     //      M = 64 accumulators hold row 16 qd + lane
     {
@@ -443,6 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     tc_fence_before();
     __syncthreads();
 
+    GDR_PHASE(6);
     // ---- MMA3: Y S0 and Q_pi S0 (K = DK)
     if (tid == 0) {
       tc_fence_after();
@@ -459,6 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     }
     if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
 
+    GDR_PHASE(7);
     // ---- V~ = U - Y S0 -> bf16 (rows = tokens)
     {
       float u[32], d[32];
@@ -478,6 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     tc_fence_before();
     __syncthreads();
 
+    GDR_PHASE(8);
     // ---- MMA4: K~^T V~ (M = DK) and O += M V~ (M = C); K = C
     if (tid == 0) {
       tc_fence_after();
@@ -495,6 +509,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     }
     if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
 
+    GDR_PHASE(9);
     // ---- state update (fp32) and outputs
     {
       float d[32];
@@ -523,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    GDR_PHASE(10);
   }
 
   if (ok && p.S_T) {
