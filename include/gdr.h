@@ -1,7 +1,7 @@
 /*
  * gdr.h -- C ABI of libgdr: the generalized delta-rule matrix memory on B200.
  *
- * The recurrence (spec column form; the state S is d_v x d_k):
+ * The recurrence (column form; the state S is d_v x d_k):
  *
  *     e_t = S_{t-1} u_t
  *     S_t = S_{t-1} Diag(w_t) - e_t z_t^T + v_t k_t^T  = S_{t-1}(Diag(w_t) - u_t z_t^T) + v_t k_t^T
@@ -37,7 +37,8 @@
  *
  * Memory and ownership.  The caller owns every buffer; pointers are device
  * pointers unless stated otherwise.  libgdr allocates no device memory, keeps no
- * global state between calls, and never synchronizes the stream except where a
+ * global state between calls (apart from the fixed scratch array behind
+ * gdr_forward_chunked_noalloc), and never synchronizes the stream except where a
  * function says so.  Everything is enqueued asynchronously on the given stream
  * (a cudaStream_t passed as void*, NULL = legacy default stream).
  *
@@ -123,8 +124,12 @@ gdr_status gdr_forward_workspace_size(const gdr_fwd_args *args, size_t *bytes);
  * the unit lower-triangular system T V~ = V^ - K^_pi S0, S_C and O as matrix
  * products) and section 4.2 eq. (10) (outputs and end state affine in S0),
  * generalized to a separate erase key z (e_t and v_t carried as two write streams).
- * Cumulative decays are formed in log space and only exponentiated at non-positive
- * arguments (section 4.2, boundary-pivoted splitting), so nothing overflows.
+ * Cumulative decays are formed in log space and exponentiated only as differences:
+ * the fp32 kernel at non-positive arguments; the tensor-core kernel splits each
+ * pairwise decay at the chunk's first token, with both exponents bounded by 80
+ * (checked per chunk and channel; a chunk that decays more forms its products from
+ * the exact pairwise decays) -- the role section 4.2's boundary pivots play on the
+ * Muir page.  No factor is divided out and nothing overflows.
  */
 gdr_status gdr_forward_chunked(const gdr_fwd_args *args, void *stream);
 
