@@ -54,7 +54,7 @@ using namespace sm100;
 constexpr int kC = 64;
 constexpr int kDK = 128;
 constexpr int kThreads = 256;
-constexpr int kLD = kC + 1;                   // fp32 C x C row stride
+constexpr int kLD = kC + 4;                   // fp32 C x C row stride (16-byte rows)
 constexpr float kMaxChunkDecay = 80.f;        // nats
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint32_t kTmemCols = 256;
@@ -77,7 +77,8 @@ struct TcSmem {
   static constexpr uint32_t PIN = TI + kC * kLD * 4;            // fp32 exp(Lam_n) DK
   static constexpr uint32_t A1 = PIN + kDK * 4;                 // fp32 alpha_1 = exp(Lam_1) DK
   static constexpr uint32_t ED = A1 + kDK * 4;                  // fp32 exp(Lam_n - Lam_1) DK
-  static constexpr uint32_t MISC = ED + kDK * 4;                // mbarrier, TMEM slot, flags
+  static constexpr uint32_t TOT = ED + kDK * 4;                 // fp32 first-half log-decay DK
+  static constexpr uint32_t MISC = TOT + kDK * 4;               // mbarrier, TMEM slot, flags
   static constexpr uint32_t TOTAL = MISC + 64;
   static constexpr uint32_t ALLOC = TOTAL + 1024;               // + alignment slack
   static_assert(A_LM % 1024 == 0 && B_LM % 1024 == 0 && KT % 1024 == 0 && VH % 1024 == 0 &&
@@ -113,22 +114,24 @@ __device__ __forceinline__ void st_smem16(uint8_t *base, uint32_t off, const uin
   *reinterpret_cast<uint4 *>(base + off) = v;
 }
 
-// All threads: bounded wait for the MMA group committed to `bar`, then a CTA
-// barrier so every thread takes the same branch.  Returns false (after setting
-// the shared abort flag) when the wait ran out.
+// Bounded wait for the MMA group committed to `bar`: thread 0 polls the
+// mbarrier, then a CTA barrier passes the completion on (and makes every thread
+// take the same branch).  Returns false, with the shared abort flag set, when the
+// wait ran out.
 __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t &phase, volatile int *abort) {
-  if (!mbar_wait_bounded(bar, phase, kWaitLimitNs)) *abort = 1;
+  if (threadIdx.x == 0 && !mbar_wait_bounded(bar, phase, kWaitLimitNs)) *abort = 1;
   phase ^= 1u;
   __syncthreads();
   tc_fence_after();
   return *abort == 0;
 }
 
-// T^-1 for the unit lower-triangular T = I + L (L strictly lower, fp32, stride kLD),
-// by blocks: 16 x 16 diagonal blocks by forward substitution, then two merge levels
-// X21 = -T_R^-1 L_RL T_L^-1 (eq. (11) of the Muir page).  Writes the lower
-// triangle of Ti; the strictly-upper blocks of Ti are used as scratch.
-__device__ void invert_unit_lower(const float *Lm, float *Ti, int tid) {
+// T^-1 for the unit lower-triangular T = I + L (L strictly lower, fp32, row stride
+// kLD), by blocks (eq. (11) of the Muir page): the four 16 x 16 diagonal blocks by
+// forward substitution, then two merge levels X21 = -T_R^-1 (L_RL T_L^-1).  Writes
+// all of Ti (zeros above the diagonal); overwrites the merged L_RL blocks of Lm
+// with the products L_RL T_L^-1.  All 256 threads; ends with a CTA barrier.
+__device__ void invert_unit_lower(float *Lm, float *Ti, int tid) {
   if (tid < 64) {
     const int blk = tid >> 4, c = tid & 15, o = 16 * blk;
     float x[16];
@@ -141,36 +144,62 @@ __device__ void invert_unit_lower(const float *Lm, float *Ti, int tid) {
     }
 #pragma unroll
     for (int t = 0; t < 16; ++t) Ti[(o + t) * kLD + o + c] = x[t];
+  } else {
+    // zero the strictly-upper blocks the merge products read
+    for (int i = tid - 64; i < 32 * 32 + 2 * 16 * 16; i += kThreads - 64) {
+      int r, c;
+      if (i < 1024) { r = i >> 5; c = 32 + (i & 31); }
+      else { const int k = i - 1024, p = k >> 8; r = 32 * p + ((k >> 4) & 15); c = 32 * p + 16 + (k & 15); }
+      Ti[r * kLD + c] = 0.f;
+    }
   }
   __syncthreads();
-  // level 1: pairs of 16-blocks -> 32-blocks.  W = L_RL T_L^-1 into the upper block.
-  for (int it = tid; it < 2 * 256; it += kThreads) {
-    const int pr = it >> 8, i = (it >> 4) & 15, j = it & 15, o = 32 * pr;
-    float acc = 0.f;
-    for (int k = j; k < 16; ++k) acc += Lm[(o + 16 + i) * kLD + o + k] * Ti[(o + k) * kLD + o + j];
-    Ti[(o + i) * kLD + o + 16 + j] = acc;
+  // level 1: pairs (blocks 0,1) and (2,3).  Thread: pair p, row i, columns 2jq, 2jq+1.
+  {
+    const int p = tid >> 7, i = (tid >> 3) & 15, j = 2 * (tid & 7), o = 32 * p;
+    float w0 = 0.f, w1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float l = Lm[(o + 16 + i) * kLD + o + k];
+      const float2 t = *reinterpret_cast<const float2 *>(Ti + (o + k) * kLD + o + j);
+      w0 += l * t.x;
+      w1 += l * t.y;
+    }
+    __syncthreads();
+    *reinterpret_cast<float2 *>(Lm + (o + 16 + i) * kLD + o + j) = make_float2(w0, w1);
+    __syncthreads();
+    float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float t = Ti[(o + 16 + i) * kLD + o + 16 + k];
+      const float2 w = *reinterpret_cast<const float2 *>(Lm + (o + 16 + k) * kLD + o + j);
+      x0 += t * w.x;
+      x1 += t * w.y;
+    }
+    *reinterpret_cast<float2 *>(Ti + (o + 16 + i) * kLD + o + j) = make_float2(-x0, -x1);
   }
   __syncthreads();
-  for (int it = tid; it < 2 * 256; it += kThreads) {
-    const int pr = it >> 8, i = (it >> 4) & 15, j = it & 15, o = 32 * pr;
-    float acc = 0.f;
-    for (int k = 0; k <= i; ++k) acc += Ti[(o + 16 + i) * kLD + o + 16 + k] * Ti[(o + k) * kLD + o + 16 + j];
-    Ti[(o + 16 + i) * kLD + o + j] = -acc;
-  }
-  __syncthreads();
-  // level 2: 32-blocks -> 64.  W = L[32:64, 0:32] T[0:32,0:32]^-1 into rows 0..31, cols 32..63.
-  for (int it = tid; it < 1024; it += kThreads) {
-    const int i = it >> 5, j = it & 31;
-    float acc = 0.f;
-    for (int k = j; k < 32; ++k) acc += Lm[(32 + i) * kLD + k] * Ti[k * kLD + j];
-    Ti[i * kLD + 32 + j] = acc;
-  }
-  __syncthreads();
-  for (int it = tid; it < 1024; it += kThreads) {
-    const int i = it >> 5, j = it & 31;
-    float acc = 0.f;
-    for (int k = 0; k <= i; ++k) acc += Ti[(32 + i) * kLD + 32 + k] * Ti[k * kLD + 32 + j];
-    Ti[(32 + i) * kLD + j] = -acc;
+  // level 2: rows 32..63 x columns 0..31.  Thread: row i, columns 4jq .. 4jq+3.
+  {
+    const int i = tid >> 3, j = 4 * (tid & 7);
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float l = Lm[(32 + i) * kLD + k];
+      const float4 t = *reinterpret_cast<const float4 *>(Ti + k * kLD + j);
+      w.x += l * t.x; w.y += l * t.y; w.z += l * t.z; w.w += l * t.w;
+    }
+    __syncthreads();
+    *reinterpret_cast<float4 *>(Lm + (32 + i) * kLD + j) = w;
+    __syncthreads();
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const float t = Ti[(32 + i) * kLD + 32 + k];
+      const float4 v = *reinterpret_cast<const float4 *>(Lm + (32 + k) * kLD + j);
+      x.x += t * v.x; x.y += t * v.y; x.z += t * v.z; x.w += t * v.w;
+    }
+    *reinterpret_cast<float4 *>(Ti + (32 + i) * kLD + j) = make_float4(-x.x, -x.y, -x.z, -x.w);
   }
   __syncthreads();
 }
@@ -196,6 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
   float *sPiN = reinterpret_cast<float *>(smem + SL::PIN);
   float *sA1 = reinterpret_cast<float *>(smem + SL::A1);
   float *sED = reinterpret_cast<float *>(smem + SL::ED);
+  float *sTot = reinterpret_cast<float *>(smem + SL::TOT);
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + SL::MISC);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 8);
   volatile int *sflag = reinterpret_cast<volatile int *>(smem + SL::MISC + 16);  // [0] exact, [1] abort
@@ -248,63 +278,93 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
   for (int t0 = 0; t0 < T && ok; t0 += kC) {
     const int n = min(kC, T - t0);
 
-    // ---- P0: cumulative log-decay (threads = key channels); V^ = wg (.) v
-    if (tid < kDK) {
-      const int j = tid;
-      float lw[kC];
+    // ---- every global read of the chunk is issued first, before any use
+    // log w: thread (channel jc, half hh) holds tokens [32 hh, 32 hh + 32)
+    const int jc = tid & (kDK - 1), hh = tid >> 7;
+    float lw[32];
 #pragma unroll
-      for (int t = 0; t < kC; ++t)
-        lw[t] = (t < n) ? __ldg(p.log_w + (((size_t)b * T + t0 + t) * H + h) * kDK + j) : 0.f;
-      float acc = 0.f;
+    for (int t = 0; t < 32; ++t) {
+      const int tt = 32 * hh + t;
+      lw[t] = (tt < n) ? __ldg(p.log_w + (((size_t)b * T + t0 + tt) * H + h) * kDK + jc) : 0.f;
+    }
+    // operand inputs: items (t, 8-channel group g), 4 per thread
+    uint4 rk[4], rb[4], rq[4];
 #pragma unroll
-      for (int t = 0; t < kC; ++t) {
-        acc += lw[t];
-        sLam[t * kDK + j] = acc;
-      }
-      sPiN[j] = __expf(acc);
-      sA1[j] = __expf(lw[0]);
-      sED[j] = __expf(acc - lw[0]);
-      if (lw[0] - acc > kMaxChunkDecay) sflag[0] = 1;
-    } else {
-      for (int it = tid - kDK; it < kC * (NV / 8); it += kThreads - kDK) {
-        const int t = it / (NV / 8), g = it % (NV / 8);
-        float o8[8];
-        if (t < n) {
-          const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + c0 + 8 * g;
-          float v8[8], w8[8];
-          unpack8(ld16(gv + off), v8);
-          if (gw) {
-            unpack8(ld16(gw + off), w8);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w8[e] = 1.f;
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o8[e] = v8[e] * w8[e];
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) o8[e] = 0.f;
-        }
-        st_smem16(smem, SL::VH + sw128_offset(t, 8 * g, kC * 128), pack8(o8));
+    for (int u = 0; u < 4; ++u) {
+      const int it = tid + u * kThreads, t = it >> 4, g = it & 15;
+      if (t < n) {
+        const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + 8 * g;
+        rk[u] = ld16(gk + off);
+        rb[u] = ld16(gb + off);
+        rq[u] = ld16(gq + off);
+      } else {
+        rk[u] = rb[u] = rq[u] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    __syncthreads();
+    // value inputs: items (t, g < NV / 8), 2 per thread
+    constexpr int kVItems = kC * (NV / 8) / kThreads;
+    uint4 rv[kVItems], rw[kVItems];
+#pragma unroll
+    for (int u = 0; u < kVItems; ++u) {
+      const int it = tid + u * kThreads, t = it / (NV / 8), g = it % (NV / 8);
+      if (t < n) {
+        const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + c0 + 8 * g;
+        rv[u] = ld16(gv + off);
+        rw[u] = gw ? ld16(gw + off) : make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+      } else {
+        rv[u] = rw[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+
+    // ---- V^ = wg (.) v (needs no decay)
+#pragma unroll
+    for (int u = 0; u < kVItems; ++u) {
+      const int it = tid + u * kThreads, t = it / (NV / 8), g = it % (NV / 8);
+      float v8[8], w8[8];
+      unpack8(rv[u], v8);
+      unpack8(rw[u], w8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+      st_smem16(smem, SL::VH + sw128_offset(t, 8 * g, kC * 128), pack8(v8));
+    }
+
+    // ---- P0: cumulative log-decay Lam_t (two halves of the chunk, then joined)
+    {
+      float acc = 0.f;
+#pragma unroll
+      for (int t = 0; t < 32; ++t) {
+        acc += lw[t];
+        lw[t] = acc;
+      }
+      if (hh == 0) {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) sLam[t * kDK + jc] = lw[t];
+        sTot[jc] = acc;
+      }
+      __syncthreads();
+      if (hh == 1) {
+        const float base = sTot[jc], lam1 = sLam[jc];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) sLam[(32 + t) * kDK + jc] = base + lw[t];
+        const float lamn = base + acc;
+        sPiN[jc] = __expf(lamn);
+        sA1[jc] = __expf(lam1);
+        sED[jc] = __expf(lamn - lam1);
+        if (lam1 - lamn > kMaxChunkDecay) sflag[0] = 1;
+      }
+      __syncthreads();
+    }
     const bool exact = sflag[0] != 0;
 
     GDR_PHASE(0);
     // ---- P1: operand tiles [K^ f; Q f], K g, K~, Q_pi
-    for (int it = tid; it < kC * (kDK / 8); it += kThreads) {
-      const int t = it >> 4, g = it & 15, j0 = 8 * g;
-      float k8[8], b8[8], q8[8];
-      if (t < n) {
-        const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + j0;
-        unpack8(ld16(gk + off), k8);
-        unpack8(ld16(gb + off), b8);
-        unpack8(ld16(gq + off), q8);
-      } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) k8[e] = b8[e] = q8[e] = 0.f;
-      }
+    for (int u = 0; u < 4; ++u) {
+      const int it = tid + u * kThreads, t = it >> 4, g = it & 15, j0 = 8 * g;
+      float k8[8], b8[8], q8[8];
+      unpack8(rk[u], k8);
+      unpack8(rb[u], b8);
+      unpack8(rq[u], q8);
       const float4 *lp = reinterpret_cast<const float4 *>(sLam + t * kDK + j0);
       const float4 *l1p = reinterpret_cast<const float4 *>(sLam + j0);
       const float4 *ln = reinterpret_cast<const float4 *>(sLam + (kC - 1) * kDK + j0);
@@ -360,10 +420,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
       const int r = 32 * qd + lane;
       if (r < kC) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int s = 32 * hf + i;
-          sL[r * kLD + s] = (s < r) ? x[i] : 0.f;
-        }
+        for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i < r) ? x[i] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4 *>(sL + r * kLD + 32 * hf + i) =
+              make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
       } else {
         const int t = r - kC;
 #pragma unroll
@@ -400,11 +461,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     invert_unit_lower(sL, sTi, tid);
     for (int it = tid; it < kC * (kC / 8); it += kThreads) {
       const int t = it >> 3, g = it & 7;
-      float x[8];
+      const float4 y0 = *reinterpret_cast<const float4 *>(sTi + t * kLD + 8 * g);
+      const float4 y1 = *reinterpret_cast<const float4 *>(sTi + t * kLD + 8 * g + 4);
+      float x[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int s = 8 * g + e;
-        x[e] = (s < t) ? sTi[t * kLD + s] : (s == t ? 1.f : 0.f);
+        x[e] = (s < t) ? x[e] : (s == t ? 1.f : 0.f);
       }
       st_smem16(smem, SL::TINV + sw128_offset(t, 8 * g, kC * 128), pack8(x));
     }
