@@ -297,8 +297,16 @@ def bench_forward(ctx, args, gdr):
         raise RuntimeError(f"device status after the timed steps: {status}")
     ms_total = ctx.max_over_ranks(t0.elapsed_time(t1))
     ms_kernel = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    # launches per call: the tensor-core path with a full workspace runs a prep and a
+    # chain kernel; every other path is one kernel
+    full_ws = ws.numel() >= gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"],
+                                                            d["log_w"], d["e1"], d["e2"],
+                                                            w.chunk, "tc") > 256
+    per_call = 2 if (args.algo in ("auto", "tc") and full_ws and w.form == "gdn2"
+                     and w.dtype == "bf16" and w.dk == w.dv == 128 and w.chunk == 64) else 1
     res = {"w": w, "ms_per_step": ms_total / args.steps, "ms_kernel": ms_kernel,
-           "clocks": clk.summary(), "launches": args.steps}
+           "clocks": clk.summary(), "launches": args.steps * per_call,
+           "launches_per_call": per_call}
     if args.only == "all":
         res["e2e"] = bench_e2e(ctx, args, gdr, w, inp, names, step, o)
     return res
@@ -436,7 +444,10 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": ctx.peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / ctx.peaks["hbm_gbs"],
                          "traffic": None, "peak_source": ctx.peaks["source"],
-                         "bytes_per_launch": nbytes, "kernel_ms": fwd["ms_kernel"]},
+                         "bytes_per_launch": nbytes, "kernel_ms": fwd["ms_kernel"],
+                         "scope": "one forward call (%d kernel launch%s)" % (
+                             fwd["launches_per_call"],
+                             "es" if fwd["launches_per_call"] > 1 else "")},
             "tensor": {"flops_per_launch": nflops, "achieved_tflops": tflops,
                        "peak_tflops": ctx.peaks["bf16_tflops"],
                        "frac": tflops / ctx.peaks["bf16_tflops"]},

@@ -33,7 +33,35 @@ gdr_status check_token_ptrs(gdr_form form, size_t tokens, const void *q, const v
   return GDR_OK;
 }
 
-constexpr size_t kStatusBytes = 256;  // status word, padded to the workspace alignment
+using gdr::kStatusBytes;
+
+// FwdParams of a forward call (pointers as given).
+gdr::FwdParams fwd_params(const gdr_fwd_args *a) {
+  gdr::FwdParams p;
+  p.form = a->form;
+  p.B = a->B;
+  p.H = a->H;
+  p.T = a->T;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.chunk = a->chunk;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.e1 = a->e1;
+  p.e2 = a->e2;
+  p.log_w = a->log_w;
+  p.S0 = a->S0;
+  p.o = a->o;
+  p.S_T = a->S_T;
+  p.status = static_cast<uint32_t *>(a->workspace);
+  return p;
+}
+
+bool uses_tc(const gdr_fwd_args *a, const gdr::FwdParams &p) {
+  return (a->algo == GDR_ALGO_TC || a->algo == GDR_ALGO_AUTO) &&
+         gdr::forward_tc_supported(p, a->dtype);
+}
 
 }  // namespace
 
@@ -58,6 +86,10 @@ int gdr_version(void) { return 100; }
 gdr_status gdr_forward_workspace_size(const gdr_fwd_args *a, size_t *bytes) {
   if (!a || !bytes) return GDR_ERR_INVALID_ARG;
   *bytes = kStatusBytes;
+  if (a->B > 0 && a->H > 0 && a->T > 0 && dtype_ok(a->dtype) && form_ok(a->form)) {
+    const gdr::FwdParams p = fwd_params(a);
+    if (uses_tc(a, p)) *bytes = gdr::forward_tc_split_workspace_bytes(p);
+  }
   return GDR_OK;
 }
 
@@ -96,21 +128,15 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
     return gdr_state_init(a->S_T, a->B, a->H, a->dk, a->dv, a->S0, stream);
   }
 
-  gdr::FwdParams p;
-  p.form = a->form;
-  p.B = a->B; p.H = a->H; p.T = a->T; p.dk = a->dk; p.dv = a->dv; p.chunk = a->chunk;
-  p.q = a->q; p.k = a->k; p.v = a->v; p.e1 = a->e1;
-  p.e2 = a->e2;
-  p.log_w = a->log_w;
-  p.S0 = a->S0;
-  p.o = a->o;
-  p.S_T = a->S_T;
-  p.status = static_cast<uint32_t *>(a->workspace);
-
+  const gdr::FwdParams p = fwd_params(a);
   const bool tc_ok = gdr::forward_tc_supported(p, a->dtype);
   if (a->algo == GDR_ALGO_TC || (a->algo == GDR_ALGO_AUTO && tc_ok)) {
     if (!tc_ok) return GDR_ERR_UNSUPPORTED;
     if (!a->workspace || a->workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
+    // the two-kernel path when the workspace holds its per-chunk records, else the
+    // single-kernel path (status word only)
+    if (a->workspace_bytes >= gdr::forward_tc_split_workspace_bytes(p))
+      return cuda_status(gdr::launch_forward_tc_split(p, a->workspace, s));
     return cuda_status(gdr::launch_forward_tc(p, s));
   }
   if (!gdr::forward_fp32_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;

@@ -38,8 +38,7 @@
 //   MMA4  K~^T x V~,  M x V~                                     -> S_C increment, O
 // The fp32 state slice lives in registers (thread = key channel, 32 columns);
 // its bf16 copy in shared memory is the B operand of MMA3.
-#include "gdr_internal.cuh"
-#include "gdr_sm100.cuh"
+#include "gdr_tc_common.cuh"
 
 // Phase hooks for an external timing harness; empty in the library build.
 #ifndef GDR_PHASE
@@ -49,15 +48,9 @@
 namespace gdr {
 namespace {
 
-using namespace sm100;
 
-constexpr int kC = 64;
-constexpr int kDK = 128;
-constexpr int kThreads = 256;
-constexpr int kLD = kC + 4;                   // fp32 C x C row stride (16-byte rows)
-constexpr float kMaxChunkDecay = 80.f;        // nats
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
-constexpr uint32_t kTmemCols = 256;
+using namespace tc;
+using Ix = PaddedIdx;
 
 template <int NV>
 struct TcSmem {
@@ -72,9 +65,9 @@ struct TcSmem {
   static constexpr uint32_t S0B = VT + kC * NV * 2;             // bf16 S0       DK x NV
   static constexpr uint32_t QP = S0B + kDK * NV * 2;            // Q_pi          C x DK
   static constexpr uint32_t LAM = QP + kC * kDK * 2;            // fp32 Lambda   C x DK
-  static constexpr uint32_t LF = LAM + kC * kDK * 4;            // fp32 L        C x kLD
-  static constexpr uint32_t TI = LF + kC * kLD * 4;             // fp32 T^-1     C x kLD
-  static constexpr uint32_t PIN = TI + kC * kLD * 4;            // fp32 exp(Lam_n) DK
+  static constexpr uint32_t LF = LAM + kC * kDK * 4;            // fp32 L        (padded rows)
+  static constexpr uint32_t TI = LF + Ix::kBytes;               // fp32 T^-1     (padded rows)
+  static constexpr uint32_t PIN = TI + Ix::kBytes;              // fp32 exp(Lam_n) DK
   static constexpr uint32_t A1 = PIN + kDK * 4;                 // fp32 alpha_1 = exp(Lam_1) DK
   static constexpr uint32_t ED = A1 + kDK * 4;                  // fp32 exp(Lam_n - Lam_1) DK
   static constexpr uint32_t TOT = ED + kDK * 4;                 // fp32 first-half log-decay DK
@@ -86,123 +79,6 @@ struct TcSmem {
                     S0B % 1024 == 0 && QP % 1024 == 0,
                 "MMA tiles must be 1024-byte aligned");
 };
-
-__device__ __forceinline__ uint4 ld16(const __nv_bfloat16 *p) {
-  return __ldg(reinterpret_cast<const uint4 *>(p));
-}
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 x = __bfloat1622float2(h[i]);
-    f[2 * i] = x.x;
-    f[2 * i + 1] = x.y;
-  }
-}
-
-__device__ __forceinline__ uint32_t pack2(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ uint4 pack8(const float *f) {
-  return make_uint4(pack2(f[0], f[1]), pack2(f[2], f[3]), pack2(f[4], f[5]), pack2(f[6], f[7]));
-}
-
-__device__ __forceinline__ void st_smem16(uint8_t *base, uint32_t off, const uint4 &v) {
-  *reinterpret_cast<uint4 *>(base + off) = v;
-}
-
-// Bounded wait for the MMA group committed to `bar`: thread 0 polls the
-// mbarrier, then a CTA barrier passes the completion on (and makes every thread
-// take the same branch).  Returns false, with the shared abort flag set, when the
-// wait ran out.
-__device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t &phase, volatile int *abort) {
-  if (threadIdx.x == 0 && !mbar_wait_bounded(bar, phase, kWaitLimitNs)) *abort = 1;
-  phase ^= 1u;
-  __syncthreads();
-  tc_fence_after();
-  return *abort == 0;
-}
-
-// T^-1 for the unit lower-triangular T = I + L (L strictly lower, fp32, row stride
-// kLD), by blocks (eq. (11) of the Muir page): the four 16 x 16 diagonal blocks by
-// forward substitution, then two merge levels X21 = -T_R^-1 (L_RL T_L^-1).  Writes
-// all of Ti (zeros above the diagonal); overwrites the merged L_RL blocks of Lm
-// with the products L_RL T_L^-1.  All 256 threads; ends with a CTA barrier.
-__device__ void invert_unit_lower(float *Lm, float *Ti, int tid) {
-  if (tid < 64) {
-    const int blk = tid >> 4, c = tid & 15, o = 16 * blk;
-    float x[16];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      float acc = (t == c) ? 1.f : 0.f;
-#pragma unroll
-      for (int s = 0; s < t; ++s) acc -= Lm[(o + t) * kLD + o + s] * x[s];
-      x[t] = acc;
-    }
-#pragma unroll
-    for (int t = 0; t < 16; ++t) Ti[(o + t) * kLD + o + c] = x[t];
-  } else {
-    // zero the strictly-upper blocks the merge products read
-    for (int i = tid - 64; i < 32 * 32 + 2 * 16 * 16; i += kThreads - 64) {
-      int r, c;
-      if (i < 1024) { r = i >> 5; c = 32 + (i & 31); }
-      else { const int k = i - 1024, p = k >> 8; r = 32 * p + ((k >> 4) & 15); c = 32 * p + 16 + (k & 15); }
-      Ti[r * kLD + c] = 0.f;
-    }
-  }
-  __syncthreads();
-  // level 1: pairs (blocks 0,1) and (2,3).  Thread: pair p, row i, columns 2jq, 2jq+1.
-  {
-    const int p = tid >> 7, i = (tid >> 3) & 15, j = 2 * (tid & 7), o = 32 * p;
-    float w0 = 0.f, w1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float l = Lm[(o + 16 + i) * kLD + o + k];
-      const float2 t = *reinterpret_cast<const float2 *>(Ti + (o + k) * kLD + o + j);
-      w0 += l * t.x;
-      w1 += l * t.y;
-    }
-    __syncthreads();
-    *reinterpret_cast<float2 *>(Lm + (o + 16 + i) * kLD + o + j) = make_float2(w0, w1);
-    __syncthreads();
-    float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float t = Ti[(o + 16 + i) * kLD + o + 16 + k];
-      const float2 w = *reinterpret_cast<const float2 *>(Lm + (o + 16 + k) * kLD + o + j);
-      x0 += t * w.x;
-      x1 += t * w.y;
-    }
-    *reinterpret_cast<float2 *>(Ti + (o + 16 + i) * kLD + o + j) = make_float2(-x0, -x1);
-  }
-  __syncthreads();
-  // level 2: rows 32..63 x columns 0..31.  Thread: row i, columns 4jq .. 4jq+3.
-  {
-    const int i = tid >> 3, j = 4 * (tid & 7);
-    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const float l = Lm[(32 + i) * kLD + k];
-      const float4 t = *reinterpret_cast<const float4 *>(Ti + k * kLD + j);
-      w.x += l * t.x; w.y += l * t.y; w.z += l * t.z; w.w += l * t.w;
-    }
-    __syncthreads();
-    *reinterpret_cast<float4 *>(Lm + (32 + i) * kLD + j) = w;
-    __syncthreads();
-    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k < 32; ++k) {
-      const float t = Ti[(32 + i) * kLD + 32 + k];
-      const float4 v = *reinterpret_cast<const float4 *>(Lm + (32 + k) * kLD + j);
-      x.x += t * v.x; x.y += t * v.y; x.z += t * v.z; x.w += t * v.w;
-    }
-    *reinterpret_cast<float4 *>(Ti + (32 + i) * kLD + j) = make_float4(-x.x, -x.y, -x.z, -x.w);
-  }
-  __syncthreads();
-}
 
 template <int NV>
 __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
@@ -423,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
         for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i < r) ? x[i] : 0.f;
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4 *>(sL + r * kLD + 32 * hf + i) =
+          *reinterpret_cast<float4 *>(sL + Ix::at(r, 32 * hf + i)) =
               make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
       } else {
         const int t = r - kC;
@@ -449,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
             l += __bfloat162float(gb[ot + j]) * __bfloat162float(gk[ot + j]) * d * ks;
           }
         }
-        sL[t * kLD + s] = (s < t) ? l : 0.f;
+        sL[Ix::at(t, s)] = (s < t) ? l : 0.f;
         *reinterpret_cast<__nv_bfloat16 *>(smem + SL::MM + sw128_offset(t, s, kC * 128)) =
             __float2bfloat16_rn(m);
       }
@@ -458,11 +334,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
 
     GDR_PHASE(3);
     // ---- T^-1 (fp32), then bf16 copy as the A operand of MMA2
-    invert_unit_lower(sL, sTi, tid);
+    invert_unit_lower<Ix, Ix>(sL, sTi, tid);
     for (int it = tid; it < kC * (kC / 8); it += kThreads) {
       const int t = it >> 3, g = it & 7;
-      const float4 y0 = *reinterpret_cast<const float4 *>(sTi + t * kLD + 8 * g);
-      const float4 y1 = *reinterpret_cast<const float4 *>(sTi + t * kLD + 8 * g + 4);
+      const float4 y0 = *reinterpret_cast<const float4 *>(sTi + Ix::at(t, 8 * g));
+      const float4 y1 = *reinterpret_cast<const float4 *>(sTi + Ix::at(t, 8 * g + 4));
       float x[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {

@@ -1,0 +1,602 @@
+// gdr_fwd_tc_split.cu -- chunked forward on the tensor cores as two kernels.
+//
+// Same algorithm and numerics as gdr_fwd_tc.cu ("Muir: Linear Attention with
+// Sensitivity-Allocated Gating and Matched-Filter Readout", section 2.2 and
+// section 4.2; GDN-2 form, bf16 inputs, d_k = d_v = 128, C = 64), split where the
+// chunkwise form itself splits:
+//
+//  * prep: everything that does not depend on the chunk's initial state S0 --
+//    the cumulative log-decay, the decay-weighted products L and M (one tcgen05
+//    MMA), T^-1 (fp32), U = T^-1 V^ and Y = T^-1 K^_pi (one MMA group), and the
+//    operand tiles Q_pi and K~.  Chunks are independent, so one CTA per
+//    (b, h, chunk) runs them all in parallel (about 107 KB of shared memory, two
+//    CTAs per SM).  Each CTA writes a record of bf16 MMA tiles, already in the
+//    128-byte-swizzled shared-memory layout, to the workspace.
+//  * chain: the inter-chunk state carry and the outputs, sequential over chunks
+//    for each (b, h, 64-column value slice):
+//        V~ = U - Y S0,   S_C = Diag(pi_n) S0 + K~^T V~,   O = Q_pi S0 + M V~.
+//    Records are fetched with bulk (TMA) copies two chunks ahead into a
+//    double buffer, so every chunk step is two MMA groups and two short
+//    CUDA-core phases.
+//
+// The workspace holds one record (74752 bytes) per (b, h, chunk) after a
+// 1024-byte header whose first word is the device status word.
+#include "gdr_tc_common.cuh"
+
+namespace gdr {
+namespace {
+
+using namespace tc;
+using Ix = SwizzledIdx;
+
+// One chunk's record: bf16 tiles in the sw128 layout (64-column blocks of C*128 B).
+struct Rec {
+  static constexpr uint32_t Y = 0;                     // Y       C x DK  (K-major A of Y S0)
+  static constexpr uint32_t QP = Y + kC * kDK * 2;      // Q_pi    C x DK  (K-major A of Q S0)
+  static constexpr uint32_t KT = QP + kC * kDK * 2;     // K~      C x DK  (MN-major A of K~^T V~)
+  static constexpr uint32_t MM = KT + kC * kDK * 2;     // M       C x C   (K-major A of M V~)
+  static constexpr uint32_t U = MM + kC * kC * 2;       // U       C x DV  (rows = tokens)
+  static constexpr uint32_t PI = U + kC * kDK * 2;      // exp(Lam_n), DK fp32
+  static constexpr uint32_t BYTES = PI + 1024;
+  static constexpr uint32_t FRONT = U;                  // Y | QP | KT | MM, copied as one block
+  static_assert(Y % 1024 == 0 && QP % 1024 == 0 && KT % 1024 == 0 && MM % 1024 == 0 &&
+                    U % 1024 == 0 && PI % 1024 == 0 && BYTES % 1024 == 0,
+                "record tiles must stay 1024-byte aligned");
+};
+constexpr size_t kHeaderBytes = 1024;
+
+__host__ __device__ inline int num_chunks(int T) { return (T + kC - 1) / kC; }
+
+// ============================================================== prep kernel
+// fp32 64 x 64 T^-1 in the Q rows of the [K^ f; Q f] tile once MMA1 has read them:
+// those rows are two 8 KB pieces (one per 64-column atom), rows 0..31 in the
+// first and 32..63 in the second; 16-byte groups XOR-permuted by (r & 15).
+struct QRowsIdx {
+  static __device__ __forceinline__ int at(int r, int s) {
+    return (r < 32 ? kC * 32 : kC * 96) + (r & 31) * kC + ((((s >> 2) ^ (r & 15))) << 2) + (s & 3);
+  }
+};
+
+struct PrepSmem {
+  static constexpr uint32_t A_LM = 0;                       // [K^ f; Q f]  2C x DK bf16; Q rows
+                                                            //   then hold fp32 T^-1 (QRowsIdx)
+  static constexpr uint32_t B_LM = A_LM + 2 * kC * kDK * 2;  // K g          C x DK bf16; then fp32 L
+  static constexpr uint32_t VH = B_LM + kC * kDK * 2;        // V^           C x DV bf16
+  static constexpr uint32_t TINV = VH + kC * kDK * 2;        // T^-1         C x C bf16
+  static constexpr uint32_t LAM = TINV + kC * kC * 2;        // fp32 Lambda  C x DK
+  static constexpr uint32_t A1 = LAM + kC * kDK * 4;         // fp32 alpha_1       DK
+  static constexpr uint32_t ED = A1 + kDK * 4;               // fp32 exp(Lam_n - Lam_1)
+  static constexpr uint32_t PIN = ED + kDK * 4;              // fp32 exp(Lam_n)
+  static constexpr uint32_t TOT = PIN + kDK * 4;             // fp32 first-half log-decay
+  static constexpr uint32_t MISC = TOT + kDK * 4;            // mbarrier, TMEM slot, flags
+  static constexpr uint32_t ALLOC = MISC + 64 + 1024;
+  static_assert(Ix::kBytes <= kC * kDK * 2, "fp32 L / T^-1 must fit the reused bf16 tiles");
+};
+
+__global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8_t *records) {
+  using SL = PrepSmem;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sb = smem_u32(smem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hf = warp >> 2;
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int T = p.T, H = p.H, t0 = c * kC, n = min(kC, T - t0);
+  uint8_t *rec = records + ((size_t)((size_t)b * H + h) * num_chunks(T) + c) * Rec::BYTES;
+
+  float *sLam = reinterpret_cast<float *>(smem + SL::LAM);
+  float *sL = reinterpret_cast<float *>(smem + SL::B_LM);
+  float *sTi = reinterpret_cast<float *>(smem + SL::A_LM);
+  float *sA1 = reinterpret_cast<float *>(smem + SL::A1);
+  float *sED = reinterpret_cast<float *>(smem + SL::ED);
+  float *sPiN = reinterpret_cast<float *>(smem + SL::PIN);
+  float *sTot = reinterpret_cast<float *>(smem + SL::TOT);
+  uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + SL::MISC);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 8);
+  volatile int *sflag = reinterpret_cast<volatile int *>(smem + SL::MISC + 16);  // exact, abort
+
+  const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
+  const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
+  const __nv_bfloat16 *gv = static_cast<const __nv_bfloat16 *>(p.v);
+  const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
+  const __nv_bfloat16 *gw = static_cast<const __nv_bfloat16 *>(p.e2);
+
+  // ---- global reads first: log w (channel jc, half hh) and the k, b, q items
+  const int jc = tid & (kDK - 1), hh = tid >> 7;
+  float lw[32];
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    const int tt = 32 * hh + t;
+    lw[t] = (tt < n) ? __ldg(p.log_w + (((size_t)b * T + t0 + tt) * H + h) * kDK + jc) : 0.f;
+  }
+  uint4 rk[4], rb[4], rq[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int it = tid + u * kThreads, t = it >> 4, g = it & 15;
+    if (t < n) {
+      const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + 8 * g;
+      rk[u] = ld16(gk + off);
+      rb[u] = ld16(gb + off);
+      rq[u] = ld16(gq + off);
+    } else {
+      rk[u] = rb[u] = rq[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(mbar, 1);
+    fence_mbar_init();
+    sflag[0] = 0;
+    sflag[1] = 0;
+  }
+
+  // ---- cumulative log-decay Lam_t (two halves of the chunk, then joined)
+  {
+    float acc = 0.f;
+#pragma unroll
+    for (int t = 0; t < 32; ++t) {
+      acc += lw[t];
+      lw[t] = acc;
+    }
+    if (hh == 0) {
+#pragma unroll
+      for (int t = 0; t < 32; ++t) sLam[t * kDK + jc] = lw[t];
+      sTot[jc] = acc;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (hh == 1) {
+      const float base = sTot[jc], lam1 = sLam[jc];
+#pragma unroll
+      for (int t = 0; t < 32; ++t) sLam[(32 + t) * kDK + jc] = base + lw[t];
+      const float lamn = base + acc;
+      sPiN[jc] = __expf(lamn);
+      sA1[jc] = __expf(lam1);
+      sED[jc] = __expf(lamn - lam1);
+      if (lam1 - lamn > kMaxChunkDecay) sflag[0] = 1;
+    }
+  }
+  // ---- V^ = wg (.) v over the full d_v
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int it = tid + u * kThreads, t = it >> 4, g = it & 15;
+    float v8[8], w8[8];
+    if (t < n) {
+      const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + 8 * g;
+      unpack8(ld16(gv + off), v8);
+      if (gw) {
+        unpack8(ld16(gw + off), w8);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w8[e] = 1.f;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v8[e] = w8[e] = 0.f;
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+    st_smem16(smem, SL::VH + sw128_offset(t, 8 * g, kC * 128), pack8(v8));
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool exact = sflag[0] != 0;
+
+  // ---- operand tiles: [K^ f; Q f], K g in shared memory; Q_pi, K~ straight to the record
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int it = tid + u * kThreads, t = it >> 4, g = it & 15, j0 = 8 * g;
+    float k8[8], b8[8], q8[8];
+    unpack8(rk[u], k8);
+    unpack8(rb[u], b8);
+    unpack8(rq[u], q8);
+    const float4 *lp = reinterpret_cast<const float4 *>(sLam + t * kDK + j0);
+    const float4 *l1p = reinterpret_cast<const float4 *>(sLam + j0);
+    const float4 *ln = reinterpret_cast<const float4 *>(sLam + (kC - 1) * kDK + j0);
+    const float4 l0 = lp[0], l1 = lp[1], f0 = l1p[0], f1 = l1p[1], n0 = ln[0], n1 = ln[1];
+    const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+    const float lam1[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
+    const float lamn[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+    float a1[8], a2[8], bl[8], kt[8], qp[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float f = __expf(lam[e] - lam1[e]);
+      a1[e] = b8[e] * k8[e] * f;
+      a2[e] = q8[e] * f;
+      qp[e] = a2[e] * sA1[j0 + e];
+      if (!exact) {
+        bl[e] = k8[e] * __expf(lam1[e] - lam[e]);
+        kt[e] = bl[e] * sED[j0 + e];
+      } else {
+        bl[e] = 0.f;
+        kt[e] = k8[e] * __expf(lamn[e] - lam[e]);
+      }
+    }
+    const uint32_t o64 = sw128_offset(t, j0, kC * 128);
+    st_smem16(smem, SL::A_LM + sw128_offset(t, j0, 2 * kC * 128), pack8(a1));
+    st_smem16(smem, SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128), pack8(a2));
+    st_smem16(smem, SL::B_LM + o64, pack8(bl));
+    *reinterpret_cast<uint4 *>(rec + Rec::QP + o64) = pack8(qp);
+    *reinterpret_cast<uint4 *>(rec + Rec::KT + o64) = pack8(kt);
+  }
+  fence_proxy_async_smem();
+  __syncthreads();
+
+  uint32_t phase = 0;
+  bool ok = true;
+  // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
+  if (tid == 0) {
+    tc_fence_after();
+    constexpr uint32_t id = idesc_bf16_f32(128, kC, false, false);
+#pragma unroll
+    for (int s = 0; s < kDK / 16; ++s) {
+      const uint64_t ad = sdesc_sw128(sb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
+      const uint64_t bd = sdesc_sw128(sb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
+      mma_bf16(tmem, ad, bd, id, s > 0);
+    }
+    mma_commit(mbar);
+  }
+  ok = wait_mma(mbar, phase, sflag + 1);
+
+  if (ok) {
+    // ---- L (fp32, strictly lower; into the dead K g tile) and M (bf16 -> record)
+    if (!exact) {
+      float x[32];
+      tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * hf, x);
+      tmem_ld_wait();
+      const int r = 32 * qd + lane;
+      if (r < kC) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i < r) ? x[i] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4 *>(sL + Ix::at(r, 32 * hf + i)) =
+              make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+      } else {
+        const int t = r - kC;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i <= t) ? x[i] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4 *>(rec + Rec::MM + sw128_offset(t, 32 * hf + i, kC * 128)) =
+              pack8(x + i);
+      }
+    } else {
+      // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound)
+      for (int it = tid; it < kC * kC; it += kThreads) {
+        const int t = it / kC, s = it % kC;
+        float l = 0.f, m = 0.f;
+        if (s <= t && t < n) {
+          const size_t ot = (((size_t)b * T + t0 + t) * H + h) * kDK;
+          const size_t os = (((size_t)b * T + t0 + s) * H + h) * kDK;
+          for (int j = 0; j < kDK; ++j) {
+            const float d = __expf(sLam[t * kDK + j] - sLam[s * kDK + j]);
+            const float ks = __bfloat162float(gk[os + j]);
+            m += __bfloat162float(gq[ot + j]) * d * ks;
+            l += __bfloat162float(gb[ot + j]) * __bfloat162float(gk[ot + j]) * d * ks;
+          }
+        }
+        sL[Ix::at(t, s)] = (s < t) ? l : 0.f;
+        *reinterpret_cast<__nv_bfloat16 *>(rec + Rec::MM + sw128_offset(t, s, kC * 128)) =
+            __float2bfloat16_rn(m);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- T^-1 (fp32, into the dead Q f half of A_LM), bf16 copy for MMA2
+    invert_unit_lower<Ix, QRowsIdx>(sL, sTi, tid);
+    for (int it = tid; it < kC * (kC / 8); it += kThreads) {
+      const int t = it >> 3, g = it & 7;
+      const float4 y0 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * g));
+      const float4 y1 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * g + 4));
+      float x[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int s = 8 * g + e;
+        x[e] = (s < t) ? x[e] : (s == t ? 1.f : 0.f);
+      }
+      st_smem16(smem, SL::TINV + sw128_offset(t, 8 * g, kC * 128), pack8(x));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16_f32(64, kDK, false, true);
+#pragma unroll
+      for (int s = 0; s < kC / 16; ++s) {
+        const uint64_t ad = sdesc_sw128(sb + SL::TINV + s * 32, 16, 1024);
+        const uint64_t bu = sdesc_sw128(sb + SL::VH + s * 2048, kC * 128, 1024);
+        const uint64_t by = sdesc_sw128(sb + SL::A_LM + s * 2048, 2 * kC * 128, 1024);
+        mma_bf16(tmem, ad, bu, id, s > 0);
+        mma_bf16(tmem + kDK, ad, by, id, s > 0);
+      }
+      mma_commit(mbar);
+    }
+    ok = wait_mma(mbar, phase, sflag + 1);
+  }
+
+  if (ok) {
+    // ---- U and Y (x alpha_1) -> bf16 record tiles; M = 64 accumulators: row 16 qd + lane
+    const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
+    float x[32];
+#pragma unroll
+    for (int part = 0; part < 4; ++part) {
+      const int col = 64 * hf + 32 * (part & 1);        // 0..127 within U or Y
+      const bool is_y = part >= 2;
+      tmem_ld_32x32b_x32(tmem + lane_q + (is_y ? kDK : 0) + col, x);
+      tmem_ld_wait();
+      if (lane < 16) {
+        const int t = 16 * qd + lane;
+        if (is_y) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] *= sA1[col + i];
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4 *>(rec + (is_y ? Rec::Y : Rec::U) +
+                                     sw128_offset(t, col + i, kC * 128)) = pack8(x + i);
+      }
+    }
+    if (tid < kDK) reinterpret_cast<float *>(rec + Rec::PI)[tid] = sPiN[tid];
+  } else if (tid == 0 && p.status) {
+    atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ============================================================== chain kernel
+template <int NV>
+struct ChainSmem {
+  // per buffer: Y | QP | KT | MM (as in the record) | U slice (C x NV) | pi
+  static constexpr uint32_t B_U = Rec::FRONT;
+  static constexpr uint32_t B_PI = B_U + kC * NV * 2;
+  static constexpr uint32_t BUF = ((B_PI + kDK * 4 + 1023) / 1024) * 1024;
+  static constexpr uint32_t S0B = 2 * BUF;                    // bf16 S0   DK x NV
+  static constexpr uint32_t VT = S0B + kDK * NV * 2;          // bf16 V~   C x NV
+  static constexpr uint32_t MISC = VT + kC * NV * 2;          // full[2], mma, TMEM slot, abort
+  static constexpr uint32_t ALLOC = MISC + 64 + 1024;
+  static constexpr uint32_t TX = Rec::FRONT + kC * NV * 2 + kDK * 4;  // bytes per record fetch
+  static_assert(NV == 64, "one 64-column block of U per CTA");
+};
+
+template <int NV>
+__global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, const uint8_t *records) {
+  using SL = ChainSmem<NV>;
+  constexpr int HALF = NV / 2;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  const uint32_t sb = smem_u32(smem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int qd = warp & 3, hf = warp >> 2;
+  const int slice = blockIdx.x, c0 = slice * NV, h = blockIdx.y, b = blockIdx.z;
+  const int T = p.T, H = p.H, nch = num_chunks(T);
+  const uint8_t *recs = records + (size_t)((size_t)b * H + h) * nch * Rec::BYTES;
+
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::MISC);       // [2]
+  uint64_t *mbar = full + 2;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 24);
+  volatile int *sabort = reinterpret_cast<volatile int *>(smem + SL::MISC + 32);
+
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(full, 1);
+    mbar_init(full + 1, 1);
+    mbar_init(mbar, 1);
+    fence_mbar_init();
+    *sabort = 0;
+  }
+  uint32_t fissue[2] = {0u, 0u}, fdone[2] = {0u, 0u};   // thread 0's fetch bookkeeping
+  if (tid == 0) {
+    for (int cc = 0; cc < 2 && cc < nch; ++cc) {
+      ++fissue[cc];
+      uint8_t *dst = smem + cc * SL::BUF;
+      const uint8_t *src = recs + (size_t)cc * Rec::BYTES;
+      mbar_arrive_expect_tx(full + cc, SL::TX);
+      bulk_g2s(dst, src, Rec::FRONT, full + cc);
+      bulk_g2s(dst + SL::B_U, src + Rec::U + slice * (kC * 128), kC * NV * 2, full + cc);
+      bulk_g2s(dst + SL::B_PI, src + Rec::PI, kDK * 4, full + cc);
+    }
+  }
+
+  // fp32 state: key channel jrow, value columns [hf*HALF, hf*HALF + HALF) of this slice
+  const int jrow = 32 * qd + lane;
+  const size_t s_off = (((size_t)b * H + h) * kDK + jrow) * kDK + c0 + hf * HALF;
+  float st[HALF];
+#pragma unroll
+  for (int i = 0; i < HALF; i += 4) {
+    float4 x = p.S0 ? __ldg(reinterpret_cast<const float4 *>(p.S0 + s_off + i))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+    st[i] = x.x; st[i + 1] = x.y; st[i + 2] = x.z; st[i + 3] = x.w;
+  }
+#pragma unroll
+  for (int i = 0; i < HALF; i += 8)
+    st_smem16(smem, SL::S0B + sw128_offset(jrow, hf * HALF + i, kDK * 128), pack8(st + i));
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tD1 = tmem, tDO = tmem + 64, tDS = tmem + 128;
+  const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
+
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int c = 0; c < nch && ok; ++c) {
+    const int buf = c & 1, t0 = c * kC, n = min(kC, T - t0);
+    const uint32_t bb = sb + buf * SL::BUF;
+    uint8_t *bsm = smem + buf * SL::BUF;
+    // ---- record of chunk c present?
+    if (tid == 0) {
+      if (mbar_wait_bounded(full + buf, (c >> 1) & 1, kWaitLimitNs)) ++fdone[buf];
+      else *sabort = 1;
+    }
+    __syncthreads();
+    if (*sabort) { ok = false; break; }
+    const float pn = reinterpret_cast<const float *>(bsm + SL::B_PI)[jrow];
+
+    // ---- MMA3: Y S0 and Q_pi S0 (K = DK)
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16_f32(64, NV, false, true);
+#pragma unroll
+      for (int s = 0; s < kDK / 16; ++s) {
+        const uint32_t ko = (s >> 2) * (kC * 128) + (s & 3) * 32;
+        const uint64_t ay = sdesc_sw128(bb + Rec::Y + ko, 16, 1024);
+        const uint64_t aq = sdesc_sw128(bb + Rec::QP + ko, 16, 1024);
+        const uint64_t bs = sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
+        mma_bf16(tD1, ay, bs, id, s > 0);
+        mma_bf16(tDO, aq, bs, id, s > 0);
+      }
+      mma_commit(mbar);
+    }
+    if (!(ok = wait_mma(mbar, phase, sabort))) break;
+
+    // ---- V~ = U - Y S0 -> bf16 (rows = tokens)
+    {
+      float d[32];
+      tmem_ld_32x32b_x32(tD1 + lane_q + hf * HALF, d);
+      tmem_ld_wait();
+      if (lane < 16) {
+        const int t = 16 * qd + lane;
+        float u[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+          float u8[8];
+          unpack8(*reinterpret_cast<const uint4 *>(bsm + SL::B_U +
+                                                  sw128_offset(t, hf * HALF + i, kC * 128)), u8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) u[i + e] = (t < n) ? u8[e] - d[i + e] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          st_smem16(smem, SL::VT + sw128_offset(t, hf * HALF + i, kC * 128), pack8(u + i));
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- MMA4: K~^T V~ (M = DK) and O += M V~ (M = C); K = C
+    if (tid == 0) {
+      tc_fence_after();
+      constexpr uint32_t ids = idesc_bf16_f32(128, NV, true, true);
+      constexpr uint32_t ido = idesc_bf16_f32(64, NV, false, true);
+#pragma unroll
+      for (int s = 0; s < kC / 16; ++s) {
+        const uint64_t ak = sdesc_sw128(bb + Rec::KT + s * 2048, kC * 128, 1024);
+        const uint64_t bv = sdesc_sw128(sb + SL::VT + s * 2048, kC * 128, 1024);
+        const uint64_t am = sdesc_sw128(bb + Rec::MM + s * 32, 16, 1024);
+        mma_bf16(tDS, ak, bv, ids, s > 0);
+        mma_bf16(tDO, am, bv, ido, 1);
+      }
+      mma_commit(mbar);
+    }
+    if (!(ok = wait_mma(mbar, phase, sabort))) break;
+
+    // ---- the buffer is free: fetch chunk c + 2
+    if (tid == 0 && c + 2 < nch) {
+      fence_proxy_async_smem();   // this CTA's reads of the buffer come before the refill
+      ++fissue[buf];
+      const uint8_t *src = recs + (size_t)(c + 2) * Rec::BYTES;
+      mbar_arrive_expect_tx(full + buf, SL::TX);
+      bulk_g2s(bsm, src, Rec::FRONT, full + buf);
+      bulk_g2s(bsm + SL::B_U, src + Rec::U + slice * (kC * 128), kC * NV * 2, full + buf);
+      bulk_g2s(bsm + SL::B_PI, src + Rec::PI, kDK * 4, full + buf);
+    }
+
+    // ---- state update (fp32) and outputs
+    {
+      float d[32];
+      tmem_ld_32x32b_x32(tDS + lane_q + hf * HALF, d);
+      tmem_ld_wait();
+#pragma unroll
+      for (int i = 0; i < HALF; ++i) st[i] = pn * st[i] + d[i];
+#pragma unroll
+      for (int i = 0; i < HALF; i += 8)
+        st_smem16(smem, SL::S0B + sw128_offset(jrow, hf * HALF + i, kDK * 128), pack8(st + i));
+      float o[32];
+      tmem_ld_32x32b_x32(tDO + lane_q + hf * HALF, o);
+      tmem_ld_wait();
+      if (lane < 16) {
+        const int t = 16 * qd + lane;
+        if (t < n) {
+          float4 *dst = reinterpret_cast<float4 *>(
+              p.o + (((size_t)b * T + t0 + t) * H + h) * kDK + c0 + hf * HALF);
+#pragma unroll
+          for (int i = 0; i < HALF; i += 4) dst[i / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+  }
+
+  if (ok && p.S_T) {
+#pragma unroll
+    for (int i = 0; i < HALF; i += 4)
+      *reinterpret_cast<float4 *>(p.S_T + s_off + i) = make_float4(st[i], st[i + 1], st[i + 2], st[i + 3]);
+  }
+  if (!ok && tid == 0) {
+    if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
+    // let MMAs and record copies already in flight land before the CTA exits
+    mbar_wait_bounded(mbar, phase, kWaitLimitNs);
+    for (int bq = 0; bq < 2; ++bq)
+      while (fdone[bq] < fissue[bq]) {
+        if (!mbar_wait_bounded(full + bq, fdone[bq] & 1, kWaitLimitNs)) break;
+        ++fdone[bq];
+      }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+size_t forward_tc_split_workspace_bytes(const FwdParams &p) {
+  return kHeaderBytes + (size_t)p.B * p.H * num_chunks(p.T) * Rec::BYTES;
+}
+
+cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStream_t stream) {
+  constexpr int NV = 64;
+  uint8_t *records = static_cast<uint8_t *>(workspace) + kHeaderBytes;
+  cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)PrepSmem::ALLOC);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(tc_chain_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)ChainSmem<NV>::ALLOC);
+  if (e != cudaSuccess) return e;
+  dim3 gp(num_chunks(p.T), p.H, p.B);
+  tc_prep_kernel<<<gp, kThreads, PrepSmem::ALLOC, stream>>>(p, records);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  dim3 gc(p.dv / NV, p.H, p.B);
+  tc_chain_kernel<NV><<<gc, kThreads, ChainSmem<NV>::ALLOC, stream>>>(p, records);
+  return cudaGetLastError();
+}
+
+}  // namespace gdr

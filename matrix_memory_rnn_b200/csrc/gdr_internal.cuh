@@ -64,6 +64,12 @@ cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_
 bool forward_fp32_supported(int dk, int dv);
 cudaError_t launch_forward_tc(const FwdParams &p, cudaStream_t stream);
 bool forward_tc_supported(const FwdParams &p, gdr_dtype dtype);
+// Two-kernel tensor-core path: per-chunk records in the workspace.
+size_t forward_tc_split_workspace_bytes(const FwdParams &p);
+cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStream_t stream);
+
+// Smallest workspace any forward path accepts (the device status word, padded).
+constexpr size_t kStatusBytes = 256;
 size_t forward_fp32_smem_bytes(int dk, int dv, int chunk);
 
 }  // namespace gdr

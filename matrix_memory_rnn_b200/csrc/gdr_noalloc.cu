@@ -49,10 +49,11 @@ gdr_status scratch_for_current_device(void **out) {
 
 extern "C" gdr_status gdr_forward_chunked_noalloc(const gdr_fwd_args *args, void *stream) {
   if (!args) return GDR_ERR_INVALID_ARG;
-  size_t need = 0;
-  gdr_status st = gdr_forward_workspace_size(args, &need);
-  if (st != GDR_OK) return st;
+  // The smallest workspace gdr_forward_chunked accepts: with it the tensor-core
+  // path runs as a single kernel (the two-kernel path needs per-chunk records).
+  const size_t need = gdr::kStatusBytes;
   if (need > kNoAllocScratchBytes) return GDR_ERR_WORKSPACE;
+  gdr_status st = GDR_OK;
   void *scratch = nullptr;
   st = scratch_for_current_device(&scratch);
   if (st != GDR_OK) return st;

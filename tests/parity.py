@@ -43,13 +43,17 @@ def oracle_forward(w, inp, S0=None, heads=None):
     return outs
 
 
-def gpu_forward(w, inp, algo="auto", chunk=None, S0=None, device="cuda"):
+def gpu_forward(w, inp, algo="auto", chunk=None, S0=None, device="cuda", workspace_bytes=None):
+    """``workspace_bytes`` = None sizes the workspace with gdr_forward_workspace_size (the
+    fastest path); a small value (e.g. 256) selects the single-kernel tensor-core path."""
     d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, w.dtype,
                       device)
     s0 = inp.get("S0") if S0 is None else S0
     s0 = None if s0 is None else torch.from_numpy(np.ascontiguousarray(s0, np.float32)).to(device)
+    ws = None if workspace_bytes is None else gdr.new_workspace(workspace_bytes, device)
     o, S_T = gdr.gdr_forward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
-                                     d["e2"], s0, chunk=chunk or w.chunk, algo=algo)
+                                     d["e2"], s0, chunk=chunk or w.chunk, algo=algo,
+                                     workspace=ws)
     torch.cuda.synchronize()
     return o.cpu().numpy(), S_T.cpu().numpy()
 

@@ -125,22 +125,40 @@ def test_eviction_on_gpu():
     assert abs(ratio - (1 - c) ** T) < 1e-5
 
 
+# the two tensor-core paths: "split" (prep + chain kernels, full workspace) and
+# "fused" (one kernel, the 256-byte minimum workspace)
+TC_PATHS = {"split": None, "fused": 256}
+
+
+@pytest.mark.parametrize("path", sorted(TC_PATHS))
 @pytest.mark.parametrize("T", [1, 64, 100, 257])
 @pytest.mark.parametrize("with_state", [False, True])
-def test_tc_kernel_gdn2(T, with_state):
-    """Tensor-core kernel (GDN-2, bf16, d = 128, C = 64) against the oracle, with a ragged tail."""
+def test_tc_kernel_gdn2(T, with_state, path):
+    """Tensor-core kernels (GDN-2, bf16, d = 128, C = 64) against the oracle, with a ragged tail."""
     w = small("gdn2", "bf16", dk=128, dv=128, T=T, B=2, H=3, chunk=64)
     inp = synth.forward_inputs(w)
     if with_state:
         inp["S0"] = synth.round_f32(np.random.default_rng(7).normal(0, 0.5, (w.B, w.H, 128, 128)))
-    o, S = gpu_forward(w, inp, algo="tc")
+    o, S = gpu_forward(w, inp, algo="tc", workspace_bytes=TC_PATHS[path])
     o_ref, S_ref = oracle_forward(w, inp)
     eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
-    print(f"tc T={T} S0={with_state}: o {eo:.3e} S {es:.3e}")
+    print(f"tc-{path} T={T} S0={with_state}: o {eo:.3e} S {es:.3e}")
     assert eo < TOL["bf16"] and es < TOL["bf16"]
 
 
-def test_tc_kernel_strong_decay_uses_exact_path():
+@pytest.mark.parametrize("path", sorted(TC_PATHS))
+def test_tc_full_size_gdn2(path):
+    w = synth.PRESETS["gdn2_bf16"]
+    inp = synth.forward_inputs(w)
+    o, S = gpu_forward(w, inp, algo="tc", workspace_bytes=TC_PATHS[path])
+    o_ref, S_ref = oracle_forward(w, inp)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    print(f"tc-{path} gdn2_bf16: o {eo:.3e} S {es:.3e}")
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
+@pytest.mark.parametrize("path", sorted(TC_PATHS))
+def test_tc_kernel_strong_decay_uses_exact_path(path):
     """Channels whose decay over a chunk exceeds e^-80 take the exact pairwise path."""
     w = small("gdn2", "bf16", dk=128, dv=128, T=200, B=1, H=2, chunk=64)
     inp = synth.forward_inputs(w)
@@ -148,7 +166,7 @@ def test_tc_kernel_strong_decay_uses_exact_path():
     lw[:, :, :, ::7] = -3.0          # 64 tokens x 3 nats = 192 nats per chunk on these channels
     lw[:, 70:80, 1, 5] = -60.0       # a burst of very strong decay on one head
     inp["log_w"] = lw.astype(np.float32)
-    o, S = gpu_forward(w, inp, algo="tc")
+    o, S = gpu_forward(w, inp, algo="tc", workspace_bytes=TC_PATHS[path])
     o_ref, S_ref = oracle_forward(w, inp)
     eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
     print(f"tc strong decay: o {eo:.3e} S {es:.3e}")
