@@ -23,6 +23,14 @@
 // 1024-byte header whose first word is the device status word.
 #include "gdr_tc_common.cuh"
 
+// Phase hooks for an external timing harness; empty in the library build.
+#ifndef GDR_PREP_PHASE
+#define GDR_PREP_PHASE(i)
+#endif
+#ifndef GDR_CHAIN_PHASE
+#define GDR_CHAIN_PHASE(i)
+#endif
+
 namespace gdr {
 namespace {
 
@@ -136,6 +144,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     sflag[1] = 0;
   }
 
+  GDR_PREP_PHASE(0);
   // ---- cumulative log-decay Lam_t (two halves of the chunk, then joined)
   {
     float acc = 0.f;
@@ -162,6 +171,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
       if (lam1 - lamn > kMaxChunkDecay) sflag[0] = 1;
     }
   }
+  GDR_PREP_PHASE(1);
   // ---- V^ = wg (.) v over the full d_v
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -189,6 +199,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   const uint32_t tmem = *tmem_slot;
   const bool exact = sflag[0] != 0;
 
+  GDR_PREP_PHASE(2);
   // ---- operand tiles: [K^ f; Q f], K g in shared memory; Q_pi, K~ straight to the record
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -231,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
 
   uint32_t phase = 0;
   bool ok = true;
+  GDR_PREP_PHASE(3);
   // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
   if (tid == 0) {
     tc_fence_after();
@@ -246,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   ok = wait_mma(mbar, phase, sflag + 1);
 
   if (ok) {
+    GDR_PREP_PHASE(4);
     // ---- L (fp32, strictly lower; into the dead K g tile) and M (bf16 -> record)
     if (!exact) {
       float x[32];
@@ -291,6 +304,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     tc_fence_before();
     __syncthreads();
 
+    GDR_PREP_PHASE(5);
     // ---- T^-1 (fp32, into the dead Q f half of A_LM), bf16 copy for MMA2
     invert_unit_lower<Ix, QRowsIdx>(sL, sTi, tid);
     for (int it = tid; it < kC * (kC / 8); it += kThreads) {
@@ -309,6 +323,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     tc_fence_before();
     __syncthreads();
 
+    GDR_PREP_PHASE(6);
     // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
     if (tid == 0) {
       tc_fence_after();
@@ -327,6 +342,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   }
 
   if (ok) {
+    GDR_PREP_PHASE(7);
     // ---- U and Y (x alpha_1) -> bf16 record tiles; M = 64 accumulators: row 16 qd + lane
     const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
     float x[32];
@@ -352,6 +368,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   } else if (tid == 0 && p.status) {
     atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
   }
+  GDR_PREP_PHASE(8);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -455,6 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     if (*sabort) { ok = false; break; }
     const float pn = reinterpret_cast<const float *>(bsm + SL::B_PI)[jrow];
 
+    GDR_CHAIN_PHASE(0);
     // ---- MMA3: Y S0 and Q_pi S0 (K = DK)
     if (tid == 0) {
       tc_fence_after();
@@ -472,6 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
 
+    GDR_CHAIN_PHASE(1);
     // ---- V~ = U - Y S0 -> bf16 (rows = tokens)
     {
       float d[32];
@@ -497,6 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     tc_fence_before();
     __syncthreads();
 
+    GDR_CHAIN_PHASE(2);
     // ---- MMA4: K~^T V~ (M = DK) and O += M V~ (M = C); K = C
     if (tid == 0) {
       tc_fence_after();
@@ -514,6 +534,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
 
+    GDR_CHAIN_PHASE(3);
     // ---- the buffer is free: fetch chunk c + 2
     if (tid == 0 && c + 2 < nch) {
       fence_proxy_async_smem();   // this CTA's reads of the buffer come before the refill
@@ -525,6 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
       bulk_g2s(bsm + SL::B_PI, src + Rec::PI, kDK * 4, full + buf);
     }
 
+    GDR_CHAIN_PHASE(4);
     // ---- state update (fp32) and outputs
     {
       float d[32];
@@ -551,6 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    GDR_CHAIN_PHASE(5);
   }
 
   if (ok && p.S_T) {
