@@ -20,9 +20,14 @@
 // state (1 GiB at B=256, H=32, d=128) is far larger than L2 and is not reused
 // within a step.
 #include "gdr_internal.cuh"
+#include "gdr_sm100.cuh"
 
 namespace gdr {
 namespace {
+
+using sm100::cp_async16;
+using sm100::cp_async_commit;
+using sm100::cp_async_wait;
 
 template <int DK, int DV>
 struct DecodeShape {
@@ -153,18 +158,6 @@ decode_step_kernel(gdr_form form, const Tin *__restrict__ q, const Tin *__restri
 // and the CTA then meets at a barrier, so no wait depends on another CTA.
 // While head i is reduced and written back from registers, heads i+1 and i+2
 // are in flight: about 130 KB per SM, enough to cover HBM latency.
-__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                   static_cast<uint32_t>(__cvta_generic_to_shared(dst_smem))),
-               "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 template <typename Tin>
 struct PipeShape {
   static constexpr int DK = 128, DV = 128, NST = 3, NT = 256;

@@ -30,6 +30,10 @@
 #ifndef GDR_CHAIN_PHASE
 #define GDR_CHAIN_PHASE(i)
 #endif
+#ifndef GDR_PHASE_INIT
+#define GDR_PHASE_INIT
+#define GDR_PHASE_FINI(slot)
+#endif
 
 namespace gdr {
 namespace {
@@ -68,19 +72,21 @@ struct QRowsIdx {
 struct PrepSmem {
   static constexpr uint32_t A_LM = 0;                       // [K^ f; Q f]  2C x DK bf16; Q rows
                                                             //   then hold fp32 T^-1 (QRowsIdx)
-  static constexpr uint32_t B_LM = A_LM + 2 * kC * kDK * 2;  // K g          C x DK bf16; then fp32 L
-  static constexpr uint32_t VH = B_LM + kC * kDK * 2;        // V^           C x DV bf16
-  static constexpr uint32_t TINV = VH + kC * kDK * 2;        // T^-1         C x C bf16
-  static constexpr uint32_t LAM = TINV + kC * kC * 2;        // fp32 Lambda  C x DK
-  static constexpr uint32_t A1 = LAM + kC * kDK * 4;         // fp32 alpha_1       DK
-  static constexpr uint32_t ED = A1 + kDK * 4;               // fp32 exp(Lam_n - Lam_1)
-  static constexpr uint32_t PIN = ED + kDK * 4;              // fp32 exp(Lam_n)
-  static constexpr uint32_t TOT = PIN + kDK * 4;             // fp32 first-half log-decay
-  static constexpr uint32_t MISC = TOT + kDK * 4;            // mbarrier, TMEM slot, flags
+  static constexpr uint32_t B_LM = A_LM + 2 * kC * kDK * 2;  // K g          C x DK bf16; then fp32 L;
+                                                            //   then bf16 T^-1 (first 8 KB)
+  static constexpr uint32_t VH = B_LM + kC * kDK * 2;        // v, then V^ = wg v in place, C x DV bf16
+  static constexpr uint32_t WG = VH + kC * kDK * 2;          // write gate  C x DV bf16
+  static constexpr uint32_t SCAN = WG + kC * kDK * 2;        // fp32 [16 token blocks][DK] log-decay sums
+  static constexpr uint32_t L1 = SCAN + 16 * kDK * 4;        // fp32 Lam_1 per channel
+  static constexpr uint32_t A1 = L1 + kDK * 4;               // fp32 alpha_1 per channel
+  static constexpr uint32_t MISC = A1 + kDK * 4;             // mbarrier, TMEM slot, flags
   static constexpr uint32_t ALLOC = MISC + 64 + 1024;
-  static_assert(Ix::kBytes <= kC * kDK * 2, "fp32 L / T^-1 must fit the reused bf16 tiles");
+  static_assert(Ix::kBytes <= kC * kDK * 2, "fp32 L must fit the reused bf16 tile");
 };
 
+// Thread layout of the elementwise phases: thread = (channel group g of 8 channels,
+// token block tb of 4 consecutive tokens); a warp covers two token blocks, and the
+// 16 threads of a token row read its 256 contiguous bytes.
 __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8_t *records) {
   using SL = PrepSmem;
   extern __shared__ uint8_t smem_raw[];
@@ -93,14 +99,14 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int T = p.T, H = p.H, t0 = c * kC, n = min(kC, T - t0);
   uint8_t *rec = records + ((size_t)((size_t)b * H + h) * num_chunks(T) + c) * Rec::BYTES;
+  const int g = tid & 15, tb = tid >> 4, j0 = 8 * g;
+  GDR_PHASE_INIT
 
-  float *sLam = reinterpret_cast<float *>(smem + SL::LAM);
   float *sL = reinterpret_cast<float *>(smem + SL::B_LM);
   float *sTi = reinterpret_cast<float *>(smem + SL::A_LM);
+  float *sScan = reinterpret_cast<float *>(smem + SL::SCAN);
+  float *sL1 = reinterpret_cast<float *>(smem + SL::L1);
   float *sA1 = reinterpret_cast<float *>(smem + SL::A1);
-  float *sED = reinterpret_cast<float *>(smem + SL::ED);
-  float *sPiN = reinterpret_cast<float *>(smem + SL::PIN);
-  float *sTot = reinterpret_cast<float *>(smem + SL::TOT);
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + SL::MISC);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 8);
   volatile int *sflag = reinterpret_cast<volatile int *>(smem + SL::MISC + 16);  // exact, abort
@@ -110,28 +116,41 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   const __nv_bfloat16 *gv = static_cast<const __nv_bfloat16 *>(p.v);
   const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
   const __nv_bfloat16 *gw = static_cast<const __nv_bfloat16 *>(p.e2);
+  auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
 
-  // ---- global reads first: log w (channel jc, half hh) and the k, b, q items
-  const int jc = tid & (kDK - 1), hh = tid >> 7;
-  float lw[32];
-#pragma unroll
-  for (int t = 0; t < 32; ++t) {
-    const int tt = 32 * hh + t;
-    lw[t] = (tt < n) ? __ldg(p.log_w + (((size_t)b * T + t0 + tt) * H + h) * kDK + jc) : 0.f;
-  }
+  // ---- every global read is issued here: log w, k, b, q into registers (this
+  //      thread's 4 tokens x 8 channels); v and wg by cp.async into their swizzled
+  //      positions (zero-filled past the end of the sequence)
+  float lam[4][8];
   uint4 rk[4], rb[4], rq[4];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int it = tid + u * kThreads, t = it >> 4, g = it & 15;
+  for (int i = 0; i < 4; ++i) {
+    const int t = 4 * tb + i;
     if (t < n) {
-      const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + 8 * g;
-      rk[u] = ld16(gk + off);
-      rb[u] = ld16(gb + off);
-      rq[u] = ld16(gq + off);
+      const size_t off = tok_off(t) + j0;
+      const float4 x0 = __ldg(reinterpret_cast<const float4 *>(p.log_w + off));
+      const float4 x1 = __ldg(reinterpret_cast<const float4 *>(p.log_w + off + 4));
+      lam[i][0] = x0.x; lam[i][1] = x0.y; lam[i][2] = x0.z; lam[i][3] = x0.w;
+      lam[i][4] = x1.x; lam[i][5] = x1.y; lam[i][6] = x1.z; lam[i][7] = x1.w;
+      rk[i] = ld16(gk + off);
+      rb[i] = ld16(gb + off);
+      rq[i] = ld16(gq + off);
     } else {
-      rk[u] = rb[u] = rq[u] = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) lam[i][e] = 0.f;
+      rk[i] = rb[i] = rq[i] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int it = tid + u * kThreads, t = it >> 4, gg = it & 15;
+    const bool valid = t < n;
+    const size_t off = valid ? tok_off(t) + 8 * gg : 0;
+    const uint32_t so = sw128_offset(t, 8 * gg, kC * 128);
+    cp_async16(smem + SL::VH + so, gv + off, valid);
+    if (gw) cp_async16(smem + SL::WG + so, gw + off, valid);
+  }
+  cp_async_commit();
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -145,104 +164,122 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   }
 
   GDR_PREP_PHASE(0);
-  // ---- cumulative log-decay Lam_t (two halves of the chunk, then joined)
+  // ---- cumulative log-decay: prefix within the thread's 4 tokens, then across the
+  //      16 token blocks through shared memory
   {
-    float acc = 0.f;
+    float tot[8];
 #pragma unroll
-    for (int t = 0; t < 32; ++t) {
-      acc += lw[t];
-      lw[t] = acc;
-    }
-    if (hh == 0) {
+    for (int e = 0; e < 8; ++e) {
+      float acc = 0.f;
 #pragma unroll
-      for (int t = 0; t < 32; ++t) sLam[t * kDK + jc] = lw[t];
-      sTot[jc] = acc;
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (hh == 1) {
-      const float base = sTot[jc], lam1 = sLam[jc];
-#pragma unroll
-      for (int t = 0; t < 32; ++t) sLam[(32 + t) * kDK + jc] = base + lw[t];
-      const float lamn = base + acc;
-      sPiN[jc] = __expf(lamn);
-      sA1[jc] = __expf(lam1);
-      sED[jc] = __expf(lamn - lam1);
-      if (lam1 - lamn > kMaxChunkDecay) sflag[0] = 1;
-    }
-  }
-  GDR_PREP_PHASE(1);
-  // ---- V^ = wg (.) v over the full d_v
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int it = tid + u * kThreads, t = it >> 4, g = it & 15;
-    float v8[8], w8[8];
-    if (t < n) {
-      const size_t off = (((size_t)b * T + t0 + t) * H + h) * kDK + 8 * g;
-      unpack8(ld16(gv + off), v8);
-      if (gw) {
-        unpack8(ld16(gw + off), w8);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w8[e] = 1.f;
+      for (int i = 0; i < 4; ++i) {
+        acc += lam[i][e];
+        lam[i][e] = acc;
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v8[e] = w8[e] = 0.f;
+      tot[e] = acc;
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
-    st_smem16(smem, SL::VH + sw128_offset(t, 8 * g, kC * 128), pack8(v8));
+    float4 *dst = reinterpret_cast<float4 *>(sScan + tb * kDK + j0);
+    dst[0] = make_float4(tot[0], tot[1], tot[2], tot[3]);
+    dst[1] = make_float4(tot[4], tot[5], tot[6], tot[7]);
+    if (tb == 0) {
+      float4 *l1 = reinterpret_cast<float4 *>(sL1 + j0);
+      l1[0] = make_float4(lam[0][0], lam[0][1], lam[0][2], lam[0][3]);
+      l1[1] = make_float4(lam[0][4], lam[0][5], lam[0][6], lam[0][7]);
+    }
   }
+  tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const bool exact = sflag[0] != 0;
-
-  GDR_PREP_PHASE(2);
-  // ---- operand tiles: [K^ f; Q f], K g in shared memory; Q_pi, K~ straight to the record
+  // lam[i][e] becomes Lam_t - Lam_1 (the pivot at the chunk's first token); dn = Lam_n - Lam_1
+  float dn[8], a1[8], ed[8];
+  {
+    float excl[8], all[8];
 #pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int it = tid + u * kThreads, t = it >> 4, g = it & 15, j0 = 8 * g;
-    float k8[8], b8[8], q8[8];
-    unpack8(rk[u], k8);
-    unpack8(rb[u], b8);
-    unpack8(rq[u], q8);
-    const float4 *lp = reinterpret_cast<const float4 *>(sLam + t * kDK + j0);
-    const float4 *l1p = reinterpret_cast<const float4 *>(sLam + j0);
-    const float4 *ln = reinterpret_cast<const float4 *>(sLam + (kC - 1) * kDK + j0);
-    const float4 l0 = lp[0], l1 = lp[1], f0 = l1p[0], f1 = l1p[1], n0 = ln[0], n1 = ln[1];
-    const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
-    const float lam1[8] = {f0.x, f0.y, f0.z, f0.w, f1.x, f1.y, f1.z, f1.w};
-    const float lamn[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-    float a1[8], a2[8], bl[8], kt[8], qp[8];
+    for (int e = 0; e < 8; ++e) excl[e] = all[e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const float4 *src = reinterpret_cast<const float4 *>(sScan + r * kDK + j0);
+      const float4 x0 = src[0], x1 = src[1];
+      const float v8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        all[e] += v8[e];
+        if (r < tb) excl[e] += v8[e];
+      }
+    }
+    const float4 *l1 = reinterpret_cast<const float4 *>(sL1 + j0);
+    const float4 y0 = l1[0], y1 = l1[1];
+    const float l1v[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+    bool over = false;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      const float f = __expf(lam[e] - lam1[e]);
-      a1[e] = b8[e] * k8[e] * f;
-      a2[e] = q8[e] * f;
-      qp[e] = a2[e] * sA1[j0 + e];
-      if (!exact) {
-        bl[e] = k8[e] * __expf(lam1[e] - lam[e]);
-        kt[e] = bl[e] * sED[j0 + e];
-      } else {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) lam[i][e] += excl[e] - l1v[e];
+      dn[e] = all[e] - l1v[e];
+      a1[e] = __expf(l1v[e]);
+      ed[e] = __expf(dn[e]);
+      over |= dn[e] < -kMaxChunkDecay;
+    }
+    if (over) sflag[0] = 1;
+    if (tb == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sA1[j0 + e] = a1[e];
+        reinterpret_cast<float *>(rec + Rec::PI)[j0 + e] = __expf(all[e]);
+      }
+    }
+  }
+
+  GDR_PREP_PHASE(1);
+  // ---- operand tiles: [K^ f; Q f], K g in shared memory; Q_pi, K~ straight to the record
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = 4 * tb + i;
+    float k8[8], b8[8], q8[8];
+    unpack8(rk[i], k8);
+    unpack8(rb[i], b8);
+    unpack8(rq[i], q8);
+    float av[8], aq[8], bl[8], kt[8], qp[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float f = __expf(lam[i][e]);
+      av[e] = b8[e] * k8[e] * f;
+      aq[e] = q8[e] * f;
+      qp[e] = aq[e] * a1[e];
+      if (dn[e] >= -kMaxChunkDecay) {
+        bl[e] = k8[e] * __expf(-lam[i][e]);
+        kt[e] = bl[e] * ed[e];
+      } else {           // this chunk takes the exact path; K g is not used
         bl[e] = 0.f;
-        kt[e] = k8[e] * __expf(lamn[e] - lam[e]);
+        kt[e] = k8[e] * __expf(dn[e] - lam[i][e]);
       }
     }
     const uint32_t o64 = sw128_offset(t, j0, kC * 128);
-    st_smem16(smem, SL::A_LM + sw128_offset(t, j0, 2 * kC * 128), pack8(a1));
-    st_smem16(smem, SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128), pack8(a2));
+    st_smem16(smem, SL::A_LM + sw128_offset(t, j0, 2 * kC * 128), pack8(av));
+    st_smem16(smem, SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128), pack8(aq));
     st_smem16(smem, SL::B_LM + o64, pack8(bl));
     *reinterpret_cast<uint4 *>(rec + Rec::QP + o64) = pack8(qp);
     *reinterpret_cast<uint4 *>(rec + Rec::KT + o64) = pack8(kt);
   }
   fence_proxy_async_smem();
   __syncthreads();
+  const bool exact = sflag[0] != 0;
+  // the exact path needs Lam_t - Lam_1 for every (token, channel): park it in the
+  // record's Y and U tiles, which are written only at the end
+  if (exact) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = 4 * tb + i;
+      float *dst = reinterpret_cast<float *>(rec + (t < 32 ? Rec::Y : Rec::U)) + (t & 31) * kDK + j0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) dst[e] = lam[i][e];
+    }
+  }
 
   uint32_t phase = 0;
   bool ok = true;
-  GDR_PREP_PHASE(3);
+  GDR_PREP_PHASE(2);
   // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
   if (tid == 0) {
     tc_fence_after();
@@ -255,6 +292,23 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     }
     mma_commit(mbar);
   }
+  // ---- while it runs: V^ = wg (.) v in place (each thread scales the chunks it copied)
+  cp_async_wait<0>();
+  if (gw) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int it = tid + u * kThreads, t = it >> 4, gg = it & 15;
+      const uint32_t so = sw128_offset(t, 8 * gg, kC * 128);
+      float v8[8], w8[8];
+      unpack8(*reinterpret_cast<const uint4 *>(smem + SL::VH + so), v8);
+      unpack8(*reinterpret_cast<const uint4 *>(smem + SL::WG + so), w8);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+      st_smem16(smem, SL::VH + so, pack8(v8));
+    }
+  }
+  fence_proxy_async_smem();
+  GDR_PREP_PHASE(3);
   ok = wait_mma(mbar, phase, sflag + 1);
 
   if (ok) {
@@ -283,14 +337,17 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
       }
     } else {
       // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound)
+      const float *lamg = reinterpret_cast<const float *>(rec + Rec::Y);
+      const float *lamg2 = reinterpret_cast<const float *>(rec + Rec::U);
       for (int it = tid; it < kC * kC; it += kThreads) {
         const int t = it / kC, s = it % kC;
         float l = 0.f, m = 0.f;
         if (s <= t && t < n) {
-          const size_t ot = (((size_t)b * T + t0 + t) * H + h) * kDK;
-          const size_t os = (((size_t)b * T + t0 + s) * H + h) * kDK;
+          const float *lt = (t < 32 ? lamg : lamg2) + (t & 31) * kDK;
+          const float *ls = (s < 32 ? lamg : lamg2) + (s & 31) * kDK;
+          const size_t ot = tok_off(t), os = tok_off(s);
           for (int j = 0; j < kDK; ++j) {
-            const float d = __expf(sLam[t * kDK + j] - sLam[s * kDK + j]);
+            const float d = __expf(__ldcg(lt + j) - __ldcg(ls + j));
             const float ks = __bfloat162float(gk[os + j]);
             m += __bfloat162float(gq[ot + j]) * d * ks;
             l += __bfloat162float(gb[ot + j]) * __bfloat162float(gk[ot + j]) * d * ks;
@@ -305,19 +362,19 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     __syncthreads();
 
     GDR_PREP_PHASE(5);
-    // ---- T^-1 (fp32, into the dead Q f half of A_LM), bf16 copy for MMA2
+    // ---- T^-1 (fp32, into the dead Q rows of A_LM), bf16 copy (into the dead L tile)
     invert_unit_lower<Ix, QRowsIdx>(sL, sTi, tid);
     for (int it = tid; it < kC * (kC / 8); it += kThreads) {
-      const int t = it >> 3, g = it & 7;
-      const float4 y0 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * g));
-      const float4 y1 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * g + 4));
+      const int t = it >> 3, gg = it & 7;
+      const float4 y0 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg));
+      const float4 y1 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg + 4));
       float x[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const int s = 8 * g + e;
+        const int s = 8 * gg + e;
         x[e] = (s < t) ? x[e] : (s == t ? 1.f : 0.f);
       }
-      st_smem16(smem, SL::TINV + sw128_offset(t, 8 * g, kC * 128), pack8(x));
+      st_smem16(smem, SL::B_LM + sw128_offset(t, 8 * gg, kC * 128), pack8(x));
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -330,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
       constexpr uint32_t id = idesc_bf16_f32(64, kDK, false, true);
 #pragma unroll
       for (int s = 0; s < kC / 16; ++s) {
-        const uint64_t ad = sdesc_sw128(sb + SL::TINV + s * 32, 16, 1024);
+        const uint64_t ad = sdesc_sw128(sb + SL::B_LM + s * 32, 16, 1024);
         const uint64_t bu = sdesc_sw128(sb + SL::VH + s * 2048, kC * 128, 1024);
         const uint64_t by = sdesc_sw128(sb + SL::A_LM + s * 2048, 2 * kC * 128, 1024);
         mma_bf16(tmem, ad, bu, id, s > 0);
@@ -364,11 +421,11 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
                                      sw128_offset(t, col + i, kC * 128)) = pack8(x + i);
       }
     }
-    if (tid < kDK) reinterpret_cast<float *>(rec + Rec::PI)[tid] = sPiN[tid];
   } else if (tid == 0 && p.status) {
     atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
   }
   GDR_PREP_PHASE(8);
+  GDR_PHASE_FINI(1)
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -381,21 +438,56 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
 template <int NV>
 struct ChainSmem {
   // per buffer: Y | QP | KT | MM (as in the record) | U slice (C x NV) | pi
+  static constexpr int NBUF = 3;
   static constexpr uint32_t B_U = Rec::FRONT;
   static constexpr uint32_t B_PI = B_U + kC * NV * 2;
   static constexpr uint32_t BUF = ((B_PI + kDK * 4 + 1023) / 1024) * 1024;
-  static constexpr uint32_t S0B = 2 * BUF;                    // bf16 S0   DK x NV
+  static constexpr uint32_t S0B = NBUF * BUF;                 // bf16 S0   DK x NV
   static constexpr uint32_t VT = S0B + kDK * NV * 2;          // bf16 V~   C x NV
-  static constexpr uint32_t MISC = VT + kC * NV * 2;          // full[2], mma, TMEM slot, abort
+  static constexpr uint32_t MISC = VT + kC * NV * 2;          // full[3], mma, TMEM slot, abort
   static constexpr uint32_t ALLOC = MISC + 64 + 1024;
   static constexpr uint32_t TX = Rec::FRONT + kC * NV * 2 + kDK * 4;  // bytes per record fetch
   static_assert(NV == 64, "one 64-column block of U per CTA");
+  static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
+
+// Thread 0: fetch record `c` of this CTA's sequence into buffer c % NBUF.
+template <int NV>
+__device__ __forceinline__ void fetch_record(uint8_t *smem, uint64_t *full, const uint8_t *recs,
+                                             int c, int slice) {
+  using SL = ChainSmem<NV>;
+  const int buf = c % SL::NBUF;
+  uint8_t *dst = smem + buf * SL::BUF;
+  const uint8_t *src = recs + (size_t)c * Rec::BYTES;
+  mbar_arrive_expect_tx(full + buf, SL::TX);
+  bulk_g2s(dst, src, Rec::FRONT, full + buf);
+  bulk_g2s(dst + SL::B_U, src + Rec::U + slice * (kC * 128), kC * NV * 2, full + buf);
+  bulk_g2s(dst + SL::B_PI, src + Rec::PI, kDK * 4, full + buf);
+}
+
+// Thread 0: MMA3 of chunk c -- D1 = Y S0 and DO[c & 1] = Q_pi S0 (K = DK).
+template <int NV>
+__device__ __forceinline__ void issue_mma3(uint32_t sb, uint32_t tmem, int c, uint64_t *mbar) {
+  using SL = ChainSmem<NV>;
+  const uint32_t bb = sb + (c % SL::NBUF) * SL::BUF;
+  constexpr uint32_t id = idesc_bf16_f32(64, NV, false, true);
+  tc_fence_after();
+#pragma unroll
+  for (int s = 0; s < kDK / 16; ++s) {
+    const uint32_t ko = (s >> 2) * (kC * 128) + (s & 3) * 32;
+    const uint64_t ay = sdesc_sw128(bb + Rec::Y + ko, 16, 1024);
+    const uint64_t aq = sdesc_sw128(bb + Rec::QP + ko, 16, 1024);
+    const uint64_t bs = sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
+    mma_bf16(tmem, ay, bs, id, s > 0);
+    mma_bf16(tmem + 64 + 64 * (c & 1), aq, bs, id, s > 0);
+  }
+  mma_commit(mbar);
+}
 
 template <int NV>
 __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, const uint8_t *records) {
   using SL = ChainSmem<NV>;
-  constexpr int HALF = NV / 2;
+  constexpr int HALF = NV / 2, NBUF = SL::NBUF;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -406,33 +498,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
   const int slice = blockIdx.x, c0 = slice * NV, h = blockIdx.y, b = blockIdx.z;
   const int T = p.T, H = p.H, nch = num_chunks(T);
   const uint8_t *recs = records + (size_t)((size_t)b * H + h) * nch * Rec::BYTES;
+  GDR_PHASE_INIT
 
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::MISC);       // [2]
-  uint64_t *mbar = full + 2;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 24);
-  volatile int *sabort = reinterpret_cast<volatile int *>(smem + SL::MISC + 32);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::MISC);       // [NBUF]
+  uint64_t *mbar = full + NBUF;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 8 * (NBUF + 1));
+  volatile int *sabort = reinterpret_cast<volatile int *>(smem + SL::MISC + 8 * (NBUF + 1) + 8);
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  uint32_t fissue[NBUF] = {}, fdone[NBUF] = {};   // thread 0's fetch bookkeeping
   if (tid == 0) {
-    mbar_init(full, 1);
-    mbar_init(full + 1, 1);
+    for (int i = 0; i < NBUF; ++i) mbar_init(full + i, 1);
     mbar_init(mbar, 1);
     fence_mbar_init();
     *sabort = 0;
-  }
-  uint32_t fissue[2] = {0u, 0u}, fdone[2] = {0u, 0u};   // thread 0's fetch bookkeeping
-  if (tid == 0) {
-    for (int cc = 0; cc < 2 && cc < nch; ++cc) {
+    for (int cc = 0; cc < NBUF && cc < nch; ++cc) {
       ++fissue[cc];
-      uint8_t *dst = smem + cc * SL::BUF;
-      const uint8_t *src = recs + (size_t)cc * Rec::BYTES;
-      mbar_arrive_expect_tx(full + cc, SL::TX);
-      bulk_g2s(dst, src, Rec::FRONT, full + cc);
-      bulk_g2s(dst + SL::B_U, src + Rec::U + slice * (kC * 128), kC * NV * 2, full + cc);
-      bulk_g2s(dst + SL::B_PI, src + Rec::PI, kDK * 4, full + cc);
+      fetch_record<NV>(smem, full, recs, cc, slice);
     }
   }
 
@@ -454,41 +539,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tD1 = tmem, tDO = tmem + 64, tDS = tmem + 128;
+  const uint32_t tD1 = tmem, tDS = tmem + 192;
   const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
+
+  // ---- MMA3 of chunk 0
+  if (tid == 0) {
+    if (mbar_wait_bounded(full, 0, kWaitLimitNs)) {
+      ++fdone[0];
+      issue_mma3<NV>(sb, tmem, 0, mbar);
+    } else {
+      *sabort = 1;
+    }
+  }
 
   uint32_t phase = 0;
   bool ok = true;
-  for (int c = 0; c < nch && ok; ++c) {
-    const int buf = c & 1, t0 = c * kC, n = min(kC, T - t0);
+  for (int c = 0; c < nch; ++c) {
+    const int buf = c % NBUF, t0 = c * kC, n = min(kC, T - t0);
     const uint32_t bb = sb + buf * SL::BUF;
-    uint8_t *bsm = smem + buf * SL::BUF;
-    // ---- record of chunk c present?
-    if (tid == 0) {
-      if (mbar_wait_bounded(full + buf, (c >> 1) & 1, kWaitLimitNs)) ++fdone[buf];
-      else *sabort = 1;
-    }
-    __syncthreads();
-    if (*sabort) { ok = false; break; }
-    const float pn = reinterpret_cast<const float *>(bsm + SL::B_PI)[jrow];
-
+    const uint8_t *bsm = smem + buf * SL::BUF;
     GDR_CHAIN_PHASE(0);
-    // ---- MMA3: Y S0 and Q_pi S0 (K = DK)
-    if (tid == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_bf16_f32(64, NV, false, true);
-#pragma unroll
-      for (int s = 0; s < kDK / 16; ++s) {
-        const uint32_t ko = (s >> 2) * (kC * 128) + (s & 3) * 32;
-        const uint64_t ay = sdesc_sw128(bb + Rec::Y + ko, 16, 1024);
-        const uint64_t aq = sdesc_sw128(bb + Rec::QP + ko, 16, 1024);
-        const uint64_t bs = sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
-        mma_bf16(tD1, ay, bs, id, s > 0);
-        mma_bf16(tDO, aq, bs, id, s > 0);
-      }
-      mma_commit(mbar);
-    }
+    // ---- wait for MMA3 (c): Y S0 in D1, Q_pi S0 in DO[c & 1]
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    const float pn = reinterpret_cast<const float *>(bsm + SL::B_PI)[jrow];
 
     GDR_CHAIN_PHASE(1);
     // ---- V~ = U - Y S0 -> bf16 (rows = tokens)
@@ -517,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     __syncthreads();
 
     GDR_CHAIN_PHASE(2);
-    // ---- MMA4: K~^T V~ (M = DK) and O += M V~ (M = C); K = C
+    // ---- MMA4: K~^T V~ (M = DK) and DO[c & 1] += M V~ (M = C); K = C
     if (tid == 0) {
       tc_fence_after();
       constexpr uint32_t ids = idesc_bf16_f32(128, NV, true, true);
@@ -528,26 +601,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
         const uint64_t bv = sdesc_sw128(sb + SL::VT + s * 2048, kC * 128, 1024);
         const uint64_t am = sdesc_sw128(bb + Rec::MM + s * 32, 16, 1024);
         mma_bf16(tDS, ak, bv, ids, s > 0);
-        mma_bf16(tDO, am, bv, ido, 1);
+        mma_bf16(tmem + 64 + 64 * (c & 1), am, bv, ido, 1);
       }
       mma_commit(mbar);
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
 
     GDR_CHAIN_PHASE(3);
-    // ---- the buffer is free: fetch chunk c + 2
-    if (tid == 0 && c + 2 < nch) {
-      fence_proxy_async_smem();   // this CTA's reads of the buffer come before the refill
-      ++fissue[buf];
-      const uint8_t *src = recs + (size_t)(c + 2) * Rec::BYTES;
-      mbar_arrive_expect_tx(full + buf, SL::TX);
-      bulk_g2s(bsm, src, Rec::FRONT, full + buf);
-      bulk_g2s(bsm + SL::B_U, src + Rec::U + slice * (kC * 128), kC * NV * 2, full + buf);
-      bulk_g2s(bsm + SL::B_PI, src + Rec::PI, kDK * 4, full + buf);
-    }
-
-    GDR_CHAIN_PHASE(4);
-    // ---- state update (fp32) and outputs
+    // ---- state update (fp32) and its bf16 copy for the next MMA3
     {
       float d[32];
       tmem_ld_32x32b_x32(tDS + lane_q + hf * HALF, d);
@@ -557,8 +618,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
 #pragma unroll
       for (int i = 0; i < HALF; i += 8)
         st_smem16(smem, SL::S0B + sw128_offset(jrow, hf * HALF + i, kDK * 128), pack8(st + i));
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    GDR_CHAIN_PHASE(4);
+    // ---- start chunk c + 1 (MMA3) and refill this chunk's buffer, then store O (c)
+    //      while that MMA runs
+    if (tid == 0 && c + 1 < nch && !*sabort) {
+      const int nb = (c + 1) % NBUF;
+      if (mbar_wait_bounded(full + nb, ((c + 1) / NBUF) & 1, kWaitLimitNs)) {
+        ++fdone[nb];
+        issue_mma3<NV>(sb, tmem, c + 1, mbar);
+        if (c + NBUF < nch) {
+          fence_proxy_async_smem();   // this CTA's reads of the buffer come before the refill
+          ++fissue[buf];
+          fetch_record<NV>(smem, full, recs, c + NBUF, slice);
+        }
+      } else {
+        *sabort = 1;
+      }
+    }
+    {
       float o[32];
-      tmem_ld_32x32b_x32(tDO + lane_q + hf * HALF, o);
+      tmem_ld_32x32b_x32(tmem + 64 + 64 * (c & 1) + lane_q + hf * HALF, o);
       tmem_ld_wait();
       if (lane < 16) {
         const int t = 16 * qd + lane;
@@ -570,12 +654,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
         }
       }
     }
-    fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
     GDR_CHAIN_PHASE(5);
   }
 
+  GDR_PHASE_FINI(0)
   if (ok && p.S_T) {
 #pragma unroll
     for (int i = 0; i < HALF; i += 4)
@@ -585,7 +668,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
     // let MMAs and record copies already in flight land before the CTA exits
     mbar_wait_bounded(mbar, phase, kWaitLimitNs);
-    for (int bq = 0; bq < 2; ++bq)
+    for (int bq = 0; bq < NBUF; ++bq)
       while (fdone[bq] < fissue[bq]) {
         if (!mbar_wait_bounded(full + bq, fdone[bq] & 1, kWaitLimitNs)) break;
         ++fdone[bq];

@@ -50,7 +50,7 @@ __device__ __forceinline__ void st_smem16(uint8_t *base, uint32_t off, const uin
 // take the same branch).  Returns false, with the shared abort flag set, when the
 // wait ran out.
 __device__ __forceinline__ bool wait_mma(uint64_t *bar, uint32_t &phase, volatile int *abort) {
-  if (threadIdx.x == 0 && !mbar_wait_bounded(bar, phase, kWaitLimitNs)) *abort = 1;
+  if (threadIdx.x == 0 && *abort == 0 && !mbar_wait_bounded(bar, phase, kWaitLimitNs)) *abort = 1;
   phase ^= 1u;
   __syncthreads();
   tc_fence_after();
