@@ -30,6 +30,10 @@
 #ifndef GDR_CHAIN_PHASE
 #define GDR_CHAIN_PHASE(i)
 #endif
+#ifndef GDR_SUB_DECL
+#define GDR_SUB_DECL
+#define GDR_SUB(i)
+#endif
 #ifndef GDR_PHASE_INIT
 #define GDR_PHASE_INIT
 #define GDR_PHASE_FINI(slot)
@@ -43,18 +47,28 @@ using Ix = SwizzledIdx;
 
 // One chunk's record: bf16 tiles in the sw128 layout (64-column blocks of C*128 B).
 struct Rec {
-  static constexpr uint32_t Y = 0;                     // Y       C x DK  (K-major A of Y S0)
-  static constexpr uint32_t QP = Y + kC * kDK * 2;      // Q_pi    C x DK  (K-major A of Q S0)
-  static constexpr uint32_t KT = QP + kC * kDK * 2;     // K~      C x DK  (MN-major A of K~^T V~)
+  static constexpr uint32_t QY = 0;                     // [Q_pi; Y] 2C x DK (K-major A of one
+                                                        //   M = 2C MMA with S0): rows 0..C-1
+                                                        //   Q_pi, rows C..2C-1 Y
+  static constexpr uint32_t KT = QY + 2 * kC * kDK * 2;  // K~      C x DK  (MN-major A of K~^T V~)
   static constexpr uint32_t MM = KT + kC * kDK * 2;     // M       C x C   (K-major A of M V~)
   static constexpr uint32_t U = MM + kC * kC * 2;       // U       C x DV  (rows = tokens)
   static constexpr uint32_t PI = U + kC * kDK * 2;      // exp(Lam_n), DK fp32
   static constexpr uint32_t BYTES = PI + 1024;
-  static constexpr uint32_t FRONT = U;                  // Y | QP | KT | MM, copied as one block
-  static_assert(Y % 1024 == 0 && QP % 1024 == 0 && KT % 1024 == 0 && MM % 1024 == 0 &&
-                    U % 1024 == 0 && PI % 1024 == 0 && BYTES % 1024 == 0,
+  static constexpr uint32_t FRONT = U;                  // QY | KT | MM, copied as one block
+  static constexpr uint32_t QY_STRIDE = 2 * kC * 128;   // bytes between QY's 64-column blocks
+  static_assert(QY % 1024 == 0 && KT % 1024 == 0 && MM % 1024 == 0 && U % 1024 == 0 &&
+                    PI % 1024 == 0 && BYTES % 1024 == 0,
                 "record tiles must stay 1024-byte aligned");
 };
+
+// Where a chunk that takes the exact path parks Lam_t - Lam_1 (token t, DK fp32):
+// the record's Y rows (two 8 KB pieces) and its U tile, all written only at the end.
+__device__ __forceinline__ uint32_t park_row(int t) {
+  return t < 16   ? Rec::QY + kC * 128 + t * kDK * 4
+         : t < 32 ? Rec::QY + Rec::QY_STRIDE + kC * 128 + (t - 16) * kDK * 4
+                  : Rec::U + (t - 32) * kDK * 4;
+}
 constexpr size_t kHeaderBytes = 1024;
 
 __host__ __device__ inline int num_chunks(int T) { return (T + kC - 1) / kC; }
@@ -190,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   // lam[i][e] becomes Lam_t - Lam_1 (the pivot at the chunk's first token); dn = Lam_n - Lam_1
   float dn[8], a1[8], ed[8];
   {
@@ -259,19 +273,21 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     st_smem16(smem, SL::A_LM + sw128_offset(t, j0, 2 * kC * 128), pack8(av));
     st_smem16(smem, SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128), pack8(aq));
     st_smem16(smem, SL::B_LM + o64, pack8(bl));
-    *reinterpret_cast<uint4 *>(rec + Rec::QP + o64) = pack8(qp);
+    *reinterpret_cast<uint4 *>(rec + Rec::QY + sw128_offset(t, j0, Rec::QY_STRIDE)) = pack8(qp);
     *reinterpret_cast<uint4 *>(rec + Rec::KT + o64) = pack8(kt);
   }
+  GDR_PREP_PHASE(9);
   fence_proxy_async_smem();
+  GDR_PREP_PHASE(10);
   __syncthreads();
   const bool exact = sflag[0] != 0;
   // the exact path needs Lam_t - Lam_1 for every (token, channel): park it in the
-  // record's Y and U tiles, which are written only at the end
+  // record's Y rows and U tile, which are written only at the end
   if (exact) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = 4 * tb + i;
-      float *dst = reinterpret_cast<float *>(rec + (t < 32 ? Rec::Y : Rec::U)) + (t & 31) * kDK + j0;
+      float *dst = reinterpret_cast<float *>(rec + park_row(t)) + j0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) dst[e] = lam[i][e];
     }
@@ -281,16 +297,16 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   bool ok = true;
   GDR_PREP_PHASE(2);
   // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
-  if (tid == 0) {
+  if (warp == 0) {
     tc_fence_after();
     constexpr uint32_t id = idesc_bf16_f32(128, kC, false, false);
 #pragma unroll
     for (int s = 0; s < kDK / 16; ++s) {
       const uint64_t ad = sdesc_sw128(sb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
       const uint64_t bd = sdesc_sw128(sb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
-      mma_bf16(tmem, ad, bd, id, s > 0);
+      mma_bf16_warp(tmem, ad, bd, id, s > 0);
     }
-    mma_commit(mbar);
+    mma_commit_warp(mbar);
   }
   // ---- while it runs: V^ = wg (.) v in place (each thread scales the chunks it copied)
   cp_async_wait<0>();
@@ -337,14 +353,12 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
       }
     } else {
       // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound)
-      const float *lamg = reinterpret_cast<const float *>(rec + Rec::Y);
-      const float *lamg2 = reinterpret_cast<const float *>(rec + Rec::U);
       for (int it = tid; it < kC * kC; it += kThreads) {
         const int t = it / kC, s = it % kC;
         float l = 0.f, m = 0.f;
         if (s <= t && t < n) {
-          const float *lt = (t < 32 ? lamg : lamg2) + (t & 31) * kDK;
-          const float *ls = (s < 32 ? lamg : lamg2) + (s & 31) * kDK;
+          const float *lt = reinterpret_cast<const float *>(rec + park_row(t));
+          const float *ls = reinterpret_cast<const float *>(rec + park_row(s));
           const size_t ot = tok_off(t), os = tok_off(s);
           for (int j = 0; j < kDK; ++j) {
             const float d = __expf(__ldcg(lt + j) - __ldcg(ls + j));
@@ -382,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
 
     GDR_PREP_PHASE(6);
     // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
-    if (tid == 0) {
+    if (warp == 0) {
       tc_fence_after();
       constexpr uint32_t id = idesc_bf16_f32(64, kDK, false, true);
 #pragma unroll
@@ -390,10 +404,10 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
         const uint64_t ad = sdesc_sw128(sb + SL::B_LM + s * 32, 16, 1024);
         const uint64_t bu = sdesc_sw128(sb + SL::VH + s * 2048, kC * 128, 1024);
         const uint64_t by = sdesc_sw128(sb + SL::A_LM + s * 2048, 2 * kC * 128, 1024);
-        mma_bf16(tmem, ad, bu, id, s > 0);
-        mma_bf16(tmem + kDK, ad, by, id, s > 0);
+        mma_bf16_warp(tmem, ad, bu, id, s > 0);
+        mma_bf16_warp(tmem + kDK, ad, by, id, s > 0);
       }
-      mma_commit(mbar);
+      mma_commit_warp(mbar);
     }
     ok = wait_mma(mbar, phase, sflag + 1);
   }
@@ -417,8 +431,9 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
         }
 #pragma unroll
         for (int i = 0; i < 32; i += 8)
-          *reinterpret_cast<uint4 *>(rec + (is_y ? Rec::Y : Rec::U) +
-                                     sw128_offset(t, col + i, kC * 128)) = pack8(x + i);
+          *reinterpret_cast<uint4 *>(
+              rec + (is_y ? Rec::QY + sw128_offset(kC + t, col + i, Rec::QY_STRIDE)
+                          : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
       }
     }
   } else if (tid == 0 && p.status) {
@@ -435,53 +450,91 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
 }
 
 // ============================================================== chain kernel
+// Per chunk, for one (b, h, 64-column value slice), with S0 the bf16 copy of the
+// fp32 state kept in registers:
+//   MMA3   D[c&1] = [Q_pi; Y] S0          (M = 2C = 128, K = DK)   rows 0..C-1: Q_pi S0
+//   V~ = U - (Y S0)                        (warps on TMEM lanes C..2C-1)
+//   MMA4   DS = K~^T V~                    (M = DK, K = C)
+//          D[c&1] += [M; *] V~             (M = 128, K = C; rows C..2C-1 are discarded)
+//   S <- Diag(pi_n) S + DS                 (fp32, all warps)
+//   O = rows 0..C-1 of D[c&1]              (read while MMA3 of chunk c + 1 runs)
+// Warp 0 issues the MMAs (lane 0, from converged code); warp 2 refills the record
+// ring three chunks ahead.
 template <int NV>
 struct ChainSmem {
-  // per buffer: Y | QP | KT | MM (as in the record) | U slice (C x NV) | pi
+  // per buffer: QY | KT | MM | U slice (C x NV) | pi.  The U slice sits directly after
+  // M, so [M; U slice] is a valid 128-row K-major operand whose lower half only
+  // feeds accumulator rows that are discarded.
   static constexpr int NBUF = 3;
   static constexpr uint32_t B_U = Rec::FRONT;
   static constexpr uint32_t B_PI = B_U + kC * NV * 2;
   static constexpr uint32_t BUF = ((B_PI + kDK * 4 + 1023) / 1024) * 1024;
   static constexpr uint32_t S0B = NBUF * BUF;                 // bf16 S0   DK x NV
   static constexpr uint32_t VT = S0B + kDK * NV * 2;          // bf16 V~   C x NV
-  static constexpr uint32_t MISC = VT + kC * NV * 2;          // full[3], mma, TMEM slot, abort
-  static constexpr uint32_t ALLOC = MISC + 64 + 1024;
+  static constexpr uint32_t MISC = VT + kC * NV * 2;          // barriers, TMEM slot, flags
+  static constexpr uint32_t ALLOC = MISC + 128 + 1024;
   static constexpr uint32_t TX = Rec::FRONT + kC * NV * 2 + kDK * 4;  // bytes per record fetch
   static_assert(NV == 64, "one 64-column block of U per CTA");
+  static_assert(B_U == Rec::MM + kC * kC * 2 && kC * NV * 2 == kC * kC * 2,
+                "[M; U slice] must form one 128-row operand");
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-// Thread 0: fetch record `c` of this CTA's sequence into buffer c % NBUF.
+struct ChainMisc {          // byte offsets inside ChainSmem::MISC
+  static constexpr uint32_t FULL = 0;      // uint64_t [NBUF] record-arrival barriers
+  static constexpr uint32_t BAR3 = 24;     // uint64_t MMA3 completion
+  static constexpr uint32_t BAR4 = 32;     // uint64_t MMA4 completion
+  static constexpr uint32_t SLOT = 40;     // uint32_t TMEM base
+  static constexpr uint32_t ABORT = 44;    // int      a bounded wait ran out
+  static constexpr uint32_t FISS = 48;     // uint32_t [NBUF] fetches issued per buffer
+  static constexpr uint32_t FDONE = 64;    // uint32_t [NBUF] fetches waited for per buffer
+};
+
+// One lane: fetch record `c` of this CTA's sequence into buffer c % NBUF.
 template <int NV>
-__device__ __forceinline__ void fetch_record(uint8_t *smem, uint64_t *full, const uint8_t *recs,
-                                             int c, int slice) {
+__device__ __forceinline__ void fetch_record(uint8_t *smem, uint64_t *full, uint32_t *fiss,
+                                             const uint8_t *recs, int c, int slice) {
   using SL = ChainSmem<NV>;
   const int buf = c % SL::NBUF;
   uint8_t *dst = smem + buf * SL::BUF;
   const uint8_t *src = recs + (size_t)c * Rec::BYTES;
+  ++fiss[buf];
   mbar_arrive_expect_tx(full + buf, SL::TX);
   bulk_g2s(dst, src, Rec::FRONT, full + buf);
   bulk_g2s(dst + SL::B_U, src + Rec::U + slice * (kC * 128), kC * NV * 2, full + buf);
   bulk_g2s(dst + SL::B_PI, src + Rec::PI, kDK * 4, full + buf);
 }
 
-// Thread 0: MMA3 of chunk c -- D1 = Y S0 and DO[c & 1] = Q_pi S0 (K = DK).
+// Warp 0 (all lanes): wait for record c, then MMA3 of chunk c into D[c & 1].
+// Returns false (and issues nothing) if the record did not arrive in time.
 template <int NV>
-__device__ __forceinline__ void issue_mma3(uint32_t sb, uint32_t tmem, int c, uint64_t *mbar) {
+__device__ __forceinline__ bool start_chunk(uint8_t *smem, uint32_t sb, uint32_t tmem, int c) {
   using SL = ChainSmem<NV>;
-  const uint32_t bb = sb + (c % SL::NBUF) * SL::BUF;
-  constexpr uint32_t id = idesc_bf16_f32(64, NV, false, true);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::MISC + ChainMisc::FULL);
+  uint32_t *fdone = reinterpret_cast<uint32_t *>(smem + SL::MISC + ChainMisc::FDONE);
+  const int buf = c % SL::NBUF;
+  GDR_SUB_DECL
+  bool got = true;
+  if ((threadIdx.x & 31) == 0) {
+    got = mbar_wait_bounded(full + buf, (c / SL::NBUF) & 1, kWaitLimitNs);
+    if (got) ++fdone[buf];
+  }
+  got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+  GDR_SUB(0);
+  if (!got) return false;
+  const uint32_t bb = sb + buf * SL::BUF;
+  constexpr uint32_t id = idesc_bf16_f32(2 * kC, NV, false, true);
   tc_fence_after();
 #pragma unroll
   for (int s = 0; s < kDK / 16; ++s) {
-    const uint32_t ko = (s >> 2) * (kC * 128) + (s & 3) * 32;
-    const uint64_t ay = sdesc_sw128(bb + Rec::Y + ko, 16, 1024);
-    const uint64_t aq = sdesc_sw128(bb + Rec::QP + ko, 16, 1024);
+    const uint64_t a = sdesc_sw128(bb + Rec::QY + (s >> 2) * Rec::QY_STRIDE + (s & 3) * 32, 16, 1024);
     const uint64_t bs = sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
-    mma_bf16(tmem, ay, bs, id, s > 0);
-    mma_bf16(tmem + 64 + 64 * (c & 1), aq, bs, id, s > 0);
+    mma_bf16_warp(tmem + 64 * (c & 1), a, bs, id, s > 0);
   }
-  mma_commit(mbar);
+  GDR_SUB(1);
+  mma_commit_warp(reinterpret_cast<uint64_t *>(smem + SL::MISC + ChainMisc::BAR3));
+  GDR_SUB(2);
+  return true;
 }
 
 template <int NV>
@@ -500,25 +553,29 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
   const uint8_t *recs = records + (size_t)((size_t)b * H + h) * nch * Rec::BYTES;
   GDR_PHASE_INIT
 
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::MISC);       // [NBUF]
-  uint64_t *mbar = full + NBUF;
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 8 * (NBUF + 1));
-  volatile int *sabort = reinterpret_cast<volatile int *>(smem + SL::MISC + 8 * (NBUF + 1) + 8);
+  uint8_t *misc = smem + SL::MISC;
+  uint64_t *full = reinterpret_cast<uint64_t *>(misc + ChainMisc::FULL);
+  uint64_t *bar3 = reinterpret_cast<uint64_t *>(misc + ChainMisc::BAR3);
+  uint64_t *bar4 = reinterpret_cast<uint64_t *>(misc + ChainMisc::BAR4);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + ChainMisc::SLOT);
+  volatile int *sabort = reinterpret_cast<volatile int *>(misc + ChainMisc::ABORT);
+  uint32_t *fiss = reinterpret_cast<uint32_t *>(misc + ChainMisc::FISS);
+  uint32_t *fdone = reinterpret_cast<uint32_t *>(misc + ChainMisc::FDONE);
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  uint32_t fissue[NBUF] = {}, fdone[NBUF] = {};   // thread 0's fetch bookkeeping
   if (tid == 0) {
-    for (int i = 0; i < NBUF; ++i) mbar_init(full + i, 1);
-    mbar_init(mbar, 1);
+    for (int i = 0; i < NBUF; ++i) {
+      mbar_init(full + i, 1);
+      fiss[i] = fdone[i] = 0;
+    }
+    mbar_init(bar3, 1);
+    mbar_init(bar4, 1);
     fence_mbar_init();
     *sabort = 0;
-    for (int cc = 0; cc < NBUF && cc < nch; ++cc) {
-      ++fissue[cc];
-      fetch_record<NV>(smem, full, recs, cc, slice);
-    }
+    for (int cc = 0; cc < NBUF && cc < nch; ++cc) fetch_record<NV>(smem, full, fiss, recs, cc, slice);
   }
 
   // fp32 state: key channel jrow, value columns [hf*HALF, hf*HALF + HALF) of this slice
@@ -538,51 +595,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const uint32_t tD1 = tmem, tDS = tmem + 192;
+  const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
+  const uint32_t tDS = tmem + 128;
   const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
 
-  // ---- MMA3 of chunk 0
-  if (tid == 0) {
-    if (mbar_wait_bounded(full, 0, kWaitLimitNs)) {
-      ++fdone[0];
-      issue_mma3<NV>(sb, tmem, 0, mbar);
-    } else {
-      *sabort = 1;
-    }
+  uint32_t iss3 = 0, iss4 = 0;   // MMA groups committed (counted by warp 0)
+  uint32_t ph3 = 0, ph4 = 0;     // completions every thread has waited for
+  if (warp == 0) {
+    if (start_chunk<NV>(smem, sb, tmem, 0)) ++iss3;
+    else if (lane == 0) *sabort = 1;
   }
 
-  uint32_t phase = 0;
   bool ok = true;
   for (int c = 0; c < nch; ++c) {
     const int buf = c % NBUF, t0 = c * kC, n = min(kC, T - t0);
     const uint32_t bb = sb + buf * SL::BUF;
     const uint8_t *bsm = smem + buf * SL::BUF;
+    const uint32_t tD = tmem + 64 * (c & 1);
     GDR_CHAIN_PHASE(0);
-    // ---- wait for MMA3 (c): Y S0 in D1, Q_pi S0 in DO[c & 1]
-    if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    // ---- wait for MMA3 (c): [Q_pi S0; Y S0] in D[c & 1]
+    if (!(ok = wait_mma(bar3, ph3, sabort))) break;
     const float pn = reinterpret_cast<const float *>(bsm + SL::B_PI)[jrow];
 
     GDR_CHAIN_PHASE(1);
-    // ---- V~ = U - Y S0 -> bf16 (rows = tokens)
-    {
+    // ---- V~ = U - Y S0 -> bf16 (rows = tokens), on the warps that own lanes C..2C-1
+    if (qd >= 2) {
+      const int t = 32 * (qd - 2) + lane;
       float d[32];
-      tmem_ld_32x32b_x32(tD1 + lane_q + hf * HALF, d);
+      tmem_ld_32x32b_x32(tD + lane_q + hf * HALF, d);
       tmem_ld_wait();
-      if (lane < 16) {
-        const int t = 16 * qd + lane;
-        float u[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-          float u8[8];
-          unpack8(*reinterpret_cast<const uint4 *>(bsm + SL::B_U +
-                                                  sw128_offset(t, hf * HALF + i, kC * 128)), u8);
+      for (int i = 0; i < HALF; i += 8) {
+        float u8[8];
+        unpack8(*reinterpret_cast<const uint4 *>(bsm + SL::B_U + sw128_offset(t, hf * HALF + i, kC * 128)), u8);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) u[i + e] = (t < n) ? u8[e] - d[i + e] : 0.f;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          st_smem16(smem, SL::VT + sw128_offset(t, hf * HALF + i, kC * 128), pack8(u + i));
+        for (int e = 0; e < 8; ++e) u8[e] = (t < n) ? u8[e] - d[i + e] : 0.f;
+        st_smem16(smem, SL::VT + sw128_offset(t, hf * HALF + i, kC * 128), pack8(u8));
       }
     }
     fence_proxy_async_smem();
@@ -590,22 +638,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     __syncthreads();
 
     GDR_CHAIN_PHASE(2);
-    // ---- MMA4: K~^T V~ (M = DK) and DO[c & 1] += M V~ (M = C); K = C
-    if (tid == 0) {
+    // ---- MMA4: DS = K~^T V~ (M = DK) and D[c & 1] += [M; *] V~ (M = 128); K = C
+    if (warp == 0) {
       tc_fence_after();
       constexpr uint32_t ids = idesc_bf16_f32(128, NV, true, true);
-      constexpr uint32_t ido = idesc_bf16_f32(64, NV, false, true);
+      constexpr uint32_t ido = idesc_bf16_f32(128, NV, false, true);
 #pragma unroll
       for (int s = 0; s < kC / 16; ++s) {
         const uint64_t ak = sdesc_sw128(bb + Rec::KT + s * 2048, kC * 128, 1024);
         const uint64_t bv = sdesc_sw128(sb + SL::VT + s * 2048, kC * 128, 1024);
         const uint64_t am = sdesc_sw128(bb + Rec::MM + s * 32, 16, 1024);
-        mma_bf16(tDS, ak, bv, ids, s > 0);
-        mma_bf16(tmem + 64 + 64 * (c & 1), am, bv, ido, 1);
+        mma_bf16_warp(tDS, ak, bv, ids, s > 0);
+        mma_bf16_warp(tD, am, bv, ido, 1);
       }
-      mma_commit(mbar);
+      mma_commit_warp(bar4);
+      ++iss4;
     }
-    if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    if (!(ok = wait_mma(bar4, ph4, sabort))) break;
 
     GDR_CHAIN_PHASE(3);
     // ---- state update (fp32) and its bf16 copy for the next MMA3
@@ -624,38 +673,31 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     __syncthreads();
 
     GDR_CHAIN_PHASE(4);
-    // ---- start chunk c + 1 (MMA3) and refill this chunk's buffer, then store O (c)
-    //      while that MMA runs
-    if (tid == 0 && c + 1 < nch && !*sabort) {
-      const int nb = (c + 1) % NBUF;
-      if (mbar_wait_bounded(full + nb, ((c + 1) / NBUF) & 1, kWaitLimitNs)) {
-        ++fdone[nb];
-        issue_mma3<NV>(sb, tmem, c + 1, mbar);
-        if (c + NBUF < nch) {
-          fence_proxy_async_smem();   // this CTA's reads of the buffer come before the refill
-          ++fissue[buf];
-          fetch_record<NV>(smem, full, recs, c + NBUF, slice);
-        }
-      } else {
-        *sabort = 1;
-      }
+    // ---- warp 0 starts chunk c + 1; warp 2 refills this chunk's buffer (every read
+    //      of it is done); warps owning lanes 0..C-1 store O (c) meanwhile
+    if (warp == 0 && c + 1 < nch && !*sabort) {
+      if (start_chunk<NV>(smem, sb, tmem, c + 1)) ++iss3;
+      else if (lane == 0) *sabort = 1;
     }
-    {
+    if (warp == 2 && lane == 0 && c + NBUF < nch && !*sabort) {
+      fence_proxy_async_smem();   // the CTA's reads of the buffer come before the refill
+      fetch_record<NV>(smem, full, fiss, recs, c + NBUF, slice);
+    }
+    GDR_CHAIN_PHASE(5);
+    if (qd < 2) {
       float o[32];
-      tmem_ld_32x32b_x32(tmem + 64 + 64 * (c & 1) + lane_q + hf * HALF, o);
+      tmem_ld_32x32b_x32(tD + lane_q + hf * HALF, o);
       tmem_ld_wait();
-      if (lane < 16) {
-        const int t = 16 * qd + lane;
-        if (t < n) {
-          float4 *dst = reinterpret_cast<float4 *>(
-              p.o + (((size_t)b * T + t0 + t) * H + h) * kDK + c0 + hf * HALF);
+      const int t = 32 * qd + lane;
+      if (t < n) {
+        float4 *dst = reinterpret_cast<float4 *>(
+            p.o + (((size_t)b * T + t0 + t) * H + h) * kDK + c0 + hf * HALF);
 #pragma unroll
-          for (int i = 0; i < HALF; i += 4) dst[i / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
-        }
+        for (int i = 0; i < HALF; i += 4) dst[i / 4] = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
       }
     }
     tc_fence_before();
-    GDR_CHAIN_PHASE(5);
+    GDR_CHAIN_PHASE(6);
   }
 
   GDR_PHASE_FINI(0)
@@ -664,12 +706,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     for (int i = 0; i < HALF; i += 4)
       *reinterpret_cast<float4 *>(p.S_T + s_off + i) = make_float4(st[i], st[i + 1], st[i + 2], st[i + 3]);
   }
-  if (!ok && tid == 0) {
+  // after a timeout: let the MMAs and record copies already in flight land before
+  // the CTA exits (every wait bounded)
+  __syncthreads();
+  if (!ok && tid == 0) {   // thread 0 is warp 0's issuing lane: iss3 / iss4 are its counts
     if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
-    // let MMAs and record copies already in flight land before the CTA exits
-    mbar_wait_bounded(mbar, phase, kWaitLimitNs);
+    // groups complete in order: wait for the last one committed on each barrier
+    if (iss3 > 0) mbar_wait_bounded(bar3, (iss3 - 1) & 1, kWaitLimitNs);
+    if (iss4 > 0) mbar_wait_bounded(bar4, (iss4 - 1) & 1, kWaitLimitNs);
     for (int bq = 0; bq < NBUF; ++bq)
-      while (fdone[bq] < fissue[bq]) {
+      while (fdone[bq] < fiss[bq]) {
         if (!mbar_wait_bounded(full + bq, fdone[bq] & 1, kWaitLimitNs)) break;
         ++fdone[bq];
       }

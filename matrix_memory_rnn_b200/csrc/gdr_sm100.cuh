@@ -152,6 +152,33 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// Warp-collective forms: every lane of a converged warp executes the call, so the
+// operands are computed as warp-uniform values, and lane 0 alone issues the
+// instruction (a predicate inside the asm, not a divergent branch).  Issued this
+// way a tcgen05.mma costs about half the issue time of the same instruction from
+// a lone thread behind `if (threadIdx.x == 0)`.  The MMAs and the commit that
+// tracks them come from the same lane, as tcgen05.commit requires.
+__device__ __forceinline__ void mma_bf16_warp(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t.reg .u32 l;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "mov.u32 l, %%laneid;\n\t"
+      "setp.eq.u32 e, l, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_warp(uint64_t *bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t.reg .u32 l;\n\t"
+      "mov.u32 l, %%laneid;\n\t"
+      "setp.eq.u32 e, l, 0;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
 // Arrives (once) on `bar` when every tcgen05 operation this thread issued so far completes.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile(
