@@ -7,20 +7,24 @@
 //
 //  * prep: everything that does not depend on the chunk's initial state S0 --
 //    the cumulative log-decay, the decay-weighted products L and M (one tcgen05
-//    MMA), T^-1 (fp32), U = T^-1 V^ and Y = T^-1 K^_pi (one MMA group), and the
-//    operand tiles Q_pi and K~.  Chunks are independent, so one CTA per
-//    (b, h, chunk) runs them all in parallel (about 107 KB of shared memory, two
-//    CTAs per SM).  Each CTA writes a record of bf16 MMA tiles, already in the
-//    128-byte-swizzled shared-memory layout, to the workspace.
+//    MMA), T^-1 (fp32 diagonal blocks, tf32 warp-MMA merges), U = T^-1 V^ and
+//    Y = T^-1 K^_pi (one tcgen05 MMA group), and the operand tiles Q_pi and K~.
+//    Chunks are independent: a persistent grid of one 512-thread CTA per SM walks
+//    them, staging each chunk's inputs in shared memory with cp.async while the
+//    previous chunk's MMAs, T^-1 and readouts run.  Each chunk's result is a
+//    record of bf16 MMA tiles, already in the 128-byte-swizzled shared-memory
+//    layout, in the workspace.
 //  * chain: the inter-chunk state carry and the outputs, sequential over chunks
 //    for each (b, h, 64-column value slice):
 //        V~ = U - Y S0,   S_C = Diag(pi_n) S0 + K~^T V~,   O = Q_pi S0 + M V~.
-//    Records are fetched with bulk (TMA) copies two chunks ahead into a
-//    double buffer, so every chunk step is two MMA groups and two short
-//    CUDA-core phases.
+//    Records are fetched with bulk (TMA) copies three chunks ahead into a ring of
+//    three buffers, so every chunk step is two MMA groups and two short CUDA-core
+//    phases.
 //
 // The workspace holds one record (74752 bytes) per (b, h, chunk) after a
 // 1024-byte header whose first word is the device status word.
+#include <type_traits>
+
 #include "gdr_tc_common.cuh"
 
 // Phase hooks for an external timing harness; empty in the library build.
@@ -74,6 +78,13 @@ constexpr size_t kHeaderBytes = 1024;
 __host__ __device__ inline int num_chunks(int T) { return (T + kC - 1) / kC; }
 
 // ============================================================== prep kernel
+// Persistent: one CTA of 512 threads per SM walks the chunks (b, h, c) with a
+// stride of gridDim.x.  A chunk's inputs are staged in shared memory by cp.async;
+// the copies for the CTA's next chunk are issued as soon as this chunk's
+// element-wise phase has consumed the staging area, so they land while the MMAs,
+// T^-1 and the readouts of this chunk run.
+constexpr int kPrepThreads = 512;
+
 // fp32 64 x 64 T^-1 in the Q rows of the [K^ f; Q f] tile once MMA1 has read them:
 // those rows are two 8 KB pieces (one per 64-column atom), rows 0..31 in the
 // first and 32..63 in the second; 16-byte groups XOR-permuted by (r & 15).
@@ -84,24 +95,63 @@ struct QRowsIdx {
 };
 
 struct PrepSmem {
-  static constexpr uint32_t A_LM = 0;                       // [K^ f; Q f]  2C x DK bf16; Q rows
-                                                            //   then hold fp32 T^-1 (QRowsIdx)
-  static constexpr uint32_t B_LM = A_LM + 2 * kC * kDK * 2;  // K g          C x DK bf16; then fp32 L;
-                                                            //   then bf16 T^-1 (first 8 KB)
-  static constexpr uint32_t VH = B_LM + kC * kDK * 2;        // v, then V^ = wg v in place, C x DV bf16
-  static constexpr uint32_t WG = VH + kC * kDK * 2;          // write gate  C x DV bf16
-  static constexpr uint32_t SCAN = WG + kC * kDK * 2;        // fp32 [16 token blocks][DK] log-decay sums
-  static constexpr uint32_t L1 = SCAN + 16 * kDK * 4;        // fp32 Lam_1 per channel
-  static constexpr uint32_t A1 = L1 + kDK * 4;               // fp32 alpha_1 per channel
-  static constexpr uint32_t MISC = A1 + kDK * 4;             // mbarrier, TMEM slot, flags
+  // staging: row-major token rows (bf16 256 B, fp32 512 B), zero past the sequence end
+  static constexpr uint32_t SK = 0;
+  static constexpr uint32_t SB = SK + kC * kDK * 2;
+  static constexpr uint32_t SQ = SB + kC * kDK * 2;
+  static constexpr uint32_t SV = SQ + kC * kDK * 2;
+  static constexpr uint32_t SW = SV + kC * kDK * 2;
+  static constexpr uint32_t SLW = SW + kC * kDK * 2;          // log w, then Lam_t - Lam_1
+  static constexpr uint32_t A_LM = SLW + kC * kDK * 4;        // [K^ f; Q f] 2C x DK bf16; Q rows
+                                                              //   then hold fp32 T^-1 (QRowsIdx)
+  static constexpr uint32_t B_LM = A_LM + 2 * kC * kDK * 2;   // K g  C x DK bf16; then fp32 L;
+                                                              //   then bf16 T^-1 (first 8 KB)
+  static constexpr uint32_t VH = B_LM + kC * kDK * 2;         // V^ = wg (.) v  C x DV bf16
+  static constexpr uint32_t QT = VH + kC * kDK * 2;           // fp32 [4][DK] quarter sums of log w
+  static constexpr uint32_t L1 = QT + 4 * kDK * 4;            // fp32 Lam_1 per channel
+  static constexpr uint32_t DN = L1 + kDK * 4;                // fp32 Lam_n - Lam_1 per channel
+  static constexpr uint32_t A1 = DN + kDK * 4;                // fp32 alpha_1 = exp(Lam_1)
+  static constexpr uint32_t MISC = A1 + kDK * 4;              // mbarrier, TMEM slot, flags
   static constexpr uint32_t ALLOC = MISC + 64 + 1024;
+  static_assert(A_LM % 1024 == 0 && B_LM % 1024 == 0 && VH % 1024 == 0, "MMA tiles 1024-aligned");
   static_assert(Ix::kBytes <= kC * kDK * 2, "fp32 L must fit the reused bf16 tile");
+  static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-// Thread layout of the elementwise phases: thread = (channel group g of 8 channels,
-// token block tb of 4 consecutive tokens); a warp covers two token blocks, and the
-// 16 threads of a token row read its 256 contiguous bytes.
-__global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8_t *records) {
+// All threads: cp.async one chunk's q, k, b, v, wg and log w into the staging area
+// (rows t >= n are zero-filled), as one commit group.
+__device__ __forceinline__ void stage_chunk(uint8_t *smem, const FwdParams &p, int b, int h, int t0,
+                                            int n, int tid) {
+  using SL = PrepSmem;
+  const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
+  const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
+  const __nv_bfloat16 *gv = static_cast<const __nv_bfloat16 *>(p.v);
+  const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
+  const __nv_bfloat16 *gw = static_cast<const __nv_bfloat16 *>(p.e2);
+  const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;   // token row of t0 in [B][T][H]
+#pragma unroll
+  for (int u = 0; u < kC * 16 / kPrepThreads; ++u) {
+    const int it = tid + u * kPrepThreads, t = it >> 4, cc = it & 15;
+    const bool valid = t < n;
+    const size_t off = valid ? (row0 + (size_t)t * p.H) * kDK + cc * 8 : 0;
+    const uint32_t so = t * 256 + cc * 16;
+    cp_async16(smem + SL::SK + so, gk + off, valid);
+    cp_async16(smem + SL::SB + so, gb + off, valid);
+    cp_async16(smem + SL::SQ + so, gq + off, valid);
+    cp_async16(smem + SL::SV + so, gv + off, valid);
+    if (gw) cp_async16(smem + SL::SW + so, gw + off, valid);
+  }
+#pragma unroll
+  for (int u = 0; u < kC * 32 / kPrepThreads; ++u) {
+    const int it = tid + u * kPrepThreads, t = it >> 5, cc = it & 31;
+    const bool valid = t < n;
+    const size_t off = valid ? (row0 + (size_t)t * p.H) * kDK + cc * 4 : 0;
+    cp_async16(smem + SL::SLW + t * 512 + cc * 16, p.log_w + off, valid);
+  }
+  cp_async_commit();
+}
+
+__global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(FwdParams p, uint8_t *records) {
   using SL = PrepSmem;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -109,62 +159,25 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   const uint32_t sb = smem_u32(smem);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, hf = warp >> 2;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int T = p.T, H = p.H, t0 = c * kC, n = min(kC, T - t0);
-  uint8_t *rec = records + ((size_t)((size_t)b * H + h) * num_chunks(T) + c) * Rec::BYTES;
-  const int g = tid & 15, tb = tid >> 4, j0 = 8 * g;
+  const int qd = warp & 3, cpart = warp >> 2;             // TMEM lane quarter, column part
+  const int T = p.T, H = p.H, nch = num_chunks(T);
+  const int items = p.B * H * nch;
   GDR_PHASE_INIT
 
+  float *sLW = reinterpret_cast<float *>(smem + SL::SLW);
   float *sL = reinterpret_cast<float *>(smem + SL::B_LM);
   float *sTi = reinterpret_cast<float *>(smem + SL::A_LM);
-  float *sScan = reinterpret_cast<float *>(smem + SL::SCAN);
+  float *sQT = reinterpret_cast<float *>(smem + SL::QT);
   float *sL1 = reinterpret_cast<float *>(smem + SL::L1);
+  float *sDN = reinterpret_cast<float *>(smem + SL::DN);
   float *sA1 = reinterpret_cast<float *>(smem + SL::A1);
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + SL::MISC);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 8);
   volatile int *sflag = reinterpret_cast<volatile int *>(smem + SL::MISC + 16);  // exact, abort
-
   const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
-  const __nv_bfloat16 *gv = static_cast<const __nv_bfloat16 *>(p.v);
   const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
-  const __nv_bfloat16 *gw = static_cast<const __nv_bfloat16 *>(p.e2);
-  auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
-
-  // ---- every global read is issued here: log w, k, b, q into registers (this
-  //      thread's 4 tokens x 8 channels); v and wg by cp.async into their swizzled
-  //      positions (zero-filled past the end of the sequence)
-  float lam[4][8];
-  uint4 rk[4], rb[4], rq[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = 4 * tb + i;
-    if (t < n) {
-      const size_t off = tok_off(t) + j0;
-      const float4 x0 = __ldg(reinterpret_cast<const float4 *>(p.log_w + off));
-      const float4 x1 = __ldg(reinterpret_cast<const float4 *>(p.log_w + off + 4));
-      lam[i][0] = x0.x; lam[i][1] = x0.y; lam[i][2] = x0.z; lam[i][3] = x0.w;
-      lam[i][4] = x1.x; lam[i][5] = x1.y; lam[i][6] = x1.z; lam[i][7] = x1.w;
-      rk[i] = ld16(gk + off);
-      rb[i] = ld16(gb + off);
-      rq[i] = ld16(gq + off);
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) lam[i][e] = 0.f;
-      rk[i] = rb[i] = rq[i] = make_uint4(0u, 0u, 0u, 0u);
-    }
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int it = tid + u * kThreads, t = it >> 4, gg = it & 15;
-    const bool valid = t < n;
-    const size_t off = valid ? tok_off(t) + 8 * gg : 0;
-    const uint32_t so = sw128_offset(t, 8 * gg, kC * 128);
-    cp_async16(smem + SL::VH + so, gv + off, valid);
-    if (gw) cp_async16(smem + SL::WG + so, gw + off, valid);
-  }
-  cp_async_commit();
+  const bool has_wg = p.e2 != nullptr;
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -173,187 +186,196 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
   if (tid == 0) {
     mbar_init(mbar, 1);
     fence_mbar_init();
-    sflag[0] = 0;
     sflag[1] = 0;
   }
-
-  GDR_PREP_PHASE(0);
-  // ---- cumulative log-decay: prefix within the thread's 4 tokens, then across the
-  //      16 token blocks through shared memory
-  {
-    float tot[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        acc += lam[i][e];
-        lam[i][e] = acc;
-      }
-      tot[e] = acc;
-    }
-    float4 *dst = reinterpret_cast<float4 *>(sScan + tb * kDK + j0);
-    dst[0] = make_float4(tot[0], tot[1], tot[2], tot[3]);
-    dst[1] = make_float4(tot[4], tot[5], tot[6], tot[7]);
-    if (tb == 0) {
-      float4 *l1 = reinterpret_cast<float4 *>(sL1 + j0);
-      l1[0] = make_float4(lam[0][0], lam[0][1], lam[0][2], lam[0][3]);
-      l1[1] = make_float4(lam[0][4], lam[0][5], lam[0][6], lam[0][7]);
-    }
+  int item = blockIdx.x;
+  if (item < items) {
+    const int c = item % nch, bh = item / nch;
+    stage_chunk(smem, p, bh / H, bh % H, c * kC, min(kC, T - c * kC), tid);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
-  // lam[i][e] becomes Lam_t - Lam_1 (the pivot at the chunk's first token); dn = Lam_n - Lam_1
-  float dn[8], a1[8], ed[8];
-  {
-    float excl[8], all[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) excl[e] = all[e] = 0.f;
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const float4 *src = reinterpret_cast<const float4 *>(sScan + r * kDK + j0);
-      const float4 x0 = src[0], x1 = src[1];
-      const float v8[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        all[e] += v8[e];
-        if (r < tb) excl[e] += v8[e];
-      }
-    }
-    const float4 *l1 = reinterpret_cast<const float4 *>(sL1 + j0);
-    const float4 y0 = l1[0], y1 = l1[1];
-    const float l1v[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-    bool over = false;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) lam[i][e] += excl[e] - l1v[e];
-      dn[e] = all[e] - l1v[e];
-      a1[e] = __expf(l1v[e]);
-      ed[e] = __expf(dn[e]);
-      over |= dn[e] < -kMaxChunkDecay;
-    }
-    if (over) sflag[0] = 1;
-    if (tb == 0) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        sA1[j0 + e] = a1[e];
-        reinterpret_cast<float *>(rec + Rec::PI)[j0 + e] = __expf(all[e]);
-      }
-    }
-  }
-
-  GDR_PREP_PHASE(1);
-  // ---- operand tiles: [K^ f; Q f], K g in shared memory; Q_pi, K~ straight to the record
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = 4 * tb + i;
-    float k8[8], b8[8], q8[8];
-    unpack8(rk[i], k8);
-    unpack8(rb[i], b8);
-    unpack8(rq[i], q8);
-    float av[8], aq[8], bl[8], kt[8], qp[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float f = __expf(lam[i][e]);
-      av[e] = b8[e] * k8[e] * f;
-      aq[e] = q8[e] * f;
-      qp[e] = aq[e] * a1[e];
-      if (dn[e] >= -kMaxChunkDecay) {
-        bl[e] = k8[e] * __expf(-lam[i][e]);
-        kt[e] = bl[e] * ed[e];
-      } else {           // this chunk takes the exact path; K g is not used
-        bl[e] = 0.f;
-        kt[e] = k8[e] * __expf(dn[e] - lam[i][e]);
-      }
-    }
-    const uint32_t o64 = sw128_offset(t, j0, kC * 128);
-    st_smem16(smem, SL::A_LM + sw128_offset(t, j0, 2 * kC * 128), pack8(av));
-    st_smem16(smem, SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128), pack8(aq));
-    st_smem16(smem, SL::B_LM + o64, pack8(bl));
-    *reinterpret_cast<uint4 *>(rec + Rec::QY + sw128_offset(t, j0, Rec::QY_STRIDE)) = pack8(qp);
-    *reinterpret_cast<uint4 *>(rec + Rec::KT + o64) = pack8(kt);
-  }
-  GDR_PREP_PHASE(9);
-  fence_proxy_async_smem();
-  GDR_PREP_PHASE(10);
-  __syncthreads();
-  const bool exact = sflag[0] != 0;
-  // the exact path needs Lam_t - Lam_1 for every (token, channel): park it in the
-  // record's Y rows and U tile, which are written only at the end
-  if (exact) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = 4 * tb + i;
-      float *dst = reinterpret_cast<float *>(rec + park_row(t)) + j0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dst[e] = lam[i][e];
-    }
-  }
-
   uint32_t phase = 0;
   bool ok = true;
-  GDR_PREP_PHASE(2);
-  // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
-  if (warp == 0) {
-    tc_fence_after();
-    constexpr uint32_t id = idesc_bf16_f32(128, kC, false, false);
-#pragma unroll
-    for (int s = 0; s < kDK / 16; ++s) {
-      const uint64_t ad = sdesc_sw128(sb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
-      const uint64_t bd = sdesc_sw128(sb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
-      mma_bf16_warp(tmem, ad, bd, id, s > 0);
-    }
-    mma_commit_warp(mbar);
-  }
-  // ---- while it runs: V^ = wg (.) v in place (each thread scales the chunks it copied)
-  cp_async_wait<0>();
-  if (gw) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int it = tid + u * kThreads, t = it >> 4, gg = it & 15;
-      const uint32_t so = sw128_offset(t, 8 * gg, kC * 128);
-      float v8[8], w8[8];
-      unpack8(*reinterpret_cast<const uint4 *>(smem + SL::VH + so), v8);
-      unpack8(*reinterpret_cast<const uint4 *>(smem + SL::WG + so), w8);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
-      st_smem16(smem, SL::VH + so, pack8(v8));
-    }
-  }
-  fence_proxy_async_smem();
-  GDR_PREP_PHASE(3);
-  ok = wait_mma(mbar, phase, sflag + 1);
 
-  if (ok) {
+  for (; item < items; item += gridDim.x) {
+    const int c = item % nch, bh = item / nch, h = bh % H, b = bh / H;
+    const int t0 = c * kC, n = min(kC, T - t0);
+    uint8_t *rec = records + (size_t)item * Rec::BYTES;   // item order = (b, h, c) record order
+    auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
+    GDR_PREP_PHASE(0);
+
+    cp_async_wait<0>();
+    if (tid == 0) sflag[0] = 0;
+    __syncthreads();
+
+    // ---- cumulative log-decay: thread = (channel ch, token quarter qt), in place
+    {
+      const int ch = tid & (kDK - 1), qt = tid >> 7;
+      float x[16];
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        acc += sLW[(16 * qt + i) * kDK + ch];
+        x[i] = acc;
+      }
+      sQT[qt * kDK + ch] = acc;
+      if (qt == 0) sL1[ch] = x[0];
+      __syncthreads();
+      float excl = 0.f, all = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float v = sQT[q * kDK + ch];
+        all += v;
+        excl += (q < qt) ? v : 0.f;
+      }
+      const float l1 = sL1[ch], shift = excl - l1;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sLW[(16 * qt + i) * kDK + ch] = x[i] + shift;
+      if (qt == 0) {
+        const float dn = all - l1;
+        sDN[ch] = dn;
+        sA1[ch] = __expf(l1);
+        reinterpret_cast<float *>(rec + Rec::PI)[ch] = __expf(all);
+        if (dn < -kMaxChunkDecay) sflag[0] = 1;
+      }
+    }
+    __syncthreads();
+    const bool exact = sflag[0] != 0;
+    GDR_PREP_PHASE(1);
+
+    // ---- operand tiles: [K^ f; Q f], K g in shared memory; Q_pi, K~ to the record.
+    //      Thread = (channel group g of 8, token pair tb); the exact path also parks
+    //      Lam_t - Lam_1 in the record.
+    {
+      const int g = tid & 15, tb = tid >> 4, j0 = 8 * g;
+      float dn[8], a1[8], ed[8];
+      {
+        const float4 d0 = *reinterpret_cast<const float4 *>(sDN + j0);
+        const float4 d1 = *reinterpret_cast<const float4 *>(sDN + j0 + 4);
+        const float4 a0 = *reinterpret_cast<const float4 *>(sA1 + j0);
+        const float4 a4 = *reinterpret_cast<const float4 *>(sA1 + j0 + 4);
+        dn[0] = d0.x; dn[1] = d0.y; dn[2] = d0.z; dn[3] = d0.w;
+        dn[4] = d1.x; dn[5] = d1.y; dn[6] = d1.z; dn[7] = d1.w;
+        a1[0] = a0.x; a1[1] = a0.y; a1[2] = a0.z; a1[3] = a0.w;
+        a1[4] = a4.x; a1[5] = a4.y; a1[6] = a4.z; a1[7] = a4.w;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ed[e] = __expf(dn[e]);
+      }
+      auto operands = [&](auto exact_path) {
+        constexpr bool kExact = decltype(exact_path)::value;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int t = 2 * tb + i;
+          const float4 l0 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0);
+          const float4 l4 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0 + 4);
+          const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l4.x, l4.y, l4.z, l4.w};
+          float k8[8], b8[8], q8[8];
+          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SK + t * 256 + g * 16), k8);
+          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SB + t * 256 + g * 16), b8);
+          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SQ + t * 256 + g * 16), q8);
+          float av[8], aq[8], bl[8], kt[8], qp[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float f = __expf(lam[e]);
+            av[e] = b8[e] * k8[e] * f;
+            aq[e] = q8[e] * f;
+            qp[e] = aq[e] * a1[e];
+            if (!kExact) {
+              bl[e] = k8[e] * __expf(-lam[e]);
+              kt[e] = bl[e] * ed[e];
+            } else if (dn[e] >= -kMaxChunkDecay) {
+              kt[e] = k8[e] * __expf(-lam[e]) * ed[e];
+              bl[e] = 0.f;     // the exact path forms L and M without K g
+            } else {
+              kt[e] = k8[e] * __expf(dn[e] - lam[e]);
+              bl[e] = 0.f;
+            }
+          }
+          const uint32_t o64 = sw128_offset(t, j0, kC * 128);
+          st_smem16(smem, SL::A_LM + sw128_offset(t, j0, 2 * kC * 128), pack8(av));
+          st_smem16(smem, SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128), pack8(aq));
+          st_smem16(smem, SL::B_LM + o64, pack8(bl));
+          *reinterpret_cast<uint4 *>(rec + Rec::QY + sw128_offset(t, j0, Rec::QY_STRIDE)) = pack8(qp);
+          *reinterpret_cast<uint4 *>(rec + Rec::KT + o64) = pack8(kt);
+          if (kExact) {
+            float4 *dst = reinterpret_cast<float4 *>(rec + park_row(t)) + g * 2;
+            dst[0] = l0;
+            dst[1] = l4;
+          }
+        }
+      };
+      if (!exact) operands(std::false_type{});
+      else operands(std::true_type{});
+    }
+    // ---- V^ = wg (.) v into its swizzled tile
+#pragma unroll
+    for (int u = 0; u < kC * 16 / kPrepThreads; ++u) {
+      const int it = tid + u * kPrepThreads, t = it >> 4, gg = it & 15;
+      uint4 vv = *reinterpret_cast<const uint4 *>(smem + SL::SV + t * 256 + gg * 16);
+      if (has_wg) {
+        float v8[8], w8[8];
+        unpack8(vv, v8);
+        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SW + t * 256 + gg * 16), w8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+        vv = pack8(v8);
+      }
+      st_smem16(smem, SL::VH + sw128_offset(t, 8 * gg, kC * 128), vv);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    GDR_PREP_PHASE(2);
+
+    // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
+    if (warp == 0) {
+      tc_fence_after();
+      constexpr uint32_t id = idesc_bf16_f32(128, kC, false, false);
+#pragma unroll
+      for (int s = 0; s < kDK / 16; ++s) {
+        const uint64_t ad = sdesc_sw128(sb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(sb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
+        mma_bf16_warp(tmem, ad, bd, id, s > 0);
+      }
+      mma_commit_warp(mbar);
+    }
+    // ---- the staging area is free: start the CTA's next chunk's copies
+    {
+      const int nx = item + gridDim.x;
+      if (nx < items) {
+        const int cn = nx % nch, bhn = nx / nch;
+        stage_chunk(smem, p, bhn / H, bhn % H, cn * kC, min(kC, T - cn * kC), tid);
+      }
+    }
+    GDR_PREP_PHASE(3);
+    if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
     GDR_PREP_PHASE(4);
+
     // ---- L (fp32, strictly lower; into the dead K g tile) and M (bf16 -> record)
     if (!exact) {
-      float x[32];
-      tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * qd) << 16) + 32 * hf, x);
+      float x[16];
+      tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * qd) << 16) + 16 * cpart, x);
       tmem_ld_wait();
-      const int r = 32 * qd + lane;
+      const int r = 32 * qd + lane, col = 16 * cpart;
       if (r < kC) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i < r) ? x[i] : 0.f;
+        for (int i = 0; i < 16; ++i) x[i] = (col + i < r) ? x[i] : 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          *reinterpret_cast<float4 *>(sL + Ix::at(r, 32 * hf + i)) =
-              make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        for (int i = 0; i < 16; i += 4)
+          *reinterpret_cast<float4 *>(sL + Ix::at(r, col + i)) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
       } else {
         const int t = r - kC;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = (32 * hf + i <= t) ? x[i] : 0.f;
+        for (int i = 0; i < 16; ++i) x[i] = (col + i <= t) ? x[i] : 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          *reinterpret_cast<uint4 *>(rec + Rec::MM + sw128_offset(t, 32 * hf + i, kC * 128)) =
-              pack8(x + i);
+        for (int i = 0; i < 16; i += 8)
+          *reinterpret_cast<uint4 *>(rec + Rec::MM + sw128_offset(t, col + i, kC * 128)) = pack8(x + i);
       }
     } else {
       // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound)
-      for (int it = tid; it < kC * kC; it += kThreads) {
+      for (int it = tid; it < kC * kC; it += kPrepThreads) {
         const int t = it / kC, s = it % kC;
         float l = 0.f, m = 0.f;
         if (s <= t && t < n) {
@@ -374,12 +396,14 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     }
     tc_fence_before();
     __syncthreads();
-
     GDR_PREP_PHASE(5);
+
     // ---- T^-1 (fp32, into the dead Q rows of A_LM), bf16 copy (into the dead L tile)
-    invert_unit_lower<Ix, QRowsIdx>(sL, sTi, tid);
-    for (int it = tid; it < kC * (kC / 8); it += kThreads) {
-      const int t = it >> 3, gg = it & 7;
+    invert_diag_blocks<Ix, QRowsIdx, kPrepThreads>(sL, sTi, tid);
+    GDR_PREP_PHASE(9);
+    invert_merge_levels<Ix, QRowsIdx, kPrepThreads>(sL, sTi, tid);
+    {
+      const int t = tid >> 3, gg = tid & 7;
       const float4 y0 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg));
       const float4 y1 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg + 4));
       float x[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
@@ -393,8 +417,8 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
-
     GDR_PREP_PHASE(6);
+
     // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
     if (warp == 0) {
       tc_fence_after();
@@ -409,38 +433,48 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
       }
       mma_commit_warp(mbar);
     }
-    ok = wait_mma(mbar, phase, sflag + 1);
-  }
-
-  if (ok) {
+    if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
     GDR_PREP_PHASE(7);
-    // ---- U and Y (x alpha_1) -> bf16 record tiles; M = 64 accumulators: row 16 qd + lane
-    const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
-    float x[32];
+
+    // ---- U and Y (x alpha_1) -> bf16 record tiles; M = 64 accumulators: row 16 qd + lane.
+    //      Column part cpart: 0, 1 -> U columns, 2, 3 -> Y columns (64 each).
+    {
+      const bool is_y = cpart >= 2;
+      const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
 #pragma unroll
-    for (int part = 0; part < 4; ++part) {
-      const int col = 64 * hf + 32 * (part & 1);        // 0..127 within U or Y
-      const bool is_y = part >= 2;
-      tmem_ld_32x32b_x32(tmem + lane_q + (is_y ? kDK : 0) + col, x);
-      tmem_ld_wait();
-      if (lane < 16) {
-        const int t = 16 * qd + lane;
-        if (is_y) {
+      for (int half = 0; half < 2; ++half) {
+        const int col = 64 * (cpart & 1) + 32 * half;    // 0..127 within U or Y
+        float x[32];
+        tmem_ld_32x32b_x32(tmem + lane_q + (is_y ? kDK : 0) + col, x);
+        tmem_ld_wait();
+        if (lane < 16) {
+          const int t = 16 * qd + lane;
+          if (is_y) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) x[i] *= sA1[col + i];
+            for (int i = 0; i < 32; i += 4) {
+              const float4 a = *reinterpret_cast<const float4 *>(sA1 + col + i);
+              x[i] *= a.x; x[i + 1] *= a.y; x[i + 2] *= a.z; x[i + 3] *= a.w;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 32; i += 8)
+            *reinterpret_cast<uint4 *>(
+                rec + (is_y ? Rec::QY + sw128_offset(kC + t, col + i, Rec::QY_STRIDE)
+                            : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
         }
-#pragma unroll
-        for (int i = 0; i < 32; i += 8)
-          *reinterpret_cast<uint4 *>(
-              rec + (is_y ? Rec::QY + sw128_offset(kC + t, col + i, Rec::QY_STRIDE)
-                          : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
       }
     }
-  } else if (tid == 0 && p.status) {
-    atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
+    tc_fence_before();
+    GDR_PREP_PHASE(8);
   }
-  GDR_PREP_PHASE(8);
+
   GDR_PHASE_FINI(1)
+  cp_async_wait<0>();
+  if (!ok && tid == 0) {
+    if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
+    // the MMA group whose wait ran out may still be running: let it finish (bounded)
+    mbar_wait_bounded(mbar, phase ^ 1u, kWaitLimitNs);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -459,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 2) tc_prep_kernel(FwdParams p, uint8
 //   S <- Diag(pi_n) S + DS                 (fp32, all warps)
 //   O = rows 0..C-1 of D[c&1]              (read while MMA3 of chunk c + 1 runs)
 // Warp 0 issues the MMAs (lane 0, from converged code); warp 2 refills the record
-// ring three chunks ahead.
+// ring three chunks ahead as soon as MMA4 has released a buffer.
 template <int NV>
 struct ChainSmem {
   // per buffer: QY | KT | MM | U slice (C x NV) | pi.  The U slice sits directly after
@@ -655,6 +689,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
       ++iss4;
     }
     if (!(ok = wait_mma(bar4, ph4, sabort))) break;
+    // every read of this chunk's buffer is done: refill it three chunks ahead
+    if (warp == 2 && lane == 0 && c + NBUF < nch && !*sabort) {
+      fence_proxy_async_smem();   // the CTA's reads of the buffer come before the refill
+      fetch_record<NV>(smem, full, fiss, recs, c + NBUF, slice);
+    }
 
     GDR_CHAIN_PHASE(3);
     // ---- state update (fp32) and its bf16 copy for the next MMA3
@@ -673,15 +712,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     __syncthreads();
 
     GDR_CHAIN_PHASE(4);
-    // ---- warp 0 starts chunk c + 1; warp 2 refills this chunk's buffer (every read
-    //      of it is done); warps owning lanes 0..C-1 store O (c) meanwhile
+    // ---- warp 0 starts chunk c + 1; warps owning lanes 0..C-1 store O (c) meanwhile
     if (warp == 0 && c + 1 < nch && !*sabort) {
       if (start_chunk<NV>(smem, sb, tmem, c + 1)) ++iss3;
       else if (lane == 0) *sabort = 1;
-    }
-    if (warp == 2 && lane == 0 && c + NBUF < nch && !*sabort) {
-      fence_proxy_async_smem();   // the CTA's reads of the buffer come before the refill
-      fetch_record<NV>(smem, full, fiss, recs, c + NBUF, slice);
     }
     GDR_CHAIN_PHASE(5);
     if (qd < 2) {
@@ -743,8 +777,11 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   e = cudaFuncSetAttribute(tc_chain_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)ChainSmem<NV>::ALLOC);
   if (e != cudaSuccess) return e;
-  dim3 gp(num_chunks(p.T), p.H, p.B);
-  tc_prep_kernel<<<gp, kThreads, PrepSmem::ALLOC, stream>>>(p, records);
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int items = p.B * p.H * num_chunks(p.T);
+  tc_prep_kernel<<<min(items, sms), kPrepThreads, PrepSmem::ALLOC, stream>>>(p, records);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 gc(p.dv / NV, p.H, p.B);
   tc_chain_kernel<NV><<<gc, kThreads, ChainSmem<NV>::ALLOC, stream>>>(p, records);

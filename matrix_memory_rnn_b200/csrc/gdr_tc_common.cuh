@@ -137,6 +137,116 @@ __device__ void invert_unit_lower(float *Lm, float *Ti, int tid) {
 }
 
 
+// fp32 -> tf32 (round to nearest, ties away), as the operand of mma.sync .tf32.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// d += a (16 x 8, row-major) * b (8 x 8), tf32 operands, fp32 accumulate; warp-wide.
+// Fragments (lane = 4 g + t): a0 (g, t) a1 (g+8, t) a2 (g, t+4) a3 (g+8, t+4);
+// b0 (k = t, n = g) b1 (k = t+4, n = g); d0 (g, 2t) d1 (g, 2t+1) d2 (g+8, 2t) d3 (g+8, 2t+1).
+__device__ __forceinline__ void mma_tf32_16x8x8(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                                uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One 16 x 8 tile of D = A B with A (16 x K) at rows r0.., columns k0.. of X (index
+// IxA) and B (K x 8) at rows kb.., columns n0.. of Y (index IxB); K a multiple of 8.
+template <class IxA, class IxB, int K>
+__device__ __forceinline__ void tile_16x8(float (&d)[4], const float *X, int r0, int k0,
+                                          const float *Y, int kb, int n0, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int ks = 0; ks < K; ks += 8) {
+    mma_tf32_16x8x8(d, to_tf32(X[IxA::at(r0 + g, k0 + ks + t)]), to_tf32(X[IxA::at(r0 + g + 8, k0 + ks + t)]),
+                    to_tf32(X[IxA::at(r0 + g, k0 + ks + t + 4)]),
+                    to_tf32(X[IxA::at(r0 + g + 8, k0 + ks + t + 4)]),
+                    to_tf32(Y[IxB::at(kb + ks + t, n0 + g)]), to_tf32(Y[IxB::at(kb + ks + t + 4, n0 + g)]));
+  }
+}
+
+// Stores a 16 x 8 tile (times `sign`) at rows r0.., columns n0.. of Z (index IxZ).
+template <class IxZ>
+__device__ __forceinline__ void store_16x8(const float (&d)[4], float sign, float *Z, int r0, int n0,
+                                           int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  *reinterpret_cast<float2 *>(Z + IxZ::at(r0 + g, n0 + 2 * t)) = make_float2(sign * d[0], sign * d[1]);
+  *reinterpret_cast<float2 *>(Z + IxZ::at(r0 + g + 8, n0 + 2 * t)) = make_float2(sign * d[2], sign * d[3]);
+}
+
+// T^-1 for T = I + L as invert_unit_lower (same blocks, same merge order), for a
+// CTA of NT threads, with the merge products X21 = -T_R^-1 (L_RL T_L^-1) on the
+// tensor cores as warp-level tf32 MMAs (16 x 8 tiles, fp32 accumulate): the
+// diagonal 16 x 16 blocks stay fp32 forward substitution.  Ends with a CTA barrier.
+// Step 1: the four diagonal 16 x 16 blocks (and zeros in the upper blocks level 2 reads).
+template <class IxL, class IxT, int NT>
+__device__ void invert_diag_blocks(const float *Lm, float *Ti, int tid) {
+  if (tid < 64) {
+    const int blk = tid >> 4, c = tid & 15, o = 16 * blk;
+    float x[16];
+#pragma unroll
+    for (int t = 0; t < 16; ++t) {
+      float acc = (t == c) ? 1.f : 0.f;
+#pragma unroll
+      for (int s = 0; s < t; ++s) acc -= Lm[IxL::at(o + t, o + s)] * x[s];
+      x[t] = acc;
+    }
+#pragma unroll
+    for (int t = 0; t < 16; ++t) Ti[IxT::at(o + t, o + c)] = x[t];
+  } else if (tid < 64 + 2 * 256 / 4) {
+    // zero the upper 16 x 16 blocks of the two diagonal 32 x 32 blocks (read by level 2)
+    const int k = (tid - 64) * 4, q = k >> 8, r = 32 * q + ((k >> 4) & 15), c = 32 * q + 16 + (k & 15);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Ti[IxT::at(r, c + e)] = 0.f;
+  }
+  __syncthreads();
+}
+
+// Step 2: the two merge levels on the tensor cores.
+template <class IxL, class IxT, int NT>
+__device__ void invert_merge_levels(float *Lm, float *Ti, int tid) {
+  static_assert(NT >= 256, "level 2 uses eight warps");
+  const int warp = tid >> 5, lane = tid & 31;
+  // level 1: pair q (blocks 2q, 2q+1), column tile nt: W = L_RL T_L^-1, X = -T_R^-1 W
+  const int q1 = warp >> 1, nt1 = warp & 1, o1 = 32 * q1;
+  float w1[4] = {0.f, 0.f, 0.f, 0.f};
+  if (warp < 4) tile_16x8<IxL, IxT, 16>(w1, Lm, o1 + 16, o1, Ti, o1, o1 + 8 * nt1, lane);
+  __syncthreads();
+  if (warp < 4) store_16x8<IxL>(w1, 1.f, Lm, o1 + 16, o1 + 8 * nt1, lane);
+  __syncthreads();
+  if (warp < 4) {
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    tile_16x8<IxT, IxL, 16>(x, Ti, o1 + 16, o1 + 16, Lm, o1 + 16, o1 + 8 * nt1, lane);
+    store_16x8<IxT>(x, -1.f, Ti, o1 + 16, o1 + 8 * nt1, lane);
+  }
+  __syncthreads();
+  // level 2: rows 32..63 x columns 0..31; row tile mt, column tile nt
+  const int mt = warp >> 2, nt2 = warp & 3;
+  float w2[4] = {0.f, 0.f, 0.f, 0.f};
+  if (warp < 8) tile_16x8<IxL, IxT, 32>(w2, Lm, 32 + 16 * mt, 0, Ti, 0, 8 * nt2, lane);
+  __syncthreads();
+  if (warp < 8) store_16x8<IxL>(w2, 1.f, Lm, 32 + 16 * mt, 8 * nt2, lane);
+  __syncthreads();
+  if (warp < 8) {
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    tile_16x8<IxT, IxL, 32>(x, Ti, 32 + 16 * mt, 32, Lm, 32, 8 * nt2, lane);
+    store_16x8<IxT>(x, -1.f, Ti, 32 + 16 * mt, 8 * nt2, lane);
+  }
+  __syncthreads();
+}
+
+template <class IxL, class IxT, int NT>
+__device__ void invert_unit_lower_mma(float *Lm, float *Ti, int tid) {
+  invert_diag_blocks<IxL, IxT, NT>(Lm, Ti, tid);
+  invert_merge_levels<IxL, IxT, NT>(Lm, Ti, tid);
+}
+
 // Row-major C x C fp32 storage for invert_unit_lower: padded rows (68 floats, 16-byte
 // aligned, conflict-free column writes) or exactly 64 floats with the 16-byte
 // groups of row r XOR-permuted by (r & 15) (same properties, no padding).
