@@ -10,8 +10,8 @@
 //    MMA), T^-1 (fp32 diagonal blocks, tf32 warp-MMA merges), U = T^-1 V^ and
 //    Y = T^-1 K^_pi (one tcgen05 MMA group), and the operand tiles Q_pi and K~.
 //    Chunks are independent: a persistent grid of one 512-thread CTA per SM walks
-//    them, staging each chunk's inputs in shared memory with cp.async while the
-//    previous chunk's MMAs, T^-1 and readouts run.  Each chunk's result is a
+//    them; each chunk's inputs arrive in shared memory as six TMA tensor tiles,
+//    issued while the previous chunk's MMAs, T^-1 and readouts run.  Each chunk's result is a
 //    record of bf16 MMA tiles, already in the 128-byte-swizzled shared-memory
 //    layout, in the workspace.
 //  * chain: the inter-chunk state carry and the outputs, sequential over chunks
@@ -23,6 +23,11 @@
 //
 // The workspace holds one record (74752 bytes) per (b, h, chunk) after a
 // 1024-byte header whose first word is the device status word.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+#include <mutex>
 #include <type_traits>
 
 #include "gdr_tc_common.cuh"
@@ -118,40 +123,29 @@ struct PrepSmem {
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-// All threads: cp.async one chunk's q, k, b, v, wg and log w into the staging area
-// (rows t >= n are zero-filled), as one commit group.
-__device__ __forceinline__ void stage_chunk(uint8_t *smem, const FwdParams &p, int b, int h, int t0,
-                                            int n, int tid) {
+// Tensor maps of the prep inputs, each 4-D (channel, head, token, batch) with a box
+// of one chunk of one head: 128 channels x 64 tokens, i.e. 16 KB of bf16 or 32 KB
+// of fp32 in row-major token rows -- the staging layout.  Tokens past T read as 0.
+struct PrepMaps {
+  CUtensorMap k, b, q, v, wg, lw;
+};
+
+// One thread: TMA loads of one chunk's k, b, q, v, (wg,) log w into the staging
+// area, completing on `bar`.
+__device__ __forceinline__ void stage_chunk(uint8_t *smem, const PrepMaps &m, uint64_t *bar, int b,
+                                            int h, int t0, bool has_wg) {
   using SL = PrepSmem;
-  const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
-  const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
-  const __nv_bfloat16 *gv = static_cast<const __nv_bfloat16 *>(p.v);
-  const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
-  const __nv_bfloat16 *gw = static_cast<const __nv_bfloat16 *>(p.e2);
-  const size_t row0 = ((size_t)b * p.T + t0) * p.H + h;   // token row of t0 in [B][T][H]
-#pragma unroll
-  for (int u = 0; u < kC * 16 / kPrepThreads; ++u) {
-    const int it = tid + u * kPrepThreads, t = it >> 4, cc = it & 15;
-    const bool valid = t < n;
-    const size_t off = valid ? (row0 + (size_t)t * p.H) * kDK + cc * 8 : 0;
-    const uint32_t so = t * 256 + cc * 16;
-    cp_async16(smem + SL::SK + so, gk + off, valid);
-    cp_async16(smem + SL::SB + so, gb + off, valid);
-    cp_async16(smem + SL::SQ + so, gq + off, valid);
-    cp_async16(smem + SL::SV + so, gv + off, valid);
-    if (gw) cp_async16(smem + SL::SW + so, gw + off, valid);
-  }
-#pragma unroll
-  for (int u = 0; u < kC * 32 / kPrepThreads; ++u) {
-    const int it = tid + u * kPrepThreads, t = it >> 5, cc = it & 31;
-    const bool valid = t < n;
-    const size_t off = valid ? (row0 + (size_t)t * p.H) * kDK + cc * 4 : 0;
-    cp_async16(smem + SL::SLW + t * 512 + cc * 16, p.log_w + off, valid);
-  }
-  cp_async_commit();
+  mbar_arrive_expect_tx(bar, (has_wg ? 5u : 4u) * kC * kDK * 2 + kC * kDK * 4);
+  tma_load_4d(smem + SL::SK, &m.k, 0, h, t0, b, bar);
+  tma_load_4d(smem + SL::SB, &m.b, 0, h, t0, b, bar);
+  tma_load_4d(smem + SL::SQ, &m.q, 0, h, t0, b, bar);
+  tma_load_4d(smem + SL::SV, &m.v, 0, h, t0, b, bar);
+  if (has_wg) tma_load_4d(smem + SL::SW, &m.wg, 0, h, t0, b, bar);
+  tma_load_4d(smem + SL::SLW, &m.lw, 0, h, t0, b, bar);
 }
 
-__global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(FwdParams p, uint8_t *records) {
+__global__ void __launch_bounds__(kPrepThreads, 1)
+    tc_prep_kernel(FwdParams p, uint8_t *records, const __grid_constant__ PrepMaps maps) {
   using SL = PrepSmem;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -172,8 +166,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(FwdParams p, u
   float *sDN = reinterpret_cast<float *>(smem + SL::DN);
   float *sA1 = reinterpret_cast<float *>(smem + SL::A1);
   uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + SL::MISC);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 8);
-  volatile int *sflag = reinterpret_cast<volatile int *>(smem + SL::MISC + 16);  // exact, abort
+  uint64_t *sbar = reinterpret_cast<uint64_t *>(smem + SL::MISC + 8);               // staging full
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 16);
+  volatile int *sflag = reinterpret_cast<volatile int *>(smem + SL::MISC + 24);  // exact, abort
   const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
   const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
@@ -183,21 +178,23 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(FwdParams p, u
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  int item = blockIdx.x;
   if (tid == 0) {
     mbar_init(mbar, 1);
+    mbar_init(sbar, 1);
     fence_mbar_init();
     sflag[1] = 0;
-  }
-  int item = blockIdx.x;
-  if (item < items) {
-    const int c = item % nch, bh = item / nch;
-    stage_chunk(smem, p, bh / H, bh % H, c * kC, min(kC, T - c * kC), tid);
+    if (item < items) {
+      const int c = item % nch, bh = item / nch;
+      stage_chunk(smem, maps, sbar, bh / H, bh % H, c * kC, has_wg);
+    }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
   uint32_t phase = 0;
+  uint32_t s_issued = item < items ? 1u : 0u, s_landed = 0;   // staging loads (uniform counts)
   bool ok = true;
 
   for (; item < items; item += gridDim.x) {
@@ -207,9 +204,14 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(FwdParams p, u
     auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
     GDR_PREP_PHASE(0);
 
-    cp_async_wait<0>();
-    if (tid == 0) sflag[0] = 0;
+    // this chunk's inputs have landed (load number s_landed completes that phase)
+    if (tid == 0) {
+      sflag[0] = 0;
+      if (!sflag[1] && !mbar_wait_bounded(sbar, s_landed & 1u, kWaitLimitNs)) sflag[1] = 1;
+    }
     __syncthreads();
+    if (!(ok = sflag[1] == 0)) break;
+    ++s_landed;
 
     // ---- cumulative log-decay: thread = (channel ch, token quarter qt), in place
     {
@@ -341,12 +343,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(FwdParams p, u
       }
       mma_commit_warp(mbar);
     }
-    // ---- the staging area is free: start the CTA's next chunk's copies
+    // ---- the staging area is free: load the CTA's next chunk
     {
       const int nx = item + gridDim.x;
       if (nx < items) {
-        const int cn = nx % nch, bhn = nx / nch;
-        stage_chunk(smem, p, bhn / H, bhn % H, cn * kC, min(kC, T - cn * kC), tid);
+        if (tid == 32) {
+          fence_proxy_async_smem();   // the CTA's reads of the staging area come first
+          const int cn = nx % nch, bhn = nx / nch;
+          stage_chunk(smem, maps, sbar, bhn / H, bhn % H, cn * kC, has_wg);
+        }
+        ++s_issued;
       }
     }
     GDR_PREP_PHASE(3);
@@ -469,11 +475,11 @@ __global__ void __launch_bounds__(kPrepThreads, 1) tc_prep_kernel(FwdParams p, u
   }
 
   GDR_PHASE_FINI(1)
-  cp_async_wait<0>();
   if (!ok && tid == 0) {
     if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
-    // the MMA group whose wait ran out may still be running: let it finish (bounded)
+    // an MMA group or a staging load may still be in flight: let them land (bounded)
     mbar_wait_bounded(mbar, phase ^ 1u, kWaitLimitNs);
+    if (s_issued > s_landed) mbar_wait_bounded(sbar, s_landed & 1u, kWaitLimitNs);
   }
   tc_fence_before();
   __syncthreads();
@@ -768,8 +774,48 @@ size_t forward_tc_split_workspace_bytes(const FwdParams &p) {
   return kHeaderBytes + (size_t)p.B * p.H * num_chunks(p.T) * Rec::BYTES;
 }
 
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [B][T][H][128] tensor of `elem` bytes as a 4-D map with a (128, 1, 64, 1) box.
+bool encode_input_map(CUtensorMap *m, const void *base, CUtensorMapDataType type, int elem,
+                      const FwdParams &p) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)kDK, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kDK * elem, (cuuint64_t)p.H * kDK * elem,
+                                 (cuuint64_t)p.T * p.H * kDK * elem};
+  const cuuint32_t box[4] = {(cuuint32_t)kDK, 1, (cuuint32_t)kC, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, type, 4, const_cast<void *>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStream_t stream) {
   constexpr int NV = 64;
+  PrepMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (!encode_input_map(&maps.k, p.k, bf, 2, p) || !encode_input_map(&maps.b, p.e1, bf, 2, p) ||
+      !encode_input_map(&maps.q, p.q, bf, 2, p) || !encode_input_map(&maps.v, p.v, bf, 2, p) ||
+      (p.e2 && !encode_input_map(&maps.wg, p.e2, bf, 2, p)) ||
+      !encode_input_map(&maps.lw, p.log_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p))
+    return cudaErrorInvalidValue;
   uint8_t *records = static_cast<uint8_t *>(workspace) + kHeaderBytes;
   cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)PrepSmem::ALLOC);
@@ -781,7 +827,7 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int items = p.B * p.H * num_chunks(p.T);
-  tc_prep_kernel<<<min(items, sms), kPrepThreads, PrepSmem::ALLOC, stream>>>(p, records);
+  tc_prep_kernel<<<min(items, sms), kPrepThreads, PrepSmem::ALLOC, stream>>>(p, records, maps);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 gc(p.dv / NV, p.H, p.B);
   tc_chain_kernel<NV><<<gc, kThreads, ChainSmem<NV>::ALLOC, stream>>>(p, records);

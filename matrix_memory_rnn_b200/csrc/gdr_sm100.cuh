@@ -75,6 +75,19 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
       : "memory");
 }
 
+// Tiled 4-D tensor load (TMA, no multicast) of one box of `map` at coordinates
+// (x, y, z, w) into shared memory; completes as transactions on `bar`.  Elements
+// outside the tensor are written as zeros.  x times the element size must be a
+// multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_4d(void *dst_smem, const void *map, int x, int y, int z,
+                                            int w, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst_smem)),
+      "l"(map), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async (16 bytes)
 // Copies 16 bytes global -> shared; when `valid` is false it writes 16 zero bytes
 // and reads nothing (src-size 0).
