@@ -10,8 +10,9 @@
 //    MMA), T^-1 (fp32 diagonal blocks, tf32 warp-MMA merges), U = T^-1 V^ and
 //    Y = T^-1 K^_pi (one tcgen05 MMA group), and the operand tiles Q_pi and K~.
 //    Chunks are independent: a persistent grid of one 512-thread CTA per SM walks
-//    them; each chunk's inputs arrive in shared memory as six TMA tensor tiles,
-//    issued while the previous chunk's MMAs, T^-1 and readouts run.  Each chunk's result is a
+//    them as a two-stage pipeline of warp groups (element-wise phase + MMA1 on
+//    one chunk while T^-1 + MMA2 run on the previous one); inputs arrive by TMA,
+//    the bf16 ones straight into the MMA tiles.  Each chunk's result is a
 //    record of bf16 MMA tiles, already in the 128-byte-swizzled shared-memory
 //    layout, in the workspace.
 //  * chain: the inter-chunk state carry and the outputs, sequential over chunks
@@ -84,11 +85,21 @@ __host__ __device__ inline int num_chunks(int T) { return (T + kC - 1) / kC; }
 
 // ============================================================== prep kernel
 // Persistent: one CTA of 512 threads per SM walks the chunks (b, h, c) with a
-// stride of gridDim.x.  A chunk's inputs are staged in shared memory by cp.async;
-// the copies for the CTA's next chunk are issued as soon as this chunk's
-// element-wise phase has consumed the staging area, so they land while the MMAs,
-// T^-1 and the readouts of this chunk run.
+// stride of gridDim.x, as a two-stage pipeline of warp groups over two chunk
+// buffers:
+//   front (warps 8..15): log-decay scan, operand tiles, MMA1, L / M readout of
+//                        chunk j;
+//   back  (warps 0..7):  T^-1, MMA2, U / Y readout of chunk j - 1.
+// Inputs arrive by TMA: k, b, q, v straight into the chunk buffer's MMA tiles
+// (128-byte swizzle, the tcgen05 operand layout), where the element-wise phase
+// turns them into K g, K^ f, Q f, V^ in place; wg and log w into a staging area.
+// The back group issues chunk j + 2's tile loads as soon as MMA2 of chunk j has
+// released its buffer; the front group loads the next staging area as soon as it
+// has read the current one.
 constexpr int kPrepThreads = 512;
+constexpr int kGroup = 256;                    // threads per warp group
+using FrontSync = GroupSync<1, kGroup>;
+using BackSync = GroupSync<2, kGroup>;
 
 // fp32 64 x 64 T^-1 in the Q rows of the [K^ f; Q f] tile once MMA1 has read them:
 // those rows are two 8 KB pieces (one per 64-column atom), rows 0..31 in the
@@ -100,48 +111,96 @@ struct QRowsIdx {
 };
 
 struct PrepSmem {
-  // staging: row-major token rows (bf16 256 B, fp32 512 B), zero past the sequence end
-  static constexpr uint32_t SK = 0;
-  static constexpr uint32_t SB = SK + kC * kDK * 2;
-  static constexpr uint32_t SQ = SB + kC * kDK * 2;
-  static constexpr uint32_t SV = SQ + kC * kDK * 2;
-  static constexpr uint32_t SW = SV + kC * kDK * 2;
+  // chunk buffer (x2): tiles in the sw128 layout, 64-column blocks
+  static constexpr uint32_t A_LM = 0;                         // [K^ f; Q f] 2C x DK (b, q land here);
+                                                              //   Q rows then hold fp32 T^-1
+  static constexpr uint32_t B_LM = A_LM + 2 * kC * kDK * 2;   // K g  C x DK (k lands here); then
+                                                              //   fp32 L; then bf16 T^-1 (first 8 KB)
+  static constexpr uint32_t VH = B_LM + kC * kDK * 2;         // V^ = wg (.) v (v lands here)
+  static constexpr uint32_t BUF = VH + kC * kDK * 2;          // 64 KB per buffer
+  // staging (single): write gate (sw128, same offsets as v), log w (row-major fp32)
+  static constexpr uint32_t SW = 2 * BUF;
   static constexpr uint32_t SLW = SW + kC * kDK * 2;          // log w, then Lam_t - Lam_1
-  static constexpr uint32_t A_LM = SLW + kC * kDK * 4;        // [K^ f; Q f] 2C x DK bf16; Q rows
-                                                              //   then hold fp32 T^-1 (QRowsIdx)
-  static constexpr uint32_t B_LM = A_LM + 2 * kC * kDK * 2;   // K g  C x DK bf16; then fp32 L;
-                                                              //   then bf16 T^-1 (first 8 KB)
-  static constexpr uint32_t VH = B_LM + kC * kDK * 2;         // V^ = wg (.) v  C x DV bf16
-  static constexpr uint32_t QT = VH + kC * kDK * 2;           // fp32 [4][DK] quarter sums of log w
-  static constexpr uint32_t L1 = QT + 4 * kDK * 4;            // fp32 Lam_1 per channel
+  static constexpr uint32_t QT = SLW + kC * kDK * 4;          // fp32 [2][DK] half sums of log w
+  static constexpr uint32_t L1 = QT + 2 * kDK * 4;            // fp32 Lam_1 per channel
   static constexpr uint32_t DN = L1 + kDK * 4;                // fp32 Lam_n - Lam_1 per channel
-  static constexpr uint32_t A1 = DN + kDK * 4;                // fp32 alpha_1 = exp(Lam_1)
-  static constexpr uint32_t MISC = A1 + kDK * 4;              // mbarrier, TMEM slot, flags
-  static constexpr uint32_t ALLOC = MISC + 64 + 1024;
-  static_assert(A_LM % 1024 == 0 && B_LM % 1024 == 0 && VH % 1024 == 0, "MMA tiles 1024-aligned");
+  static constexpr uint32_t A1 = DN + kDK * 4;                // fp32 [4][DK] alpha_1, by chunk & 3
+  static constexpr uint32_t MISC = A1 + 4 * kDK * 4;
+  static constexpr uint32_t ALLOC = MISC + 256 + 1024;
+  static_assert(BUF % 1024 == 0 && SW % 1024 == 0, "MMA tiles 1024-aligned");
   static_assert(Ix::kBytes <= kC * kDK * 2, "fp32 L must fit the reused bf16 tile");
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
-// Tensor maps of the prep inputs, each 4-D (channel, head, token, batch) with a box
-// of one chunk of one head: 128 channels x 64 tokens, i.e. 16 KB of bf16 or 32 KB
-// of fp32 in row-major token rows -- the staging layout.  Tokens past T read as 0.
+struct PrepMisc {             // byte offsets inside PrepSmem::MISC
+  static constexpr uint32_t BFULL = 0;      // uint64_t [2] chunk-buffer tiles landed
+  static constexpr uint32_t AFULL = 16;     // uint64_t     staging landed
+  static constexpr uint32_t READY = 24;     // uint64_t [2] front -> back: buffer holds L, V^, K^ f
+  static constexpr uint32_t BAR1 = 40;      // uint64_t     MMA1 done (front)
+  static constexpr uint32_t BAR2 = 48;      // uint64_t     MMA2 done (back)
+  static constexpr uint32_t SLOT = 56;      // uint32_t     TMEM base
+  static constexpr uint32_t ABORT = 60;     // int          a bounded wait ran out
+  static constexpr uint32_t EXACT = 64;     // int          front: this chunk takes the exact path
+  static constexpr uint32_t CNT = 128;      // uint32_t [8] issued / completed counts (drain)
+};
+enum { kBIss0, kBIss1, kBDone0, kBDone1, kAIss, kADone, kM2Iss, kM1Iss };
+
+// Tensor maps of the prep inputs, each 4-D (channel, head, token, batch).  k, b, q,
+// v, wg: bf16 boxes of 64 channels x 64 tokens with the 128-byte swizzle (one
+// 64-column block of an MMA tile); log w: fp32 box of 128 channels x 64 tokens,
+// row-major.  Tokens past T read as 0.
 struct PrepMaps {
   CUtensorMap k, b, q, v, wg, lw;
 };
 
-// One thread: TMA loads of one chunk's k, b, q, v, (wg,) log w into the staging
-// area, completing on `bar`.
-__device__ __forceinline__ void stage_chunk(uint8_t *smem, const PrepMaps &m, uint64_t *bar, int b,
-                                            int h, int t0, bool has_wg) {
+// One thread: the chunk buffer's tile loads (k, b, q, v) for chunk (b, h, t0).
+__device__ __forceinline__ void load_tiles(uint8_t *buf, const PrepMaps &m, uint64_t *bar, int b,
+                                           int h, int t0) {
   using SL = PrepSmem;
-  mbar_arrive_expect_tx(bar, (has_wg ? 5u : 4u) * kC * kDK * 2 + kC * kDK * 4);
-  tma_load_4d(smem + SL::SK, &m.k, 0, h, t0, b, bar);
-  tma_load_4d(smem + SL::SB, &m.b, 0, h, t0, b, bar);
-  tma_load_4d(smem + SL::SQ, &m.q, 0, h, t0, b, bar);
-  tma_load_4d(smem + SL::SV, &m.v, 0, h, t0, b, bar);
-  if (has_wg) tma_load_4d(smem + SL::SW, &m.wg, 0, h, t0, b, bar);
+  mbar_arrive_expect_tx(bar, 4u * kC * kDK * 2);
+#pragma unroll
+  for (int blk = 0; blk < 2; ++blk) {
+    tma_load_4d(buf + SL::B_LM + blk * (kC * 128), &m.k, 64 * blk, h, t0, b, bar);
+    tma_load_4d(buf + SL::A_LM + blk * (2 * kC * 128), &m.b, 64 * blk, h, t0, b, bar);
+    tma_load_4d(buf + SL::A_LM + blk * (2 * kC * 128) + kC * 128, &m.q, 64 * blk, h, t0, b, bar);
+    tma_load_4d(buf + SL::VH + blk * (kC * 128), &m.v, 64 * blk, h, t0, b, bar);
+  }
+}
+
+// One thread: the staging loads (wg if present, log w) for chunk (b, h, t0).
+__device__ __forceinline__ void load_staging(uint8_t *smem, const PrepMaps &m, uint64_t *bar, int b,
+                                             int h, int t0, bool has_wg) {
+  using SL = PrepSmem;
+  mbar_arrive_expect_tx(bar, (has_wg ? kC * kDK * 2u : 0u) + kC * kDK * 4u);
+  if (has_wg) {
+    tma_load_4d(smem + SL::SW, &m.wg, 0, h, t0, b, bar);
+    tma_load_4d(smem + SL::SW + kC * 128, &m.wg, 64, h, t0, b, bar);
+  }
   tma_load_4d(smem + SL::SLW, &m.lw, 0, h, t0, b, bar);
+}
+
+// One thread of a group polls `bar` for `parity` (bounded; gives up at once when the
+// CTA is aborting), then the group meets at a barrier that ORs every thread's view
+// of the abort flag, so the whole group takes the same branch even while the other
+// group sets the flag.  Returns false (for the whole group) when the CTA aborts.
+template <class Sync>
+__device__ __forceinline__ bool group_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                           bool poller) {
+  bool failed = *abort != 0;
+  if (poller && !failed) {
+    bool done = mbar_try_wait(bar, parity);
+    if (!done) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!(done = mbar_try_wait(bar, parity)) && *abort == 0) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+      }
+    }
+    if (!done) {
+      *abort = 1;
+      failed = true;
+    }
+  }
+  return !Sync::sync_or(failed);
 }
 
 __global__ void __launch_bounds__(kPrepThreads, 1)
@@ -153,339 +212,388 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   const uint32_t sb = smem_u32(smem);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int qd = warp & 3, cpart = warp >> 2;             // TMEM lane quarter, column part
+  const bool front = tid >= kGroup;
+  const int gt = tid & (kGroup - 1);                      // index within the group
+  const int qd = warp & 3, cpart = (warp >> 2) & 1;       // TMEM lane quarter, column half
   const int T = p.T, H = p.H, nch = num_chunks(T);
   const int items = p.B * H * nch;
+  const int nloc = items > (int)blockIdx.x ? (items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   GDR_PHASE_INIT
 
+  uint8_t *misc = smem + SL::MISC;
+  uint64_t *bfull = reinterpret_cast<uint64_t *>(misc + PrepMisc::BFULL);
+  uint64_t *afull = reinterpret_cast<uint64_t *>(misc + PrepMisc::AFULL);
+  uint64_t *ready = reinterpret_cast<uint64_t *>(misc + PrepMisc::READY);
+  uint64_t *bar1 = reinterpret_cast<uint64_t *>(misc + PrepMisc::BAR1);
+  uint64_t *bar2 = reinterpret_cast<uint64_t *>(misc + PrepMisc::BAR2);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + PrepMisc::SLOT);
+  volatile int *sabort = reinterpret_cast<volatile int *>(misc + PrepMisc::ABORT);
+  volatile int *sexact = reinterpret_cast<volatile int *>(misc + PrepMisc::EXACT);
+  uint32_t *cnt = reinterpret_cast<uint32_t *>(misc + PrepMisc::CNT);
   float *sLW = reinterpret_cast<float *>(smem + SL::SLW);
-  float *sL = reinterpret_cast<float *>(smem + SL::B_LM);
-  float *sTi = reinterpret_cast<float *>(smem + SL::A_LM);
   float *sQT = reinterpret_cast<float *>(smem + SL::QT);
   float *sL1 = reinterpret_cast<float *>(smem + SL::L1);
   float *sDN = reinterpret_cast<float *>(smem + SL::DN);
   float *sA1 = reinterpret_cast<float *>(smem + SL::A1);
-  uint64_t *mbar = reinterpret_cast<uint64_t *>(smem + SL::MISC);
-  uint64_t *sbar = reinterpret_cast<uint64_t *>(smem + SL::MISC + 8);               // staging full
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + SL::MISC + 16);
-  volatile int *sflag = reinterpret_cast<volatile int *>(smem + SL::MISC + 24);  // exact, abort
   const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
   const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
   const bool has_wg = p.e2 != nullptr;
+  auto item_of = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
 
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, 2 * kTmemCols);
     tmem_relinquish();
   }
-  int item = blockIdx.x;
   if (tid == 0) {
-    mbar_init(mbar, 1);
-    mbar_init(sbar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bfull + i, 1);
+      mbar_init(ready + i, 1);
+    }
+    mbar_init(afull, 1);
+    mbar_init(bar1, 1);
+    mbar_init(bar2, 1);
     fence_mbar_init();
-    sflag[1] = 0;
-    if (item < items) {
-      const int c = item % nch, bh = item / nch;
-      stage_chunk(smem, maps, sbar, bh / H, bh % H, c * kC, has_wg);
+    *sabort = 0;
+    for (int i = 0; i < 8; ++i) cnt[i] = 0;
+    for (int j = 0; j < 2 && j < nloc; ++j) {
+      const int it = item_of(j), c = it % nch, bh = it / nch;
+      load_tiles(smem + j * SL::BUF, maps, bfull + j, bh / H, bh % H, c * kC);
+      ++cnt[kBIss0 + j];
+    }
+    if (nloc > 0) {
+      const int it = item_of(0), c = it % nch, bh = it / nch;
+      load_staging(smem, maps, afull, bh / H, bh % H, c * kC, has_wg);
+      ++cnt[kAIss];
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
-  uint32_t phase = 0;
-  uint32_t s_issued = item < items ? 1u : 0u, s_landed = 0;   // staging loads (uniform counts)
-  bool ok = true;
+  const uint32_t tD1 = tmem + 2 * kDK;                    // front: L | M accumulator (64 columns)
 
-  for (; item < items; item += gridDim.x) {
-    const int c = item % nch, bh = item / nch, h = bh % H, b = bh / H;
-    const int t0 = c * kC, n = min(kC, T - t0);
-    uint8_t *rec = records + (size_t)item * Rec::BYTES;   // item order = (b, h, c) record order
-    auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
-    GDR_PREP_PHASE(0);
+  if (front) {
+    // =========================================================== front group
+    const bool poller = gt == 0;
+    for (int j = 0; j < nloc; ++j) {
+      const int item = item_of(j), c = item % nch, bh = item / nch, h = bh % H, b = bh / H;
+      const int t0 = c * kC, n = min(kC, T - t0), bi = j & 1;
+      uint8_t *buf = smem + bi * SL::BUF;
+      float *sL = reinterpret_cast<float *>(buf + SL::B_LM);
+      uint8_t *rec = records + (size_t)item * Rec::BYTES;
+      float *a1s = sA1 + (j & 3) * kDK;
+      auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
+      GDR_PREP_PHASE(0);
 
-    // this chunk's inputs have landed (load number s_landed completes that phase)
-    if (tid == 0) {
-      sflag[0] = 0;
-      if (!sflag[1] && !mbar_wait_bounded(sbar, s_landed & 1u, kWaitLimitNs)) sflag[1] = 1;
-    }
-    __syncthreads();
-    if (!(ok = sflag[1] == 0)) break;
-    ++s_landed;
-
-    // ---- cumulative log-decay: thread = (channel ch, token quarter qt), in place
-    {
-      const int ch = tid & (kDK - 1), qt = tid >> 7;
-      float x[16];
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        acc += sLW[(16 * qt + i) * kDK + ch];
-        x[i] = acc;
+      // chunk j's staging and tiles have landed
+      if (poller) *sexact = 0;
+      if (!group_wait<FrontSync>(afull, j & 1, sabort, poller)) break;
+      if (!group_wait<FrontSync>(bfull + bi, (j >> 1) & 1, sabort, poller)) break;
+      if (poller) {
+        cnt[kADone] = j + 1;
+        cnt[kBDone0 + bi] += 1;
       }
-      sQT[qt * kDK + ch] = acc;
-      if (qt == 0) sL1[ch] = x[0];
-      __syncthreads();
-      float excl = 0.f, all = 0.f;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float v = sQT[q * kDK + ch];
-        all += v;
-        excl += (q < qt) ? v : 0.f;
-      }
-      const float l1 = sL1[ch], shift = excl - l1;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) sLW[(16 * qt + i) * kDK + ch] = x[i] + shift;
-      if (qt == 0) {
-        const float dn = all - l1;
-        sDN[ch] = dn;
-        sA1[ch] = __expf(l1);
-        reinterpret_cast<float *>(rec + Rec::PI)[ch] = __expf(all);
-        if (dn < -kMaxChunkDecay) sflag[0] = 1;
-      }
-    }
-    __syncthreads();
-    const bool exact = sflag[0] != 0;
-    GDR_PREP_PHASE(1);
+      GDR_PREP_PHASE(1);
 
-    // ---- operand tiles: [K^ f; Q f], K g in shared memory; Q_pi, K~ to the record.
-    //      Thread = (channel group g of 8, token pair tb); the exact path also parks
-    //      Lam_t - Lam_1 in the record.
-    {
-      const int g = tid & 15, tb = tid >> 4, j0 = 8 * g;
-      float dn[8], a1[8], ed[8];
+      // ---- cumulative log-decay: thread = (channel ch, token half), in place
       {
-        const float4 d0 = *reinterpret_cast<const float4 *>(sDN + j0);
-        const float4 d1 = *reinterpret_cast<const float4 *>(sDN + j0 + 4);
-        const float4 a0 = *reinterpret_cast<const float4 *>(sA1 + j0);
-        const float4 a4 = *reinterpret_cast<const float4 *>(sA1 + j0 + 4);
-        dn[0] = d0.x; dn[1] = d0.y; dn[2] = d0.z; dn[3] = d0.w;
-        dn[4] = d1.x; dn[5] = d1.y; dn[6] = d1.z; dn[7] = d1.w;
-        a1[0] = a0.x; a1[1] = a0.y; a1[2] = a0.z; a1[3] = a0.w;
-        a1[4] = a4.x; a1[5] = a4.y; a1[6] = a4.z; a1[7] = a4.w;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ed[e] = __expf(dn[e]);
-      }
-      auto operands = [&](auto exact_path) {
-        constexpr bool kExact = decltype(exact_path)::value;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int t = 2 * tb + i;
-          const float4 l0 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0);
-          const float4 l4 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0 + 4);
-          const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l4.x, l4.y, l4.z, l4.w};
-          float k8[8], b8[8], q8[8];
-          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SK + t * 256 + g * 16), k8);
-          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SB + t * 256 + g * 16), b8);
-          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SQ + t * 256 + g * 16), q8);
-          float av[8], aq[8], bl[8], kt[8], qp[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float f = __expf(lam[e]);
-            av[e] = b8[e] * k8[e] * f;
-            aq[e] = q8[e] * f;
-            qp[e] = aq[e] * a1[e];
-            if (!kExact) {
-              bl[e] = k8[e] * __expf(-lam[e]);
-              kt[e] = bl[e] * ed[e];
-            } else if (dn[e] >= -kMaxChunkDecay) {
-              kt[e] = k8[e] * __expf(-lam[e]) * ed[e];
-              bl[e] = 0.f;     // the exact path forms L and M without K g
-            } else {
-              kt[e] = k8[e] * __expf(dn[e] - lam[e]);
-              bl[e] = 0.f;
-            }
-          }
-          const uint32_t o64 = sw128_offset(t, j0, kC * 128);
-          st_smem16(smem, SL::A_LM + sw128_offset(t, j0, 2 * kC * 128), pack8(av));
-          st_smem16(smem, SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128), pack8(aq));
-          st_smem16(smem, SL::B_LM + o64, pack8(bl));
-          *reinterpret_cast<uint4 *>(rec + Rec::QY + sw128_offset(t, j0, Rec::QY_STRIDE)) = pack8(qp);
-          *reinterpret_cast<uint4 *>(rec + Rec::KT + o64) = pack8(kt);
-          if (kExact) {
-            float4 *dst = reinterpret_cast<float4 *>(rec + park_row(t)) + g * 2;
-            dst[0] = l0;
-            dst[1] = l4;
-          }
-        }
-      };
-      if (!exact) operands(std::false_type{});
-      else operands(std::true_type{});
-    }
-    // ---- V^ = wg (.) v into its swizzled tile
-#pragma unroll
-    for (int u = 0; u < kC * 16 / kPrepThreads; ++u) {
-      const int it = tid + u * kPrepThreads, t = it >> 4, gg = it & 15;
-      uint4 vv = *reinterpret_cast<const uint4 *>(smem + SL::SV + t * 256 + gg * 16);
-      if (has_wg) {
-        float v8[8], w8[8];
-        unpack8(vv, v8);
-        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SW + t * 256 + gg * 16), w8);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
-        vv = pack8(v8);
-      }
-      st_smem16(smem, SL::VH + sw128_offset(t, 8 * gg, kC * 128), vv);
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    GDR_PREP_PHASE(2);
-
-    // ---- MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
-    if (warp == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_bf16_f32(128, kC, false, false);
-#pragma unroll
-      for (int s = 0; s < kDK / 16; ++s) {
-        const uint64_t ad = sdesc_sw128(sb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
-        mma_bf16_warp(tmem, ad, bd, id, s > 0);
-      }
-      mma_commit_warp(mbar);
-    }
-    // ---- the staging area is free: load the CTA's next chunk
-    {
-      const int nx = item + gridDim.x;
-      if (nx < items) {
-        if (tid == 32) {
-          fence_proxy_async_smem();   // the CTA's reads of the staging area come first
-          const int cn = nx % nch, bhn = nx / nch;
-          stage_chunk(smem, maps, sbar, bhn / H, bhn % H, cn * kC, has_wg);
-        }
-        ++s_issued;
-      }
-    }
-    GDR_PREP_PHASE(3);
-    if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
-    GDR_PREP_PHASE(4);
-
-    // ---- L (fp32, strictly lower; into the dead K g tile) and M (bf16 -> record)
-    if (!exact) {
-      float x[16];
-      tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * qd) << 16) + 16 * cpart, x);
-      tmem_ld_wait();
-      const int r = 32 * qd + lane, col = 16 * cpart;
-      if (r < kC) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = (col + i < r) ? x[i] : 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; i += 4)
-          *reinterpret_cast<float4 *>(sL + Ix::at(r, col + i)) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
-      } else {
-        const int t = r - kC;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) x[i] = (col + i <= t) ? x[i] : 0.f;
-#pragma unroll
-        for (int i = 0; i < 16; i += 8)
-          *reinterpret_cast<uint4 *>(rec + Rec::MM + sw128_offset(t, col + i, kC * 128)) = pack8(x + i);
-      }
-    } else {
-      // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound)
-      for (int it = tid; it < kC * kC; it += kPrepThreads) {
-        const int t = it / kC, s = it % kC;
-        float l = 0.f, m = 0.f;
-        if (s <= t && t < n) {
-          const float *lt = reinterpret_cast<const float *>(rec + park_row(t));
-          const float *ls = reinterpret_cast<const float *>(rec + park_row(s));
-          const size_t ot = tok_off(t), os = tok_off(s);
-          for (int j = 0; j < kDK; ++j) {
-            const float d = __expf(__ldcg(lt + j) - __ldcg(ls + j));
-            const float ks = __bfloat162float(gk[os + j]);
-            m += __bfloat162float(gq[ot + j]) * d * ks;
-            l += __bfloat162float(gb[ot + j]) * __bfloat162float(gk[ot + j]) * d * ks;
-          }
-        }
-        sL[Ix::at(t, s)] = (s < t) ? l : 0.f;
-        *reinterpret_cast<__nv_bfloat16 *>(rec + Rec::MM + sw128_offset(t, s, kC * 128)) =
-            __float2bfloat16_rn(m);
-      }
-    }
-    tc_fence_before();
-    __syncthreads();
-    GDR_PREP_PHASE(5);
-
-    // ---- T^-1 (fp32, into the dead Q rows of A_LM), bf16 copy (into the dead L tile)
-    invert_diag_blocks<Ix, QRowsIdx, kPrepThreads>(sL, sTi, tid);
-    GDR_PREP_PHASE(9);
-    invert_merge_levels<Ix, QRowsIdx, kPrepThreads>(sL, sTi, tid);
-    {
-      const int t = tid >> 3, gg = tid & 7;
-      const float4 y0 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg));
-      const float4 y1 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg + 4));
-      float x[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int s = 8 * gg + e;
-        x[e] = (s < t) ? x[e] : (s == t ? 1.f : 0.f);
-      }
-      st_smem16(smem, SL::B_LM + sw128_offset(t, 8 * gg, kC * 128), pack8(x));
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    GDR_PREP_PHASE(6);
-
-    // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
-    if (warp == 0) {
-      tc_fence_after();
-      constexpr uint32_t id = idesc_bf16_f32(64, kDK, false, true);
-#pragma unroll
-      for (int s = 0; s < kC / 16; ++s) {
-        const uint64_t ad = sdesc_sw128(sb + SL::B_LM + s * 32, 16, 1024);
-        const uint64_t bu = sdesc_sw128(sb + SL::VH + s * 2048, kC * 128, 1024);
-        const uint64_t by = sdesc_sw128(sb + SL::A_LM + s * 2048, 2 * kC * 128, 1024);
-        mma_bf16_warp(tmem, ad, bu, id, s > 0);
-        mma_bf16_warp(tmem + kDK, ad, by, id, s > 0);
-      }
-      mma_commit_warp(mbar);
-    }
-    if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
-    GDR_PREP_PHASE(7);
-
-    // ---- U and Y (x alpha_1) -> bf16 record tiles; M = 64 accumulators: row 16 qd + lane.
-    //      Column part cpart: 0, 1 -> U columns, 2, 3 -> Y columns (64 each).
-    {
-      const bool is_y = cpart >= 2;
-      const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int col = 64 * (cpart & 1) + 32 * half;    // 0..127 within U or Y
+        const int ch = gt & (kDK - 1), hv = gt >> 7;
         float x[32];
-        tmem_ld_32x32b_x32(tmem + lane_q + (is_y ? kDK : 0) + col, x);
-        tmem_ld_wait();
-        if (lane < 16) {
-          const int t = 16 * qd + lane;
-          if (is_y) {
+        float acc = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 a = *reinterpret_cast<const float4 *>(sA1 + col + i);
-              x[i] *= a.x; x[i + 1] *= a.y; x[i + 2] *= a.z; x[i + 3] *= a.w;
+        for (int i = 0; i < 32; ++i) {
+          acc += sLW[(32 * hv + i) * kDK + ch];
+          x[i] = acc;
+        }
+        sQT[hv * kDK + ch] = acc;
+        if (hv == 0) sL1[ch] = x[0];
+        FrontSync::sync();
+        const float q0 = sQT[ch], all = q0 + sQT[kDK + ch];
+        const float l1 = sL1[ch], shift = (hv ? q0 : 0.f) - l1;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sLW[(32 * hv + i) * kDK + ch] = x[i] + shift;
+        if (hv == 0) {
+          const float dn = all - l1;
+          sDN[ch] = dn;
+          a1s[ch] = __expf(l1);
+          reinterpret_cast<float *>(rec + Rec::PI)[ch] = __expf(all);
+          if (dn < -kMaxChunkDecay) *sexact = 1;
+        }
+      }
+      FrontSync::sync();
+      const bool exact = *sexact != 0;
+      GDR_PREP_PHASE(2);
+
+      // ---- operand tiles, in place: k -> K g, b -> K^ f, q -> Q f; Q_pi, K~ to the
+      //      record.  Thread = (channel group g of 8, token block tb of 4).
+      {
+        const int g = gt & 15, tb = gt >> 4, j0 = 8 * g;
+        float dn[8], a1[8], ed[8];
+        {
+          const float4 d0 = *reinterpret_cast<const float4 *>(sDN + j0);
+          const float4 d1 = *reinterpret_cast<const float4 *>(sDN + j0 + 4);
+          const float4 a0 = *reinterpret_cast<const float4 *>(a1s + j0);
+          const float4 a4 = *reinterpret_cast<const float4 *>(a1s + j0 + 4);
+          dn[0] = d0.x; dn[1] = d0.y; dn[2] = d0.z; dn[3] = d0.w;
+          dn[4] = d1.x; dn[5] = d1.y; dn[6] = d1.z; dn[7] = d1.w;
+          a1[0] = a0.x; a1[1] = a0.y; a1[2] = a0.z; a1[3] = a0.w;
+          a1[4] = a4.x; a1[5] = a4.y; a1[6] = a4.z; a1[7] = a4.w;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ed[e] = __expf(dn[e]);
+        }
+        auto operands = [&](auto exact_path) {
+          constexpr bool kExact = decltype(exact_path)::value;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int t = 4 * tb + i;
+            const float4 l0 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0);
+            const float4 l4 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0 + 4);
+            const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l4.x, l4.y, l4.z, l4.w};
+            const uint32_t ok_ = sw128_offset(t, j0, kC * 128);
+            const uint32_t ob = SL::A_LM + sw128_offset(t, j0, 2 * kC * 128);
+            const uint32_t oq = SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128);
+            float k8[8], b8[8], q8[8];
+            unpack8(*reinterpret_cast<const uint4 *>(buf + SL::B_LM + ok_), k8);
+            unpack8(*reinterpret_cast<const uint4 *>(buf + ob), b8);
+            unpack8(*reinterpret_cast<const uint4 *>(buf + oq), q8);
+            float av[8], aq[8], bl[8], kt[8], qp[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float f = __expf(lam[e]);
+              av[e] = b8[e] * k8[e] * f;
+              aq[e] = q8[e] * f;
+              qp[e] = aq[e] * a1[e];
+              if (!kExact) {
+                bl[e] = k8[e] * __expf(-lam[e]);
+                kt[e] = bl[e] * ed[e];
+              } else if (dn[e] >= -kMaxChunkDecay) {
+                kt[e] = k8[e] * __expf(-lam[e]) * ed[e];
+                bl[e] = 0.f;     // the exact path forms L and M without K g
+              } else {
+                kt[e] = k8[e] * __expf(dn[e] - lam[e]);
+                bl[e] = 0.f;
+              }
+            }
+            st_smem16(buf, ob, pack8(av));
+            st_smem16(buf, oq, pack8(aq));
+            st_smem16(buf, SL::B_LM + ok_, pack8(bl));
+            *reinterpret_cast<uint4 *>(rec + Rec::QY + sw128_offset(t, j0, Rec::QY_STRIDE)) = pack8(qp);
+            *reinterpret_cast<uint4 *>(rec + Rec::KT + ok_) = pack8(kt);
+            if (kExact) {
+              float4 *dst = reinterpret_cast<float4 *>(rec + park_row(t)) + g * 2;
+              dst[0] = l0;
+              dst[1] = l4;
             }
           }
+        };
+        if (!exact) operands(std::false_type{});
+        else operands(std::true_type{});
+      }
+      // ---- V^ = wg (.) v in place (wg staged at the same swizzled offsets)
+      if (has_wg) {
+#pragma unroll
+        for (int u = 0; u < kC * 16 / kGroup; ++u) {
+          const uint32_t off = (uint32_t)(gt + u * kGroup) * 16;
+          float v8[8], w8[8];
+          unpack8(*reinterpret_cast<const uint4 *>(buf + SL::VH + off), v8);
+          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SW + off), w8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+          st_smem16(buf, SL::VH + off, pack8(v8));
+        }
+      }
+      fence_proxy_async_smem();
+      FrontSync::sync();
+      GDR_PREP_PHASE(3);
+
+      // ---- the staging area is read: load the next chunk's; MMA1 on this chunk
+      if (gt == 32 && j + 1 < nloc) {
+        fence_proxy_async_smem();
+        const int it = item_of(j + 1), cn = it % nch, bhn = it / nch;
+        load_staging(smem, maps, afull, bhn / H, bhn % H, cn * kC, has_wg);
+        cnt[kAIss] = j + 2;
+      }
+      if (warp == 8) {
+        // MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
+        tc_fence_after();
+        const uint32_t bb = sb + bi * SL::BUF;
+        constexpr uint32_t id = idesc_bf16_f32(128, kC, false, false);
+#pragma unroll
+        for (int s = 0; s < kDK / 16; ++s) {
+          const uint64_t ad = sdesc_sw128(bb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(bb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
+          mma_bf16_warp(tD1, ad, bd, id, s > 0);
+        }
+        mma_commit_warp(bar1);
+        if (lane == 0) cnt[kM1Iss] = j + 1;
+      }
+      if (!group_wait<FrontSync>(bar1, j & 1, sabort, poller)) break;
+      tc_fence_after();
+      GDR_PREP_PHASE(4);
+
+      // ---- L (fp32, strictly lower; over the dead K g tile) and M (bf16 -> record)
+      if (!exact) {
+        float x[32];
+        tmem_ld_32x32b_x32(tD1 + ((uint32_t)(32 * qd) << 16) + 32 * cpart, x);
+        tmem_ld_wait();
+        const int r = 32 * qd + lane, col = 32 * cpart;
+        if (r < kC) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = (col + i < r) ? x[i] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4 *>(sL + Ix::at(r, col + i)) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+        } else {
+          const int t = r - kC;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) x[i] = (col + i <= t) ? x[i] : 0.f;
 #pragma unroll
           for (int i = 0; i < 32; i += 8)
-            *reinterpret_cast<uint4 *>(
-                rec + (is_y ? Rec::QY + sw128_offset(kC + t, col + i, Rec::QY_STRIDE)
-                            : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
+            *reinterpret_cast<uint4 *>(rec + Rec::MM + sw128_offset(t, col + i, kC * 128)) = pack8(x + i);
+        }
+      } else {
+        // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound)
+        for (int it = gt; it < kC * kC; it += kGroup) {
+          const int t = it / kC, s = it % kC;
+          float l = 0.f, m = 0.f;
+          if (s <= t && t < n) {
+            const float *lt = reinterpret_cast<const float *>(rec + park_row(t));
+            const float *ls = reinterpret_cast<const float *>(rec + park_row(s));
+            const size_t ot = tok_off(t), os = tok_off(s);
+            for (int jj = 0; jj < kDK; ++jj) {
+              const float d = __expf(__ldcg(lt + jj) - __ldcg(ls + jj));
+              const float ks = __bfloat162float(gk[os + jj]);
+              m += __bfloat162float(gq[ot + jj]) * d * ks;
+              l += __bfloat162float(gb[ot + jj]) * __bfloat162float(gk[ot + jj]) * d * ks;
+            }
+          }
+          sL[Ix::at(t, s)] = (s < t) ? l : 0.f;
+          *reinterpret_cast<__nv_bfloat16 *>(rec + Rec::MM + sw128_offset(t, s, kC * 128)) =
+              __float2bfloat16_rn(m);
         }
       }
+      tc_fence_before();
+      FrontSync::sync();
+      if (poller) mbar_arrive(ready + bi);                 // hand the buffer to the back group
+      GDR_PREP_PHASE(5);
     }
-    tc_fence_before();
-    GDR_PREP_PHASE(8);
+  } else {
+    // =========================================================== back group
+    const bool poller = gt == 0;
+    for (int j = 0; j < nloc; ++j) {
+      const int item = item_of(j), bi = j & 1;
+      uint8_t *buf = smem + bi * SL::BUF;
+      float *sL = reinterpret_cast<float *>(buf + SL::B_LM);
+      float *sTi = reinterpret_cast<float *>(buf + SL::A_LM);
+      uint8_t *rec = records + (size_t)item * Rec::BYTES;
+      const float *a1s = sA1 + (j & 3) * kDK;
+      GDR_PREP_PHASE(8);
+      if (!group_wait<BackSync>(ready + bi, (j >> 1) & 1, sabort, poller)) break;
+      tc_fence_after();
+      GDR_PREP_PHASE(9);
+
+      // ---- T^-1 (fp32, into the dead Q rows of A_LM), bf16 copy (into the dead L tile)
+      invert_diag_blocks<Ix, QRowsIdx, kGroup, BackSync>(sL, sTi, gt);
+      invert_merge_levels<Ix, QRowsIdx, kGroup, BackSync>(sL, sTi, gt);
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int it = gt + u * kGroup, t = it >> 3, gg = it & 7;
+        const float4 y0 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg));
+        const float4 y1 = *reinterpret_cast<const float4 *>(sTi + QRowsIdx::at(t, 8 * gg + 4));
+        float x[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int s = 8 * gg + e;
+          x[e] = (s < t) ? x[e] : (s == t ? 1.f : 0.f);
+        }
+        st_smem16(buf, SL::B_LM + sw128_offset(t, 8 * gg, kC * 128), pack8(x));
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      BackSync::sync();
+      GDR_PREP_PHASE(10);
+
+      // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
+      if (warp == 0) {
+        tc_fence_after();
+        const uint32_t bb = sb + bi * SL::BUF;
+        constexpr uint32_t id = idesc_bf16_f32(64, kDK, false, true);
+#pragma unroll
+        for (int s = 0; s < kC / 16; ++s) {
+          const uint64_t ad = sdesc_sw128(bb + SL::B_LM + s * 32, 16, 1024);
+          const uint64_t bu = sdesc_sw128(bb + SL::VH + s * 2048, kC * 128, 1024);
+          const uint64_t by = sdesc_sw128(bb + SL::A_LM + s * 2048, 2 * kC * 128, 1024);
+          mma_bf16_warp(tmem, ad, bu, id, s > 0);
+          mma_bf16_warp(tmem + kDK, ad, by, id, s > 0);
+        }
+        mma_commit_warp(bar2);
+        if (lane == 0) cnt[kM2Iss] = j + 1;
+      }
+      if (!group_wait<BackSync>(bar2, j & 1, sabort, poller)) break;
+      tc_fence_after();
+      GDR_PREP_PHASE(11);
+
+      // ---- the buffer is free: load chunk j + 2's tiles into it
+      if (gt == 32 && j + 2 < nloc) {
+        fence_proxy_async_smem();
+        const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
+        load_tiles(buf, maps, bfull + bi, bhn / H, bhn % H, cn * kC);
+        cnt[kBIss0 + bi] += 1;
+      }
+
+      // ---- U and Y (x alpha_1) -> bf16 record tiles; M = 64 accumulators: row 16 qd + lane.
+      //      cpart 0: U columns, 1: Y columns (128 each, four loads of 32).
+      {
+        const bool is_y = cpart == 1;
+        const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
+#pragma unroll
+        for (int part = 0; part < 4; ++part) {
+          const int col = 32 * part;
+          float x[32];
+          tmem_ld_32x32b_x32(tmem + lane_q + (is_y ? kDK : 0) + col, x);
+          tmem_ld_wait();
+          if (lane < 16) {
+            const int t = 16 * qd + lane;
+            if (is_y) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(a1s + col + i);
+                x[i] *= a.x; x[i + 1] *= a.y; x[i + 2] *= a.z; x[i + 3] *= a.w;
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 32; i += 8)
+              *reinterpret_cast<uint4 *>(
+                  rec + (is_y ? Rec::QY + sw128_offset(kC + t, col + i, Rec::QY_STRIDE)
+                              : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
+          }
+        }
+      }
+      tc_fence_before();
+      BackSync::sync();          // U / Y read before the next MMA2 overwrites them
+      GDR_PREP_PHASE(12);
+    }
   }
 
   GDR_PHASE_FINI(1)
-  if (!ok && tid == 0) {
+  __syncthreads();
+  if (tid == 0 && *sabort) {
     if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
-    // an MMA group or a staging load may still be in flight: let them land (bounded)
-    mbar_wait_bounded(mbar, phase ^ 1u, kWaitLimitNs);
-    if (s_issued > s_landed) mbar_wait_bounded(sbar, s_landed & 1u, kWaitLimitNs);
+    // let every TMA load and MMA group still in flight land (each wait bounded)
+    for (int bq = 0; bq < 2; ++bq)
+      for (uint32_t d = cnt[kBDone0 + bq]; d < cnt[kBIss0 + bq]; ++d)
+        if (!mbar_wait_bounded(bfull + bq, d & 1, kWaitLimitNs)) break;
+    for (uint32_t d = cnt[kADone]; d < cnt[kAIss]; ++d)
+      if (!mbar_wait_bounded(afull, d & 1, kWaitLimitNs)) break;
+    if (cnt[kM1Iss] > 0) mbar_wait_bounded(bar1, (cnt[kM1Iss] - 1) & 1, kWaitLimitNs);
+    if (cnt[kM2Iss] > 0) mbar_wait_bounded(bar2, (cnt[kM2Iss] - 1) & 1, kWaitLimitNs);
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, 2 * kTmemCols);
   }
 }
 
@@ -789,19 +897,20 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// [B][T][H][128] tensor of `elem` bytes as a 4-D map with a (128, 1, 64, 1) box.
+// [B][T][H][128] tensor of `elem` bytes as a 4-D map (channel, head, token, batch)
+// with a (box0, 1, C, 1) box.
 bool encode_input_map(CUtensorMap *m, const void *base, CUtensorMapDataType type, int elem,
-                      const FwdParams &p) {
+                      int box0, CUtensorMapSwizzle swizzle, const FwdParams &p) {
   PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
   if (!enc) return false;
   const cuuint64_t dims[4] = {(cuuint64_t)kDK, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
   const cuuint64_t strides[3] = {(cuuint64_t)kDK * elem, (cuuint64_t)p.H * kDK * elem,
                                  (cuuint64_t)p.T * p.H * kDK * elem};
-  const cuuint32_t box[4] = {(cuuint32_t)kDK, 1, (cuuint32_t)kC, 1};
+  const cuuint32_t box[4] = {(cuuint32_t)box0, 1, (cuuint32_t)kC, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   return enc(m, type, 4, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -810,11 +919,17 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   constexpr int NV = 64;
   PrepMaps maps;
   memset(&maps, 0, sizeof(maps));
+  // bf16 tiles: 64-channel boxes with the 128-byte swizzle (the MMA operand layout);
+  // log w: one 128-channel fp32 box, row-major
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-  if (!encode_input_map(&maps.k, p.k, bf, 2, p) || !encode_input_map(&maps.b, p.e1, bf, 2, p) ||
-      !encode_input_map(&maps.q, p.q, bf, 2, p) || !encode_input_map(&maps.v, p.v, bf, 2, p) ||
-      (p.e2 && !encode_input_map(&maps.wg, p.e2, bf, 2, p)) ||
-      !encode_input_map(&maps.lw, p.log_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p))
+  const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!encode_input_map(&maps.k, p.k, bf, 2, 64, sw, p) ||
+      !encode_input_map(&maps.b, p.e1, bf, 2, 64, sw, p) ||
+      !encode_input_map(&maps.q, p.q, bf, 2, 64, sw, p) ||
+      !encode_input_map(&maps.v, p.v, bf, 2, 64, sw, p) ||
+      (p.e2 && !encode_input_map(&maps.wg, p.e2, bf, 2, 64, sw, p)) ||
+      !encode_input_map(&maps.lw, p.log_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, p))
     return cudaErrorInvalidValue;
   uint8_t *records = static_cast<uint8_t *>(workspace) + kHeaderBytes;
   cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -184,8 +184,34 @@ __device__ __forceinline__ void store_16x8(const float (&d)[4], float sign, floa
 // CTA of NT threads, with the merge products X21 = -T_R^-1 (L_RL T_L^-1) on the
 // tensor cores as warp-level tf32 MMAs (16 x 8 tiles, fp32 accumulate): the
 // diagonal 16 x 16 blocks stay fp32 forward substitution.  Ends with a CTA barrier.
+// Barrier policies for the helpers below: the whole CTA, or a named barrier shared
+// by one group of N threads (warp-specialised kernels).
+struct CtaSync {
+  static __device__ __forceinline__ void sync() { __syncthreads(); }
+};
+template <int ID, int N>
+struct GroupSync {
+  static __device__ __forceinline__ void sync() {
+    asm volatile("bar.sync %0, %1;" ::"n"(ID), "n"(N) : "memory");
+  }
+  // Barrier that also returns, to every thread of the group, the OR of `v` over it.
+  static __device__ __forceinline__ bool sync_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred pi, po;\n\t"
+        "setp.ne.u32 pi, %1, 0;\n\t"
+        "bar.red.or.pred po, %2, %3, pi;\n\t"
+        "selp.u32 %0, 1, 0, po;\n\t}"
+        : "=r"(r)
+        : "r"(v ? 1u : 0u), "n"(ID), "n"(N)
+        : "memory");
+    return r != 0;
+  }
+};
+
 // Step 1: the four diagonal 16 x 16 blocks (and zeros in the upper blocks level 2 reads).
-template <class IxL, class IxT, int NT>
+// `tid` is the thread's index within the group that runs the inverse.
+template <class IxL, class IxT, int NT, class Sync = CtaSync>
 __device__ void invert_diag_blocks(const float *Lm, float *Ti, int tid) {
   if (tid < 64) {
     const int blk = tid >> 4, c = tid & 15, o = 16 * blk;
@@ -205,11 +231,11 @@ __device__ void invert_diag_blocks(const float *Lm, float *Ti, int tid) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) Ti[IxT::at(r, c + e)] = 0.f;
   }
-  __syncthreads();
+  Sync::sync();
 }
 
 // Step 2: the two merge levels on the tensor cores.
-template <class IxL, class IxT, int NT>
+template <class IxL, class IxT, int NT, class Sync = CtaSync>
 __device__ void invert_merge_levels(float *Lm, float *Ti, int tid) {
   static_assert(NT >= 256, "level 2 uses eight warps");
   const int warp = tid >> 5, lane = tid & 31;
@@ -217,28 +243,28 @@ __device__ void invert_merge_levels(float *Lm, float *Ti, int tid) {
   const int q1 = warp >> 1, nt1 = warp & 1, o1 = 32 * q1;
   float w1[4] = {0.f, 0.f, 0.f, 0.f};
   if (warp < 4) tile_16x8<IxL, IxT, 16>(w1, Lm, o1 + 16, o1, Ti, o1, o1 + 8 * nt1, lane);
-  __syncthreads();
+  Sync::sync();
   if (warp < 4) store_16x8<IxL>(w1, 1.f, Lm, o1 + 16, o1 + 8 * nt1, lane);
-  __syncthreads();
+  Sync::sync();
   if (warp < 4) {
     float x[4] = {0.f, 0.f, 0.f, 0.f};
     tile_16x8<IxT, IxL, 16>(x, Ti, o1 + 16, o1 + 16, Lm, o1 + 16, o1 + 8 * nt1, lane);
     store_16x8<IxT>(x, -1.f, Ti, o1 + 16, o1 + 8 * nt1, lane);
   }
-  __syncthreads();
+  Sync::sync();
   // level 2: rows 32..63 x columns 0..31; row tile mt, column tile nt
   const int mt = warp >> 2, nt2 = warp & 3;
   float w2[4] = {0.f, 0.f, 0.f, 0.f};
   if (warp < 8) tile_16x8<IxL, IxT, 32>(w2, Lm, 32 + 16 * mt, 0, Ti, 0, 8 * nt2, lane);
-  __syncthreads();
+  Sync::sync();
   if (warp < 8) store_16x8<IxL>(w2, 1.f, Lm, 32 + 16 * mt, 8 * nt2, lane);
-  __syncthreads();
+  Sync::sync();
   if (warp < 8) {
     float x[4] = {0.f, 0.f, 0.f, 0.f};
     tile_16x8<IxT, IxL, 32>(x, Ti, 32 + 16 * mt, 32, Lm, 32, 8 * nt2, lane);
     store_16x8<IxT>(x, -1.f, Ti, 32 + 16 * mt, 8 * nt2, lane);
   }
-  __syncthreads();
+  Sync::sync();
 }
 
 template <class IxL, class IxT, int NT>
