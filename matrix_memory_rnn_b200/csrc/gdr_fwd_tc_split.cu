@@ -7,7 +7,8 @@
 //
 //  * prep: everything that does not depend on the chunk's initial state S0 --
 //    the cumulative log-decay, the decay-weighted products L and M (one tcgen05
-//    MMA), T^-1 (fp32 diagonal blocks, tf32 warp-MMA merges), U = T^-1 V^ and
+//    MMA), T^-1 (fp32 8 x 8 diagonal blocks and 16 x 16 merge, tf32 warp-MMA
+//    merges at 32 and 64), U = T^-1 V^ and
 //    Y = T^-1 K^_pi (one tcgen05 MMA group), and the operand tiles Q_pi and K~.
 //    Chunks are independent: a persistent grid of one 512-thread CTA per SM walks
 //    them as a two-stage pipeline of warp groups (element-wise phase + MMA1 on
@@ -494,7 +495,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       GDR_PREP_PHASE(9);
 
       // ---- T^-1 (fp32, into the dead Q rows of A_LM), bf16 copy (into the dead L tile)
-      invert_diag_blocks<Ix, QRowsIdx, kGroup, BackSync>(sL, sTi, gt);
+      invert_diag_blocks8<Ix, QRowsIdx, kGroup, BackSync>(sL, sTi, gt);
       invert_merge_levels<Ix, QRowsIdx, kGroup, BackSync>(sL, sTi, gt);
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
@@ -542,32 +543,32 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         cnt[kBIss0 + bi] += 1;
       }
 
-      // ---- U and Y (x alpha_1) -> bf16 record tiles; M = 64 accumulators: row 16 qd + lane.
-      //      cpart 0: U columns, 1: Y columns (128 each, four loads of 32).
+      // ---- U and Y (x alpha_1) -> bf16 record tiles.  M = 64 accumulators: row
+      //      16 qd + r in TMEM lane 32 qd + r.  Warp (qd, cpart) reads U (cpart 0) or
+      //      Y (cpart 1) of its 16 rows, 64 columns per load: lanes 0..15 the first
+      //      32, lanes 16..31 the next 32.
       {
         const bool is_y = cpart == 1;
         const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
+        const int t = 16 * qd + (lane & 15);
 #pragma unroll
-        for (int part = 0; part < 4; ++part) {
-          const int col = 32 * part;
+        for (int part = 0; part < 2; ++part) {
+          const int col = 64 * part + 32 * (lane >> 4);
           float x[32];
-          tmem_ld_32x32b_x32(tmem + lane_q + (is_y ? kDK : 0) + col, x);
+          tmem_ld_16x32bx2_x32_split32(tmem + lane_q + (is_y ? kDK : 0) + 64 * part, x);
           tmem_ld_wait();
-          if (lane < 16) {
-            const int t = 16 * qd + lane;
-            if (is_y) {
+          if (is_y) {
 #pragma unroll
-              for (int i = 0; i < 32; i += 4) {
-                const float4 a = *reinterpret_cast<const float4 *>(a1s + col + i);
-                x[i] *= a.x; x[i + 1] *= a.y; x[i + 2] *= a.z; x[i + 3] *= a.w;
-              }
+            for (int i = 0; i < 32; i += 4) {
+              const float4 a = *reinterpret_cast<const float4 *>(a1s + col + i);
+              x[i] *= a.x; x[i + 1] *= a.y; x[i + 2] *= a.z; x[i + 3] *= a.w;
             }
-#pragma unroll
-            for (int i = 0; i < 32; i += 8)
-              *reinterpret_cast<uint4 *>(
-                  rec + (is_y ? Rec::QY + sw128_offset(kC + t, col + i, Rec::QY_STRIDE)
-                              : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
           }
+#pragma unroll
+          for (int i = 0; i < 32; i += 8)
+            *reinterpret_cast<uint4 *>(
+                rec + (is_y ? Rec::QY + sw128_offset(kC + t, col + i, Rec::QY_STRIDE)
+                            : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
         }
       }
       tc_fence_before();

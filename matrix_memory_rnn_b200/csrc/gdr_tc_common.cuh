@@ -234,6 +234,58 @@ __device__ void invert_diag_blocks(const float *Lm, float *Ti, int tid) {
   Sync::sync();
 }
 
+// Step 1 with shorter dependency chains: the eight 8 x 8 diagonal blocks by forward
+// substitution (64 threads), then each 16 x 16 block's lower-left 8 x 8 by the same
+// merge X21 = -T_R^-1 (L_RL T_L^-1) (one thread per entry).  Needs NT >= 256.
+template <class IxL, class IxT, int NT, class Sync = CtaSync>
+__device__ void invert_diag_blocks8(float *Lm, float *Ti, int tid) {
+  static_assert(NT >= 256, "one thread per entry of the four 8 x 8 merges");
+  if (tid < 64) {
+    const int o = 8 * (tid >> 3), c = tid & 7;
+    float x[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      float acc = (t == c) ? 1.f : 0.f;
+#pragma unroll
+      for (int s = 0; s < t; ++s) acc -= Lm[IxL::at(o + t, o + s)] * x[s];
+      x[t] = acc;
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) Ti[IxT::at(o + t, o + c)] = x[t];
+  } else if (tid < 64 + 128) {
+    // zeros: the upper-right 8 x 8 of each 16 x 16 block (2 entries per thread) and
+    // the upper 16 x 16 blocks of the two 32 x 32 blocks (4 entries per thread)
+    const int u = tid - 64;
+    {
+      const int p = u >> 5, r = (u >> 2) & 7, c = 2 * (u & 3);
+      Ti[IxT::at(16 * p + r, 16 * p + 8 + c)] = 0.f;
+      Ti[IxT::at(16 * p + r, 16 * p + 8 + c + 1)] = 0.f;
+    }
+    const int k = u * 4, q = k >> 8, r = 32 * q + ((k >> 4) & 15), c = 32 * q + 16 + (k & 15);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) Ti[IxT::at(r, c + e)] = 0.f;
+  }
+  Sync::sync();
+  {
+    const int p = (tid >> 6) & 3, r = (tid >> 3) & 7, c = tid & 7, o = 16 * p;
+    float w = 0.f;
+    if (tid < 256) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) w += Lm[IxL::at(o + 8 + r, o + k)] * Ti[IxT::at(o + k, o + c)];
+    }
+    Sync::sync();
+    if (tid < 256) Lm[IxL::at(o + 8 + r, o + c)] = w;
+    Sync::sync();
+    if (tid < 256) {
+      float x = 0.f;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) x += Ti[IxT::at(o + 8 + r, o + 8 + k)] * Lm[IxL::at(o + 8 + k, o + c)];
+      Ti[IxT::at(o + 8 + r, o + c)] = -x;
+    }
+  }
+  Sync::sync();
+}
+
 // Step 2: the two merge levels on the tensor cores.
 template <class IxL, class IxT, int NT, class Sync = CtaSync>
 __device__ void invert_merge_levels(float *Lm, float *Ti, int tid) {
