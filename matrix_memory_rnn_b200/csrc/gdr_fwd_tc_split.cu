@@ -11,9 +11,9 @@
 //    merges at 32 and 64), U = T^-1 V^ and
 //    Y = T^-1 K^_pi (one tcgen05 MMA group), and the operand tiles Q_pi and K~.
 //    Chunks are independent: a persistent grid of one 512-thread CTA per SM walks
-//    them as a two-stage pipeline of warp groups (element-wise phase + MMA1 on
-//    one chunk while T^-1 + MMA2 run on the previous one); inputs arrive by TMA,
-//    the bf16 ones straight into the MMA tiles.  Each chunk's result is a
+//    them as a two-stage pipeline of warp groups (scan, element-wise phase and
+//    MMA1 on one chunk while L readout, T^-1 and MMA2 run on the previous one);
+//    inputs arrive by TMA, the bf16 ones straight into the MMA tiles.  Each chunk's result is a
 //    record of bf16 MMA tiles, already in the 128-byte-swizzled shared-memory
 //    layout, in the workspace.
 //  * chain: the inter-chunk state carry and the outputs, sequential over chunks
@@ -88,15 +88,14 @@ __host__ __device__ inline int num_chunks(int T) { return (T + kC - 1) / kC; }
 // Persistent: one CTA of 512 threads per SM walks the chunks (b, h, c) with a
 // stride of gridDim.x, as a two-stage pipeline of warp groups over two chunk
 // buffers:
-//   front (warps 8..15): log-decay scan, operand tiles, MMA1, L / M readout of
-//                        chunk j;
-//   back  (warps 0..7):  T^-1, MMA2, U / Y readout of chunk j - 1.
+//   front (warps 8..15): log-decay scan, operand tiles and MMA1 of chunk j;
+//   back  (warps 0..7):  L / M readout, T^-1, MMA2 and U / Y readout of chunk j - 1.
 // Inputs arrive by TMA: k, b, q, v straight into the chunk buffer's MMA tiles
 // (128-byte swizzle, the tcgen05 operand layout), where the element-wise phase
-// turns them into K g, K^ f, Q f, V^ in place; wg and log w into a staging area.
-// The back group issues chunk j + 2's tile loads as soon as MMA2 of chunk j has
-// released its buffer; the front group loads the next staging area as soon as it
-// has read the current one.
+// turns them into K g, K^ f, Q f, V^ in place; wg into one of two staging tiles,
+// log w into a staging area that the scan releases as soon as it has read it.
+// The back group loads chunk j + 2's tiles as soon as MMA2 of chunk j has
+// released its buffer.
 constexpr int kPrepThreads = 512;
 constexpr int kGroup = 256;                    // threads per warp group
 using FrontSync = GroupSync<1, kGroup>;
@@ -119,13 +118,12 @@ struct PrepSmem {
                                                               //   fp32 L; then bf16 T^-1 (first 8 KB)
   static constexpr uint32_t VH = B_LM + kC * kDK * 2;         // V^ = wg (.) v (v lands here)
   static constexpr uint32_t BUF = VH + kC * kDK * 2;          // 64 KB per buffer
-  // staging (single): write gate (sw128, same offsets as v), log w (row-major fp32)
-  static constexpr uint32_t SW = 2 * BUF;
-  static constexpr uint32_t SLW = SW + kC * kDK * 2;          // log w, then Lam_t - Lam_1
-  static constexpr uint32_t QT = SLW + kC * kDK * 4;          // fp32 [2][DK] half sums of log w
-  static constexpr uint32_t L1 = QT + 2 * kDK * 4;            // fp32 Lam_1 per channel
-  static constexpr uint32_t DN = L1 + kDK * 4;                // fp32 Lam_n - Lam_1 per channel
-  static constexpr uint32_t A1 = DN + kDK * 4;                // fp32 [4][DK] alpha_1, by chunk & 3
+  static constexpr uint32_t SW = 2 * BUF;                     // write gate x2 (sw128, offsets as v)
+  static constexpr uint32_t SLW = SW + 2 * kC * kDK * 2;      // log w, row-major fp32
+  static constexpr uint32_t BT = SLW + kC * kDK * 4;          // fp32 [16][DK] block sums -> prefixes
+  static constexpr uint32_t TOT = BT + 16 * kDK * 4;          // fp32 Lam_n per channel
+  static constexpr uint32_t L1 = TOT + kDK * 4;               // fp32 Lam_1 per channel
+  static constexpr uint32_t A1 = L1 + kDK * 4;                // fp32 [4][DK] alpha_1, by chunk & 3
   static constexpr uint32_t MISC = A1 + 4 * kDK * 4;
   static constexpr uint32_t ALLOC = MISC + 256 + 1024;
   static_assert(BUF % 1024 == 0 && SW % 1024 == 0, "MMA tiles 1024-aligned");
@@ -135,16 +133,20 @@ struct PrepSmem {
 
 struct PrepMisc {             // byte offsets inside PrepSmem::MISC
   static constexpr uint32_t BFULL = 0;      // uint64_t [2] chunk-buffer tiles landed
-  static constexpr uint32_t AFULL = 16;     // uint64_t     staging landed
-  static constexpr uint32_t READY = 24;     // uint64_t [2] front -> back: buffer holds L, V^, K^ f
-  static constexpr uint32_t BAR1 = 40;      // uint64_t     MMA1 done (front)
-  static constexpr uint32_t BAR2 = 48;      // uint64_t     MMA2 done (back)
-  static constexpr uint32_t SLOT = 56;      // uint32_t     TMEM base
-  static constexpr uint32_t ABORT = 60;     // int          a bounded wait ran out
-  static constexpr uint32_t EXACT = 64;     // int          front: this chunk takes the exact path
-  static constexpr uint32_t CNT = 128;      // uint32_t [8] issued / completed counts (drain)
+  static constexpr uint32_t WFULL = 16;     // uint64_t [2] write-gate staging landed
+  static constexpr uint32_t LFULL = 32;     // uint64_t     log-w staging landed
+  static constexpr uint32_t READY = 40;     // uint64_t [2] front -> back: operand tiles written
+  static constexpr uint32_t BAR1 = 56;      // uint64_t [2] MMA1 done, per buffer
+  static constexpr uint32_t BAR2 = 72;      // uint64_t     MMA2 done
+  static constexpr uint32_t SLOT = 80;      // uint32_t     TMEM base
+  static constexpr uint32_t ABORT = 84;     // int          a bounded wait ran out
+  static constexpr uint32_t EXACT = 88;     // int [2]      the buffer's chunk takes the exact path
+  static constexpr uint32_t CNT = 128;      // uint32_t [16] issued / completed counts (drain)
 };
-enum { kBIss0, kBIss1, kBDone0, kBDone1, kAIss, kADone, kM2Iss, kM1Iss };
+enum {
+  kBIss0, kBIss1, kBDone0, kBDone1, kWIss0, kWIss1, kWDone0, kWDone1,
+  kLIss, kLDone, kM1Iss0, kM1Iss1, kM1Done0, kM1Done1, kM2Iss, kNCnt
+};
 
 // Tensor maps of the prep inputs, each 4-D (channel, head, token, batch).  k, b, q,
 // v, wg: bf16 boxes of 64 channels x 64 tokens with the 128-byte swizzle (one
@@ -168,16 +170,19 @@ __device__ __forceinline__ void load_tiles(uint8_t *buf, const PrepMaps &m, uint
   }
 }
 
-// One thread: the staging loads (wg if present, log w) for chunk (b, h, t0).
-__device__ __forceinline__ void load_staging(uint8_t *smem, const PrepMaps &m, uint64_t *bar, int b,
-                                             int h, int t0, bool has_wg) {
-  using SL = PrepSmem;
-  mbar_arrive_expect_tx(bar, (has_wg ? kC * kDK * 2u : 0u) + kC * kDK * 4u);
-  if (has_wg) {
-    tma_load_4d(smem + SL::SW, &m.wg, 0, h, t0, b, bar);
-    tma_load_4d(smem + SL::SW + kC * 128, &m.wg, 64, h, t0, b, bar);
-  }
-  tma_load_4d(smem + SL::SLW, &m.lw, 0, h, t0, b, bar);
+// One thread: the write gate of chunk (b, h, t0) into staging tile `sw`.
+__device__ __forceinline__ void load_gate(uint8_t *sw, const PrepMaps &m, uint64_t *bar, int b, int h,
+                                          int t0) {
+  mbar_arrive_expect_tx(bar, kC * kDK * 2u);
+  tma_load_4d(sw, &m.wg, 0, h, t0, b, bar);
+  tma_load_4d(sw + kC * 128, &m.wg, 64, h, t0, b, bar);
+}
+
+// One thread: log w of chunk (b, h, t0) into the log-w staging area.
+__device__ __forceinline__ void load_logw(uint8_t *slw, const PrepMaps &m, uint64_t *bar, int b, int h,
+                                          int t0) {
+  mbar_arrive_expect_tx(bar, kC * kDK * 4u);
+  tma_load_4d(slw, &m.lw, 0, h, t0, b, bar);
 }
 
 // One thread of a group polls `bar` for `parity` (bounded; gives up at once when the
@@ -223,7 +228,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 
   uint8_t *misc = smem + SL::MISC;
   uint64_t *bfull = reinterpret_cast<uint64_t *>(misc + PrepMisc::BFULL);
-  uint64_t *afull = reinterpret_cast<uint64_t *>(misc + PrepMisc::AFULL);
+  uint64_t *wfull = reinterpret_cast<uint64_t *>(misc + PrepMisc::WFULL);
+  uint64_t *lfull = reinterpret_cast<uint64_t *>(misc + PrepMisc::LFULL);
   uint64_t *ready = reinterpret_cast<uint64_t *>(misc + PrepMisc::READY);
   uint64_t *bar1 = reinterpret_cast<uint64_t *>(misc + PrepMisc::BAR1);
   uint64_t *bar2 = reinterpret_cast<uint64_t *>(misc + PrepMisc::BAR2);
@@ -231,10 +237,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   volatile int *sabort = reinterpret_cast<volatile int *>(misc + PrepMisc::ABORT);
   volatile int *sexact = reinterpret_cast<volatile int *>(misc + PrepMisc::EXACT);
   uint32_t *cnt = reinterpret_cast<uint32_t *>(misc + PrepMisc::CNT);
-  float *sLW = reinterpret_cast<float *>(smem + SL::SLW);
-  float *sQT = reinterpret_cast<float *>(smem + SL::QT);
+  const float *sLW = reinterpret_cast<const float *>(smem + SL::SLW);
+  float *sBT = reinterpret_cast<float *>(smem + SL::BT);
+  float *sTOT = reinterpret_cast<float *>(smem + SL::TOT);
   float *sL1 = reinterpret_cast<float *>(smem + SL::L1);
-  float *sDN = reinterpret_cast<float *>(smem + SL::DN);
   float *sA1 = reinterpret_cast<float *>(smem + SL::A1);
   const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
@@ -249,108 +255,158 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(bfull + i, 1);
+      mbar_init(wfull + i, 1);
       mbar_init(ready + i, 1);
+      mbar_init(bar1 + i, 1);
+      sexact[i] = 0;
     }
-    mbar_init(afull, 1);
-    mbar_init(bar1, 1);
+    mbar_init(lfull, 1);
     mbar_init(bar2, 1);
     fence_mbar_init();
     *sabort = 0;
-    for (int i = 0; i < 8; ++i) cnt[i] = 0;
+    for (int i = 0; i < kNCnt; ++i) cnt[i] = 0;
     for (int j = 0; j < 2 && j < nloc; ++j) {
       const int it = item_of(j), c = it % nch, bh = it / nch;
       load_tiles(smem + j * SL::BUF, maps, bfull + j, bh / H, bh % H, c * kC);
       ++cnt[kBIss0 + j];
-    }
-    if (nloc > 0) {
-      const int it = item_of(0), c = it % nch, bh = it / nch;
-      load_staging(smem, maps, afull, bh / H, bh % H, c * kC, has_wg);
-      ++cnt[kAIss];
+      if (has_wg) {
+        load_gate(smem + SL::SW + j * (kC * kDK * 2), maps, wfull + j, bh / H, bh % H, c * kC);
+        ++cnt[kWIss0 + j];
+      }
+      if (j == 0) {
+        load_logw(smem + SL::SLW, maps, lfull, bh / H, bh % H, c * kC);
+        ++cnt[kLIss];
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
-  const uint32_t tD1 = tmem + 2 * kDK;                    // front: L | M accumulator (64 columns)
+  const uint32_t tD1 = tmem + 2 * kDK;                    // L | M accumulators, 64 columns x 2
 
   if (front) {
     // =========================================================== front group
     const bool poller = gt == 0;
+    const int g = gt & 15, tb = gt >> 4, j0 = 8 * g;      // 8 channels x 4 tokens per thread
     for (int j = 0; j < nloc; ++j) {
-      const int item = item_of(j), c = item % nch, bh = item / nch, h = bh % H, b = bh / H;
-      const int t0 = c * kC, n = min(kC, T - t0), bi = j & 1;
+      const int item = item_of(j), bi = j & 1;
       uint8_t *buf = smem + bi * SL::BUF;
-      float *sL = reinterpret_cast<float *>(buf + SL::B_LM);
       uint8_t *rec = records + (size_t)item * Rec::BYTES;
       float *a1s = sA1 + (j & 3) * kDK;
-      auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
       GDR_PREP_PHASE(0);
 
-      // chunk j's staging and tiles have landed
-      if (poller) *sexact = 0;
-      if (!group_wait<FrontSync>(afull, j & 1, sabort, poller)) break;
+      // chunk j's log w, tiles and write gate have landed
+      if (poller) sexact[bi] = 0;
+      if (!group_wait<FrontSync>(lfull, j & 1, sabort, poller)) break;
       if (!group_wait<FrontSync>(bfull + bi, (j >> 1) & 1, sabort, poller)) break;
+      if (has_wg && !group_wait<FrontSync>(wfull + bi, (j >> 1) & 1, sabort, poller)) break;
       if (poller) {
-        cnt[kADone] = j + 1;
+        cnt[kLDone] = j + 1;
         cnt[kBDone0 + bi] += 1;
+        if (has_wg) cnt[kWDone0 + bi] += 1;
       }
       GDR_PREP_PHASE(1);
 
-      // ---- cumulative log-decay: thread = (channel ch, token half), in place
+      // ---- cumulative log-decay in registers: prefix over the thread's 4 tokens,
+      //      then the exclusive prefix over the 16 token blocks (one thread per channel)
+      float lam[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 x0 = *reinterpret_cast<const float4 *>(sLW + (4 * tb + i) * kDK + j0);
+        const float4 x1 = *reinterpret_cast<const float4 *>(sLW + (4 * tb + i) * kDK + j0 + 4);
+        lam[i][0] = x0.x; lam[i][1] = x0.y; lam[i][2] = x0.z; lam[i][3] = x0.w;
+        lam[i][4] = x1.x; lam[i][5] = x1.y; lam[i][6] = x1.z; lam[i][7] = x1.w;
+      }
       {
-        const int ch = gt & (kDK - 1), hv = gt >> 7;
-        float x[32];
-        float acc = 0.f;
+        float tot[8];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          acc += sLW[(32 * hv + i) * kDK + ch];
-          x[i] = acc;
+        for (int e = 0; e < 8; ++e) {
+          float acc = 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            acc += lam[i][e];
+            lam[i][e] = acc;
+          }
+          tot[e] = acc;
         }
-        sQT[hv * kDK + ch] = acc;
-        if (hv == 0) sL1[ch] = x[0];
-        FrontSync::sync();
-        const float q0 = sQT[ch], all = q0 + sQT[kDK + ch];
-        const float l1 = sL1[ch], shift = (hv ? q0 : 0.f) - l1;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) sLW[(32 * hv + i) * kDK + ch] = x[i] + shift;
-        if (hv == 0) {
-          const float dn = all - l1;
-          sDN[ch] = dn;
-          a1s[ch] = __expf(l1);
-          reinterpret_cast<float *>(rec + Rec::PI)[ch] = __expf(all);
-          if (dn < -kMaxChunkDecay) *sexact = 1;
+        float4 *bt = reinterpret_cast<float4 *>(sBT + tb * kDK + j0);
+        bt[0] = make_float4(tot[0], tot[1], tot[2], tot[3]);
+        bt[1] = make_float4(tot[4], tot[5], tot[6], tot[7]);
+        if (tb == 0) {
+          float4 *l1 = reinterpret_cast<float4 *>(sL1 + j0);
+          l1[0] = make_float4(lam[0][0], lam[0][1], lam[0][2], lam[0][3]);
+          l1[1] = make_float4(lam[0][4], lam[0][5], lam[0][6], lam[0][7]);
         }
       }
       FrontSync::sync();
-      const bool exact = *sexact != 0;
+      // the log-w staging has been read: load the next chunk's
+      if (gt == 32 && j + 1 < nloc) {
+        fence_proxy_async_smem();
+        const int it = item_of(j + 1), cn = it % nch, bhn = it / nch;
+        load_logw(smem + SL::SLW, maps, lfull, bhn / H, bhn % H, cn * kC);
+        cnt[kLIss] = j + 2;
+      }
+      if (gt < kDK) {
+        float run = 0.f;
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+          const float v = sBT[r * kDK + gt];
+          sBT[r * kDK + gt] = run;
+          run += v;
+        }
+        sTOT[gt] = run;
+      }
+      FrontSync::sync();
+      // lam[i][e] becomes Lam_t - Lam_1 (the pivot at the chunk's first token)
+      float dn[8], ed[8];
+      {
+        const float4 e0 = *reinterpret_cast<const float4 *>(sBT + tb * kDK + j0);
+        const float4 e1 = *reinterpret_cast<const float4 *>(sBT + tb * kDK + j0 + 4);
+        const float4 a0 = *reinterpret_cast<const float4 *>(sTOT + j0);
+        const float4 a4 = *reinterpret_cast<const float4 *>(sTOT + j0 + 4);
+        const float4 f0 = *reinterpret_cast<const float4 *>(sL1 + j0);
+        const float4 f4 = *reinterpret_cast<const float4 *>(sL1 + j0 + 4);
+        const float excl[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+        const float all[8] = {a0.x, a0.y, a0.z, a0.w, a4.x, a4.y, a4.z, a4.w};
+        const float l1[8] = {f0.x, f0.y, f0.z, f0.w, f4.x, f4.y, f4.z, f4.w};
+        bool over = false;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) lam[i][e] += excl[e] - l1[e];
+          dn[e] = all[e] - l1[e];
+          ed[e] = __expf(dn[e]);
+          over |= dn[e] < -kMaxChunkDecay;
+        }
+        if (over) sexact[bi] = 1;
+        if (tb == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            a1s[j0 + e] = __expf(l1[e]);
+            reinterpret_cast<float *>(rec + Rec::PI)[j0 + e] = __expf(all[e]);
+          }
+        }
+      }
+      FrontSync::sync();
+      const bool exact = sexact[bi] != 0;
       GDR_PREP_PHASE(2);
 
       // ---- operand tiles, in place: k -> K g, b -> K^ f, q -> Q f; Q_pi, K~ to the
-      //      record.  Thread = (channel group g of 8, token block tb of 4).
+      //      record (the exact path also parks Lam_t - Lam_1 there)
       {
-        const int g = gt & 15, tb = gt >> 4, j0 = 8 * g;
-        float dn[8], a1[8], ed[8];
+        float a1[8];
         {
-          const float4 d0 = *reinterpret_cast<const float4 *>(sDN + j0);
-          const float4 d1 = *reinterpret_cast<const float4 *>(sDN + j0 + 4);
           const float4 a0 = *reinterpret_cast<const float4 *>(a1s + j0);
           const float4 a4 = *reinterpret_cast<const float4 *>(a1s + j0 + 4);
-          dn[0] = d0.x; dn[1] = d0.y; dn[2] = d0.z; dn[3] = d0.w;
-          dn[4] = d1.x; dn[5] = d1.y; dn[6] = d1.z; dn[7] = d1.w;
           a1[0] = a0.x; a1[1] = a0.y; a1[2] = a0.z; a1[3] = a0.w;
           a1[4] = a4.x; a1[5] = a4.y; a1[6] = a4.z; a1[7] = a4.w;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) ed[e] = __expf(dn[e]);
         }
         auto operands = [&](auto exact_path) {
           constexpr bool kExact = decltype(exact_path)::value;
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const int t = 4 * tb + i;
-            const float4 l0 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0);
-            const float4 l4 = *reinterpret_cast<const float4 *>(sLW + t * kDK + j0 + 4);
-            const float lam[8] = {l0.x, l0.y, l0.z, l0.w, l4.x, l4.y, l4.z, l4.w};
             const uint32_t ok_ = sw128_offset(t, j0, kC * 128);
             const uint32_t ob = SL::A_LM + sw128_offset(t, j0, 2 * kC * 128);
             const uint32_t oq = SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128);
@@ -361,18 +417,18 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             float av[8], aq[8], bl[8], kt[8], qp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float f = __expf(lam[e]);
+              const float f = __expf(lam[i][e]);
               av[e] = b8[e] * k8[e] * f;
               aq[e] = q8[e] * f;
               qp[e] = aq[e] * a1[e];
               if (!kExact) {
-                bl[e] = k8[e] * __expf(-lam[e]);
+                bl[e] = k8[e] * __expf(-lam[i][e]);
                 kt[e] = bl[e] * ed[e];
               } else if (dn[e] >= -kMaxChunkDecay) {
-                kt[e] = k8[e] * __expf(-lam[e]) * ed[e];
+                kt[e] = k8[e] * __expf(-lam[i][e]) * ed[e];
                 bl[e] = 0.f;     // the exact path forms L and M without K g
               } else {
-                kt[e] = k8[e] * __expf(dn[e] - lam[e]);
+                kt[e] = k8[e] * __expf(dn[e] - lam[i][e]);
                 bl[e] = 0.f;
               }
             }
@@ -383,8 +439,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             *reinterpret_cast<uint4 *>(rec + Rec::KT + ok_) = pack8(kt);
             if (kExact) {
               float4 *dst = reinterpret_cast<float4 *>(rec + park_row(t)) + g * 2;
-              dst[0] = l0;
-              dst[1] = l4;
+              dst[0] = make_float4(lam[i][0], lam[i][1], lam[i][2], lam[i][3]);
+              dst[1] = make_float4(lam[i][4], lam[i][5], lam[i][6], lam[i][7]);
             }
           }
         };
@@ -393,12 +449,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       }
       // ---- V^ = wg (.) v in place (wg staged at the same swizzled offsets)
       if (has_wg) {
+        const uint8_t *sw = smem + SL::SW + bi * (kC * kDK * 2);
 #pragma unroll
         for (int u = 0; u < kC * 16 / kGroup; ++u) {
           const uint32_t off = (uint32_t)(gt + u * kGroup) * 16;
           float v8[8], w8[8];
           unpack8(*reinterpret_cast<const uint4 *>(buf + SL::VH + off), v8);
-          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::SW + off), w8);
+          unpack8(*reinterpret_cast<const uint4 *>(sw + off), w8);
 #pragma unroll
           for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
           st_smem16(buf, SL::VH + off, pack8(v8));
@@ -408,12 +465,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       FrontSync::sync();
       GDR_PREP_PHASE(3);
 
-      // ---- the staging area is read: load the next chunk's; MMA1 on this chunk
-      if (gt == 32 && j + 1 < nloc) {
+      // ---- the write-gate staging tile is read: load chunk j + 2's; MMA1 on this chunk
+      if (gt == 32 && has_wg && j + 2 < nloc) {
         fence_proxy_async_smem();
-        const int it = item_of(j + 1), cn = it % nch, bhn = it / nch;
-        load_staging(smem, maps, afull, bhn / H, bhn % H, cn * kC, has_wg);
-        cnt[kAIss] = j + 2;
+        const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
+        load_gate(smem + SL::SW + bi * (kC * kDK * 2), maps, wfull + bi, bhn / H, bhn % H, cn * kC);
+        cnt[kWIss0 + bi] += 1;
       }
       if (warp == 8) {
         // MMA1: [K^ f; Q f] (M = 128) x (K g)^T (N = C), K = DK  -> L, M
@@ -424,19 +481,38 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         for (int s = 0; s < kDK / 16; ++s) {
           const uint64_t ad = sdesc_sw128(bb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
           const uint64_t bd = sdesc_sw128(bb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
-          mma_bf16_warp(tD1, ad, bd, id, s > 0);
+          mma_bf16_warp(tD1 + 64 * bi, ad, bd, id, s > 0);
         }
-        mma_commit_warp(bar1);
-        if (lane == 0) cnt[kM1Iss] = j + 1;
+        mma_commit_warp(bar1 + bi);
+        if (lane == 0) cnt[kM1Iss0 + bi] += 1;
       }
-      if (!group_wait<FrontSync>(bar1, j & 1, sabort, poller)) break;
-      tc_fence_after();
+      if (poller) mbar_arrive(ready + bi);                 // hand the chunk to the back group
       GDR_PREP_PHASE(4);
+    }
+  } else {
+    // =========================================================== back group
+    const bool poller = gt == 0;
+    for (int j = 0; j < nloc; ++j) {
+      const int item = item_of(j), c = item % nch, bh = item / nch, h = bh % H, b = bh / H;
+      const int t0 = c * kC, n = min(kC, T - t0), bi = j & 1;
+      uint8_t *buf = smem + bi * SL::BUF;
+      float *sL = reinterpret_cast<float *>(buf + SL::B_LM);
+      float *sTi = reinterpret_cast<float *>(buf + SL::A_LM);
+      uint8_t *rec = records + (size_t)item * Rec::BYTES;
+      const float *a1s = sA1 + (j & 3) * kDK;
+      auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
+      GDR_PREP_PHASE(8);
+      if (!group_wait<BackSync>(ready + bi, (j >> 1) & 1, sabort, poller)) break;
+      if (!group_wait<BackSync>(bar1 + bi, (j >> 1) & 1, sabort, poller)) break;
+      if (poller) cnt[kM1Done0 + bi] += 1;
+      tc_fence_after();
+      const bool exact = sexact[bi] != 0;
+      GDR_PREP_PHASE(9);
 
       // ---- L (fp32, strictly lower; over the dead K g tile) and M (bf16 -> record)
       if (!exact) {
         float x[32];
-        tmem_ld_32x32b_x32(tD1 + ((uint32_t)(32 * qd) << 16) + 32 * cpart, x);
+        tmem_ld_32x32b_x32(tD1 + 64 * bi + ((uint32_t)(32 * qd) << 16) + 32 * cpart, x);
         tmem_ld_wait();
         const int r = 32 * qd + lane, col = 32 * cpart;
         if (r < kC) {
@@ -475,24 +551,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         }
       }
       tc_fence_before();
-      FrontSync::sync();
-      if (poller) mbar_arrive(ready + bi);                 // hand the buffer to the back group
-      GDR_PREP_PHASE(5);
-    }
-  } else {
-    // =========================================================== back group
-    const bool poller = gt == 0;
-    for (int j = 0; j < nloc; ++j) {
-      const int item = item_of(j), bi = j & 1;
-      uint8_t *buf = smem + bi * SL::BUF;
-      float *sL = reinterpret_cast<float *>(buf + SL::B_LM);
-      float *sTi = reinterpret_cast<float *>(buf + SL::A_LM);
-      uint8_t *rec = records + (size_t)item * Rec::BYTES;
-      const float *a1s = sA1 + (j & 3) * kDK;
-      GDR_PREP_PHASE(8);
-      if (!group_wait<BackSync>(ready + bi, (j >> 1) & 1, sabort, poller)) break;
-      tc_fence_after();
-      GDR_PREP_PHASE(9);
+      BackSync::sync();
+      GDR_PREP_PHASE(10);
 
       // ---- T^-1 (fp32, into the dead Q rows of A_LM), bf16 copy (into the dead L tile)
       invert_diag_blocks8<Ix, QRowsIdx, kGroup, BackSync>(sL, sTi, gt);
@@ -513,7 +573,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       BackSync::sync();
-      GDR_PREP_PHASE(10);
+      GDR_PREP_PHASE(11);
 
       // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
       if (warp == 0) {
@@ -533,7 +593,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       }
       if (!group_wait<BackSync>(bar2, j & 1, sabort, poller)) break;
       tc_fence_after();
-      GDR_PREP_PHASE(11);
+      GDR_PREP_PHASE(12);
 
       // ---- the buffer is free: load chunk j + 2's tiles into it
       if (gt == 32 && j + 2 < nloc) {
@@ -573,7 +633,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       }
       tc_fence_before();
       BackSync::sync();          // U / Y read before the next MMA2 overwrites them
-      GDR_PREP_PHASE(12);
+      GDR_PREP_PHASE(13);
     }
   }
 
@@ -582,12 +642,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   if (tid == 0 && *sabort) {
     if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
     // let every TMA load and MMA group still in flight land (each wait bounded)
-    for (int bq = 0; bq < 2; ++bq)
+    for (int bq = 0; bq < 2; ++bq) {
       for (uint32_t d = cnt[kBDone0 + bq]; d < cnt[kBIss0 + bq]; ++d)
         if (!mbar_wait_bounded(bfull + bq, d & 1, kWaitLimitNs)) break;
-    for (uint32_t d = cnt[kADone]; d < cnt[kAIss]; ++d)
-      if (!mbar_wait_bounded(afull, d & 1, kWaitLimitNs)) break;
-    if (cnt[kM1Iss] > 0) mbar_wait_bounded(bar1, (cnt[kM1Iss] - 1) & 1, kWaitLimitNs);
+      for (uint32_t d = cnt[kWDone0 + bq]; d < cnt[kWIss0 + bq]; ++d)
+        if (!mbar_wait_bounded(wfull + bq, d & 1, kWaitLimitNs)) break;
+      for (uint32_t d = cnt[kM1Done0 + bq]; d < cnt[kM1Iss0 + bq]; ++d)
+        if (!mbar_wait_bounded(bar1 + bq, d & 1, kWaitLimitNs)) break;
+    }
+    for (uint32_t d = cnt[kLDone]; d < cnt[kLIss]; ++d)
+      if (!mbar_wait_bounded(lfull, d & 1, kWaitLimitNs)) break;
     if (cnt[kM2Iss] > 0) mbar_wait_bounded(bar2, (cnt[kM2Iss] - 1) & 1, kWaitLimitNs);
   }
   tc_fence_before();
