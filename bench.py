@@ -55,6 +55,14 @@ def fwd_flops(w) -> int:
     return int(w.B * w.T * w.H * (6 * d * d + 5 * C * d + C * C / 3))
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of the
+# current kernels on a quarter-size case, scaled by the units processed).  Forward: prep +
+# chain, per (b, h, 64-token chunk) of the GDN-2 bf16 d = 128 tensor-core path; decode: per
+# (b, h) step of the d = 128 persistent kernel.  Must be re-measured when those kernels change.
+FWD_TC_TRAFFIC_PER_CHUNK = (117.6e6 + 32.0e6 + 76.1e6 + 11.1e6) / 1024
+DEC_TRAFFIC_PER_HEAD = (137.9e6 + 81.0e6) / (64 * 32)
+
+
 def dec_algorithmic_bytes(w) -> int:
     eb = 2
     state = 2 * w.B * w.H * w.dk * w.dv * 4
@@ -256,7 +264,7 @@ class Ctx:
 def bench_forward(ctx, args, gdr):
     """Device-resident chunked forward: K timed steps, kernel time per launch."""
     torch = ctx.torch
-    w = FWD
+    w = FWD if args.fwd_batch is None else FWD.with_(B=args.fwd_batch)
     inp = synth.forward_inputs(w, seed=w.seed + 1000 * ctx.rank)
     names = ("q", "k", "v", "log_w", "e1", "e2")
     d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
@@ -303,7 +311,7 @@ def bench_forward(ctx, args, gdr):
                                                             d["log_w"], d["e1"], d["e2"],
                                                             w.chunk, "tc") > 256
     per_call = 2 if (args.algo in ("auto", "tc") and full_ws and w.form == "gdn2"
-                     and w.dtype == "bf16" and w.dk == w.dv == 128 and w.chunk == 64) else 1
+                     and w.dtype == "bf16" and w.dk == w.dv == 128 and w.chunk in (64, 128)) else 1
     res = {"w": w, "ms_per_step": ms_total / args.steps, "ms_kernel": ms_kernel,
            "clocks": clk.summary(), "launches": args.steps * per_call,
            "launches_per_call": per_call}
@@ -351,7 +359,7 @@ def bench_e2e(ctx, args, gdr, w, inp, names, step, o):
 def bench_decode(ctx, args, gdr):
     """Decode step on the resident 1 GiB state, inputs cycled from 8 seeded steps."""
     torch = ctx.torch
-    dw = DEC
+    dw = DEC if args.dec_batch is None else DEC.with_(B=args.dec_batch)
     S = torch.from_numpy(synth.decode_state(dw, seed=dw.seed + 1000 * ctx.rank)).to(ctx.dev)
     names = ("q", "k", "v", "log_w", "e1", "e2")
     pool = [gdr.to_device({k: p[k] for k in names}, "bf16", ctx.dev)
@@ -382,7 +390,9 @@ def bench_decode(ctx, args, gdr):
             "dv": dw.dv, "steps": args.decode_steps, "steps_per_s": 1e3 / ms,
             "ms_per_step": ms,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"], "traffic": None,
+                         "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],
+                         "traffic": (DEC_TRAFFIC_PER_HEAD * dw.B * dw.H
+                                     if dw.dk == dw.dv == 128 and dw.form != "rwkv7" else None),
                          "bytes_per_launch": nbytes, "peak_source": ctx.peaks["source"]},
             "gpu_launches": args.decode_steps, "clocks": clk.summary()}
 
@@ -397,6 +407,11 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=15.0)
+    ap.add_argument("--fwd-batch", type=int, default=None,
+                    help="forward batch B (default: the workload's); smaller values make "
+                         "profiler captures cheaper and are not bench results")
+    ap.add_argument("--dec-batch", type=int, default=None,
+                    help="decode batch B (default: the workload's); for profiler captures")
     ap.add_argument("--only", default="all", choices=["all", "forward", "decode"],
                     help="time one part only (profiling runs); the default line needs 'all'")
     args = ap.parse_args()
@@ -443,7 +458,9 @@ def main():
                        "l2": f"inputs larger than L2 ({nbytes / 2**20:.0f} MiB per step > 126 MiB)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": ctx.peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / ctx.peaks["hbm_gbs"],
-                         "traffic": None, "peak_source": ctx.peaks["source"],
+                         "traffic": (FWD_TC_TRAFFIC_PER_CHUNK * w.B * w.H * -(-w.T // 64)
+                                     if fwd["launches_per_call"] == 2 else None),
+                         "peak_source": ctx.peaks["source"],
                          "bytes_per_launch": nbytes, "kernel_ms": fwd["ms_kernel"],
                          "scope": "one forward call (%d kernel launch%s)" % (
                              fwd["launches_per_call"],

@@ -102,7 +102,10 @@ typedef struct {
   int B, H, T, dk, dv;  /* B, H, T >= 0 (zero sizes are a no-op apart from S_T = S0);
                            dk, dv in {16, 32, 64, 128}                                  */
   int chunk;            /* chunk length C of the chunkwise form: 16, 32, 64 or 128.
-                           T need not be a multiple of C (the last chunk is partial).   */
+                           T need not be a multiple of C (the last chunk is partial).
+                           The kernels may split a chunk further: the fp32 kernel uses
+                           min(C, 64, 4096 / dk), the tensor-core kernels 64 for C >= 64.
+                           The result depends on the chunk length only through rounding. */
   gdr_algo algo;
   const void *q, *k, *v;
   const float *log_w;   /* log of the decay, must be <= 0 (decay w = exp(log_w) in (0,1]) */

@@ -503,9 +503,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
 
 }  // namespace
 
+// The tensor-core kernels evaluate the chunkwise form with C = 64; a requested chunk
+// of 128 is served with two 64-token chunks (the result depends on the chunk length
+// only through rounding).  Smaller requested chunks go to the fp32 kernel.
 bool forward_tc_supported(const FwdParams &p, gdr_dtype dtype) {
   return p.form == GDR_FORM_GDN2 && dtype == GDR_BF16 && p.dk == kDK && p.dv == kDK &&
-         p.chunk == kC;
+         (p.chunk == kC || p.chunk == 2 * kC);
 }
 
 cudaError_t launch_forward_tc(const FwdParams &p, cudaStream_t stream) {

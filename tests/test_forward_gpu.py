@@ -147,6 +147,19 @@ def test_tc_kernel_gdn2(T, with_state, path):
 
 
 @pytest.mark.parametrize("path", sorted(TC_PATHS))
+def test_tc_kernel_serves_chunk_128(path):
+    """A requested chunk of 128 runs on the tensor-core kernels as two 64-token chunks."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=300, B=1, H=2, chunk=128)
+    inp = synth.forward_inputs(w)
+    o, S = gpu_forward(w, inp, algo="tc", workspace_bytes=TC_PATHS[path])
+    o_ref, S_ref = oracle_forward(w, inp)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+    o64, S64 = gpu_forward(w.with_(chunk=64), inp, algo="tc", workspace_bytes=TC_PATHS[path])
+    assert np.array_equal(o, o64) and np.array_equal(S, S64)
+
+
+@pytest.mark.parametrize("path", sorted(TC_PATHS))
 def test_tc_full_size_gdn2(path):
     w = synth.PRESETS["gdn2_bf16"]
     inp = synth.forward_inputs(w)
