@@ -62,6 +62,10 @@ bool uses_tc(const gdr_fwd_args *a, const gdr::FwdParams &p) {
   return (a->algo == GDR_ALGO_TC || a->algo == GDR_ALGO_AUTO) &&
          gdr::forward_tc_supported(p, a->dtype);
 }
+bool uses_tc_general(const gdr_fwd_args *a, const gdr::FwdParams &p) {
+  return (a->algo == GDR_ALGO_TC || a->algo == GDR_ALGO_AUTO) &&
+         gdr::forward_tc_general_supported(p, a->dtype);
+}
 
 }  // namespace
 
@@ -129,6 +133,10 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
   }
 
   const gdr::FwdParams p = fwd_params(a);
+  if (uses_tc_general(a, p)) {   // two-stream forms, d = 64: one fused kernel, status word only
+    if (!a->workspace || a->workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
+    return cuda_status(gdr::launch_forward_tc_general(p, s));
+  }
   const bool tc_ok = gdr::forward_tc_supported(p, a->dtype);
   if (a->algo == GDR_ALGO_TC || (a->algo == GDR_ALGO_AUTO && tc_ok)) {
     if (!tc_ok) return GDR_ERR_UNSUPPORTED;

@@ -64,6 +64,10 @@ cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_
 bool forward_fp32_supported(int dk, int dv);
 cudaError_t launch_forward_tc(const FwdParams &p, cudaStream_t stream);
 bool forward_tc_supported(const FwdParams &p, gdr_dtype dtype);
+// Tensor-core path for the two-stream forms (general, RWKV-7), d_k = d_v = 64: one
+// fused kernel per (b, h); needs only the status word as workspace.
+bool forward_tc_general_supported(const FwdParams &p, gdr_dtype dtype);
+cudaError_t launch_forward_tc_general(const FwdParams &p, cudaStream_t stream);
 // Two-kernel tensor-core path: per-chunk records in the workspace.
 size_t forward_tc_split_workspace_bytes(const FwdParams &p);
 cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStream_t stream);
