@@ -83,8 +83,12 @@ typedef enum {
 typedef enum {
   GDR_ALGO_AUTO = 0,   /* tensor-core kernel where it applies, else the fp32 kernel        */
   GDR_ALGO_FP32 = 1,   /* fp32 CUDA-core kernel: every product in fp32 (all forms, all dtypes) */
-  GDR_ALGO_TC = 2      /* tcgen05/TMEM kernel: bf16 operands, fp32 accumulate and state;
-                          GDR_ERR_UNSUPPORTED where it does not apply                       */
+  GDR_ALGO_TC = 2      /* tcgen05/TMEM kernels: bf16 operands, fp32 accumulate and state.
+                          They apply to bf16 inputs with chunk >= 64 for
+                            GDN2, dk = dv = 128 (two kernels with a per-chunk record
+                                 workspace, or one kernel with the status word only), and
+                            GENERAL / RWKV7, dk = dv = 64 (one kernel, status word only);
+                          GDR_ERR_UNSUPPORTED elsewhere.                                  */
 } gdr_algo;
 
 /*
