@@ -42,9 +42,14 @@ L2_BYTES = 126 * 2 ** 20
 
 
 def fwd_algorithmic_bytes(w) -> int:
-    """q, k, v, erase gate, write gate (bf16), log_w (fp32) in; o (fp32) and S_T out."""
+    """Token inputs in (q, k, v and the form's erase arguments at the input dtype, log_w
+    fp32), o (fp32) and S_T out."""
     eb = 2 if w.dtype == "bf16" else 4
-    per_token_head = eb * (3 * w.dk + w.dv + w.dv) + 4 * w.dk + 4 * w.dv
+    extra = {"gdn2": w.dk + w.dv,        # erase gate b, write gate wg
+             "rwkv7": w.dk + 1,          # removal direction a, coefficient c
+             "general": 2 * w.dk,        # u, z
+             "gla": 0}[w.form]
+    per_token_head = eb * (2 * w.dk + w.dv + extra) + 4 * w.dk + 4 * w.dv
     return w.B * w.T * w.H * per_token_head + w.B * w.H * w.dk * w.dv * 4
 
 
@@ -264,7 +269,9 @@ class Ctx:
 def bench_forward(ctx, args, gdr):
     """Device-resident chunked forward: K timed steps, kernel time per launch."""
     torch = ctx.torch
-    w = FWD if args.fwd_batch is None else FWD.with_(B=args.fwd_batch)
+    w = FWD if args.fwd_workload is None else synth.PRESETS[args.fwd_workload]
+    if args.fwd_batch is not None:
+        w = w.with_(B=args.fwd_batch)
     inp = synth.forward_inputs(w, seed=w.seed + 1000 * ctx.rank)
     names = ("q", "k", "v", "log_w", "e1", "e2")
     d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
@@ -318,6 +325,52 @@ def bench_forward(ctx, args, gdr):
     if args.only == "all":
         res["e2e"] = bench_e2e(ctx, args, gdr, w, inp, names, step, o)
     return res
+
+
+def bench_other_workloads(ctx, args, gdr):
+    """The other forward workloads, device-resident, through the same call (algo auto):
+    milliseconds per call and the HBM roofline fraction of their algorithmic bytes."""
+    torch = ctx.torch
+    out = []
+    for name in ("rwkv7_bf16", "gdn2_long", "rwkv7_f32"):
+        w = synth.PRESETS[name]
+        inp = synth.forward_inputs(w, seed=w.seed + 1000 * ctx.rank)
+        names = ("q", "k", "v", "log_w", "e1", "e2")
+        d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
+        del inp
+        ws = gdr.new_workspace(gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"],
+                                                              d["log_w"], d["e1"], d["e2"],
+                                                              w.chunk, args.algo), ctx.dev)
+
+        def call():
+            return gdr.gdr_forward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
+                                           d["e2"], None, chunk=w.chunk, algo=args.algo,
+                                           workspace=ws)
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = ctx.event(), ctx.event()
+        n = 5
+        e0.record(ctx.stream)
+        for _ in range(n):
+            call()
+        e1.record(ctx.stream)
+        torch.cuda.synchronize()
+        status = gdr.gdr_read_status(ws)
+        if status != "GDR_OK":
+            raise RuntimeError(f"device status after {name}: {status}")
+        ms = ctx.max_over_ranks(e0.elapsed_time(e1)) / n
+        nbytes = fwd_algorithmic_bytes(w)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.append({"workload": name, "form": w.form, "dtype": w.dtype, "B": w.B, "H": w.H,
+                    "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "ms_per_call": ms,
+                    "tokens_per_s": w.tokens * ctx.world / (ms * 1e-3),
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
+                                 "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],
+                                 "bytes_per_call": nbytes}})
+        del d, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def bench_e2e(ctx, args, gdr, w, inp, names, step, o):
@@ -407,11 +460,15 @@ def main():
     ap.add_argument("--decode-steps", type=int, default=50)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=15.0)
+    ap.add_argument("--fwd-workload", default=None, choices=sorted(synth.PRESETS),
+                    help="forward workload (default: the GDN-2 headline); for profiler captures")
     ap.add_argument("--fwd-batch", type=int, default=None,
                     help="forward batch B (default: the workload's); smaller values make "
                          "profiler captures cheaper and are not bench results")
     ap.add_argument("--dec-batch", type=int, default=None,
                     help="decode batch B (default: the workload's); for profiler captures")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the timing of the other forward workloads")
     ap.add_argument("--only", default="all", choices=["all", "forward", "decode"],
                     help="time one part only (profiling runs); the default line needs 'all'")
     args = ap.parse_args()
@@ -477,6 +534,8 @@ def main():
                                     "kind": "oracle", "sample": sample}
     if dec is not None:
         line["decode"] = dec
+    if args.only == "all" and not args.no_other_workloads:
+        line["other_workloads"] = bench_other_workloads(ctx, args, gdr)
     print(json.dumps(line), flush=True)
     return 0
 
