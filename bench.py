@@ -75,6 +75,11 @@ def dec_algorithmic_bytes(w) -> int:
     return state + tok
 
 
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own shard of sequences (weak scaling, no collective)."""
+    return base + 1000 * rank
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -240,16 +245,19 @@ def run_reference(args):
 class Ctx:
     """Device, stream and the rank plumbing (barrier, max over ranks)."""
 
-    def __init__(self, torch, dist, world, rank, local):
+    def __init__(self, torch, dist, world, rank, local, device=None):
         self.torch, self.dist = torch, dist
         self.world, self.rank, self.local = world, rank, local
-        self.dev = torch.device("cuda", local)
-        self.stream = torch.cuda.current_stream()
+        # the rank plumbing also runs on the host (gloo) for the multi-process tests
+        self.dev = device if device is not None else torch.device("cuda", local)
+        self.stream = torch.cuda.current_stream() if self.dev.type == "cuda" else None
         self.peaks = load_peaks()
-        try:
-            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
-        except Exception:
-            self.uuid = str(local)
+        self.uuid = str(local)
+        if self.dev.type == "cuda":
+            try:
+                self.uuid = "GPU-" + str(torch.cuda.get_device_properties(self.dev).uuid)
+            except Exception:
+                pass
 
     def barrier(self):
         if self.world > 1:
@@ -272,7 +280,7 @@ def bench_forward(ctx, args, gdr):
     w = FWD if args.fwd_workload is None else synth.PRESETS[args.fwd_workload]
     if args.fwd_batch is not None:
         w = w.with_(B=args.fwd_batch)
-    inp = synth.forward_inputs(w, seed=w.seed + 1000 * ctx.rank)
+    inp = synth.forward_inputs(w, seed=rank_seed(w.seed, ctx.rank))
     names = ("q", "k", "v", "log_w", "e1", "e2")
     d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
     o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=ctx.dev)
@@ -334,7 +342,7 @@ def bench_other_workloads(ctx, args, gdr):
     out = []
     for name in ("rwkv7_bf16", "gdn2_long", "rwkv7_f32"):
         w = synth.PRESETS[name]
-        inp = synth.forward_inputs(w, seed=w.seed + 1000 * ctx.rank)
+        inp = synth.forward_inputs(w, seed=rank_seed(w.seed, ctx.rank))
         names = ("q", "k", "v", "log_w", "e1", "e2")
         d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
         del inp
@@ -413,10 +421,10 @@ def bench_decode(ctx, args, gdr):
     """Decode step on the resident 1 GiB state, inputs cycled from 8 seeded steps."""
     torch = ctx.torch
     dw = DEC if args.dec_batch is None else DEC.with_(B=args.dec_batch)
-    S = torch.from_numpy(synth.decode_state(dw, seed=dw.seed + 1000 * ctx.rank)).to(ctx.dev)
+    S = torch.from_numpy(synth.decode_state(dw, seed=rank_seed(dw.seed, ctx.rank))).to(ctx.dev)
     names = ("q", "k", "v", "log_w", "e1", "e2")
     pool = [gdr.to_device({k: p[k] for k in names}, "bf16", ctx.dev)
-            for p in (synth.decode_step_inputs(dw, s, seed=dw.seed + 1000 * ctx.rank)
+            for p in (synth.decode_step_inputs(dw, s, seed=rank_seed(dw.seed, ctx.rank))
                       for s in range(8))]
     o_dec = torch.empty((dw.B, dw.H, dw.dv), dtype=torch.float32, device=ctx.dev)
 
