@@ -48,6 +48,10 @@
  * Kernels that wait on an mbarrier bound each wait; a wait that runs out writes
  * GDR_ERR_TIMEOUT into the caller's workspace status word, which
  * gdr_read_status() returns.  No function aborts, exits or traps.
+ * For tests of that path, the environment variable GDR_DEBUG_FAULT=skip_handoff
+ * makes the two-kernel tensor-core forward withhold a hand-off between its warp
+ * groups, so a bounded wait runs out (about 2 s) and GDR_ERR_TIMEOUT is reported;
+ * the context stays usable.
  */
 #ifndef GDR_H_
 #define GDR_H_

@@ -1,6 +1,7 @@
 // gdr_api.cu -- the extern "C" entry points of libgdr: argument validation,
 // kernel selection and launch.  Declarations and the contract: include/gdr.h.
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 
 #include "gdr_internal.cuh"
@@ -55,6 +56,8 @@ gdr::FwdParams fwd_params(const gdr_fwd_args *a) {
   p.o = a->o;
   p.S_T = a->S_T;
   p.status = static_cast<uint32_t *>(a->workspace);
+  const char *fault = getenv("GDR_DEBUG_FAULT");
+  p.debug = (fault && strcmp(fault, "skip_handoff") == 0) ? gdr::kDebugSkipHandoff : 0u;
   return p;
 }
 

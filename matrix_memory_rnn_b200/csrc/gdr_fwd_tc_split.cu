@@ -486,7 +486,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         mma_commit_warp(bar1 + bi);
         if (lane == 0) cnt[kM1Iss0 + bi] += 1;
       }
-      if (poller) mbar_arrive(ready + bi);                 // hand the chunk to the back group
+      // hand the chunk to the back group (the fault-injection hook withholds it)
+      if (poller && !(p.debug & kDebugSkipHandoff)) mbar_arrive(ready + bi);
       GDR_PREP_PHASE(4);
     }
   } else {

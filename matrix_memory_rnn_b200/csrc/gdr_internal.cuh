@@ -56,7 +56,13 @@ struct FwdParams {
   float *o;
   float *S_T;
   uint32_t *status;  // device status word (workspace), may be null
+  uint32_t debug;    // fault-injection bits (kDebug...), 0 in normal use
 };
+
+// Fault injection for the tests of the bounded waits (set through the environment
+// variable GDR_DEBUG_FAULT, read per call on the host): the prep kernel's front warp
+// group never hands its chunks to the back group, whose bounded wait then runs out.
+constexpr uint32_t kDebugSkipHandoff = 1u;
 
 // Launchers (host).  Return cudaSuccess or the launch error.
 cudaError_t launch_decode(const gdr_step_args &a, cudaStream_t stream);

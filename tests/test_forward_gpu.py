@@ -226,3 +226,26 @@ def test_tc_rejects_what_it_does_not_cover():
     with pytest.raises(gdr.GdrError) as ei:
         gpu_forward(w, inp, algo="tc")
     assert ei.value.code == 2
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(monkeypatch):
+    """Fault injection on the host: the prep kernel's front group withholds its hand-off,
+    the back group's bounded wait runs out, the call reports GDR_ERR_TIMEOUT through the
+    workspace status word, and the next call on the same context is correct."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=192, B=1, H=2, chunk=64)
+    inp = synth.forward_inputs(w)
+    d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "bf16")
+    ws = gdr.new_workspace(gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"],
+                                                          d["log_w"], d["e1"], d["e2"], 64,
+                                                          "tc"), "cuda")
+    monkeypatch.setenv("GDR_DEBUG_FAULT", "skip_handoff")
+    gdr.gdr_forward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"], d["e2"],
+                            None, chunk=64, algo="tc", workspace=ws)
+    assert gdr.gdr_read_status(ws) == "GDR_ERR_TIMEOUT"
+    monkeypatch.delenv("GDR_DEBUG_FAULT")
+    o, S = gdr.gdr_forward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
+                                   d["e2"], None, chunk=64, algo="tc", workspace=ws)
+    assert gdr.gdr_read_status(ws) == "GDR_OK"
+    o_ref, S_ref = oracle_forward(w, inp)
+    assert head_rel_err(o.cpu().numpy(), o_ref, (0, 2)) < TOL["bf16"]
+    assert head_rel_err(S.cpu().numpy(), S_ref, (0, 1)) < TOL["bf16"]
