@@ -21,7 +21,8 @@
 // M_k V.
 //
 // One CTA of 256 threads per (b, h) walks its chunks in order (fused: the
-// sequences are many and short in the workloads this serves).  Per chunk, five
+// sequences are many and short in the workloads this serves); shared-memory
+// slots are reused across the chunk's phases so that two CTAs share an SM.  Per chunk, five
 // tcgen05 MMA groups with bf16 operands in 128-byte-swizzled shared memory and
 // fp32 accumulators in TMEM, CUDA-core phases in between:
 //   MMA1   [U f'; Q f] (M = 128) x [Z g; K g]^T (N = 128), K = d_k   -> A, B, M_z, M_k
@@ -50,38 +51,47 @@ constexpr int kD = 64;                      // d_k = d_v
 constexpr int kGT = 256;                    // threads per CTA
 constexpr uint32_t kTile = kC * kD * 2;     // one 64 x 64 bf16 tile in the sw128 layout (8 KB)
 
-// Shared memory (bytes from a 1024-aligned base).  All bf16 tiles are 64 rows of
-// 128 B in the sw128 layout (rows = tokens unless stated).
+// Shared memory: thirteen 8 KB slots (bf16 64 x 64 tiles in the sw128 layout, rows =
+// tokens unless stated) from a 1024-aligned base, reused as the chunk goes on, so two
+// CTAs fit on an SM:
+//   slot 0      v (TMA)                                   -> next chunk's v after MMA3
+//   slot 1      S0' [j][c], bf16 copy of the state (B operand of MMA3)
+//   slot 2      U_pi                        } B operand of MMA2: two atoms, U_pi first
+//   slot 3      K~ [s][j] (MN-major A; slot 4 is its junk atom)
+//   slot 4      Z~ [s][j] (MN-major A; slot 5 is its junk atom)
+//   slots 5-6   u | q (TMA) -> [U f'; Q f] in place (MMA1 A) -> fp32 T^-1 (or, on the
+//               exact path, Lam first) -> -W (5), V~ (6)
+//   slots 7-8   z | k (TMA) -> [Z g; K g] in place (MMA1 B) -> fp32 A -> bf16 T^-1 (7),
+//               B V (8)                     } second atom of MMA2's B operand
+//   slots 9-10  log w (TMA, fp32 row-major) -> Lam - Lam_0 -> M_k (9), M_z (10)
+//   slots 11-12 [Q_pi; B] -> [Q_pi; Y_u] (MMA3 A)
 struct GenSmem {
-  static constexpr uint32_t V = 0;                 // input v [s][c]; B operand (MN-major)
-  static constexpr uint32_t Q = V + kTile;         // input q
-  static constexpr uint32_t K = Q + kTile;         // input k
-  static constexpr uint32_t E1 = K + kTile;        // input u (general) / a (RWKV-7)
-  static constexpr uint32_t E2 = E1 + kTile;       // input z (general)
-  static constexpr uint32_t LW = E2 + kTile;       // log w, row-major fp32 (16 KB); then Lam_t - Lam_0
-  static constexpr uint32_t A1 = LW + 2 * kTile;   // [U f'; Q f] 128 x 64 (K-major A); then fp32 T^-1
-  static constexpr uint32_t B1 = A1 + 2 * kTile;   // [Z g; K g] 128 x 64 (K-major B); then fp32 A;
-                                                   //   then bf16 T^-1 (first 8 KB)
-  static constexpr uint32_t QY = B1 + 2 * kTile;   // [Q_pi; Y_u] 128 x 64 (K-major A of MMA3)
-  static constexpr uint32_t UP = QY + 2 * kTile;   // U_pi   } MMA2 B operand, two atoms
-  static constexpr uint32_t BV = UP + kTile;       // B V    } 8 KB apart
-  static constexpr uint32_t KT = BV + kTile;       // K~ [s][j] (MN-major A; next tile = junk atom)
-  static constexpr uint32_t ZT = KT + kTile;       // Z~ [s][j] (MN-major A; next tile = junk atom)
-  static constexpr uint32_t BB = ZT + kTile;       // B [t][s] (K-major A of B V)
-  static constexpr uint32_t MK = BB + kTile;       // M_k [t][s] (K-major; next tile = junk rows)
-  static constexpr uint32_t MZ = MK + kTile;       // M_z [t][s] (K-major; next tile = junk rows)
-  static constexpr uint32_t UW = MZ + kTile;       // -W [t][c]
-  static constexpr uint32_t VT = UW + kTile;       // V~ [t][c] (B operand of MMA4)
-  static constexpr uint32_t S0B = VT + kTile;      // S0' [j][c] (B operand of MMA3, MN-major)
-  static constexpr uint32_t PI = S0B + kTile;      // fp32 pi_C per channel
+  static constexpr uint32_t V = 0 * kTile;
+  static constexpr uint32_t S0B = 1 * kTile;
+  static constexpr uint32_t UP = 2 * kTile;
+  static constexpr uint32_t KT = 3 * kTile;
+  static constexpr uint32_t ZT = 4 * kTile;
+  static constexpr uint32_t A1 = 5 * kTile;        // [U f'; Q f]: u lands in the first half, q in the second
+  static constexpr uint32_t B1 = 7 * kTile;        // [Z g; K g]: z lands in the first half, k in the second
+  static constexpr uint32_t LW = 9 * kTile;        // log w (16 KB)
+  static constexpr uint32_t QY = 11 * kTile;       // [Q_pi; B then Y_u]
+  static constexpr uint32_t UW = A1;               // -W
+  static constexpr uint32_t VT = A1 + kTile;       // V~ (B operand of MMA4)
+  static constexpr uint32_t TI = B1;               // bf16 T^-1 (A operand of MMA2)
+  static constexpr uint32_t BV = B1 + kTile;       // B V
+  static constexpr uint32_t MK = LW;               // M_k [t][s] (K-major; M_z is its junk rows)
+  static constexpr uint32_t MZ = LW + kTile;       // M_z [t][s] (K-major; Q_pi is its junk rows)
+  static constexpr uint32_t BB = QY + kTile;       // B [t][s] (K-major A of B V)
+  static constexpr uint32_t PI = 13 * kTile;       // fp32 pi_C per channel
   static constexpr uint32_t A1V = PI + kD * 4;     // fp32 alpha_0 = e^{Lam_0} per channel
   static constexpr uint32_t DN = A1V + kD * 4;     // fp32 Lam_63 - Lam_0 per channel
   static constexpr uint32_t QT = DN + kD * 4;      // fp32 [4][d] quarter sums of log w
   static constexpr uint32_t CS = QT + 4 * kD * 4;  // fp32 RWKV-7 c per token
   static constexpr uint32_t MISC = CS + kC * 4;    // barriers, TMEM slot, flags
   static constexpr uint32_t ALLOC = MISC + 128 + 1024;
-  static_assert(ALLOC <= 227 * 1024, "shared memory");
+  static_assert(ALLOC <= 113 * 1024, "two CTAs per SM");
   static_assert(Ix::kBytes <= 2 * kTile, "fp32 64 x 64 must fit a 16 KB region");
+  static_assert(BV > UP, "MMA2's B operand: the B V atom follows the U_pi atom");
 };
 
 struct GenMisc {
@@ -107,10 +117,10 @@ __device__ __forceinline__ void load_in1(uint8_t *smem, const GenMaps &m, uint64
                                          int t0) {
   using SL = GenSmem;
   mbar_arrive_expect_tx(bar, (kRwkv ? 3u : 4u) * kTile + kC * kD * 4u);
-  tma_load_4d(smem + SL::Q, &m.q, 0, h, t0, b, bar);
-  tma_load_4d(smem + SL::K, &m.k, 0, h, t0, b, bar);
-  tma_load_4d(smem + SL::E1, &m.e1, 0, h, t0, b, bar);
-  if (!kRwkv) tma_load_4d(smem + SL::E2, &m.e2, 0, h, t0, b, bar);
+  tma_load_4d(smem + SL::A1, &m.e1, 0, h, t0, b, bar);
+  tma_load_4d(smem + SL::A1 + kTile, &m.q, 0, h, t0, b, bar);
+  if (!kRwkv) tma_load_4d(smem + SL::B1, &m.e2, 0, h, t0, b, bar);
+  tma_load_4d(smem + SL::B1 + kTile, &m.k, 0, h, t0, b, bar);
   tma_load_4d(smem + SL::LW, &m.lw, 0, h, t0, b, bar);
 }
 
@@ -120,13 +130,48 @@ __device__ __forceinline__ void load_in2(uint8_t *smem, const GenMaps &m, uint64
   tma_load_4d(smem + GenSmem::V, &m.v, 0, h, t0, b, bar);
 }
 
-// Thread 0 polls the MMA barrier (bounded), then the CTA meets.
-__device__ __forceinline__ bool gen_wait(uint64_t *bar, uint32_t &phase, volatile int *abort) {
-  return wait_mma(bar, phase, abort);
+// Cumulative log-decay of one chunk, Lam_t - Lam_0 in place in `lw` (row-major
+// [t][d] fp32; rows past the sequence are zero).  Thread = (channel, token quarter).
+// Also per channel: alpha_0 = e^{Lam_0}, dn = Lam_63 - Lam_0, pi_C = e^{Lam_63}, and
+// the exact-path flag when dn < -80.  Ends with a CTA barrier.
+__device__ __forceinline__ void chunk_scan(float *lw, float *sQT, float *sA1, float *sDN,
+                                           float *sPI, volatile int *sexact, int tid) {
+  const int ch = tid & (kD - 1), qt = tid >> 6;
+  float x[16];
+  float acc = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    acc += lw[(16 * qt + i) * kD + ch];
+    x[i] = acc;
+  }
+  sQT[qt * kD + ch] = acc;
+  __syncthreads();
+  float excl = 0.f, all = 0.f;
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const float v = sQT[q4 * kD + ch];
+    all += v;
+    excl += (q4 < qt) ? v : 0.f;
+  }
+  if (qt == 0) sA1[ch] = x[0];             // Lam_0 (token 0), replaced by alpha_0 below
+  __syncthreads();
+  const float lam0 = sA1[ch];
+  const float shift = excl - lam0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) lw[(16 * qt + i) * kD + ch] = x[i] + shift;
+  __syncthreads();
+  if (qt == 0) {
+    const float dn = all - lam0;
+    sDN[ch] = dn;
+    sA1[ch] = __expf(lam0);
+    sPI[ch] = __expf(all);
+    if (dn < -kMaxChunkDecay) *sexact = 1;
+  }
+  __syncthreads();
 }
 
 template <bool kRwkv>
-__global__ void __launch_bounds__(kGT, 1)
+__global__ void __launch_bounds__(kGT, 2)
     tc_general_kernel(FwdParams p, const __grid_constant__ GenMaps maps) {
   using SL = GenSmem;
   extern __shared__ uint8_t smem_raw[];
@@ -154,7 +199,10 @@ __global__ void __launch_bounds__(kGT, 1)
   float *sDN = reinterpret_cast<float *>(smem + SL::DN);
   float *sQT = reinterpret_cast<float *>(smem + SL::QT);
   float *sC = reinterpret_cast<float *>(smem + SL::CS);
-  const __nv_bfloat16 *gc = static_cast<const __nv_bfloat16 *>(p.e2);   // RWKV-7 c [B][T][H]
+  const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
+  const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
+  const __nv_bfloat16 *ge1 = static_cast<const __nv_bfloat16 *>(p.e1);
+  const __nv_bfloat16 *ge2 = static_cast<const __nv_bfloat16 *>(p.e2);   // z, or RWKV-7 c [B][T][H]
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -177,7 +225,7 @@ __global__ void __launch_bounds__(kGT, 1)
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
       const int t = 2 * lane + i;
-      cnext[i] = t < T ? __bfloat162float(gc[((size_t)b * T + t) * H + h]) : 0.f;
+      cnext[i] = t < T ? __bfloat162float(ge2[((size_t)b * T + t) * H + h]) : 0.f;
     }
   }
 
@@ -228,47 +276,16 @@ __global__ void __launch_bounds__(kGT, 1)
     __syncthreads();
     if (!(ok = *sabort == 0)) break;
 
-    // ---- cumulative log-decay in place: thread = (channel ch, token quarter qt)
-    {
-      const int ch = tid & (kD - 1), qt = tid >> 6;
-      float x[16];
-      float acc = 0.f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        acc += sLW[(16 * qt + i) * kD + ch];
-        x[i] = acc;
-      }
-      sQT[qt * kD + ch] = acc;
-      __syncthreads();
-      float excl = 0.f, all = 0.f;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const float v = sQT[q4 * kD + ch];
-        all += v;
-        excl += (q4 < qt) ? v : 0.f;
-      }
-      if (qt == 0) sA1[ch] = x[0];             // Lam_0 (token 0), replaced by alpha_0 below
-      __syncthreads();
-      const float lam0 = sA1[ch];
-      const float shift = excl - lam0;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) sLW[(16 * qt + i) * kD + ch] = x[i] + shift;
-      __syncthreads();
-      if (qt == 0) {
-        const float dn = all - lam0;
-        sDN[ch] = dn;
-        sA1[ch] = __expf(lam0);
-        sPI[ch] = __expf(all);
-        if (dn < -kMaxChunkDecay) *sexact = 1;
-      }
-    }
-    __syncthreads();
+    // ---- cumulative log-decay in place (slots 9-10)
+    chunk_scan(sLW, sQT, sA1, sDN, sPI, sexact, tid);
     const bool exact = *sexact != 0;
 
-    // ---- operand tiles.  Thread = (channel group g of 8, token pair tp).
-    //      Pivot-split (MMA1): U f' (f' = e^{lam_{t-1}}, row 0 zero), Q f (f = e^{lam_t}),
-    //      Z g, K g (g = e^{-lam_s}).  Direct (<= 1): Q_pi = Q f alpha_0, U_pi = U f' alpha_0
-    //      (row 0: u_0), K~, Z~ = (k, z) e^{dn - lam_s}.  lam = Lam - Lam_0.
+    // ---- operand tiles.  Thread = (channel group g of 8, token pair tp); each input
+    //      element is read and its outputs written at the same swizzled offset, so the
+    //      pivot-split MMA1 operands replace u, q, z, k in place:
+    //        U f' (f' = e^{lam_{t-1}}, row 0 zero), Q f (f = e^{lam_t}), Z g, K g (g = e^{-lam_s});
+    //      and the direct (<= 1) tiles go to their own slots:
+    //        Q_pi = Q f alpha_0, U_pi = U f' alpha_0 (row 0: u_0), K~, Z~ = (k, z) e^{dn - lam_s}.
     {
       const int g = tid & 7, tp = tid >> 3, j0 = 8 * g;
       float dn[8], a0[8];
@@ -285,27 +302,28 @@ __global__ void __launch_bounds__(kGT, 1)
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int t = 2 * tp + i;
-        float lam[8], lamp[8];
+        const uint32_t o = sw128_offset(t, j0, kC * 128);
+        float lam[8], fp[8], q8[8], k8[8], u8[8], z8[8], x[8];
         {
           const float4 l0 = *reinterpret_cast<const float4 *>(sLW + t * kD + j0);
           const float4 l1 = *reinterpret_cast<const float4 *>(sLW + t * kD + j0 + 4);
           lam[0] = l0.x; lam[1] = l0.y; lam[2] = l0.z; lam[3] = l0.w;
           lam[4] = l1.x; lam[5] = l1.y; lam[6] = l1.z; lam[7] = l1.w;
-          if (t > 0) {
-            const float4 m0 = *reinterpret_cast<const float4 *>(sLW + (t - 1) * kD + j0);
-            const float4 m1 = *reinterpret_cast<const float4 *>(sLW + (t - 1) * kD + j0 + 4);
-            lamp[0] = m0.x; lamp[1] = m0.y; lamp[2] = m0.z; lamp[3] = m0.w;
-            lamp[4] = m1.x; lamp[5] = m1.y; lamp[6] = m1.z; lamp[7] = m1.w;
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) lamp[e] = 0.f;
-          }
         }
-        const uint32_t o = sw128_offset(t, j0, kC * 128);
-        float q8[8], k8[8], u8[8], z8[8];
-        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::Q + o), q8);
-        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::K + o), k8);
-        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::E1 + o), u8);
+        if (t > 0) {
+          const float4 m0 = *reinterpret_cast<const float4 *>(sLW + (t - 1) * kD + j0);
+          const float4 m1 = *reinterpret_cast<const float4 *>(sLW + (t - 1) * kD + j0 + 4);
+          fp[0] = m0.x; fp[1] = m0.y; fp[2] = m0.z; fp[3] = m0.w;
+          fp[4] = m1.x; fp[5] = m1.y; fp[6] = m1.z; fp[7] = m1.w;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) fp[e] = __expf(fp[e]);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) fp[e] = 0.f;
+        }
+        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::A1 + kTile + o), q8);
+        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::B1 + kTile + o), k8);
+        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::A1 + o), u8);
         if (kRwkv) {
           const float ct = sC[t];
 #pragma unroll
@@ -314,37 +332,39 @@ __global__ void __launch_bounds__(kGT, 1)
             u8[e] *= ct;          // u = c a
           }
         } else {
-          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::E2 + o), z8);
+          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::B1 + o), z8);
         }
-        float uf[8], qf[8], zg[8], kg[8], qpi[8], upi[8], kt[8], zt[8];
+        // U f' (in place over u) and U_pi
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float f = __expf(lam[e]);
-          const float fp = (t > 0) ? __expf(lamp[e]) : 0.f;
-          qf[e] = q8[e] * f;
-          uf[e] = u8[e] * fp;
-          qpi[e] = qf[e] * a0[e];
-          upi[e] = (t > 0) ? uf[e] * a0[e] : u8[e];
-          const float r = __expf(dn[e] - lam[e]);          // e^{Lam_63 - Lam_t} <= 1
-          kt[e] = k8[e] * r;
-          zt[e] = z8[e] * r;
-          if (!exact) {
-            const float gg = __expf(-lam[e]);
-            zg[e] = z8[e] * gg;
-            kg[e] = k8[e] * gg;
-          } else {             // the exact path forms A, B, M_z, M_k without the pivot split
-            zg[e] = 0.f;
-            kg[e] = 0.f;
-          }
-        }
-        st_smem16(smem, SL::A1 + o, pack8(uf));
-        st_smem16(smem, SL::A1 + kTile + o, pack8(qf));
-        st_smem16(smem, SL::B1 + o, pack8(zg));
-        st_smem16(smem, SL::B1 + kTile + o, pack8(kg));
-        st_smem16(smem, SL::QY + o, pack8(qpi));
-        st_smem16(smem, SL::UP + o, pack8(upi));
-        st_smem16(smem, SL::KT + o, pack8(kt));
-        st_smem16(smem, SL::ZT + o, pack8(zt));
+        for (int e = 0; e < 8; ++e) x[e] = u8[e] * fp[e];
+        st_smem16(smem, SL::A1 + o, pack8(x));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = (t > 0) ? x[e] * a0[e] : u8[e];
+        st_smem16(smem, SL::UP + o, pack8(x));
+        // Q f (in place over q) and Q_pi
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = q8[e] * __expf(lam[e]);
+        st_smem16(smem, SL::A1 + kTile + o, pack8(x));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] *= a0[e];
+        st_smem16(smem, SL::QY + o, pack8(x));
+        // K~, Z~ (direct) and Z g, K g (pivot split; zero on the exact path)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fp[e] = __expf(dn[e] - lam[e]);   // e^{Lam_63 - Lam_t} <= 1
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = k8[e] * fp[e];
+        st_smem16(smem, SL::KT + o, pack8(x));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = z8[e] * fp[e];
+        st_smem16(smem, SL::ZT + o, pack8(x));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fp[e] = exact ? 0.f : __expf(-lam[e]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = z8[e] * fp[e];
+        st_smem16(smem, SL::B1 + o, pack8(x));
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = k8[e] * fp[e];
+        st_smem16(smem, SL::B1 + kTile + o, pack8(x));
       }
     }
     fence_proxy_async_smem();
@@ -364,18 +384,17 @@ __global__ void __launch_bounds__(kGT, 1)
       mma_commit_warp(mbar);
       if (lane == 0) ++issued_mma;
     }
-    if (!(ok = gen_wait(mbar, phase, sabort))) break;
+    if (!(ok = wait_mma(mbar, phase, sabort))) break;
 
-    // ---- A (fp32, strictly lower -> sA over B1), B (bf16 -> BB), M_z, M_k (bf16).
-    //      Row r = 32 qd + lane: r < 64 the U rows (t = r), else the Q rows (t = r - 64);
-    //      hf = 0: the Z columns (s), hf = 1: the K columns.
+    // ---- A (fp32, strictly lower -> over the MMA1 B operand), B (bf16, below Q_pi),
+    //      M_k, M_z (bf16, over log w).  Row r = 32 qd + lane: r < 64 the U rows
+    //      (t = r), else the Q rows (t = r - 64); hf = 0: the Z columns, 1: the K columns.
     if (!exact) {
       const int r = 32 * qd + lane, t = r & 63;
       float x[32], y[32];
       tmem_ld_32x32b_x32(tmem + kT_D1 + lane_q + 64 * hf, x);
       tmem_ld_32x32b_x32(tmem + kT_D1 + lane_q + 64 * hf + 32, y);
       tmem_ld_wait();
-      __syncthreads();        // every thread has read B1 (MMA1 is done with it): sA may land
       const bool urow = r < kC;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -397,28 +416,51 @@ __global__ void __launch_bounds__(kGT, 1)
         }
       }
     } else {
-      __syncthreads();
-      // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound)
+      // exact pairwise decays (a chunk whose log-decay exceeds the pivot bound): Lam
+      // again from global log w into the dead MMA1 A operand, inputs from global
+      float *lam = sTi;
+      {
+        const int ch = tid & (kD - 1), qt = tid >> 6;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int t = 16 * qt + i;
+          lam[t * kD + ch] = t < n ? __ldg(p.log_w + (((size_t)b * T + t0 + t) * H + h) * kD + ch) : 0.f;
+        }
+        __syncthreads();
+        float x[16];
+        float acc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          acc += lam[(16 * qt + i) * kD + ch];
+          x[i] = acc;
+        }
+        sQT[qt * kD + ch] = acc;
+        __syncthreads();
+        float excl = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) excl += (q4 < qt) ? sQT[q4 * kD + ch] : 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) lam[(16 * qt + i) * kD + ch] = x[i] + excl;   // Lam_t
+        __syncthreads();
+      }
+      auto tok = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kD; };
       for (int it = tid; it < kC * kC; it += kGT) {
         const int t = it / kC, s = it % kC;
         float av = 0.f, bv = 0.f, mz = 0.f, mk = 0.f;
         if (s <= t && t < n) {
+          const size_t ot = tok(t), os = tok(s);
+          const float ct = kRwkv ? sC[t] : 1.f;
           for (int j = 0; j < kD; ++j) {
-            const uint32_t ot = sw128_offset(t, j, kC * 128), os = sw128_offset(s, j, kC * 128);
-            const float ls = sLW[s * kD + j], lt = sLW[t * kD + j];
-            const float zs = kRwkv ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(smem + SL::E1 + os))
-                                   : __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(smem + SL::E2 + os));
-            const float ks = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(smem + SL::K + os));
-            const float qt = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(smem + SL::Q + ot));
-            const float dq = __expf(lt - ls);
-            mz += qt * dq * zs;
-            mk += qt * dq * ks;
+            const float ls = lam[s * kD + j], lt = lam[t * kD + j];
+            const float zs = kRwkv ? __bfloat162float(ge1[os + j]) : __bfloat162float(ge2[os + j]);
+            const float ks = __bfloat162float(gk[os + j]);
+            const float dq = __expf(lt - ls) * __bfloat162float(gq[ot + j]);
+            mz += dq * zs;
+            mk += dq * ks;
             if (s < t) {
-              float ut = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(smem + SL::E1 + ot));
-              if (kRwkv) ut *= sC[t];
-              const float du = __expf(sLW[(t - 1) * kD + j] - ls);
-              av += ut * du * zs;
-              bv += ut * du * ks;
+              const float du = __expf(lam[(t - 1) * kD + j] - ls) * __bfloat162float(ge1[ot + j]) * ct;
+              av += du * zs;
+              bv += du * ks;
             }
           }
         }
@@ -431,23 +473,17 @@ __global__ void __launch_bounds__(kGT, 1)
             __float2bfloat16_rn(mk);
       }
     }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- the inputs q, k, e1, e2, log w are consumed: load the next chunk's
-    if (tid == 0 && c + 1 < nch) {
-      fence_proxy_async_smem();
-      load_in1<kRwkv>(smem, maps, in1, b, h, t0 + kC);
-      ++in1_iss;
-    }
     if (kRwkv && warp == 0 && c + 1 < nch) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int t = t0 + kC + 2 * lane + i;
-        cnext[i] = t < T ? __bfloat162float(gc[((size_t)b * T + t) * H + h]) : 0.f;
+        cnext[i] = t < T ? __bfloat162float(ge2[((size_t)b * T + t) * H + h]) : 0.f;
       }
     }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
     // ---- MMA-BV: B V (M = 64) -> TMEM; state accumulator = K~^T V ([K~ | *], M = 128).
     //      They run while T^-1 is formed.
     if (warp == 0) {
@@ -465,7 +501,7 @@ __global__ void __launch_bounds__(kGT, 1)
       mma_commit_warp(mbar);
       if (lane == 0) ++issued_mma;
     }
-    // ---- T^-1 (fp32 into the dead A1), bf16 copy (into the first half of the dead B1)
+    // ---- T^-1 (fp32 over the dead MMA1 A operand), bf16 copy over the dead fp32 A
     invert_diag_blocks8<Ix, Ix, kGT>(sA, sTi, tid);
     invert_merge_levels<Ix, Ix, kGT>(sA, sTi, tid);
 #pragma unroll
@@ -479,9 +515,9 @@ __global__ void __launch_bounds__(kGT, 1)
         const int s = 8 * gg + e;
         x[e] = (s < t) ? x[e] : (s == t ? 1.f : 0.f);
       }
-      st_smem16(smem, SL::B1 + sw128_offset(t, 8 * gg, kC * 128), pack8(x));
+      st_smem16(smem, SL::TI + sw128_offset(t, 8 * gg, kC * 128), pack8(x));
     }
-    if (!(ok = gen_wait(mbar, phase, sabort))) break;    // B V and K~^T V
+    if (!(ok = wait_mma(mbar, phase, sabort))) break;    // B V and K~^T V
 
     // ---- B V (M = 64 accumulator: row 16 qd + r at lane 32 qd + r) -> bf16 tile
     if (hf == 0) {
@@ -502,16 +538,16 @@ __global__ void __launch_bounds__(kGT, 1)
       constexpr uint32_t id = idesc_bf16_f32(64, 128, false, true);
 #pragma unroll
       for (int s = 0; s < kC / 16; ++s) {
-        const uint64_t ad = sdesc_sw128(sb + SL::B1 + s * 32, 16, 1024);
-        const uint64_t bd = sdesc_sw128(sb + SL::UP + s * 2048, kTile, 1024);
+        const uint64_t ad = sdesc_sw128(sb + SL::TI + s * 32, 16, 1024);
+        const uint64_t bd = sdesc_sw128(sb + SL::UP + s * 2048, SL::BV - SL::UP, 1024);
         mma_bf16_warp(tmem + kT_M2, ad, bd, id, s > 0);
       }
       mma_commit_warp(mbar);
       if (lane == 0) ++issued_mma;
     }
-    if (!(ok = gen_wait(mbar, phase, sabort))) break;
+    if (!(ok = wait_mma(mbar, phase, sabort))) break;
 
-    // ---- Y_u -> rows 64..127 of [Q_pi; Y_u]; -W -> UW.  hf 0: Y_u columns, 1: W columns
+    // ---- Y_u -> rows 64..127 of [Q_pi; Y_u]; -W -> its tile.  hf 0: Y_u columns, 1: W columns
     {
       float x[32];
       tmem_ld_16x32bx2_x32_split32(tmem + kT_M2 + lane_q + 64 * hf, x);
@@ -552,7 +588,13 @@ __global__ void __launch_bounds__(kGT, 1)
       mma_commit_warp(mbar);
       if (lane == 0) ++issued_mma;
     }
-    if (!(ok = gen_wait(mbar, phase, sabort))) break;
+    if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    // ---- v is consumed: load the next chunk's
+    if (tid == 0 && c + 1 < nch) {
+      fence_proxy_async_smem();
+      load_in2(smem, maps, in2, b, h, t0 + kC);
+      ++in2_iss;
+    }
 
     // ---- V~ = -W - Y_u S0 -> bf16 (rows = tokens), on the warps owning lanes 64..127
     if (qd >= 2) {
@@ -589,40 +631,39 @@ __global__ void __launch_bounds__(kGT, 1)
       mma_commit_warp(mbar);
       if (lane == 0) ++issued_mma;
     }
-    if (!(ok = gen_wait(mbar, phase, sabort))) break;
-
-    // ---- v is consumed: load the next chunk's
+    if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    // ---- u, q, z, k, log w are consumed (and their slots' later tenants): load the next chunk's
     if (tid == 0 && c + 1 < nch) {
       fence_proxy_async_smem();
-      load_in2(smem, maps, in2, b, h, t0 + kC);
-      ++in2_iss;
+      load_in1<kRwkv>(smem, maps, in1, b, h, t0 + kC);
+      ++in1_iss;
     }
+
     // ---- state update and output (warps owning lanes 0..63: key rows / token rows)
     if (owner) {
       float d[32];
       tmem_ld_32x32b_x32(tmem + kT_DS + lane_q + 32 * hf, d);
       tmem_ld_wait();
       const float pn = sPI[jrow];
-      float x[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         st[i] = pn * st[i] + d[i];
-        x[i] = st[i];
+        d[i] = st[i];
       }
 #pragma unroll
       for (int i = 0; i < 32; i += 8)
-        st_smem16(smem, SL::S0B + sw128_offset(jrow, 32 * hf + i, kC * 128), pack8(x + i));
-      float o1[32], o2[32];
+        st_smem16(smem, SL::S0B + sw128_offset(jrow, 32 * hf + i, kC * 128), pack8(d + i));
+      float o1[32];
       tmem_ld_32x32b_x32(tmem + kT_D3 + lane_q + 32 * hf, o1);
-      tmem_ld_32x32b_x32(tmem + kT_DO + lane_q + 32 * hf, o2);
+      tmem_ld_32x32b_x32(tmem + kT_DO + lane_q + 32 * hf, d);
       tmem_ld_wait();
       const int t = jrow;
       if (t < n) {
         float4 *dst = reinterpret_cast<float4 *>(p.o + (((size_t)b * T + t0 + t) * H + h) * kD + 32 * hf);
 #pragma unroll
         for (int i = 0; i < 32; i += 4)
-          dst[i / 4] = make_float4(o1[i] + o2[i], o1[i + 1] + o2[i + 1], o1[i + 2] + o2[i + 2],
-                                   o1[i + 3] + o2[i + 3]);
+          dst[i / 4] = make_float4(o1[i] + d[i], o1[i + 1] + d[i + 1], o1[i + 2] + d[i + 2],
+                                   o1[i + 3] + d[i + 3]);
       }
     }
     fence_proxy_async_smem();
