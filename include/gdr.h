@@ -89,9 +89,11 @@ typedef enum {
   GDR_ALGO_FP32 = 1,   /* fp32 CUDA-core kernel: every product in fp32 (all forms, all dtypes) */
   GDR_ALGO_TC = 2      /* tcgen05/TMEM kernels: bf16 operands, fp32 accumulate and state.
                           They apply to bf16 inputs with chunk >= 64 for
-                            GDN2, dk = dv = 128 (two kernels with a per-chunk record
-                                 workspace, or one kernel with the status word only), and
-                            GENERAL / RWKV7, dk = dv = 64 (one kernel, status word only);
+                            GDN2, dk = dv = 128: two kernels with a per-chunk record
+                                 workspace, or one kernel with the status word only;
+                            GLA, dk = dv = 128: the two kernels (GDR_ERR_WORKSPACE
+                                 without the record workspace; AUTO then takes fp32);
+                            every form, dk = dv = 64: one kernel, status word only;
                           GDR_ERR_UNSUPPORTED elsewhere.                                  */
 } gdr_algo;
 

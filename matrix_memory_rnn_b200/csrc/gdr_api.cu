@@ -63,7 +63,7 @@ gdr::FwdParams fwd_params(const gdr_fwd_args *a) {
 
 bool uses_tc(const gdr_fwd_args *a, const gdr::FwdParams &p) {
   return (a->algo == GDR_ALGO_TC || a->algo == GDR_ALGO_AUTO) &&
-         gdr::forward_tc_supported(p, a->dtype);
+         gdr::forward_tc_split_supported(p, a->dtype);
 }
 bool uses_tc_general(const gdr_fwd_args *a, const gdr::FwdParams &p) {
   return (a->algo == GDR_ALGO_TC || a->algo == GDR_ALGO_AUTO) &&
@@ -140,15 +140,16 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
     if (!a->workspace || a->workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
     return cuda_status(gdr::launch_forward_tc_general(p, s));
   }
-  const bool tc_ok = gdr::forward_tc_supported(p, a->dtype);
+  const bool tc_ok = gdr::forward_tc_split_supported(p, a->dtype);
   if (a->algo == GDR_ALGO_TC || (a->algo == GDR_ALGO_AUTO && tc_ok)) {
     if (!tc_ok) return GDR_ERR_UNSUPPORTED;
     if (!a->workspace || a->workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
     // the two-kernel path when the workspace holds its per-chunk records, else the
-    // single-kernel path (status word only)
+    // single-kernel path (status word only; GDN-2 alone)
     if (a->workspace_bytes >= gdr::forward_tc_split_workspace_bytes(p))
       return cuda_status(gdr::launch_forward_tc_split(p, a->workspace, s));
-    return cuda_status(gdr::launch_forward_tc(p, s));
+    if (gdr::forward_tc_supported(p, a->dtype)) return cuda_status(gdr::launch_forward_tc(p, s));
+    if (a->algo == GDR_ALGO_TC) return GDR_ERR_WORKSPACE;
   }
   if (!gdr::forward_fp32_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
   return cuda_status(gdr::launch_forward_fp32(p, a->dtype, s));

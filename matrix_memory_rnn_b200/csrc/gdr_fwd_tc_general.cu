@@ -1,6 +1,8 @@
-// gdr_fwd_tc_general.cu -- chunked forward of the two-stream (general) form on the
-// tensor cores: GDR_FORM_GENERAL (u, z given) and GDR_FORM_RWKV7 (u = c a, z = a),
-// bf16 inputs, d_k = d_v = 64, chunks of C = 64 tokens.
+// gdr_fwd_tc_general.cu -- chunked forward of the generalized delta rule on the
+// tensor cores at d_k = d_v = 64 (bf16 inputs, chunks of C = 64 tokens), written for
+// the two-stream form and serving every form through its mapping:
+// GDR_FORM_GENERAL (u, z given), GDR_FORM_RWKV7 (u = c a, z = a), GDR_FORM_GDN2
+// (u = alpha (.) b (.) k, z = k, written value wg (.) v) and GDR_FORM_GLA (u = z = 0).
 //
 // "Exponential gates and matrix memory: xLSTM and RWKV-7", section 13.3 (the
 // generalized delta rule; the erase reads the undecayed state S_{t-1}), evaluated
@@ -112,14 +114,24 @@ struct GenMaps {
   CUtensorMap q, k, v, e1, e2, lw;
 };
 
-template <bool kRwkv>
+// Which tiles a form stages: e1 (u, a or the erase gate b) in the first half of the
+// MMA1 A operand, e2 (z, or GDN-2's write gate) in the first half of its B operand.
+template <int kForm>
+__device__ __forceinline__ bool form_has_e1() { return kForm != GDR_FORM_GLA; }
+template <int kForm>
+__device__ __forceinline__ bool form_has_e2(bool has_wg) {
+  return kForm == GDR_FORM_GENERAL || (kForm == GDR_FORM_GDN2 && has_wg);
+}
+
+template <int kForm>
 __device__ __forceinline__ void load_in1(uint8_t *smem, const GenMaps &m, uint64_t *bar, int b, int h,
-                                         int t0) {
+                                         int t0, bool has_wg) {
   using SL = GenSmem;
-  mbar_arrive_expect_tx(bar, (kRwkv ? 3u : 4u) * kTile + kC * kD * 4u);
-  tma_load_4d(smem + SL::A1, &m.e1, 0, h, t0, b, bar);
+  const bool e1 = form_has_e1<kForm>(), e2 = form_has_e2<kForm>(has_wg);
+  mbar_arrive_expect_tx(bar, (2u + (e1 ? 1u : 0u) + (e2 ? 1u : 0u)) * kTile + kC * kD * 4u);
+  if (e1) tma_load_4d(smem + SL::A1, &m.e1, 0, h, t0, b, bar);
   tma_load_4d(smem + SL::A1 + kTile, &m.q, 0, h, t0, b, bar);
-  if (!kRwkv) tma_load_4d(smem + SL::B1, &m.e2, 0, h, t0, b, bar);
+  if (e2) tma_load_4d(smem + SL::B1, &m.e2, 0, h, t0, b, bar);
   tma_load_4d(smem + SL::B1 + kTile, &m.k, 0, h, t0, b, bar);
   tma_load_4d(smem + SL::LW, &m.lw, 0, h, t0, b, bar);
 }
@@ -170,9 +182,10 @@ __device__ __forceinline__ void chunk_scan(float *lw, float *sQT, float *sA1, fl
   __syncthreads();
 }
 
-template <bool kRwkv>
+template <int kForm>
 __global__ void __launch_bounds__(kGT, 2)
     tc_general_kernel(FwdParams p, const __grid_constant__ GenMaps maps) {
+  constexpr bool kRwkv = kForm == GDR_FORM_RWKV7;
   using SL = GenSmem;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -202,7 +215,8 @@ __global__ void __launch_bounds__(kGT, 2)
   const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
   const __nv_bfloat16 *ge1 = static_cast<const __nv_bfloat16 *>(p.e1);
-  const __nv_bfloat16 *ge2 = static_cast<const __nv_bfloat16 *>(p.e2);   // z, or RWKV-7 c [B][T][H]
+  const __nv_bfloat16 *ge2 = static_cast<const __nv_bfloat16 *>(p.e2);   // z, RWKV-7 c [B][T][H], or wg
+  const bool has_wg = kForm == GDR_FORM_GDN2 && p.e2 != nullptr;
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -215,7 +229,7 @@ __global__ void __launch_bounds__(kGT, 2)
     fence_mbar_init();
     *sabort = 0;
     if (nch > 0) {
-      load_in1<kRwkv>(smem, maps, in1, b, h, 0);
+      load_in1<kForm>(smem, maps, in1, b, h, 0, has_wg);
       load_in2(smem, maps, in2, b, h, 0);
     }
   }
@@ -310,29 +324,59 @@ __global__ void __launch_bounds__(kGT, 2)
           lam[0] = l0.x; lam[1] = l0.y; lam[2] = l0.z; lam[3] = l0.w;
           lam[4] = l1.x; lam[5] = l1.y; lam[6] = l1.z; lam[7] = l1.w;
         }
+        // fp: lam_{t-1} (GDN-2 first takes its own decay alpha_t = e^{lam_t - lam_{t-1}}
+        // from it, alpha_0 = e^{Lam_0}), then f' = e^{lam_{t-1}} (row 0: unused, 0)
+        float at[8];
         if (t > 0) {
           const float4 m0 = *reinterpret_cast<const float4 *>(sLW + (t - 1) * kD + j0);
           const float4 m1 = *reinterpret_cast<const float4 *>(sLW + (t - 1) * kD + j0 + 4);
           fp[0] = m0.x; fp[1] = m0.y; fp[2] = m0.z; fp[3] = m0.w;
           fp[4] = m1.x; fp[5] = m1.y; fp[6] = m1.z; fp[7] = m1.w;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) fp[e] = __expf(fp[e]);
+          for (int e = 0; e < 8; ++e) {
+            if (kForm == GDR_FORM_GDN2) at[e] = __expf(lam[e] - fp[e]);
+            fp[e] = __expf(fp[e]);
+          }
         } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) fp[e] = 0.f;
+          for (int e = 0; e < 8; ++e) {
+            if (kForm == GDR_FORM_GDN2) at[e] = a0[e];
+            fp[e] = 0.f;
+          }
         }
         unpack8(*reinterpret_cast<const uint4 *>(smem + SL::A1 + kTile + o), q8);
         unpack8(*reinterpret_cast<const uint4 *>(smem + SL::B1 + kTile + o), k8);
-        unpack8(*reinterpret_cast<const uint4 *>(smem + SL::A1 + o), u8);
-        if (kRwkv) {
+        if (kForm == GDR_FORM_GLA) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) u8[e] = z8[e] = 0.f;
+        } else {
+          unpack8(*reinterpret_cast<const uint4 *>(smem + SL::A1 + o), u8);
+        }
+        if (kForm == GDR_FORM_RWKV7) {
           const float ct = sC[t];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             z8[e] = u8[e];        // z = a
             u8[e] *= ct;          // u = c a
           }
-        } else {
+        } else if (kForm == GDR_FORM_GENERAL) {
           unpack8(*reinterpret_cast<const uint4 *>(smem + SL::B1 + o), z8);
+        } else if (kForm == GDR_FORM_GDN2) {
+          // u = alpha_t b k with alpha_t = e^{Lam_t - Lam_{t-1}} (alpha_0 = e^{Lam_0}), z = k;
+          // the written value wg (.) v replaces v in place
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            u8[e] = at[e] * u8[e] * k8[e];
+            z8[e] = k8[e];
+          }
+          if (has_wg) {
+            float w8[8], v8[8];
+            unpack8(*reinterpret_cast<const uint4 *>(smem + SL::B1 + o), w8);
+            unpack8(*reinterpret_cast<const uint4 *>(smem + SL::V + o), v8);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+            st_smem16(smem, SL::V + o, pack8(v8));
+          }
         }
         // U f' (in place over u) and U_pi
 #pragma unroll
@@ -452,13 +496,25 @@ __global__ void __launch_bounds__(kGT, 2)
           const float ct = kRwkv ? sC[t] : 1.f;
           for (int j = 0; j < kD; ++j) {
             const float ls = lam[s * kD + j], lt = lam[t * kD + j];
-            const float zs = kRwkv ? __bfloat162float(ge1[os + j]) : __bfloat162float(ge2[os + j]);
             const float ks = __bfloat162float(gk[os + j]);
+            // the form's erase key z_s and erase vector u_t
+            float zs = 0.f, ut = 0.f;
+            if (kForm == GDR_FORM_GENERAL) {
+              zs = __bfloat162float(ge2[os + j]);
+              ut = __bfloat162float(ge1[ot + j]);
+            } else if (kForm == GDR_FORM_RWKV7) {
+              zs = __bfloat162float(ge1[os + j]);
+              ut = __bfloat162float(ge1[ot + j]) * ct;
+            } else if (kForm == GDR_FORM_GDN2) {
+              zs = ks;
+              ut = __expf(__ldg(p.log_w + ot + j)) * __bfloat162float(ge1[ot + j]) *
+                   __bfloat162float(gk[ot + j]);
+            }
             const float dq = __expf(lt - ls) * __bfloat162float(gq[ot + j]);
             mz += dq * zs;
             mk += dq * ks;
             if (s < t) {
-              const float du = __expf(lam[(t - 1) * kD + j] - ls) * __bfloat162float(ge1[ot + j]) * ct;
+              const float du = __expf(lam[(t - 1) * kD + j] - ls) * ut;
               av += du * zs;
               bv += du * ks;
             }
@@ -635,7 +691,7 @@ __global__ void __launch_bounds__(kGT, 2)
     // ---- u, q, z, k, log w are consumed (and their slots' later tenants): load the next chunk's
     if (tid == 0 && c + 1 < nch) {
       fence_proxy_async_smem();
-      load_in1<kRwkv>(smem, maps, in1, b, h, t0 + kC);
+      load_in1<kForm>(smem, maps, in1, b, h, t0 + kC, has_wg);
       ++in1_iss;
     }
 
@@ -725,20 +781,27 @@ bool encode_gen_map(CUtensorMap *m, const void *base, bool bf16, const FwdParams
 }  // namespace
 
 bool forward_tc_general_supported(const FwdParams &p, gdr_dtype dtype) {
-  return (p.form == GDR_FORM_GENERAL || p.form == GDR_FORM_RWKV7) && dtype == GDR_BF16 &&
-         p.dk == kD && p.dv == kD && (p.chunk == kC || p.chunk == 2 * kC);
+  return dtype == GDR_BF16 && p.dk == kD && p.dv == kD && (p.chunk == kC || p.chunk == 2 * kC);
 }
 
 cudaError_t launch_forward_tc_general(const FwdParams &p, cudaStream_t stream) {
-  const bool rwkv = p.form == GDR_FORM_RWKV7;
   GenMaps maps;
   memset(&maps, 0, sizeof(maps));
+  // e1: u, a or b (not GLA); e2: z (general) or the optional write gate (GDN-2)
+  const bool e1 = p.form != GDR_FORM_GLA;
+  const bool e2 = p.form == GDR_FORM_GENERAL || (p.form == GDR_FORM_GDN2 && p.e2);
   if (!encode_gen_map(&maps.q, p.q, true, p) || !encode_gen_map(&maps.k, p.k, true, p) ||
-      !encode_gen_map(&maps.v, p.v, true, p) || !encode_gen_map(&maps.e1, p.e1, true, p) ||
-      (!rwkv && !encode_gen_map(&maps.e2, p.e2, true, p)) ||
+      !encode_gen_map(&maps.v, p.v, true, p) || (e1 && !encode_gen_map(&maps.e1, p.e1, true, p)) ||
+      (e2 && !encode_gen_map(&maps.e2, p.e2, true, p)) ||
       !encode_gen_map(&maps.lw, p.log_w, false, p))
     return cudaErrorInvalidValue;
-  auto kern = rwkv ? tc_general_kernel<true> : tc_general_kernel<false>;
+  void (*kern)(FwdParams, const GenMaps) = nullptr;
+  switch (p.form) {
+    case GDR_FORM_GENERAL: kern = tc_general_kernel<GDR_FORM_GENERAL>; break;
+    case GDR_FORM_RWKV7: kern = tc_general_kernel<GDR_FORM_RWKV7>; break;
+    case GDR_FORM_GDN2: kern = tc_general_kernel<GDR_FORM_GDN2>; break;
+    default: kern = tc_general_kernel<GDR_FORM_GLA>; break;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)GenSmem::ALLOC);
   if (e != cudaSuccess) return e;

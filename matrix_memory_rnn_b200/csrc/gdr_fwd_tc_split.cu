@@ -156,15 +156,17 @@ struct PrepMaps {
   CUtensorMap k, b, q, v, wg, lw;
 };
 
-// One thread: the chunk buffer's tile loads (k, b, q, v) for chunk (b, h, t0).
+// One thread: the chunk buffer's tile loads (k, b, q, v) for chunk (b, h, t0); GLA
+// (has_b false) has no erase gate and skips b.
 __device__ __forceinline__ void load_tiles(uint8_t *buf, const PrepMaps &m, uint64_t *bar, int b,
-                                           int h, int t0) {
+                                           int h, int t0, bool has_b) {
   using SL = PrepSmem;
-  mbar_arrive_expect_tx(bar, 4u * kC * kDK * 2);
+  mbar_arrive_expect_tx(bar, (has_b ? 4u : 3u) * kC * kDK * 2);
 #pragma unroll
   for (int blk = 0; blk < 2; ++blk) {
     tma_load_4d(buf + SL::B_LM + blk * (kC * 128), &m.k, 64 * blk, h, t0, b, bar);
-    tma_load_4d(buf + SL::A_LM + blk * (2 * kC * 128), &m.b, 64 * blk, h, t0, b, bar);
+    if (has_b)
+      tma_load_4d(buf + SL::A_LM + blk * (2 * kC * 128), &m.b, 64 * blk, h, t0, b, bar);
     tma_load_4d(buf + SL::A_LM + blk * (2 * kC * 128) + kC * 128, &m.q, 64 * blk, h, t0, b, bar);
     tma_load_4d(buf + SL::VH + blk * (kC * 128), &m.v, 64 * blk, h, t0, b, bar);
   }
@@ -245,7 +247,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   const __nv_bfloat16 *gq = static_cast<const __nv_bfloat16 *>(p.q);
   const __nv_bfloat16 *gk = static_cast<const __nv_bfloat16 *>(p.k);
   const __nv_bfloat16 *gb = static_cast<const __nv_bfloat16 *>(p.e1);
-  const bool has_wg = p.e2 != nullptr;
+  // GDN-2 (erase gate b, optional write gate) or GLA (u = 0: no b, no write gate)
+  const bool has_b = p.form == GDR_FORM_GDN2;
+  const bool has_wg = has_b && p.e2 != nullptr;
   auto item_of = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
 
   if (warp == 0) {
@@ -267,7 +271,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     for (int i = 0; i < kNCnt; ++i) cnt[i] = 0;
     for (int j = 0; j < 2 && j < nloc; ++j) {
       const int it = item_of(j), c = it % nch, bh = it / nch;
-      load_tiles(smem + j * SL::BUF, maps, bfull + j, bh / H, bh % H, c * kC);
+      load_tiles(smem + j * SL::BUF, maps, bfull + j, bh / H, bh % H, c * kC, has_b);
       ++cnt[kBIss0 + j];
       if (has_wg) {
         load_gate(smem + SL::SW + j * (kC * kDK * 2), maps, wfull + j, bh / H, bh % H, c * kC);
@@ -412,7 +416,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             const uint32_t oq = SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128);
             float k8[8], b8[8], q8[8];
             unpack8(*reinterpret_cast<const uint4 *>(buf + SL::B_LM + ok_), k8);
-            unpack8(*reinterpret_cast<const uint4 *>(buf + ob), b8);
+            if (has_b) {
+              unpack8(*reinterpret_cast<const uint4 *>(buf + ob), b8);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) b8[e] = 0.f;
+            }
             unpack8(*reinterpret_cast<const uint4 *>(buf + oq), q8);
             float av[8], aq[8], bl[8], kt[8], qp[8];
 #pragma unroll
@@ -543,7 +552,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
               const float d = __expf(__ldcg(lt + jj) - __ldcg(ls + jj));
               const float ks = __bfloat162float(gk[os + jj]);
               m += __bfloat162float(gq[ot + jj]) * d * ks;
-              l += __bfloat162float(gb[ot + jj]) * __bfloat162float(gk[ot + jj]) * d * ks;
+              if (has_b) l += __bfloat162float(gb[ot + jj]) * __bfloat162float(gk[ot + jj]) * d * ks;
             }
           }
           sL[Ix::at(t, s)] = (s < t) ? l : 0.f;
@@ -600,7 +609,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       if (gt == 32 && j + 2 < nloc) {
         fence_proxy_async_smem();
         const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
-        load_tiles(buf, maps, bfull + bi, bhn / H, bhn % H, cn * kC);
+        load_tiles(buf, maps, bfull + bi, bhn / H, bhn % H, cn * kC, has_b);
         cnt[kBIss0 + bi] += 1;
       }
 
@@ -944,6 +953,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
 
 }  // namespace
 
+// GDN-2 and GLA (GDN-2 with b = 0), bf16, d_k = d_v = 128; chunk 64, or 128 served
+// as two 64-token chunks.
+bool forward_tc_split_supported(const FwdParams &p, gdr_dtype dtype) {
+  return (p.form == GDR_FORM_GDN2 || p.form == GDR_FORM_GLA) && dtype == GDR_BF16 &&
+         p.dk == kDK && p.dv == kDK && (p.chunk == kC || p.chunk == 2 * kC);
+}
+
 size_t forward_tc_split_workspace_bytes(const FwdParams &p) {
   return kHeaderBytes + (size_t)p.B * p.H * num_chunks(p.T) * Rec::BYTES;
 }
@@ -989,11 +1005,12 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   // log w: one 128-channel fp32 box, row-major
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  const bool has_b = p.form == GDR_FORM_GDN2;
   if (!encode_input_map(&maps.k, p.k, bf, 2, 64, sw, p) ||
-      !encode_input_map(&maps.b, p.e1, bf, 2, 64, sw, p) ||
+      (has_b && !encode_input_map(&maps.b, p.e1, bf, 2, 64, sw, p)) ||
       !encode_input_map(&maps.q, p.q, bf, 2, 64, sw, p) ||
       !encode_input_map(&maps.v, p.v, bf, 2, 64, sw, p) ||
-      (p.e2 && !encode_input_map(&maps.wg, p.e2, bf, 2, 64, sw, p)) ||
+      (has_b && p.e2 && !encode_input_map(&maps.wg, p.e2, bf, 2, 64, sw, p)) ||
       !encode_input_map(&maps.lw, p.log_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK,
                         CU_TENSOR_MAP_SWIZZLE_NONE, p))
     return cudaErrorInvalidValue;

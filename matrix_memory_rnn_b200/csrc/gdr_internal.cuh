@@ -75,6 +75,7 @@ bool forward_tc_supported(const FwdParams &p, gdr_dtype dtype);
 bool forward_tc_general_supported(const FwdParams &p, gdr_dtype dtype);
 cudaError_t launch_forward_tc_general(const FwdParams &p, cudaStream_t stream);
 // Two-kernel tensor-core path: per-chunk records in the workspace.
+bool forward_tc_split_supported(const FwdParams &p, gdr_dtype dtype);
 size_t forward_tc_split_workspace_bytes(const FwdParams &p);
 cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStream_t stream);
 

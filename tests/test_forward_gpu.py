@@ -187,11 +187,11 @@ def test_tc_kernel_strong_decay_uses_exact_path(path):
     assert eo < TOL["bf16"] and es < TOL["bf16"]
 
 
-@pytest.mark.parametrize("form", ["rwkv7", "general"])
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("T", [1, 64, 100, 257])
 @pytest.mark.parametrize("with_state", [False, True])
 def test_tc_general_kernel(form, T, with_state):
-    """Two-stream tensor-core kernel (RWKV-7 / general, bf16, d = 64, C = 64) against the oracle."""
+    """Two-stream tensor-core kernel (every form, bf16, d = 64, C = 64) against the oracle."""
     w = small(form, "bf16", dk=64, dv=64, T=T, B=2, H=3, chunk=64)
     inp = synth.forward_inputs(w)
     if with_state:
@@ -203,7 +203,18 @@ def test_tc_general_kernel(form, T, with_state):
     assert eo < TOL["bf16"] and es < TOL["bf16"]
 
 
-@pytest.mark.parametrize("form", ["rwkv7", "general"])
+def test_tc_general_gdn2_without_write_gate():
+    """GDN-2 with no write gate (written value v) on the two-stream kernel."""
+    w = small("gdn2", "bf16", dk=64, dv=64, T=150, B=2, H=3, chunk=64)
+    inp = synth.forward_inputs(w)
+    inp["e2"] = None
+    o, S = gpu_forward(w, inp, algo="tc")
+    o_ref, S_ref = oracle_forward(w, inp)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
+@pytest.mark.parametrize("form", FORMS)
 def test_tc_general_strong_decay_uses_exact_path(form):
     """Channels whose decay over a chunk exceeds e^-80 take the exact pairwise path."""
     w = small(form, "bf16", dk=64, dv=64, T=200, B=1, H=2, chunk=64)
@@ -218,6 +229,42 @@ def test_tc_general_strong_decay_uses_exact_path(form):
     print(f"tc-general strong decay {form}: o {eo:.3e} S {es:.3e}")
     assert np.isfinite(o).all() and np.isfinite(S).all()
     assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
+@pytest.mark.parametrize("T", [1, 100, 257])
+@pytest.mark.parametrize("with_state", [False, True])
+def test_tc_split_gla(T, with_state):
+    """GLA at d = 128 on the prep + chain kernels (GDN-2's chunk algebra with b = 0)."""
+    w = small("gla", "bf16", dk=128, dv=128, T=T, B=2, H=3, chunk=64)
+    inp = synth.forward_inputs(w)
+    if with_state:
+        inp["S0"] = synth.round_f32(np.random.default_rng(9).normal(0, 0.5, (w.B, w.H, 128, 128)))
+    o, S = gpu_forward(w, inp, algo="tc")
+    o_ref, S_ref = oracle_forward(w, inp)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    print(f"tc-split gla T={T} S0={with_state}: o {eo:.3e} S {es:.3e}")
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
+def test_tc_split_gla_strong_decay_and_small_workspace():
+    """GLA at d = 128: the exact pairwise path, and without the record workspace algo=tc
+    reports GDR_ERR_WORKSPACE while algo=auto takes the fp32 kernel."""
+    w = small("gla", "bf16", dk=128, dv=128, T=200, B=1, H=2, chunk=64)
+    inp = synth.forward_inputs(w)
+    lw = inp["log_w"].copy()
+    lw[:, :, :, ::7] = -3.0
+    lw[:, 70:80, 1, 5] = -60.0
+    inp["log_w"] = lw.astype(np.float32)
+    o_ref, S_ref = oracle_forward(w, inp)
+    o, S = gpu_forward(w, inp, algo="tc")
+    assert head_rel_err(o, o_ref, (0, 2)) < TOL["bf16"]
+    assert head_rel_err(S, S_ref, (0, 1)) < TOL["bf16"]
+    with pytest.raises(gdr.GdrError) as ei:
+        gpu_forward(w, inp, algo="tc", workspace_bytes=256)
+    assert ei.value.code == 7
+    o, S = gpu_forward(w, inp, algo="auto", workspace_bytes=256)
+    assert head_rel_err(o, o_ref, (0, 2)) < TOL["bf16"]
+    assert head_rel_err(S, S_ref, (0, 1)) < TOL["bf16"]
 
 
 def test_tc_rejects_what_it_does_not_cover():
