@@ -41,14 +41,18 @@
 
 enum { OR_GENERAL = 0, OR_GDN2 = 1, OR_RWKV7 = 2, OR_GLA = 3 };
 
-/* One (b, h) sequence.  S is d_v x d_k (column form), row-major: S[c * dk + j]. */
+/* Tokens [t_begin, t_end) of one (b, h) sequence.  S is d_v x d_k (column form),
+ * row-major: S[c * dk + j].  o may be NULL (no readout).  On return u, z, w, vv
+ * and e hold the last token's erase vector, erase key, decay, written value and
+ * e = S_{t-1} u. */
 static void run_sequence(int form, int b, int h, int B, int T, int H, int dk, int dv,
+                         int t_begin, int t_end,
                          const double *q, const double *k, const double *v,
                          const double *log_w, const double *e1, const double *e2,
                          double *S, double *o, double *u, double *z, double *w,
                          double *vv, double *e) {
   (void)B;
-  for (int t = 0; t < T; ++t) {
+  for (int t = t_begin; t < t_end; ++t) {
     const size_t tk = (((size_t)b * T + t) * H + h) * (size_t)dk;  /* [b][t][h][.] over dk */
     const size_t tv = (((size_t)b * T + t) * H + h) * (size_t)dv;  /* [b][t][h][.] over dv */
     const size_t ts = ((size_t)b * T + t) * H + h;                 /* [b][t][h] scalar     */
@@ -86,7 +90,7 @@ static void run_sequence(int form, int b, int h, int B, int T, int H, int dk, in
       for (int j = 0; j < dk; ++j)
         S[(size_t)c * dk + j] = S[(size_t)c * dk + j] * w[j] - e[c] * z[j] + vv[c] * k[tk + j];
     /* o_t = S q_t */
-    for (int c = 0; c < dv; ++c) {
+    for (int c = 0; o && c < dv; ++c) {
       double acc = 0.0;
       for (int j = 0; j < dk; ++j) acc += S[(size_t)c * dk + j] * q[tk + j];
       o[tv + c] = acc;
@@ -136,7 +140,7 @@ int oracle_forward(int form, int B, int T, int H, int dk, int dv,
         for (int j = 0; j < dk; ++j)
           S[(size_t)c * dk + j] = S0 ? S0[so + (size_t)j * dv + c] : 0.0;
       double *u = scratch, *z = u + dk, *w = z + dk, *vv = w + dk, *e = vv + dv;
-      run_sequence(form, b, h, B, T, H, dk, dv, q, k, v, log_w, e1, e2, S, o,
+      run_sequence(form, b, h, B, T, H, dk, dv, 0, T, q, k, v, log_w, e1, e2, S, o,
                    u, z, w, vv, e);
       if (S_T)
         for (int c = 0; c < dv; ++c)
@@ -155,4 +159,203 @@ int oracle_max_threads(void) {
 #else
   return 1;
 #endif
+}
+
+/*
+ * Reverse mode of the same loop (the adjoint of each statement of run_sequence,
+ * taken in reverse token order).  With the loss L = <dO, o> + <dS_T, S_T>, the
+ * adjoint dS of the state after token t collects dO_t q_t^T from the readout and
+ * the propagated adjoint of the next token; then, for
+ * S_t = S_{t-1} Diag(w) - e z^T + vv k^T with e = S_{t-1} u:
+ *
+ *     dq = S_t^T dO_t          dvv = dS k          dk  = dS^T vv
+ *     de = -dS z               dz  = -dS^T e       dw  = diag(S_{t-1}^T dS)
+ *     du = S_{t-1}^T de        dS_{t-1} = dS Diag(w) + de u^T
+ *
+ * and the form's mapping is differentiated back to its raw arguments:
+ *   all forms: d log_w = dw (.) w                        (w = exp(log_w))
+ *   general  : d e1 = du, d e2 = dz
+ *   GDN-2    : u = w (.) b (.) k, z = k, vv = wg (.) v:
+ *              dk += dz + du (.) w (.) b,  d b = du (.) w (.) k,  d log_w += du (.) u,
+ *              dv = dvv (.) wg,  d wg = dvv (.) v
+ *   RWKV-7   : u = c a, z = a:  d a = c du + dz,  d c = <du, a>
+ *   GLA      : u = z = 0 (no erase gradients)
+ *
+ * States are recomputed from checkpoints taken every kSeg tokens (plain
+ * recomputation; the arithmetic is the forward's own loop).
+ *
+ * Inputs as oracle_forward, plus dO [B][T][H][dv] and dS_T [B][H][dk][dv] (NULL =
+ * 0).  Outputs: dq, dk, dlog_w [B][T][H][dk]; dv [B][T][H][dv]; de1 shaped like
+ * e1 and de2 like e2 (NULL for a form without them); dS0 [B][H][dk][dv] (may be
+ * NULL).  Returns 0, -1 on bad arguments, -2 when scratch memory ran out.
+ */
+enum { kSeg = 64 };
+
+static void reverse_token(int form, int dk, int dv, size_t tk, size_t tv, size_t ts,
+                          const double *q, const double *k, const double *v,
+                          const double *e1, const double *e2, const double *dO,
+                          const double *S_prev, const double *S_cur, const double *u,
+                          const double *z, const double *w, const double *vv,
+                          const double *e, double *dS, double *de, double *dvv,
+                          double *dq, double *dk_, double *dv_, double *dlog_w,
+                          double *de1, double *de2) {
+  /* readout o_t = S_t q_t */
+  for (int j = 0; j < dk; ++j) {
+    double acc = 0.0;
+    for (int c = 0; c < dv; ++c) acc += S_cur[(size_t)c * dk + j] * dO[tv + c];
+    dq[tk + j] = acc;
+  }
+  for (int c = 0; c < dv; ++c)
+    for (int j = 0; j < dk; ++j) dS[(size_t)c * dk + j] += dO[tv + c] * q[tk + j];
+  /* S_t = S_{t-1} Diag(w) - e z^T + vv k^T */
+  for (int c = 0; c < dv; ++c) {
+    double a = 0.0, b = 0.0;
+    for (int j = 0; j < dk; ++j) {
+      a += dS[(size_t)c * dk + j] * k[tk + j];
+      b += dS[(size_t)c * dk + j] * z[j];
+    }
+    dvv[c] = a;
+    de[c] = -b;
+  }
+  for (int j = 0; j < dk; ++j) {
+    double kw = 0.0, zz = 0.0, ww = 0.0, uu = 0.0;
+    for (int c = 0; c < dv; ++c) {
+      const double g = dS[(size_t)c * dk + j];
+      kw += g * vv[c];
+      zz -= g * e[c];
+      ww += g * S_prev[(size_t)c * dk + j];
+      uu += S_prev[(size_t)c * dk + j] * de[c];   /* e = S_{t-1} u */
+    }
+    double dkj = kw, dlw = ww * w[j];
+    switch (form) {
+      case OR_GENERAL:
+        de1[tk + j] = uu;
+        de2[tk + j] = zz;
+        break;
+      case OR_GDN2:
+        dkj += zz + uu * w[j] * e1[tk + j];
+        de1[tk + j] = uu * w[j] * k[tk + j];
+        dlw += uu * u[j];
+        break;
+      case OR_RWKV7:
+        de1[tk + j] = uu * e2[ts] + zz;
+        break;
+      default:
+        break;
+    }
+    dk_[tk + j] = dkj;
+    dlog_w[tk + j] = dlw;
+  }
+  if (form == OR_RWKV7) {
+    double acc = 0.0;
+    for (int j = 0; j < dk; ++j) {
+      double uu = 0.0;
+      for (int c = 0; c < dv; ++c) uu += S_prev[(size_t)c * dk + j] * de[c];
+      acc += uu * e1[tk + j];
+    }
+    de2[ts] = acc;
+  }
+  for (int c = 0; c < dv; ++c) {
+    if (form == OR_GDN2 && e2) {
+      dv_[tv + c] = dvv[c] * e2[tv + c];
+      de2[tv + c] = dvv[c] * v[tv + c];
+    } else {
+      dv_[tv + c] = dvv[c];
+    }
+  }
+  /* adjoint of S_{t-1} */
+  for (int c = 0; c < dv; ++c)
+    for (int j = 0; j < dk; ++j)
+      dS[(size_t)c * dk + j] = dS[(size_t)c * dk + j] * w[j] + de[c] * u[j];
+}
+
+int oracle_backward(int form, int B, int T, int H, int dk, int dv,
+                    const double *q, const double *k, const double *v,
+                    const double *log_w, const double *e1, const double *e2,
+                    const double *S0, const double *dO, const double *dS_T,
+                    double *dq, double *dk_, double *dv_, double *dlog_w,
+                    double *de1, double *de2, double *dS0, int n_threads) {
+  if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+  if (form < OR_GENERAL || form > OR_GLA) return -1;
+  if (T > 0 && (!q || !k || !v || !log_w || !dO || !dq || !dk_ || !dv_ || !dlog_w)) return -1;
+  if (T > 0 && form == OR_GENERAL && (!e1 || !e2 || !de1 || !de2)) return -1;
+  if (T > 0 && form == OR_GDN2 && (!e1 || !de1 || (e2 && !de2))) return -1;
+  if (T > 0 && form == OR_RWKV7 && (!e1 || !e2 || !de1 || !de2)) return -1;
+
+  const int n_seq = B * H;
+  const int n_ck = (T + kSeg - 1) / kSeg + 1;
+  const size_t dd = (size_t)dk * dv;
+  int failed = 0;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel
+#endif
+  {
+    double *ck = (double *)malloc(sizeof(double) * dd * (size_t)n_ck);        /* checkpoints */
+    double *st = (double *)malloc(sizeof(double) * dd * (size_t)(kSeg + 1));  /* segment states */
+    double *par = (double *)malloc(sizeof(double) * (size_t)kSeg * (3 * dk + 2 * dv));
+    double *dS = (double *)malloc(sizeof(double) * dd);
+    double *scratch = (double *)malloc(sizeof(double) * (size_t)(3 * dk + 4 * dv));
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+    for (int sq = 0; sq < n_seq; ++sq) {
+      if (!ck || !st || !par || !dS || !scratch) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+        failed = 1;
+        continue;
+      }
+      const int b = sq / H, h = sq % H;
+      const size_t so = (size_t)sq * dd;
+      double *u = scratch, *z = u + dk, *w = z + dk, *vv = w + dk, *e = vv + dv;
+      double *de = e + dv, *dvv = de + dv;
+      /* forward pass: checkpoints at t = 0, kSeg, 2 kSeg, ... */
+      for (int c = 0; c < dv; ++c)
+        for (int j = 0; j < dk; ++j)
+          ck[(size_t)c * dk + j] = S0 ? S0[so + j * (size_t)dv + c] : 0.0;
+      for (int g = 0; g + 1 < n_ck; ++g) {
+        memcpy(ck + (size_t)(g + 1) * dd, ck + (size_t)g * dd, sizeof(double) * dd);
+        const int t1 = (g + 1) * kSeg < T ? (g + 1) * kSeg : T;
+        run_sequence(form, b, h, B, T, H, dk, dv, g * kSeg, t1, q, k, v, log_w, e1, e2,
+                     ck + (size_t)(g + 1) * dd, NULL, u, z, w, vv, e);
+      }
+      /* reverse pass */
+      for (int c = 0; c < dv; ++c)
+        for (int j = 0; j < dk; ++j)
+          dS[(size_t)c * dk + j] = dS_T ? dS_T[so + (size_t)j * dv + c] : 0.0;
+      for (int g = n_ck - 2; g >= 0; --g) {
+        const int t0 = g * kSeg, n = (t0 + kSeg < T ? t0 + kSeg : T) - t0;
+        memcpy(st, ck + (size_t)g * dd, sizeof(double) * dd);
+        for (int i = 0; i < n; ++i) {
+          double *S = st + (size_t)(i + 1) * dd;
+          double *pp = par + (size_t)i * (3 * dk + 2 * dv);
+          memcpy(S, st + (size_t)i * dd, sizeof(double) * dd);
+          run_sequence(form, b, h, B, T, H, dk, dv, t0 + i, t0 + i + 1, q, k, v, log_w, e1, e2,
+                       S, NULL, pp, pp + dk, pp + 2 * dk, pp + 3 * dk, pp + 3 * dk + dv);
+        }
+        for (int i = n - 1; i >= 0; --i) {
+          const int t = t0 + i;
+          const size_t tk = (((size_t)b * T + t) * H + h) * (size_t)dk;
+          const size_t tv = (((size_t)b * T + t) * H + h) * (size_t)dv;
+          const size_t ts = ((size_t)b * T + t) * H + h;
+          const double *pp = par + (size_t)i * (3 * dk + 2 * dv);
+          reverse_token(form, dk, dv, tk, tv, ts, q, k, v, e1, e2, dO, st + (size_t)i * dd,
+                        st + (size_t)(i + 1) * dd, pp, pp + dk, pp + 2 * dk, pp + 3 * dk,
+                        pp + 3 * dk + dv, dS, de, dvv, dq, dk_, dv_, dlog_w, de1, de2);
+        }
+      }
+      if (dS0)
+        for (int c = 0; c < dv; ++c)
+          for (int j = 0; j < dk; ++j)
+            dS0[so + j * (size_t)dv + c] = dS[(size_t)c * dk + j];
+    }
+    free(ck);
+    free(st);
+    free(par);
+    free(dS);
+    free(scratch);
+  }
+  return failed ? -2 : 0;
 }

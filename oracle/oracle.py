@@ -48,6 +48,8 @@ def load_library(path: str):
     lib.oracle_forward.restype = ctypes.c_int
     lib.oracle_forward.argtypes = [ctypes.c_int] * 6 + [dp] * 9 + [ctypes.c_int]
     lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_backward.restype = ctypes.c_int
+    lib.oracle_backward.argtypes = [ctypes.c_int] * 6 + [dp] * 16 + [ctypes.c_int]
     return lib
 
 
@@ -100,6 +102,35 @@ def forward(form: str, q, k, v, log_w, e1=None, e2=None, S0=None, n_threads: int
     if rc != 0:
         raise ValueError(f"oracle_forward failed with code {rc}")
     return o, S_T
+
+
+def backward(form: str, q, k, v, log_w, e1=None, e2=None, S0=None, dO=None, dS_T=None,
+             n_threads: int = 0, lib=None):
+    """Gradients of L = <dO, o> + <dS_T, S_T> through the token-by-token recurrence.
+
+    Same inputs as ``forward`` plus ``dO`` [B, T, H, dv] and ``dS_T`` [B, H, dk, dv]
+    (None = 0).  Returns a dict with ``q, k, v, log_w`` (shaped like the inputs),
+    ``e1`` / ``e2`` (None where the form has no such input) and ``S0`` [B, H, dk, dv].
+    """
+    lib = _load() if lib is None else lib
+    q, k, v, log_w, e1, e2, S0, dO, dS_T = map(_f64, (q, k, v, log_w, e1, e2, S0, dO, dS_T))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, T, H, dk) and log_w.shape == (B, T, H, dk)
+    assert v.shape == (B, T, H, dv) and dO is not None and dO.shape == (B, T, H, dv)
+    if dS_T is not None:
+        assert dS_T.shape == (B, H, dk, dv)
+    g = {n: np.zeros_like(x) for n, x in (("q", q), ("k", k), ("v", v), ("log_w", log_w))}
+    g["e1"] = None if e1 is None else np.zeros_like(e1)
+    g["e2"] = None if e2 is None else np.zeros_like(e2)
+    g["S0"] = np.zeros((B, H, dk, dv), dtype=np.float64)
+    rc = lib.oracle_backward(FORMS[form], B, T, H, dk, dv, _ptr(q), _ptr(k), _ptr(v),
+                             _ptr(log_w), _ptr(e1), _ptr(e2), _ptr(S0), _ptr(dO), _ptr(dS_T),
+                             _ptr(g["q"]), _ptr(g["k"]), _ptr(g["v"]), _ptr(g["log_w"]),
+                             _ptr(g["e1"]), _ptr(g["e2"]), _ptr(g["S0"]), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_backward failed with code {rc}")
+    return g
 
 
 def decode_step(form: str, q, k, v, log_w, e1, e2, S, n_threads: int = 0):
