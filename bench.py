@@ -53,6 +53,16 @@ def fwd_algorithmic_bytes(w) -> int:
     return w.B * w.T * w.H * per_token_head + w.B * w.H * w.dk * w.dv * 4
 
 
+def bwd_algorithmic_bytes(w) -> int:
+    """Reverse mode: the forward's token inputs and dO (fp32) in, every gradient out
+    (fp32: q, k, log_w, v and the form's erase arguments)."""
+    eb = 2 if w.dtype == "bf16" else 4
+    extra = {"gdn2": w.dk + w.dv, "rwkv7": w.dk + 1, "general": 2 * w.dk, "gla": 0}[w.form]
+    per_in = eb * (2 * w.dk + w.dv + extra) + 4 * w.dk + 4 * w.dv
+    per_out = 4 * (3 * w.dk + w.dv + extra)
+    return w.B * w.T * w.H * (per_in + per_out) + w.B * w.H * w.dk * w.dv * 4
+
+
 def fwd_flops(w) -> int:
     """Algorithmic flops of the single-write (GDN-2) chunk form per token-head:
     6 d^2 (state GEMMs Y S0, Q S0, K~^T V~) + 5 C d (L, M, [U Y], M V~) + C^2 / 3 (T^-1)."""
@@ -381,6 +391,54 @@ def bench_other_workloads(ctx, args, gdr):
     return out
 
 
+def bench_backward(ctx, args, gdr):
+    """gdr_backward_chunked on the bf16 forward workloads, device-resident (S0 = 0,
+    dS_T = 0, random dO): milliseconds per call and the HBM roofline fraction of the
+    algorithmic bytes (inputs and dO in, every gradient out)."""
+    torch = ctx.torch
+    out = []
+    for name in ("gdn2_bf16", "rwkv7_bf16"):
+        w = synth.PRESETS[name]
+        inp = synth.forward_inputs(w, seed=rank_seed(w.seed, ctx.rank))
+        names = ("q", "k", "v", "log_w", "e1", "e2")
+        d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
+        del inp
+        gen = torch.Generator(device=ctx.dev).manual_seed(rank_seed(w.seed + 100, ctx.rank))
+        dO = torch.randn((w.B, w.T, w.H, w.dv), generator=gen, device=ctx.dev)
+        ws = gdr.new_workspace(gdr.gdr_backward_workspace_size(w.form, d["q"], d["k"], d["v"],
+                                                               d["log_w"], d["e1"], d["e2"]),
+                               ctx.dev)
+        grads = None
+
+        def call():
+            return gdr.gdr_backward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
+                                            d["e2"], None, dO, None, workspace=ws, grads=grads)
+        grads = call()
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = ctx.event(), ctx.event()
+        n = 5
+        e0.record(ctx.stream)
+        for _ in range(n):
+            call()
+        e1.record(ctx.stream)
+        torch.cuda.synchronize()
+        ms = ctx.max_over_ranks(e0.elapsed_time(e1)) / n
+        nbytes = bwd_algorithmic_bytes(w)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.append({"workload": name, "form": w.form, "dtype": w.dtype, "B": w.B, "H": w.H,
+                    "T": w.T, "dk": w.dk, "dv": w.dv, "ms_per_call": ms, "launches_per_call": 3,
+                    "tokens_per_s": w.tokens * ctx.world / (ms * 1e-3),
+                    "workspace_bytes": int(ws.numel()),
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
+                                 "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],
+                                 "bytes_per_call": nbytes}})
+        del d, ws, grads, dO
+        torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(ctx, args, gdr, w, inp, names, step, o):
     """Same call with host inputs: pinned H2D copies, the forward, D2H of o, all timed."""
     torch = ctx.torch
@@ -477,6 +535,8 @@ def main():
                     help="decode batch B (default: the workload's); for profiler captures")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip the timing of the other forward workloads")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the timing of the reverse mode (gdr_backward_chunked)")
     ap.add_argument("--only", default="all", choices=["all", "forward", "decode"],
                     help="time one part only (profiling runs); the default line needs 'all'")
     args = ap.parse_args()
@@ -500,6 +560,10 @@ def main():
 
     fwd = bench_forward(ctx, args, gdr) if args.only in ("all", "forward") else None
     dec = bench_decode(ctx, args, gdr) if args.only in ("all", "decode") else None
+    # every rank times its own shard of these too (same collective steps on all ranks)
+    others = (bench_other_workloads(ctx, args, gdr)
+              if args.only == "all" and not args.no_other_workloads else None)
+    bwd = bench_backward(ctx, args, gdr) if args.only == "all" and not args.no_backward else None
     ctx.barrier()
     if world > 1:
         dist.destroy_process_group()
@@ -542,8 +606,10 @@ def main():
                                     "kind": "oracle", "sample": sample}
     if dec is not None:
         line["decode"] = dec
-    if args.only == "all" and not args.no_other_workloads:
-        line["other_workloads"] = bench_other_workloads(ctx, args, gdr)
+    if others is not None:
+        line["other_workloads"] = others
+    if bwd is not None:
+        line["backward"] = bwd
     print(json.dumps(line), flush=True)
     return 0
 

@@ -174,6 +174,64 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *args, void *stream);
 gdr_status gdr_forward_chunked_noalloc(const gdr_fwd_args *args, void *stream);
 
 /*
+ * Arguments of gdr_backward_chunked: the forward's inputs plus the loss gradient.
+ * With L the caller's loss, dO = dL/do [B][T][H][dv] fp32 (required) and
+ * dS_T = dL/dS_T [B][H][dk][dv] fp32 (NULL = 0).  Outputs g_x = dL/dx, all fp32,
+ * each the full gradient (overwritten, not accumulated):
+ *   g_q, g_k, g_log_w : [B][T][H][dk]          g_v : [B][T][H][dv]
+ *   g_e1              : shaped like e1 (GENERAL, GDN2, RWKV7; NULL for GLA)
+ *   g_e2              : shaped like e2 (GENERAL; RWKV7 [B][T][H]; GDN2 when e2 != NULL)
+ *   g_S0              : [B][H][dk][dv], or NULL when not wanted
+ * GDN2's gradients are those of its raw arguments (k receives the write, erase-key
+ * and erase-vector terms; log_w includes alpha's share in u); RWKV7's those of a
+ * and c.  dtype, shapes and forms as in gdr_fwd_args; dk, dv in {64, 128}.
+ */
+typedef struct {
+  gdr_form form;
+  gdr_dtype dtype;
+  int B, H, T, dk, dv;
+  int chunk;            /* accepted values as gdr_fwd_args; the kernels use 32-token
+                           chunks whatever is passed (the result depends on it only
+                           through rounding)                                          */
+  const void *q, *k, *v;
+  const float *log_w;
+  const void *e1, *e2;
+  const float *S0;      /* initial state of the forward, or NULL (= 0)                */
+  const float *dO;
+  const float *dS_T;
+  float *g_q, *g_k, *g_v, *g_log_w, *g_e1, *g_e2, *g_S0;
+  void *workspace;      /* device scratch of gdr_backward_workspace_size bytes, 256-B aligned */
+  size_t workspace_bytes;
+} gdr_bwd_args;
+
+/* Workspace bytes gdr_backward_chunked needs (host-only, no CUDA call).  About
+ * (2 dk dv / 32 + 5 dk) * 4 bytes per token and head: the chunk-start states, their
+ * adjoints and the per-chunk records of the two chains. */
+gdr_status gdr_backward_workspace_size(const gdr_bwd_args *args, size_t *bytes);
+
+/*
+ * Reverse mode of gdr_forward_chunked: every gradient of L = <dO, o> + <dS_T, S_T>.
+ * Chunkwise adjoint of the same algebra ("Muir ...", section 2.2 and section 4.2
+ * eq. (10): outputs and end state are affine in the chunk's start state, so the
+ * adjoint of the start state is the same affine map transposed, carried backwards
+ * over the chunks).  Per 32-token chunk, with W = T^-1 U~ and the decayed keys
+ * K~, Z~ of the forward:
+ *     S_end   = Diag(pi) S - Z~^T (W S) + (K~ - (T^-1 B)^T Z~)^T V      (forward chain)
+ *     dS      = Diag(pi) dS_end - W^T (Z~ dS_end) + (Q~ - M_z W)^T dO    (adjoint chain)
+ * and the token gradients follow chunk-parallel from S and dS_end by the adjoints
+ * of E = T^-1 (U~ S + B V), O = Q~ S + M_k V - M_z E, S_end = Diag(pi) S + K~^T V - Z~^T E.
+ * The decay gradient is a reverse cumulative sum over the sequence:
+ *     dlog_w_t = sum_{r >= t} (q dq - k dk - z dz + u du)_r - u_t du_t + diag(S_T^T dS_T)
+ * (effective u, z, k of the form; for GDN2 the last two terms cancel the share of
+ * alpha in u).  Products on the tensor cores (tf32 operands with fp32 accumulate;
+ * bf16 inputs use one tf32 product, fp32 inputs three, which keeps fp32 accuracy).
+ * Four kernels, no device waits.  Errors as gdr_forward_chunked; GDR_ERR_UNSUPPORTED
+ * for dk or dv outside {64, 128}; GDR_ERR_WORKSPACE when the workspace is missing
+ * or too small.
+ */
+gdr_status gdr_backward_chunked(const gdr_bwd_args *args, void *stream);
+
+/*
  * Arguments of gdr_decode_step: one token for each (b, h).
  *   q, k, log_w, e1 (GENERAL/GDN2/RWKV7) : [B][H][dk]
  *   v, o, e2 (GDN2)                      : [B][H][dv]

@@ -170,6 +170,70 @@ gdr_status gdr_decode_step(const gdr_step_args *a, void *stream) {
   return cuda_status(gdr::launch_decode(*a, static_cast<cudaStream_t>(stream)));
 }
 
+gdr_status gdr_backward_workspace_size(const gdr_bwd_args *a, size_t *bytes) {
+  if (!a || !bytes) return GDR_ERR_INVALID_ARG;
+  *bytes = kStatusBytes;
+  if (a->B > 0 && a->H > 0 && a->T > 0 && form_ok(a->form) && gdr::backward_supported(a->dk, a->dv))
+    *bytes = gdr::backward_workspace_bytes(a->form, a->B, a->H, a->T, a->dk, a->dv);
+  return GDR_OK;
+}
+
+gdr_status gdr_backward_chunked(const gdr_bwd_args *a, void *stream) {
+  if (!a) return GDR_ERR_INVALID_ARG;
+  if (!form_ok(a->form) || !dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 0 || a->T < 0) return GDR_ERR_INVALID_ARG;
+  if (!chunk_ok(a->chunk)) return GDR_ERR_UNSUPPORTED;
+  if (!dim_ok(a->dk) || !dim_ok(a->dv)) return GDR_ERR_UNSUPPORTED;
+  if (!gdr::backward_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
+  const size_t tokens = (size_t)a->B * a->T * a->H;
+  gdr_status st = check_token_ptrs(a->form, tokens, a->q, a->k, a->v, a->log_w, a->e1, a->e2,
+                                   a->dO);
+  if (st != GDR_OK) return st;
+  if (tokens > 0) {
+    if (!a->g_q || !a->g_k || !a->g_v || !a->g_log_w) return GDR_ERR_INVALID_ARG;
+    if (needs_e1(a->form) && !a->g_e1) return GDR_ERR_INVALID_ARG;
+    if (a->e2 && a->form != GDR_FORM_GLA && !a->g_e2) return GDR_ERR_INVALID_ARG;
+  }
+  const void *outs[] = {a->S0, a->dS_T, a->g_q, a->g_k, a->g_v, a->g_log_w, a->g_e1, a->g_e2,
+                        a->g_S0};
+  for (const void *p : outs)
+    if (p && !aligned16(p)) return GDR_ERR_MISALIGNED;
+  if (a->B == 0 || a->H == 0) return GDR_OK;
+  if (a->T == 0) {  // no tokens: dL/dS0 = dS_T
+    if (!a->g_S0) return GDR_OK;
+    return gdr_state_init(a->g_S0, a->B, a->H, a->dk, a->dv, a->dS_T, stream);
+  }
+  const size_t need = gdr::backward_workspace_bytes(a->form, a->B, a->H, a->T, a->dk, a->dv);
+  if (!a->workspace || a->workspace_bytes < need) return GDR_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return GDR_ERR_MISALIGNED;
+  gdr::BwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.form = a->form;
+  p.B = a->B;
+  p.H = a->H;
+  p.T = a->T;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.e1 = a->e1;
+  p.e2 = a->form == GDR_FORM_GLA ? nullptr : a->e2;
+  p.log_w = a->log_w;
+  p.S0 = a->S0;
+  p.dO = a->dO;
+  p.dS_T = a->dS_T;
+  p.gq = a->g_q;
+  p.gk = a->g_k;
+  p.gv = a->g_v;
+  p.glw = a->g_log_w;
+  p.ge1 = a->g_e1;
+  p.ge2 = a->g_e2;
+  p.gS0 = a->g_S0;
+  return cuda_status(gdr::launch_backward(p, a->dtype, a->workspace,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 gdr_status gdr_read_status(void *workspace, void *stream, gdr_status *device_status) {
   if (!workspace || !device_status) return GDR_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

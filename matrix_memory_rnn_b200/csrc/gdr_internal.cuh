@@ -64,6 +64,24 @@ struct FwdParams {
 // group never hands its chunks to the back group, whose bounded wait then runs out.
 constexpr uint32_t kDebugSkipHandoff = 1u;
 
+// Reverse mode (gdr_backward_chunked).  Chunks of kBwdChunk tokens, nc of them per
+// sequence; the workspace sections hold, per chunk, the records of the two chains
+// (rec), the chunk-start states plus the final state (states, nc + 1 per sequence)
+// and the adjoints of the chunk-end states (adj).
+constexpr int kBwdChunk = 32;
+struct BwdParams {
+  gdr_form form;
+  int B, H, T, dk, dv, nc;
+  const void *q, *k, *v, *e1, *e2;
+  const float *log_w, *S0, *dO, *dS_T;
+  float *gq, *gk, *gv, *glw, *ge1, *ge2, *gS0;
+  float *rec, *states, *adj;
+};
+size_t backward_workspace_bytes(int form, int B, int H, int T, int dk, int dv);
+bool backward_supported(int dk, int dv);
+cudaError_t launch_backward(const BwdParams &p, gdr_dtype dtype, void *workspace,
+                            cudaStream_t stream);
+
 // Launchers (host).  Return cudaSuccess or the launch error.
 cudaError_t launch_decode(const gdr_step_args &a, cudaStream_t stream);
 cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_t stream);

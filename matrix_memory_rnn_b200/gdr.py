@@ -40,6 +40,15 @@ class gdr_step_args(ctypes.Structure):
                 ("log_w", _fp), ("e1", _vp), ("e2", _vp), ("S", _fp), ("o", _fp)]
 
 
+class gdr_bwd_args(ctypes.Structure):
+    _fields_ = [("form", _c_int), ("dtype", _c_int), ("B", _c_int), ("H", _c_int),
+                ("T", _c_int), ("dk", _c_int), ("dv", _c_int), ("chunk", _c_int),
+                ("q", _vp), ("k", _vp), ("v", _vp), ("log_w", _fp), ("e1", _vp), ("e2", _vp),
+                ("S0", _fp), ("dO", _fp), ("dS_T", _fp), ("g_q", _fp), ("g_k", _fp),
+                ("g_v", _fp), ("g_log_w", _fp), ("g_e1", _fp), ("g_e2", _fp), ("g_S0", _fp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 class GdrError(RuntimeError):
     def __init__(self, fn, code):
         self.code = int(code)
@@ -61,12 +70,16 @@ def _load():
             lib.gdr_forward_chunked.argtypes = [ctypes.POINTER(gdr_fwd_args), _vp]
             lib.gdr_forward_workspace_size.argtypes = [ctypes.POINTER(gdr_fwd_args),
                                                        ctypes.POINTER(ctypes.c_size_t)]
+            lib.gdr_backward_chunked.argtypes = [ctypes.POINTER(gdr_bwd_args), _vp]
+            lib.gdr_backward_workspace_size.argtypes = [ctypes.POINTER(gdr_bwd_args),
+                                                        ctypes.POINTER(ctypes.c_size_t)]
             lib.gdr_decode_step.argtypes = [ctypes.POINTER(gdr_step_args), _vp]
             lib.gdr_state_init.argtypes = [_fp, _c_int, _c_int, _c_int, _c_int, _fp, _vp]
             lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
             lib.gdr_status_string.restype = ctypes.c_char_p
             lib.gdr_status_string.argtypes = [_c_int]
-            for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size", "gdr_decode_step",
+            for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size",
+                       "gdr_backward_chunked", "gdr_backward_workspace_size", "gdr_decode_step",
                        "gdr_state_init", "gdr_read_status", "gdr_version"):
                 getattr(lib, fn).restype = _c_int
             _lib = lib
@@ -188,6 +201,92 @@ def gdr_forward_chunked(form, q, k, v, log_w, e1=None, e2=None, S0=None, *, chun
     a = _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, workspace)
     _check("gdr_forward_chunked", _load().gdr_forward_chunked(ctypes.byref(a), _stream(stream)))
     return o, S_T
+
+
+def _bwd_struct(form, q, k, v, log_w, e1, e2, S0, dO, dS_T, grads, chunk, workspace):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dname, tdt = _dtype_of(q)
+    _need(q, "q", tdt, (B, T, H, dk))
+    _need(k, "k", tdt, (B, T, H, dk))
+    _need(v, "v", tdt, (B, T, H, dv))
+    _need(log_w, "log_w", torch.float32, (B, T, H, dk))
+    s1, s2 = _e_shapes(form, (B, T, H), dk, dv)
+    if s1 is not None:
+        _need(e1, "e1", tdt, s1)
+    if e2 is not None or form in ("general", "rwkv7"):
+        _need(e2, "e2", tdt, s2)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv))
+    _need(dO, "dO", torch.float32, (B, T, H, dv))
+    if dS_T is not None:
+        _need(dS_T, "dS_T", torch.float32, (B, H, dk, dv))
+    a = gdr_bwd_args()
+    a.form, a.dtype = FORMS[form], DTYPES[dname]
+    a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, dv, chunk
+    a.q, a.k, a.v, a.log_w = _ptr(q), _ptr(k), _ptr(v), _ptr(log_w)
+    a.e1, a.e2, a.S0, a.dO, a.dS_T = _ptr(e1), _ptr(e2), _ptr(S0), _ptr(dO), _ptr(dS_T)
+    if grads is not None:
+        for name in ("q", "k", "v", "log_w", "e1", "e2", "S0"):
+            setattr(a, "g_" + name, _ptr(grads.get(name)))
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    return a
+
+
+def gdr_backward_workspace_size(form, q, k, v, log_w, e1=None, e2=None, chunk=64):
+    """Bytes of device workspace ``gdr_backward_chunked`` needs for these inputs."""
+    B, T, H, dk = q.shape
+    a = gdr_bwd_args()
+    a.form, a.dtype = FORMS[form], DTYPES[_dtype_of(q)[0]]
+    a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, v.shape[-1], chunk
+    n = ctypes.c_size_t(0)
+    _check("gdr_backward_workspace_size",
+           _load().gdr_backward_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    return int(n.value)
+
+
+def gdr_backward_chunked(form, q, k, v, log_w, e1=None, e2=None, S0=None, dO=None, dS_T=None, *,
+                         chunk=64, want_S0=True, grads=None, workspace=None, stream=None):
+    """Reverse mode of ``gdr_forward_chunked``: gradients of <dO, o> + <dS_T, S_T>.
+
+    Returns a dict with fp32 tensors ``q, k, v, log_w`` (shaped like the inputs),
+    ``e1`` / ``e2`` (None where the form has no such input) and ``S0`` [B, H, dk, dv]
+    (None when ``want_S0`` is False).  ``grads`` may hold preallocated outputs.
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    g = dict(grads or {})
+
+    def out(name, shape):
+        if g.get(name) is None:
+            g[name] = torch.empty(shape, dtype=torch.float32, device=dev)
+        _need(g[name], "grad " + name, torch.float32, shape)
+
+    out("q", (B, T, H, dk))
+    out("k", (B, T, H, dk))
+    out("v", (B, T, H, dv))
+    out("log_w", (B, T, H, dk))
+    s1, s2 = _e_shapes(form, (B, T, H), dk, dv)
+    if s1 is not None:
+        out("e1", s1)
+    else:
+        g["e1"] = None
+    if s2 is not None and (e2 is not None or form in ("general", "rwkv7")):
+        out("e2", s2)
+    else:
+        g["e2"] = None
+    if want_S0:
+        out("S0", (B, H, dk, dv))
+    else:
+        g["S0"] = None
+    if workspace is None:
+        workspace = new_workspace(gdr_backward_workspace_size(form, q, k, v, log_w, e1, e2, chunk),
+                                  dev)
+    a = _bwd_struct(form, q, k, v, log_w, e1, e2, S0, dO, dS_T, g, chunk, workspace)
+    _check("gdr_backward_chunked", _load().gdr_backward_chunked(ctypes.byref(a), _stream(stream)))
+    return g
 
 
 def gdr_decode_step(form, q, k, v, log_w, e1, e2, S, *, o=None, stream=None):
