@@ -397,8 +397,10 @@ def bench_backward(ctx, args, gdr):
     algorithmic bytes (inputs and dO in, every gradient out)."""
     torch = ctx.torch
     out = []
-    for name in ("gdn2_bf16", "rwkv7_bf16"):
+    for name in ((args.bwd_workload,) if args.bwd_workload else ("gdn2_bf16", "rwkv7_bf16")):
         w = synth.PRESETS[name]
+        if args.bwd_batch:
+            w = w.with_(B=args.bwd_batch)
         inp = synth.forward_inputs(w, seed=rank_seed(w.seed, ctx.rank))
         names = ("q", "k", "v", "log_w", "e1", "e2")
         d = gdr.to_device({k: inp[k] for k in names}, w.dtype, ctx.dev)
@@ -537,7 +539,11 @@ def main():
                     help="skip the timing of the other forward workloads")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the timing of the reverse mode (gdr_backward_chunked)")
-    ap.add_argument("--only", default="all", choices=["all", "forward", "decode"],
+    ap.add_argument("--bwd-workload", default=None, choices=["gdn2_bf16", "rwkv7_bf16"],
+                    help="reverse-mode workload (default: both); for profiler captures")
+    ap.add_argument("--bwd-batch", type=int, default=None,
+                    help="reverse-mode batch B (default: the workload's); for profiler captures")
+    ap.add_argument("--only", default="all", choices=["all", "forward", "decode", "backward"],
                     help="time one part only (profiling runs); the default line needs 'all'")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -563,7 +569,8 @@ def main():
     # every rank times its own shard of these too (same collective steps on all ranks)
     others = (bench_other_workloads(ctx, args, gdr)
               if args.only == "all" and not args.no_other_workloads else None)
-    bwd = bench_backward(ctx, args, gdr) if args.only == "all" and not args.no_backward else None
+    bwd = (bench_backward(ctx, args, gdr)
+           if (args.only == "all" and not args.no_backward) or args.only == "backward" else None)
     ctx.barrier()
     if world > 1:
         dist.destroy_process_group()
