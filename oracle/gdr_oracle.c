@@ -359,3 +359,89 @@ int oracle_backward(int form, int B, int T, int H, int dk, int dv,
   }
   return failed ? -2 : 0;
 }
+
+/*
+ * The Muir token mixer around the recurrence ("Muir ...", section 2.1 and section 4,
+ * eqs. (8)-(9)): from pre-activations (after the projections and the depthwise causal
+ * convolution) and gate logits,
+ *
+ *     q = l2norm(silu(q_pre)),  k = l2norm(silu(k_pre))  (per head, over d_k),  v = silu(v_pre)
+ *     log alpha = -exp(a_log[h]) softplus(z_f),  b = 2 sigmoid(z_b),  w = sigmoid(z_w),
+ *     gamma = gamma_stat (.) 2 sigmoid(z_q),     g = z_g
+ *     GDN-2 recurrence with q^ = gamma (.) q, erase gate b, write gate w, decay alpha
+ *     y_t = rmsnorm(o_t) (.) silu(g_t),  rmsnorm(o)_c = rho_c o_c / sqrt(mean_c o_c^2 + eps)
+ *
+ * l2norm(x) = x / max(||x||, 1e-12) (a zero vector stays zero).  gamma_stat [H][dk] and
+ * rho [dv] may be NULL (all ones).  Inputs [B][T][H][.] as oracle_forward; a_log [H].
+ * Outputs y [B][T][H][dv] and, if S_T != NULL, the final state.  Returns as oracle_forward.
+ */
+static double silu(double x) { return x / (1.0 + exp(-x)); }
+static double sigm(double x) { return 1.0 / (1.0 + exp(-x)); }
+static double softplus(double x) { return x > 30.0 ? x : log1p(exp(x)); }
+
+int oracle_muir_forward(int B, int T, int H, int dk, int dv,
+                        const double *q_pre, const double *k_pre, const double *v_pre,
+                        const double *zf, const double *zb, const double *zw,
+                        const double *zq, const double *zg, const double *a_log,
+                        const double *gamma_stat, const double *rho, double eps,
+                        const double *S0, double *y, double *S_T, int n_threads) {
+  if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+  if (T > 0 && (!q_pre || !k_pre || !v_pre || !zf || !zb || !zw || !zq || !zg || !a_log || !y))
+    return -1;
+  const size_t nk = (size_t)B * T * H * dk, nv = (size_t)B * T * H * dv;
+  double *q = (double *)calloc(nk ? nk : 1, sizeof(double));
+  double *k = (double *)calloc(nk ? nk : 1, sizeof(double));
+  double *v = (double *)calloc(nv ? nv : 1, sizeof(double));
+  double *lw = (double *)calloc(nk ? nk : 1, sizeof(double));
+  double *bg = (double *)calloc(nk ? nk : 1, sizeof(double));
+  double *wg = (double *)calloc(nv ? nv : 1, sizeof(double));
+  double *o = (double *)calloc(nv ? nv : 1, sizeof(double));
+  int rc = -2;
+  if (!q || !k || !v || !lw || !bg || !wg || !o) goto done;
+  for (size_t tok = 0; tok < (size_t)B * T * H; ++tok) {
+    const int h = (int)(tok % H);
+    const size_t ok = tok * dk, ov = tok * dv;
+    double nq = 0.0, nk2 = 0.0;
+    for (int j = 0; j < dk; ++j) {
+      q[ok + j] = silu(q_pre[ok + j]);
+      k[ok + j] = silu(k_pre[ok + j]);
+      nq += q[ok + j] * q[ok + j];
+      nk2 += k[ok + j] * k[ok + j];
+    }
+    nq = sqrt(nq);
+    nk2 = sqrt(nk2);
+    if (nq < 1e-12) nq = 1e-12;
+    if (nk2 < 1e-12) nk2 = 1e-12;
+    const double rate = exp(a_log[h]);
+    for (int j = 0; j < dk; ++j) {
+      const double gam = (gamma_stat ? gamma_stat[(size_t)h * dk + j] : 1.0) * 2.0 * sigm(zq[ok + j]);
+      q[ok + j] = gam * q[ok + j] / nq;
+      k[ok + j] /= nk2;
+      lw[ok + j] = -rate * softplus(zf[ok + j]);
+      bg[ok + j] = 2.0 * sigm(zb[ok + j]);
+    }
+    for (int c = 0; c < dv; ++c) {
+      v[ov + c] = silu(v_pre[ov + c]);
+      wg[ov + c] = sigm(zw[ov + c]);
+    }
+  }
+  rc = oracle_forward(OR_GDN2, B, T, H, dk, dv, q, k, v, lw, bg, wg, S0, o, S_T, n_threads);
+  if (rc != 0) goto done;
+  for (size_t tok = 0; tok < (size_t)B * T * H; ++tok) {
+    const size_t ov = tok * dv;
+    double ms = 0.0;
+    for (int c = 0; c < dv; ++c) ms += o[ov + c] * o[ov + c];
+    const double inv = 1.0 / sqrt(ms / dv + eps);
+    for (int c = 0; c < dv; ++c)
+      y[ov + c] = (rho ? rho[c] : 1.0) * o[ov + c] * inv * silu(zg[ov + c]);
+  }
+done:
+  free(q);
+  free(k);
+  free(v);
+  free(lw);
+  free(bg);
+  free(wg);
+  free(o);
+  return rc;
+}

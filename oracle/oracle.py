@@ -48,6 +48,9 @@ def load_library(path: str):
     lib.oracle_forward.restype = ctypes.c_int
     lib.oracle_forward.argtypes = [ctypes.c_int] * 6 + [dp] * 9 + [ctypes.c_int]
     lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_muir_forward.restype = ctypes.c_int
+    lib.oracle_muir_forward.argtypes = ([ctypes.c_int] * 5 + [dp] * 11 + [ctypes.c_double] +
+                                        [dp] * 3 + [ctypes.c_int])
     lib.oracle_backward.restype = ctypes.c_int
     lib.oracle_backward.argtypes = [ctypes.c_int] * 6 + [dp] * 16 + [ctypes.c_int]
     return lib
@@ -131,6 +134,30 @@ def backward(form: str, q, k, v, log_w, e1=None, e2=None, S0=None, dO=None, dS_T
     if rc != 0:
         raise ValueError(f"oracle_backward failed with code {rc}")
     return g
+
+
+def muir_forward(q_pre, k_pre, v_pre, zf, zb, zw, zq, zg, a_log, gamma_stat=None, rho=None,
+                 eps=1e-6, S0=None, n_threads: int = 0, lib=None):
+    """The Muir token mixer around the GDN-2 recurrence (``oracle_muir_forward``):
+    pre-activations and gate logits [B, T, H, .], a_log [H], gamma_stat [H, dk] or None,
+    rho [dv] or None.  Returns ``(y [B, T, H, dv], S_T [B, H, dk, dv])``."""
+    lib = _load() if lib is None else lib
+    arrs = map(_f64, (q_pre, k_pre, v_pre, zf, zb, zw, zq, zg, a_log, gamma_stat, rho, S0))
+    q_pre, k_pre, v_pre, zf, zb, zw, zq, zg, a_log, gamma_stat, rho, S0 = arrs
+    B, T, H, dk = q_pre.shape
+    dv = v_pre.shape[-1]
+    for a, d in ((k_pre, dk), (zf, dk), (zb, dk), (zq, dk), (v_pre, dv), (zw, dv), (zg, dv)):
+        assert a.shape == (B, T, H, d)
+    assert a_log.shape == (H,)
+    y = np.zeros((B, T, H, dv), dtype=np.float64)
+    S_T = np.zeros((B, H, dk, dv), dtype=np.float64)
+    rc = lib.oracle_muir_forward(B, T, H, dk, dv, _ptr(q_pre), _ptr(k_pre), _ptr(v_pre), _ptr(zf),
+                                 _ptr(zb), _ptr(zw), _ptr(zq), _ptr(zg), _ptr(a_log),
+                                 _ptr(gamma_stat), _ptr(rho), float(eps), _ptr(S0), _ptr(y),
+                                 _ptr(S_T), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_muir_forward failed with code {rc}")
+    return y, S_T
 
 
 def decode_step(form: str, q, k, v, log_w, e1, e2, S, n_threads: int = 0):
