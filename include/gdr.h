@@ -232,6 +232,52 @@ gdr_status gdr_backward_workspace_size(const gdr_bwd_args *args, size_t *bytes);
 gdr_status gdr_backward_chunked(const gdr_bwd_args *args, void *stream);
 
 /*
+ * Arguments of gdr_muir_forward: the Muir token mixer around the GDN-2 recurrence
+ * ("Muir ...", section 2.1 and section 4.1, eqs. (8)-(9)), from the activations that
+ * leave the projections and the depthwise causal convolution:
+ *   q, k, zf, zb, zq : [B][T][H][dk]      v, zw, zg : [B][T][H][dv]     (element type dtype)
+ *   a_log            : [H] fp32, the per-head log decay rate
+ *   gamma_stat       : [H][dk] fp32 static readout gain, or NULL (= 1)
+ *   rms_weight       : [dv] fp32 RMSNorm weight shared by the heads, or NULL (= 1)
+ *   y                : [B][T][H][dv] fp32, required;  S0, S_T as gdr_fwd_args
+ * It computes, per token and head,
+ *   q^ = gamma_stat (.) 2 sigmoid(zq) (.) l2norm(silu(q)),  k^ = l2norm(silu(k)),  v^ = silu(v)
+ *   log alpha = -exp(a_log) softplus(zf),  b = 2 sigmoid(zb),  w = sigmoid(zw)
+ *   o = the GDN-2 recurrence on (q^, k^, v^, log alpha, b, w)   (as gdr_forward_chunked)
+ *   y = rms_weight (.) o / sqrt(mean_c o_c^2 + rms_eps) (.) silu(zg)
+ * with l2norm(x) = x / max(||x||_2, 1e-12).
+ */
+typedef struct {
+  gdr_dtype dtype;
+  int B, H, T, dk, dv, chunk;
+  gdr_algo algo;
+  const void *q, *k, *v;
+  const void *zf, *zb, *zw, *zq, *zg;
+  const float *a_log;
+  const float *gamma_stat;
+  const float *rms_weight;
+  float rms_eps;
+  const float *S0;
+  float *y;
+  float *S_T;
+  void *workspace;      /* device scratch of gdr_muir_workspace_size bytes, 256-B aligned */
+  size_t workspace_bytes;
+} gdr_muir_args;
+
+/* Workspace bytes gdr_muir_forward needs (host-only, no CUDA call). */
+gdr_status gdr_muir_workspace_size(const gdr_muir_args *args, size_t *bytes);
+
+/*
+ * The Muir mixer above.  For bf16 inputs with dk = dv = 128 (algo AUTO or TC) the
+ * activations run inside the tensor-core forward's chunk-parallel kernel, on the tiles
+ * it loads (no activated copy of the inputs is written), and one light kernel applies
+ * RMSNorm (.) SiLU(zg) to o; elsewhere a prologue kernel writes the activated inputs
+ * into the workspace, gdr_forward_chunked runs on them, and the same epilogue follows.
+ * Errors as gdr_forward_chunked.
+ */
+gdr_status gdr_muir_forward(const gdr_muir_args *args, void *stream);
+
+/*
  * Arguments of gdr_decode_step: one token for each (b, h).
  *   q, k, log_w, e1 (GENERAL/GDN2/RWKV7) : [B][H][dk]
  *   v, o, e2 (GDN2)                      : [B][H][dv]

@@ -70,6 +70,49 @@ bool uses_tc_general(const gdr_fwd_args *a, const gdr::FwdParams &p) {
          gdr::forward_tc_general_supported(p, a->dtype);
 }
 
+// Workspace of gdr_muir_forward: the forward's own workspace, then (generic path) the
+// activated inputs and o, each section 256-byte aligned.
+struct MuirLayout {
+  size_t fwd, qh, kh, bh, vh, wh, lw, o, total;
+};
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+gdr_fwd_args muir_fwd_args(const gdr_muir_args *a) {
+  gdr_fwd_args f;
+  memset(&f, 0, sizeof(f));
+  f.form = GDR_FORM_GDN2;
+  f.dtype = a->dtype;
+  f.B = a->B;
+  f.H = a->H;
+  f.T = a->T;
+  f.dk = a->dk;
+  f.dv = a->dv;
+  f.chunk = a->chunk;
+  f.algo = a->algo;
+  f.S0 = a->S0;
+  f.S_T = a->S_T;
+  return f;
+}
+
+MuirLayout muir_layout(const gdr_muir_args *a) {
+  MuirLayout L;
+  const gdr_fwd_args f = muir_fwd_args(a);
+  size_t fwd = kStatusBytes;
+  gdr_forward_workspace_size(&f, &fwd);
+  const size_t n = (size_t)a->B * a->T * a->H, eb = a->dtype == GDR_BF16 ? 2 : 4;
+  size_t off = 0;
+  L.fwd = off; off = align256(off + fwd);
+  L.qh = off; off = align256(off + n * a->dk * eb);
+  L.kh = off; off = align256(off + n * a->dk * eb);
+  L.bh = off; off = align256(off + n * a->dk * eb);
+  L.vh = off; off = align256(off + n * a->dv * eb);
+  L.wh = off; off = align256(off + n * a->dv * eb);
+  L.lw = off; off = align256(off + n * a->dk * 4);
+  L.o = off; off = align256(off + n * a->dv * 4);
+  L.total = off;
+  return L;
+}
+
 }  // namespace
 
 extern "C" {
@@ -232,6 +275,80 @@ gdr_status gdr_backward_chunked(const gdr_bwd_args *a, void *stream) {
   p.gS0 = a->g_S0;
   return cuda_status(gdr::launch_backward(p, a->dtype, a->workspace,
                                           static_cast<cudaStream_t>(stream)));
+}
+
+gdr_status gdr_muir_workspace_size(const gdr_muir_args *a, size_t *bytes) {
+  if (!a || !bytes) return GDR_ERR_INVALID_ARG;
+  *bytes = kStatusBytes;
+  if (a->B > 0 && a->H > 0 && a->T > 0 && dtype_ok(a->dtype) && dim_ok(a->dk) && dim_ok(a->dv))
+    *bytes = muir_layout(a).total;
+  return GDR_OK;
+}
+
+gdr_status gdr_muir_forward(const gdr_muir_args *a, void *stream) {
+  if (!a) return GDR_ERR_INVALID_ARG;
+  if (!dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 0 || a->T < 0) return GDR_ERR_INVALID_ARG;
+  if (!dim_ok(a->dk) || !dim_ok(a->dv) || !chunk_ok(a->chunk)) return GDR_ERR_UNSUPPORTED;
+  if (a->algo < GDR_ALGO_AUTO || a->algo > GDR_ALGO_TC) return GDR_ERR_INVALID_ARG;
+  if (!(a->rms_eps >= 0.f)) return GDR_ERR_INVALID_ARG;
+  const size_t tokens = (size_t)a->B * a->T * a->H;
+  if (tokens > 0) {
+    const void *need[] = {a->q, a->k, a->v, a->zf, a->zb, a->zw, a->zq, a->zg, a->a_log, a->y};
+    for (const void *p : need)
+      if (!p) return GDR_ERR_INVALID_ARG;
+    const void *al[] = {a->q, a->k, a->v, a->zf, a->zb, a->zw, a->zq, a->zg, a->y};
+    for (const void *p : al)
+      if (!aligned16(p)) return GDR_ERR_MISALIGNED;
+  }
+  if ((a->S0 && !aligned16(a->S0)) || (a->S_T && !aligned16(a->S_T))) return GDR_ERR_MISALIGNED;
+  if (a->B == 0 || a->H == 0) return GDR_OK;
+  if (a->T == 0) {
+    if (!a->S_T) return GDR_OK;
+    return gdr_state_init(a->S_T, a->B, a->H, a->dk, a->dv, a->S0, stream);
+  }
+  const MuirLayout L = muir_layout(a);
+  if (!a->workspace || a->workspace_bytes < L.total) return GDR_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(a->workspace) & 255u) return GDR_ERR_MISALIGNED;
+  uint8_t *ws = static_cast<uint8_t *>(a->workspace);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gdr::MuirParams m;
+  m.B = a->B;
+  m.H = a->H;
+  m.T = a->T;
+  m.dk = a->dk;
+  m.dv = a->dv;
+  m.q = a->q;
+  m.k = a->k;
+  m.v = a->v;
+  m.zf = a->zf;
+  m.zb = a->zb;
+  m.zw = a->zw;
+  m.zq = a->zq;
+  m.zg = a->zg;
+  m.a_log = a->a_log;
+  m.gamma_stat = a->gamma_stat;
+  m.rms_weight = a->rms_weight;
+  m.rms_eps = a->rms_eps;
+  float *o = reinterpret_cast<float *>(ws + L.o);
+  // activated inputs, then the GDN-2 forward on them, then the readout
+  gdr_status st = cuda_status(gdr::launch_muir_prologue(
+      m, a->dtype, ws + L.qh, ws + L.kh, ws + L.vh, ws + L.bh, ws + L.wh,
+      reinterpret_cast<float *>(ws + L.lw), s));
+  if (st != GDR_OK) return st;
+  gdr_fwd_args f = muir_fwd_args(a);
+  f.q = ws + L.qh;
+  f.k = ws + L.kh;
+  f.v = ws + L.vh;
+  f.log_w = reinterpret_cast<const float *>(ws + L.lw);
+  f.e1 = ws + L.bh;
+  f.e2 = ws + L.wh;
+  f.o = o;
+  f.workspace = ws + L.fwd;
+  f.workspace_bytes = L.qh - L.fwd;
+  st = gdr_forward_chunked(&f, stream);
+  if (st != GDR_OK) return st;
+  return cuda_status(gdr::launch_muir_epilogue(m, a->dtype, o, a->y, s));
 }
 
 gdr_status gdr_read_status(void *workspace, void *stream, gdr_status *device_status) {

@@ -82,6 +82,20 @@ bool backward_supported(int dk, int dv);
 cudaError_t launch_backward(const BwdParams &p, gdr_dtype dtype, void *workspace,
                             cudaStream_t stream);
 
+// The Muir token mixer (gdr_muir_forward): raw activations and gate logits.
+struct MuirParams {
+  int B, H, T, dk, dv;
+  const void *q, *k, *v, *zf, *zb, *zw, *zq, *zg;
+  const float *a_log, *gamma_stat, *rms_weight;
+  float rms_eps;
+};
+// Prologue into activated inputs of the GDN-2 forward (q^, k^, v^, b, w at the input
+// type; log alpha fp32), and the RMSNorm (.) SiLU(zg) epilogue of o into y.
+cudaError_t launch_muir_prologue(const MuirParams &m, gdr_dtype dtype, void *qh, void *kh,
+                                 void *vh, void *b, void *w, float *log_w, cudaStream_t stream);
+cudaError_t launch_muir_epilogue(const MuirParams &m, gdr_dtype dtype, const float *o, float *y,
+                                 cudaStream_t stream);
+
 // Launchers (host).  Return cudaSuccess or the launch error.
 cudaError_t launch_decode(const gdr_step_args &a, cudaStream_t stream);
 cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_t stream);

@@ -49,6 +49,15 @@ class gdr_bwd_args(ctypes.Structure):
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class gdr_muir_args(ctypes.Structure):
+    _fields_ = [("dtype", _c_int), ("B", _c_int), ("H", _c_int), ("T", _c_int), ("dk", _c_int),
+                ("dv", _c_int), ("chunk", _c_int), ("algo", _c_int), ("q", _vp), ("k", _vp),
+                ("v", _vp), ("zf", _vp), ("zb", _vp), ("zw", _vp), ("zq", _vp), ("zg", _vp),
+                ("a_log", _fp), ("gamma_stat", _fp), ("rms_weight", _fp),
+                ("rms_eps", ctypes.c_float), ("S0", _fp), ("y", _fp), ("S_T", _fp),
+                ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
+
+
 class GdrError(RuntimeError):
     def __init__(self, fn, code):
         self.code = int(code)
@@ -73,13 +82,17 @@ def _load():
             lib.gdr_backward_chunked.argtypes = [ctypes.POINTER(gdr_bwd_args), _vp]
             lib.gdr_backward_workspace_size.argtypes = [ctypes.POINTER(gdr_bwd_args),
                                                         ctypes.POINTER(ctypes.c_size_t)]
+            lib.gdr_muir_forward.argtypes = [ctypes.POINTER(gdr_muir_args), _vp]
+            lib.gdr_muir_workspace_size.argtypes = [ctypes.POINTER(gdr_muir_args),
+                                                    ctypes.POINTER(ctypes.c_size_t)]
             lib.gdr_decode_step.argtypes = [ctypes.POINTER(gdr_step_args), _vp]
             lib.gdr_state_init.argtypes = [_fp, _c_int, _c_int, _c_int, _c_int, _fp, _vp]
             lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
             lib.gdr_status_string.restype = ctypes.c_char_p
             lib.gdr_status_string.argtypes = [_c_int]
             for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size",
-                       "gdr_backward_chunked", "gdr_backward_workspace_size", "gdr_decode_step",
+                       "gdr_backward_chunked", "gdr_backward_workspace_size",
+                       "gdr_muir_forward", "gdr_muir_workspace_size", "gdr_decode_step",
                        "gdr_state_init", "gdr_read_status", "gdr_version"):
                 getattr(lib, fn).restype = _c_int
             _lib = lib
@@ -287,6 +300,70 @@ def gdr_backward_chunked(form, q, k, v, log_w, e1=None, e2=None, S0=None, dO=Non
     a = _bwd_struct(form, q, k, v, log_w, e1, e2, S0, dO, dS_T, g, chunk, workspace)
     _check("gdr_backward_chunked", _load().gdr_backward_chunked(ctypes.byref(a), _stream(stream)))
     return g
+
+
+def _muir_struct(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat, rms_weight, rms_eps, S0, y,
+                 S_T, chunk, algo, workspace):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dname, tdt = _dtype_of(q)
+    for t, name, d in ((q, "q", dk), (k, "k", dk), (zf, "zf", dk), (zb, "zb", dk), (zq, "zq", dk),
+                       (v, "v", dv), (zw, "zw", dv), (zg, "zg", dv)):
+        _need(t, name, tdt, (B, T, H, d))
+    _need(a_log, "a_log", torch.float32, (H,))
+    if gamma_stat is not None:
+        _need(gamma_stat, "gamma_stat", torch.float32, (H, dk))
+    if rms_weight is not None:
+        _need(rms_weight, "rms_weight", torch.float32, (dv,))
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dk, dv))
+    if y is not None:
+        _need(y, "y", torch.float32, (B, T, H, dv))
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (B, H, dk, dv))
+    a = gdr_muir_args()
+    a.dtype, a.algo = DTYPES[dname], ALGOS[algo]
+    a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, dv, chunk
+    for name, t in (("q", q), ("k", k), ("v", v), ("zf", zf), ("zb", zb), ("zw", zw), ("zq", zq),
+                    ("zg", zg), ("a_log", a_log), ("gamma_stat", gamma_stat),
+                    ("rms_weight", rms_weight), ("S0", S0), ("y", y), ("S_T", S_T)):
+        setattr(a, name, _ptr(t))
+    a.rms_eps = float(rms_eps)
+    if workspace is not None:
+        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    return a
+
+
+def gdr_muir_workspace_size(q, k, v, chunk=64, algo="auto"):
+    """Bytes of device workspace ``gdr_muir_forward`` needs for inputs of these shapes."""
+    B, T, H, dk = q.shape
+    a = gdr_muir_args()
+    a.dtype, a.algo = DTYPES[_dtype_of(q)[0]], ALGOS[algo]
+    a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, v.shape[-1], chunk
+    n = ctypes.c_size_t(0)
+    _check("gdr_muir_workspace_size",
+           _load().gdr_muir_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    return int(n.value)
+
+
+def gdr_muir_forward(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat=None, rms_weight=None,
+                     rms_eps=1e-6, S0=None, *, chunk=64, algo="auto", y=None, S_T=None,
+                     want_state=True, workspace=None, stream=None):
+    """The Muir token mixer around the GDN-2 recurrence (include/gdr.h, gdr_muir_forward):
+    pre-activations q, k, v and gate logits zf, zb, zw, zq, zg [B, T, H, .] (bf16 or fp32),
+    a_log [H], optional gamma_stat [H, dk] and rms_weight [dv] (fp32).  Returns (y, S_T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if y is None:
+        y = torch.empty((B, T, H, dv), dtype=torch.float32, device=q.device)
+    if S_T is None and want_state:
+        S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = new_workspace(gdr_muir_workspace_size(q, k, v, chunk, algo), q.device)
+    a = _muir_struct(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat, rms_weight, rms_eps, S0, y,
+                     S_T, chunk, algo, workspace)
+    _check("gdr_muir_forward", _load().gdr_muir_forward(ctypes.byref(a), _stream(stream)))
+    return y, S_T
 
 
 def gdr_decode_step(form, q, k, v, log_w, e1, e2, S, *, o=None, stream=None):

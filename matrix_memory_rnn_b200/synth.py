@@ -25,7 +25,7 @@ from dataclasses import dataclass, replace
 import numpy as np
 
 __all__ = ["Workload", "PRESETS", "round_bf16", "round_f32", "forward_inputs",
-           "decode_state", "decode_step_inputs"]
+           "decode_state", "decode_step_inputs", "muir_inputs"]
 
 
 def round_f32(x) -> np.ndarray:
@@ -169,3 +169,25 @@ def decode_step_inputs(w: Workload, step: int, seed: int | None = None) -> dict:
     """Inputs of decode step ``step``: q, k, v, log_w, e1, e2 shaped [B, H, .]."""
     rng = np.random.default_rng((w.seed if seed is None else seed, step))
     return _draw(rng, w, (w.B, w.H))
+
+
+def muir_inputs(w: Workload, seed: int | None = None, static_gains: bool = True) -> dict:
+    """Inputs of one Muir-mixer call (shapes of ``w``; form ignored): the activations
+    after the projections and the causal convolution q, k, v ~ N(0, 1), and the gate logits
+    z_f ~ N(-4, 1) (softplus ~ 0.02: decays 0.75-0.98 per token with the rates below),
+    z_b, z_w, z_q, z_g ~ N(0, 1), all at the storage dtype; a_log ~ U[log 1, log 16] per head,
+    gamma_stat ~ U[0.5, 1.5] per (head, key channel) and the RMSNorm weight ~ U[0.5, 1.5]
+    per value channel (fp32; ones when ``static_gains`` is False, their initial values)."""
+    rng = np.random.default_rng(w.seed + 10 if seed is None else seed)
+    sk = (w.B, w.T, w.H, w.dk)
+    sv = (w.B, w.T, w.H, w.dv)
+    r = lambda shape, m=0.0: _round(rng.normal(m, 1.0, size=shape), w.dtype)
+    out = {"q": r(sk), "k": r(sk), "v": r(sv), "zf": r(sk, -4.0), "zb": r(sk), "zw": r(sv),
+           "zq": r(sk), "zg": r(sv),
+           "a_log": round_f32(rng.uniform(0.0, np.log(16.0), size=w.H))}
+    if static_gains:
+        out["gamma_stat"] = round_f32(rng.uniform(0.5, 1.5, size=(w.H, w.dk)))
+        out["rms_weight"] = round_f32(rng.uniform(0.5, 1.5, size=w.dv))
+    else:
+        out["gamma_stat"] = out["rms_weight"] = None
+    return out
