@@ -63,6 +63,14 @@ def bwd_algorithmic_bytes(w) -> int:
     return w.B * w.T * w.H * (per_in + per_out) + w.B * w.H * w.dk * w.dv * 4
 
 
+def muir_algorithmic_bytes(w) -> int:
+    """The Muir mixer: the activations q, k, v and the gate logits z_f, z_b, z_w, z_q, z_g
+    in (input dtype), y out (fp32), S_T out."""
+    eb = 2 if w.dtype == "bf16" else 4
+    per_token_head = eb * (5 * w.dk + 3 * w.dv) + 4 * w.dv
+    return w.B * w.T * w.H * per_token_head + w.B * w.H * w.dk * w.dv * 4
+
+
 def fwd_flops(w) -> int:
     """Algorithmic flops of the single-write (GDN-2) chunk form per token-head:
     6 d^2 (state GEMMs Y S0, Q S0, K~^T V~) + 5 C d (L, M, [U Y], M V~) + C^2 / 3 (T^-1)."""
@@ -441,6 +449,50 @@ def bench_backward(ctx, args, gdr):
     return out
 
 
+def bench_muir(ctx, args, gdr):
+    """gdr_muir_forward (the Muir token mixer around the GDN-2 recurrence) on the headline
+    shapes, device-resident, fused (activations inside the tensor-core forward) and with
+    the separate prologue kernel: milliseconds per call and the HBM roofline fraction."""
+    torch = ctx.torch
+    w = synth.PRESETS["gdn2_bf16"]
+    inp = synth.muir_inputs(w, seed=rank_seed(w.seed + 10, ctx.rank))
+    names = ("q", "k", "v", "zf", "zb", "zw", "zq", "zg")
+    d = {k: torch.from_numpy(inp[k]).to(ctx.dev, torch.bfloat16) for k in names}
+    par = {k: torch.from_numpy(inp[k]).to(ctx.dev) for k in ("a_log", "gamma_stat", "rms_weight")}
+    out = {"workload": "muir on " + w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv}
+    nbytes = muir_algorithmic_bytes(w)
+    for key, unfused in (("fused", False), ("unfused", True)):
+        ws = gdr.new_workspace(gdr.gdr_muir_workspace_size(d["q"], d["k"], d["v"], w.chunk,
+                                                           args.algo, unfused), ctx.dev)
+        y = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=ctx.dev)
+
+        def call():
+            gdr.gdr_muir_forward(*(d[k] for k in names), par["a_log"], par["gamma_stat"],
+                                 par["rms_weight"], 1e-6, None, chunk=w.chunk, algo=args.algo,
+                                 unfused=unfused, y=y, want_state=False, workspace=ws)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = ctx.event(), ctx.event()
+        n = 5
+        e0.record(ctx.stream)
+        for _ in range(n):
+            call()
+        e1.record(ctx.stream)
+        torch.cuda.synchronize()
+        ms = ctx.max_over_ranks(e0.elapsed_time(e1)) / n
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[key] = {"ms_per_call": ms, "tokens_per_s": w.tokens * ctx.world / (ms * 1e-3),
+                    "launches_per_call": 3 if not unfused else 4,
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
+                                 "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],
+                                 "bytes_per_call": nbytes}}
+        del ws, y
+    del d, par
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(ctx, args, gdr, w, inp, names, step, o):
     """Same call with host inputs: pinned H2D copies, the forward, D2H of o, all timed."""
     torch = ctx.torch
@@ -537,6 +589,8 @@ def main():
                     help="decode batch B (default: the workload's); for profiler captures")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip the timing of the other forward workloads")
+    ap.add_argument("--no-muir", action="store_true",
+                    help="skip the timing of the Muir mixer (gdr_muir_forward)")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the timing of the reverse mode (gdr_backward_chunked)")
     ap.add_argument("--bwd-workload", default=None, choices=["gdn2_bf16", "rwkv7_bf16"],
@@ -571,6 +625,7 @@ def main():
               if args.only == "all" and not args.no_other_workloads else None)
     bwd = (bench_backward(ctx, args, gdr)
            if (args.only == "all" and not args.no_backward) or args.only == "backward" else None)
+    muir = bench_muir(ctx, args, gdr) if args.only == "all" and not args.no_muir else None
     ctx.barrier()
     if world > 1:
         dist.destroy_process_group()
@@ -617,6 +672,8 @@ def main():
         line["other_workloads"] = others
     if bwd is not None:
         line["backward"] = bwd
+    if muir is not None:
+        line["muir"] = muir
     print(json.dumps(line), flush=True)
     return 0
 

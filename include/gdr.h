@@ -257,6 +257,8 @@ typedef struct {
   const float *gamma_stat;
   const float *rms_weight;
   float rms_eps;
+  int unfused;          /* 0: the activations run inside the tensor-core forward where it
+                           applies (bf16, dk = dv = 128); 1: always the separate prologue */
   const float *S0;
   float *y;
   float *S_T;
@@ -268,12 +270,12 @@ typedef struct {
 gdr_status gdr_muir_workspace_size(const gdr_muir_args *args, size_t *bytes);
 
 /*
- * The Muir mixer above.  For bf16 inputs with dk = dv = 128 (algo AUTO or TC) the
- * activations run inside the tensor-core forward's chunk-parallel kernel, on the tiles
- * it loads (no activated copy of the inputs is written), and one light kernel applies
- * RMSNorm (.) SiLU(zg) to o; elsewhere a prologue kernel writes the activated inputs
- * into the workspace, gdr_forward_chunked runs on them, and the same epilogue follows.
- * Errors as gdr_forward_chunked.
+ * The Muir mixer above.  Fused (unfused = 0; bf16 inputs, dk = dv = 128, algo AUTO or
+ * TC): the activations run inside the tensor-core forward's chunk-parallel kernel, on
+ * the tiles it loads (no activated copy of the inputs is written), and one light kernel
+ * applies RMSNorm (.) SiLU(zg) to o.  Otherwise a prologue kernel writes the activated
+ * inputs into the workspace, gdr_forward_chunked runs on them, and the same epilogue
+ * follows.  Errors as gdr_forward_chunked.
  */
 gdr_status gdr_muir_forward(const gdr_muir_args *args, void *stream);
 

@@ -38,7 +38,7 @@ using gdr::kStatusBytes;
 
 // FwdParams of a forward call (pointers as given).
 gdr::FwdParams fwd_params(const gdr_fwd_args *a) {
-  gdr::FwdParams p;
+  gdr::FwdParams p{};
   p.form = a->form;
   p.B = a->B;
   p.H = a->H;
@@ -94,13 +94,51 @@ gdr_fwd_args muir_fwd_args(const gdr_muir_args *a) {
   return f;
 }
 
+// The fused path: bf16, d_k = d_v = 128, the two-kernel tensor-core forward with the
+// mixer's activations in its chunk-parallel kernel.
+gdr::FwdParams muir_fused_params(const gdr_muir_args *a) {
+  gdr::FwdParams p{};
+  p.form = GDR_FORM_GDN2;
+  p.B = a->B;
+  p.H = a->H;
+  p.T = a->T;
+  p.dk = a->dk;
+  p.dv = a->dv;
+  p.chunk = a->chunk;
+  p.q = a->q;
+  p.k = a->k;
+  p.v = a->v;
+  p.e1 = a->zb;
+  p.e2 = a->zw;
+  p.S0 = a->S0;
+  p.S_T = a->S_T;
+  p.status = static_cast<uint32_t *>(a->workspace);
+  p.muir = true;
+  p.zf = a->zf;
+  p.zq = a->zq;
+  p.a_log = a->a_log;
+  p.gamma_stat = a->gamma_stat;
+  return p;
+}
+bool muir_fused(const gdr_muir_args *a) {
+  return !a->unfused && a->algo != GDR_ALGO_FP32 &&
+         gdr::forward_tc_split_supported(muir_fused_params(a), a->dtype);
+}
+
 MuirLayout muir_layout(const gdr_muir_args *a) {
   MuirLayout L;
+  const size_t n = (size_t)a->B * a->T * a->H, eb = a->dtype == GDR_BF16 ? 2 : 4;
+  size_t off = 0;
+  if (muir_fused(a)) {
+    L.fwd = off; off = align256(off + gdr::forward_tc_split_workspace_bytes(muir_fused_params(a)));
+    L.qh = L.kh = L.bh = L.vh = L.wh = L.lw = off;
+    L.o = off; off = align256(off + n * a->dv * 4);
+    L.total = off;
+    return L;
+  }
   const gdr_fwd_args f = muir_fwd_args(a);
   size_t fwd = kStatusBytes;
   gdr_forward_workspace_size(&f, &fwd);
-  const size_t n = (size_t)a->B * a->T * a->H, eb = a->dtype == GDR_BF16 ? 2 : 4;
-  size_t off = 0;
   L.fwd = off; off = align256(off + fwd);
   L.qh = off; off = align256(off + n * a->dk * eb);
   L.kh = off; off = align256(off + n * a->dk * eb);
@@ -331,6 +369,13 @@ gdr_status gdr_muir_forward(const gdr_muir_args *a, void *stream) {
   m.rms_weight = a->rms_weight;
   m.rms_eps = a->rms_eps;
   float *o = reinterpret_cast<float *>(ws + L.o);
+  if (muir_fused(a)) {   // activations inside the forward's chunk-parallel kernel, then the readout
+    gdr::FwdParams p = muir_fused_params(a);
+    p.o = o;
+    gdr_status st = cuda_status(gdr::launch_forward_tc_split(p, ws + L.fwd, s));
+    if (st != GDR_OK) return st;
+    return cuda_status(gdr::launch_muir_epilogue(m, a->dtype, o, a->y, s));
+  }
   // activated inputs, then the GDN-2 forward on them, then the readout
   gdr_status st = cuda_status(gdr::launch_muir_prologue(
       m, a->dtype, ws + L.qh, ws + L.kh, ws + L.vh, ws + L.bh, ws + L.wh,

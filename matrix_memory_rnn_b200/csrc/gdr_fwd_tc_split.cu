@@ -124,7 +124,8 @@ struct PrepSmem {
   static constexpr uint32_t TOT = BT + 16 * kDK * 4;          // fp32 Lam_n per channel
   static constexpr uint32_t L1 = TOT + kDK * 4;               // fp32 Lam_1 per channel
   static constexpr uint32_t A1 = L1 + kDK * 4;                // fp32 [4][DK] alpha_1, by chunk & 3
-  static constexpr uint32_t MISC = A1 + 4 * kDK * 4;
+  static constexpr uint32_t NRM = A1 + 4 * kDK * 4;           // fp32 [2][2][C] Muir 1/|q|, 1/|k|
+  static constexpr uint32_t MISC = NRM + 4 * kC * 4;
   static constexpr uint32_t ALLOC = MISC + 256 + 1024;
   static_assert(BUF % 1024 == 0 && SW % 1024 == 0, "MMA tiles 1024-aligned");
   static_assert(Ix::kBytes <= kC * kDK * 2, "fp32 L must fit the reused bf16 tile");
@@ -180,10 +181,12 @@ __device__ __forceinline__ void load_gate(uint8_t *sw, const PrepMaps &m, uint64
   tma_load_4d(sw + kC * 128, &m.wg, 64, h, t0, b, bar);
 }
 
-// One thread: log w of chunk (b, h, t0) into the log-w staging area.
+// One thread: log w of chunk (b, h, t0) into the log-w staging area (fp32; for the
+// Muir mixer the decay logits z_f, bf16).
+template <bool kMuir>
 __device__ __forceinline__ void load_logw(uint8_t *slw, const PrepMaps &m, uint64_t *bar, int b, int h,
                                           int t0) {
-  mbar_arrive_expect_tx(bar, kC * kDK * 4u);
+  mbar_arrive_expect_tx(bar, kC * kDK * (kMuir ? 2u : 4u));
   tma_load_4d(slw, &m.lw, 0, h, t0, b, bar);
 }
 
@@ -211,6 +214,31 @@ __device__ __forceinline__ bool group_wait(uint64_t *bar, uint32_t parity, volat
   return !Sync::sync_or(failed);
 }
 
+// The Muir mixer's activations on the tiles as loaded ("Muir ...", section 2.1 and
+// section 4.1): SiLU, the head's l2 norm (the 16 lanes holding one token's 128
+// channels reduce with shuffles), the readout gain and the gates.  Seven of these per
+// element ride on a kernel that is issue- and latency-bound, so they use the hardware
+// exponential, logarithm and approximate division (a few ulp; the operands are rounded
+// to bf16 next).  The argument of the exponential is clamped at 80 so that 1 + e^-x
+// stays finite and inside the approximate division's range; softplus switches to its
+// asymptotes where 1 + e^x would round.
+__device__ __forceinline__ float sigmoid_f(float x) {
+  return __fdividef(1.f, 1.f + __expf(-fmaxf(x, -80.f)));
+}
+__device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
+__device__ __forceinline__ float softplus_f(float x) {
+  return x > 15.f ? x : (x < -15.f ? __expf(x) : __logf(1.f + __expf(x)));
+}
+__device__ __forceinline__ float inv_norm16(const float (&x)[8]) {
+  float s = 0.f;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s += x[e] * x[e];
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  return rsqrtf(fmaxf(s, 1e-24f));
+}
+
+template <bool kMuir>
 __global__ void __launch_bounds__(kPrepThreads, 1)
     tc_prep_kernel(FwdParams p, uint8_t *records, const __grid_constant__ PrepMaps maps) {
   using SL = PrepSmem;
@@ -250,6 +278,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   // GDN-2 (erase gate b, optional write gate) or GLA (u = 0: no b, no write gate)
   const bool has_b = p.form == GDR_FORM_GDN2;
   const bool has_wg = has_b && p.e2 != nullptr;
+  float *sNRM = reinterpret_cast<float *>(smem + SL::NRM);   // [buffer][q, k][token]
+  const __nv_bfloat16 *gzq = static_cast<const __nv_bfloat16 *>(p.zq);
   auto item_of = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
 
   if (warp == 0) {
@@ -278,7 +308,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         ++cnt[kWIss0 + j];
       }
       if (j == 0) {
-        load_logw(smem + SL::SLW, maps, lfull, bh / H, bh % H, c * kC);
+        load_logw<kMuir>(smem + SL::SLW, maps, lfull, bh / H, bh % H, c * kC);
         ++cnt[kLIss];
       }
     }
@@ -299,6 +329,28 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       uint8_t *rec = records + (size_t)item * Rec::BYTES;
       float *a1s = sA1 + (j & 3) * kDK;
       GDR_PREP_PHASE(0);
+      // Muir: this thread's 4 tokens x 8 channels of z_q and 8 static gains, loaded now so
+      // that their latency overlaps the waits and the scan
+      uint4 zq_raw[4];
+      float gs8[8];
+      if constexpr (kMuir) {
+        const int bh = item / nch, hh = bh % H;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int tt = (item % nch) * kC + 4 * tb + i;
+          zq_raw[i] = tt < T ? ld16(gzq + (((size_t)(bh / H) * T + tt) * H + hh) * kDK + j0)
+                             : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (p.gamma_stat) {
+          const float4 a = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0));
+          const float4 c = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0 + 4));
+          gs8[0] = a.x; gs8[1] = a.y; gs8[2] = a.z; gs8[3] = a.w;
+          gs8[4] = c.x; gs8[5] = c.y; gs8[6] = c.z; gs8[7] = c.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) gs8[e] = 1.f;
+        }
+      }
 
       // chunk j's log w, tiles and write gate have landed
       if (poller) sexact[bi] = 0;
@@ -315,12 +367,27 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       // ---- cumulative log-decay in registers: prefix over the thread's 4 tokens,
       //      then the exclusive prefix over the 16 token blocks (one thread per channel)
       float lam[4][8];
+      if constexpr (kMuir) {
+        // log alpha = -exp(a_log[h]) softplus(z_f); tokens past T keep the state (log alpha
+        // = 0), as the zero-filled log w of the plain path does
+        const float rate = __expf(p.a_log[(item / nch) % H]);
+        const int tpad = T - (item % nch) * kC;
+        const __nv_bfloat16 *zl = reinterpret_cast<const __nv_bfloat16 *>(smem + SL::SLW);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 x0 = *reinterpret_cast<const float4 *>(sLW + (4 * tb + i) * kDK + j0);
-        const float4 x1 = *reinterpret_cast<const float4 *>(sLW + (4 * tb + i) * kDK + j0 + 4);
-        lam[i][0] = x0.x; lam[i][1] = x0.y; lam[i][2] = x0.z; lam[i][3] = x0.w;
-        lam[i][4] = x1.x; lam[i][5] = x1.y; lam[i][6] = x1.z; lam[i][7] = x1.w;
+        for (int i = 0; i < 4; ++i) {
+          unpack8(*reinterpret_cast<const uint4 *>(zl + (4 * tb + i) * kDK + j0), lam[i]);
+          const bool real = 4 * tb + i < tpad;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) lam[i][e] = real ? -rate * softplus_f(lam[i][e]) : 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float4 x0 = *reinterpret_cast<const float4 *>(sLW + (4 * tb + i) * kDK + j0);
+          const float4 x1 = *reinterpret_cast<const float4 *>(sLW + (4 * tb + i) * kDK + j0 + 4);
+          lam[i][0] = x0.x; lam[i][1] = x0.y; lam[i][2] = x0.z; lam[i][3] = x0.w;
+          lam[i][4] = x1.x; lam[i][5] = x1.y; lam[i][6] = x1.z; lam[i][7] = x1.w;
+        }
       }
       {
         float tot[8];
@@ -348,7 +415,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       if (gt == 32 && j + 1 < nloc) {
         fence_proxy_async_smem();
         const int it = item_of(j + 1), cn = it % nch, bhn = it / nch;
-        load_logw(smem + SL::SLW, maps, lfull, bhn / H, bhn % H, cn * kC);
+        load_logw<kMuir>(smem + SL::SLW, maps, lfull, bhn / H, bhn % H, cn * kC);
         cnt[kLIss] = j + 2;
       }
       if (gt < kDK) {
@@ -423,6 +490,27 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
               for (int e = 0; e < 8; ++e) b8[e] = 0.f;
             }
             unpack8(*reinterpret_cast<const uint4 *>(buf + oq), q8);
+            if constexpr (kMuir) {
+              // k = l2norm(silu(k)), q^ = gamma_stat 2 sigmoid(z_q) l2norm(silu(q)), b = 2 sigmoid(z_b)
+              float zq8[8];
+              unpack8(zq_raw[i], zq8);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                k8[e] = silu_f(k8[e]);
+                q8[e] = silu_f(q8[e]);
+                b8[e] = 2.f * sigmoid_f(b8[e]);
+              }
+              const float nk = inv_norm16(k8), nq = inv_norm16(q8);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                k8[e] *= nk;
+                q8[e] *= nq * gs8[e] * 2.f * sigmoid_f(zq8[e]);
+              }
+              if (g == 0) {
+                sNRM[bi * 2 * kC + t] = nq;
+                sNRM[bi * 2 * kC + kC + t] = nk;
+              }
+            }
             float av[8], aq[8], bl[8], kt[8], qp[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -465,8 +553,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
           float v8[8], w8[8];
           unpack8(*reinterpret_cast<const uint4 *>(buf + SL::VH + off), v8);
           unpack8(*reinterpret_cast<const uint4 *>(sw + off), w8);
+          if constexpr (kMuir) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+            for (int e = 0; e < 8; ++e) v8[e] = silu_f(v8[e]) * sigmoid_f(w8[e]);   // silu(v) sigmoid(z_w)
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
+          }
           st_smem16(buf, SL::VH + off, pack8(v8));
         }
       }
@@ -550,9 +643,18 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             const size_t ot = tok_off(t), os = tok_off(s);
             for (int jj = 0; jj < kDK; ++jj) {
               const float d = __expf(__ldcg(lt + jj) - __ldcg(ls + jj));
-              const float ks = __bfloat162float(gk[os + jj]);
-              m += __bfloat162float(gq[ot + jj]) * d * ks;
-              if (has_b) l += __bfloat162float(gb[ot + jj]) * __bfloat162float(gk[ot + jj]) * d * ks;
+              float ks = __bfloat162float(gk[os + jj]), kt = __bfloat162float(gk[ot + jj]);
+              float qt = __bfloat162float(gq[ot + jj]), bt = has_b ? __bfloat162float(gb[ot + jj]) : 0.f;
+              if constexpr (kMuir) {   // the activations of the front group's operand tiles
+                const float *nrm = sNRM + bi * 2 * kC;
+                const float gs = p.gamma_stat ? __ldg(p.gamma_stat + h * kDK + jj) : 1.f;
+                ks = silu_f(ks) * nrm[kC + s];
+                kt = silu_f(kt) * nrm[kC + t];
+                qt = silu_f(qt) * nrm[t] * gs * 2.f * sigmoid_f(__bfloat162float(gzq[ot + jj]));
+                bt = 2.f * sigmoid_f(bt);
+              }
+              m += qt * d * ks;
+              if (has_b) l += bt * kt * d * ks;
             }
           }
           sL[Ix::at(t, s)] = (s < t) ? l : 0.f;
@@ -1006,16 +1108,19 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B;
   const bool has_b = p.form == GDR_FORM_GDN2;
+  const bool lw_ok = p.muir ? encode_input_map(&maps.lw, p.zf, bf, 2, kDK, CU_TENSOR_MAP_SWIZZLE_NONE, p)
+                            : encode_input_map(&maps.lw, p.log_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4,
+                                               kDK, CU_TENSOR_MAP_SWIZZLE_NONE, p);
   if (!encode_input_map(&maps.k, p.k, bf, 2, 64, sw, p) ||
       (has_b && !encode_input_map(&maps.b, p.e1, bf, 2, 64, sw, p)) ||
       !encode_input_map(&maps.q, p.q, bf, 2, 64, sw, p) ||
       !encode_input_map(&maps.v, p.v, bf, 2, 64, sw, p) ||
-      (has_b && p.e2 && !encode_input_map(&maps.wg, p.e2, bf, 2, 64, sw, p)) ||
-      !encode_input_map(&maps.lw, p.log_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, kDK,
-                        CU_TENSOR_MAP_SWIZZLE_NONE, p))
+      (has_b && p.e2 && !encode_input_map(&maps.wg, p.e2, bf, 2, 64, sw, p)) || !lw_ok)
     return cudaErrorInvalidValue;
+  if (p.muir && (!has_b || !p.e2 || !p.zq || !p.a_log)) return cudaErrorInvalidValue;
   uint8_t *records = static_cast<uint8_t *>(workspace) + kHeaderBytes;
-  cudaError_t e = cudaFuncSetAttribute(tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto prep = p.muir ? tc_prep_kernel<true> : tc_prep_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)PrepSmem::ALLOC);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(tc_chain_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1025,7 +1130,7 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int items = p.B * p.H * num_chunks(p.T);
-  tc_prep_kernel<<<min(items, sms), kPrepThreads, PrepSmem::ALLOC, stream>>>(p, records, maps);
+  prep<<<min(items, sms), kPrepThreads, PrepSmem::ALLOC, stream>>>(p, records, maps);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 gc(p.dv / NV, p.H, p.B);
   tc_chain_kernel<NV><<<gc, kThreads, ChainSmem<NV>::ALLOC, stream>>>(p, records);

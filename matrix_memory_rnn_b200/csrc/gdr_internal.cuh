@@ -57,6 +57,12 @@ struct FwdParams {
   float *S_T;
   uint32_t *status;  // device status word (workspace), may be null
   uint32_t debug;    // fault-injection bits (kDebug...), 0 in normal use
+  // The Muir mixer's prologue inside the tensor-core forward (gdr_muir_forward):
+  // q, k, v, e1, e2 then hold the raw q, k, v, z_b, z_w, and the decay comes from
+  // z_f and a_log instead of log_w.
+  bool muir;
+  const void *zf, *zq;
+  const float *a_log, *gamma_stat;
 };
 
 // Fault injection for the tests of the bounded waits (set through the environment

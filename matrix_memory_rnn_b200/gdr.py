@@ -54,7 +54,8 @@ class gdr_muir_args(ctypes.Structure):
                 ("dv", _c_int), ("chunk", _c_int), ("algo", _c_int), ("q", _vp), ("k", _vp),
                 ("v", _vp), ("zf", _vp), ("zb", _vp), ("zw", _vp), ("zq", _vp), ("zg", _vp),
                 ("a_log", _fp), ("gamma_stat", _fp), ("rms_weight", _fp),
-                ("rms_eps", ctypes.c_float), ("S0", _fp), ("y", _fp), ("S_T", _fp),
+                ("rms_eps", ctypes.c_float), ("unfused", _c_int), ("S0", _fp), ("y", _fp),
+                ("S_T", _fp),
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
@@ -303,7 +304,7 @@ def gdr_backward_chunked(form, q, k, v, log_w, e1=None, e2=None, S0=None, dO=Non
 
 
 def _muir_struct(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat, rms_weight, rms_eps, S0, y,
-                 S_T, chunk, algo, workspace):
+                 S_T, chunk, algo, workspace, unfused=False):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dname, tdt = _dtype_of(q)
@@ -329,16 +330,18 @@ def _muir_struct(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat, rms_weight, rms
                     ("rms_weight", rms_weight), ("S0", S0), ("y", y), ("S_T", S_T)):
         setattr(a, name, _ptr(t))
     a.rms_eps = float(rms_eps)
+    a.unfused = int(bool(unfused))
     if workspace is not None:
         a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
     return a
 
 
-def gdr_muir_workspace_size(q, k, v, chunk=64, algo="auto"):
+def gdr_muir_workspace_size(q, k, v, chunk=64, algo="auto", unfused=False):
     """Bytes of device workspace ``gdr_muir_forward`` needs for inputs of these shapes."""
     B, T, H, dk = q.shape
     a = gdr_muir_args()
     a.dtype, a.algo = DTYPES[_dtype_of(q)[0]], ALGOS[algo]
+    a.unfused = int(bool(unfused))
     a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, v.shape[-1], chunk
     n = ctypes.c_size_t(0)
     _check("gdr_muir_workspace_size",
@@ -347,8 +350,8 @@ def gdr_muir_workspace_size(q, k, v, chunk=64, algo="auto"):
 
 
 def gdr_muir_forward(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat=None, rms_weight=None,
-                     rms_eps=1e-6, S0=None, *, chunk=64, algo="auto", y=None, S_T=None,
-                     want_state=True, workspace=None, stream=None):
+                     rms_eps=1e-6, S0=None, *, chunk=64, algo="auto", unfused=False, y=None,
+                     S_T=None, want_state=True, workspace=None, stream=None):
     """The Muir token mixer around the GDN-2 recurrence (include/gdr.h, gdr_muir_forward):
     pre-activations q, k, v and gate logits zf, zb, zw, zq, zg [B, T, H, .] (bf16 or fp32),
     a_log [H], optional gamma_stat [H, dk] and rms_weight [dv] (fp32).  Returns (y, S_T)."""
@@ -359,9 +362,9 @@ def gdr_muir_forward(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat=None, rms_we
     if S_T is None and want_state:
         S_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
     if workspace is None:
-        workspace = new_workspace(gdr_muir_workspace_size(q, k, v, chunk, algo), q.device)
+        workspace = new_workspace(gdr_muir_workspace_size(q, k, v, chunk, algo, unfused), q.device)
     a = _muir_struct(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat, rms_weight, rms_eps, S0, y,
-                     S_T, chunk, algo, workspace)
+                     S_T, chunk, algo, workspace, unfused)
     _check("gdr_muir_forward", _load().gdr_muir_forward(ctypes.byref(a), _stream(stream)))
     return y, S_T
 

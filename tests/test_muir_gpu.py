@@ -14,14 +14,14 @@ pytestmark = pytest.mark.gpu
 TOKEN = ("q", "k", "v", "zf", "zb", "zw", "zq", "zg")
 
 
-def _run(w, inp, S0=None, algo="auto", workspace_bytes=None):
+def _run(w, inp, S0=None, algo="auto", workspace_bytes=None, unfused=False):
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     d = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to("cuda", tdt) for k in TOKEN}
     f32 = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a, np.float32)).cuda()
     ws = None if workspace_bytes is None else gdr.new_workspace(workspace_bytes, "cuda")
     y, S_T = gdr.gdr_muir_forward(*(d[k] for k in TOKEN), f32(inp["a_log"]), f32(inp["gamma_stat"]),
                                   f32(inp["rms_weight"]), 1e-6, f32(S0), chunk=w.chunk, algo=algo,
-                                  workspace=ws)
+                                  unfused=unfused, workspace=ws)
     torch.cuda.synchronize()
     return y.cpu().numpy(), S_T.cpu().numpy()
 
@@ -69,3 +69,43 @@ def test_muir_zero_length():
     S0 = np.random.default_rng(1).standard_normal((1, 2, 64, 64)).astype(np.float32)
     y, S = _run(w, inp, S0)
     assert y.shape == (1, 0, 2, 64) and np.array_equal(S, S0)
+
+
+def test_muir_fused_strong_decay_uses_exact_path():
+    """bf16, d = 128 runs the mixer inside the tensor-core forward; decay logits that make
+    some channels decay by more than 80 nats per chunk take its exact pairwise path."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=150, B=1, H=2, chunk=64)
+    inp = synth.muir_inputs(w)
+    zf = inp["zf"].copy()
+    zf[:, :, :, ::9] = 6.0          # softplus ~ 6: log alpha ~ -6 exp(a_log) per token
+    inp["zf"] = synth.round_bf16(zf)
+    inp["a_log"] = np.full(w.H, np.log(4.0), np.float32)
+    y, S = _run(w, inp)
+    y_ref, S_ref = _ref(inp)
+    ey, es = head_rel_err(y, y_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    print(f"muir fused strong decay: y {ey:.2e} S {es:.2e}")
+    assert np.isfinite(y).all() and ey < TOL["bf16"] and es < TOL["bf16"]
+
+
+def test_muir_fused_against_unfused():
+    """The fused path (activations inside the forward) and the unfused one (prologue
+    kernel, fp32 forward, epilogue) on the same inputs."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=200, B=2, H=2, chunk=64)
+    inp = synth.muir_inputs(w)
+    y_f, S_f = _run(w, inp, algo="auto")
+    y_u, S_u = _run(w, inp, algo="fp32")
+    assert head_rel_err(y_f, y_u, (0, 2)) < TOL["bf16"]
+    assert head_rel_err(S_f, S_u, (0, 1)) < TOL["bf16"]
+
+
+@pytest.mark.parametrize("unfused", [False, True])
+def test_muir_bf16_d128_both_paths(unfused):
+    """bf16, d = 128: the fused path and the separate prologue (both on the tensor-core
+    forward) against the oracle, with a ragged tail and an initial state."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=333, B=2, H=3, chunk=64)
+    inp = synth.muir_inputs(w)
+    S0 = synth.round_f32(np.random.default_rng(13).normal(0, 0.5, (w.B, w.H, 128, 128)))
+    y, S = _run(w, inp, S0, unfused=unfused)
+    y_ref, S_ref = _ref(inp, S0)
+    assert head_rel_err(y, y_ref, (0, 2)) < TOL["bf16"]
+    assert head_rel_err(S, S_ref, (0, 1)) < TOL["bf16"]
