@@ -5,4 +5,4 @@ TEST INFRASTRUCTURE: only ``tests/``, ``__graft_entry__.smoke()`` and the
 package.  The product path (``matrix_memory_rnn_b200``) never does.
 """
 from .oracle import (FORMS, backward, build, decode_step, forward, library_path, load_library,
-                     max_threads, muir_forward)  # noqa: F401
+                     max_threads, mlstm_forward, muir_forward)  # noqa: F401

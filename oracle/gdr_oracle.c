@@ -445,3 +445,101 @@ done:
   free(o);
   return rc;
 }
+
+/*
+ * xLSTM's mLSTM cell ("Exponential gates and matrix memory: xLSTM and RWKV-7", section
+ * 13.4 and the solution to Exercise 13.6), one head at a time: matrix memory C (d_v x d_k),
+ * normalizer n (d_k), scalar gates per (b, t, h): forget f_t = sigmoid(f~_t), input
+ * i_t = exp(i~_t).
+ *
+ *   naive       C_t = f_t C_{t-1} + i_t v_t k_t^T,  n_t = f_t n_{t-1} + i_t k_t,
+ *               h_t = C_t q_t / max(|n_t^T q_t|, 1)
+ *   stabilized  m_t = max(log f_t + m_{t-1}, i~_t)   (m_0 = -inf for an empty memory)
+ *               f'_t = exp(log f_t + m_{t-1} - m_t),  i'_t = exp(i~_t - m_t)
+ *               C_t = f'_t C_{t-1} + i'_t v_t k_t^T,  n_t = f'_t n_{t-1} + i'_t k_t
+ *               h_t = C_t q_t / max(|n_t^T q_t|, exp(-m_t))
+ *
+ * (the stabilized memory is the naive one times exp(-m_t); the readout floor scales with
+ * it).  Inputs: q, k [B][T][H][dk], v [B][T][H][dv], f_pre, i_pre [B][T][H].  Initial
+ * state: C0 [B][H][dk][dv] (storage layout, the transpose of C), n0 [B][H][dk], m0 [B][H];
+ * all NULL for an empty memory (stabilized: m0 = -inf).  In the naive mode C0 and n0 are
+ * the unscaled memory and m0 is ignored.  Outputs h [B][T][H][dv] and, when non-NULL, the
+ * final C_T, n_T, m_T (the naive mode writes m_T = 0).  Returns as oracle_forward.
+ */
+static double log_sigmoid(double x) { return x >= 0.0 ? -log1p(exp(-x)) : x - log1p(exp(x)); }
+
+int oracle_mlstm_forward(int B, int T, int H, int dk, int dv, int naive,
+                         const double *q, const double *k, const double *v,
+                         const double *f_pre, const double *i_pre,
+                         const double *C0, const double *n0, const double *m0,
+                         double *h, double *C_T, double *n_T, double *m_T, int n_threads) {
+  if (B < 0 || T < 0 || H < 0 || dk <= 0 || dv <= 0) return -1;
+  if (T > 0 && (!q || !k || !v || !f_pre || !i_pre || !h)) return -1;
+  const int n_seq = B * H;
+  int failed = 0;
+#ifdef _OPENMP
+  if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel
+#endif
+  {
+    double *C = (double *)malloc(sizeof(double) * (size_t)dk * dv);
+    double *nv = (double *)malloc(sizeof(double) * (size_t)dk);
+#ifdef _OPENMP
+#pragma omp for schedule(dynamic, 1)
+#endif
+    for (int sq = 0; sq < n_seq; ++sq) {
+      if (!C || !nv) {
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+        failed = 1;
+        continue;
+      }
+      const int b = sq / H, hh = sq % H;
+      const size_t so = (size_t)sq * dk * dv;
+      for (int c = 0; c < dv; ++c)
+        for (int j = 0; j < dk; ++j) C[(size_t)c * dk + j] = C0 ? C0[so + (size_t)j * dv + c] : 0.0;
+      for (int j = 0; j < dk; ++j) nv[j] = n0 ? n0[(size_t)sq * dk + j] : 0.0;
+      double m = m0 ? m0[sq] : -INFINITY;
+      for (int t = 0; t < T; ++t) {
+        const size_t ts = ((size_t)b * T + t) * H + hh;
+        const size_t tk = ts * (size_t)dk, tv = ts * (size_t)dv;
+        const double lf = log_sigmoid(f_pre[ts]), li = i_pre[ts];
+        double fs, is;
+        if (naive) {
+          fs = exp(lf);
+          is = exp(li);
+        } else {
+          const double mn = fmax(lf + m, li);
+          fs = exp(lf + m - mn);   /* 0 when m = -inf: the empty memory is discarded */
+          is = exp(li - mn);
+          m = mn;
+        }
+        for (int c = 0; c < dv; ++c)
+          for (int j = 0; j < dk; ++j)
+            C[(size_t)c * dk + j] = fs * C[(size_t)c * dk + j] + is * v[tv + c] * k[tk + j];
+        double den = 0.0;
+        for (int j = 0; j < dk; ++j) {
+          nv[j] = fs * nv[j] + is * k[tk + j];
+          den += nv[j] * q[tk + j];
+        }
+        const double floor_ = naive ? 1.0 : exp(-m);
+        const double dd = fmax(fabs(den), floor_);
+        for (int c = 0; c < dv; ++c) {
+          double acc = 0.0;
+          for (int j = 0; j < dk; ++j) acc += C[(size_t)c * dk + j] * q[tk + j];
+          h[tv + c] = acc / dd;
+        }
+      }
+      if (C_T)
+        for (int c = 0; c < dv; ++c)
+          for (int j = 0; j < dk; ++j) C_T[so + (size_t)j * dv + c] = C[(size_t)c * dk + j];
+      if (n_T)
+        for (int j = 0; j < dk; ++j) n_T[(size_t)sq * dk + j] = nv[j];
+      if (m_T) m_T[sq] = naive ? 0.0 : m;
+    }
+    free(C);
+    free(nv);
+  }
+  return failed ? -2 : 0;
+}

@@ -51,6 +51,8 @@ def load_library(path: str):
     lib.oracle_muir_forward.restype = ctypes.c_int
     lib.oracle_muir_forward.argtypes = ([ctypes.c_int] * 5 + [dp] * 11 + [ctypes.c_double] +
                                         [dp] * 3 + [ctypes.c_int])
+    lib.oracle_mlstm_forward.restype = ctypes.c_int
+    lib.oracle_mlstm_forward.argtypes = [ctypes.c_int] * 6 + [dp] * 12 + [ctypes.c_int]
     lib.oracle_backward.restype = ctypes.c_int
     lib.oracle_backward.argtypes = [ctypes.c_int] * 6 + [dp] * 16 + [ctypes.c_int]
     return lib
@@ -158,6 +160,29 @@ def muir_forward(q_pre, k_pre, v_pre, zf, zb, zw, zq, zg, a_log, gamma_stat=None
     if rc != 0:
         raise ValueError(f"oracle_muir_forward failed with code {rc}")
     return y, S_T
+
+
+def mlstm_forward(q, k, v, f_pre, i_pre, C0=None, n0=None, m0=None, naive=False,
+                  n_threads: int = 0, lib=None):
+    """xLSTM's mLSTM cell (``oracle_mlstm_forward``), stabilized unless ``naive``:
+    q, k [B, T, H, dk], v [B, T, H, dv], f_pre, i_pre [B, T, H]; optional initial
+    C0 [B, H, dk, dv], n0 [B, H, dk], m0 [B, H].  Returns (h, C_T, n_T, m_T)."""
+    lib = _load() if lib is None else lib
+    q, k, v, f_pre, i_pre, C0, n0, m0 = map(_f64, (q, k, v, f_pre, i_pre, C0, n0, m0))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    assert k.shape == (B, T, H, dk) and v.shape == (B, T, H, dv)
+    assert f_pre.shape == (B, T, H) and i_pre.shape == (B, T, H)
+    h = np.zeros((B, T, H, dv))
+    C_T = np.zeros((B, H, dk, dv))
+    n_T = np.zeros((B, H, dk))
+    m_T = np.zeros((B, H))
+    rc = lib.oracle_mlstm_forward(B, T, H, dk, dv, int(bool(naive)), _ptr(q), _ptr(k), _ptr(v),
+                                  _ptr(f_pre), _ptr(i_pre), _ptr(C0), _ptr(n0), _ptr(m0), _ptr(h),
+                                  _ptr(C_T), _ptr(n_T), _ptr(m_T), int(n_threads))
+    if rc != 0:
+        raise ValueError(f"oracle_mlstm_forward failed with code {rc}")
+    return h, C_T, n_T, m_T
 
 
 def decode_step(form: str, q, k, v, log_w, e1, e2, S, n_threads: int = 0):
