@@ -280,6 +280,42 @@ gdr_status gdr_muir_workspace_size(const gdr_muir_args *args, size_t *bytes);
 gdr_status gdr_muir_forward(const gdr_muir_args *args, void *stream);
 
 /*
+ * Arguments of gdr_mlstm_forward: xLSTM's mLSTM cell ("Exponential gates and matrix
+ * memory: xLSTM and RWKV-7", section 13.4 and the solution to Exercise 13.6).
+ *   q, k : [B][T][H][dk]    v : [B][T][H][dv]    (element type dtype)
+ *   f_pre, i_pre : [B][T][H] fp32, forget and input gate pre-activations f~, i~
+ *   C0 [B][H][dk][dv], n0 [B][H][dk], m0 [B][H] : the stabilized state (memory in the
+ *       storage orientation, normalizer, running max), or all NULL for an empty memory
+ *   h : [B][T][H][dv] fp32, required;  C_T, n_T, m_T : the final state, or NULL
+ * Per (b, h), with f_t = sigmoid(f~_t) and i_t = exp(i~_t):
+ *   m_t = max(log f_t + m_{t-1}, i~_t)      (m_0 = -inf for an empty memory)
+ *   C_t = e^{log f_t + m_{t-1} - m_t} C_{t-1} + e^{i~_t - m_t} v_t k_t^T,  n_t likewise with k_t
+ *   h_t = C_t q_t / max(|n_t . q_t|, e^{-m_t})
+ * i.e. the naive recurrence (C_t = f_t C_{t-1} + i_t v_t k_t^T, floor 1) carried in the
+ * coordinates C e^{-m_t}, which never overflow.
+ */
+typedef struct {
+  gdr_dtype dtype;
+  int B, H, T, dk, dv;  /* dk, dv in {64, 128} */
+  const void *q, *k, *v;
+  const float *f_pre, *i_pre;
+  const float *C0, *n0, *m0;
+  float *h;
+  float *C_T, *n_T, *m_T;
+} gdr_mlstm_args;
+
+/*
+ * The mLSTM cell over whole sequences, chunkwise: per 64-token chunk with A_t the
+ * cumulative log f_t inside the chunk and (C, n, m) carried from the previous chunk,
+ *   m_t = A_t + max(m, max_{s <= t} (i~_s - A_s)),
+ *   h_t = (sum_{s<=t} w_ts (q_t.k_s) v_s + g_t C q_t) / max(|sum_{s<=t} w_ts (q_t.k_s) + g_t n.q_t|, e^{-m_t})
+ * with w_ts = e^{A_t - A_s + i~_s - m_t} and g_t = e^{A_t + m - m_t}, all <= 1; the chunk's
+ * products on the tensor cores (tf32, three products for fp32 inputs).  No workspace.
+ * Errors as gdr_forward_chunked; GDR_ERR_UNSUPPORTED for dk or dv outside {64, 128}.
+ */
+gdr_status gdr_mlstm_forward(const gdr_mlstm_args *args, void *stream);
+
+/*
  * Arguments of gdr_decode_step: one token for each (b, h).
  *   q, k, log_w, e1 (GENERAL/GDN2/RWKV7) : [B][H][dk]
  *   v, o, e2 (GDN2)                      : [B][H][dv]

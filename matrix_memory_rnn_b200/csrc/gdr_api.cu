@@ -1,5 +1,6 @@
 // gdr_api.cu -- the extern "C" entry points of libgdr: argument validation,
 // kernel selection and launch.  Declarations and the contract: include/gdr.h.
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -394,6 +395,42 @@ gdr_status gdr_muir_forward(const gdr_muir_args *a, void *stream) {
   st = gdr_forward_chunked(&f, stream);
   if (st != GDR_OK) return st;
   return cuda_status(gdr::launch_muir_epilogue(m, a->dtype, o, a->y, s));
+}
+
+gdr_status gdr_mlstm_forward(const gdr_mlstm_args *a, void *stream) {
+  if (!a) return GDR_ERR_INVALID_ARG;
+  if (!dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 0 || a->T < 0) return GDR_ERR_INVALID_ARG;
+  if ((a->dk != 64 && a->dk != 128) || (a->dv != 64 && a->dv != 128)) return GDR_ERR_UNSUPPORTED;
+  const size_t tokens = (size_t)a->B * a->T * a->H;
+  if (tokens > 0 && (!a->q || !a->k || !a->v || !a->f_pre || !a->i_pre || !a->h))
+    return GDR_ERR_INVALID_ARG;
+  // the state comes whole or not at all
+  if ((a->C0 != nullptr) != (a->n0 != nullptr) || (a->C0 != nullptr) != (a->m0 != nullptr))
+    return GDR_ERR_INVALID_ARG;
+  const void *al[] = {a->q, a->k, a->v, a->h, a->C0, a->C_T};
+  for (const void *p : al)
+    if (p && !aligned16(p)) return GDR_ERR_MISALIGNED;
+  if (a->B == 0 || a->H == 0) return GDR_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (a->T == 0) {   // no tokens: the final state is the initial one (empty: zeros, m = -inf)
+    const size_t nbh = (size_t)a->B * a->H;
+    if (a->C_T) {
+      gdr_status st = gdr_state_init(a->C_T, a->B, a->H, a->dk, a->dv, a->C0, stream);
+      if (st != GDR_OK) return st;
+    }
+    if (a->n_T) {
+      cudaError_t e = a->n0 ? cudaMemcpyAsync(a->n_T, a->n0, nbh * a->dk * 4, cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(a->n_T, 0, nbh * a->dk * 4, s);
+      if (e != cudaSuccess) return GDR_ERR_CUDA;
+    }
+    if (a->m_T) {
+      if (a->m0) return cuda_status(cudaMemcpyAsync(a->m_T, a->m0, nbh * 4, cudaMemcpyDeviceToDevice, s));
+      return cuda_status(gdr::fill_f32(a->m_T, nbh, -INFINITY, s));
+    }
+    return GDR_OK;
+  }
+  return cuda_status(gdr::launch_mlstm(*a, s));
 }
 
 gdr_status gdr_read_status(void *workspace, void *stream, gdr_status *device_status) {

@@ -102,6 +102,10 @@ cudaError_t launch_muir_prologue(const MuirParams &m, gdr_dtype dtype, void *qh,
 cudaError_t launch_muir_epilogue(const MuirParams &m, gdr_dtype dtype, const float *o, float *y,
                                  cudaStream_t stream);
 
+// xLSTM's mLSTM cell (gdr_mlstm_forward); p[0 .. n) = x.
+cudaError_t launch_mlstm(const gdr_mlstm_args &a, cudaStream_t stream);
+cudaError_t fill_f32(float *p, size_t n, float x, cudaStream_t stream);
+
 // Launchers (host).  Return cudaSuccess or the launch error.
 cudaError_t launch_decode(const gdr_step_args &a, cudaStream_t stream);
 cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_t stream);

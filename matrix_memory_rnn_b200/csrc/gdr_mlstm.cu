@@ -1,0 +1,251 @@
+// gdr_mlstm.cu -- xLSTM's mLSTM cell with the log-domain stabilizer ("Exponential gates
+// and matrix memory: xLSTM and RWKV-7", section 13.4 and the solution to Exercise 13.6),
+// chunkwise.
+//
+// The stabilizer is a running maximum of the log-weights of everything the memory holds:
+// unrolled, m_t = max(F_t + m_0, max_{s<=t} (F_t - F_s + i~_s)) with F the cumulative
+// log forget gate.  Inside a chunk (local cumulative A_t, carried state C, n, m) that is
+//   m_t = A_t + max(m, P_t),   P_t = max_{s<=t} (i~_s - A_s)   (a prefix maximum),
+// and every weight of the readout and of the carried state is an exponential of a
+// non-positive argument:
+//   w_ts = e^{A_t - A_s + i~_s - m_t} (s <= t),   g_t = e^{A_t + m - m_t},
+//   num_t = sum_s w_ts (q_t . k_s) v_s + g_t C q_t,   den_t = sum_s w_ts (q_t . k_s) + g_t n . q_t,
+//   h_t = num_t / max(|den_t|, e^{-m_t}),
+//   C <- g_L C + sum_s w_Ls v_s k_s^T,   n <- g_L n + sum_s w_Ls k_s,   m <- m_L.
+// One CTA per (b, h, 64 value columns) walks the chunks of its sequence with the state
+// slice in shared memory; Q K^T, P V + diag(g) Q C, and the state update K^T diag(w_L) V
+// are warp-level tf32 MMAs (three products for fp32 inputs).  Tokens past T are padding
+// with log f = 0 and i~ = -inf (no write, no decay).
+#include <math.h>
+
+#include "gdr_internal.cuh"
+#include "gdr_warp_mma.cuh"
+
+namespace gdr {
+namespace {
+
+using wmma_tf32::for_acc;
+using wmma_tf32::mma_seg;
+using wmma_tf32::zero_acc;
+
+constexpr int kL = 64;          // chunk
+constexpr int kNV = 64;         // value columns per CTA
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kLDL = kL + 4;
+constexpr int kLDN = kNV + 4;
+
+struct MlstmSmem {
+  int LDK;
+  size_t Q, K, V, P, C, n, A, lf, ib, m, g, den, total;
+  __host__ __device__ explicit MlstmSmem(int dk) {
+    LDK = dk + 4;
+    size_t off = 0;
+    Q = off; off += (size_t)kL * LDK;
+    K = off; off += (size_t)kL * LDK;
+    V = off; off += (size_t)kL * kLDN;
+    P = off; off += (size_t)kL * kLDL;
+    C = off; off += (size_t)dk * kLDN;
+    n = off; off += dk;
+    A = off; off += kL;
+    lf = off; off += kL;
+    ib = off; off += kL;
+    m = off; off += kL;
+    g = off; off += kL;
+    den = off; off += kL;
+    total = off + 4;
+  }
+};
+
+__device__ __forceinline__ float ld_elem(const float *p, size_t i) { return __ldg(p + i); }
+__device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
+
+template <typename Tin, bool kSplit>
+__global__ void __launch_bounds__(kThreads, 1) mlstm_kernel(gdr_mlstm_args a) {
+  extern __shared__ float sm[];
+  const int dk = a.dk, dv = a.dv, T = a.T, H = a.H;
+  const MlstmSmem L(dk);
+  const int LDK = L.LDK;
+  const int c0 = blockIdx.x * kNV, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float *Q = sm + L.Q, *K = sm + L.K, *V = sm + L.V, *P = sm + L.P, *C = sm + L.C, *nn = sm + L.n;
+  float *A = sm + L.A, *lf = sm + L.lf, *ib = sm + L.ib, *mt = sm + L.m, *gt = sm + L.g;
+  float *den = sm + L.den;
+  float *mcar = sm + L.total - 4;   // the carried running max
+  const Tin *q = static_cast<const Tin *>(a.q), *k = static_cast<const Tin *>(a.k);
+  const Tin *v = static_cast<const Tin *>(a.v);
+  const size_t bh = (size_t)b * H + h;
+
+  for (int i = tid; i < dk * kNV; i += kThreads) {
+    const int j = i / kNV, c = i % kNV;
+    C[j * kLDN + c] = a.C0 ? a.C0[bh * dk * dv + (size_t)j * dv + c0 + c] : 0.f;
+  }
+  for (int j = tid; j < dk; j += kThreads) nn[j] = a.n0 ? a.n0[bh * dk + j] : 0.f;
+  if (tid == 0) *mcar = a.m0 ? a.m0[bh] : -INFINITY;
+
+  for (int t0 = 0; t0 < T; t0 += kL) {
+    const int n = min(kL, T - t0);
+    __syncthreads();   // the previous chunk is done with every buffer
+    // ---- chunk tiles and gates (padding: q = k = v = 0, log f = 0, i~ = -inf)
+    for (int i = tid; i < kL * dk; i += kThreads) {
+      const int t = i / dk, j = i % dk;
+      const size_t ik = (((size_t)b * T + t0 + t) * H + h) * dk + j;
+      Q[t * LDK + j] = t < n ? ld_elem(q, ik) : 0.f;
+      K[t * LDK + j] = t < n ? ld_elem(k, ik) : 0.f;
+    }
+    for (int i = tid; i < kL * kNV; i += kThreads) {
+      const int t = i / kNV, c = i % kNV;
+      V[t * kLDN + c] = t < n ? ld_elem(v, (((size_t)b * T + t0 + t) * H + h) * dv + c0 + c) : 0.f;
+    }
+    if (tid < kL) {
+      const int t = tid;
+      const size_t ts = ((size_t)b * T + t0 + t) * H + h;
+      if (t < n) {
+        const float x = __ldg(a.f_pre + ts);
+        lf[t] = x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));   // log sigmoid
+        ib[t] = __ldg(a.i_pre + ts);
+      } else {
+        lf[t] = 0.f;
+        ib[t] = -INFINITY;
+      }
+    }
+    __syncthreads();
+    // ---- A (inclusive prefix of log f), the prefix max of i~ - A, m_t and g_t (warp 0)
+    if (warp == 0) {
+      float a0 = lf[lane], a1 = lf[lane + 32];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float x0 = __shfl_up_sync(0xffffffffu, a0, o), x1 = __shfl_up_sync(0xffffffffu, a1, o);
+        if (lane >= o) {
+          a0 += x0;
+          a1 += x1;
+        }
+      }
+      a1 += __shfl_sync(0xffffffffu, a0, 31);
+      float p0 = ib[lane] - a0, p1 = ib[lane + 32] - a1;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float x0 = __shfl_up_sync(0xffffffffu, p0, o), x1 = __shfl_up_sync(0xffffffffu, p1, o);
+        if (lane >= o) {
+          p0 = fmaxf(p0, x0);
+          p1 = fmaxf(p1, x1);
+        }
+      }
+      p1 = fmaxf(p1, __shfl_sync(0xffffffffu, p0, 31));
+      const float mc = *mcar;
+      const float m0 = a0 + fmaxf(mc, p0), m1 = a1 + fmaxf(mc, p1);
+      A[lane] = a0;
+      A[lane + 32] = a1;
+      mt[lane] = m0;
+      mt[lane + 32] = m1;
+      gt[lane] = expf(a0 + mc - m0);      // 0 for an empty memory (mc = -inf)
+      gt[lane + 32] = expf(a1 + mc - m1);
+    }
+    __syncthreads();
+    // ---- P = (Q K^T) (.) w, w_ts = e^{A_t - A_s + i~_s - m_t} (s <= t)
+    {
+      const int r0 = 16 * (warp >> 1), cc0 = 32 * (warp & 1);
+      float acc[4][4];
+      zero_acc(acc);
+      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return Q[m * LDK + kk]; },
+                      [&](int kk, int nn2) { return K[nn2 * LDK + kk]; }, lane);
+      for_acc(acc, r0, cc0, lane, [&](int t, int s, float x) {
+        P[t * kLDL + s] = s <= t ? x * expf(A[t] - A[s] + ib[s] - mt[t]) : 0.f;
+      });
+    }
+    __syncthreads();
+    // ---- den_t = sum_s P_ts + g_t n . q_t (4 threads per row)
+    {
+      const int t = tid >> 2, part = tid & 3;
+      float s = 0.f;
+      for (int u = part; u < kL; u += 4) s += P[t * kLDL + u];
+      for (int j = part; j < dk; j += 4) s += gt[t] * nn[j] * Q[t * LDK + j];
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      if (part == 0) den[t] = s;
+    }
+    __syncthreads();
+    // ---- h = (P V + diag(g) Q C) / max(|den|, e^{-m})
+    {
+      const int r0 = 16 * (warp >> 1), cc0 = 32 * (warp & 1);
+      float acc[4][4];
+      zero_acc(acc);
+      mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int kk) { return P[m * kLDL + kk]; },
+                      [&](int kk, int nn2) { return V[kk * kLDN + nn2]; }, lane);
+      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return gt[m] * Q[m * LDK + kk]; },
+                      [&](int kk, int nn2) { return C[kk * kLDN + nn2]; }, lane);
+      for_acc(acc, r0, cc0, lane, [&](int t, int c, float x) {
+        if (t < n)
+          a.h[(((size_t)b * T + t0 + t) * H + h) * dv + c0 + c] =
+              x / fmaxf(fabsf(den[t]), expf(-mt[t]));
+      });
+    }
+    __syncthreads();   // C and n are read above; they change below
+    // ---- state: C <- g_L C + K^T diag(w_L) V, n <- g_L n + K^T w_L, m <- m_L
+    {
+      const float mL = mt[kL - 1], gL = gt[kL - 1];
+      float *wl = den;   // den is read above: w_Ls = e^{A_L - A_s + i~_s - m_L} in its place
+      if (tid < kL) wl[tid] = expf(A[kL - 1] - A[tid] + ib[tid] - mL);
+      __syncthreads();
+      auto wL = [&](int s) { return wl[s]; };
+      for (int wt = warp; wt < dk / 8; wt += kWarps) {
+        const int r0 = 16 * (wt >> 1), cc0 = 32 * (wt & 1);
+        float acc[4][4];
+        zero_acc(acc);
+        mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int s) { return K[s * LDK + m] * wL(s); },
+                        [&](int s, int nn2) { return V[s * kLDN + nn2]; }, lane);
+        for_acc(acc, r0, cc0, lane, [&](int j, int c, float x) {
+          C[j * kLDN + c] = gL * C[j * kLDN + c] + x;
+        });
+      }
+      for (int j = tid; j < dk; j += kThreads) {
+        float s = 0.f;
+        for (int u = 0; u < kL; ++u) s += wL(u) * K[u * LDK + j];
+        nn[j] = gL * nn[j] + s;
+      }
+      __syncthreads();
+      if (tid == 0) *mcar = mL;
+    }
+  }
+  __syncthreads();
+  if (a.C_T)
+    for (int i = tid; i < dk * kNV; i += kThreads) {
+      const int j = i / kNV, c = i % kNV;
+      a.C_T[bh * dk * dv + (size_t)j * dv + c0 + c] = C[j * kLDN + c];
+    }
+  if (blockIdx.x == 0) {
+    if (a.n_T)
+      for (int j = tid; j < dk; j += kThreads) a.n_T[bh * dk + j] = nn[j];
+    if (a.m_T && tid == 0) a.m_T[bh] = *mcar;
+  }
+}
+
+template <typename Tin, bool kSplit>
+cudaError_t launch_typed(const gdr_mlstm_args &a, cudaStream_t stream) {
+  const size_t smem = MlstmSmem(a.dk).total * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(mlstm_kernel<Tin, kSplit>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  mlstm_kernel<Tin, kSplit><<<dim3(a.dv / kNV, a.H, a.B), kThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+__global__ void fill_kernel(float *p, size_t n, float x) {
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x)
+    p[i] = x;
+}
+
+}  // namespace
+
+cudaError_t fill_f32(float *p, size_t n, float x, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  fill_kernel<<<(unsigned)((n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024), 256, 0, stream>>>(p, n, x);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mlstm(const gdr_mlstm_args &a, cudaStream_t stream) {
+  return a.dtype == GDR_BF16 ? launch_typed<__nv_bfloat16, false>(a, stream)
+                             : launch_typed<float, true>(a, stream);
+}
+
+}  // namespace gdr

@@ -59,6 +59,13 @@ class gdr_muir_args(ctypes.Structure):
                 ("workspace", _vp), ("workspace_bytes", ctypes.c_size_t)]
 
 
+class gdr_mlstm_args(ctypes.Structure):
+    _fields_ = [("dtype", _c_int), ("B", _c_int), ("H", _c_int), ("T", _c_int), ("dk", _c_int),
+                ("dv", _c_int), ("q", _vp), ("k", _vp), ("v", _vp), ("f_pre", _fp), ("i_pre", _fp),
+                ("C0", _fp), ("n0", _fp), ("m0", _fp), ("h", _fp), ("C_T", _fp), ("n_T", _fp),
+                ("m_T", _fp)]
+
+
 class GdrError(RuntimeError):
     def __init__(self, fn, code):
         self.code = int(code)
@@ -86,6 +93,7 @@ def _load():
             lib.gdr_muir_forward.argtypes = [ctypes.POINTER(gdr_muir_args), _vp]
             lib.gdr_muir_workspace_size.argtypes = [ctypes.POINTER(gdr_muir_args),
                                                     ctypes.POINTER(ctypes.c_size_t)]
+            lib.gdr_mlstm_forward.argtypes = [ctypes.POINTER(gdr_mlstm_args), _vp]
             lib.gdr_decode_step.argtypes = [ctypes.POINTER(gdr_step_args), _vp]
             lib.gdr_state_init.argtypes = [_fp, _c_int, _c_int, _c_int, _c_int, _fp, _vp]
             lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
@@ -93,7 +101,8 @@ def _load():
             lib.gdr_status_string.argtypes = [_c_int]
             for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size",
                        "gdr_backward_chunked", "gdr_backward_workspace_size",
-                       "gdr_muir_forward", "gdr_muir_workspace_size", "gdr_decode_step",
+                       "gdr_muir_forward", "gdr_muir_workspace_size", "gdr_mlstm_forward",
+                       "gdr_decode_step",
                        "gdr_state_init", "gdr_read_status", "gdr_version"):
                 getattr(lib, fn).restype = _c_int
             _lib = lib
@@ -367,6 +376,40 @@ def gdr_muir_forward(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat=None, rms_we
                      S_T, chunk, algo, workspace, unfused)
     _check("gdr_muir_forward", _load().gdr_muir_forward(ctypes.byref(a), _stream(stream)))
     return y, S_T
+
+
+def gdr_mlstm_forward(q, k, v, f_pre, i_pre, C0=None, n0=None, m0=None, *, h=None,
+                      want_state=True, stream=None):
+    """xLSTM's mLSTM cell (include/gdr.h, gdr_mlstm_forward): q, k [B, T, H, dk], v
+    [B, T, H, dv] (bf16 or fp32), gate pre-activations f_pre, i_pre [B, T, H] fp32, optional
+    stabilized state C0 [B, H, dk, dv], n0 [B, H, dk], m0 [B, H].  Returns (h, C_T, n_T, m_T)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dname, tdt = _dtype_of(q)
+    _need(q, "q", tdt, (B, T, H, dk))
+    _need(k, "k", tdt, (B, T, H, dk))
+    _need(v, "v", tdt, (B, T, H, dv))
+    _need(f_pre, "f_pre", torch.float32, (B, T, H))
+    _need(i_pre, "i_pre", torch.float32, (B, T, H))
+    if C0 is not None:
+        _need(C0, "C0", torch.float32, (B, H, dk, dv))
+        _need(n0, "n0", torch.float32, (B, H, dk))
+        _need(m0, "m0", torch.float32, (B, H))
+    dev = q.device
+    if h is None:
+        h = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    C_T = n_T = m_T = None
+    if want_state:
+        C_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+        n_T = torch.empty((B, H, dk), dtype=torch.float32, device=dev)
+        m_T = torch.empty((B, H), dtype=torch.float32, device=dev)
+    a = gdr_mlstm_args()
+    a.dtype, a.B, a.H, a.T, a.dk, a.dv = DTYPES[dname], B, H, T, dk, dv
+    for name, t in (("q", q), ("k", k), ("v", v), ("f_pre", f_pre), ("i_pre", i_pre), ("C0", C0),
+                    ("n0", n0), ("m0", m0), ("h", h), ("C_T", C_T), ("n_T", n_T), ("m_T", m_T)):
+        setattr(a, name, _ptr(t))
+    _check("gdr_mlstm_forward", _load().gdr_mlstm_forward(ctypes.byref(a), _stream(stream)))
+    return h, C_T, n_T, m_T
 
 
 def gdr_decode_step(form, q, k, v, log_w, e1, e2, S, *, o=None, stream=None):

@@ -25,7 +25,7 @@ from dataclasses import dataclass, replace
 import numpy as np
 
 __all__ = ["Workload", "PRESETS", "round_bf16", "round_f32", "forward_inputs",
-           "decode_state", "decode_step_inputs", "muir_inputs"]
+           "decode_state", "decode_step_inputs", "muir_inputs", "mlstm_inputs"]
 
 
 def round_f32(x) -> np.ndarray:
@@ -191,3 +191,17 @@ def muir_inputs(w: Workload, seed: int | None = None, static_gains: bool = True)
     else:
         out["gamma_stat"] = out["rms_weight"] = None
     return out
+
+
+def mlstm_inputs(w: Workload, seed: int | None = None, i_mu: float = 0.0, i_sd: float = 1.0) -> dict:
+    """Inputs of one mLSTM call (shapes of ``w``): q, k ~ N(0, 1/d_k) per entry (the scaled
+    keys of the cell), v ~ N(0, 1) at the storage dtype, and fp32 gate pre-activations
+    f~ ~ N(3, 1) (forget gates near sigmoid(3) = 0.95) and i~ ~ N(i_mu, i_sd)."""
+    rng = np.random.default_rng(w.seed + 20 if seed is None else seed)
+    sk = (w.B, w.T, w.H, w.dk)
+    sv = (w.B, w.T, w.H, w.dv)
+    s = 1.0 / np.sqrt(w.dk)
+    return {"q": _round(rng.normal(0.0, s, sk), w.dtype), "k": _round(rng.normal(0.0, s, sk), w.dtype),
+            "v": _round(rng.standard_normal(sv), w.dtype),
+            "f_pre": round_f32(rng.normal(3.0, 1.0, (w.B, w.T, w.H))),
+            "i_pre": round_f32(rng.normal(i_mu, i_sd, (w.B, w.T, w.H)))}
