@@ -71,6 +71,14 @@ def muir_algorithmic_bytes(w) -> int:
     return w.B * w.T * w.H * per_token_head + w.B * w.H * w.dk * w.dv * 4
 
 
+def mlstm_algorithmic_bytes(w) -> int:
+    """xLSTM's mLSTM cell: q, k, v in (input dtype), the two fp32 gate pre-activations in,
+    h out (fp32), the final state out."""
+    eb = 2 if w.dtype == "bf16" else 4
+    per_token_head = eb * (2 * w.dk + w.dv) + 8 + 4 * w.dv
+    return w.B * w.T * w.H * per_token_head + w.B * w.H * (w.dk * w.dv + w.dk + 1) * 4
+
+
 def fwd_flops(w) -> int:
     """Algorithmic flops of the single-write (GDN-2) chunk form per token-head:
     6 d^2 (state GEMMs Y S0, Q S0, K~^T V~) + 5 C d (L, M, [U Y], M V~) + C^2 / 3 (T^-1)."""
@@ -493,6 +501,46 @@ def bench_muir(ctx, args, gdr):
     return out
 
 
+def bench_mlstm(ctx, args, gdr):
+    """gdr_mlstm_forward (xLSTM's mLSTM cell with the stabilizer) on the bf16 shapes of the
+    two forward workloads, device-resident: milliseconds per call and the HBM roofline
+    fraction of the algorithmic bytes."""
+    torch = ctx.torch
+    out = []
+    for name in ("gdn2_bf16", "rwkv7_bf16"):
+        w = synth.PRESETS[name]
+        inp = synth.mlstm_inputs(w, seed=rank_seed(w.seed + 20, ctx.rank))
+        d = {k: torch.from_numpy(inp[k]).to(ctx.dev, torch.bfloat16) for k in ("q", "k", "v")}
+        g = {k: torch.from_numpy(inp[k]).to(ctx.dev) for k in ("f_pre", "i_pre")}
+        h = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=ctx.dev)
+
+        def call():
+            gdr.gdr_mlstm_forward(d["q"], d["k"], d["v"], g["f_pre"], g["i_pre"], h=h,
+                                  want_state=False)
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        e0, e1 = ctx.event(), ctx.event()
+        n = 5
+        e0.record(ctx.stream)
+        for _ in range(n):
+            call()
+        e1.record(ctx.stream)
+        torch.cuda.synchronize()
+        ms = ctx.max_over_ranks(e0.elapsed_time(e1)) / n
+        nbytes = mlstm_algorithmic_bytes(w)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out.append({"workload": "mlstm on " + name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk,
+                    "dv": w.dv, "ms_per_call": ms, "launches_per_call": 1,
+                    "tokens_per_s": w.tokens * ctx.world / (ms * 1e-3),
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
+                                 "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],
+                                 "bytes_per_call": nbytes}})
+        del d, g, h
+        torch.cuda.empty_cache()
+    return out
+
+
 def bench_e2e(ctx, args, gdr, w, inp, names, step, o):
     """Same call with host inputs: pinned H2D copies, the forward, D2H of o, all timed."""
     torch = ctx.torch
@@ -589,6 +637,8 @@ def main():
                     help="decode batch B (default: the workload's); for profiler captures")
     ap.add_argument("--no-other-workloads", action="store_true",
                     help="skip the timing of the other forward workloads")
+    ap.add_argument("--no-mlstm", action="store_true",
+                    help="skip the timing of the mLSTM cell (gdr_mlstm_forward)")
     ap.add_argument("--no-muir", action="store_true",
                     help="skip the timing of the Muir mixer (gdr_muir_forward)")
     ap.add_argument("--no-backward", action="store_true",
@@ -626,6 +676,7 @@ def main():
     bwd = (bench_backward(ctx, args, gdr)
            if (args.only == "all" and not args.no_backward) or args.only == "backward" else None)
     muir = bench_muir(ctx, args, gdr) if args.only == "all" and not args.no_muir else None
+    mlstm = bench_mlstm(ctx, args, gdr) if args.only == "all" and not args.no_mlstm else None
     ctx.barrier()
     if world > 1:
         dist.destroy_process_group()
@@ -674,6 +725,8 @@ def main():
         line["backward"] = bwd
     if muir is not None:
         line["muir"] = muir
+    if mlstm is not None:
+        line["mlstm"] = mlstm
     print(json.dumps(line), flush=True)
     return 0
 

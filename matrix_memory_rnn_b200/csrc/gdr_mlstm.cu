@@ -57,8 +57,28 @@ struct MlstmSmem {
   }
 };
 
-__device__ __forceinline__ float ld_elem(const float *p, size_t i) { return __ldg(p + i); }
-__device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p, size_t i) { return __bfloat162float(p[i]); }
+// 16-byte pieces of the chunk's q, k (64 x dk) and v slice (64 x 64) held in registers:
+// the next chunk is loaded while the current one is computed.  kE = elements per piece.
+template <typename Tin>
+struct ChunkRegs {
+  static constexpr int kE = 16 / sizeof(Tin);
+  static constexpr int kQK = kL * 128 / kE / kThreads;   // pieces per thread of q (and of k), d_k = 128
+  static constexpr int kV = kL * kNV / kE / kThreads;
+  uint4 q[kQK], k[kQK], v[kV];
+  float lf, ib;
+};
+__device__ __forceinline__ void widen(const uint4 &u, float *dst, const __nv_bfloat16 *) {
+  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 x = __bfloat1622float2(h[i]);
+    dst[2 * i] = x.x;
+    dst[2 * i + 1] = x.y;
+  }
+}
+__device__ __forceinline__ void widen(const uint4 &u, float *dst, const float *) {
+  *reinterpret_cast<float4 *>(dst) = *reinterpret_cast<const float4 *>(&u);
+}
 
 template <typename Tin, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1) mlstm_kernel(gdr_mlstm_args a) {
@@ -83,32 +103,61 @@ __global__ void __launch_bounds__(kThreads, 1) mlstm_kernel(gdr_mlstm_args a) {
   for (int j = tid; j < dk; j += kThreads) nn[j] = a.n0 ? a.n0[bh * dk + j] : 0.f;
   if (tid == 0) *mcar = a.m0 ? a.m0[bh] : -INFINITY;
 
+  // ---- chunk loads (padding: q = k = v = 0, log f = 0, i~ = -inf), one chunk ahead
+  using R = ChunkRegs<Tin>;
+  R rg;
+  const int gq = dk / R::kE;                 // pieces per row of q / k
+  const int nq = kL * gq / kThreads;         // pieces per thread (d_k = 64: half of kQK)
+  auto fetch = [&](int t0) {
+#pragma unroll
+    for (int u = 0; u < R::kQK; ++u) {
+      if (u >= nq) break;
+      const int i = tid + u * kThreads, t = i / gq, j = (i % gq) * R::kE;
+      const size_t ik = (((size_t)b * T + t0 + t) * H + h) * dk + j;
+      const bool in = t0 + t < T;
+      rg.q[u] = in ? __ldg(reinterpret_cast<const uint4 *>(q + ik)) : make_uint4(0u, 0u, 0u, 0u);
+      rg.k[u] = in ? __ldg(reinterpret_cast<const uint4 *>(k + ik)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < R::kV; ++u) {
+      const int i = tid + u * kThreads, t = i / (kNV / R::kE), c = (i % (kNV / R::kE)) * R::kE;
+      const bool in = t0 + t < T;
+      rg.v[u] = in ? __ldg(reinterpret_cast<const uint4 *>(v + (((size_t)b * T + t0 + t) * H + h) * dv + c0 + c))
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (tid < kL) {
+      const bool in = t0 + tid < T;
+      const size_t ts = ((size_t)b * T + t0 + tid) * H + h;
+      rg.lf = in ? __ldg(a.f_pre + ts) : 0.f;
+      rg.ib = in ? __ldg(a.i_pre + ts) : -INFINITY;
+    }
+  };
+  auto commit = [&](int n) {
+#pragma unroll
+    for (int u = 0; u < R::kQK; ++u) {
+      if (u >= nq) break;
+      const int i = tid + u * kThreads, t = i / gq, j = (i % gq) * R::kE;
+      widen(rg.q[u], Q + t * LDK + j, q);
+      widen(rg.k[u], K + t * LDK + j, k);
+    }
+#pragma unroll
+    for (int u = 0; u < R::kV; ++u) {
+      const int i = tid + u * kThreads, t = i / (kNV / R::kE), c = (i % (kNV / R::kE)) * R::kE;
+      widen(rg.v[u], V + t * kLDN + c, v);
+    }
+    if (tid < kL) {
+      const float x = rg.lf;   // log sigmoid; padding keeps log f = 0
+      lf[tid] = tid < n ? (x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x))) : 0.f;
+      ib[tid] = rg.ib;
+    }
+  };
+  fetch(0);
+
   for (int t0 = 0; t0 < T; t0 += kL) {
     const int n = min(kL, T - t0);
     __syncthreads();   // the previous chunk is done with every buffer
-    // ---- chunk tiles and gates (padding: q = k = v = 0, log f = 0, i~ = -inf)
-    for (int i = tid; i < kL * dk; i += kThreads) {
-      const int t = i / dk, j = i % dk;
-      const size_t ik = (((size_t)b * T + t0 + t) * H + h) * dk + j;
-      Q[t * LDK + j] = t < n ? ld_elem(q, ik) : 0.f;
-      K[t * LDK + j] = t < n ? ld_elem(k, ik) : 0.f;
-    }
-    for (int i = tid; i < kL * kNV; i += kThreads) {
-      const int t = i / kNV, c = i % kNV;
-      V[t * kLDN + c] = t < n ? ld_elem(v, (((size_t)b * T + t0 + t) * H + h) * dv + c0 + c) : 0.f;
-    }
-    if (tid < kL) {
-      const int t = tid;
-      const size_t ts = ((size_t)b * T + t0 + t) * H + h;
-      if (t < n) {
-        const float x = __ldg(a.f_pre + ts);
-        lf[t] = x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));   // log sigmoid
-        ib[t] = __ldg(a.i_pre + ts);
-      } else {
-        lf[t] = 0.f;
-        ib[t] = -INFINITY;
-      }
-    }
+    commit(n);
+    if (t0 + kL < T) fetch(t0 + kL);
     __syncthreads();
     // ---- A (inclusive prefix of log f), the prefix max of i~ - A, m_t and g_t (warp 0)
     if (warp == 0) {
