@@ -342,6 +342,19 @@ typedef struct {
  */
 gdr_status gdr_decode_step(const gdr_step_args *args, void *stream);
 
+/*
+ * S_out[i] = M[i] S_in[i] + Q[i] for i < BH: M [BH][dk][dk], S_in, Q, S_out [BH][dk][dv],
+ * fp32 (S_in or Q NULL = 0; S_out may alias Q, not S_in).  In the storage orientation a
+ * sequence segment maps its entry state affinely to its exit state, S_out = M S_in + Q
+ * ("Muir ...", section 4.2 eq. (10): the chunk's end state is affine in its start state,
+ * and so is any run of chunks); M is the segment run from S_in = I with v = 0, Q the run
+ * from S_in = 0.  Composing the maps of consecutive segments gives each segment its entry
+ * state (sequence parallelism).  Products as tf32 with the three-product split (fp32
+ * accuracy).  dk, dv in {16, 32, 64, 128}.
+ */
+gdr_status gdr_state_compose(float *S_out, const float *M, const float *S_in, const float *Q,
+                             int BH, int dk, int dv, void *stream);
+
 /* S[B][H][dk][dv] = src (device pointer, same layout) or 0 when src == NULL. */
 gdr_status gdr_state_init(float *S, int B, int H, int dk, int dv, const float *src, void *stream);
 

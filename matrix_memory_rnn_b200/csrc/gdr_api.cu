@@ -433,6 +433,16 @@ gdr_status gdr_mlstm_forward(const gdr_mlstm_args *a, void *stream) {
   return cuda_status(gdr::launch_mlstm(*a, s));
 }
 
+gdr_status gdr_state_compose(float *S_out, const float *M, const float *S_in, const float *Q,
+                             int BH, int dk, int dv, void *stream) {
+  if (BH < 0 || !dim_ok(dk) || !dim_ok(dv)) return GDR_ERR_INVALID_ARG;
+  if (BH == 0) return GDR_OK;
+  if (!S_out || !M) return GDR_ERR_INVALID_ARG;
+  if (S_in && S_in == S_out) return GDR_ERR_INVALID_ARG;
+  return cuda_status(gdr::launch_state_compose(S_out, M, S_in, Q, BH, dk, dv,
+                                               static_cast<cudaStream_t>(stream)));
+}
+
 gdr_status gdr_read_status(void *workspace, void *stream, gdr_status *device_status) {
   if (!workspace || !device_status) return GDR_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

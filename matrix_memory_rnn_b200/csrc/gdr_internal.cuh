@@ -102,6 +102,10 @@ cudaError_t launch_muir_prologue(const MuirParams &m, gdr_dtype dtype, void *qh,
 cudaError_t launch_muir_epilogue(const MuirParams &m, gdr_dtype dtype, const float *o, float *y,
                                  cudaStream_t stream);
 
+// S_out = M S_in + Q per head (gdr_state_compose).
+cudaError_t launch_state_compose(float *S_out, const float *M, const float *S_in, const float *Q,
+                                 int BH, int dk, int dv, cudaStream_t stream);
+
 // xLSTM's mLSTM cell (gdr_mlstm_forward); p[0 .. n) = x.
 cudaError_t launch_mlstm(const gdr_mlstm_args &a, cudaStream_t stream);
 cudaError_t fill_f32(float *p, size_t n, float x, cudaStream_t stream);

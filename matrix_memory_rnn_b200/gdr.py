@@ -94,6 +94,7 @@ def _load():
             lib.gdr_muir_workspace_size.argtypes = [ctypes.POINTER(gdr_muir_args),
                                                     ctypes.POINTER(ctypes.c_size_t)]
             lib.gdr_mlstm_forward.argtypes = [ctypes.POINTER(gdr_mlstm_args), _vp]
+            lib.gdr_state_compose.argtypes = [_fp, _fp, _fp, _fp, _c_int, _c_int, _c_int, _vp]
             lib.gdr_decode_step.argtypes = [ctypes.POINTER(gdr_step_args), _vp]
             lib.gdr_state_init.argtypes = [_fp, _c_int, _c_int, _c_int, _c_int, _fp, _vp]
             lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
@@ -102,6 +103,7 @@ def _load():
             for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size",
                        "gdr_backward_chunked", "gdr_backward_workspace_size",
                        "gdr_muir_forward", "gdr_muir_workspace_size", "gdr_mlstm_forward",
+                       "gdr_state_compose",
                        "gdr_decode_step",
                        "gdr_state_init", "gdr_read_status", "gdr_version"):
                 getattr(lib, fn).restype = _c_int
@@ -437,6 +439,20 @@ def gdr_decode_step(form, q, k, v, log_w, e1, e2, S, *, o=None, stream=None):
     a.e1, a.e2, a.S, a.o = _ptr(e1), _ptr(e2), _ptr(S), _ptr(o)
     _check("gdr_decode_step", _load().gdr_decode_step(ctypes.byref(a), _stream(stream)))
     return o
+
+
+def gdr_state_compose(M, S_in, Q, *, out=None, stream=None):
+    """M [B, H, dk, dk] S_in [B, H, dk, dv] + Q [B, H, dk, dv] per head (S_in None = 0)."""
+    B, H, dk, dv = Q.shape
+    _need(M, "M", torch.float32, (B, H, dk, dk))
+    _need(Q, "Q", torch.float32, (B, H, dk, dv))
+    if S_in is not None:
+        _need(S_in, "S_in", torch.float32, (B, H, dk, dv))
+    if out is None:
+        out = torch.empty_like(Q)
+    _check("gdr_state_compose", _load().gdr_state_compose(_ptr(out), _ptr(M), _ptr(S_in), _ptr(Q),
+                                                          B * H, dk, dv, _stream(stream)))
+    return out
 
 
 def gdr_state_init(S, src=None, *, stream=None):
