@@ -106,3 +106,84 @@ def test_state_init_rejects_bad_arguments_on_host(lib):
     assert lib.gdr_state_init(None, 1, 1, 64, 64, None, None) == 1
     assert lib.gdr_state_init(None, 0, 1, 64, 64, None, None) == 0
     assert lib.gdr_state_init(None, 1, 1, 48, 64, None, None) == 1
+
+
+def _bwd_args(**kw):
+    a = gdr.gdr_bwd_args()
+    a.form, a.dtype, a.B, a.H, a.T, a.dk, a.dv, a.chunk = 1, 1, 1, 1, 8, 64, 64, 64
+    fake = ctypes.c_void_p(0x10000)
+    for name in ("q", "k", "v", "log_w", "e1", "dO", "g_q", "g_k", "g_v", "g_log_w", "g_e1"):
+        setattr(a, name, fake)
+    for name, val in kw.items():
+        setattr(a, name, val)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=32), 2), (dict(dv=16), 2), (dict(chunk=24), 2), (dict(form=9), 1), (dict(T=-1), 1),
+    (dict(dO=None), 1), (dict(g_q=None), 1), (dict(g_e1=None), 1),
+    (dict(g_k=ctypes.c_void_p(0x10004)), 3), (dict(workspace=None), 7),
+])
+def test_backward_rejects_bad_arguments_on_host(lib, kw, code):
+    a = _bwd_args(**kw)
+    assert lib.gdr_backward_chunked(ctypes.byref(a), None) == code
+
+
+def test_backward_workspace_size(lib):
+    a = _bwd_args()
+    n = ctypes.c_size_t(0)
+    assert lib.gdr_backward_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    assert n.value >= 3 * 64 * 64 * 4 and n.value % 256 == 0   # two states, one adjoint at T = 8
+    a = _bwd_args(B=0)
+    assert lib.gdr_backward_chunked(ctypes.byref(a), None) == 0
+
+
+def _muir_args(**kw):
+    a = gdr.gdr_muir_args()
+    a.dtype, a.B, a.H, a.T, a.dk, a.dv, a.chunk = 1, 1, 1, 8, 64, 64, 64
+    fake = ctypes.c_void_p(0x10000)
+    for name in ("q", "k", "v", "zf", "zb", "zw", "zq", "zg", "a_log", "y"):
+        setattr(a, name, fake)
+    a.rms_eps = 1e-6
+    for name, val in kw.items():
+        setattr(a, name, val)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=48), 2), (dict(chunk=24), 2), (dict(dtype=4), 1), (dict(algo=9), 1),
+    (dict(zq=None), 1), (dict(a_log=None), 1), (dict(y=None), 1), (dict(rms_eps=-1.0), 1),
+    (dict(zg=ctypes.c_void_p(0x10002)), 3), (dict(workspace=None), 7),
+])
+def test_muir_rejects_bad_arguments_on_host(lib, kw, code):
+    a = _muir_args(**kw)
+    assert lib.gdr_muir_forward(ctypes.byref(a), None) == code
+
+
+def _mlstm_args(**kw):
+    a = gdr.gdr_mlstm_args()
+    a.dtype, a.B, a.H, a.T, a.dk, a.dv = 1, 1, 1, 8, 64, 64
+    fake = ctypes.c_void_p(0x10000)
+    for name in ("q", "k", "v", "f_pre", "i_pre", "h"):
+        setattr(a, name, fake)
+    for name, val in kw.items():
+        setattr(a, name, val)
+    return a
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(dk=32), 2), (dict(dv=16), 2), (dict(dtype=3), 1), (dict(T=-2), 1),
+    (dict(i_pre=None), 1), (dict(h=None), 1), (dict(C0=ctypes.c_void_p(0x10000)), 1),
+    (dict(v=ctypes.c_void_p(0x10008)), 3),
+])
+def test_mlstm_rejects_bad_arguments_on_host(lib, kw, code):
+    a = _mlstm_args(**kw)
+    assert lib.gdr_mlstm_forward(ctypes.byref(a), None) == code
+
+
+def test_state_compose_rejects_bad_arguments_on_host(lib):
+    fake = ctypes.c_void_p(0x10000)
+    assert lib.gdr_state_compose(None, fake, None, fake, 2, 64, 64, None) == 1
+    assert lib.gdr_state_compose(fake, fake, fake, fake, 2, 48, 64, None) == 1
+    assert lib.gdr_state_compose(fake, fake, fake, None, 2, 64, 64, None) == 1   # S_in aliases S_out
+    assert lib.gdr_state_compose(fake, fake, None, None, 0, 64, 64, None) == 0
