@@ -90,7 +90,7 @@ def fwd_flops(w) -> int:
 # current kernels on a quarter-size case, scaled by the units processed).  Forward: prep +
 # chain, per (b, h, 64-token chunk) of the GDN-2 bf16 d = 128 tensor-core path; decode: per
 # (b, h) step of the d = 128 persistent kernel.  Must be re-measured when those kernels change.
-FWD_TC_TRAFFIC_PER_CHUNK = (117.6e6 + 32.0e6 + 76.1e6 + 11.1e6) / 1024
+FWD_TC_TRAFFIC_PER_CHUNK = (117.6e6 + 33.9e6 + 76.1e6 + 4.7e6) / 1024
 DEC_TRAFFIC_PER_HEAD = (137.9e6 + 81.0e6) / (64 * 32)
 
 
