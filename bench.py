@@ -357,7 +357,7 @@ def bench_forward(ctx, args, gdr):
            "clocks": clk.summary(), "launches": args.steps * per_call,
            "launches_per_call": per_call}
     if args.only == "all":
-        res["e2e"] = bench_e2e(ctx, args, gdr, w, inp, names, step, o)
+        res["e2e"] = bench_e2e(ctx, args, gdr, w, inp, names, ws)
     return res
 
 
@@ -541,40 +541,64 @@ def bench_mlstm(ctx, args, gdr):
     return out
 
 
-def bench_e2e(ctx, args, gdr, w, inp, names, step, o):
-    """Same call with host inputs: pinned H2D copies, the forward, D2H of o, all timed."""
+def bench_e2e(ctx, args, gdr, w, inp, names, ws):
+    """The same call with host inputs, as a pipelined loop: every step copies its inputs
+    from pinned host memory to the device, runs the forward and copies o back to pinned
+    host memory, all inside the timed region.  Two buffer sets on three streams (upload,
+    compute, download) let step i + 1's upload and step i - 1's download overlap step i
+    (PCIe is full duplex); a buffer is reused only after the step that used it finished."""
     torch = ctx.torch
     host = {k: None if inp[k] is None else torch.from_numpy(inp[k]) for k in names}
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     pinned = {k: None if t is None else
               t.to(torch.float32 if k == "log_w" else tdt).pin_memory() for k, t in host.items()}
-    dev_bufs = {k: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=ctx.dev)
-                for k, t in pinned.items()}
-    o_host = torch.empty(o.shape, dtype=torch.float32, pin_memory=True)
+    dev = [{k: None if t is None else torch.empty(t.shape, dtype=t.dtype, device=ctx.dev)
+            for k, t in pinned.items()} for _ in range(2)]
+    o = [torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=ctx.dev) for _ in range(2)]
+    o_host = [torch.empty(o[0].shape, dtype=torch.float32, pin_memory=True) for _ in range(2)]
     h2d = sum(t.numel() * t.element_size() for t in pinned.values() if t is not None)
-    d2h = o.numel() * 4
+    d2h = o[0].numel() * 4
+    s_in, s_out, s_comp = torch.cuda.Stream(), torch.cuda.Stream(), ctx.stream
+    in_done, comp_done, out_done = ([ctx.event() for _ in range(2)] for _ in range(3))
 
-    def e2e_step():
-        for k, t in pinned.items():
-            if t is not None:
-                dev_bufs[k].copy_(t, non_blocking=True)
-        step(dev_bufs)
-        o_host.copy_(o, non_blocking=True)
+    def e2e_step(i):
+        b = i % 2
+        s_in.wait_event(comp_done[b])        # the step that last read dev[b] has finished
+        with torch.cuda.stream(s_in):
+            for k, t in pinned.items():
+                if t is not None:
+                    dev[b][k].copy_(t, non_blocking=True)
+            in_done[b].record(s_in)
+        s_comp.wait_event(in_done[b])
+        s_comp.wait_event(out_done[b])       # o[b] has been read back
+        with torch.cuda.stream(s_comp):
+            bb = dev[b]
+            gdr.gdr_forward_chunked(w.form, bb["q"], bb["k"], bb["v"], bb["log_w"], bb["e1"],
+                                    bb["e2"], None, chunk=w.chunk, algo=args.algo, o=o[b],
+                                    want_state=False, workspace=ws, stream=s_comp)
+            comp_done[b].record(s_comp)
+        s_out.wait_event(comp_done[b])
+        with torch.cuda.stream(s_out):
+            o_host[b].copy_(o[b], non_blocking=True)
+            out_done[b].record(s_out)
 
     n = max(3, min(args.steps, 10))
-    for _ in range(2):
-        e2e_step()
+    for i in range(2):
+        e2e_step(i)
     torch.cuda.synchronize()
     ctx.barrier()
     e0, e1 = ctx.event(), ctx.event()
-    e0.record(ctx.stream)
-    for _ in range(n):
-        e2e_step()
-    e1.record(ctx.stream)
+    e0.record(s_in)
+    s_comp.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(n):
+        e2e_step(i)
+    e1.record(s_out)
     torch.cuda.synchronize()
     ms = ctx.max_over_ranks(e0.elapsed_time(e1)) / n
     return {"value": w.tokens * ctx.world / (ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "pipeline": "2 buffer sets; upload, compute and download on separate streams"}
 
 
 def bench_decode(ctx, args, gdr):
