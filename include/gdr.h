@@ -245,7 +245,8 @@ gdr_status gdr_backward_chunked(const gdr_bwd_args *args, void *stream);
  *   log alpha = -exp(a_log) softplus(zf),  b = 2 sigmoid(zb),  w = sigmoid(zw)
  *   o = the GDN-2 recurrence on (q^, k^, v^, log alpha, b, w)   (as gdr_forward_chunked)
  *   y = rms_weight (.) o / sqrt(mean_c o_c^2 + rms_eps) (.) silu(zg)
- * with l2norm(x) = x / max(||x||_2, 1e-12).
+ * with l2norm(x) = x / max(||x||_2, 1e-12).  Every array pointer, gamma_stat and
+ * rms_weight included, must be 16-byte aligned (GDR_ERR_MISALIGNED otherwise).
  */
 typedef struct {
   gdr_dtype dtype;

@@ -341,6 +341,8 @@ gdr_status gdr_muir_forward(const gdr_muir_args *a, void *stream) {
       if (!aligned16(p)) return GDR_ERR_MISALIGNED;
   }
   if ((a->S0 && !aligned16(a->S0)) || (a->S_T && !aligned16(a->S_T))) return GDR_ERR_MISALIGNED;
+  if ((a->gamma_stat && !aligned16(a->gamma_stat)) || (a->rms_weight && !aligned16(a->rms_weight)))
+    return GDR_ERR_MISALIGNED;
   if (a->B == 0 || a->H == 0) return GDR_OK;
   if (a->T == 0) {
     if (!a->S_T) return GDR_OK;
