@@ -59,10 +59,10 @@ struct MlstmSmem {
 
 // 16-byte pieces of the chunk's q, k (64 x dk) and v slice (64 x 64) held in registers:
 // the next chunk is loaded while the current one is computed.  kE = elements per piece.
-template <typename Tin>
+template <typename Tin, int kDK>
 struct ChunkRegs {
   static constexpr int kE = 16 / sizeof(Tin);
-  static constexpr int kQK = kL * 128 / kE / kThreads;   // pieces per thread of q (and of k), d_k = 128
+  static constexpr int kQK = kL * kDK / kE / kThreads;   // pieces per thread of q (and of k)
   static constexpr int kV = kL * kNV / kE / kThreads;
   uint4 q[kQK], k[kQK], v[kV];
   float lf, ib;
@@ -80,10 +80,12 @@ __device__ __forceinline__ void widen(const uint4 &u, float *dst, const float *)
   *reinterpret_cast<float4 *>(dst) = *reinterpret_cast<const float4 *>(&u);
 }
 
-template <typename Tin, bool kSplit>
-__global__ void __launch_bounds__(kThreads, 1) mlstm_kernel(gdr_mlstm_args a) {
+// d_k = 64 keeps two CTAs per SM (registers and shared memory), d_k = 128 one.
+template <typename Tin, bool kSplit, int kDK>
+__global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_mlstm_args a) {
   extern __shared__ float sm[];
-  const int dk = a.dk, dv = a.dv, T = a.T, H = a.H;
+  constexpr int dk = kDK;
+  const int dv = a.dv, T = a.T, H = a.H;
   const MlstmSmem L(dk);
   const int LDK = L.LDK;
   const int c0 = blockIdx.x * kNV, h = blockIdx.y, b = blockIdx.z;
@@ -104,7 +106,7 @@ __global__ void __launch_bounds__(kThreads, 1) mlstm_kernel(gdr_mlstm_args a) {
   if (tid == 0) *mcar = a.m0 ? a.m0[bh] : -INFINITY;
 
   // ---- chunk loads (padding: q = k = v = 0, log f = 0, i~ = -inf), one chunk ahead
-  using R = ChunkRegs<Tin>;
+  using R = ChunkRegs<Tin, kDK>;
   R rg;
   const int gq = dk / R::kE;                 // pieces per row of q / k
   const int nq = kL * gq / kThreads;         // pieces per thread (d_k = 64: half of kQK)
@@ -269,13 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1) mlstm_kernel(gdr_mlstm_args a) {
   }
 }
 
-template <typename Tin, bool kSplit>
+template <typename Tin, bool kSplit, int kDK>
 cudaError_t launch_typed(const gdr_mlstm_args &a, cudaStream_t stream) {
-  const size_t smem = MlstmSmem(a.dk).total * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(mlstm_kernel<Tin, kSplit>,
+  const size_t smem = MlstmSmem(kDK).total * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(mlstm_kernel<Tin, kSplit, kDK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  mlstm_kernel<Tin, kSplit><<<dim3(a.dv / kNV, a.H, a.B), kThreads, smem, stream>>>(a);
+  mlstm_kernel<Tin, kSplit, kDK><<<dim3(a.dv / kNV, a.H, a.B), kThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -293,8 +295,10 @@ cudaError_t fill_f32(float *p, size_t n, float x, cudaStream_t stream) {
 }
 
 cudaError_t launch_mlstm(const gdr_mlstm_args &a, cudaStream_t stream) {
-  return a.dtype == GDR_BF16 ? launch_typed<__nv_bfloat16, false>(a, stream)
-                             : launch_typed<float, true>(a, stream);
+  if (a.dtype == GDR_BF16)
+    return a.dk == 64 ? launch_typed<__nv_bfloat16, false, 64>(a, stream)
+                      : launch_typed<__nv_bfloat16, false, 128>(a, stream);
+  return a.dk == 64 ? launch_typed<float, true, 64>(a, stream) : launch_typed<float, true, 128>(a, stream);
 }
 
 }  // namespace gdr
