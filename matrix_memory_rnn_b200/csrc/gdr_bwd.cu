@@ -162,10 +162,11 @@ struct ChunkSmem {
 // Loads one chunk (rows past n zero), forms lam and pi, decides the exact path and,
 // on the pivot path, scales Q -> Q~, U -> U~, K -> K', Z -> Z' in place.  With
 // `grads` also loads V (GDN-2: wg (.) v) and dO.  Returns the exact-path flag.
-template <typename Tin>
+template <typename Tin, int kDK, int kDV>
 __device__ bool load_chunk(const BwdParams &p, const ChunkSmem &L, float *sm, int b, int h,
                            int t0, int n, bool grads) {
-  const int dk = p.dk, dv = p.dv, T = p.T, H = p.H, LDK = L.LDK, LDV = L.LDV;
+  constexpr int dk = kDK, dv = kDV;
+  const int T = p.T, H = p.H, LDK = L.LDK, LDV = L.LDV;
   const int tid = threadIdx.x;
   const Tin *q = static_cast<const Tin *>(p.q), *k = static_cast<const Tin *>(p.k);
   const Tin *v = static_cast<const Tin *>(p.v), *e1 = static_cast<const Tin *>(p.e1);
@@ -268,8 +269,8 @@ __device__ bool load_chunk(const BwdParams &p, const ChunkSmem &L, float *sm, in
 
 // The chunk's C x C matrices A, B (strictly lower), M_z and, with `with_mk`, M_k
 // (lower, diagonal included).  Ends with a CTA barrier.
-template <bool kSplit>
-__device__ void chunk_matrices(const ChunkSmem &L, float *sm, int dk, bool exact, bool with_mk) {
+template <bool kSplit, int dk>
+__device__ void chunk_matrices(const ChunkSmem &L, float *sm, bool exact, bool with_mk) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, LDK = L.LDK;
   const float *lam = sm + L.lam, *Q = sm + L.Q, *K = sm + L.K, *U = sm + L.U, *Z = sm + L.Z;
   if (!exact) {
@@ -356,15 +357,16 @@ struct Decayed {
 // bwd_prep: per chunk W = T^-1 U~, Z~, K~ - N^T Z~ (N = T^-1 B), X = Q~ - M_z W, pi.
 // Record layout [W | Z~ | K~ - N^T Z~ | X] (32 x dk each, row-major) then pi [dk].
 // ---------------------------------------------------------------------------
-template <typename Tin, bool kSplit>
+template <typename Tin, bool kSplit, int kDK, int kDV>
 __global__ void __launch_bounds__(kThreads, kSplit ? 1 : 2) bwd_prep_kernel(BwdParams p) {
   extern __shared__ float sm[];
-  const ChunkSmem L(p.dk, p.dv, false);
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, dk = p.dk, LDK = L.LDK;
+  constexpr int dk = kDK;
+  const ChunkSmem L(kDK, kDV, false);
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, LDK = L.LDK;
   const int t0 = c * kC, n = min(kC, p.T - t0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool exact = load_chunk<Tin>(p, L, sm, b, h, t0, n, false);
-  chunk_matrices<kSplit>(L, sm, dk, exact, false);
+  const bool exact = load_chunk<Tin, kDK, kDV>(p, L, sm, b, h, t0, n, false);
+  chunk_matrices<kSplit, kDK>(L, sm, exact, false);
   invert_unit_lower32(sm + L.A, sm + L.Ti);
 
   const size_t cid = ((size_t)b * p.H + h) * p.nc + c;
@@ -598,12 +600,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) bwd_chain_kernel(BwdParams p
 // bwd_grads: one CTA per (chunk, h, b).  Every token gradient of the chunk and the
 // chunk's log-decay gradients.  S and dS_end are staged into shared memory in slabs.
 // ---------------------------------------------------------------------------
-template <typename Tin, bool kSplit>
+template <typename Tin, bool kSplit, int kDK, int kDV>
 __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
   extern __shared__ float sm[];
-  const ChunkSmem L(p.dk, p.dv, true);
+  constexpr int dk = kDK, dv = kDV;
+  const ChunkSmem L(kDK, kDV, true);
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int dk = p.dk, dv = p.dv, T = p.T, H = p.H, LDK = L.LDK, LDV = L.LDV;
+  const int T = p.T, H = p.H, LDK = L.LDK, LDV = L.LDV;
   const int t0 = c * kC, n = min(kC, T - t0);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const size_t bh = (size_t)b * H + h, cid = bh * p.nc + c;
@@ -611,8 +614,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
   const float *Send = S + (size_t)dk * dv;                             // chunk-end state
   const float *G = p.adj + cid * dk * dv;                              // its adjoint
 
-  const bool exact = load_chunk<Tin>(p, L, sm, b, h, t0, n, true);
-  chunk_matrices<kSplit>(L, sm, dk, exact, true);
+  const bool exact = load_chunk<Tin, kDK, kDV>(p, L, sm, b, h, t0, n, true);
+  chunk_matrices<kSplit, kDK>(L, sm, exact, true);
   invert_unit_lower32(sm + L.A, sm + L.Ti);
 
   const float *lam = sm + L.lam, *pi = sm + L.pi;
@@ -935,23 +938,31 @@ cudaError_t launch_chain(const BwdParams &p, cudaStream_t stream) {
   return cudaSuccess;
 }
 
-template <typename Tin, bool kSplit>
-cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
-  const ChunkSmem Lp(p.dk, p.dv, false), Lg(p.dk, p.dv, true);
+template <typename Tin, bool kSplit, int kDK, int kDV>
+cudaError_t launch_sized(const BwdParams &p, cudaStream_t stream) {
+  const ChunkSmem Lp(kDK, kDV, false), Lg(kDK, kDV, true);
   const size_t sp = Lp.total * 4, sg = Lg.total * 4;
   cudaError_t e;
-  if ((e = cudaFuncSetAttribute(bwd_prep_kernel<Tin, kSplit>,
+  if ((e = cudaFuncSetAttribute(bwd_prep_kernel<Tin, kSplit, kDK, kDV>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sp)) != cudaSuccess)
     return e;
-  if ((e = cudaFuncSetAttribute(bwd_grads_kernel<Tin, kSplit>,
+  if ((e = cudaFuncSetAttribute(bwd_grads_kernel<Tin, kSplit, kDK, kDV>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sg)) != cudaSuccess)
     return e;
   const dim3 chunks(p.nc, p.H, p.B);
-  bwd_prep_kernel<Tin, kSplit><<<chunks, kThreads, sp, stream>>>(p);
-  e = p.dk == 64 ? launch_chain<Tin, kSplit, 64>(p, stream) : launch_chain<Tin, kSplit, 128>(p, stream);
-  if (e != cudaSuccess) return e;
-  bwd_grads_kernel<Tin, kSplit><<<chunks, kThreads, sg, stream>>>(p);
+  bwd_prep_kernel<Tin, kSplit, kDK, kDV><<<chunks, kThreads, sp, stream>>>(p);
+  if ((e = launch_chain<Tin, kSplit, kDK>(p, stream)) != cudaSuccess) return e;
+  bwd_grads_kernel<Tin, kSplit, kDK, kDV><<<chunks, kThreads, sg, stream>>>(p);
   return cudaGetLastError();
+}
+
+template <typename Tin, bool kSplit>
+cudaError_t launch_typed(const BwdParams &p, cudaStream_t stream) {
+  if (p.dk == 64)
+    return p.dv == 64 ? launch_sized<Tin, kSplit, 64, 64>(p, stream)
+                      : launch_sized<Tin, kSplit, 64, 128>(p, stream);
+  return p.dv == 64 ? launch_sized<Tin, kSplit, 128, 64>(p, stream)
+                    : launch_sized<Tin, kSplit, 128, 128>(p, stream);
 }
 
 }  // namespace
