@@ -671,7 +671,8 @@ def main():
                     help="reverse-mode workload (default: both); for profiler captures")
     ap.add_argument("--bwd-batch", type=int, default=None,
                     help="reverse-mode batch B (default: the workload's); for profiler captures")
-    ap.add_argument("--only", default="all", choices=["all", "forward", "decode", "backward"],
+    ap.add_argument("--only", default="all",
+                    choices=["all", "forward", "decode", "backward", "muir", "mlstm"],
                     help="time one part only (profiling runs); the default line needs 'all'")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -699,8 +700,10 @@ def main():
               if args.only == "all" and not args.no_other_workloads else None)
     bwd = (bench_backward(ctx, args, gdr)
            if (args.only == "all" and not args.no_backward) or args.only == "backward" else None)
-    muir = bench_muir(ctx, args, gdr) if args.only == "all" and not args.no_muir else None
-    mlstm = bench_mlstm(ctx, args, gdr) if args.only == "all" and not args.no_mlstm else None
+    muir = (bench_muir(ctx, args, gdr)
+            if (args.only == "all" and not args.no_muir) or args.only == "muir" else None)
+    mlstm = (bench_mlstm(ctx, args, gdr)
+             if (args.only == "all" and not args.no_mlstm) or args.only == "mlstm" else None)
     ctx.barrier()
     if world > 1:
         dist.destroy_process_group()
