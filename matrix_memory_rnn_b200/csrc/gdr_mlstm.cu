@@ -35,15 +35,17 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kLDL = kL + 4;
 constexpr int kLDN = kNV + 4;
 
+// Shared memory: fp32 arrays (offsets in floats), then the q, k, v tiles at the input's
+// element type (offsets in bytes from `tiles`): bf16 inputs keep their exact values in
+// half the space, and are widened as they are read.
 struct MlstmSmem {
-  int LDK;
-  size_t Q, K, V, P, C, n, A, lf, ib, m, g, den, total;
-  __host__ __device__ explicit MlstmSmem(int dk) {
-    LDK = dk + 4;
+  int LDK, LDV;  // row strides of the q / k and v tiles, in elements (16-byte rows)
+  size_t P, C, n, A, lf, ib, m, g, den, mcar, tiles, Q, K, V, bytes;
+  __host__ __device__ MlstmSmem(int dk, int esize) {
+    const int pad = 16 / esize;
+    LDK = dk + pad;
+    LDV = kNV + pad;
     size_t off = 0;
-    Q = off; off += (size_t)kL * LDK;
-    K = off; off += (size_t)kL * LDK;
-    V = off; off += (size_t)kL * kLDN;
     P = off; off += (size_t)kL * kLDL;
     C = off; off += (size_t)dk * kLDN;
     n = off; off += dk;
@@ -53,9 +55,16 @@ struct MlstmSmem {
     m = off; off += kL;
     g = off; off += kL;
     den = off; off += kL;
-    total = off + 4;
+    mcar = off; off += 4;
+    tiles = off * 4;
+    Q = 0;
+    K = Q + (size_t)kL * LDK * esize;
+    V = K + (size_t)kL * LDK * esize;
+    bytes = tiles + V + (size_t)kL * LDV * esize;
   }
 };
+__device__ __forceinline__ float widen1(float x) { return x; }
+__device__ __forceinline__ float widen1(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // 16-byte pieces of the chunk's q, k (64 x dk) and v slice (64 x 64) held in registers:
 // the next chunk is loaded while the current one is computed.  kE = elements per piece.
@@ -67,33 +76,25 @@ struct ChunkRegs {
   uint4 q[kQK], k[kQK], v[kV];
   float lf, ib;
 };
-__device__ __forceinline__ void widen(const uint4 &u, float *dst, const __nv_bfloat16 *) {
-  const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 x = __bfloat1622float2(h[i]);
-    dst[2 * i] = x.x;
-    dst[2 * i + 1] = x.y;
-  }
-}
-__device__ __forceinline__ void widen(const uint4 &u, float *dst, const float *) {
-  *reinterpret_cast<float4 *>(dst) = *reinterpret_cast<const float4 *>(&u);
-}
-
-// d_k = 64 keeps two CTAs per SM (registers and shared memory), d_k = 128 one.
 template <typename Tin, bool kSplit, int kDK>
-__global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_mlstm_args a) {
+__global__ void __launch_bounds__(kThreads, kSplit ? 1 : 2) mlstm_kernel(gdr_mlstm_args a) {
   extern __shared__ float sm[];
   constexpr int dk = kDK;
   const int dv = a.dv, T = a.T, H = a.H;
-  const MlstmSmem L(dk);
-  const int LDK = L.LDK;
+  const MlstmSmem L(dk, sizeof(Tin));
+  const int LDK = L.LDK, LDV = L.LDV;
   const int c0 = blockIdx.x * kNV, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float *Q = sm + L.Q, *K = sm + L.K, *V = sm + L.V, *P = sm + L.P, *C = sm + L.C, *nn = sm + L.n;
+  float *P = sm + L.P, *C = sm + L.C, *nn = sm + L.n;
   float *A = sm + L.A, *lf = sm + L.lf, *ib = sm + L.ib, *mt = sm + L.m, *gt = sm + L.g;
   float *den = sm + L.den;
-  float *mcar = sm + L.total - 4;   // the carried running max
+  float *mcar = sm + L.mcar;   // the carried running max
+  uint8_t *tiles = reinterpret_cast<uint8_t *>(sm) + L.tiles;
+  Tin *Qs = reinterpret_cast<Tin *>(tiles + L.Q), *Ks = reinterpret_cast<Tin *>(tiles + L.K);
+  Tin *Vs = reinterpret_cast<Tin *>(tiles + L.V);
+  auto Q = [&](int r, int c) { return widen1(Qs[r * LDK + c]); };
+  auto K = [&](int r, int c) { return widen1(Ks[r * LDK + c]); };
+  auto V = [&](int r, int c) { return widen1(Vs[r * LDV + c]); };
   const Tin *q = static_cast<const Tin *>(a.q), *k = static_cast<const Tin *>(a.k);
   const Tin *v = static_cast<const Tin *>(a.v);
   const size_t bh = (size_t)b * H + h;
@@ -139,13 +140,13 @@ __global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_
     for (int u = 0; u < R::kQK; ++u) {
       if (u >= nq) break;
       const int i = tid + u * kThreads, t = i / gq, j = (i % gq) * R::kE;
-      widen(rg.q[u], Q + t * LDK + j, q);
-      widen(rg.k[u], K + t * LDK + j, k);
+      *reinterpret_cast<uint4 *>(Qs + t * LDK + j) = rg.q[u];
+      *reinterpret_cast<uint4 *>(Ks + t * LDK + j) = rg.k[u];
     }
 #pragma unroll
     for (int u = 0; u < R::kV; ++u) {
       const int i = tid + u * kThreads, t = i / (kNV / R::kE), c = (i % (kNV / R::kE)) * R::kE;
-      widen(rg.v[u], V + t * kLDN + c, v);
+      *reinterpret_cast<uint4 *>(Vs + t * LDV + c) = rg.v[u];
     }
     if (tid < kL) {
       const float x = rg.lf;   // log sigmoid; padding keeps log f = 0
@@ -198,8 +199,8 @@ __global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_
       const int r0 = 16 * (warp >> 1), cc0 = 32 * (warp & 1);
       float acc[4][4];
       zero_acc(acc);
-      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return Q[m * LDK + kk]; },
-                      [&](int kk, int nn2) { return K[nn2 * LDK + kk]; }, lane);
+      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return Q(m, kk); },
+                      [&](int kk, int nn2) { return K(nn2, kk); }, lane);
       for_acc(acc, r0, cc0, lane, [&](int t, int s, float x) {
         P[t * kLDL + s] = s <= t ? x * expf(A[t] - A[s] + ib[s] - mt[t]) : 0.f;
       });
@@ -210,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_
       const int t = tid >> 2, part = tid & 3;
       float s = 0.f;
       for (int u = part; u < kL; u += 4) s += P[t * kLDL + u];
-      for (int j = part; j < dk; j += 4) s += gt[t] * nn[j] * Q[t * LDK + j];
+      for (int j = part; j < dk; j += 4) s += gt[t] * nn[j] * Q(t, j);
       s += __shfl_xor_sync(0xffffffffu, s, 1);
       s += __shfl_xor_sync(0xffffffffu, s, 2);
       if (part == 0) den[t] = s;
@@ -222,8 +223,8 @@ __global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_
       float acc[4][4];
       zero_acc(acc);
       mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int kk) { return P[m * kLDL + kk]; },
-                      [&](int kk, int nn2) { return V[kk * kLDN + nn2]; }, lane);
-      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return gt[m] * Q[m * LDK + kk]; },
+                      [&](int kk, int nn2) { return V(kk, nn2); }, lane);
+      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return gt[m] * Q(m, kk); },
                       [&](int kk, int nn2) { return C[kk * kLDN + nn2]; }, lane);
       for_acc(acc, r0, cc0, lane, [&](int t, int c, float x) {
         if (t < n)
@@ -243,15 +244,15 @@ __global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_
         const int r0 = 16 * (wt >> 1), cc0 = 32 * (wt & 1);
         float acc[4][4];
         zero_acc(acc);
-        mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int s) { return K[s * LDK + m] * wL(s); },
-                        [&](int s, int nn2) { return V[s * kLDN + nn2]; }, lane);
+        mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int s) { return K(s, m) * wL(s); },
+                        [&](int s, int nn2) { return V(s, nn2); }, lane);
         for_acc(acc, r0, cc0, lane, [&](int j, int c, float x) {
           C[j * kLDN + c] = gL * C[j * kLDN + c] + x;
         });
       }
       for (int j = tid; j < dk; j += kThreads) {
         float s = 0.f;
-        for (int u = 0; u < kL; ++u) s += wL(u) * K[u * LDK + j];
+        for (int u = 0; u < kL; ++u) s += wL(u) * K(u, j);
         nn[j] = gL * nn[j] + s;
       }
       __syncthreads();
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, kDK == 64 ? 2 : 1) mlstm_kernel(gdr_
 
 template <typename Tin, bool kSplit, int kDK>
 cudaError_t launch_typed(const gdr_mlstm_args &a, cudaStream_t stream) {
-  const size_t smem = MlstmSmem(kDK).total * sizeof(float);
+  const size_t smem = MlstmSmem(kDK, sizeof(Tin)).bytes;
   cudaError_t e = cudaFuncSetAttribute(mlstm_kernel<Tin, kSplit, kDK>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
