@@ -267,6 +267,34 @@ def test_tc_split_gla_strong_decay_and_small_workspace():
     assert head_rel_err(S, S_ref, (0, 1)) < TOL["bf16"]
 
 
+@pytest.mark.parametrize("d,algo,ws", [(128, "auto", None), (128, "tc", 256), (64, "tc", None),
+                                       (64, "fp32", None)])
+def test_deltanet_through_gdn2_form(d, algo, ws):
+    """Plain DeltaNet (no decay, u = beta k, z = k, write beta v k^T) is the GDN-2 form with
+    log w = 0 and the erase and write gates both set to the per-token strength beta.  The
+    oracle runs it in the general form with that mapping written out in fp64."""
+    B, T, H = 2, 200, 2
+    rng = np.random.default_rng(21)
+    q = synth.round_bf16(rng.standard_normal((B, T, H, d)))
+    kk = rng.standard_normal((B, T, H, d))
+    k = synth.round_bf16(kk / np.linalg.norm(kk, axis=-1, keepdims=True))
+    v = synth.round_bf16(rng.standard_normal((B, T, H, d)))
+    beta = synth.round_bf16(1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, H, 1)))))
+    gate = np.broadcast_to(beta, (B, T, H, d)).copy()
+    log_w = np.zeros((B, T, H, d), np.float32)
+    dev = gdr.to_device(dict(q=q, k=k, v=v, log_w=log_w, e1=gate, e2=gate), "bf16")
+    o, S_T = gdr.gdr_forward_chunked("gdn2", dev["q"], dev["k"], dev["v"], dev["log_w"],
+                                     dev["e1"], dev["e2"], None, chunk=64, algo=algo,
+                                     workspace=None if ws is None else gdr.new_workspace(ws, "cuda"))
+    torch.cuda.synchronize()
+    b64, k64 = beta.astype(np.float64), k.astype(np.float64)
+    o_ref, S_ref = oracle.forward("general", q, k, b64 * v, log_w, b64 * k64, k, None)
+    eo = head_rel_err(o.cpu().numpy(), o_ref, (0, 2))
+    es = head_rel_err(S_T.cpu().numpy(), S_ref, (0, 1))
+    print(f"deltanet d={d} {algo}: o {eo:.3e} S {es:.3e}")
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
 def test_tc_rejects_what_it_does_not_cover():
     w = small("rwkv7", "bf16", dk=32, dv=32, T=64, B=1, H=1, chunk=64)
     inp = synth.forward_inputs(w)
