@@ -217,14 +217,17 @@ __device__ __forceinline__ bool group_wait(uint64_t *bar, uint32_t parity, volat
 // The Muir mixer's activations on the tiles as loaded ("Muir ...", section 2.1 and
 // section 4.1): SiLU, the head's l2 norm (the 16 lanes holding one token's 128
 // channels reduce with shuffles), the readout gain and the gates.  Seven of these per
-// element ride on a kernel that is issue- and latency-bound, so they use the hardware
-// exponential, logarithm and approximate division (a few ulp; the operands are rounded
-// to bf16 next).  The argument of the exponential is clamped at 80 so that 1 + e^-x
-// stays finite and inside the approximate division's range; softplus switches to its
-// asymptotes where 1 + e^x would round.
-__device__ __forceinline__ float sigmoid_f(float x) {
-  return __fdividef(1.f, 1.f + __expf(-fmaxf(x, -80.f)));
+// element ride on a kernel that is issue- and latency-bound, so they use the hardware's
+// special-function unit directly: sigma(x) = (1 + tanh(x / 2)) / 2 with its tanh (one
+// operation where an exponential and a reciprocal take two; absolute error about 2.5e-4,
+// and every result is rounded to bf16 next), and its exponential and logarithm for
+// softplus, which switches to its asymptotes where 1 + e^x would round.
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
+__device__ __forceinline__ float sigmoid_f(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 __device__ __forceinline__ float silu_f(float x) { return x * sigmoid_f(x); }
 __device__ __forceinline__ float softplus_f(float x) {
   return x > 15.f ? x : (x < -15.f ? __expf(x) : __logf(1.f + __expf(x)));

@@ -13,10 +13,13 @@
 //   h_t = num_t / max(|den_t|, e^{-m_t}),
 //   C <- g_L C + sum_s w_Ls v_s k_s^T,   n <- g_L n + sum_s w_Ls k_s,   m <- m_L.
 // One CTA per (b, h, 64 value columns) walks the chunks of its sequence with the state
-// slice in shared memory; Q K^T, P V + diag(g) Q C, and the state update K^T diag(w_L) V
-// are warp-level tf32 MMAs (three products for fp32 inputs).  Tokens past T are padding
-// with log f = 0 and i~ = -inf (no write, no decay).
+// slice in shared memory.  Q K^T takes bf16 MMAs for bf16 inputs (exact products) and
+// tf32 otherwise; P V, Q C and the state update K^T diag(w_L) V are tf32 (three products
+// for fp32 inputs).  Tokens past T are padding with log f = 0 and i~ = -inf (no write, no
+// decay).
 #include <math.h>
+
+#include <type_traits>
 
 #include "gdr_internal.cuh"
 #include "gdr_warp_mma.cuh"
@@ -25,7 +28,9 @@ namespace gdr {
 namespace {
 
 using wmma_tf32::for_acc;
+using wmma_tf32::mma_bf16_abt;
 using wmma_tf32::mma_seg;
+using wmma_tf32::tf32_exact;
 using wmma_tf32::zero_acc;
 
 constexpr int kL = 64;          // chunk
@@ -63,8 +68,160 @@ struct MlstmSmem {
     bytes = tiles + V + (size_t)kL * LDV * esize;
   }
 };
-__device__ __forceinline__ float widen1(float x) { return x; }
-__device__ __forceinline__ float widen1(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Views of one CTA's shared memory.
+template <typename Tin>
+struct Views {
+  float *P, *C, *nn, *A, *lf, *ib, *mt, *gt, *den, *mcar;
+  Tin *Qs, *Ks, *Vs;
+  int LDK, LDV;
+  __device__ Views(float *sm, const MlstmSmem &L) {
+    P = sm + L.P; C = sm + L.C; nn = sm + L.n; A = sm + L.A; lf = sm + L.lf; ib = sm + L.ib;
+    mt = sm + L.m; gt = sm + L.g; den = sm + L.den; mcar = sm + L.mcar;
+    uint8_t *tiles = reinterpret_cast<uint8_t *>(sm) + L.tiles;
+    Qs = reinterpret_cast<Tin *>(tiles + L.Q);
+    Ks = reinterpret_cast<Tin *>(tiles + L.K);
+    Vs = reinterpret_cast<Tin *>(tiles + L.V);
+    LDK = L.LDK;
+    LDV = L.LDV;
+  }
+  __device__ float Q(int r, int c) const { return widen(Qs[r * LDK + c]); }
+  __device__ float K(int r, int c) const { return widen(Ks[r * LDK + c]); }
+  // the tiles as MMA operands (a bf16 value is exact in tf32)
+  __device__ auto Qx(int r, int c) const { return tf32_exact(Qs[r * LDK + c]); }
+  __device__ auto Kx(int r, int c) const { return tf32_exact(Ks[r * LDK + c]); }
+  __device__ auto Vx(int r, int c) const { return tf32_exact(Vs[r * LDV + c]); }
+  static __device__ float widen(float x) { return x; }
+  static __device__ float widen(__nv_bfloat16 x) { return __bfloat162float(x); }
+};
+
+__device__ __forceinline__ float log_sigmoid(float x) {
+  return x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));
+}
+
+// Warp 0: A (inclusive prefix of log f), the prefix max of i~ - A, m_t and g_t, from the
+// carried running max mc.
+__device__ __forceinline__ void scan_chunk(const float *lf, const float *ib, float mc, float *A,
+                                           float *mt, float *gt, int lane) {
+  float a0 = lf[lane], a1 = lf[lane + 32];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float x0 = __shfl_up_sync(0xffffffffu, a0, o), x1 = __shfl_up_sync(0xffffffffu, a1, o);
+    if (lane >= o) {
+      a0 += x0;
+      a1 += x1;
+    }
+  }
+  a1 += __shfl_sync(0xffffffffu, a0, 31);
+  float p0 = ib[lane] - a0, p1 = ib[lane + 32] - a1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const float x0 = __shfl_up_sync(0xffffffffu, p0, o), x1 = __shfl_up_sync(0xffffffffu, p1, o);
+    if (lane >= o) {
+      p0 = fmaxf(p0, x0);
+      p1 = fmaxf(p1, x1);
+    }
+  }
+  p1 = fmaxf(p1, __shfl_sync(0xffffffffu, p0, 31));
+  const float m0 = a0 + fmaxf(mc, p0), m1 = a1 + fmaxf(mc, p1);
+  A[lane] = a0;
+  A[lane + 32] = a1;
+  mt[lane] = m0;
+  mt[lane + 32] = m1;
+  gt[lane] = expf(a0 + mc - m0);      // 0 for an empty memory (mc = -inf)
+  gt[lane + 32] = expf(a1 + mc - m1);
+}
+
+// The chunk's readout h for value columns [c0, c0 + 64) from the scanned gates and the
+// state in shared memory; every thread calls it after a barrier that follows the scan.
+// Rows t >= n are not stored.
+template <typename Tin, bool kSplit, int kDK>
+__device__ __forceinline__ void readout(const Views<Tin> &s, float *hout, size_t hstride, int n) {
+  constexpr int dk = kDK;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r0 = 16 * (warp >> 1), cc0 = 32 * (warp & 1), g = lane >> 2, tq = lane & 3;
+  // ---- P = (Q K^T) (.) w, w_ts = e^{A_t - A_s + i~_s - m_t} (s <= t)
+  {
+    float acc[4][4];
+    zero_acc(acc);
+    if constexpr (std::is_same<Tin, __nv_bfloat16>::value)
+      mma_bf16_abt(acc, s.Qs, s.LDK, s.Ks, s.LDK, r0, cc0, 0, dk, lane);
+    else
+      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return s.Qx(m, kk); },
+                      [&](int kk, int nn2) { return s.Kx(nn2, kk); }, lane);
+    for_acc(acc, r0, cc0, lane, [&](int t, int j, float x) {
+      s.P[t * kLDL + j] = j <= t ? x * __expf(s.A[t] - s.A[j] + s.ib[j] - s.mt[t]) : 0.f;
+    });
+  }
+  __syncthreads();
+  // ---- 1 / max(|den_t|, e^{-m_t}), den_t = sum_s P_ts + g_t n . q_t (4 threads per row)
+  {
+    const int t = tid >> 2, part = tid & 3;
+    float sp = 0.f, sq = 0.f;
+    for (int u = part; u < kL; u += 4) sp += s.P[t * kLDL + u];
+    for (int j = part; j < dk; j += 4) sq += s.nn[j] * s.Q(t, j);
+    float acc = sp + s.gt[t] * sq;
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (part == 0) s.den[t] = 1.f / fmaxf(fabsf(acc), expf(-s.mt[t]));
+  }
+  __syncthreads();
+  // ---- h = (P V + diag(g) Q C) / max(|den|, e^{-m}); P V and Q C in two accumulators
+  {
+    float pv[4][4], qc[4][4];
+    zero_acc(pv);
+    zero_acc(qc);
+    mma_seg<kSplit>(pv, r0, cc0, 0, kL, [&](int m, int kk) { return s.P[m * kLDL + kk]; },
+                    [&](int kk, int nn2) { return s.Vx(kk, nn2); }, lane);
+    mma_seg<kSplit>(qc, r0, cc0, 0, dk, [&](int m, int kk) { return s.Qx(m, kk); },
+                    [&](int kk, int nn2) { return s.C[kk * kLDN + nn2]; }, lane);
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {   // rows r0 + g and r0 + g + 8
+      const int t = r0 + g + 8 * hf;
+      if (t >= n) continue;
+      const float gg = s.gt[t], rd = s.den[t];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float x0 = fmaf(gg, qc[i][2 * hf], pv[i][2 * hf]) * rd;
+        const float x1 = fmaf(gg, qc[i][2 * hf + 1], pv[i][2 * hf + 1]) * rd;
+        *reinterpret_cast<float2 *>(hout + t * hstride + cc0 + 8 * i + 2 * tq) = make_float2(x0, x1);
+      }
+    }
+  }
+}
+
+// C <- g_L C + K^T diag(w_L) V, n <- g_L n + K^T w_L, m <- m_L; every thread calls it after
+// a barrier that follows every read of C, n and den.
+template <typename Tin, bool kSplit, int kDK>
+__device__ __forceinline__ void update_state(const Views<Tin> &s) {
+  constexpr int dk = kDK;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float mL = s.mt[kL - 1], gL = s.gt[kL - 1];
+  float *wl = s.den;   // den is read: w_Ls = e^{A_L - A_s + i~_s - m_L} in its place
+  if (tid < kL) wl[tid] = expf(s.A[kL - 1] - s.A[tid] + s.ib[tid] - mL);
+  __syncthreads();
+  for (int wt = warp; wt < dk / 8; wt += kWarps) {
+    const int r0 = 16 * (wt >> 1), cc0 = 32 * (wt & 1);
+    float acc[4][4];
+    zero_acc(acc);
+    mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int j) { return s.K(j, m) * wl[j]; },
+                    [&](int j, int nn2) { return s.Vx(j, nn2); }, lane);
+    for_acc(acc, r0, cc0, lane, [&](int j, int c, float x) {
+      s.C[j * kLDN + c] = gL * s.C[j * kLDN + c] + x;
+    });
+  }
+  {   // kThreads / dk adjacent lanes per key channel
+    constexpr int kP = kThreads / kDK;
+    const int j = tid / kP, part = tid % kP;
+    float acc = 0.f;
+    for (int u = part; u < kL; u += kP) acc += wl[u] * s.K(u, j);
+#pragma unroll
+    for (int o = 1; o < kP; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (part == 0) s.nn[j] = gL * s.nn[j] + acc;
+  }
+  __syncthreads();
+  if (tid == 0) *s.mcar = mL;
+}
 
 // 16-byte pieces of the chunk's q, k (64 x dk) and v slice (64 x 64) held in registers:
 // the next chunk is loaded while the current one is computed.  kE = elements per piece.
@@ -75,201 +232,109 @@ struct ChunkRegs {
   static constexpr int kV = kL * kNV / kE / kThreads;
   uint4 q[kQK], k[kQK], v[kV];
   float lf, ib;
-};
-template <typename Tin, bool kSplit, int kDK>
-__global__ void __launch_bounds__(kThreads, kSplit ? 1 : 2) mlstm_kernel(gdr_mlstm_args a) {
-  extern __shared__ float sm[];
-  constexpr int dk = kDK;
-  const int dv = a.dv, T = a.T, H = a.H;
-  const MlstmSmem L(dk, sizeof(Tin));
-  const int LDK = L.LDK, LDV = L.LDV;
-  const int c0 = blockIdx.x * kNV, h = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  float *P = sm + L.P, *C = sm + L.C, *nn = sm + L.n;
-  float *A = sm + L.A, *lf = sm + L.lf, *ib = sm + L.ib, *mt = sm + L.m, *gt = sm + L.g;
-  float *den = sm + L.den;
-  float *mcar = sm + L.mcar;   // the carried running max
-  uint8_t *tiles = reinterpret_cast<uint8_t *>(sm) + L.tiles;
-  Tin *Qs = reinterpret_cast<Tin *>(tiles + L.Q), *Ks = reinterpret_cast<Tin *>(tiles + L.K);
-  Tin *Vs = reinterpret_cast<Tin *>(tiles + L.V);
-  auto Q = [&](int r, int c) { return widen1(Qs[r * LDK + c]); };
-  auto K = [&](int r, int c) { return widen1(Ks[r * LDK + c]); };
-  auto V = [&](int r, int c) { return widen1(Vs[r * LDV + c]); };
-  const Tin *q = static_cast<const Tin *>(a.q), *k = static_cast<const Tin *>(a.k);
-  const Tin *v = static_cast<const Tin *>(a.v);
-  const size_t bh = (size_t)b * H + h;
 
-  for (int i = tid; i < dk * kNV; i += kThreads) {
-    const int j = i / kNV, c = i % kNV;
-    C[j * kLDN + c] = a.C0 ? a.C0[bh * dk * dv + (size_t)j * dv + c0 + c] : 0.f;
-  }
-  for (int j = tid; j < dk; j += kThreads) nn[j] = a.n0 ? a.n0[bh * dk + j] : 0.f;
-  if (tid == 0) *mcar = a.m0 ? a.m0[bh] : -INFINITY;
-
-  // ---- chunk loads (padding: q = k = v = 0, log f = 0, i~ = -inf), one chunk ahead
-  using R = ChunkRegs<Tin, kDK>;
-  R rg;
-  const int gq = dk / R::kE;                 // pieces per row of q / k
-  const int nq = kL * gq / kThreads;         // pieces per thread (d_k = 64: half of kQK)
-  auto fetch = [&](int t0) {
+  __device__ void fetch(const gdr_mlstm_args &a, int b, int h, int c0, int t0) {
+    const Tin *q_ = static_cast<const Tin *>(a.q), *k_ = static_cast<const Tin *>(a.k);
+    const Tin *v_ = static_cast<const Tin *>(a.v);
+    const int tid = threadIdx.x, T = a.T, H = a.H, gq = kDK / kE;
 #pragma unroll
-    for (int u = 0; u < R::kQK; ++u) {
-      if (u >= nq) break;
-      const int i = tid + u * kThreads, t = i / gq, j = (i % gq) * R::kE;
-      const size_t ik = (((size_t)b * T + t0 + t) * H + h) * dk + j;
+    for (int u = 0; u < kQK; ++u) {
+      const int i = tid + u * kThreads, t = i / gq, j = (i % gq) * kE;
+      const size_t ik = (((size_t)b * T + t0 + t) * H + h) * kDK + j;
       const bool in = t0 + t < T;
-      rg.q[u] = in ? __ldg(reinterpret_cast<const uint4 *>(q + ik)) : make_uint4(0u, 0u, 0u, 0u);
-      rg.k[u] = in ? __ldg(reinterpret_cast<const uint4 *>(k + ik)) : make_uint4(0u, 0u, 0u, 0u);
+      q[u] = in ? __ldg(reinterpret_cast<const uint4 *>(q_ + ik)) : make_uint4(0u, 0u, 0u, 0u);
+      k[u] = in ? __ldg(reinterpret_cast<const uint4 *>(k_ + ik)) : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
-    for (int u = 0; u < R::kV; ++u) {
-      const int i = tid + u * kThreads, t = i / (kNV / R::kE), c = (i % (kNV / R::kE)) * R::kE;
+    for (int u = 0; u < kV; ++u) {
+      const int i = tid + u * kThreads, t = i / (kNV / kE), c = (i % (kNV / kE)) * kE;
       const bool in = t0 + t < T;
-      rg.v[u] = in ? __ldg(reinterpret_cast<const uint4 *>(v + (((size_t)b * T + t0 + t) * H + h) * dv + c0 + c))
-                   : make_uint4(0u, 0u, 0u, 0u);
+      v[u] = in ? __ldg(reinterpret_cast<const uint4 *>(v_ + (((size_t)b * T + t0 + t) * H + h) * a.dv + c0 + c))
+                : make_uint4(0u, 0u, 0u, 0u);
     }
     if (tid < kL) {
       const bool in = t0 + tid < T;
       const size_t ts = ((size_t)b * T + t0 + tid) * H + h;
-      rg.lf = in ? __ldg(a.f_pre + ts) : 0.f;
-      rg.ib = in ? __ldg(a.i_pre + ts) : -INFINITY;
-    }
-  };
-  auto commit = [&](int n) {
-#pragma unroll
-    for (int u = 0; u < R::kQK; ++u) {
-      if (u >= nq) break;
-      const int i = tid + u * kThreads, t = i / gq, j = (i % gq) * R::kE;
-      *reinterpret_cast<uint4 *>(Qs + t * LDK + j) = rg.q[u];
-      *reinterpret_cast<uint4 *>(Ks + t * LDK + j) = rg.k[u];
-    }
-#pragma unroll
-    for (int u = 0; u < R::kV; ++u) {
-      const int i = tid + u * kThreads, t = i / (kNV / R::kE), c = (i % (kNV / R::kE)) * R::kE;
-      *reinterpret_cast<uint4 *>(Vs + t * LDV + c) = rg.v[u];
-    }
-    if (tid < kL) {
-      const float x = rg.lf;   // log sigmoid; padding keeps log f = 0
-      lf[tid] = tid < n ? (x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x))) : 0.f;
-      ib[tid] = rg.ib;
-    }
-  };
-  fetch(0);
-
-  for (int t0 = 0; t0 < T; t0 += kL) {
-    const int n = min(kL, T - t0);
-    __syncthreads();   // the previous chunk is done with every buffer
-    commit(n);
-    if (t0 + kL < T) fetch(t0 + kL);
-    __syncthreads();
-    // ---- A (inclusive prefix of log f), the prefix max of i~ - A, m_t and g_t (warp 0)
-    if (warp == 0) {
-      float a0 = lf[lane], a1 = lf[lane + 32];
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float x0 = __shfl_up_sync(0xffffffffu, a0, o), x1 = __shfl_up_sync(0xffffffffu, a1, o);
-        if (lane >= o) {
-          a0 += x0;
-          a1 += x1;
-        }
-      }
-      a1 += __shfl_sync(0xffffffffu, a0, 31);
-      float p0 = ib[lane] - a0, p1 = ib[lane + 32] - a1;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float x0 = __shfl_up_sync(0xffffffffu, p0, o), x1 = __shfl_up_sync(0xffffffffu, p1, o);
-        if (lane >= o) {
-          p0 = fmaxf(p0, x0);
-          p1 = fmaxf(p1, x1);
-        }
-      }
-      p1 = fmaxf(p1, __shfl_sync(0xffffffffu, p0, 31));
-      const float mc = *mcar;
-      const float m0 = a0 + fmaxf(mc, p0), m1 = a1 + fmaxf(mc, p1);
-      A[lane] = a0;
-      A[lane + 32] = a1;
-      mt[lane] = m0;
-      mt[lane + 32] = m1;
-      gt[lane] = expf(a0 + mc - m0);      // 0 for an empty memory (mc = -inf)
-      gt[lane + 32] = expf(a1 + mc - m1);
-    }
-    __syncthreads();
-    // ---- P = (Q K^T) (.) w, w_ts = e^{A_t - A_s + i~_s - m_t} (s <= t)
-    {
-      const int r0 = 16 * (warp >> 1), cc0 = 32 * (warp & 1);
-      float acc[4][4];
-      zero_acc(acc);
-      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return Q(m, kk); },
-                      [&](int kk, int nn2) { return K(nn2, kk); }, lane);
-      for_acc(acc, r0, cc0, lane, [&](int t, int s, float x) {
-        P[t * kLDL + s] = s <= t ? x * expf(A[t] - A[s] + ib[s] - mt[t]) : 0.f;
-      });
-    }
-    __syncthreads();
-    // ---- den_t = sum_s P_ts + g_t n . q_t (4 threads per row)
-    {
-      const int t = tid >> 2, part = tid & 3;
-      float s = 0.f;
-      for (int u = part; u < kL; u += 4) s += P[t * kLDL + u];
-      for (int j = part; j < dk; j += 4) s += gt[t] * nn[j] * Q(t, j);
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      if (part == 0) den[t] = s;
-    }
-    __syncthreads();
-    // ---- h = (P V + diag(g) Q C) / max(|den|, e^{-m})
-    {
-      const int r0 = 16 * (warp >> 1), cc0 = 32 * (warp & 1);
-      float acc[4][4];
-      zero_acc(acc);
-      mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int kk) { return P[m * kLDL + kk]; },
-                      [&](int kk, int nn2) { return V(kk, nn2); }, lane);
-      mma_seg<kSplit>(acc, r0, cc0, 0, dk, [&](int m, int kk) { return gt[m] * Q(m, kk); },
-                      [&](int kk, int nn2) { return C[kk * kLDN + nn2]; }, lane);
-      for_acc(acc, r0, cc0, lane, [&](int t, int c, float x) {
-        if (t < n)
-          a.h[(((size_t)b * T + t0 + t) * H + h) * dv + c0 + c] =
-              x / fmaxf(fabsf(den[t]), expf(-mt[t]));
-      });
-    }
-    __syncthreads();   // C and n are read above; they change below
-    // ---- state: C <- g_L C + K^T diag(w_L) V, n <- g_L n + K^T w_L, m <- m_L
-    {
-      const float mL = mt[kL - 1], gL = gt[kL - 1];
-      float *wl = den;   // den is read above: w_Ls = e^{A_L - A_s + i~_s - m_L} in its place
-      if (tid < kL) wl[tid] = expf(A[kL - 1] - A[tid] + ib[tid] - mL);
-      __syncthreads();
-      auto wL = [&](int s) { return wl[s]; };
-      for (int wt = warp; wt < dk / 8; wt += kWarps) {
-        const int r0 = 16 * (wt >> 1), cc0 = 32 * (wt & 1);
-        float acc[4][4];
-        zero_acc(acc);
-        mma_seg<kSplit>(acc, r0, cc0, 0, kL, [&](int m, int s) { return K(s, m) * wL(s); },
-                        [&](int s, int nn2) { return V(s, nn2); }, lane);
-        for_acc(acc, r0, cc0, lane, [&](int j, int c, float x) {
-          C[j * kLDN + c] = gL * C[j * kLDN + c] + x;
-        });
-      }
-      for (int j = tid; j < dk; j += kThreads) {
-        float s = 0.f;
-        for (int u = 0; u < kL; ++u) s += wL(u) * K(u, j);
-        nn[j] = gL * nn[j] + s;
-      }
-      __syncthreads();
-      if (tid == 0) *mcar = mL;
+      lf = in ? __ldg(a.f_pre + ts) : 0.f;
+      ib = in ? __ldg(a.i_pre + ts) : -INFINITY;
     }
   }
-  __syncthreads();
+  __device__ void commit(const Views<Tin> &s, int n) const {
+    const int tid = threadIdx.x, gq = kDK / kE;
+#pragma unroll
+    for (int u = 0; u < kQK; ++u) {
+      const int i = tid + u * kThreads, t = i / gq, j = (i % gq) * kE;
+      *reinterpret_cast<uint4 *>(s.Qs + t * s.LDK + j) = q[u];
+      *reinterpret_cast<uint4 *>(s.Ks + t * s.LDK + j) = k[u];
+    }
+#pragma unroll
+    for (int u = 0; u < kV; ++u) {
+      const int i = tid + u * kThreads, t = i / (kNV / kE), c = (i % (kNV / kE)) * kE;
+      *reinterpret_cast<uint4 *>(s.Vs + t * s.LDV + c) = v[u];
+    }
+    if (tid < kL) {
+      s.lf[tid] = tid < n ? log_sigmoid(lf) : 0.f;   // padding keeps log f = 0
+      s.ib[tid] = ib;
+    }
+  }
+};
+
+// The state a CTA starts from: C0's 64 columns (or zeros), n0, m0 (or an empty memory).
+template <typename Tin, int kDK>
+__device__ __forceinline__ void load_initial_state(const Views<Tin> &s, const gdr_mlstm_args &a,
+                                                   size_t bh, int c0) {
+  const int tid = threadIdx.x, dv = a.dv;
+  for (int i = tid; i < kDK * kNV; i += kThreads) {
+    const int j = i / kNV, c = i % kNV;
+    s.C[j * kLDN + c] = a.C0 ? a.C0[bh * kDK * dv + (size_t)j * dv + c0 + c] : 0.f;
+  }
+  for (int j = tid; j < kDK; j += kThreads) s.nn[j] = a.n0 ? a.n0[bh * kDK + j] : 0.f;
+  if (tid == 0) *s.mcar = a.m0 ? a.m0[bh] : -INFINITY;
+}
+
+// The final state (C_T's 64 columns; n_T, m_T from the first column block).
+template <typename Tin, int kDK>
+__device__ __forceinline__ void store_final_state(const Views<Tin> &s, const gdr_mlstm_args &a,
+                                                  size_t bh, int c0) {
+  const int tid = threadIdx.x, dv = a.dv;
   if (a.C_T)
-    for (int i = tid; i < dk * kNV; i += kThreads) {
+    for (int i = tid; i < kDK * kNV; i += kThreads) {
       const int j = i / kNV, c = i % kNV;
-      a.C_T[bh * dk * dv + (size_t)j * dv + c0 + c] = C[j * kLDN + c];
+      a.C_T[bh * kDK * dv + (size_t)j * dv + c0 + c] = s.C[j * kLDN + c];
     }
   if (blockIdx.x == 0) {
     if (a.n_T)
-      for (int j = tid; j < dk; j += kThreads) a.n_T[bh * dk + j] = nn[j];
-    if (a.m_T && tid == 0) a.m_T[bh] = *mcar;
+      for (int j = tid; j < kDK; j += kThreads) a.n_T[bh * kDK + j] = s.nn[j];
+    if (a.m_T && tid == 0) a.m_T[bh] = *s.mcar;
   }
+}
+
+// One CTA per (b, h, 64 value columns): readout and state update, chunk after chunk.
+template <typename Tin, bool kSplit, int kDK>
+__global__ void __launch_bounds__(kThreads, kSplit ? 1 : 2) mlstm_kernel(gdr_mlstm_args a) {
+  extern __shared__ float sm[];
+  const Views<Tin> s(sm, MlstmSmem(kDK, sizeof(Tin)));
+  const int c0 = blockIdx.x * kNV, h = blockIdx.y, b = blockIdx.z;
+  const int T = a.T, H = a.H, dv = a.dv, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const size_t bh = (size_t)b * H + h;
+  load_initial_state<Tin, kDK>(s, a, bh, c0);
+
+  ChunkRegs<Tin, kDK> rg;
+  rg.fetch(a, b, h, c0, 0);
+  for (int t0 = 0; t0 < T; t0 += kL) {
+    const int n = min(kL, T - t0);
+    __syncthreads();   // the previous chunk is done with every buffer
+    rg.commit(s, n);
+    if (t0 + kL < T) rg.fetch(a, b, h, c0, t0 + kL);
+    __syncthreads();
+    if (warp == 0) scan_chunk(s.lf, s.ib, *s.mcar, s.A, s.mt, s.gt, lane);
+    __syncthreads();
+    readout<Tin, kSplit, kDK>(s, a.h + (((size_t)b * T + t0) * H + h) * dv + c0, (size_t)H * dv, n);
+    __syncthreads();   // C and n are read above; they change below
+    update_state<Tin, kSplit, kDK>(s);
+  }
+  __syncthreads();
+  store_final_state<Tin, kDK>(s, a, bh, c0);
 }
 
 template <typename Tin, bool kSplit, int kDK>
