@@ -236,7 +236,8 @@ def oracle_sample_rate(w, budget_s=15.0):
                    None, n_threads=cores)
     dt = time.perf_counter() - t0
     token_heads_per_s = n * w.T / dt
-    return token_heads_per_s / w.H, cores, f"{n} of {heads} heads x {w.T} tokens, fp64 oracle ({dt:.1f} s)"
+    return token_heads_per_s / w.H, cores, (f"{n} of {heads} heads x {w.T} tokens, fp64 oracle: "
+                                            f"{dt:.1f} s on {cores} threads = {dt * cores:.0f} CPU-s")
 
 
 def run_reference(args):

@@ -295,6 +295,23 @@ def test_deltanet_through_gdn2_form(d, algo, ws):
     assert eo < TOL["bf16"] and es < TOL["bf16"]
 
 
+@pytest.mark.parametrize("form,d,algo", [("gdn2", 128, "auto"), ("gdn2", 128, "fp32"),
+                                         ("rwkv7", 64, "auto"), ("rwkv7", 64, "fp32")])
+def test_zero_erase_reduces_to_gla(form, d, algo):
+    """With the erase strength at zero (GDN-2 b = 0, RWKV-7 c = 0) the recurrence is gated
+    linear attention: the oracle's GLA form on the same decays, with GDN-2's write gate
+    folded into v in fp64."""
+    w = small(form, "bf16", dk=d, dv=d, T=150, B=2, H=2, chunk=64)
+    inp = synth.forward_inputs(w)
+    inp["e1" if form == "gdn2" else "e2"] = np.zeros_like(inp["e1" if form == "gdn2" else "e2"])
+    o, S = gpu_forward(w, inp, algo=algo)
+    v = inp["v"].astype(np.float64) * (inp["e2"] if form == "gdn2" else 1.0)
+    o_ref, S_ref = oracle.forward("gla", inp["q"], inp["k"], v, inp["log_w"], None, None, None)
+    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
+    print(f"zero erase {form} {algo}: o {eo:.3e} S {es:.3e}")
+    assert eo < TOL["bf16"] and es < TOL["bf16"]
+
+
 def test_tc_rejects_what_it_does_not_cover():
     w = small("rwkv7", "bf16", dk=32, dv=32, T=64, B=1, H=1, chunk=64)
     inp = synth.forward_inputs(w)
