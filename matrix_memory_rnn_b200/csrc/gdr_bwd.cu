@@ -383,8 +383,13 @@ __global__ void __launch_bounds__(kThreads, kSplit ? 1 : 2) bwd_prep_kernel(BwdP
     zero_acc(acc[u]);
     if (wt < 2 * ntn) {
       const int r0 = 16 * (wt / ntn), c0 = 32 * (wt % ntn);
-      mma_seg<kSplit>(acc[u], r0, c0, 0, kC, [&](int m, int kk) { return Ti[m * kLDC + kk]; },
-                      [&](int kk, int nn) { return D.ut(U, kk, nn); }, lane);
+      // the exact and pivot paths as separate loops, so that the operand is a plain load
+      // on the pivot path
+      auto ti = [&](int m, int kk) { return Ti[m * kLDC + kk]; };
+      if (exact)
+        mma_seg<kSplit>(acc[u], r0, c0, 0, kC, ti, [&](int kk, int nn) { return D.ut(U, kk, nn); }, lane);
+      else
+        mma_seg<kSplit>(acc[u], r0, c0, 0, kC, ti, [&](int kk, int nn) { return U[kk * LDK + nn]; }, lane);
     } else if (wt < ntiles) {
       const int r0 = 16 * (wt - 2 * ntn);
       mma_seg<kSplit>(acc[u], r0, 0, 0, kC, [&](int m, int kk) { return Ti[m * kLDC + kk]; },
@@ -414,8 +419,12 @@ __global__ void __launch_bounds__(kThreads, kSplit ? 1 : 2) bwd_prep_kernel(BwdP
     float acc[4][4];
     zero_acc(acc);
     if (which == 0) {
-      mma_seg<kSplit>(acc, r0, c0, 0, kC, [&](int m, int kk) { return Nm[kk * kLDC + m]; },
-                      [&](int kk, int nn) { return D.end(Z, kk, nn); }, lane);
+      auto nt = [&](int m, int kk) { return Nm[kk * kLDC + m]; };
+      if (exact)
+        mma_seg<kSplit>(acc, r0, c0, 0, kC, nt, [&](int kk, int nn) { return D.end(Z, kk, nn); }, lane);
+      else
+        mma_seg<kSplit>(acc, r0, c0, 0, kC, nt, [&](int kk, int nn) { return Z[kk * LDK + nn] * D.pi[nn]; },
+                        lane);
       for_acc(acc, r0, c0, lane, [&](int r, int cc, float x) {
         rec[2 * kC * dk + r * dk + cc] = D.end(K, r, cc) - x;
       });
@@ -643,9 +652,13 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
       pf.store(dR, LDV, kC, dv, nullptr);
       __syncthreads();
       if (kk0 + kC < dk) pf.load(S + (size_t)(kk0 + kC) * dv, dv, kC, dv);
-      if (vt_own)
-        mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return D.ut(U, m, kk0 + kk); },
-                        [&](int kk, int nn) { return dR[kk * LDV + nn]; }, lane);
+      if (vt_own) {
+        auto st = [&](int kk, int nn) { return dR[kk * LDV + nn]; };
+        if (exact)
+          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return D.ut(U, m, kk0 + kk); }, st, lane);
+        else
+          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return U[m * LDK + kk0 + kk]; }, st, lane);
+      }
       __syncthreads();
     }
     if (vt_own) {

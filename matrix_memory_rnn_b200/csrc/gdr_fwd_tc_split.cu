@@ -281,6 +281,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   // GDN-2 (erase gate b, optional write gate) or GLA (u = 0: no b, no write gate)
   const bool has_b = p.form == GDR_FORM_GDN2;
   const bool has_wg = has_b && p.e2 != nullptr;
+  // Which group forms V^ from v and the write gate: only MMA2 (back group) reads it.  The
+  // plain gate product is cheap and stays in the front group; the Muir activations
+  // (SiLU(v) sigmoid(z_w)) go to the back group, which otherwise waits on the front.
+  const bool wg_front = has_wg && !kMuir, wg_back = has_wg && kMuir;
   float *sNRM = reinterpret_cast<float *>(smem + SL::NRM);   // [buffer][q, k][token]
   const __nv_bfloat16 *gzq = static_cast<const __nv_bfloat16 *>(p.zq);
   auto item_of = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
@@ -359,11 +363,11 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       if (poller) sexact[bi] = 0;
       if (!group_wait<FrontSync>(lfull, j & 1, sabort, poller)) break;
       if (!group_wait<FrontSync>(bfull + bi, (j >> 1) & 1, sabort, poller)) break;
-      if (has_wg && !group_wait<FrontSync>(wfull + bi, (j >> 1) & 1, sabort, poller)) break;
+      if (wg_front && !group_wait<FrontSync>(wfull + bi, (j >> 1) & 1, sabort, poller)) break;
       if (poller) {
         cnt[kLDone] = j + 1;
         cnt[kBDone0 + bi] += 1;
-        if (has_wg) cnt[kWDone0 + bi] += 1;
+        if (wg_front) cnt[kWDone0 + bi] += 1;
       }
       GDR_PREP_PHASE(1);
 
@@ -548,7 +552,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         else operands(std::true_type{});
       }
       // ---- V^ = wg (.) v in place (wg staged at the same swizzled offsets)
-      if (has_wg) {
+      if (wg_front) {
         const uint8_t *sw = smem + SL::SW + bi * (kC * kDK * 2);
 #pragma unroll
         for (int u = 0; u < kC * 16 / kGroup; ++u) {
@@ -556,13 +560,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
           float v8[8], w8[8];
           unpack8(*reinterpret_cast<const uint4 *>(buf + SL::VH + off), v8);
           unpack8(*reinterpret_cast<const uint4 *>(sw + off), w8);
-          if constexpr (kMuir) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v8[e] = silu_f(v8[e]) * sigmoid_f(w8[e]);   // silu(v) sigmoid(z_w)
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
-          }
+          for (int e = 0; e < 8; ++e) v8[e] *= w8[e];
           st_smem16(buf, SL::VH + off, pack8(v8));
         }
       }
@@ -571,7 +570,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       GDR_PREP_PHASE(3);
 
       // ---- the write-gate staging tile is read: load chunk j + 2's; MMA1 on this chunk
-      if (gt == 32 && has_wg && j + 2 < nloc) {
+      if (gt == 32 && wg_front && j + 2 < nloc) {
         fence_proxy_async_smem();
         const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
         load_gate(smem + SL::SW + bi * (kC * kDK * 2), maps, wfull + bi, bhn / H, bhn % H, cn * kC);
@@ -609,6 +608,24 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
       GDR_PREP_PHASE(8);
       if (!group_wait<BackSync>(ready + bi, (j >> 1) & 1, sabort, poller)) break;
+      // ---- Muir: V^ = SiLU(v) sigmoid(z_w) in place while MMA1 runs (v's tile landed
+      //      before the hand-off; the gate staging tile is waited for here)
+      if (wg_back) {
+        if (!group_wait<BackSync>(wfull + bi, (j >> 1) & 1, sabort, poller)) break;
+        if (poller) cnt[kWDone0 + bi] += 1;
+        const uint8_t *sw = smem + SL::SW + bi * (kC * kDK * 2);
+#pragma unroll
+        for (int u = 0; u < kC * 16 / kGroup; ++u) {
+          const uint32_t off = (uint32_t)(gt + u * kGroup) * 16;
+          float v8[8], w8[8];
+          unpack8(*reinterpret_cast<const uint4 *>(buf + SL::VH + off), v8);
+          unpack8(*reinterpret_cast<const uint4 *>(sw + off), w8);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v8[e] = silu_f(v8[e]) * sigmoid_f(w8[e]);
+          st_smem16(buf, SL::VH + off, pack8(v8));
+        }
+        fence_proxy_async_smem();   // MMA2 reads V^ after the barriers below
+      }
       if (!group_wait<BackSync>(bar1 + bi, (j >> 1) & 1, sabort, poller)) break;
       if (poller) cnt[kM1Done0 + bi] += 1;
       tc_fence_after();
@@ -668,6 +685,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       tc_fence_before();
       BackSync::sync();
       GDR_PREP_PHASE(10);
+      // Muir: every back thread has read the gate staging tile: chunk j + 2's into it
+      if (wg_back && gt == 32 && j + 2 < nloc) {
+        fence_proxy_async_smem();
+        const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
+        load_gate(smem + SL::SW + bi * (kC * kDK * 2), maps, wfull + bi, bhn / H, bhn % H, cn * kC);
+        cnt[kWIss0 + bi] += 1;
+      }
 
       // ---- T^-1 (fp32, into the dead Q rows of A_LM), bf16 copy (into the dead L tile)
       invert_diag_blocks8<Ix, QRowsIdx, kGroup, BackSync>(sL, sTi, gt);
