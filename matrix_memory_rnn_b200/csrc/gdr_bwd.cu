@@ -624,6 +624,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
   const float *G = p.adj + cid * dk * dv;                              // its adjoint
 
   const bool exact = load_chunk<Tin, kDK, kDV>(p, L, sm, b, h, t0, n, true);
+  // S's first 32 rows, in flight while the chunk matrices and T^-1 are formed
+  Prefetch<4> pfS;
+  pfS.load(S, dv, kC, dv);
   chunk_matrices<kSplit, kDK>(L, sm, exact, true);
   invert_unit_lower32(sm + L.A, sm + L.Ti);
 
@@ -646,8 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
   {
     float acc[4][4];
     zero_acc(acc);
-    Prefetch<4> pf;
-    pf.load(S, dv, kC, dv);
+    Prefetch<4> &pf = pfS;
     for (int kk0 = 0; kk0 < dk; kk0 += kC) {
       pf.store(dR, LDV, kC, dv, nullptr);
       __syncthreads();
@@ -667,6 +669,9 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
       for_acc(acc, vr0, vc0, lane, [&](int r, int cc, float x) { Tmp[r * LDV + cc] = x; });
     }
   }
+  // dS_end's first 32 rows, in flight during E = T^-1 R
+  Prefetch<4> pfG;
+  pfG.load(G, dv, kC, dv);
   __syncthreads();
   // E = T^-1 R
   if (vt_own) {
@@ -677,23 +682,27 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
     for_acc(acc, vr0, vc0, lane, [&](int r, int cc, float x) { E[r * LDV + cc] = x; });
   }
   __syncthreads();
-  // dE = -(Z~ dS_end + M_z^T dO) (into Tmp): dS_end staged into dR
+  // dE = -(Z~ dS_end + M_z^T dO) (into Tmp) and the K~ dS_end part of dV (kept in
+  // registers): dS_end staged into dR once for both
+  float accv[4][4];
+  zero_acc(accv);
   {
     float acc[4][4];
     zero_acc(acc);
-    Prefetch<4> pf;
-    pf.load(G, dv, kC, dv);
+    Prefetch<4> &pf = pfG;
     for (int kk0 = 0; kk0 < dk; kk0 += kC) {
       pf.store(dR, LDV, kC, dv, gscale ? gscale + kk0 : nullptr);
       __syncthreads();
       if (kk0 + kC < dk) pf.load(G + (size_t)(kk0 + kC) * dv, dv, kC, dv);
       if (vt_own) {
-        if (exact)
-          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return D.end(Z, m, kk0 + kk); },
-                          [&](int kk, int nn) { return dR[kk * LDV + nn]; }, lane);
-        else
-          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return Z[m * LDK + kk0 + kk]; },
-                          [&](int kk, int nn) { return dR[kk * LDV + nn]; }, lane);
+        auto gs = [&](int kk, int nn) { return dR[kk * LDV + nn]; };
+        if (exact) {
+          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return D.end(Z, m, kk0 + kk); }, gs, lane);
+          mma_seg<kSplit>(accv, vr0, vc0, 0, kC, [&](int m, int kk) { return D.end(K, m, kk0 + kk); }, gs, lane);
+        } else {
+          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return Z[m * LDK + kk0 + kk]; }, gs, lane);
+          mma_seg<kSplit>(accv, vr0, vc0, 0, kC, [&](int m, int kk) { return K[m * LDK + kk0 + kk]; }, gs, lane);
+        }
       }
       __syncthreads();
     }
@@ -713,43 +722,54 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
     for_acc(acc, vr0, vc0, lane, [&](int r, int cc, float x) { dR[r * LDV + cc] = x; });
   }
   __syncthreads();
-  // dV = K~ dS_end + M_k^T dO + B^T dR (written out): dS_end staged into Tmp
+  // the first slabs of S^T and dS_end^T for the token gradients, in flight during dV and
+  // the C x C gradients: kDepth slabs ahead (two where the registers allow)
+  constexpr int kDepth = kSplit ? 1 : 2;
+  Prefetch<2> pS[kDepth], pG[kDepth];
+#pragma unroll
+  for (int d = 0; d < kDepth; ++d)
+    if (d * kSlab < dv) {
+      pS[d].load(S + d * kSlab, dv, dk, kSlab);
+      pG[d].load(G + d * kSlab, dv, dk, kSlab);
+    }
+  // dV = K~ dS_end (above) + M_k^T dO + B^T dR (written out)
   {
     const Tin *v = static_cast<const Tin *>(p.v), *e2 = static_cast<const Tin *>(p.e2);
     const bool gated = p.form == GDR_FORM_GDN2 && e2 != nullptr;
     float acc[4][4];
-    zero_acc(acc);
-    Prefetch<4> pf;
-    pf.load(G, dv, kC, dv);
-    for (int kk0 = 0; kk0 < dk; kk0 += kC) {
-      pf.store(Tmp, LDV, kC, dv, gscale ? gscale + kk0 : nullptr);
-      __syncthreads();
-      if (kk0 + kC < dk) pf.load(G + (size_t)(kk0 + kC) * dv, dv, kC, dv);
-      if (vt_own) {
-        if (exact)
-          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return D.end(K, m, kk0 + kk); },
-                          [&](int kk, int nn) { return Tmp[kk * LDV + nn]; }, lane);
-        else
-          mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return K[m * LDK + kk0 + kk]; },
-                          [&](int kk, int nn) { return Tmp[kk * LDV + nn]; }, lane);
-      }
-      __syncthreads();
-    }
     if (vt_own) {
-      mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return Mk[kk * kLDC + m]; },
+      mma_seg<kSplit>(accv, vr0, vc0, 0, kC, [&](int m, int kk) { return Mk[kk * kLDC + m]; },
                       [&](int kk, int nn) { return dO[kk * LDV + nn]; }, lane);
-      mma_seg<kSplit>(acc, vr0, vc0, 0, kC, [&](int m, int kk) { return Bm[kk * kLDC + m]; },
+      mma_seg<kSplit>(accv, vr0, vc0, 0, kC, [&](int m, int kk) { return Bm[kk * kLDC + m]; },
                       [&](int kk, int nn) { return dR[kk * LDV + nn]; }, lane);
-      for_acc(acc, vr0, vc0, lane, [&](int r, int cc, float x) {
-        if (r >= n) return;
-        const size_t iv = (((size_t)b * T + t0 + r) * H + h) * dv + cc;
-        if (gated) {
-          p.gv[iv] = x * ld_in(e2, iv);
-          p.ge2[iv] = x * ld_in(v, iv);
-        } else {
-          p.gv[iv] = x;
+      // the write-gate and value entries of this thread's 16 outputs, loaded together
+      const int g = lane >> 2, tq = lane & 3;
+      float pw[4][4], pv[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = vr0 + g + 8 * (e >> 1), cc = vc0 + 8 * i + 2 * tq + (e & 1);
+          const size_t iv = (((size_t)b * T + t0 + r) * H + h) * dv + cc;
+          const bool in = gated && r < n;
+          pw[i][e] = in ? ld_in(e2, iv) : 0.f;
+          pv[i][e] = in ? ld_in(v, iv) : 0.f;
         }
-      });
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = vr0 + g + 8 * (e >> 1), cc = vc0 + 8 * i + 2 * tq + (e & 1);
+          if (r >= n) continue;
+          const size_t iv = (((size_t)b * T + t0 + r) * H + h) * dv + cc;
+          const float x = accv[i][e];
+          if (gated) {
+            p.gv[iv] = x * pw[i][e];
+            p.ge2[iv] = x * pv[i][e];
+          } else {
+            p.gv[iv] = x;
+          }
+        }
     }
     // 0 dM_k = tril(dO V^T), 1 dM_z = -tril(dO E^T), 2 dA = -stril(dR E^T), 3 dB = stril(dR V^T)
     {
@@ -780,16 +800,16 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
     zero_acc(au);
     zero_acc(ak);
     zero_acc(az);
-    Prefetch<2> pS, pG;
-    pS.load(S, dv, dk, kSlab);
-    pG.load(G, dv, dk, kSlab);
-    for (int cs = 0; cs < dv; cs += kSlab) {
-      pS.store(slS, kLDS, dk, kSlab, nullptr);
-      pG.store(slG, kLDS, dk, kSlab, gscale);
+    constexpr int kUnroll = kDepth > 1 ? kDV / kSlab : 1;   // two buffers alternate statically
+#pragma unroll kUnroll
+    for (int it = 0; it < dv / kSlab; ++it) {
+      const int cs = it * kSlab, q = it % kDepth;
+      pS[q].store(slS, kLDS, dk, kSlab, nullptr);
+      pG[q].store(slG, kLDS, dk, kSlab, gscale);
       __syncthreads();
-      if (cs + kSlab < dv) {
-        pS.load(S + cs + kSlab, dv, dk, kSlab);
-        pG.load(G + cs + kSlab, dv, dk, kSlab);
+      if (cs + kDepth * kSlab < dv) {
+        pS[q].load(S + cs + kDepth * kSlab, dv, dk, kSlab);
+        pG[q].load(G + cs + kDepth * kSlab, dv, dk, kSlab);
       }
       if (own) {
         auto St = [&](int kk, int nn) { return slS[nn * kLDS + kk]; };
@@ -814,6 +834,20 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
         mma_seg<kSplit>(az, r0, c0, 0, kC, [&](int m, int kk) { return dMz[kk * kLDC + m]; }, tile(Q), lane);
       }
       const int g = lane >> 2, tq = lane & 3;
+      // the form's inputs of this thread's 16 outputs (GDN-2's erase gate b, RWKV-7's c),
+      // loaded together ahead of the loop
+      float pre[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int t = r0 + g + 8 * (e >> 1), j = c0 + 8 * i + 2 * tq + (e & 1);
+          const size_t tok = ((size_t)b * T + t0 + t) * H + h;
+          pre[i][e] = t >= n ? 0.f
+                      : p.form == GDR_FORM_GDN2  ? ld_in(e1, tok * dk + j)
+                      : p.form == GDR_FORM_RWKV7 ? ld_in(e2, tok)
+                                                 : 0.f;
+        }
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -875,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
               p.ge2[ik] = dz;
               break;
             case GDR_FORM_GDN2: {
-              const float bb = ld_in(e1, ik);
+              const float bb = pre[i][e];
               p.gk[ik] = dkk + dz + du * w * bb;
               p.ge1[ik] = du * w * kr;
               lw_local = 0.f;
@@ -883,7 +917,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_grads_kernel(BwdParams p) {
             }
             case GDR_FORM_RWKV7: {
               p.gk[ik] = dkk;
-              p.ge1[ik] = ld_in(e2, tok) * du + dz;
+              p.ge1[ik] = pre[i][e] * du + dz;
               atomicAdd(sm + L.dc + t, du * z);   // z = a
               break;
             }
