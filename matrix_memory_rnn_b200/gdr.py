@@ -143,6 +143,13 @@ def _need(t, name, dtype, shape):
     return t
 
 
+def _workspace(w):
+    """A caller-supplied workspace must be device memory: a contiguous CUDA tensor."""
+    if w is not None and (not isinstance(w, torch.Tensor) or not w.is_cuda or not w.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return w
+
+
 def _dtype_of(q):
     if q.dtype == torch.bfloat16:
         return "bf16", torch.bfloat16
@@ -185,7 +192,8 @@ def _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, workspace
     a.q, a.k, a.v, a.log_w = _ptr(q), _ptr(k), _ptr(v), _ptr(log_w)
     a.e1, a.e2, a.S0, a.o, a.S_T = _ptr(e1), _ptr(e2), _ptr(S0), _ptr(o), _ptr(S_T)
     if workspace is not None:
-        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+        a.workspace = _ptr(_workspace(workspace))
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
     return a
 
 
@@ -255,7 +263,8 @@ def _bwd_struct(form, q, k, v, log_w, e1, e2, S0, dO, dS_T, grads, chunk, worksp
         for name in ("q", "k", "v", "log_w", "e1", "e2", "S0"):
             setattr(a, "g_" + name, _ptr(grads.get(name)))
     if workspace is not None:
-        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+        a.workspace = _ptr(_workspace(workspace))
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
     return a
 
 
@@ -343,7 +352,8 @@ def _muir_struct(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat, rms_weight, rms
     a.rms_eps = float(rms_eps)
     a.unfused = int(bool(unfused))
     if workspace is not None:
-        a.workspace, a.workspace_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+        a.workspace = _ptr(_workspace(workspace))
+        a.workspace_bytes = workspace.numel() * workspace.element_size()
     return a
 
 
@@ -400,6 +410,7 @@ def gdr_mlstm_forward(q, k, v, f_pre, i_pre, C0=None, n0=None, m0=None, *, h=Non
     dev = q.device
     if h is None:
         h = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    _need(h, "h", torch.float32, (B, T, H, dv))
     C_T = n_T = m_T = None
     if want_state:
         C_T = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
@@ -450,6 +461,7 @@ def gdr_state_compose(M, S_in, Q, *, out=None, stream=None):
         _need(S_in, "S_in", torch.float32, (B, H, dk, dv))
     if out is None:
         out = torch.empty_like(Q)
+    _need(out, "out", torch.float32, (B, H, dk, dv))
     _check("gdr_state_compose", _load().gdr_state_compose(_ptr(out), _ptr(M), _ptr(S_in), _ptr(Q),
                                                           B * H, dk, dv, _stream(stream)))
     return out
@@ -469,7 +481,7 @@ def gdr_state_init(S, src=None, *, stream=None):
 def gdr_read_status(workspace, *, stream=None):
     """Synchronizes and returns (and clears) the device status word of ``workspace``."""
     st = ctypes.c_int(0)
-    _check("gdr_read_status", _load().gdr_read_status(_ptr(workspace), _stream(stream),
+    _check("gdr_read_status", _load().gdr_read_status(_ptr(_workspace(workspace)), _stream(stream),
                                                       ctypes.byref(st)))
     return STATUS.get(st.value, st.value)
 

@@ -187,3 +187,18 @@ def test_state_compose_rejects_bad_arguments_on_host(lib):
     assert lib.gdr_state_compose(fake, fake, fake, fake, 2, 48, 64, None) == 1
     assert lib.gdr_state_compose(fake, fake, fake, None, 2, 64, 64, None) == 1   # S_in aliases S_out
     assert lib.gdr_state_compose(fake, fake, None, None, 0, 64, 64, None) == 0
+
+
+def test_binding_rejects_host_memory():
+    """Host tensors never reach the library: the binding checks every tensor and every
+    caller-supplied workspace for device memory before marshalling a pointer."""
+    import torch
+    with pytest.raises(ValueError):
+        gdr._workspace(torch.zeros(256, dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        gdr._need(torch.zeros(4), "x", torch.float32, (4,))
+    x = torch.zeros(1, 8, 1, 64)
+    with pytest.raises(ValueError):
+        gdr.gdr_forward_chunked("gla", x, x, x, x)
+    with pytest.raises(ValueError):
+        gdr.gdr_state_compose(torch.zeros(1, 1, 64, 64), None, torch.zeros(1, 1, 64, 64))
