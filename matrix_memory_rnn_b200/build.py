@@ -1,7 +1,10 @@
 """Builds ``libgdr.so`` (the CUDA kernels and the C ABI) in-tree with nvcc for sm_100a.
 
-Usage: ``python -m matrix_memory_rnn_b200.build [--force]``.  Objects go to
+Usage: ``python -m matrix_memory_rnn_b200.build [--force] [--timing]``.  Objects go to
 ``matrix_memory_rnn_b200/_build/``; the library to ``matrix_memory_rnn_b200/libgdr.so``.
+``--timing`` builds ``libgdr_timing.so`` instead (objects in ``_build_timing/``): the same
+kernels with the per-phase cycle hooks of ``csrc/gdr_phase_timing.cuh`` filled in, for
+``python -m matrix_memory_rnn_b200.phase_timing``; it is never loaded by the binding.
 """
 from __future__ import annotations
 
@@ -18,6 +21,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libgdr.so")
+BUILD_TIMING = os.path.join(PKG, "_build_timing")
+LIB_TIMING = os.path.join(PKG, "libgdr_timing.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -50,16 +55,18 @@ def _stale(target, deps):
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, timing: bool = False) -> str:
+    build_dir, lib = (BUILD_TIMING, LIB_TIMING) if timing else (BUILD, LIB)
+    extra = ["-DGDR_PHASE_TIMING"] if timing else []
+    os.makedirs(build_dir, exist_ok=True)
     headers = glob.glob(os.path.join(CSRC, "*.cuh")) + glob.glob(os.path.join(INCLUDE, "*.h"))
     jobs = []
     objs = []
     for src in _sources():
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or _stale(obj, [src] + headers):
-            cmd = [nvcc()] + NVCC_FLAGS + ["-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+            cmd = [nvcc()] + NVCC_FLAGS + extra + ["-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
             jobs.append(cmd)
     if jobs:
         with cf.ThreadPoolExecutor(max_workers=min(8, len(jobs))) as ex:
@@ -70,13 +77,13 @@ def build(force: bool = False, verbose: bool = False) -> str:
                     sys.stderr.write(r.stdout + r.stderr)
                 if r.returncode != 0:
                     raise RuntimeError(f"nvcc failed: {' '.join(cmd)}")
-    if force or jobs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or jobs or _stale(lib, objs):
+        tmp = lib + f".tmp{os.getpid()}"
         subprocess.check_call([nvcc(), "-shared", "-gencode", "arch=compute_100a,code=sm_100a",
                                "-o", tmp] + objs + ["-lcuda"])
-        os.replace(tmp, LIB)
-    return LIB
+        os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, timing="--timing" in sys.argv))

@@ -32,9 +32,10 @@
 #include <mutex>
 #include <type_traits>
 
+#include "gdr_phase_timing.cuh"
 #include "gdr_tc_common.cuh"
 
-// Phase hooks for an external timing harness; empty in the library build.
+// Phase hooks: filled by gdr_phase_timing.cuh in the timing build, empty in libgdr.so.
 #ifndef GDR_PREP_PHASE
 #define GDR_PREP_PHASE(i)
 #endif
@@ -1165,3 +1166,17 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
 }
 
 }  // namespace gdr
+
+#ifdef GDR_PHASE_TIMING
+// Timing build only: copies the per-phase cycle sums ([2][16]: chain, prep) and the number
+// of recording threads ([2]) to host memory, then clears them.  Returns 0 or a CUDA error.
+extern "C" int gdr_phase_timing_read(unsigned long long *cycles, unsigned long long *threads) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(cycles, gdr::g_phase_cycles, sizeof(gdr::g_phase_cycles));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(threads, gdr::g_phase_threads, sizeof(gdr::g_phase_threads));
+  static const unsigned long long zc[2][16] = {}, zt[2] = {};
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_phase_cycles, zc, sizeof(zc));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_phase_threads, zt, sizeof(zt));
+  return (int)e;
+}
+#endif
