@@ -209,34 +209,9 @@ struct GroupSync {
   }
 };
 
-// Step 1: the four diagonal 16 x 16 blocks (and zeros in the upper blocks level 2 reads).
-// `tid` is the thread's index within the group that runs the inverse.
-template <class IxL, class IxT, int NT, class Sync = CtaSync>
-__device__ void invert_diag_blocks(const float *Lm, float *Ti, int tid) {
-  if (tid < 64) {
-    const int blk = tid >> 4, c = tid & 15, o = 16 * blk;
-    float x[16];
-#pragma unroll
-    for (int t = 0; t < 16; ++t) {
-      float acc = (t == c) ? 1.f : 0.f;
-#pragma unroll
-      for (int s = 0; s < t; ++s) acc -= Lm[IxL::at(o + t, o + s)] * x[s];
-      x[t] = acc;
-    }
-#pragma unroll
-    for (int t = 0; t < 16; ++t) Ti[IxT::at(o + t, o + c)] = x[t];
-  } else if (tid < 64 + 2 * 256 / 4) {
-    // zero the upper 16 x 16 blocks of the two diagonal 32 x 32 blocks (read by level 2)
-    const int k = (tid - 64) * 4, q = k >> 8, r = 32 * q + ((k >> 4) & 15), c = 32 * q + 16 + (k & 15);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) Ti[IxT::at(r, c + e)] = 0.f;
-  }
-  Sync::sync();
-}
-
-// Step 1 with shorter dependency chains: the eight 8 x 8 diagonal blocks by forward
-// substitution (64 threads), then each 16 x 16 block's lower-left 8 x 8 by the same
-// merge X21 = -T_R^-1 (L_RL T_L^-1) (one thread per entry).  Needs NT >= 256.
+// Step 1: the eight 8 x 8 diagonal blocks by forward substitution (64 threads), then each
+// 16 x 16 block's lower-left 8 x 8 by the merge X21 = -T_R^-1 (L_RL T_L^-1) (one thread per
+// entry).  Needs NT >= 256.
 template <class IxL, class IxT, int NT, class Sync = CtaSync>
 __device__ void invert_diag_blocks8(float *Lm, float *Ti, int tid) {
   static_assert(NT >= 256, "one thread per entry of the four 8 x 8 merges");
@@ -317,12 +292,6 @@ __device__ void invert_merge_levels(float *Lm, float *Ti, int tid) {
     store_16x8<IxT>(x, -1.f, Ti, 32 + 16 * mt, 8 * nt2, lane);
   }
   Sync::sync();
-}
-
-template <class IxL, class IxT, int NT>
-__device__ void invert_unit_lower_mma(float *Lm, float *Ti, int tid) {
-  invert_diag_blocks<IxL, IxT, NT>(Lm, Ti, tid);
-  invert_merge_levels<IxL, IxT, NT>(Lm, Ti, tid);
 }
 
 // Row-major C x C fp32 storage for invert_unit_lower: padded rows (68 floats, 16-byte
