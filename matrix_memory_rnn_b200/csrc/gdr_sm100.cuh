@@ -68,7 +68,7 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
-// ---------------------------------------------------------------- bulk copy (TMA, no multicast)
+// ---------------------------------------------------------------- bulk copy (TMA, this CTA only)
 // Contiguous global -> shared copy of `bytes` (multiple of 16, both addresses
 // 16-byte aligned); completes as transactions on `bar`.
 __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, uint32_t bytes,
@@ -80,7 +80,7 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
       : "memory");
 }
 
-// Tiled 4-D tensor load (TMA, no multicast) of one box of `map` at coordinates
+// Tiled 4-D tensor load (TMA, into this CTA only) of one box of `map` at coordinates
 // (x, y, z, w) into shared memory; completes as transactions on `bar`.  Elements
 // outside the tensor are written as zeros.  x times the element size must be a
 // multiple of 16 bytes.
