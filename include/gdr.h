@@ -153,22 +153,38 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *args, void *stream);
  * Some callers are not allowed to allocate: a plugin whose host application owns
  * every device allocation, a serving loop that forbids allocation once its memory
  * plan is fixed, code where cudaMalloc is unavailable or would synchronize.  This
- * call computes exactly what gdr_forward_chunked computes, but ignores
- * args->workspace / workspace_bytes and uses a fixed scratch array compiled into
- * libgdr instead (a static __device__ array of 4096 bytes that every GPU loading
- * the library holds until process exit).  It calls no cudaMalloc, cudaFree or
- * other allocating routine.
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make that
- *     first call before any stream capture.
+ * call ignores args->workspace / workspace_bytes and uses a fixed scratch array
+ * compiled into libgdr instead (a static __device__ array of 4096 bytes that every
+ * GPU loading the library holds until process exit).  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *
+ * Kernels.  The array holds only the status word, so the call takes the paths of
+ * gdr_forward_chunked that need no per-chunk records:
+ *   - GDN2, bf16, dk = dv = 128, algo AUTO or TC: the single-kernel tensor-core
+ *     forward (not the faster two-kernel one, whose records do not fit);
+ *   - GLA, bf16, dk = dv = 128: algo TC returns GDR_ERR_WORKSPACE; algo AUTO runs
+ *     the fp32 kernel;
+ *   - every form at bf16, dk = dv = 64, algo AUTO or TC: the two-stream
+ *     tensor-core kernel, as gdr_forward_chunked;
+ *   - everything else (algo FP32, fp32 inputs, other sizes): the fp32 kernel, as
+ *     gdr_forward_chunked.
+ * The results are those of the kernel named, within the same error bars.
+ *
+ *   - Arguments are checked on the host, as gdr_forward_chunked checks them, before
+ *     anything is enqueued.
+ *   - The array's device address is looked up (cudaGetSymbolAddress, with the
+ *     device current) on a device's first call and cached with the id of the CUDA
+ *     context it belongs to; a call in another context (after cudaDeviceReset, or
+ *     once the primary context was released and created again) looks it up anew.
+ *     Make the first call of each context before any stream capture.
  *   - All calls share the one array; calls that overlap on the GPU (different
  *     streams, or different host threads on the same device) race on it.
  *     Serialize them.
  *   - The array keeps the last call's contents; each call clears the status word
  *     it uses on `stream` before the launch.
- *   - A call that would need more scratch than the array holds returns
- *     GDR_ERR_WORKSPACE.  The device status word lives in the library's array,
- *     so gdr_read_status cannot report this variant's device-side failures.
+ *   - The device status word lives in the library's array, so gdr_read_status
+ *     cannot report this variant's device-side failures (a bounded wait that ran
+ *     out leaves its outputs incomplete without a status).
  * Errors and all other arguments: as gdr_forward_chunked.
  */
 gdr_status gdr_forward_chunked_noalloc(const gdr_fwd_args *args, void *stream);

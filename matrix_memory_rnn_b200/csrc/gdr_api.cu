@@ -154,6 +154,60 @@ MuirLayout muir_layout(const gdr_muir_args *a) {
 
 }  // namespace
 
+namespace gdr {
+
+// Host validation and kernel selection of gdr_forward_chunked for a workspace of
+// `workspace_bytes` bytes; no CUDA call.
+gdr_status forward_plan(const gdr_fwd_args *a, const void *workspace, size_t workspace_bytes,
+                        FwdPath *path) {
+  if (!a || !path) return GDR_ERR_INVALID_ARG;
+  if (!form_ok(a->form) || !dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
+  if (a->B < 0 || a->H < 0 || a->T < 0) return GDR_ERR_INVALID_ARG;
+  if (!dim_ok(a->dk) || !dim_ok(a->dv) || !chunk_ok(a->chunk)) return GDR_ERR_UNSUPPORTED;
+  if (a->algo < GDR_ALGO_AUTO || a->algo > GDR_ALGO_TC) return GDR_ERR_INVALID_ARG;
+  const size_t tokens = (size_t)a->B * a->T * a->H;
+  gdr_status st = check_token_ptrs(a->form, tokens, a->q, a->k, a->v, a->log_w, a->e1, a->e2,
+                                   a->o);
+  if (st != GDR_OK) return st;
+  if ((a->S0 && !aligned16(a->S0)) || (a->S_T && !aligned16(a->S_T))) return GDR_ERR_MISALIGNED;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return GDR_ERR_MISALIGNED;
+  if (a->B == 0 || a->H == 0) {
+    *path = FwdPath::kNone;
+    return GDR_OK;
+  }
+  if (a->T == 0) {
+    *path = a->S_T ? FwdPath::kCopyState : FwdPath::kNone;
+    return GDR_OK;
+  }
+  const FwdParams p = fwd_params(a);
+  if (uses_tc_general(a, p)) {   // two-stream forms, d = 64: one fused kernel, status word only
+    if (workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
+    *path = FwdPath::kTcGeneral;
+    return GDR_OK;
+  }
+  const bool tc_ok = forward_tc_split_supported(p, a->dtype);
+  if (a->algo == GDR_ALGO_TC || (a->algo == GDR_ALGO_AUTO && tc_ok)) {
+    if (!tc_ok) return GDR_ERR_UNSUPPORTED;
+    if (workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
+    // the two-kernel path when the workspace holds its per-chunk records, else the
+    // single-kernel path (status word only; GDN-2 alone)
+    if (workspace_bytes >= forward_tc_split_workspace_bytes(p)) {
+      *path = FwdPath::kTcSplit;
+      return GDR_OK;
+    }
+    if (forward_tc_supported(p, a->dtype)) {
+      *path = FwdPath::kTcSingle;
+      return GDR_OK;
+    }
+    if (a->algo == GDR_ALGO_TC) return GDR_ERR_WORKSPACE;
+  }
+  if (!forward_fp32_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
+  *path = FwdPath::kFp32;     // needs no workspace (a status word is used when given)
+  return GDR_OK;
+}
+
+}  // namespace gdr
+
 extern "C" {
 
 const char *gdr_status_string(gdr_status s) {
@@ -197,44 +251,27 @@ gdr_status gdr_state_init(float *S, int B, int H, int dk, int dv, const float *s
 }
 
 gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
-  if (!a) return GDR_ERR_INVALID_ARG;
-  if (!form_ok(a->form) || !dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
-  if (a->B < 0 || a->H < 0 || a->T < 0) return GDR_ERR_INVALID_ARG;
-  if (!dim_ok(a->dk) || !dim_ok(a->dv) || !chunk_ok(a->chunk)) return GDR_ERR_UNSUPPORTED;
-  if (a->algo < GDR_ALGO_AUTO || a->algo > GDR_ALGO_TC) return GDR_ERR_INVALID_ARG;
-  const size_t tokens = (size_t)a->B * a->T * a->H;
-  gdr_status st = check_token_ptrs(a->form, tokens, a->q, a->k, a->v, a->log_w, a->e1, a->e2,
-                                   a->o);
+  gdr::FwdPath path;
+  const gdr_status st = gdr::forward_plan(a, a ? a->workspace : nullptr, a ? a->workspace_bytes : 0,
+                                          &path);
   if (st != GDR_OK) return st;
-  if ((a->S0 && !aligned16(a->S0)) || (a->S_T && !aligned16(a->S_T))) return GDR_ERR_MISALIGNED;
-  if (a->workspace && (reinterpret_cast<uintptr_t>(a->workspace) & 255u))
-    return GDR_ERR_MISALIGNED;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-
-  if (a->B == 0 || a->H == 0) return GDR_OK;
-  if (a->T == 0) {  // no tokens: S_T = S0
-    if (!a->S_T) return GDR_OK;
-    return gdr_state_init(a->S_T, a->B, a->H, a->dk, a->dv, a->S0, stream);
+  switch (path) {
+    case gdr::FwdPath::kNone:
+      return GDR_OK;
+    case gdr::FwdPath::kCopyState:   // no tokens: S_T = S0
+      return gdr_state_init(a->S_T, a->B, a->H, a->dk, a->dv, a->S0, stream);
+    default:
+      break;
   }
-
+  if (path != gdr::FwdPath::kFp32 && !a->workspace) return GDR_ERR_WORKSPACE;
   const gdr::FwdParams p = fwd_params(a);
-  if (uses_tc_general(a, p)) {   // two-stream forms, d = 64: one fused kernel, status word only
-    if (!a->workspace || a->workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
-    return cuda_status(gdr::launch_forward_tc_general(p, s));
+  switch (path) {
+    case gdr::FwdPath::kTcGeneral: return cuda_status(gdr::launch_forward_tc_general(p, s));
+    case gdr::FwdPath::kTcSplit: return cuda_status(gdr::launch_forward_tc_split(p, a->workspace, s));
+    case gdr::FwdPath::kTcSingle: return cuda_status(gdr::launch_forward_tc(p, s));
+    default: return cuda_status(gdr::launch_forward_fp32(p, a->dtype, s));
   }
-  const bool tc_ok = gdr::forward_tc_split_supported(p, a->dtype);
-  if (a->algo == GDR_ALGO_TC || (a->algo == GDR_ALGO_AUTO && tc_ok)) {
-    if (!tc_ok) return GDR_ERR_UNSUPPORTED;
-    if (!a->workspace || a->workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
-    // the two-kernel path when the workspace holds its per-chunk records, else the
-    // single-kernel path (status word only; GDN-2 alone)
-    if (a->workspace_bytes >= gdr::forward_tc_split_workspace_bytes(p))
-      return cuda_status(gdr::launch_forward_tc_split(p, a->workspace, s));
-    if (gdr::forward_tc_supported(p, a->dtype)) return cuda_status(gdr::launch_forward_tc(p, s));
-    if (a->algo == GDR_ALGO_TC) return GDR_ERR_WORKSPACE;
-  }
-  if (!gdr::forward_fp32_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
-  return cuda_status(gdr::launch_forward_fp32(p, a->dtype, s));
 }
 
 gdr_status gdr_decode_step(const gdr_step_args *a, void *stream) {

@@ -127,6 +127,15 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
 
 // Smallest workspace any forward path accepts (the device status word, padded).
 constexpr size_t kStatusBytes = 256;
+
+// Which kernel gdr_forward_chunked runs for given arguments and workspace size.
+enum class FwdPath { kNone, kCopyState, kTcGeneral, kTcSplit, kTcSingle, kFp32 };
+// Host validation and selection (no CUDA call): every check gdr_forward_chunked makes on
+// its arguments and on a workspace at `workspace` (alignment; may be null) of
+// `workspace_bytes` bytes, except that a null workspace on a path that needs one is
+// reported by the caller.
+gdr_status forward_plan(const gdr_fwd_args *a, const void *workspace, size_t workspace_bytes,
+                        FwdPath *path);
 size_t forward_fp32_smem_bytes(int dk, int dv, int chunk);
 
 }  // namespace gdr

@@ -6,7 +6,8 @@ import torch
 
 import oracle
 from matrix_memory_rnn_b200 import gdr, synth
-from parity import TOL, TOL_FP32_KERNEL, gpu_forward, head_rel_err, oracle_forward, small
+from parity import (TOL, TOL_FP32_KERNEL, check_parity, gpu_forward, head_rel_err, oracle_forward,
+                    small)
 
 pytestmark = pytest.mark.gpu
 
@@ -34,9 +35,8 @@ def test_preset_full_size(name):
     inp = synth.forward_inputs(w)
     o, S = gpu_forward(w, inp, algo="auto")
     o_ref, S_ref = oracle_forward(w, inp)
-    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
-    print(f"{name}: max head rel err o {eo:.3e} S {es:.3e}")
-    assert eo < TOL[w.dtype] and es < TOL[w.dtype]
+    check_parity(o, o_ref, (0, 2), TOL[w.dtype], f"{name} o")
+    check_parity(S, S_ref, (0, 1), TOL[w.dtype], f"{name} S_T")
 
 
 def test_zero_tokens_copies_state():
@@ -165,9 +165,8 @@ def test_tc_full_size_gdn2(path):
     inp = synth.forward_inputs(w)
     o, S = gpu_forward(w, inp, algo="tc", workspace_bytes=TC_PATHS[path])
     o_ref, S_ref = oracle_forward(w, inp)
-    eo, es = head_rel_err(o, o_ref, (0, 2)), head_rel_err(S, S_ref, (0, 1))
-    print(f"tc-{path} gdn2_bf16: o {eo:.3e} S {es:.3e}")
-    assert eo < TOL["bf16"] and es < TOL["bf16"]
+    check_parity(o, o_ref, (0, 2), TOL["bf16"], f"tc-{path} gdn2_bf16 o")
+    check_parity(S, S_ref, (0, 1), TOL["bf16"], f"tc-{path} gdn2_bf16 S_T")
 
 
 @pytest.mark.parametrize("path", sorted(TC_PATHS))

@@ -10,7 +10,7 @@ import torch
 
 import oracle
 from matrix_memory_rnn_b200 import gdr, synth
-from parity import TOL, head_rel_err, small
+from parity import TOL, check_parity, head_rel_err, small
 
 pytestmark = pytest.mark.gpu
 GOLD = os.path.join(os.path.dirname(__file__), "golden", "mlstm_recovery_ch13_4.json")
@@ -114,7 +114,5 @@ def test_mlstm_full_size_sampled_heads(preset):
     for b, hh in ((0, 0), (w.B - 1, w.H - 1)):
         sl = {k: x[b:b + 1, :, hh:hh + 1] for k, x in inp.items()}
         hr, Cr, _, _ = oracle.mlstm_forward(sl["q"], sl["k"], sl["v"], sl["f_pre"], sl["i_pre"])
-        eh = head_rel_err(h[b:b + 1, :, hh:hh + 1], hr, (0, 2))
-        eC = head_rel_err(C[b:b + 1, hh:hh + 1], Cr, (0, 1))
-        print(f"mlstm full size head ({b},{hh}): h {eh:.2e} C {eC:.2e}")
-        assert eh < TOL["bf16"] and eC < TOL["bf16"]
+        check_parity(h[b:b + 1, :, hh:hh + 1], hr, (0, 2), TOL["bf16"], f"mlstm full size ({b},{hh}) h")
+        check_parity(C[b:b + 1, hh:hh + 1], Cr, (0, 1), TOL["bf16"], f"mlstm full size ({b},{hh}) C")

@@ -7,7 +7,7 @@ import torch
 
 import oracle
 from matrix_memory_rnn_b200 import gdr, synth
-from parity import TOL, head_rel_err, small
+from parity import TOL, check_parity, head_rel_err, small
 
 pytestmark = pytest.mark.gpu
 
@@ -57,10 +57,8 @@ def test_muir_full_size_sampled_heads():
         sl = lambda a: a[b:b + 1, :, h:h + 1]
         sub = dict(inp, a_log=inp["a_log"][h:h + 1], gamma_stat=inp["gamma_stat"][h:h + 1])
         y_ref, S_ref = _ref(sub, None, sl)
-        ey = head_rel_err(y[b:b + 1, :, h:h + 1], y_ref, (0, 2))
-        es = head_rel_err(S[b:b + 1, h:h + 1], S_ref, (0, 1))
-        print(f"muir full size head ({b},{h}): y {ey:.2e} S {es:.2e}")
-        assert ey < TOL["bf16"] and es < TOL["bf16"]
+        check_parity(y[b:b + 1, :, h:h + 1], y_ref, (0, 2), TOL["bf16"], f"muir full size ({b},{h}) y")
+        check_parity(S[b:b + 1, h:h + 1], S_ref, (0, 1), TOL["bf16"], f"muir full size ({b},{h}) S_T")
 
 
 def test_muir_zero_length():
