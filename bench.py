@@ -41,16 +41,20 @@ DEC = synth.PRESETS["decode"]
 L2_BYTES = 126 * 2 ** 20
 
 
-def fwd_algorithmic_bytes(w) -> int:
-    """Token inputs in (q, k, v and the form's erase arguments at the input dtype, log_w
-    fp32), o (fp32) and S_T out."""
+def fwd_algorithmic_bytes(w, with_write_gate=False) -> int:
+    """Algorithmic bytes of one forward call: the recurrence's five token inputs (q, k, v
+    and the form's erase arguments at the input dtype, log w fp32) in and o (fp32) out, per
+    token and head -- 2048 B on the GDN-2 bf16 d = 128 workload.  The written value is
+    v itself (the Muir page feeds the kernel w (.) v); this API also accepts GDN-2's write
+    gate as a separate tensor, whose bytes ``with_write_gate`` adds (2304 B per token-head
+    there).  The final state (one d_k x d_v block per sequence) is not counted."""
     eb = 2 if w.dtype == "bf16" else 4
-    extra = {"gdn2": w.dk + w.dv,        # erase gate b, write gate wg
+    extra = {"gdn2": w.dk + (w.dv if with_write_gate else 0),   # erase gate b (+ write gate)
              "rwkv7": w.dk + 1,          # removal direction a, coefficient c
              "general": 2 * w.dk,        # u, z
              "gla": 0}[w.form]
     per_token_head = eb * (2 * w.dk + w.dv + extra) + 4 * w.dk + 4 * w.dv
-    return w.B * w.T * w.H * per_token_head + w.B * w.H * w.dk * w.dv * 4
+    return w.B * w.T * w.H * per_token_head
 
 
 def bwd_algorithmic_bytes(w) -> int:
@@ -397,12 +401,15 @@ def bench_other_workloads(ctx, args, gdr):
         ms = ctx.max_over_ranks(e0.elapsed_time(e1)) / n
         nbytes = fwd_algorithmic_bytes(w)
         gbs = nbytes / (ms * 1e-3) / 1e9
+        nbytes_wg = fwd_algorithmic_bytes(w, with_write_gate=True)
         out.append({"workload": name, "form": w.form, "dtype": w.dtype, "B": w.B, "H": w.H,
                     "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "ms_per_call": ms,
                     "tokens_per_s": w.tokens * ctx.world / (ms * 1e-3),
                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
                                  "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],
-                                 "bytes_per_call": nbytes}})
+                                 "bytes_per_call": nbytes,
+                                 "frac_with_write_gate": nbytes_wg / (ms * 1e-3) / 1e9
+                                 / ctx.peaks["hbm_gbs"]}})
         del d, ws
         torch.cuda.empty_cache()
     return out
@@ -542,6 +549,30 @@ def bench_mlstm(ctx, args, gdr):
     return out
 
 
+def bench_gemm_phases(ctx, fwd):
+    """The chunked forward's tensor-core phases, measured: the same kernels built with their
+    timing hooks (libgdr_timing.so) run the GDN-2 bf16 workload at B = 1; each MMA group is
+    timed from the issue of its first MMA to its completion (the issuing warp waits for every
+    group), and its bf16 FLOPs over those cycles, at the SM clock seen during the timed
+    forward steps, are compared with the measured dense bf16 peak.  Per kernel (all its
+    groups together) and per group."""
+    try:
+        from matrix_memory_rnn_b200 import phase_timing
+        m = phase_timing.measure(batch=1, calls=2)
+        clk = (fwd.get("clocks") or {}).get("sm_mhz") or 1965.0
+        fr = phase_timing.gemm_phase_fractions(m, ctx.peaks["bf16_tflops"], clk)
+        return {"method": "timing build, B=1: MMA group issue-to-completion cycles, groups waited "
+                          "for one at a time; FLOPs of the groups over their cycles at the forward's "
+                          "SM clock, against the measured bf16 peak",
+                "sm_mhz": clk, "peak_tflops": ctx.peaks["bf16_tflops"],
+                "kernels": {k: {"frac": v["frac"], "tflops": v["tflops"],
+                                "groups": [{kk: g[kk] for kk in ("group", "cycles", "frac")}
+                                           for g in v["groups"]]}
+                            for k, v in fr.items()}}
+    except Exception as exc:      # the timing build is optional: report why it is missing
+        return {"unavailable": f"{type(exc).__name__}: {exc}"}
+
+
 def bench_e2e(ctx, args, gdr, w, inp, names, ws):
     """The same call with host inputs, as a pipelined loop: every step copies its inputs
     from pinned host memory to the device, runs the forward and copies o back to pinned
@@ -672,6 +703,8 @@ def main():
                     help="reverse-mode workload (default: both); for profiler captures")
     ap.add_argument("--bwd-batch", type=int, default=None,
                     help="reverse-mode batch B (default: the workload's); for profiler captures")
+    ap.add_argument("--no-gemm-phase", action="store_true",
+                    help="skip the tensor-core GEMM-phase measurement (timing build, B = 1)")
     ap.add_argument("--only", default="all",
                     choices=["all", "forward", "decode", "backward", "muir", "mlstm"],
                     help="time one part only (profiling runs); the default line needs 'all'")
@@ -705,6 +738,9 @@ def main():
             if (args.only == "all" and not args.no_muir) or args.only == "muir" else None)
     mlstm = (bench_mlstm(ctx, args, gdr)
              if (args.only == "all" and not args.no_mlstm) or args.only == "mlstm" else None)
+    gemm = None
+    if args.only in ("all", "forward") and not args.no_gemm_phase and fwd is not None:
+        gemm = bench_gemm_phases(ctx, fwd)
     ctx.barrier()
     if world > 1:
         dist.destroy_process_group()
@@ -717,6 +753,7 @@ def main():
     if fwd is not None:
         w = fwd["w"]
         nbytes, nflops = fwd_algorithmic_bytes(w), fwd_flops(w)
+        nbytes_wg = fwd_algorithmic_bytes(w, with_write_gate=True)
         achieved = nbytes / (fwd["ms_kernel"] * 1e-3) / 1e9
         tflops = nflops / (fwd["ms_kernel"] * 1e-3) / 1e12
         line.update({
@@ -732,12 +769,16 @@ def main():
                                      if fwd["launches_per_call"] == 2 else None),
                          "peak_source": ctx.peaks["source"],
                          "bytes_per_launch": nbytes, "kernel_ms": fwd["ms_kernel"],
+                         "bytes_with_write_gate": nbytes_wg,
+                         "frac_with_write_gate": nbytes_wg / (fwd["ms_kernel"] * 1e-3) / 1e9
+                         / ctx.peaks["hbm_gbs"],
                          "scope": "one forward call (%d kernel launch%s)" % (
                              fwd["launches_per_call"],
                              "es" if fwd["launches_per_call"] > 1 else "")},
             "tensor": {"flops_per_launch": nflops, "achieved_tflops": tflops,
                        "peak_tflops": ctx.peaks["bf16_tflops"],
-                       "frac": tflops / ctx.peaks["bf16_tflops"]},
+                       "frac": tflops / ctx.peaks["bf16_tflops"],
+                       "gemm_phase": gemm},
             "gpu_launches": fwd["launches"], "clocks": fwd["clocks"]})
         if "e2e" in fwd:
             line["e2e"] = fwd["e2e"]

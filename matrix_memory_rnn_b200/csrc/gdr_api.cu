@@ -59,6 +59,9 @@ gdr::FwdParams fwd_params(const gdr_fwd_args *a) {
   p.status = static_cast<uint32_t *>(a->workspace);
   const char *fault = getenv("GDR_DEBUG_FAULT");
   p.debug = (fault && strcmp(fault, "skip_handoff") == 0) ? gdr::kDebugSkipHandoff : 0u;
+#ifdef GDR_PHASE_TIMING
+  if (getenv("GDR_TIMING_MMA")) p.debug |= gdr::kDebugTimeMma;
+#endif
   return p;
 }
 

@@ -42,13 +42,15 @@
 #ifndef GDR_CHAIN_PHASE
 #define GDR_CHAIN_PHASE(i)
 #endif
-#ifndef GDR_SUB_DECL
-#define GDR_SUB_DECL
-#define GDR_SUB(i)
-#endif
 #ifndef GDR_PHASE_INIT
 #define GDR_PHASE_INIT
 #define GDR_PHASE_FINI(slot)
+#endif
+#ifndef GDR_MMA_DECL
+#define GDR_MMA_DECL
+#define GDR_MMA_BEGIN()
+#define GDR_MMA_END(g, tbar)
+#define GDR_MMA_FINI(slot)
 #endif
 
 namespace gdr {
@@ -82,6 +84,9 @@ __device__ __forceinline__ uint32_t park_row(int t) {
                   : Rec::U + (t - 32) * kDK * 4;
 }
 constexpr size_t kHeaderBytes = 1024;
+// Sequences of at least this many chunks, whose chain CTAs fill at most a third of the
+// SMs, run prep and chain in one cooperative launch.
+constexpr int kFusedMinChunks = 32;
 
 __host__ __device__ inline int num_chunks(int T) { return (T + kC - 1) / kC; }
 
@@ -144,6 +149,7 @@ struct PrepMisc {             // byte offsets inside PrepSmem::MISC
   static constexpr uint32_t ABORT = 84;     // int          a bounded wait ran out
   static constexpr uint32_t EXACT = 88;     // int [2]      the buffer's chunk takes the exact path
   static constexpr uint32_t CNT = 128;      // uint32_t [16] issued / completed counts (drain)
+  static constexpr uint32_t TBAR = 192;     // uint64_t [2] timing build: MMA1 / MMA2 group timing
 };
 enum {
   kBIss0, kBIss1, kBDone0, kBDone1, kWIss0, kWIss1, kWDone0, kWDone1,
@@ -242,9 +248,23 @@ __device__ __forceinline__ float inv_norm16(const float (&x)[8]) {
   return rsqrtf(fmaxf(s, 1e-24f));
 }
 
+// The chunks one prep CTA walks: items pid, pid + nprep, pid + 2 nprep, ...; item i is
+// chunk c of sequence bh, numbered sequence-major (i = bh * nch + c) or, when chain CTAs
+// consume the records while they are made, chunk-major (i = c * BH + bh).
+struct PrepWork {
+  int pid, nprep, BH;
+  bool chunk_major;
+};
+
+// Publishes a finished record (release at GPU scope; the writers fenced their stores).
+__device__ __forceinline__ void publish(uint32_t *flag) {
+  __threadfence();
+  asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(1u) : "memory");
+}
+
 template <bool kMuir>
-__global__ void __launch_bounds__(kPrepThreads, 1)
-    tc_prep_kernel(FwdParams p, uint8_t *records, const __grid_constant__ PrepMaps maps) {
+__device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, const PrepMaps &maps,
+                                          const PrepWork W, uint32_t *flags) {
   using SL = PrepSmem;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -257,7 +277,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   const int qd = warp & 3, cpart = (warp >> 2) & 1;       // TMEM lane quarter, column half
   const int T = p.T, H = p.H, nch = num_chunks(T);
   const int items = p.B * H * nch;
-  const int nloc = items > (int)blockIdx.x ? (items - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int nloc = items > W.pid ? (items - 1 - W.pid) / W.nprep + 1 : 0;
   GDR_PHASE_INIT
 
   uint8_t *misc = smem + SL::MISC;
@@ -288,7 +308,13 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   const bool wg_front = has_wg && !kMuir, wg_back = has_wg && kMuir;
   float *sNRM = reinterpret_cast<float *>(smem + SL::NRM);   // [buffer][q, k][token]
   const __nv_bfloat16 *gzq = static_cast<const __nv_bfloat16 *>(p.zq);
-  auto item_of = [&](int j) { return (int)blockIdx.x + j * (int)gridDim.x; };
+  auto item_of = [&](int j) { return W.pid + j * W.nprep; };
+  auto c_of = [&](int it) { return W.chunk_major ? it / W.BH : it % nch; };
+  auto bh_of = [&](int it) { return W.chunk_major ? it % W.BH : it / nch; };
+  auto rec_of = [&](int it) { return records + (size_t)(bh_of(it) * nch + c_of(it)) * Rec::BYTES; };
+  uint64_t *tbar = reinterpret_cast<uint64_t *>(misc + PrepMisc::TBAR);
+  GDR_MMA_DECL
+  (void)tbar;
 
   if (warp == 0) {
     tmem_alloc(tmem_slot, 2 * kTmemCols);
@@ -304,11 +330,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     }
     mbar_init(lfull, 1);
     mbar_init(bar2, 1);
+#ifdef GDR_PHASE_TIMING
+    mbar_init(tbar, 1);
+    mbar_init(tbar + 1, 1);
+#endif
     fence_mbar_init();
     *sabort = 0;
     for (int i = 0; i < kNCnt; ++i) cnt[i] = 0;
     for (int j = 0; j < 2 && j < nloc; ++j) {
-      const int it = item_of(j), c = it % nch, bh = it / nch;
+      const int it = item_of(j), c = c_of(it), bh = bh_of(it);
       load_tiles(smem + j * SL::BUF, maps, bfull + j, bh / H, bh % H, c * kC, has_b);
       ++cnt[kBIss0 + j];
       if (has_wg) {
@@ -334,7 +364,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     for (int j = 0; j < nloc; ++j) {
       const int item = item_of(j), bi = j & 1;
       uint8_t *buf = smem + bi * SL::BUF;
-      uint8_t *rec = records + (size_t)item * Rec::BYTES;
+      uint8_t *rec = rec_of(item);
       float *a1s = sA1 + (j & 3) * kDK;
       GDR_PREP_PHASE(0);
       // Muir: this thread's 4 tokens x 8 channels of z_q and 8 static gains, loaded now so
@@ -342,10 +372,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       uint4 zq_raw[4];
       float gs8[8];
       if constexpr (kMuir) {
-        const int bh = item / nch, hh = bh % H;
+        const int bh = bh_of(item), hh = bh % H;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const int tt = (item % nch) * kC + 4 * tb + i;
+          const int tt = c_of(item) * kC + 4 * tb + i;
           zq_raw[i] = tt < T ? ld16(gzq + (((size_t)(bh / H) * T + tt) * H + hh) * kDK + j0)
                              : make_uint4(0u, 0u, 0u, 0u);
         }
@@ -378,8 +408,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       if constexpr (kMuir) {
         // log alpha = -exp(a_log[h]) softplus(z_f); tokens past T keep the state (log alpha
         // = 0), as the zero-filled log w of the plain path does
-        const float rate = __expf(p.a_log[(item / nch) % H]);
-        const int tpad = T - (item % nch) * kC;
+        const float rate = __expf(p.a_log[bh_of(item) % H]);
+        const int tpad = T - c_of(item) * kC;
         const __nv_bfloat16 *zl = reinterpret_cast<const __nv_bfloat16 *>(smem + SL::SLW);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -422,7 +452,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       // the log-w staging has been read: load the next chunk's
       if (gt == 32 && j + 1 < nloc) {
         fence_proxy_async_smem();
-        const int it = item_of(j + 1), cn = it % nch, bhn = it / nch;
+        const int it = item_of(j + 1), cn = c_of(it), bhn = bh_of(it);
         load_logw<kMuir>(smem + SL::SLW, maps, lfull, bhn / H, bhn % H, cn * kC);
         cnt[kLIss] = j + 2;
       }
@@ -566,6 +596,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
           st_smem16(buf, SL::VH + off, pack8(v8));
         }
       }
+      if (flags) __threadfence();      // this thread's record stores, before the back group publishes
       fence_proxy_async_smem();
       FrontSync::sync();
       GDR_PREP_PHASE(3);
@@ -573,7 +604,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       // ---- the write-gate staging tile is read: load chunk j + 2's; MMA1 on this chunk
       if (gt == 32 && wg_front && j + 2 < nloc) {
         fence_proxy_async_smem();
-        const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
+        const int it = item_of(j + 2), cn = c_of(it), bhn = bh_of(it);
         load_gate(smem + SL::SW + bi * (kC * kDK * 2), maps, wfull + bi, bhn / H, bhn % H, cn * kC);
         cnt[kWIss0 + bi] += 1;
       }
@@ -582,6 +613,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         tc_fence_after();
         const uint32_t bb = sb + bi * SL::BUF;
         constexpr uint32_t id = idesc_bf16_f32(128, kC, false, false);
+        GDR_MMA_BEGIN()
 #pragma unroll
         for (int s = 0; s < kDK / 16; ++s) {
           const uint64_t ad = sdesc_sw128(bb + SL::A_LM + (s >> 2) * (2 * kC * 128) + (s & 3) * 32, 16, 1024);
@@ -589,6 +621,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
           mma_bf16_warp(tD1 + 64 * bi, ad, bd, id, s > 0);
         }
         mma_commit_warp(bar1 + bi);
+        GDR_MMA_END(0, tbar);
         if (lane == 0) cnt[kM1Iss0 + bi] += 1;
       }
       // hand the chunk to the back group (the fault-injection hook withholds it)
@@ -599,12 +632,12 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     // =========================================================== back group
     const bool poller = gt == 0;
     for (int j = 0; j < nloc; ++j) {
-      const int item = item_of(j), c = item % nch, bh = item / nch, h = bh % H, b = bh / H;
+      const int item = item_of(j), c = c_of(item), bh = bh_of(item), h = bh % H, b = bh / H;
       const int t0 = c * kC, n = min(kC, T - t0), bi = j & 1;
       uint8_t *buf = smem + bi * SL::BUF;
       float *sL = reinterpret_cast<float *>(buf + SL::B_LM);
       float *sTi = reinterpret_cast<float *>(buf + SL::A_LM);
-      uint8_t *rec = records + (size_t)item * Rec::BYTES;
+      uint8_t *rec = rec_of(item);
       const float *a1s = sA1 + (j & 3) * kDK;
       auto tok_off = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDK; };
       GDR_PREP_PHASE(8);
@@ -689,7 +722,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       // Muir: every back thread has read the gate staging tile: chunk j + 2's into it
       if (wg_back && gt == 32 && j + 2 < nloc) {
         fence_proxy_async_smem();
-        const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
+        const int it = item_of(j + 2), cn = c_of(it), bhn = bh_of(it);
         load_gate(smem + SL::SW + bi * (kC * kDK * 2), maps, wfull + bi, bhn / H, bhn % H, cn * kC);
         cnt[kWIss0 + bi] += 1;
       }
@@ -715,11 +748,14 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       BackSync::sync();
       GDR_PREP_PHASE(11);
 
-      // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C
+      // ---- MMA2: U = T^-1 V^ (N = DV), Y Diag(1/alpha_1) = T^-1 (K^ f) (N = DK); K = C.
+      //      (Issued at M = 64: the transposed form, M = 128 and N = C, measured no faster for
+      //      these shapes, and its channel-per-thread readout is slower.)
       if (warp == 0) {
         tc_fence_after();
         const uint32_t bb = sb + bi * SL::BUF;
         constexpr uint32_t id = idesc_bf16_f32(64, kDK, false, true);
+        GDR_MMA_BEGIN()
 #pragma unroll
         for (int s = 0; s < kC / 16; ++s) {
           const uint64_t ad = sdesc_sw128(bb + SL::B_LM + s * 32, 16, 1024);
@@ -729,6 +765,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
           mma_bf16_warp(tmem + kDK, ad, by, id, s > 0);
         }
         mma_commit_warp(bar2);
+        GDR_MMA_END(1, tbar + 1);
         if (lane == 0) cnt[kM2Iss] = j + 1;
       }
       if (!group_wait<BackSync>(bar2, j & 1, sabort, poller)) break;
@@ -738,7 +775,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
       // ---- the buffer is free: load chunk j + 2's tiles into it
       if (gt == 32 && j + 2 < nloc) {
         fence_proxy_async_smem();
-        const int it = item_of(j + 2), cn = it % nch, bhn = it / nch;
+        const int it = item_of(j + 2), cn = c_of(it), bhn = bh_of(it);
         load_tiles(buf, maps, bfull + bi, bhn / H, bhn % H, cn * kC, has_b);
         cnt[kBIss0 + bi] += 1;
       }
@@ -771,13 +808,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
                             : Rec::U + sw128_offset(t, col + i, kC * 128))) = pack8(x + i);
         }
       }
+      if (flags) __threadfence();
       tc_fence_before();
       BackSync::sync();          // U / Y read before the next MMA2 overwrites them
+      if (flags && gt == 0) publish(flags + (size_t)bh * nch + c);
       GDR_PREP_PHASE(13);
     }
   }
 
   GDR_PHASE_FINI(1)
+  GDR_MMA_FINI(1)
   __syncthreads();
   if (tid == 0 && *sabort) {
     if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
@@ -802,8 +842,15 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
   }
 }
 
+template <bool kMuir>
+__global__ void __launch_bounds__(kPrepThreads, 1)
+    tc_prep_kernel(FwdParams p, uint8_t *records, const __grid_constant__ PrepMaps maps) {
+  prep_body<kMuir>(p, records, maps, PrepWork{(int)blockIdx.x, (int)gridDim.x, p.B * p.H, false},
+                   nullptr);
+}
+
 // ============================================================== chain kernel
-// Per chunk, for one (b, h, 64-column value slice), with S0 the bf16 copy of the
+// Per chunk, for one (b, h, value slice of NV = 64 or 128 columns), with S0 the bf16 copy of the
 // fp32 state kept in registers:
 //   MMA3   D[c&1] = [Q_pi; Y] S0          (M = 2C = 128, K = DK)   rows 0..C-1: Q_pi S0
 //   V~ = U - (Y S0)                        (warps on TMEM lanes C..2C-1)
@@ -812,13 +859,16 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 //   S <- Diag(pi_n) S + DS                 (fp32, all warps)
 //   O = rows 0..C-1 of D[c&1]              (read while MMA3 of chunk c + 1 runs)
 // Warp 0 issues the MMAs (lane 0, from converged code); warp 2 refills the record
-// ring three chunks ahead as soon as MMA4 has released a buffer.
+// ring (three records for NV = 64, two for NV = 128, the size shared memory allows) as
+// soon as MMA4 has released a buffer.  NV = 128 runs 512 threads, 32 columns each.
 template <int NV>
 struct ChainSmem {
   // per buffer: QY | KT | MM | U slice (C x NV) | pi.  The U slice sits directly after
   // M, so [M; U slice] is a valid 128-row K-major operand whose lower half only
   // feeds accumulator rows that are discarded.
-  static constexpr int NBUF = 3;
+  static constexpr int NBUF = NV == 64 ? 3 : 2;                // records in the ring
+  static constexpr int NT = NV == 64 ? 256 : 512;               // threads: 32 columns each
+  static constexpr uint32_t TMEM_COLS = NV == 64 ? 256 : 512;   // D x 2 and DS, NV columns each
   static constexpr uint32_t B_U = Rec::FRONT;
   static constexpr uint32_t B_PI = B_U + kC * NV * 2;
   static constexpr uint32_t BUF = ((B_PI + kDK * 4 + 1023) / 1024) * 1024;
@@ -827,9 +877,9 @@ struct ChainSmem {
   static constexpr uint32_t MISC = VT + kC * NV * 2;          // barriers, TMEM slot, flags
   static constexpr uint32_t ALLOC = MISC + 128 + 1024;
   static constexpr uint32_t TX = Rec::FRONT + kC * NV * 2 + kDK * 4;  // bytes per record fetch
-  static_assert(NV == 64, "one 64-column block of U per CTA");
-  static_assert(B_U == Rec::MM + kC * kC * 2 && kC * NV * 2 == kC * kC * 2,
-                "[M; U slice] must form one 128-row operand");
+  static_assert(NV == 64 || NV == 128, "one or both 64-column blocks of U per CTA");
+  static_assert(B_U == Rec::MM + kC * kC * 2,
+                "[M; first 64 columns of U] must form one 128-row operand");
   static_assert(ALLOC <= 227 * 1024, "shared memory");
 };
 
@@ -841,6 +891,7 @@ struct ChainMisc {          // byte offsets inside ChainSmem::MISC
   static constexpr uint32_t ABORT = 44;    // int      a bounded wait ran out
   static constexpr uint32_t FISS = 48;     // uint32_t [NBUF] fetches issued per buffer
   static constexpr uint32_t FDONE = 64;    // uint32_t [NBUF] fetches waited for per buffer
+  static constexpr uint32_t TBAR = 80;     // uint64_t timing build: MMA group timing
 };
 
 // One lane: fetch record `c` of this CTA's sequence into buffer c % NBUF.
@@ -858,42 +909,46 @@ __device__ __forceinline__ void fetch_record(uint8_t *smem, uint64_t *full, uint
   bulk_g2s(dst + SL::B_PI, src + Rec::PI, kDK * 4, full + buf);
 }
 
-// Warp 0 (all lanes): wait for record c, then MMA3 of chunk c into D[c & 1].
-// Returns false (and issues nothing) if the record did not arrive in time.
-template <int NV>
-__device__ __forceinline__ bool start_chunk(uint8_t *smem, uint32_t sb, uint32_t tmem, int c) {
-  using SL = ChainSmem<NV>;
-  uint64_t *full = reinterpret_cast<uint64_t *>(smem + SL::MISC + ChainMisc::FULL);
-  uint32_t *fdone = reinterpret_cast<uint32_t *>(smem + SL::MISC + ChainMisc::FDONE);
-  const int buf = c % SL::NBUF;
-  GDR_SUB_DECL
-  bool got = true;
-  if ((threadIdx.x & 31) == 0) {
-    got = mbar_wait_bounded(full + buf, (c / SL::NBUF) & 1, kWaitLimitNs);
-    if (got) ++fdone[buf];
+// Waits (one lane, bounded) until a prep CTA has published record `flag` of the same
+// launch; then orders the later bulk copy of it after the publishing CTA's stores.
+__device__ __forceinline__ bool wait_published(const uint32_t *flag, volatile int *abort) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+  if (v == 0) {
+    const uint64_t t0 = globaltimer_ns();
+    do {
+      if (*abort != 0 || globaltimer_ns() - t0 > kWaitLimitNs) return false;
+      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+    } while (v == 0);
   }
-  got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
-  GDR_SUB(0);
-  if (!got) return false;
-  const uint32_t bb = sb + buf * SL::BUF;
-  constexpr uint32_t id = idesc_bf16_f32(2 * kC, NV, false, true);
-  tc_fence_after();
-#pragma unroll
-  for (int s = 0; s < kDK / 16; ++s) {
-    const uint64_t a = sdesc_sw128(bb + Rec::QY + (s >> 2) * Rec::QY_STRIDE + (s & 3) * 32, 16, 1024);
-    const uint64_t bs = sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
-    mma_bf16_warp(tmem + 64 * (c & 1), a, bs, id, s > 0);
-  }
-  GDR_SUB(1);
-  mma_commit_warp(reinterpret_cast<uint64_t *>(smem + SL::MISC + ChainMisc::BAR3));
-  GDR_SUB(2);
+  asm volatile("fence.proxy.async.global;" ::: "memory");
   return true;
 }
 
+// Barrier of the chain's 256 threads (a named barrier, so that a CTA of more threads can
+// run the chain with the rest idle).
+template <int NT>
+using ChainSync = GroupSync<3, NT>;
+
+// Bounded wait for the MMA group committed to `bar`: thread 0 polls, the chain barrier
+// passes the completion on.  Returns false, with the abort flag set, when it ran out.
+template <int NT>
+__device__ __forceinline__ bool chain_wait_mma(uint64_t *bar, uint32_t &phase, volatile int *abort) {
+  if (threadIdx.x == 0 && *abort == 0 && !mbar_wait_bounded(bar, phase, kWaitLimitNs)) *abort = 1;
+  phase ^= 1u;
+  ChainSync<NT>::sync();
+  tc_fence_after();
+  return *abort == 0;
+}
+
+// The chain of one (b, h, value slice), run by threads 0 .. 255.  `flags` (or null):
+// records are published by prep CTAs of the same launch and waited for before fetching.
 template <int NV>
-__global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, const uint8_t *records) {
+__device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *records, int slice,
+                                           int h, int b, const uint32_t *flags) {
   using SL = ChainSmem<NV>;
-  constexpr int HALF = NV / 2, NBUF = SL::NBUF;
+  constexpr int NBUF = SL::NBUF, NT = SL::NT;
+  constexpr int HALF = 32;      // value columns per thread: NT / 128 column groups of 32
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -901,8 +956,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, hf = warp >> 2;
-  const int slice = blockIdx.x, c0 = slice * NV, h = blockIdx.y, b = blockIdx.z;
+  const int c0 = slice * NV;
   const int T = p.T, H = p.H, nch = num_chunks(T);
+  const uint32_t *rflags = flags ? flags + ((size_t)b * H + h) * nch : nullptr;
   const uint8_t *recs = records + (size_t)((size_t)b * H + h) * nch * Rec::BYTES;
   GDR_PHASE_INIT
 
@@ -916,7 +972,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
   uint32_t *fdone = reinterpret_cast<uint32_t *>(misc + ChainMisc::FDONE);
 
   if (warp == 0) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, SL::TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
@@ -926,9 +982,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     }
     mbar_init(bar3, 1);
     mbar_init(bar4, 1);
+#ifdef GDR_PHASE_TIMING
+    mbar_init(reinterpret_cast<uint64_t *>(misc + ChainMisc::TBAR), 1);
+#endif
     fence_mbar_init();
     *sabort = 0;
-    for (int cc = 0; cc < NBUF && cc < nch; ++cc) fetch_record<NV>(smem, full, fiss, recs, cc, slice);
+    for (int cc = 0; cc < NBUF && cc < nch; ++cc) {
+      if (rflags && !wait_published(rflags + cc, sabort)) {
+        *sabort = 1;
+        break;
+      }
+      fetch_record<NV>(smem, full, fiss, recs, cc, slice);
+    }
   }
 
   // fp32 state: key channel jrow, value columns [hf*HALF, hf*HALF + HALF) of this slice
@@ -946,16 +1011,44 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     st_smem16(smem, SL::S0B + sw128_offset(jrow, hf * HALF + i, kDK * 128), pack8(st + i));
   fence_proxy_async_smem();
   tc_fence_before();
-  __syncthreads();
+  ChainSync<NT>::sync();
   tc_fence_after();
   const uint32_t tmem = __shfl_sync(0xffffffffu, *tmem_slot, 0);
-  const uint32_t tDS = tmem + 128;
+  const uint32_t tDS = tmem + 2 * NV;
   const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
 
+  uint64_t *tbar = reinterpret_cast<uint64_t *>(misc + ChainMisc::TBAR);
+  GDR_MMA_DECL
+  (void)tbar;
+  // Warp 0 (all lanes): wait for record c, then MMA3 of chunk c into D[c & 1].  Returns
+  // false (and issues nothing) if the record did not arrive in time.
+  auto start_chunk = [&](int c) {
+    const int buf = c % NBUF;
+    bool got = true;
+    if (lane == 0) {
+      got = mbar_wait_bounded(full + buf, (c / NBUF) & 1, kWaitLimitNs);
+      if (got) ++fdone[buf];
+    }
+    got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
+    if (!got) return false;
+    const uint32_t bb = sb + buf * SL::BUF;
+    constexpr uint32_t id = idesc_bf16_f32(2 * kC, NV, false, true);
+    tc_fence_after();
+    GDR_MMA_BEGIN()
+#pragma unroll
+    for (int s = 0; s < kDK / 16; ++s) {
+      const uint64_t a = sdesc_sw128(bb + Rec::QY + (s >> 2) * Rec::QY_STRIDE + (s & 3) * 32, 16, 1024);
+      const uint64_t bs = sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
+      mma_bf16_warp(tmem + NV * (c & 1), a, bs, id, s > 0);
+    }
+    mma_commit_warp(bar3);
+    GDR_MMA_END(0, tbar);
+    return true;
+  };
   uint32_t iss3 = 0, iss4 = 0;   // MMA groups committed (counted by warp 0)
   uint32_t ph3 = 0, ph4 = 0;     // completions every thread has waited for
   if (warp == 0) {
-    if (start_chunk<NV>(smem, sb, tmem, 0)) ++iss3;
+    if (start_chunk(0)) ++iss3;
     else if (lane == 0) *sabort = 1;
   }
 
@@ -964,10 +1057,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     const int buf = c % NBUF, t0 = c * kC, n = min(kC, T - t0);
     const uint32_t bb = sb + buf * SL::BUF;
     const uint8_t *bsm = smem + buf * SL::BUF;
-    const uint32_t tD = tmem + 64 * (c & 1);
+    const uint32_t tD = tmem + NV * (c & 1);
     GDR_CHAIN_PHASE(0);
     // ---- wait for MMA3 (c): [Q_pi S0; Y S0] in D[c & 1]
-    if (!(ok = wait_mma(bar3, ph3, sabort))) break;
+    if (!(ok = chain_wait_mma<NT>(bar3, ph3, sabort))) break;
     const float pn = reinterpret_cast<const float *>(bsm + SL::B_PI)[jrow];
 
     GDR_CHAIN_PHASE(1);
@@ -988,7 +1081,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    ChainSync<NT>::sync();
 
     GDR_CHAIN_PHASE(2);
     // ---- MMA4: DS = K~^T V~ (M = DK) and D[c & 1] += [M; *] V~ (M = 128); K = C
@@ -996,6 +1089,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
       tc_fence_after();
       constexpr uint32_t ids = idesc_bf16_f32(128, NV, true, true);
       constexpr uint32_t ido = idesc_bf16_f32(128, NV, false, true);
+      GDR_MMA_BEGIN()
 #pragma unroll
       for (int s = 0; s < kC / 16; ++s) {
         const uint64_t ak = sdesc_sw128(bb + Rec::KT + s * 2048, kC * 128, 1024);
@@ -1005,13 +1099,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
         mma_bf16_warp(tD, am, bv, ido, 1);
       }
       mma_commit_warp(bar4);
+      GDR_MMA_END(1, tbar);
       ++iss4;
     }
-    if (!(ok = wait_mma(bar4, ph4, sabort))) break;
-    // every read of this chunk's buffer is done: refill it three chunks ahead
+    if (!(ok = chain_wait_mma<NT>(bar4, ph4, sabort))) break;
+    // every read of this chunk's buffer is done: refill it NBUF chunks ahead
     if (warp == 2 && lane == 0 && c + NBUF < nch && !*sabort) {
-      fence_proxy_async_smem();   // the CTA's reads of the buffer come before the refill
-      fetch_record<NV>(smem, full, fiss, recs, c + NBUF, slice);
+      if (rflags && !wait_published(rflags + c + NBUF, sabort)) {
+        *sabort = 1;
+      } else {
+        fence_proxy_async_smem();   // the CTA's reads of the buffer come before the refill
+        fetch_record<NV>(smem, full, fiss, recs, c + NBUF, slice);
+      }
     }
 
     GDR_CHAIN_PHASE(3);
@@ -1028,12 +1127,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    ChainSync<NT>::sync();
 
     GDR_CHAIN_PHASE(4);
     // ---- warp 0 starts chunk c + 1; warps owning lanes 0..C-1 store O (c) meanwhile
     if (warp == 0 && c + 1 < nch && !*sabort) {
-      if (start_chunk<NV>(smem, sb, tmem, c + 1)) ++iss3;
+      if (start_chunk(c + 1)) ++iss3;
       else if (lane == 0) *sabort = 1;
     }
     GDR_CHAIN_PHASE(5);
@@ -1054,6 +1153,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
   }
 
   GDR_PHASE_FINI(0)
+  GDR_MMA_FINI(0)
   if (ok && p.S_T) {
 #pragma unroll
     for (int i = 0; i < HALF; i += 4)
@@ -1061,7 +1161,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
   }
   // after a timeout: let the MMAs and record copies already in flight land before
   // the CTA exits (every wait bounded)
-  __syncthreads();
+  ChainSync<NT>::sync();
   if (!ok && tid == 0) {   // thread 0 is warp 0's issuing lane: iss3 / iss4 are its counts
     if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
     // groups complete in order: wait for the last one committed on each barrier
@@ -1074,10 +1174,37 @@ __global__ void __launch_bounds__(kThreads, 1) tc_chain_kernel(FwdParams p, cons
       }
   }
   tc_fence_before();
-  __syncthreads();
+  ChainSync<NT>::sync();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, SL::TMEM_COLS);
+  }
+}
+
+template <int NV>
+__global__ void __launch_bounds__(ChainSmem<NV>::NT, 1) tc_chain_kernel(FwdParams p, const uint8_t *records) {
+  chain_body<NV>(p, records, blockIdx.x, blockIdx.y, blockIdx.z, nullptr);
+}
+
+// Few long sequences (the chain CTAs leave most SMs idle): one cooperative launch in which
+// CTAs 0 .. nchain-1 run the chain of one (b, h, value slice) each while the others walk
+// the chunks chunk-major as prep CTAs and publish each finished record; a chain CTA waits
+// (bounded) for a record's flag before fetching it.  Only prep CTAs make records and they
+// wait on no chain CTA, and the cooperative launch keeps every CTA resident, so each wait
+// ends.
+template <bool kMuir, int NV>
+__global__ void __launch_bounds__(kPrepThreads, 1)
+    tc_fused_kernel(FwdParams p, uint8_t *records, const __grid_constant__ PrepMaps maps,
+                    uint32_t *flags, int nchain) {
+  static_assert(kPrepThreads >= ChainSmem<NV>::NT, "the chain runs on the first NT threads");
+  if ((int)blockIdx.x < nchain) {
+    if ((int)threadIdx.x >= ChainSmem<NV>::NT) return;   // the chain's barriers count its own threads
+    const int nsl = p.dv / NV, i = blockIdx.x;
+    chain_body<NV>(p, records, i % nsl, (i / nsl) % p.H, i / nsl / p.H, flags);
+  } else {
+    prep_body<kMuir>(p, records, maps,
+                     PrepWork{(int)blockIdx.x - nchain, (int)gridDim.x - nchain, p.B * p.H, true},
+                     flags);
   }
 }
 
@@ -1090,8 +1217,11 @@ bool forward_tc_split_supported(const FwdParams &p, gdr_dtype dtype) {
          p.dk == kDK && p.dv == kDK && (p.chunk == kC || p.chunk == 2 * kC);
 }
 
+// Header, one record per (b, h, chunk), then one publication flag per record (used when
+// the records are consumed as they are made).
 size_t forward_tc_split_workspace_bytes(const FwdParams &p) {
-  return kHeaderBytes + (size_t)p.B * p.H * num_chunks(p.T) * Rec::BYTES;
+  const size_t recs = (size_t)p.B * p.H * num_chunks(p.T);
+  return kHeaderBytes + recs * Rec::BYTES + ((recs * 4 + 255) & ~(size_t)255);
 }
 
 namespace {
@@ -1157,11 +1287,31 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  const int items = p.B * p.H * num_chunks(p.T);
+  const int nch = num_chunks(p.T);
+  const int items = p.B * p.H * nch;
+  int nchain = (p.dv / NV) * p.H * p.B;
+  if (nchain * 3 <= sms && nch >= kFusedMinChunks) {
+    // few long sequences: chains and prep in one cooperative launch (tc_fused_kernel)
+    auto fused = p.muir ? tc_fused_kernel<true, NV> : tc_fused_kernel<false, NV>;
+    const int smem = (int)(PrepSmem::ALLOC > ChainSmem<NV>::ALLOC ? PrepSmem::ALLOC : ChainSmem<NV>::ALLOC);
+    if ((e = cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
+      return e;
+    int per_sm = 0;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused, kPrepThreads, smem)) != cudaSuccess)
+      return e;
+    if (per_sm >= 1) {
+      uint32_t *flags = reinterpret_cast<uint32_t *>(records + (size_t)items * Rec::BYTES);
+      if ((e = cudaMemsetAsync(flags, 0, (size_t)items * 4, stream)) != cudaSuccess) return e;
+      FwdParams pp = p;
+      void *args[] = {&pp, &records, &maps, &flags, &nchain};
+      return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(fused), dim3(sms),
+                                         dim3(kPrepThreads), args, (size_t)smem, stream);
+    }
+  }
   prep<<<min(items, sms), kPrepThreads, PrepSmem::ALLOC, stream>>>(p, records, maps);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 gc(p.dv / NV, p.H, p.B);
-  tc_chain_kernel<NV><<<gc, kThreads, ChainSmem<NV>::ALLOC, stream>>>(p, records);
+  tc_chain_kernel<NV><<<gc, ChainSmem<NV>::NT, ChainSmem<NV>::ALLOC, stream>>>(p, records);
   return cudaGetLastError();
 }
 
@@ -1170,13 +1320,18 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
 #ifdef GDR_PHASE_TIMING
 // Timing build only: copies the per-phase cycle sums ([2][16]: chain, prep) and the number
 // of recording threads ([2]) to host memory, then clears them.  Returns 0 or a CUDA error.
-extern "C" int gdr_phase_timing_read(unsigned long long *cycles, unsigned long long *threads) {
+extern "C" int gdr_phase_timing_read(unsigned long long *cycles, unsigned long long *threads,
+                                     unsigned long long *mma_cycles, unsigned long long *mma_groups) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e == cudaSuccess) e = cudaMemcpyFromSymbol(cycles, gdr::g_phase_cycles, sizeof(gdr::g_phase_cycles));
   if (e == cudaSuccess) e = cudaMemcpyFromSymbol(threads, gdr::g_phase_threads, sizeof(gdr::g_phase_threads));
-  static const unsigned long long zc[2][16] = {}, zt[2] = {};
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(mma_cycles, gdr::g_mma_cycles, sizeof(gdr::g_mma_cycles));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(mma_groups, gdr::g_mma_groups, sizeof(gdr::g_mma_groups));
+  static const unsigned long long zc[2][16] = {}, zt[2] = {}, zm[2][8] = {};
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_phase_cycles, zc, sizeof(zc));
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_phase_threads, zt, sizeof(zt));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_mma_cycles, zm, sizeof(zm));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_mma_groups, zm, sizeof(zm));
   return (int)e;
 }
 #endif

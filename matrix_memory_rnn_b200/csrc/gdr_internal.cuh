@@ -69,6 +69,9 @@ struct FwdParams {
 // variable GDR_DEBUG_FAULT, read per call on the host): the prep kernel's front warp
 // group never hands its chunks to the back group, whose bounded wait then runs out.
 constexpr uint32_t kDebugSkipHandoff = 1u;
+// Timing build only (environment variable GDR_TIMING_MMA): the MMA-issuing warps wait for
+// each tensor-core group and time it.
+constexpr uint32_t kDebugTimeMma = 2u;
 
 // Reverse mode (gdr_backward_chunked).  Chunks of kBwdChunk tokens, nc of them per
 // sequence; the workspace sections hold, per chunk, the records of the two chains

@@ -2,10 +2,12 @@
 
 Runs the forward through ``libgdr_timing.so`` (the same kernels with their phase marks filled
 in, see ``csrc/gdr_phase_timing.cuh``) and prints, per kernel and phase, the average cycles
-per chunk of one recording thread: the prep kernel's front and back warp groups (one thread
-each) and the chain kernel (thread 0).  Each value is the interval that ends at the phase's
-mark, so it includes the time that thread waited for the others there.  The timing build runs
-somewhat slower than ``libgdr.so``: compare phases with one another, not with bench.py.
+per chunk of one recording thread per role: the prep kernel's front and back warp groups and
+the chain kernel's thread 0.  Each value is the interval that
+ends at the phase's mark, so it includes the time that thread waited for the others there.
+A second pass times each tensor-core group from the issue of its first MMA to its completion
+(the issuing warp then waits for every group, which changes the schedule, so the two passes
+are separate).
 
 Usage: ``python -m matrix_memory_rnn_b200.phase_timing [--batch B] [--calls N]`` (one GPU).
 """
@@ -31,22 +33,32 @@ CHAIN_PHASES = [
     (4, "state update and its bf16 copy"), (5, "MMA3 of the next chunk issued"), (6, "O read out"),
     (0, "to the next chunk"),
 ]
+# Tensor-core groups timed in the timing build (issue of the first MMA to completion, the
+# issuing warp waiting for each group): (slot, group, label, bf16 FLOPs per group).
+C, D, NV = 64, 128, 64
+MMA_GROUPS = [   # (slot, group, product, shape, FLOPs)
+    (1, 0, "[K^ f; Q f] (K g)^T", "M=128 N=64 K=128", 2 * 128 * C * D),
+    (1, 1, "T^-1 [V^ | K^ f]", "M=64 N=128 K=64, x2", 2 * 2 * 64 * D * C),
+    (0, 0, "[Q_pi; Y] S0", "M=128 N=64 K=128", 2 * 128 * NV * D),
+    (0, 1, "K~^T V~ and [M; *] V~", "M=128 N=64 K=64, x2", 2 * 2 * 128 * NV * C),
+]
 
 
-def main(argv=None) -> int:
-    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("--batch", type=int, default=4, help="B of the GDN-2 bf16 workload (H=16, T=4096)")
-    ap.add_argument("--calls", type=int, default=3, help="timed forward calls after one warm-up call")
-    args = ap.parse_args(argv)
-
+def load_timing_library():
     lib = ctypes.CDLL(build.build(timing=True))
     lib.gdr_forward_chunked.argtypes = [ctypes.POINTER(gdr.gdr_fwd_args), ctypes.c_void_p]
     lib.gdr_forward_chunked.restype = ctypes.c_int
     u64p = ctypes.POINTER(ctypes.c_ulonglong)
-    lib.gdr_phase_timing_read.argtypes = [u64p, u64p]
+    lib.gdr_phase_timing_read.argtypes = [u64p, u64p, u64p, u64p]
     lib.gdr_phase_timing_read.restype = ctypes.c_int
+    return lib
 
-    w = synth.PRESETS["gdn2_bf16"].with_(B=args.batch)
+
+def measure(batch=1, calls=3, lib=None):
+    """Runs the GDN-2 bf16 forward (B = batch, H = 16, T = 4096) through the timing build and
+    returns the per-phase cycle sums and the timed tensor-core groups, per chunk."""
+    lib = lib or load_timing_library()
+    w = synth.PRESETS["gdn2_bf16"].with_(B=batch)
     inp = synth.forward_inputs(w)
     d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "bf16")
     o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device="cuda")
@@ -57,35 +69,101 @@ def main(argv=None) -> int:
                         "tc", ws)
     cycles = (ctypes.c_ulonglong * 32)()
     threads = (ctypes.c_ulonglong * 2)()
+    mma_cycles = (ctypes.c_ulonglong * 16)()
+    mma_groups = (ctypes.c_ulonglong * 16)()
 
     def run(n):
         for _ in range(n):
             rc = lib.gdr_forward_chunked(ctypes.byref(a), None)
             if rc != 0:
                 raise RuntimeError(f"gdr_forward_chunked (timing build) failed: {rc}")
-        rc = lib.gdr_phase_timing_read(cycles, threads)
+        rc = lib.gdr_phase_timing_read(cycles, threads, mma_cycles, mma_groups)
         if rc != 0:
             raise RuntimeError(f"gdr_phase_timing_read failed: CUDA error {rc}")
 
+    import os
+    os.environ.pop("GDR_TIMING_MMA", None)
     run(1)            # warm-up; reading clears the sums
-    run(args.calls)
+    run(calls)        # phases, with the kernels' own schedule
+    out = {"w": w, "calls": calls, "threads": list(threads), "cycles": list(cycles)}
+    os.environ["GDR_TIMING_MMA"] = "1"
+    try:
+        run(calls)    # tensor-core groups, each waited for by its issuing warp
+    finally:
+        os.environ.pop("GDR_TIMING_MMA", None)
     nch = (w.T + 63) // 64
-    prep_chunks = w.B * w.H * nch * args.calls                # each group's recorder sees every chunk
-    chain_chunks = w.B * w.H * (w.dv // 64) * nch * args.calls
+    out.update({"prep_chunks": w.B * w.H * nch * calls,    # each recorder sees every chunk
+                "chain_chunks": w.B * w.H * (w.dv // 64) * nch * calls,
+                "mma_cycles": list(mma_cycles), "mma_groups": list(mma_groups)})
+    return out
+
+
+def gemm_phase_fractions(m, peak_tflops, sm_mhz):
+    """Per kernel: bf16 FLOPs of its timed tensor-core groups over their summed
+    issue-to-completion cycles, as TFLOP/s of the whole GPU at `sm_mhz` (every SM doing the
+    same) and as a fraction of `peak_tflops`.  Also per group."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    out = {}
+    for slot, name in ((1, "tc_prep_kernel"), (0, "tc_chain_kernel")):
+        fl = cyc = 0.0
+        groups = []
+        for s_, g, what, shape, flops in MMA_GROUPS:
+            n = m["mma_groups"][8 * slot + g]
+            if s_ != slot or not n:
+                continue
+            c = m["mma_cycles"][8 * slot + g] / n
+            tf = flops / c * sm_mhz * 1e6 * sms / 1e12
+            groups.append({"group": f"{what} ({shape})", "count": n, "cycles": c,
+                           "tflops": tf, "frac": tf / peak_tflops})
+            fl += flops * n
+            cyc += m["mma_cycles"][8 * slot + g]
+        if cyc:
+            tf = fl / cyc * sm_mhz * 1e6 * sms / 1e12
+            out[name] = {"tflops": tf, "frac": tf / peak_tflops, "groups": groups}
+    return out
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--batch", type=int, default=4, help="B of the GDN-2 bf16 workload (H=16, T=4096)")
+    ap.add_argument("--calls", type=int, default=3, help="timed forward calls after one warm-up call")
+    ap.add_argument("--peak-tflops", type=float, default=None,
+                    help="bf16 dense peak of the whole GPU (default: MEASURED_PEAKS.json's, else 1590)")
+    ap.add_argument("--sm-mhz", type=float, default=1965.0,
+                    help="SM clock of the run (the cycles are SM cycles)")
+    args = ap.parse_args(argv)
+
+    m = measure(args.batch, args.calls)
+    w = m["w"]
     print(f"GDN-2 bf16, B={w.B}, H={w.H}, T={w.T}, d=128, C=64; {args.calls} calls; "
-          f"recording threads: prep {threads[1]}, chain {threads[0]}")
-    for title, slot, phases, units in (("tc_prep_kernel", 1, PREP_PHASES, prep_chunks),
-                                      ("tc_chain_kernel", 0, CHAIN_PHASES, chain_chunks)):
+          f"recording threads: prep {m['threads'][1]}, chain {m['threads'][0]}")
+    for title, slot, phases, units in (("tc_prep_kernel", 1, PREP_PHASES, m["prep_chunks"]),
+                                      ("tc_chain_kernel", 0, CHAIN_PHASES, m["chain_chunks"])):
         print(f"\n{title}: cycles per chunk, by phase")
-        total = {"front": 0.0, "back": 0.0, "": 0.0}
+        total = {}
         for i, label in phases:
-            c = cycles[16 * slot + i] / units
+            c = m["cycles"][16 * slot + i] / units
             group = label.split(":")[0] if ":" in label else ""
-            total[group] += c
+            total[group] = total.get(group, 0.0) + c
             print(f"  {label:50s} {c:9.0f}")
         for g, t in total.items():
             if t:
                 print(f"  {'sum' + (' (' + g + ')' if g else ''):50s} {t:9.0f}")
+    peak = args.peak_tflops
+    if peak is None:
+        import json
+        import os
+        path = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                            "MEASURED_PEAKS.json")
+        peak = json.load(open(path))["bf16_tflops"] if os.path.exists(path) else 1590.0
+    fr = gemm_phase_fractions(m, peak, args.sm_mhz)
+    print(f"\ntensor-core groups, issue of the first MMA to completion (the issuing warp waits for "
+          f"each group); TFLOP/s of the GPU at {args.sm_mhz:.0f} MHz against {peak:.1f} TFLOP/s")
+    for name, r in fr.items():
+        for g in r["groups"]:
+            print(f"  {name:16s} {g['group']:44s} {g['count']:8d} x {g['cycles']:6.0f} cycles "
+                  f"= {g['tflops']:7.1f} TFLOP/s ({g['frac']:5.1%})")
+        print(f"  {name:16s} {'all GEMM phases':44s} {'':19s} = {r['tflops']:7.1f} TFLOP/s ({r['frac']:5.1%})")
     return 0
 
 

@@ -47,12 +47,14 @@ def head_max_err(x, ref, head_axes):
     return float(np.max(num / den)) if num.size else 0.0
 
 
-def check_parity(x, ref, head_axes, tol, label=""):
-    """Asserts both bars (Frobenius `tol`, elementwise ELEM_FACTOR * tol); returns both errors."""
+def check_parity(x, ref, head_axes, tol, label="", elem_tol=None):
+    """Asserts both bars (Frobenius `tol`, elementwise `elem_tol`, by default ELEM_FACTOR *
+    tol); returns both errors."""
+    elem_tol = ELEM_FACTOR * tol if elem_tol is None else elem_tol
     rel, mx = head_rel_err(x, ref, head_axes), head_max_err(x, ref, head_axes)
     print(f"{label}: max head rel err {rel:.3e}, max elementwise err / RMS {mx:.3e}")
     assert rel < tol, f"{label}: Frobenius {rel:.3e} >= {tol:.1e}"
-    assert mx < ELEM_FACTOR * tol, f"{label}: elementwise {mx:.3e} >= {ELEM_FACTOR * tol:.1e}"
+    assert mx < elem_tol, f"{label}: elementwise {mx:.3e} >= {elem_tol:.1e}"
     return rel, mx
 
 

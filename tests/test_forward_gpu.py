@@ -169,6 +169,23 @@ def test_tc_full_size_gdn2(path):
     check_parity(S, S_ref, (0, 1), TOL["bf16"], f"tc-{path} gdn2_bf16 S_T")
 
 
+@pytest.mark.parametrize("form", ["gdn2", "gla"])
+def test_tc_long_sequences_one_launch(form):
+    """Few long sequences (here 2 heads x 41 chunks): prep and chain CTAs share one
+    cooperative launch, the chain CTAs fetching each record once a prep CTA has published
+    it.  Against the oracle, with a ragged tail and an initial state; bit-identical on a
+    second call."""
+    w = small(form, "bf16", dk=128, dv=128, T=64 * 40 + 17, B=1, H=2, chunk=64)
+    inp = synth.forward_inputs(w)
+    inp["S0"] = synth.round_f32(np.random.default_rng(12).normal(0, 0.5, (w.B, w.H, 128, 128)))
+    o, S = gpu_forward(w, inp, algo="tc")
+    o_ref, S_ref = oracle_forward(w, inp)
+    check_parity(o, o_ref, (0, 2), TOL["bf16"], f"one launch {form} o")
+    check_parity(S, S_ref, (0, 1), TOL["bf16"], f"one launch {form} S_T")
+    o2, S2 = gpu_forward(w, inp, algo="tc")
+    assert np.array_equal(o, o2) and np.array_equal(S, S2)
+
+
 @pytest.mark.parametrize("path", sorted(TC_PATHS))
 def test_tc_kernel_strong_decay_uses_exact_path(path):
     """Channels whose decay over a chunk exceeds e^-80 take the exact pairwise path."""

@@ -12,6 +12,17 @@ from parity import TOL, check_parity, head_rel_err, small
 pytestmark = pytest.mark.gpu
 
 TOKEN = ("q", "k", "v", "zf", "zb", "zw", "zq", "zg")
+# Elementwise bar of the mixer's outputs.  (1) The readout y_t = rho (.) o_t / RMS(o_t) (.)
+# SiLU(z_g) normalizes each token: an error of o_t that scales with the head's output level R
+# (the bf16 rounding of the state's contribution) becomes an error of y_t scaled by
+# R / RMS(o_t), large for the few tokens whose output nearly cancels.  (2) The mixer's erase
+# gate b = 2 sigmoid(z_b) reaches 2, so the transition (I - k (b (.) k)^T) Diag(alpha) has an
+# eigenvalue near -1 along the current key: rounding errors along such directions are hardly
+# damped and gather in a few state entries over long sequences (about 0.12 elementwise on S_T
+# after 2300 tokens, with 3e-3 to 5e-3 Frobenius, for the fused path and for the separate
+# prologue with accurate activations alike).  A token or state entry that is wrong is off by
+# about 1 RMS, so 0.5 still separates it from these.
+Y_ELEM_TOL = 0.5
 
 
 def _run(w, inp, S0=None, algo="auto", workspace_bytes=None, unfused=False):
@@ -57,8 +68,10 @@ def test_muir_full_size_sampled_heads():
         sl = lambda a: a[b:b + 1, :, h:h + 1]
         sub = dict(inp, a_log=inp["a_log"][h:h + 1], gamma_stat=inp["gamma_stat"][h:h + 1])
         y_ref, S_ref = _ref(sub, None, sl)
-        check_parity(y[b:b + 1, :, h:h + 1], y_ref, (0, 2), TOL["bf16"], f"muir full size ({b},{h}) y")
-        check_parity(S[b:b + 1, h:h + 1], S_ref, (0, 1), TOL["bf16"], f"muir full size ({b},{h}) S_T")
+        check_parity(y[b:b + 1, :, h:h + 1], y_ref, (0, 2), TOL["bf16"], f"muir full size ({b},{h}) y",
+                     elem_tol=Y_ELEM_TOL)
+        check_parity(S[b:b + 1, h:h + 1], S_ref, (0, 1), TOL["bf16"], f"muir full size ({b},{h}) S_T",
+                     elem_tol=Y_ELEM_TOL)
 
 
 def test_muir_zero_length():
@@ -107,3 +120,19 @@ def test_muir_bf16_d128_both_paths(unfused):
     y_ref, S_ref = _ref(inp, S0)
     assert head_rel_err(y, y_ref, (0, 2)) < TOL["bf16"]
     assert head_rel_err(S, S_ref, (0, 1)) < TOL["bf16"]
+
+
+def test_muir_long_sequence_one_launch():
+    """A few long sequences run the fused mixer as one cooperative launch (prep CTAs with
+    the activations publish records that chain CTAs consume): against the oracle."""
+    w = small("gdn2", "bf16", dk=128, dv=128, T=64 * 36 + 5, B=1, H=2, chunk=64)
+    inp = synth.muir_inputs(w)
+    S0 = synth.round_f32(np.random.default_rng(14).normal(0, 0.5, (w.B, w.H, 128, 128)))
+    y, S = _run(w, inp, S0)
+    y_ref, S_ref = _ref(inp, S0)
+    check_parity(y, y_ref, (0, 2), TOL["bf16"], "muir one launch y", elem_tol=Y_ELEM_TOL)
+    check_parity(S, S_ref, (0, 1), TOL["bf16"], "muir one launch S_T", elem_tol=Y_ELEM_TOL)
+    # the separate prologue (accurate activations) on the same sequence
+    y_u, S_u = _run(w, inp, S0, unfused=True)
+    check_parity(y_u, y_ref, (0, 2), TOL["bf16"], "muir unfused, long y", elem_tol=Y_ELEM_TOL)
+    check_parity(S_u, S_ref, (0, 1), TOL["bf16"], "muir unfused, long S_T", elem_tol=Y_ELEM_TOL)
