@@ -91,10 +91,12 @@ def fwd_flops(w) -> int:
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of the
-# current kernels on a quarter-size case, scaled by the units processed).  Forward: prep +
-# chain, per (b, h, 64-token chunk) of the GDN-2 bf16 d = 128 tensor-core path; decode: per
-# (b, h) step of the d = 128 persistent kernel.  Must be re-measured when those kernels change.
-FWD_TC_TRAFFIC_PER_CHUNK = (117.6e6 + 33.9e6 + 76.1e6 + 4.7e6) / 1024
+# current kernels on a half-size case, scaled by the units processed).  Forward: prep +
+# chain, per (b, h, 64-token chunk) of the GDN-2 bf16 d = 128 tensor-core path (B = 2, 2048
+# chunks: prep 235.0 MB read + 107.1 MB written, chain 152.1 MB read + 37.0 MB written);
+# decode: per (b, h) step of the d = 128 persistent kernel.  Must be re-measured when those
+# kernels change.
+FWD_TC_TRAFFIC_PER_CHUNK = (234995968 + 107078400 + 152093952 + 36988416) / 2048
 DEC_TRAFFIC_PER_HEAD = (137.9e6 + 81.0e6) / (64 * 32)
 
 
@@ -551,19 +553,19 @@ def bench_mlstm(ctx, args, gdr):
 
 def bench_gemm_phases(ctx, fwd):
     """The chunked forward's tensor-core phases, measured: the same kernels built with their
-    timing hooks (libgdr_timing.so) run the GDN-2 bf16 workload at B = 1; each MMA group is
+    timing hooks (libgdr_timing.so) run the timed forward workload; each MMA group is
     timed from the issue of its first MMA to its completion (the issuing warp waits for every
     group), and its bf16 FLOPs over those cycles, at the SM clock seen during the timed
     forward steps, are compared with the measured dense bf16 peak.  Per kernel (all its
     groups together) and per group."""
     try:
         from matrix_memory_rnn_b200 import phase_timing
-        m = phase_timing.measure(batch=1, calls=2)
+        m = phase_timing.measure(batch=fwd["w"].B, calls=2)
         clk = (fwd.get("clocks") or {}).get("sm_mhz") or 1965.0
         fr = phase_timing.gemm_phase_fractions(m, ctx.peaks["bf16_tflops"], clk)
-        return {"method": "timing build, B=1: MMA group issue-to-completion cycles, groups waited "
-                          "for one at a time; FLOPs of the groups over their cycles at the forward's "
-                          "SM clock, against the measured bf16 peak",
+        return {"method": "timing build, same workload: MMA group issue-to-completion cycles, groups "
+                          "waited for one at a time; FLOPs of the groups over their cycles at the "
+                          "forward's SM clock, against the measured bf16 peak",
                 "sm_mhz": clk, "peak_tflops": ctx.peaks["bf16_tflops"],
                 "kernels": {k: {"frac": v["frac"], "tflops": v["tflops"],
                                 "groups": [{kk: g[kk] for kk in ("group", "cycles", "frac")}

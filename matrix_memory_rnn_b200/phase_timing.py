@@ -104,6 +104,7 @@ def gemm_phase_fractions(m, peak_tflops, sm_mhz):
     same) and as a fraction of `peak_tflops`.  Also per group."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     out = {}
+    fl_all = cyc_all = 0.0
     for slot, name in ((1, "tc_prep_kernel"), (0, "tc_chain_kernel")):
         fl = cyc = 0.0
         groups = []
@@ -120,6 +121,11 @@ def gemm_phase_fractions(m, peak_tflops, sm_mhz):
         if cyc:
             tf = fl / cyc * sm_mhz * 1e6 * sms / 1e12
             out[name] = {"tflops": tf, "frac": tf / peak_tflops, "groups": groups}
+            fl_all += fl
+            cyc_all += cyc
+    if cyc_all:   # the forward call as a whole: every group of both kernels
+        tf = fl_all / cyc_all * sm_mhz * 1e6 * sms / 1e12
+        out["forward"] = {"tflops": tf, "frac": tf / peak_tflops, "groups": []}
     return out
 
 
