@@ -50,8 +50,9 @@
  * gdr_read_status() returns.  No function aborts, exits or traps.
  * For tests of that path, the environment variable GDR_DEBUG_FAULT=skip_handoff
  * makes the two-kernel tensor-core forward withhold a hand-off between its warp
- * groups, so a bounded wait runs out (about 2 s) and GDR_ERR_TIMEOUT is reported;
- * the context stays usable.
+ * groups (and the tcgen05 mLSTM kernel the completion signal of one product), so a
+ * bounded wait runs out (about 2 s) and GDR_ERR_TIMEOUT is reported; the context
+ * stays usable.
  */
 #ifndef GDR_H_
 #define GDR_H_
@@ -319,6 +320,7 @@ typedef struct {
   const float *C0, *n0, *m0;
   float *h;
   float *C_T, *n_T, *m_T;
+  uint32_t *status;  /* device word or NULL: GDR_ERR_TIMEOUT after a bounded wait ran out */
 } gdr_mlstm_args;
 
 /*
@@ -327,8 +329,12 @@ typedef struct {
  *   m_t = A_t + max(m, max_{s <= t} (i~_s - A_s)),
  *   h_t = (sum_{s<=t} w_ts (q_t.k_s) v_s + g_t C q_t) / max(|sum_{s<=t} w_ts (q_t.k_s) + g_t n.q_t|, e^{-m_t})
  * with w_ts = e^{A_t - A_s + i~_s - m_t} and g_t = e^{A_t + m - m_t}, all <= 1; the chunk's
- * products on the tensor cores (tf32, three products for fp32 inputs).  No workspace.
- * Errors as gdr_forward_chunked; GDR_ERR_UNSUPPORTED for dk or dv outside {64, 128}.
+ * products on the tensor cores: tcgen05 with TMEM accumulators for bf16 at dk = dv = 128,
+ * warp-level MMAs otherwise (tf32, three products for fp32 inputs).  No workspace.
+ * Errors as gdr_forward_chunked; GDR_ERR_UNSUPPORTED for dk or dv outside {64, 128}.  The
+ * tcgen05 kernel bounds its waits on the tensor cores and copies (about 2 s); one that runs
+ * out writes GDR_ERR_TIMEOUT to `status` when given (gdr_read_status reads and clears it)
+ * and leaves h and the final state undefined.
  */
 gdr_status gdr_mlstm_forward(const gdr_mlstm_args *args, void *stream);
 

@@ -34,6 +34,7 @@
 
 #include "gdr_phase_timing.cuh"
 #include "gdr_tc_common.cuh"
+#include "gdr_tma_host.cuh"
 
 // Phase hooks: filled by gdr_phase_timing.cuh in the timing build, empty in libgdr.so.
 #ifndef GDR_PREP_PHASE
@@ -1226,33 +1227,10 @@ size_t forward_tc_split_workspace_bytes(const FwdParams &p) {
 
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
-// [B][T][H][128] tensor of `elem` bytes as a 4-D map (channel, head, token, batch)
-// with a (box0, 1, C, 1) box.
+// [B][T][H][128] input as the prep kernel's 4-D map: boxes of `box0` channels x C tokens.
 bool encode_input_map(CUtensorMap *m, const void *base, CUtensorMapDataType type, int elem,
                       int box0, CUtensorMapSwizzle swizzle, const FwdParams &p) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
-  if (!enc) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)kDK, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
-  const cuuint64_t strides[3] = {(cuuint64_t)kDK * elem, (cuuint64_t)p.H * kDK * elem,
-                                 (cuuint64_t)p.T * p.H * kDK * elem};
-  const cuuint32_t box[4] = {(cuuint32_t)box0, 1, (cuuint32_t)kC, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return enc(m, type, 4, const_cast<void *>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return tma::encode_input_map(m, base, type, elem, box0, kC, swizzle, p.H, p.T, p.B);
 }
 
 }  // namespace

@@ -67,7 +67,8 @@ struct FwdParams {
 
 // Fault injection for the tests of the bounded waits (set through the environment
 // variable GDR_DEBUG_FAULT, read per call on the host): the prep kernel's front warp
-// group never hands its chunks to the back group, whose bounded wait then runs out.
+// group never hands its chunks to the back group, and the tcgen05 mLSTM kernel never
+// commits its [P~ V | P~ 1] product; in both a bounded wait then runs out.
 constexpr uint32_t kDebugSkipHandoff = 1u;
 // Timing build only (environment variable GDR_TIMING_MMA): the MMA-issuing warps wait for
 // each tensor-core group and time it.
@@ -109,8 +110,11 @@ cudaError_t launch_muir_epilogue(const MuirParams &m, gdr_dtype dtype, const flo
 cudaError_t launch_state_compose(float *S_out, const float *M, const float *S_in, const float *Q,
                                  int BH, int dk, int dv, cudaStream_t stream);
 
-// xLSTM's mLSTM cell (gdr_mlstm_forward); p[0 .. n) = x.
+// xLSTM's mLSTM cell (gdr_mlstm_forward); p[0 .. n) = x.  bf16 inputs with d_k = d_v = 128
+// take the tensor-core kernel, the rest the warp-MMA kernel.
 cudaError_t launch_mlstm(const gdr_mlstm_args &a, cudaStream_t stream);
+bool mlstm_tc_supported(const gdr_mlstm_args &a);
+cudaError_t launch_mlstm_tc(const gdr_mlstm_args &a, cudaStream_t stream);
 cudaError_t fill_f32(float *p, size_t n, float x, cudaStream_t stream);
 
 // Launchers (host).  Return cudaSuccess or the launch error.

@@ -361,6 +361,7 @@ cudaError_t fill_f32(float *p, size_t n, float x, cudaStream_t stream) {
 }
 
 cudaError_t launch_mlstm(const gdr_mlstm_args &a, cudaStream_t stream) {
+  if (mlstm_tc_supported(a)) return launch_mlstm_tc(a, stream);   // tcgen05 kernel (gdr_mlstm_tc.cu)
   if (a.dtype == GDR_BF16)
     return a.dk == 64 ? launch_typed<__nv_bfloat16, false, 64>(a, stream)
                       : launch_typed<__nv_bfloat16, false, 128>(a, stream);

@@ -93,6 +93,33 @@ __device__ __forceinline__ void tma_load_4d(void *dst_smem, const void *map, int
       : "memory");
 }
 
+// Tiled 4-D tensor store (TMA) of one box of shared memory to `map` at coordinates
+// (x, y, z, w), in the issuing thread's bulk group (bulk_commit / bulk_wait_*).  Elements
+// outside the tensor are not written.  Every coordinate must be >= 0, and x times the
+// element size a multiple of 16 bytes.  The writes to `src_smem` must be made visible to
+// the async proxy first (fence_proxy_async_smem, then a barrier if other threads wrote).
+__device__ __forceinline__ void tma_store_4d(const void *map, const void *src_smem, int x, int y,
+                                             int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+      ::"l"(map), "r"(smem_u32(src_smem)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+// Closes the issuing thread's current bulk group (its bulk stores since the last commit).
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until at most N of the issuing thread's bulk groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Waits until at most N of the issuing thread's bulk groups are incomplete.
+template <int N>
+__device__ __forceinline__ void bulk_wait() {
+  asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory");
+}
+
 // ---------------------------------------------------------------- cp.async (16 bytes)
 // Copies 16 bytes global -> shared; when `valid` is false it writes 16 zero bytes
 // and reads nothing (src-size 0).

@@ -63,7 +63,7 @@ class gdr_mlstm_args(ctypes.Structure):
     _fields_ = [("dtype", _c_int), ("B", _c_int), ("H", _c_int), ("T", _c_int), ("dk", _c_int),
                 ("dv", _c_int), ("q", _vp), ("k", _vp), ("v", _vp), ("f_pre", _fp), ("i_pre", _fp),
                 ("C0", _fp), ("n0", _fp), ("m0", _fp), ("h", _fp), ("C_T", _fp), ("n_T", _fp),
-                ("m_T", _fp)]
+                ("m_T", _fp), ("status", _vp)]
 
 
 class GdrError(RuntimeError):
@@ -391,10 +391,12 @@ def gdr_muir_forward(q, k, v, zf, zb, zw, zq, zg, a_log, gamma_stat=None, rms_we
 
 
 def gdr_mlstm_forward(q, k, v, f_pre, i_pre, C0=None, n0=None, m0=None, *, h=None,
-                      want_state=True, stream=None):
+                      want_state=True, status=None, stream=None):
     """xLSTM's mLSTM cell (include/gdr.h, gdr_mlstm_forward): q, k [B, T, H, dk], v
     [B, T, H, dv] (bf16 or fp32), gate pre-activations f_pre, i_pre [B, T, H] fp32, optional
-    stabilized state C0 [B, H, dk, dv], n0 [B, H, dk], m0 [B, H].  Returns (h, C_T, n_T, m_T)."""
+    stabilized state C0 [B, H, dk, dv], n0 [B, H, dk], m0 [B, H].  ``status``: optional
+    contiguous CUDA tensor whose first 4 bytes receive GDR_ERR_TIMEOUT if a bounded device
+    wait runs out (read with ``gdr_read_status``).  Returns (h, C_T, n_T, m_T)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dname, tdt = _dtype_of(q)
@@ -421,6 +423,9 @@ def gdr_mlstm_forward(q, k, v, f_pre, i_pre, C0=None, n0=None, m0=None, *, h=Non
     for name, t in (("q", q), ("k", k), ("v", v), ("f_pre", f_pre), ("i_pre", i_pre), ("C0", C0),
                     ("n0", n0), ("m0", m0), ("h", h), ("C_T", C_T), ("n_T", n_T), ("m_T", m_T)):
         setattr(a, name, _ptr(t))
+    if status is not None and _workspace(status).numel() * status.element_size() < 4:
+        raise ValueError("status must hold at least 4 bytes")
+    a.status = _ptr(status)
     _check("gdr_mlstm_forward", _load().gdr_mlstm_forward(ctypes.byref(a), _stream(stream)))
     return h, C_T, n_T, m_T
 

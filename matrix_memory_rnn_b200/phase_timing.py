@@ -129,6 +129,64 @@ def gemm_phase_fractions(m, peak_tflops, sm_mhz):
     return out
 
 
+# Marks of the mLSTM kernel: (index, label) for thread 0 (a P~ / h warp) and for thread 64
+# (a K~ warp, the one that also scans the next chunk's gates), in the order of the chunk
+# loop; marks 0, 1, 11 and 12 are shared.
+MLSTM_PHASES = {
+    "thread 0 (P~ and h warps)": [
+        (1, "wait for the chunk's tiles, barrier"), (2, "P~ weights (tensor cores on S)"),
+        (3, "wait for S"), (4, "S from TMEM, times the weights"),
+        (5, "P~ stored, fence, barrier"), (6, "[P~ V | P~ 1] issued; r, g, m"),
+        (7, "wait for [P~ V | P~ 1] and [Q C | Q n]"), (8, "h"),
+        (9, "wait for [K~^T V | K~^T 1]"), (10, "state update, rows 0..63"),
+        (11, "proxy fence"), (12, "barrier (chunk done)"), (0, "to the next chunk"),
+    ],
+    "thread 64 (K~ warps)": [
+        (1, "wait for the chunk's tiles, barrier"), (2, "K~ formed and stored"),
+        (3, "barrier (K~ done)"), (4, "[K~^T V | K~^T 1] issued"),
+        (5, "next chunk's gate scan"), (6, "wait for [Q C | Q n] and [K~^T V | K~^T 1]"),
+        (10, "state update, rows 64..127"), (11, "proxy fence"), (12, "barrier (chunk done)"),
+        (0, "to the next chunk"),
+    ],
+}
+
+
+def measure_mlstm(batch=4, calls=3):
+    """The mLSTM cell (bf16, d = 128: the tensor-core kernel) on the GDN-2 bf16 workload's shapes
+    through the timing build; returns, for thread 0 and thread 64, the cycles per chunk by
+    mark index."""
+    lib = ctypes.CDLL(build.build(timing=True))
+    lib.gdr_mlstm_forward.argtypes = [ctypes.POINTER(gdr.gdr_mlstm_args), ctypes.c_void_p]
+    lib.gdr_mlstm_forward.restype = ctypes.c_int
+    lib.gdr_mlstm_timing_read.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.gdr_mlstm_timing_read.restype = ctypes.c_int
+    w = synth.PRESETS["gdn2_bf16"].with_(B=batch)
+    inp = synth.mlstm_inputs(w)
+    d = {k: torch.from_numpy(inp[k]).to("cuda", torch.bfloat16) for k in ("q", "k", "v")}
+    g = {k: torch.from_numpy(inp[k]).cuda() for k in ("f_pre", "i_pre")}
+    h = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device="cuda")
+    a = gdr.gdr_mlstm_args()
+    a.dtype, a.B, a.H, a.T, a.dk, a.dv = gdr.DTYPES["bf16"], w.B, w.H, w.T, w.dk, w.dv
+    a.q, a.k, a.v = (ctypes.c_void_p(d[x].data_ptr()) for x in ("q", "k", "v"))
+    a.f_pre, a.i_pre = ctypes.c_void_p(g["f_pre"].data_ptr()), ctypes.c_void_p(g["i_pre"].data_ptr())
+    a.h = ctypes.c_void_p(h.data_ptr())
+    cycles = (ctypes.c_ulonglong * 32)()
+
+    def run(n):
+        for _ in range(n):
+            rc = lib.gdr_mlstm_forward(ctypes.byref(a), None)
+            if rc != 0:
+                raise RuntimeError(f"gdr_mlstm_forward (timing build) failed: {rc}")
+        rc = lib.gdr_mlstm_timing_read(cycles)
+        if rc != 0:
+            raise RuntimeError(f"gdr_mlstm_timing_read failed: CUDA error {rc}")
+
+    run(1)
+    run(calls)
+    chunks = w.B * w.H * (w.dv // 64) * ((w.T + 63) // 64) * calls
+    return [{i: cycles[16 * r + i] / chunks for i in range(16)} for r in range(2)]
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--batch", type=int, default=4, help="B of the GDN-2 bf16 workload (H=16, T=4096)")
@@ -137,7 +195,19 @@ def main(argv=None) -> int:
                     help="bf16 dense peak of the whole GPU (default: MEASURED_PEAKS.json's, else 1590)")
     ap.add_argument("--sm-mhz", type=float, default=1965.0,
                     help="SM clock of the run (the cycles are SM cycles)")
+    ap.add_argument("--mlstm", action="store_true",
+                    help="the mLSTM cell's tensor-core kernel instead of the forward")
     args = ap.parse_args(argv)
+
+    if args.mlstm:
+        per = measure_mlstm(args.batch, args.calls)
+        print(f"mlstm_tc_kernel, bf16, B={args.batch}, H=16, T=4096, d=128: cycles per chunk")
+        for r, (who, phases) in enumerate(MLSTM_PHASES.items()):
+            print(f"\n{who}")
+            for i, label in phases:
+                print(f"  {label:50s} {per[r][i]:9.0f}")
+            print(f"  {'sum':50s} {sum(per[r][i] for i, _ in phases):9.0f}")
+        return 0
 
     m = measure(args.batch, args.calls)
     w = m["w"]

@@ -116,3 +116,41 @@ def test_mlstm_full_size_sampled_heads(preset):
         hr, Cr, _, _ = oracle.mlstm_forward(sl["q"], sl["k"], sl["v"], sl["f_pre"], sl["i_pre"])
         check_parity(h[b:b + 1, :, hh:hh + 1], hr, (0, 2), TOL["bf16"], f"mlstm full size ({b},{hh}) h")
         check_parity(C[b:b + 1, hh:hh + 1], Cr, (0, 1), TOL["bf16"], f"mlstm full size ({b},{hh}) C")
+
+
+def _bf16_case(T=257, B=1, H=2):
+    w = small("gdn2", "bf16", dk=128, dv=128, T=T, B=B, H=H, chunk=64)
+    inp = synth.mlstm_inputs(w)
+    d = {k: torch.from_numpy(np.ascontiguousarray(inp[k])).to("cuda", torch.bfloat16) for k in ("q", "k", "v")}
+    g = {k: torch.from_numpy(np.ascontiguousarray(inp[k], np.float32)).cuda() for k in ("f_pre", "i_pre")}
+    return w, inp, d, g
+
+
+def test_mlstm_status_word_stays_ok_and_changes_nothing():
+    """The tensor-core kernel (bf16, d = 128) leaves a given status word at GDR_OK, and the
+    outputs are bit-identical with and without it."""
+    w, inp, d, g = _bf16_case()
+    status = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    h1, C1, n1, m1 = gdr.gdr_mlstm_forward(d["q"], d["k"], d["v"], g["f_pre"], g["i_pre"], status=status)
+    assert gdr.gdr_read_status(status) == "GDR_OK"
+    h0, C0, n0, m0 = gdr.gdr_mlstm_forward(d["q"], d["k"], d["v"], g["f_pre"], g["i_pre"])
+    torch.cuda.synchronize()
+    for x, y in ((h1, h0), (C1, C0), (n1, n0), (m1, m0)):
+        assert torch.equal(x, y)
+
+
+def test_mlstm_bounded_wait_reports_timeout_and_context_survives(monkeypatch):
+    """Fault injection on the host: the kernel withholds the commit of [P~ V | P~ 1], the
+    bounded wait for it runs out (about 2 s), GDR_ERR_TIMEOUT lands in the status word, and
+    the next call on the same context matches the oracle."""
+    w, inp, d, g = _bf16_case(T=130)
+    status = torch.zeros(4, dtype=torch.uint8, device="cuda")
+    monkeypatch.setenv("GDR_DEBUG_FAULT", "skip_handoff")
+    gdr.gdr_mlstm_forward(d["q"], d["k"], d["v"], g["f_pre"], g["i_pre"], status=status)
+    assert gdr.gdr_read_status(status) == "GDR_ERR_TIMEOUT"
+    monkeypatch.delenv("GDR_DEBUG_FAULT")
+    h, C, n, m = gdr.gdr_mlstm_forward(d["q"], d["k"], d["v"], g["f_pre"], g["i_pre"], status=status)
+    assert gdr.gdr_read_status(status) == "GDR_OK"
+    hr, Cr, nr, mr = oracle.mlstm_forward(inp["q"], inp["k"], inp["v"], inp["f_pre"], inp["i_pre"])
+    check_parity(h.cpu().numpy(), hr, (0, 2), TOL["bf16"], "mlstm after a timeout: h")
+    check_parity(C.cpu().numpy(), Cr, (0, 1), TOL["bf16"], "mlstm after a timeout: C")
