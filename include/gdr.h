@@ -50,9 +50,9 @@
  * gdr_read_status() returns.  No function aborts, exits or traps.
  * For tests of that path, the environment variable GDR_DEBUG_FAULT=skip_handoff
  * makes the two-kernel tensor-core forward withhold a hand-off between its warp
- * groups (and the tcgen05 mLSTM kernel the completion signal of one product), so a
- * bounded wait runs out (about 2 s) and GDR_ERR_TIMEOUT is reported; the context
- * stays usable.
+ * groups (the single-kernel forward and the tcgen05 mLSTM kernel the completion
+ * signal of one product), so a bounded wait runs out (about 2 s) and GDR_ERR_TIMEOUT
+ * is reported; the context stays usable.
  */
 #ifndef GDR_H_
 #define GDR_H_
@@ -183,12 +183,20 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *args, void *stream);
  *     Serialize them.
  *   - The array keeps the last call's contents; each call clears the status word
  *     it uses on `stream` before the launch.
- *   - The device status word lives in the library's array, so gdr_read_status
- *     cannot report this variant's device-side failures (a bounded wait that ran
- *     out leaves its outputs incomplete without a status).
+ *   - The device status word lives in the library's array: read it with
+ *     gdr_noalloc_read_status (below), not gdr_read_status.
  * Errors and all other arguments: as gdr_forward_chunked.
  */
 gdr_status gdr_forward_chunked_noalloc(const gdr_fwd_args *args, void *stream);
+
+/*
+ * The device status word of gdr_forward_chunked_noalloc on the current device: waits for
+ * `stream` (cudaStreamSynchronize), copies the word from the library's array to
+ * *device_status (GDR_OK, or GDR_ERR_TIMEOUT after a bounded wait of a kernel ran out)
+ * and clears it, as gdr_read_status does for a caller's workspace.  Allocates nothing.
+ * Returns GDR_ERR_INVALID_ARG for a NULL device_status, GDR_ERR_CUDA if a CUDA call fails.
+ */
+gdr_status gdr_noalloc_read_status(void *stream, gdr_status *device_status);
 
 /*
  * Arguments of gdr_backward_chunked: the forward's inputs plus the loss gradient.

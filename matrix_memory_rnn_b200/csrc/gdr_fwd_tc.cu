@@ -283,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
         const uint64_t bd = sdesc_sw128(sb + SL::B_LM + (s >> 2) * (kC * 128) + (s & 3) * 32, 16, 1024);
         mma_bf16(tLM, ad, bd, id, s > 0);
       }
-      mma_commit(mbar);
+      if (!(p.debug & kDebugSkipHandoff)) mma_commit(mbar);   // (withheld in the fault test)
     }
     if (!(ok = wait_mma(mbar, phase, sflag + 1))) break;
 
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_tc_gdn2_kernel(FwdParams p) {
     // in-flight group one more bounded wait, then release TMEM.
     if (tid == 0) {
       if (p.status) atomicExch(p.status, (uint32_t)GDR_ERR_TIMEOUT);
-      mbar_wait_bounded(mbar, phase, kWaitLimitNs);
+      mbar_wait_bounded(mbar, phase ^ 1u, kWaitLimitNs);   // wait_mma advanced `phase` past it
     }
   }
   tc_fence_before();

@@ -67,8 +67,9 @@ struct FwdParams {
 
 // Fault injection for the tests of the bounded waits (set through the environment
 // variable GDR_DEBUG_FAULT, read per call on the host): the prep kernel's front warp
-// group never hands its chunks to the back group, and the tcgen05 mLSTM kernel never
-// commits its [P~ V | P~ 1] product; in both a bounded wait then runs out.
+// group never hands its chunks to the back group, the single-kernel tensor-core forward
+// never commits its first product, and the tcgen05 mLSTM kernel never commits its
+// [P~ V | P~ 1] product; in each a bounded wait then runs out.
 constexpr uint32_t kDebugSkipHandoff = 1u;
 // Timing build only (environment variable GDR_TIMING_MMA): the MMA-issuing warps wait for
 // each tensor-core group and time it.

@@ -121,3 +121,11 @@ extern "C" gdr_status gdr_forward_chunked_noalloc(const gdr_fwd_args *args, void
   a.workspace_bytes = kNoAllocScratchBytes;
   return gdr_forward_chunked(&a, stream);
 }
+
+extern "C" gdr_status gdr_noalloc_read_status(void *stream, gdr_status *device_status) {
+  if (!device_status) return GDR_ERR_INVALID_ARG;
+  void *scratch = nullptr;
+  const gdr_status st = scratch_for_current_device(&scratch);
+  if (st != GDR_OK) return st;
+  return gdr_read_status(scratch, stream, device_status);
+}

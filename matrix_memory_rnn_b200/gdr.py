@@ -529,3 +529,15 @@ def gdr_forward_chunked_noalloc(form, q, k, v, log_w, e1=None, e2=None, S0=None,
     a = _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, None)
     _check("gdr_forward_chunked_noalloc", fn(ctypes.byref(a), _stream(stream)))
     return o, S_T
+
+
+def gdr_noalloc_read_status(*, stream=None):
+    """Synchronizes ``stream`` and returns (and clears) the device status word of
+    ``gdr_forward_chunked_noalloc`` on the current device."""
+    lib = _load()
+    fn = lib.gdr_noalloc_read_status
+    fn.argtypes = [_vp, ctypes.POINTER(_c_int)]
+    fn.restype = _c_int
+    st = ctypes.c_int(0)
+    _check("gdr_noalloc_read_status", fn(_stream(stream), ctypes.byref(st)))
+    return STATUS.get(st.value, st.value)

@@ -85,3 +85,24 @@ def test_noalloc_refuses_what_needs_records():
     torch.cuda.synchronize()
     assert rc == GDR_ERR_WORKSPACE
     assert torch.isnan(o).all() and torch.isnan(S_T).all()
+
+
+def test_noalloc_reports_a_timeout_through_its_status_reader(monkeypatch):
+    """Fault injection on the host: the single-kernel forward withholds the commit of its
+    first product, its bounded wait runs out, and gdr_noalloc_read_status returns
+    GDR_ERR_TIMEOUT from the library's array (then GDR_OK: it clears the word).  The next
+    call on the same context matches the oracle."""
+    w, inp, args = _case("gdn2", 128)
+    o = torch.empty((w.B, w.T, w.H, w.dv), device="cuda")
+    S_T = torch.empty((w.B, w.H, w.dk, w.dv), device="cuda")
+    assert gdr.gdr_noalloc_read_status() == "GDR_OK"
+    monkeypatch.setenv("GDR_DEBUG_FAULT", "skip_handoff")
+    gdr.gdr_forward_chunked_noalloc(*args, algo="tc", o=o, S_T=S_T)
+    assert gdr.gdr_noalloc_read_status() == "GDR_ERR_TIMEOUT"
+    assert gdr.gdr_noalloc_read_status() == "GDR_OK"
+    monkeypatch.delenv("GDR_DEBUG_FAULT")
+    gdr.gdr_forward_chunked_noalloc(*args, algo="tc", o=o, S_T=S_T)
+    assert gdr.gdr_noalloc_read_status() == "GDR_OK"
+    o_or, S_or = oracle_forward(w, inp)
+    assert head_rel_err(o.cpu().numpy(), o_or, (0, 2)) < TOL["bf16"]
+    assert head_rel_err(S_T.cpu().numpy(), S_or, (0, 1)) < TOL["bf16"]
