@@ -22,12 +22,13 @@
 // One CTA of 256 threads per (b, h, 64 value columns), two warp groups working side by side
 // on a chunk:
 //   P~ / h warps (0, 1, 4, 5: TMEM lanes 0..63, i.e. the chunk's tokens): the weights w~
-//     while the tensor cores form S, then P~, [P~ V | P~ 1] (issued by warp 1, which also
-//     issues S and [Q C | Q n] at the chunk's start), h (staged in shared memory, written by
-//     TMA stores), and the state update of key channels 0..63;
-//   K~ warps (2, 3, 6, 7): K~, [K~^T V | K~^T 1] (issued by warp 2), the next chunk's gate
-//     scan (warp 2: A, mloc and i~ - A, which do not depend on the carried m), and the state
-//     update of key channels 64..127.
+//     while the tensor cores form S, then P~, [P~ V | P~ 1] (issued by warp 1), h (staged in
+//     shared memory, written by TMA stores), and the state update of key channels 0..63;
+//   K~ warps (2, 3, 6, 7): S and [Q C | Q n] (issued by warp 3 at the chunk's start), the
+//     next chunk's tile loads (warp 6), diag(f) [V | 1] and K^T diag(f) [V | 1] =
+//     [K~^T V | K~^T 1] (issued by warp 2), the next chunk's gates and their scan (warp 7:
+//     A, mloc and i~ - A, which do not depend on the carried m), and the state update of key
+//     channels 64..127.
 // Every thread carries m and forms its own r_t, g_t, g_L, r_L from the scanned arrays.  The
 // next chunk's q, k and value slice arrive by TMA (128-byte swizzle, straight into the MMA
 // tiles) and its gates by 4-byte cp.async while the current chunk is computed.  Every wait is
@@ -40,7 +41,8 @@
 #include "gdr_tc_common.cuh"
 #include "gdr_tma_host.cuh"
 
-// Phase marks of the timing build: thread 0 (a P~ / h warp) and thread 64 (a K~ warp) sum
+// Phase marks of the timing build: thread 0 (a P~ / h warp) and thread 224 (the K~ warp that
+// scans the gates) sum
 // the cycles between consecutive marks, over CTAs and chunks, into [2][16]; empty in
 // libgdr.so.
 #ifdef GDR_PHASE_TIMING
@@ -52,16 +54,16 @@ __device__ unsigned long long g_mlstm_cycles[2][16];
   long long mt_l_ = 0;
 #define MT_MARK(i)                                                                  \
   do {                                                                              \
-    if (threadIdx.x == 0 || threadIdx.x == 64) {                                    \
+    if (threadIdx.x == 0 || threadIdx.x == 224) {                                   \
       const long long n_ = clock64();                                               \
       if (mt_l_) mt_a_[i] += n_ - mt_l_;                                            \
       mt_l_ = n_;                                                                   \
     }                                                                               \
   } while (0)
 #define MT_FINI                                                                     \
-  if (threadIdx.x == 0 || threadIdx.x == 64)                                        \
+  if (threadIdx.x == 0 || threadIdx.x == 224)                                       \
     for (int i_ = 0; i_ < 16; ++i_)                                                 \
-      atomicAdd(&gdr::g_mlstm_cycles[threadIdx.x == 64][i_], (unsigned long long)mt_a_[i_]);
+      atomicAdd(&gdr::g_mlstm_cycles[threadIdx.x == 224][i_], (unsigned long long)mt_a_[i_]);
 #else
 #define MT_INIT
 #define MT_MARK(i)
@@ -81,7 +83,8 @@ constexpr int kMThreads = 256;
 // slice V (64 tokens x 64 columns, sw128) followed by the constant "ones" block (column 0
 // = 1, the rest 0) so that [V | 1] is one MN-major operand of 128 columns, and the raw
 // gates.  Then P~ (64 x 64, K-major A operand, with 8 KB of padding as the unused rows
-// 64..127), K~ (64 tokens x 128 channels, the MN-major A operand of K~^T), [C | n] (bf16, 128
+// 64..127), diag(f) [V | 1] (64 tokens x (64 + 64), the B operand of K^T diag(f) [V | 1]; column 0
+// of its second block holds f, the rest of that block stays 0), [C | n] (bf16, 128
 // key channels x (64 + 64): C's block then a block whose column 0 holds n), the scan's
 // per-token arrays and the barriers.
 struct MSmem {
@@ -91,13 +94,13 @@ struct MSmem {
   static constexpr uint32_t GATES = ONES + 64 * 128;          // f~[64], i~[64] fp32
   static constexpr uint32_t BUF = GATES + 1024;
   static constexpr uint32_t PT = 2 * BUF;                     // P~ (8 KB) + 8 KB padding
-  static constexpr uint32_t KT = PT + 16384;                  // K~, two blocks of 8 KB
-  static constexpr uint32_t CB = KT + 16384;                  // [C | n]: two blocks of 16 KB
+  static constexpr uint32_t VS = PT + 16384;                  // diag(f) [V | 1]: two blocks of 8 KB
+  static constexpr uint32_t CB = VS + 16384;                  // [C | n]: two blocks of 16 KB
   static constexpr uint32_t HST = CB + 32768;                 // h staging: [2][4 warps] 4 KB
   static constexpr uint32_t ARR = HST + 32768;                // fp32 A, mloc, D [64], two chunks
   static constexpr uint32_t MISC = ARR + 6 * 256;
   static constexpr uint32_t ALLOC = MISC + 128 + 1024;
-  static_assert(BUF % 1024 == 0 && PT % 1024 == 0 && KT % 1024 == 0 && CB % 1024 == 0 &&
+  static_assert(BUF % 1024 == 0 && PT % 1024 == 0 && VS % 1024 == 0 && CB % 1024 == 0 &&
                     HST % 1024 == 0,
                 "MMA tiles and swizzled TMA boxes 1024-aligned");
   static_assert(ALLOC <= 227 * 1024, "shared memory");
@@ -113,6 +116,13 @@ struct MMaps {
 };
 // TMEM columns: S 64, [Q C | Q n] 80, [P~ V | P~ 1] 80, [K~^T V | K~^T 1] 80.
 constexpr uint32_t kColS = 0, kColQC = 64, kColH = 160, kColDS = 256, kMTmemCols = 512;
+
+// 2^x by the PTX instruction ex2.approx.ftz.f32 (relative error about 2^-22; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ float log_sigmoid_f(float x) {
   return x >= 0.f ? -log1pf(expf(-x)) : x - log1pf(expf(x));
@@ -222,7 +232,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
     tmem_alloc(tmem_slot, kMTmemCols);
     tmem_relinquish();
   }
-  if (tid == 0) {
+  if (tid == 192) {   // the thread that arms `full` for the first tile loads below
     mbar_init(bar1, 1);
     mbar_init(bar2, 1);
     mbar_init(bar3, 1);
@@ -242,6 +252,8 @@ __global__ void __launch_bounds__(kMThreads, 1)
     *reinterpret_cast<uint4 *>(smem + MSmem::PT + 8192 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
   for (int i = tid; i < 16384 / 16; i += kMThreads)
     *reinterpret_cast<uint4 *>(smem + MSmem::CB + 16384 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
+  for (int i = tid; i < 8192 / 16; i += kMThreads)   // diag(f) 1: only column 0 changes per chunk
+    *reinterpret_cast<uint4 *>(smem + MSmem::VS + 8192 + i * 16) = make_uint4(0u, 0u, 0u, 0u);
 
   // fp32 state: key channel jrow, value columns [hf*32, hf*32 + 32) of the slice; n_j on hf 0.
   // Every thread carries m (mc) itself: the same arithmetic on the same values everywhere.
@@ -269,14 +281,15 @@ __global__ void __launch_bounds__(kMThreads, 1)
   store_state_bf16();
   fence_proxy_async_smem();   // the constant blocks and [C | n] are read by the tensor cores
 
-  // Thread 0 requests the tiles and counts the chunks whose tiles it requested and saw
-  // land; warp 2 loads the gates (one cp.async group per chunk) and scans them a chunk ahead.
+  // Thread 192 (warp 6, a K~ warp) requests the tiles and counts the chunks whose tiles it
+  // requested and saw land; warp 7 loads the gates (one cp.async group per chunk) and scans
+  // them a chunk ahead.
   int loads_issued = 0, loads_seen = 0;
-  if (tid == 0) {
+  if (tid == 192) {
     load_tiles(smem, maps, full, b, h, c0, 0);
     loads_issued = 1;
   }
-  if (warp == 2) {
+  if (warp == 7) {
     load_gates(smem, a, b, h, 0);
     cp_async_wait<0>();
     __syncwarp();
@@ -320,8 +333,8 @@ __global__ void __launch_bounds__(kMThreads, 1)
     const uint32_t par = (uint32_t)(c & 1);   // each MMA barrier completes once per chunk
     const float *arr = arr0 + 192 * bi;       // this chunk's A, mloc, D (scanned a chunk ahead)
     MT_MARK(0);
-    // ---- chunk c's tiles have landed (thread 0 polls, bounded); its gates are scanned
-    if (tid == 0) {
+    // ---- chunk c's tiles have landed (thread 192 polls, bounded); its gates are scanned
+    if (tid == 192) {
       if (mbar_wait_bounded(full + bi, (uint32_t)((c >> 1) & 1), kWaitLimitNs)) ++loads_seen;
       else fail = true;
     }
@@ -330,8 +343,8 @@ __global__ void __launch_bounds__(kMThreads, 1)
       break;
     }
     MT_MARK(1);
-    // ---- MMA group 1 (warp 1): S = [Q; K] K^T, then [Q C | Q n] = [Q; K] [C | n]
-    if (warp == 1) {
+    // ---- MMA group 1 (warp 3): S = [Q; K] K^T, then [Q C | Q n] = [Q; K] [C | n]
+    if (warp == 3) {
       tc_fence_after();
       constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);
       constexpr uint32_t id_qc = idesc_bf16_f32(128, 80, false, true);
@@ -352,21 +365,27 @@ __global__ void __launch_bounds__(kMThreads, 1)
     }
     // ---- the next chunk's loads, into the other buffer (chunk c - 1 is done with it)
     if (c + 1 < nch) {
-      if (tid == 0) {
+      if (tid == 192) {
         load_tiles(smem + (bi ^ 1) * MSmem::BUF, maps, full + (bi ^ 1), b, h, c0, t0 + 64);
         ++loads_issued;
       }
-      if (warp == 2) load_gates(smem + (bi ^ 1) * MSmem::BUF, a, b, h, t0 + 64);
+      if (warp == 7) load_gates(smem + (bi ^ 1) * MSmem::BUF, a, b, h, t0 + 64);
     }
     if (pw) {
       // ---- P~ = S (.) w~ for row t = 32 qd + lane, columns [32 hf, 32 hf + 32), with
       //      w~_ts = e^{(A_t - mloc_t) + D_s} for s <= t.  The weights are formed while the
       //      tensor cores compute S; the warp reads D_s as 16-byte broadcasts (32 scalar reads
       //      per thread, or 32 shuffles, were measured several times slower).
+      //      Warp 4 (tokens 0..31, keys 32..63) lies wholly above the diagonal: zeros.
       const int t = 32 * qd + lane;
+      const bool upper = qd == 0 && hf == 1;   // warp-uniform
       float w[32];
-      {
-        const float rowv = arr[t] - arr[64 + t];
+      if (upper) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) w[i] = 0.f;
+      } else {
+        constexpr float kLog2e = 1.4426950408889634f;
+        const float rowv2 = (arr[t] - arr[64 + t]) * kLog2e;
         const float4 *dcol = reinterpret_cast<const float4 *>(arr + 128 + hf * 32);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -375,7 +394,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int i = 4 * j + e;
-            w[i] = hf * 32 + i <= t ? __expf(rowv + dd[e]) : 0.f;
+            w[i] = hf * 32 + i <= t ? ex2_approx(fmaf(dd[e], kLog2e, rowv2)) : 0.f;
           }
         }
       }
@@ -384,7 +403,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
       __syncwarp();   // the warp-wide tcgen05.ld below wants the warp converged
       tc_fence_after();
       MT_MARK(3);
-      {
+      if (!upper) {
         float x[32];
         tmem_ld_32x32b_x32(tmem + kColS + lane_q + hf * 32, x);
         tmem_ld_wait();
@@ -457,41 +476,46 @@ __global__ void __launch_bounds__(kMThreads, 1)
       update_state(arr);
       MT_MARK(10);
     } else {
-      // ---- K~_s = k_s e^{A_L - mloc_L + D_s} (token s, channel half `half`)
+      // ---- diag(f) [V | 1] with f_s = e^{A_L - mloc_L + D_s} (token s, 32 value columns), so
+      //      that K~^T [V | 1] = K^T (diag(f) [V | 1]) reads K in place from the [Q; K] tile
       const int u = ((warp & 1) << 5) + ((warp >> 2) << 6) + lane;   // 0..127 over warps 2, 3, 6, 7
-      const int s = u & 63, half = u >> 6;
+      const int s = u & 63, ch = u >> 6;
       const float f = __expf(arr[63] - arr[64 + 63] + arr[128 + s]);
 #pragma unroll
-      for (int i = 0; i < 64; i += 8) {
-        float k8[8];
-        unpack8(*reinterpret_cast<const uint4 *>(buf + MSmem::QK + sw128_offset(64 + s, half * 64 + i, 16384)), k8);
+      for (int i = 0; i < 32; i += 8) {
+        float v8[8];
+        unpack8(*reinterpret_cast<const uint4 *>(buf + MSmem::V + sw128_offset(s, ch * 32 + i, 8192)), v8);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) k8[e] *= f;
-        st_smem16(smem, MSmem::KT + sw128_offset(s, half * 64 + i, 8192), pack8(k8));
+        for (int e = 0; e < 8; ++e) v8[e] *= f;
+        st_smem16(smem, MSmem::VS + sw128_offset(s, ch * 32 + i, 8192), pack8(v8));
       }
+      if (ch == 0)
+        *reinterpret_cast<__nv_bfloat16 *>(smem + MSmem::VS + sw128_offset(s, 64, 8192)) = __float2bfloat16_rn(f);
       fence_proxy_async_smem();
       MT_MARK(2);
       KSync::sync();
       MT_MARK(3);
-      // ---- MMA 2b (warp 2): [K~^T V | K~^T 1] = K~^T [V | 1]
+      // ---- MMA 2b (warp 2): [K~^T V | K~^T 1] = K^T (diag(f) [V | 1]); K^T is the MN-major
+      //      view of the k rows of the [Q; K] tile (its two 64-channel blocks 16 KB apart)
       if (warp == 2) {
         tc_fence_after();
         constexpr uint32_t id_ds = idesc_bf16_f32(128, 80, true, true);
 #pragma unroll
         for (int s4 = 0; s4 < 4; ++s4) {
-          const uint64_t ak = sdesc_sw128(sb + MSmem::KT + s4 * 2048, 8192, 1024);
-          const uint64_t bv = sdesc_sw128(bb + MSmem::V + s4 * 2048, 8192, 1024);
+          const uint64_t ak = sdesc_sw128(bb + MSmem::QK + 64 * 128 + s4 * 2048, 16384, 1024);
+          const uint64_t bv = sdesc_sw128(sb + MSmem::VS + s4 * 2048, 8192, 1024);
           mma_bf16_warp(tmem + kColDS, ak, bv, id_ds, s4 > 0);
         }
         mma_commit_warp(bar3);
-        MT_MARK(4);
-        // ---- the next chunk's carry-free scan (its gates were requested at the chunk's start)
-        if (c + 1 < nch) {
-          cp_async_wait<0>();
-          __syncwarp();
-          scan_gates(reinterpret_cast<const float *>(smem + (bi ^ 1) * MSmem::BUF + MSmem::GATES),
-                     min(64, T - t0 - 64), arr0 + 192 * (bi ^ 1));
-        }
+      }
+      MT_MARK(4);
+      // ---- the next chunk's carry-free scan (warp 7; its gates were requested at the
+      //      chunk's start)
+      if (warp == 7 && c + 1 < nch) {
+        cp_async_wait<0>();
+        __syncwarp();
+        scan_gates(reinterpret_cast<const float *>(smem + (bi ^ 1) * MSmem::BUF + MSmem::GATES),
+                   min(64, T - t0 - 64), arr0 + 192 * (bi ^ 1));
       }
       MT_MARK(5);
       // ---- the state update of key channels 64..127, once [Q C | Q n] has read [C | n]
@@ -528,7 +552,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
       if (a.n_T && hf == 0) a.n_T[bh * 128 + jrow] = nj;
       if (a.m_T && tid == 0) a.m_T[bh] = mc;
     }
-  } else if (tid == 0) {
+  } else if (tid == 192) {   // the issuing thread of the tile loads
     if (a.status) *reinterpret_cast<volatile uint32_t *>(a.status) = (uint32_t)GDR_ERR_TIMEOUT;
     // let what is still in flight land before the CTA exits: the last chunk's MMA groups
     // and the tile loads requested but not seen (each buffer's loads land in order)
@@ -559,7 +583,7 @@ bool mlstm_tc_supported(const gdr_mlstm_args &a) {
 
 #ifdef GDR_PHASE_TIMING
 // Timing build only: copies the mLSTM kernel's per-phase cycle sums ([2][16]: thread 0's,
-// then thread 64's) to host memory, then clears them.  Returns 0 or a CUDA error.
+// then thread 224's) to host memory, then clears them.  Returns 0 or a CUDA error.
 extern "C" int gdr_mlstm_timing_read(unsigned long long *cycles) {
   cudaError_t e = cudaDeviceSynchronize();
   if (e == cudaSuccess) e = cudaMemcpyFromSymbol(cycles, g_mlstm_cycles, sizeof(g_mlstm_cycles));

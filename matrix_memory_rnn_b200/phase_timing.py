@@ -129,7 +129,7 @@ def gemm_phase_fractions(m, peak_tflops, sm_mhz):
     return out
 
 
-# Marks of the mLSTM kernel: (index, label) for thread 0 (a P~ / h warp) and for thread 64
+# Marks of the mLSTM kernel: (index, label) for thread 0 (a P~ / h warp) and for thread 224
 # (a K~ warp, the one that also scans the next chunk's gates), in the order of the chunk
 # loop; marks 0, 1, 11 and 12 are shared.
 MLSTM_PHASES = {
@@ -141,9 +141,9 @@ MLSTM_PHASES = {
         (9, "wait for [K~^T V | K~^T 1]"), (10, "state update, rows 0..63"),
         (11, "proxy fence"), (12, "barrier (chunk done)"), (0, "to the next chunk"),
     ],
-    "thread 64 (K~ warps)": [
-        (1, "wait for the chunk's tiles, barrier"), (2, "K~ formed and stored"),
-        (3, "barrier (K~ done)"), (4, "[K~^T V | K~^T 1] issued"),
+    "thread 224 (K~ warps; warp 7 scans the next chunk's gates)": [
+        (1, "wait for the chunk's tiles, barrier"), (2, "diag(f) [V | 1] formed and stored"),
+        (3, "barrier (diag(f) [V | 1] done)"), (4, "(warp 2 issues [K~^T V | K~^T 1])"),
         (5, "next chunk's gate scan"), (6, "wait for [Q C | Q n] and [K~^T V | K~^T 1]"),
         (10, "state update, rows 64..127"), (11, "proxy fence"), (12, "barrier (chunk done)"),
         (0, "to the next chunk"),
@@ -153,7 +153,7 @@ MLSTM_PHASES = {
 
 def measure_mlstm(batch=4, calls=3):
     """The mLSTM cell (bf16, d = 128: the tensor-core kernel) on the GDN-2 bf16 workload's shapes
-    through the timing build; returns, for thread 0 and thread 64, the cycles per chunk by
+    through the timing build; returns, for thread 0 and thread 224, the cycles per chunk by
     mark index."""
     lib = ctypes.CDLL(build.build(timing=True))
     lib.gdr_mlstm_forward.argtypes = [ctypes.POINTER(gdr.gdr_mlstm_args), ctypes.c_void_p]
