@@ -48,7 +48,7 @@
 #define GDR_PHASE_FINI(slot)
 #endif
 #ifndef GDR_MMA_DECL
-#define GDR_MMA_DECL
+#define GDR_MMA_DECL(slot)
 #define GDR_MMA_BEGIN()
 #define GDR_MMA_END(g, tbar)
 #define GDR_MMA_FINI(slot)
@@ -314,7 +314,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
   auto bh_of = [&](int it) { return W.chunk_major ? it % W.BH : it / nch; };
   auto rec_of = [&](int it) { return records + (size_t)(bh_of(it) * nch + c_of(it)) * Rec::BYTES; };
   uint64_t *tbar = reinterpret_cast<uint64_t *>(misc + PrepMisc::TBAR);
-  GDR_MMA_DECL
+  GDR_MMA_DECL(1)
   (void)tbar;
 
   if (warp == 0) {
@@ -1019,7 +1019,7 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
   const uint32_t lane_q = (uint32_t)(32 * qd) << 16;
 
   uint64_t *tbar = reinterpret_cast<uint64_t *>(misc + ChainMisc::TBAR);
-  GDR_MMA_DECL
+  GDR_MMA_DECL(0)
   (void)tbar;
   // Warp 0 (all lanes): wait for record c, then MMA3 of chunk c into D[c & 1].  Returns
   // false (and issues nothing) if the record did not arrive in time.
@@ -1310,6 +1310,20 @@ extern "C" int gdr_phase_timing_read(unsigned long long *cycles, unsigned long l
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_phase_threads, zt, sizeof(zt));
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_mma_cycles, zm, sizeof(zm));
   if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_mma_groups, zm, sizeof(zm));
+  return (int)e;
+}
+
+// Timing build only: copies the MMA-group interval log (g_mma_log [2][256][256][2],
+// g_mma_log_group [2][256][256], g_mma_log_n [2][256]) to host memory and clears the counts.
+// Returns 0 or a CUDA error.
+extern "C" int gdr_phase_timing_read_log(unsigned long long *intervals, unsigned int *groups,
+                                         unsigned int *counts) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(intervals, gdr::g_mma_log, sizeof(gdr::g_mma_log));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(groups, gdr::g_mma_log_group, sizeof(gdr::g_mma_log_group));
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(counts, gdr::g_mma_log_n, sizeof(gdr::g_mma_log_n));
+  static const unsigned int zn[2][gdr::kMmaLogCtas] = {};
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_mma_log_n, zn, sizeof(zn));
   return (int)e;
 }
 #endif

@@ -19,19 +19,29 @@ __device__ unsigned long long g_phase_threads[2];
 // group's first MMA to the arrival of its completion, and the number of groups timed.
 __device__ unsigned long long g_mma_cycles[2][8];
 __device__ unsigned long long g_mma_groups[2][8];
+// The same groups as intervals, per kernel and CTA (linear block index): [start, end] in the
+// SM's clock64 and the group, for the first kMmaLogEntries groups of the first kMmaLogCtas
+// CTAs; so that the host can take the union of the intervals in which a CTA had a group in
+// flight (the prep kernel's two warp groups overlap theirs).
+constexpr int kMmaLogCtas = 256, kMmaLogEntries = 256;
+__device__ unsigned long long g_mma_log[2][kMmaLogCtas][kMmaLogEntries][2];
+__device__ unsigned int g_mma_log_group[2][kMmaLogCtas][kMmaLogEntries];
+__device__ unsigned int g_mma_log_n[2][kMmaLogCtas];
 }  // namespace gdr
 
-// MMA-group timing, in the issuing warp: GDR_MMA_BEGIN before a group's first MMA;
+// MMA-group timing, in the issuing warp (GDR_MMA_DECL(slot): 0 the chain, 1 prep):
+// GDR_MMA_BEGIN before a group's first MMA;
 // GDR_MMA_END(g, tbar) after its commit commits once more to the timing-only mbarrier
 // `tbar`, waits for it (bounded), and adds the elapsed cycles to group g.  The issuing
 // warp thus waits for each group before issuing the next, so the measured interval is
 // the group's own issue, execution and completion, not time queued behind other groups
 // of the same warp.
-#define GDR_MMA_DECL                                       \
+#define GDR_MMA_DECL(slot)                                 \
   long long gdr_mc_[8] = {0};                              \
   unsigned gdr_mn_[8] = {0};                               \
   uint32_t gdr_mp_ = 0;                                    \
-  long long gdr_mb_ = 0;
+  long long gdr_mb_ = 0;                                   \
+  const int gdr_ms_ = (slot);
 #define GDR_MMA_BEGIN() gdr_mb_ = clock64();
 // (only when the call asked for it: the waits change the kernel's schedule, so the phase
 // accounting above is taken in a separate pass without them)
@@ -42,8 +52,18 @@ __device__ unsigned long long g_mma_groups[2][8];
       if ((threadIdx.x & 31) == 0) mbar_wait_bounded(tbar, gdr_mp_ & 1u, 1000000000ull); \
       __syncwarp();                                                            \
       ++gdr_mp_;                                                               \
-      gdr_mc_[g] += clock64() - gdr_mb_;                                       \
+      const long long gdr_me_ = clock64();                                     \
+      gdr_mc_[g] += gdr_me_ - gdr_mb_;                                         \
       ++gdr_mn_[g];                                                            \
+      const unsigned gdr_cta_ = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z); \
+      if ((threadIdx.x & 31) == 0 && gdr_cta_ < (unsigned)gdr::kMmaLogCtas) {   \
+        const unsigned k_ = atomicAdd(&gdr::g_mma_log_n[gdr_ms_][gdr_cta_], 1u); \
+        if (k_ < (unsigned)gdr::kMmaLogEntries) {                              \
+          gdr::g_mma_log[gdr_ms_][gdr_cta_][k_][0] = (unsigned long long)gdr_mb_; \
+          gdr::g_mma_log[gdr_ms_][gdr_cta_][k_][1] = (unsigned long long)gdr_me_; \
+          gdr::g_mma_log_group[gdr_ms_][gdr_cta_][k_] = (unsigned)(g);          \
+        }                                                                      \
+      }                                                                        \
     }                                                                          \
   } while (0)
 #define GDR_MMA_FINI(slot)                                                      \

@@ -51,7 +51,49 @@ def load_timing_library():
     u64p = ctypes.POINTER(ctypes.c_ulonglong)
     lib.gdr_phase_timing_read.argtypes = [u64p, u64p, u64p, u64p]
     lib.gdr_phase_timing_read.restype = ctypes.c_int
+    lib.gdr_phase_timing_read_log.argtypes = [u64p, ctypes.POINTER(ctypes.c_uint), ctypes.POINTER(ctypes.c_uint)]
+    lib.gdr_phase_timing_read_log.restype = ctypes.c_int
     return lib
+
+
+LOG_CTAS, LOG_ENTRIES = 256, 256   # the timing build's interval log (gdr_phase_timing.cuh)
+
+
+def read_union(lib, flops_of):
+    """Reads (and clears) the timing build's MMA interval log and returns, per kernel slot,
+    [bf16 FLOPs of the logged groups, the summed per-CTA union of their [start, end]
+    intervals in SM cycles, groups logged, groups dropped].  The union counts the cycles in
+    which a CTA had at least one group in flight once, however many groups overlapped."""
+    iv = (ctypes.c_ulonglong * (2 * LOG_CTAS * LOG_ENTRIES * 2))()
+    gr = (ctypes.c_uint * (2 * LOG_CTAS * LOG_ENTRIES))()
+    cn = (ctypes.c_uint * (2 * LOG_CTAS))()
+    rc = lib.gdr_phase_timing_read_log(iv, gr, cn)
+    if rc != 0:
+        raise RuntimeError(f"gdr_phase_timing_read_log failed: CUDA error {rc}")
+    out = {}
+    for slot in (0, 1):
+        fl = cyc = 0.0
+        logged = dropped = 0
+        for cta in range(LOG_CTAS):
+            n = cn[slot * LOG_CTAS + cta]
+            if not n:
+                continue
+            k = min(n, LOG_ENTRIES)
+            dropped += n - k
+            logged += k
+            base = (slot * LOG_CTAS + cta) * LOG_ENTRIES
+            spans = sorted((iv[2 * (base + j)], iv[2 * (base + j) + 1]) for j in range(k))
+            fl += sum(flops_of[(slot, gr[base + j])] for j in range(k))
+            lo, hi = spans[0]
+            for a, b in spans[1:]:
+                if a > hi:
+                    cyc += hi - lo
+                    lo, hi = a, b
+                else:
+                    hi = max(hi, b)
+            cyc += hi - lo
+        out[slot] = [fl, cyc, logged, dropped]
+    return out
 
 
 def measure(batch=1, calls=3, lib=None):
@@ -87,10 +129,17 @@ def measure(batch=1, calls=3, lib=None):
     run(calls)        # phases, with the kernels' own schedule
     out = {"w": w, "calls": calls, "threads": list(threads), "cycles": list(cycles)}
     os.environ["GDR_TIMING_MMA"] = "1"
+    flops_of = {(s_, g): fl for s_, g, _, _, fl in MMA_GROUPS}
+    union = {0: [0.0, 0.0, 0, 0], 1: [0.0, 0.0, 0, 0]}
     try:
-        run(calls)    # tensor-core groups, each waited for by its issuing warp
+        read_union(lib, flops_of)     # clear what earlier runs left in the log
+        for _ in range(calls):        # tensor-core groups, each waited for by its issuing warp
+            run(1)
+            for slot, v in read_union(lib, flops_of).items():
+                union[slot] = [x + y for x, y in zip(union[slot], v)]
     finally:
         os.environ.pop("GDR_TIMING_MMA", None)
+    out["union"] = union
     nch = (w.T + 63) // 64
     out.update({"prep_chunks": w.B * w.H * nch * calls,    # each recorder sees every chunk
                 "chain_chunks": w.B * w.H * (w.dv // 64) * nch * calls,
@@ -101,10 +150,12 @@ def measure(batch=1, calls=3, lib=None):
 def gemm_phase_fractions(m, peak_tflops, sm_mhz):
     """Per kernel: bf16 FLOPs of its timed tensor-core groups over their summed
     issue-to-completion cycles, as TFLOP/s of the whole GPU at `sm_mhz` (every SM doing the
-    same) and as a fraction of `peak_tflops`.  Also per group."""
+    same) and as a fraction of `peak_tflops`.  Also per group, and ("union_*") the same FLOPs
+    over the cycles in which each CTA had at least one group in flight (overlapping groups
+    counted once)."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     out = {}
-    fl_all = cyc_all = 0.0
+    fl_all = cyc_all = ufl_all = ucyc_all = 0.0
     for slot, name in ((1, "tc_prep_kernel"), (0, "tc_chain_kernel")):
         fl = cyc = 0.0
         groups = []
@@ -121,11 +172,21 @@ def gemm_phase_fractions(m, peak_tflops, sm_mhz):
         if cyc:
             tf = fl / cyc * sm_mhz * 1e6 * sms / 1e12
             out[name] = {"tflops": tf, "frac": tf / peak_tflops, "groups": groups}
+            u = m.get("union", {}).get(slot)
+            if u and u[1]:
+                tu = u[0] / u[1] * sm_mhz * 1e6 * sms / 1e12
+                out[name].update({"union_tflops": tu, "union_frac": tu / peak_tflops,
+                                  "union_groups_logged": u[2], "union_groups_dropped": u[3]})
+                ufl_all += u[0]
+                ucyc_all += u[1]
             fl_all += fl
             cyc_all += cyc
     if cyc_all:   # the forward call as a whole: every group of both kernels
         tf = fl_all / cyc_all * sm_mhz * 1e6 * sms / 1e12
         out["forward"] = {"tflops": tf, "frac": tf / peak_tflops, "groups": []}
+        if ucyc_all:
+            tu = ufl_all / ucyc_all * sm_mhz * 1e6 * sms / 1e12
+            out["forward"].update({"union_tflops": tu, "union_frac": tu / peak_tflops})
     return out
 
 
@@ -240,6 +301,11 @@ def main(argv=None) -> int:
             print(f"  {name:16s} {g['group']:44s} {g['count']:8d} x {g['cycles']:6.0f} cycles "
                   f"= {g['tflops']:7.1f} TFLOP/s ({g['frac']:5.1%})")
         print(f"  {name:16s} {'all GEMM phases':44s} {'':19s} = {r['tflops']:7.1f} TFLOP/s ({r['frac']:5.1%})")
+        if "union_tflops" in r:
+            extra = (f"  [{r['union_groups_logged']} groups logged, {r['union_groups_dropped']} dropped]"
+                     if "union_groups_logged" in r else "")
+            print(f"  {name:16s} {'the same over the busy-interval union':44s} {'':19s} = "
+                  f"{r['union_tflops']:7.1f} TFLOP/s ({r['union_frac']:5.1%}){extra}")
     return 0
 
 
