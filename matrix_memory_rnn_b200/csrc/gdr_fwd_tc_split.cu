@@ -428,6 +428,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
           lam[i][4] = x1.x; lam[i][5] = x1.y; lam[i][6] = x1.z; lam[i][7] = x1.w;
         }
       }
+      GDR_PREP_PHASE(5);
       {
         float tot[8];
 #pragma unroll
@@ -450,6 +451,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
         }
       }
       FrontSync::sync();
+      GDR_PREP_PHASE(6);
       // the log-w staging has been read: load the next chunk's
       if (gt == 32 && j + 1 < nloc) {
         fence_proxy_async_smem();
@@ -468,6 +470,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
         sTOT[gt] = run;
       }
       FrontSync::sync();
+      GDR_PREP_PHASE(7);
       // lam[i][e] becomes Lam_t - Lam_1 (the pivot at the chunk's first token)
       float dn[8], ed[8];
       {
@@ -1032,6 +1035,7 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
     }
     got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
     if (!got) return false;
+    GDR_CHAIN_PHASE(7);   // the record has arrived
     const uint32_t bb = sb + buf * SL::BUF;
     constexpr uint32_t id = idesc_bf16_f32(2 * kC, NV, false, true);
     tc_fence_after();

@@ -76,6 +76,33 @@ _lock = threading.Lock()
 _lib = None
 
 
+def _declare(lib):
+    """Argument and result types of the C ABI on a loaded libgdr (or its timing build)."""
+    lib.gdr_forward_chunked.argtypes = [ctypes.POINTER(gdr_fwd_args), _vp]
+    lib.gdr_forward_workspace_size.argtypes = [ctypes.POINTER(gdr_fwd_args),
+                                               ctypes.POINTER(ctypes.c_size_t)]
+    lib.gdr_backward_chunked.argtypes = [ctypes.POINTER(gdr_bwd_args), _vp]
+    lib.gdr_backward_workspace_size.argtypes = [ctypes.POINTER(gdr_bwd_args),
+                                                ctypes.POINTER(ctypes.c_size_t)]
+    lib.gdr_muir_forward.argtypes = [ctypes.POINTER(gdr_muir_args), _vp]
+    lib.gdr_muir_workspace_size.argtypes = [ctypes.POINTER(gdr_muir_args),
+                                            ctypes.POINTER(ctypes.c_size_t)]
+    lib.gdr_mlstm_forward.argtypes = [ctypes.POINTER(gdr_mlstm_args), _vp]
+    lib.gdr_state_compose.argtypes = [_fp, _fp, _fp, _fp, _c_int, _c_int, _c_int, _vp]
+    lib.gdr_decode_step.argtypes = [ctypes.POINTER(gdr_step_args), _vp]
+    lib.gdr_state_init.argtypes = [_fp, _c_int, _c_int, _c_int, _c_int, _fp, _vp]
+    lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
+    lib.gdr_status_string.restype = ctypes.c_char_p
+    lib.gdr_status_string.argtypes = [_c_int]
+    for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size",
+               "gdr_backward_chunked", "gdr_backward_workspace_size",
+               "gdr_muir_forward", "gdr_muir_workspace_size", "gdr_mlstm_forward",
+               "gdr_state_compose",
+               "gdr_decode_step",
+               "gdr_state_init", "gdr_read_status", "gdr_version"):
+        getattr(lib, fn).restype = _c_int
+
+
 def _load():
     global _lib
     with _lock:
@@ -84,29 +111,7 @@ def _load():
                 from . import build as _build   # nvcc is required; raises if absent
                 _build.build()
             lib = ctypes.CDLL(LIB_PATH)
-            lib.gdr_forward_chunked.argtypes = [ctypes.POINTER(gdr_fwd_args), _vp]
-            lib.gdr_forward_workspace_size.argtypes = [ctypes.POINTER(gdr_fwd_args),
-                                                       ctypes.POINTER(ctypes.c_size_t)]
-            lib.gdr_backward_chunked.argtypes = [ctypes.POINTER(gdr_bwd_args), _vp]
-            lib.gdr_backward_workspace_size.argtypes = [ctypes.POINTER(gdr_bwd_args),
-                                                        ctypes.POINTER(ctypes.c_size_t)]
-            lib.gdr_muir_forward.argtypes = [ctypes.POINTER(gdr_muir_args), _vp]
-            lib.gdr_muir_workspace_size.argtypes = [ctypes.POINTER(gdr_muir_args),
-                                                    ctypes.POINTER(ctypes.c_size_t)]
-            lib.gdr_mlstm_forward.argtypes = [ctypes.POINTER(gdr_mlstm_args), _vp]
-            lib.gdr_state_compose.argtypes = [_fp, _fp, _fp, _fp, _c_int, _c_int, _c_int, _vp]
-            lib.gdr_decode_step.argtypes = [ctypes.POINTER(gdr_step_args), _vp]
-            lib.gdr_state_init.argtypes = [_fp, _c_int, _c_int, _c_int, _c_int, _fp, _vp]
-            lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
-            lib.gdr_status_string.restype = ctypes.c_char_p
-            lib.gdr_status_string.argtypes = [_c_int]
-            for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size",
-                       "gdr_backward_chunked", "gdr_backward_workspace_size",
-                       "gdr_muir_forward", "gdr_muir_workspace_size", "gdr_mlstm_forward",
-                       "gdr_state_compose",
-                       "gdr_decode_step",
-                       "gdr_state_init", "gdr_read_status", "gdr_version"):
-                getattr(lib, fn).restype = _c_int
+            _declare(lib)
             _lib = lib
     return _lib
 

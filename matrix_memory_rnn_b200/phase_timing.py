@@ -21,7 +21,9 @@ import torch
 from . import build, gdr, synth
 
 PREP_PHASES = [
-    (1, "front: wait for log w, tiles and write gate"), (2, "front: log-decay scan"),
+    (1, "front: wait for log w, tiles and write gate"), (5, "front: scan: log decay per thread"),
+    (6, "front: scan: block totals, barrier"), (7, "front: scan: exclusive prefix, barrier"),
+    (2, "front: scan: pivot and exponentials, barrier"),
     (3, "front: operand tiles and V^"), (4, "front: MMA1 issued, chunk handed over"),
     (0, "front: to the next chunk"),
     (9, "back: wait for the hand-over and MMA1"), (10, "back: L and M"),
@@ -30,7 +32,8 @@ PREP_PHASES = [
 ]
 CHAIN_PHASES = [
     (1, "wait for MMA3 ([Q_pi; Y] S0)"), (2, "V~ = U - Y S0"), (3, "MMA4 issued and waited for"),
-    (4, "state update and its bf16 copy"), (5, "MMA3 of the next chunk issued"), (6, "O read out"),
+    (4, "state update and its bf16 copy"), (7, "wait for the next chunk's record"),
+    (5, "MMA3 of the next chunk issued"), (6, "O read out"),
     (0, "to the next chunk"),
 ]
 # Tensor-core groups timed in the timing build (issue of the first MMA to completion, the
@@ -96,11 +99,50 @@ def read_union(lib, flops_of):
     return out
 
 
-def measure(batch=1, calls=3, lib=None):
-    """Runs the GDN-2 bf16 forward (B = batch, H = 16, T = 4096) through the timing build and
-    returns the per-phase cycle sums and the timed tensor-core groups, per chunk."""
-    lib = lib or load_timing_library()
+def measure_muir(batch=4, calls=3):
+    """The Muir mixer, fused (activations inside the prep kernel), on the gdn2_bf16 shapes with
+    B = batch, through the timing build: per-phase cycle sums of its prep and chain kernels,
+    per chunk (no tensor-core pass)."""
+    lib = load_timing_library()
+    gdr._declare(lib)
     w = synth.PRESETS["gdn2_bf16"].with_(B=batch)
+    inp = synth.muir_inputs(w)
+    names = ("q", "k", "v", "zf", "zb", "zw", "zq", "zg")
+    d = {k: torch.from_numpy(inp[k]).to("cuda", torch.bfloat16) for k in names}
+    par = {k: torch.from_numpy(inp[k]).cuda() for k in ("a_log", "gamma_stat", "rms_weight")}
+    cycles = (ctypes.c_ulonglong * 32)()
+    threads = (ctypes.c_ulonglong * 2)()
+    mma = [(ctypes.c_ulonglong * 16)() for _ in range(2)]
+    saved = gdr._lib
+    gdr._lib = lib           # the binding's calls go to the timing build meanwhile
+    try:
+        ws = gdr.new_workspace(gdr.gdr_muir_workspace_size(d["q"], d["k"], d["v"], 64, "tc", False), "cuda")
+        y = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device="cuda")
+
+        def run(n):
+            for _ in range(n):
+                gdr.gdr_muir_forward(*(d[k] for k in names), par["a_log"], par["gamma_stat"],
+                                     par["rms_weight"], 1e-6, None, chunk=64, algo="tc",
+                                     unfused=False, y=y, want_state=False, workspace=ws)
+            rc = lib.gdr_phase_timing_read(cycles, threads, mma[0], mma[1])
+            if rc != 0:
+                raise RuntimeError(f"gdr_phase_timing_read failed: CUDA error {rc}")
+
+        run(1)
+        run(calls)
+    finally:
+        gdr._lib = saved
+    nch = (w.T + 63) // 64
+    return {"w": w, "calls": calls, "threads": list(threads), "cycles": list(cycles),
+            "prep_chunks": w.B * w.H * nch * calls, "chain_chunks": w.B * w.H * (w.dv // 64) * nch * calls}
+
+
+def measure(batch=1, calls=3, lib=None, preset="gdn2_bf16"):
+    """Runs a GDN-2 bf16 forward workload (default gdn2_bf16: H = 16, T = 4096, with
+    B = batch) through the timing build and returns the per-phase cycle sums and the timed
+    tensor-core groups, per chunk."""
+    lib = lib or load_timing_library()
+    w = synth.PRESETS[preset].with_(B=batch)
     inp = synth.forward_inputs(w)
     d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "bf16")
     o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device="cuda")
@@ -256,6 +298,10 @@ def main(argv=None) -> int:
                     help="bf16 dense peak of the whole GPU (default: MEASURED_PEAKS.json's, else 1590)")
     ap.add_argument("--sm-mhz", type=float, default=1965.0,
                     help="SM clock of the run (the cycles are SM cycles)")
+    ap.add_argument("--preset", default="gdn2_bf16", choices=["gdn2_bf16", "gdn2_long"],
+                    help="forward workload (gdn2_long: B=1, T=65536, the one-launch path)")
+    ap.add_argument("--muir", action="store_true",
+                    help="the Muir mixer's fused forward (phases only)")
     ap.add_argument("--mlstm", action="store_true",
                     help="the mLSTM cell's tensor-core kernel instead of the forward")
     args = ap.parse_args(argv)
@@ -270,9 +316,10 @@ def main(argv=None) -> int:
             print(f"  {'sum':50s} {sum(per[r][i] for i, _ in phases):9.0f}")
         return 0
 
-    m = measure(args.batch, args.calls)
+    m = (measure_muir(args.batch, args.calls) if args.muir
+         else measure(args.batch, args.calls, preset=args.preset))
     w = m["w"]
-    print(f"GDN-2 bf16, B={w.B}, H={w.H}, T={w.T}, d=128, C=64; {args.calls} calls; "
+    print(f"{'Muir mixer (fused) on ' if args.muir else ''}GDN-2 bf16, B={w.B}, H={w.H}, T={w.T}, d=128, C=64; {args.calls} calls; "
           f"recording threads: prep {m['threads'][1]}, chain {m['threads'][0]}")
     for title, slot, phases, units in (("tc_prep_kernel", 1, PREP_PHASES, m["prep_chunks"]),
                                       ("tc_chain_kernel", 0, CHAIN_PHASES, m["chain_chunks"])):
@@ -286,6 +333,8 @@ def main(argv=None) -> int:
         for g, t in total.items():
             if t:
                 print(f"  {'sum' + (' (' + g + ')' if g else ''):50s} {t:9.0f}")
+    if args.muir:
+        return 0
     peak = args.peak_tflops
     if peak is None:
         import json
