@@ -1067,6 +1067,12 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
     // ---- wait for MMA3 (c): [Q_pi S0; Y S0] in D[c & 1]
     if (!(ok = chain_wait_mma<NT>(bar3, ph3, sabort))) break;
     const float pn = reinterpret_cast<const float *>(bsm + SL::B_PI)[jrow];
+    // one-launch path: warp 1 (idle while V~ is formed) sees whether record c + NBUF has
+    // been published, so that the acquire's round trip overlaps V~; the same lane issues
+    // the refill below
+    bool published = true;
+    if (rflags && warp == 1 && lane == 0 && c + NBUF < nch && !*sabort)
+      published = wait_published(rflags + c + NBUF, sabort);
 
     GDR_CHAIN_PHASE(1);
     // ---- V~ = U - Y S0 -> bf16 (rows = tokens), on the warps that own lanes C..2C-1
@@ -1109,8 +1115,8 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
     }
     if (!(ok = chain_wait_mma<NT>(bar4, ph4, sabort))) break;
     // every read of this chunk's buffer is done: refill it NBUF chunks ahead
-    if (warp == 2 && lane == 0 && c + NBUF < nch && !*sabort) {
-      if (rflags && !wait_published(rflags + c + NBUF, sabort)) {
+    if (warp == 1 && lane == 0 && c + NBUF < nch && !*sabort) {
+      if (!published) {
         *sabort = 1;
       } else {
         fence_proxy_async_smem();   // the CTA's reads of the buffer come before the refill
