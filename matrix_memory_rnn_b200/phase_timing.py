@@ -62,6 +62,20 @@ def load_timing_library():
 LOG_CTAS, LOG_ENTRIES = 256, 256   # the timing build's interval log (gdr_phase_timing.cuh)
 
 
+def union_length(spans):
+    """Total length of the union of closed intervals [start, end] (each start <= end)."""
+    total = 0
+    lo = hi = None
+    for a, b in sorted(spans):
+        if hi is None or a > hi:
+            if hi is not None:
+                total += hi - lo
+            lo, hi = a, b
+        else:
+            hi = max(hi, b)
+    return total + (hi - lo if hi is not None else 0)
+
+
 def read_union(lib, flops_of):
     """Reads (and clears) the timing build's MMA interval log and returns, per kernel slot,
     [bf16 FLOPs of the logged groups, the summed per-CTA union of their [start, end]
@@ -85,16 +99,8 @@ def read_union(lib, flops_of):
             dropped += n - k
             logged += k
             base = (slot * LOG_CTAS + cta) * LOG_ENTRIES
-            spans = sorted((iv[2 * (base + j)], iv[2 * (base + j) + 1]) for j in range(k))
             fl += sum(flops_of[(slot, gr[base + j])] for j in range(k))
-            lo, hi = spans[0]
-            for a, b in spans[1:]:
-                if a > hi:
-                    cyc += hi - lo
-                    lo, hi = a, b
-                else:
-                    hi = max(hi, b)
-            cyc += hi - lo
+            cyc += union_length((iv[2 * (base + j)], iv[2 * (base + j) + 1]) for j in range(k))
         out[slot] = [fl, cyc, logged, dropped]
     return out
 
