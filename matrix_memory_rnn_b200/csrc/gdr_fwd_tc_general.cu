@@ -44,6 +44,32 @@
 
 #include "gdr_tc_common.cuh"
 
+// Phase marks of the timing build (thread 0, cycles summed over CTAs and chunks into
+// g_general_cycles); empty in libgdr.so.
+#ifdef GDR_PHASE_TIMING
+namespace gdr {
+__device__ unsigned long long g_general_cycles[16];
+}
+#define GT_INIT                                                                     \
+  long long gt_a_[16] = {0};                                                        \
+  long long gt_l_ = 0;
+#define GT_MARK(i)                                                                  \
+  do {                                                                              \
+    if (threadIdx.x == 0) {                                                         \
+      const long long n_ = clock64();                                               \
+      if (gt_l_) gt_a_[i] += n_ - gt_l_;                                            \
+      gt_l_ = n_;                                                                   \
+    }                                                                               \
+  } while (0)
+#define GT_FINI                                                                     \
+  if (threadIdx.x == 0)                                                             \
+    for (int i_ = 0; i_ < 16; ++i_) atomicAdd(&gdr::g_general_cycles[i_], (unsigned long long)gt_a_[i_]);
+#else
+#define GT_INIT
+#define GT_MARK(i)
+#define GT_FINI
+#endif
+
 namespace gdr {
 namespace {
 
@@ -273,8 +299,10 @@ __global__ void __launch_bounds__(kGT, 2)
   // thread 0's counts: MMA groups committed, input loads issued / waited for
   uint32_t issued_mma = 0, in1_iss = nch > 0 ? 1u : 0u, in2_iss = in1_iss, in1_done = 0, in2_done = 0;
   bool ok = true;
+  GT_INIT
   for (int c = 0; c < nch; ++c) {
     const int t0 = c * kC, n = min(kC, T - t0);
+    GT_MARK(0);
     // ---- this chunk's inputs have landed
     if (tid == 0 && !*sabort) {
       if (mbar_wait_bounded(in1, c & 1, kWaitLimitNs)) ++in1_done;
@@ -289,10 +317,12 @@ __global__ void __launch_bounds__(kGT, 2)
     }
     __syncthreads();
     if (!(ok = *sabort == 0)) break;
+    GT_MARK(1);
 
     // ---- cumulative log-decay in place (slots 9-10)
     chunk_scan(sLW, sQT, sA1, sDN, sPI, sexact, tid);
     const bool exact = *sexact != 0;
+    GT_MARK(2);
 
     // ---- operand tiles.  Thread = (channel group g of 8, token pair tp); each input
     //      element is read and its outputs written at the same swizzled offset, so the
@@ -414,6 +444,7 @@ __global__ void __launch_bounds__(kGT, 2)
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    GT_MARK(3);
 
     // ---- MMA1: [U f'; Q f] (M = 128) x [Z g; K g]^T (N = 128), K = d_k
     if (warp == 0) {
@@ -429,6 +460,7 @@ __global__ void __launch_bounds__(kGT, 2)
       if (lane == 0) ++issued_mma;
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    GT_MARK(4);
 
     // ---- A (fp32, strictly lower -> over the MMA1 B operand), B (bf16, below Q_pi),
     //      M_k, M_z (bf16, over log w).  Row r = 32 qd + lane: r < 64 the U rows
@@ -540,6 +572,7 @@ __global__ void __launch_bounds__(kGT, 2)
     tc_fence_before();
     __syncthreads();
 
+    GT_MARK(5);
     // ---- MMA-BV: B V (M = 64) -> TMEM; state accumulator = K~^T V ([K~ | *], M = 128).
     //      They run while T^-1 is formed.
     if (warp == 0) {
@@ -574,6 +607,7 @@ __global__ void __launch_bounds__(kGT, 2)
       st_smem16(smem, SL::TI + sw128_offset(t, 8 * gg, kC * 128), pack8(x));
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;    // B V and K~^T V
+    GT_MARK(6);
 
     // ---- B V (M = 64 accumulator: row 16 qd + r at lane 32 qd + r) -> bf16 tile
     if (hf == 0) {
@@ -588,6 +622,7 @@ __global__ void __launch_bounds__(kGT, 2)
     tc_fence_before();
     __syncthreads();
 
+    GT_MARK(7);
     // ---- MMA2: [Y_u | W] = T^-1 [U_pi | B V] (M = 64, N = 128), K = C
     if (warp == 0) {
       tc_fence_after();
@@ -602,6 +637,7 @@ __global__ void __launch_bounds__(kGT, 2)
       if (lane == 0) ++issued_mma;
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    GT_MARK(8);
 
     // ---- Y_u -> rows 64..127 of [Q_pi; Y_u]; -W -> its tile.  hf 0: Y_u columns, 1: W columns
     {
@@ -625,6 +661,7 @@ __global__ void __launch_bounds__(kGT, 2)
     tc_fence_before();
     __syncthreads();
 
+    GT_MARK(9);
     // ---- MMA3: [Q_pi; Y_u] S0' (M = 128), K = d_k; output extra = [M_k; *] V (M = 128), K = C
     if (warp == 0) {
       tc_fence_after();
@@ -645,6 +682,7 @@ __global__ void __launch_bounds__(kGT, 2)
       if (lane == 0) ++issued_mma;
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    GT_MARK(10);
     // ---- v is consumed: load the next chunk's
     if (tid == 0 && c + 1 < nch) {
       fence_proxy_async_smem();
@@ -671,6 +709,7 @@ __global__ void __launch_bounds__(kGT, 2)
     tc_fence_before();
     __syncthreads();
 
+    GT_MARK(11);
     // ---- MMA4: state acc += [Z~ | *]^T V~ (M = 128); output extra += [M_z; *] V~ (M = 128)
     if (warp == 0) {
       tc_fence_after();
@@ -688,6 +727,7 @@ __global__ void __launch_bounds__(kGT, 2)
       if (lane == 0) ++issued_mma;
     }
     if (!(ok = wait_mma(mbar, phase, sabort))) break;
+    GT_MARK(12);
     // ---- u, q, z, k, log w are consumed (and their slots' later tenants): load the next chunk's
     if (tid == 0 && c + 1 < nch) {
       fence_proxy_async_smem();
@@ -725,7 +765,9 @@ __global__ void __launch_bounds__(kGT, 2)
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    GT_MARK(13);
   }
+  GT_FINI
 
   if (ok && owner && p.S_T) {
 #pragma unroll
@@ -811,3 +853,15 @@ cudaError_t launch_forward_tc_general(const FwdParams &p, cudaStream_t stream) {
 }
 
 }  // namespace gdr
+
+#ifdef GDR_PHASE_TIMING
+// Timing build only: copies the two-stream kernel's per-phase cycle sums ([16], thread 0 of
+// every CTA, every chunk) to host memory, then clears them.  Returns 0 or a CUDA error.
+extern "C" int gdr_general_timing_read(unsigned long long *cycles) {
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e == cudaSuccess) e = cudaMemcpyFromSymbol(cycles, gdr::g_general_cycles, sizeof(gdr::g_general_cycles));
+  static const unsigned long long z[16] = {};
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(gdr::g_general_cycles, z, sizeof(z));
+  return (int)e;
+}
+#endif

@@ -105,6 +105,50 @@ def read_union(lib, flops_of):
     return out
 
 
+# Marks of the two-stream kernel (every form at d = 64): (index, label), thread 0 per CTA.
+GENERAL_PHASES = [
+    (1, "wait for the chunk's inputs, barrier"), (2, "log-decay scan"),
+    (3, "operand tiles, barrier"), (4, "MMA1 issued and waited for"),
+    (5, "A, B, M_z, M_k formed"), (6, "B V, K~^T V issued; T^-1; waited for"),
+    (7, "B V as bf16"), (8, "MMA2 [Y_u | W] issued and waited for"),
+    (9, "Y_u, W to their tiles"), (10, "MMA3 [Q_pi; Y_u] S0' + M_k V issued and waited for"),
+    (11, "V~ formed"), (12, "MMA4 issued and waited for"), (13, "state update and output, barrier"),
+    (0, "to the next chunk"),
+]
+
+
+def measure_general(preset="rwkv7_bf16", calls=3):
+    """The two-stream tensor-core forward (d = 64) on `preset` through the timing build:
+    thread 0's cycles per chunk by phase."""
+    lib = load_timing_library()
+    lib.gdr_general_timing_read.argtypes = [ctypes.POINTER(ctypes.c_ulonglong)]
+    lib.gdr_general_timing_read.restype = ctypes.c_int
+    w = synth.PRESETS[preset]
+    inp = synth.forward_inputs(w)
+    d = gdr.to_device({k: inp[k] for k in ("q", "k", "v", "log_w", "e1", "e2")}, "bf16")
+    o = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device="cuda")
+    S_T = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device="cuda")
+    ws = gdr.new_workspace(gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"], d["log_w"],
+                                                          d["e1"], d["e2"], 64, "tc"), "cuda")
+    a = gdr._fwd_struct(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"], d["e2"], None, o, S_T, 64,
+                        "tc", ws)
+    cycles = (ctypes.c_ulonglong * 16)()
+
+    def run(n):
+        for _ in range(n):
+            rc = lib.gdr_forward_chunked(ctypes.byref(a), None)
+            if rc != 0:
+                raise RuntimeError(f"gdr_forward_chunked (timing build) failed: {rc}")
+        rc = lib.gdr_general_timing_read(cycles)
+        if rc != 0:
+            raise RuntimeError(f"gdr_general_timing_read failed: CUDA error {rc}")
+
+    run(1)
+    run(calls)
+    chunks = w.B * w.H * ((w.T + 63) // 64) * calls
+    return w, {i: cycles[i] / chunks for i in range(16)}
+
+
 def measure_muir(batch=4, calls=3):
     """The Muir mixer, fused (activations inside the prep kernel), on the gdn2_bf16 shapes with
     B = batch, through the timing build: per-phase cycle sums of its prep and chain kernels,
@@ -306,6 +350,8 @@ def main(argv=None) -> int:
                     help="SM clock of the run (the cycles are SM cycles)")
     ap.add_argument("--preset", default="gdn2_bf16", choices=["gdn2_bf16", "gdn2_long"],
                     help="forward workload (gdn2_long: B=1, T=65536, the one-launch path)")
+    ap.add_argument("--general", action="store_true",
+                    help="the two-stream kernel (every form at d = 64) on rwkv7_bf16")
     ap.add_argument("--muir", action="store_true",
                     help="the Muir mixer's fused forward (phases only)")
     ap.add_argument("--mlstm", action="store_true",
@@ -322,6 +368,13 @@ def main(argv=None) -> int:
             print(f"  {'sum':50s} {sum(per[r][i] for i, _ in phases):9.0f}")
         return 0
 
+    if args.general:
+        w, per = measure_general(calls=args.calls)
+        print(f"tc_general_kernel, {w.form} bf16, B={w.B}, H={w.H}, T={w.T}, d={w.dk}: thread 0's cycles per chunk")
+        for i, label in GENERAL_PHASES:
+            print(f"  {label:55s} {per[i]:9.0f}")
+        print(f"  {'sum':55s} {sum(per[i] for i, _ in GENERAL_PHASES):9.0f}")
+        return 0
     m = (measure_muir(args.batch, args.calls) if args.muir
          else measure(args.batch, args.calls, preset=args.preset))
     w = m["w"]
