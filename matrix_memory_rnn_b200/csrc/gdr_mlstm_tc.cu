@@ -85,8 +85,9 @@ constexpr int kMThreads = 256;
 // gates.  Then P~ (64 x 64, K-major A operand, with 8 KB of padding as the unused rows
 // 64..127), diag(f) [V | 1] (64 tokens x (64 + 64), the B operand of K^T diag(f) [V | 1]; column 0
 // of its second block holds f, the rest of that block stays 0), [C | n] (bf16, 128
-// key channels x (64 + 64): C's block then a block whose column 0 holds n), the scan's
-// per-token arrays and the barriers.
+// key channels x (64 + 64): C's block then a block whose column 0 holds n), the h staging
+// (per chunk parity, four warps' 32 tokens x 32 fp32 columns, 128-byte swizzled for the TMA
+// stores), the scan's per-token arrays (two chunks) and the barriers.
 struct MSmem {
   static constexpr uint32_t QK = 0;
   static constexpr uint32_t V = QK + 2 * 128 * 128;           // 32 KB
@@ -117,7 +118,8 @@ struct MMaps {
 // TMEM columns: S 64, [Q C | Q n] 80, [P~ V | P~ 1] 80, [K~^T V | K~^T 1] 80.
 constexpr uint32_t kColS = 0, kColQC = 64, kColH = 160, kColDS = 256, kMTmemCols = 512;
 
-// 2^x by the PTX instruction ex2.approx.ftz.f32 (relative error about 2^-22; 2^-inf = 0).
+// 2^x by the PTX instruction ex2.approx.ftz.f32 (an approximation; 2^-inf = 0).  The
+// weights it forms are rounded to bf16 next.
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
