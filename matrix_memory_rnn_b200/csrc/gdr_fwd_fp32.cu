@@ -21,9 +21,14 @@
 // For GDN-2 (z = k, u = alpha b k) this reduces exactly to section 2.2 with
 // A = Bm = L_strict and V~ = V - E.
 //
-// This kernel evaluates every product in fp32 on the CUDA cores with the exact
-// pairwise decay (one exp per pair and channel).  It is the accurate path (fp32
-// inputs) and the reference kernel for the tensor-core path.  One CTA per
+// This kernel evaluates every product in fp32 on the CUDA cores.  When no channel
+// decays by more than 80 nats over the chunk, each pair's decay e^{Lam[a] - Lam[b]} (a
+// the later index) splits as e^{Lam[a] - P} e^{P - Lam[b]} with P the channel's Lam at
+// the chunk's middle, every factor in [e^-80, e^80]: q and u take the first factor, k
+// and z the second, in place, and the pairwise products become plain dot products (one
+// exponential per element instead of up to three per pair and channel).  A chunk that
+// decays more takes the exact pairwise decay (one exp per pair and channel).  It is the
+// accurate path (fp32 inputs) and the reference kernel for the tensor-core path.  One CTA per
 // (b, h, slice of NV value columns), looping over the chunks; the chunk is held
 // in shared memory, so the kernel caps its chunk at 64 tokens and at
 // 4096 / dk tokens (32 at dk = 128); the result does not depend on the chunk
@@ -34,6 +39,7 @@ namespace gdr {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr float kMaxSpan = 80.f;   // nats of decay over a chunk for the pivot path
 
 __host__ __device__ inline int fp32_chunk(int dk, int chunk) {
   int c = chunk < 64 ? chunk : 64;
@@ -45,7 +51,7 @@ __host__ __device__ inline int fp32_nv(int dv) { return dv < 32 ? dv : 32; }
 struct Smem {
   int LD;  // padded row stride of the d_k-wide arrays (dk + 1: conflict-free columns)
   int C, NV, dk;
-  size_t lam, q, k, u, z, v, e, r, A, Bm, Mk, Mz, S, total;  // float offsets
+  size_t lam, q, k, u, z, v, e, r, A, Bm, Mk, Mz, S, fac, flag, total;  // float offsets
   __host__ __device__ Smem(int dk_, int dv, int chunk) {
     dk = dk_;
     LD = dk + 1;
@@ -65,6 +71,8 @@ struct Smem {
     Mk = off; off += (size_t)C * C;
     Mz = off; off += (size_t)C * C;
     S = off; off += (size_t)dk * NV;
+    fac = off; off += (size_t)3 * dk;   // pivot path: e^P, e^(Lam[n] - P), e^Lam[n] per channel
+    flag = off; off += 4;               // int: this chunk takes the exact pairwise path
     total = off;
   }
 };
@@ -80,6 +88,8 @@ __global__ void __launch_bounds__(kThreads) fwd_fp32_kernel(FwdParams p) {
   float *lam = sm + L.lam, *Q = sm + L.q, *K = sm + L.k, *U = sm + L.u, *Z = sm + L.z;
   float *V = sm + L.v, *E = sm + L.e, *R = sm + L.r;
   float *A = sm + L.A, *Bm = sm + L.Bm, *Mk = sm + L.Mk, *Mz = sm + L.Mz, *S = sm + L.S;
+  float *fac = sm + L.fac;
+  volatile int *sflag = reinterpret_cast<volatile int *>(sm + L.flag);
   const Tin *q = static_cast<const Tin *>(p.q), *k = static_cast<const Tin *>(p.k);
   const Tin *v = static_cast<const Tin *>(p.v), *e1 = static_cast<const Tin *>(p.e1);
   const Tin *e2 = static_cast<const Tin *>(p.e2);
@@ -118,7 +128,10 @@ __global__ void __launch_bounds__(kThreads) fwd_fp32_kernel(FwdParams p) {
     }
     __syncthreads();
 
-    // 2. cumulative log-decay (one thread per channel)
+    // 2. cumulative log-decay (one thread per channel); a channel that decays by more
+    //    than 80 nats over the chunk sends the chunk to the exact pairwise path
+    if (tid == 0) *sflag = 0;
+    __syncthreads();
     for (int j = tid; j < dk; j += kThreads) {
       float acc = 0.f;
       lam[j] = 0.f;
@@ -126,14 +139,52 @@ __global__ void __launch_bounds__(kThreads) fwd_fp32_kernel(FwdParams p) {
         acc += lam[t * LD + j];
         lam[t * LD + j] = acc;
       }
+      if (!(acc >= -kMaxSpan)) *sflag = 1;   // (NaN too)
     }
     __syncthreads();
+    const bool exact = *sflag != 0;
+
+    // 2b. pivot path: q_t *= e^(Lam[t+1] - P), u_t *= e^(Lam[t] - P), k_s, z_s *= e^(P - Lam[s+1])
+    //     in place, P = Lam[n/2] per channel; then the three per-channel factors the later
+    //     steps use in place of their exponentials of Lam
+    if (!exact) {
+      const int pv = n / 2;
+      for (int i = tid; i < n * dk; i += kThreads) {
+        const int t = i / dk, j = i % dk;
+        const float P = lam[pv * LD + j], l1 = lam[(t + 1) * LD + j];
+        Q[t * LD + j] *= expf(l1 - P);
+        K[t * LD + j] *= expf(P - l1);
+        if (has_erase) {
+          U[t * LD + j] *= expf(lam[t * LD + j] - P);
+          Z[t * LD + j] *= expf(P - l1);
+        }
+      }
+      for (int j = tid; j < dk; j += kThreads) {
+        const float P = lam[pv * LD + j], ln = lam[n * LD + j];
+        fac[j] = expf(P);
+        fac[dk + j] = expf(ln - P);
+        fac[2 * dk + j] = expf(ln);
+      }
+      __syncthreads();
+    }
 
     // 3. pairwise decay-weighted products
     for (int i = tid; i < n * n; i += kThreads) {
       const int t = i / n, s = i % n;
       float a = 0.f, bm = 0.f, mk = 0.f, mz = 0.f;
-      if (s <= t) {
+      if (s <= t && !exact) {   // the decays are in the scaled rows
+        const float *qt = Q + t * LD, *ut = U + t * LD, *ks = K + s * LD, *zs = Z + s * LD;
+        for (int j = 0; j < dk; ++j) {
+          mk += qt[j] * ks[j];
+          if (has_erase) {
+            mz += qt[j] * zs[j];
+            if (s < t) {
+              a += ut[j] * zs[j];
+              bm += ut[j] * ks[j];
+            }
+          }
+        }
+      } else if (s <= t) {
         const float *lt = lam + t * LD, *lt1 = lam + (t + 1) * LD, *ls1 = lam + (s + 1) * LD;
         const float *qt = Q + t * LD, *ut = U + t * LD, *ks = K + s * LD, *zs = Z + s * LD;
         for (int j = 0; j < dk; ++j) {
@@ -162,7 +213,10 @@ __global__ void __launch_bounds__(kThreads) fwd_fp32_kernel(FwdParams p) {
         const int t = i / NV, c = i % NV;
         float acc = 0.f;
         const float *lt = lam + t * LD, *ut = U + t * LD;
-        for (int j = 0; j < dk; ++j) acc += ut[j] * __expf(lt[j]) * S[j * NV + c];
+        if (exact)
+          for (int j = 0; j < dk; ++j) acc += ut[j] * __expf(lt[j]) * S[j * NV + c];
+        else   // u_t e^(Lam[t] - P) e^P
+          for (int j = 0; j < dk; ++j) acc += ut[j] * fac[j] * S[j * NV + c];
         for (int s = 0; s < t; ++s) acc += Bm[t * n + s] * V[s * NV + c];
         R[i] = acc;
       }
@@ -191,7 +245,10 @@ __global__ void __launch_bounds__(kThreads) fwd_fp32_kernel(FwdParams p) {
       const int t = i / NV, c = i % NV;
       float acc = 0.f;
       const float *lt1 = lam + (t + 1) * LD, *qt = Q + t * LD;
-      for (int j = 0; j < dk; ++j) acc += qt[j] * __expf(lt1[j]) * S[j * NV + c];
+      if (exact)
+        for (int j = 0; j < dk; ++j) acc += qt[j] * __expf(lt1[j]) * S[j * NV + c];
+      else   // q_t e^(Lam[t+1] - P) e^P
+        for (int j = 0; j < dk; ++j) acc += qt[j] * fac[j] * S[j * NV + c];
       for (int s = 0; s <= t; ++s) {
         acc += Mk[t * n + s] * V[s * NV + c];
         if (has_erase) acc -= Mz[t * n + s] * E[s * NV + c];
@@ -202,7 +259,8 @@ __global__ void __launch_bounds__(kThreads) fwd_fp32_kernel(FwdParams p) {
     __syncthreads();
     for (int i = tid; i < n * dk; i += kThreads) {
       const int s = i / dk, j = i % dk;
-      const float d = __expf(lam[n * LD + j] - lam[(s + 1) * LD + j]);
+      // (pivot path: k_s e^(P - Lam[s+1]) e^(Lam[n] - P))
+      const float d = exact ? __expf(lam[n * LD + j] - lam[(s + 1) * LD + j]) : fac[dk + j];
       K[s * LD + j] *= d;
       Z[s * LD + j] *= d;
     }
@@ -211,7 +269,7 @@ __global__ void __launch_bounds__(kThreads) fwd_fp32_kernel(FwdParams p) {
     // 7. state update
     for (int i = tid; i < dk * NV; i += kThreads) {
       const int j = i / NV, c = i % NV;
-      float acc = __expf(lam[n * LD + j]) * S[i];
+      float acc = (exact ? __expf(lam[n * LD + j]) : fac[2 * dk + j]) * S[i];
       for (int s = 0; s < n; ++s) {
         acc += K[s * LD + j] * V[s * NV + c];
         if (has_erase) acc -= Z[s * LD + j] * E[s * NV + c];
