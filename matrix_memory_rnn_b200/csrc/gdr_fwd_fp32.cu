@@ -38,7 +38,7 @@
 namespace gdr {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr float kMaxSpan = 80.f;   // nats of decay over a chunk for the pivot path
 
 __host__ __device__ inline int fp32_chunk(int dk, int chunk) {
