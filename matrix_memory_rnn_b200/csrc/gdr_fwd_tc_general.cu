@@ -471,11 +471,16 @@ __global__ void __launch_bounds__(kGT, 2)
       tmem_ld_32x32b_x32(tmem + kT_D1 + lane_q + 64 * hf, x);
       tmem_ld_32x32b_x32(tmem + kT_D1 + lane_q + 64 * hf + 32, y);
       tmem_ld_wait();
+      GT_MARK(14);
       const bool urow = r < kC;
+      // columns below lim are kept (strictly lower for A and B, lower with the diagonal for
+      // M_z and M_k); one compare per element against a per-lane limit (a nested
+      // condition per element here was measured at several times the cost)
+      const int lim = urow ? t : t + 1;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        x[i] = (urow ? (i < t) : (i <= t)) ? x[i] : 0.f;
-        y[i] = (urow ? (32 + i < t) : (32 + i <= t)) ? y[i] : 0.f;
+        x[i] = i < lim ? x[i] : 0.f;
+        y[i] = 32 + i < lim ? y[i] : 0.f;
       }
       if (urow && hf == 0) {
 #pragma unroll
@@ -561,6 +566,7 @@ __global__ void __launch_bounds__(kGT, 2)
             __float2bfloat16_rn(mk);
       }
     }
+    GT_MARK(15);
     if (kRwkv && warp == 0 && c + 1 < nch) {
 #pragma unroll
       for (int i = 0; i < 2; ++i) {

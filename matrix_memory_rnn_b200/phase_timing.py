@@ -109,7 +109,8 @@ def read_union(lib, flops_of):
 GENERAL_PHASES = [
     (1, "wait for the chunk's inputs, barrier"), (2, "log-decay scan"),
     (3, "operand tiles, barrier"), (4, "MMA1 issued and waited for"),
-    (5, "A, B, M_z, M_k formed"), (6, "B V, K~^T V issued; T^-1; waited for"),
+    (14, "A, B, M_z, M_k: from TMEM"), (15, "A, B, M_z, M_k: masked, stored"),
+    (5, "A, B, M_z, M_k: gate loads, fence, barrier"), (6, "B V, K~^T V issued; T^-1; waited for"),
     (7, "B V as bf16"), (8, "MMA2 [Y_u | W] issued and waited for"),
     (9, "Y_u, W to their tiles"), (10, "MMA3 [Q_pi; Y_u] S0' + M_k V issued and waited for"),
     (11, "V~ formed"), (12, "MMA4 issued and waited for"), (13, "state update and output, barrier"),
