@@ -343,6 +343,11 @@ __global__ void __launch_bounds__(kGT, 2)
         a0[0] = x0.x; a0[1] = x0.y; a0[2] = x0.z; a0[3] = x0.w;
         a0[4] = x1.x; a0[5] = x1.y; a0[6] = x1.z; a0[7] = x1.w;
       }
+      // pivot path: e^{dn} per channel, so that K~'s e^{dn - lam} = e^{dn} e^{-lam} reuses
+      // the e^{-lam} of K g; e^{lam} of the thread's first token is the second's f'
+      float edn[8], elam_prev[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) edn[e] = exact ? 0.f : __expf(dn[e]);
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
         const int t = 2 * tp + i;
@@ -365,7 +370,7 @@ __global__ void __launch_bounds__(kGT, 2)
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             if (kForm == GDR_FORM_GDN2) at[e] = __expf(lam[e] - fp[e]);
-            fp[e] = __expf(fp[e]);
+            fp[e] = (i == 1 && !exact) ? elam_prev[e] : __expf(fp[e]);
           }
         } else {
 #pragma unroll
@@ -417,14 +422,21 @@ __global__ void __launch_bounds__(kGT, 2)
         st_smem16(smem, SL::UP + o, pack8(x));
         // Q f (in place over q) and Q_pi
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = q8[e] * __expf(lam[e]);
+        for (int e = 0; e < 8; ++e) {
+          elam_prev[e] = __expf(lam[e]);
+          x[e] = q8[e] * elam_prev[e];
+        }
         st_smem16(smem, SL::A1 + kTile + o, pack8(x));
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] *= a0[e];
         st_smem16(smem, SL::QY + o, pack8(x));
-        // K~, Z~ (direct) and Z g, K g (pivot split; zero on the exact path)
+        // K~, Z~ (direct: e^{Lam_63 - Lam_t} <= 1, as e^{dn} e^{-lam} on the pivot path, where
+        // both factors lie in [e^-80, e^80]) and Z g, K g (pivot split; zero on the exact path)
+        float eml[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) fp[e] = __expf(dn[e] - lam[e]);   // e^{Lam_63 - Lam_t} <= 1
+        for (int e = 0; e < 8; ++e) eml[e] = exact ? 0.f : __expf(-lam[e]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) fp[e] = exact ? __expf(dn[e] - lam[e]) : edn[e] * eml[e];
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = k8[e] * fp[e];
         st_smem16(smem, SL::KT + o, pack8(x));
@@ -432,7 +444,7 @@ __global__ void __launch_bounds__(kGT, 2)
         for (int e = 0; e < 8; ++e) x[e] = z8[e] * fp[e];
         st_smem16(smem, SL::ZT + o, pack8(x));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) fp[e] = exact ? 0.f : __expf(-lam[e]);
+        for (int e = 0; e < 8; ++e) fp[e] = eml[e];
 #pragma unroll
         for (int e = 0; e < 8; ++e) x[e] = z8[e] * fp[e];
         st_smem16(smem, SL::B1 + o, pack8(x));
