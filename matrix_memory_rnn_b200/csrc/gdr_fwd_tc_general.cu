@@ -138,6 +138,7 @@ constexpr uint32_t kT_D1 = 0, kT_BV = 128, kT_DS = 192, kT_M2 = 0, kT_D3 = 0, kT
 
 struct GenMaps {
   CUtensorMap q, k, v, e1, e2, lw;
+  CUtensorMap o;   // stores: boxes of 32 fp32 columns x 32 tokens, 128-byte swizzle
 };
 
 // Which tiles a form stages: e1 (u, a or the erase gate b) in the first half of the
@@ -303,7 +304,9 @@ __global__ void __launch_bounds__(kGT, 2)
   for (int c = 0; c < nch; ++c) {
     const int t0 = c * kC, n = min(kC, T - t0);
     GT_MARK(0);
-    // ---- this chunk's inputs have landed
+    // ---- this chunk's inputs have landed; the previous chunk's o stores have read the
+    //      staging that this chunk's operand tiles overwrite
+    if (tid == 0) bulk_wait_read<0>();
     if (tid == 0 && !*sabort) {
       if (mbar_wait_bounded(in1, c & 1, kWaitLimitNs)) ++in1_done;
       else *sabort = 1;
@@ -771,21 +774,30 @@ __global__ void __launch_bounds__(kGT, 2)
       tmem_ld_32x32b_x32(tmem + kT_D3 + lane_q + 32 * hf, o1);
       tmem_ld_32x32b_x32(tmem + kT_DO + lane_q + 32 * hf, d);
       tmem_ld_wait();
-      const int t = jrow;
-      if (t < n) {
-        float4 *dst = reinterpret_cast<float4 *>(p.o + (((size_t)b * T + t0 + t) * H + h) * kD + 32 * hf);
+      // o staged over [Q_pi; Y_u] (read by MMA3, rewritten only by the next chunk's
+      // operand tiles) as four boxes of 32 tokens x 32 columns, 128-byte swizzled, for
+      // thread 0's TMA stores after the barrier below; rows past T are clipped by the copy
+      uint8_t *box = smem + SL::QY + ((2 * qd + hf) << 12);
 #pragma unroll
-        for (int i = 0; i < 32; i += 4)
-          dst[i / 4] = make_float4(o1[i] + d[i], o1[i + 1] + d[i + 1], o1[i + 2] + d[i + 2],
-                                   o1[i + 3] + d[i + 3]);
-      }
+      for (int i = 0; i < 32; i += 4)
+        *reinterpret_cast<float4 *>(box + lane * 128 + (((i >> 2) ^ (lane & 7)) << 4)) =
+            make_float4(o1[i] + d[i], o1[i + 1] + d[i + 1], o1[i + 2] + d[i + 2], o1[i + 3] + d[i + 3]);
     }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) {   // this chunk's o: four TMA stores from the staging
+#pragma unroll
+      for (int bx = 0; bx < 4; ++bx) {
+        const int tok = t0 + 32 * (bx >> 1);
+        if (tok < T) tma_store_4d(&maps.o, smem + SL::QY + (bx << 12), 32 * (bx & 1), h, tok, b);
+      }
+      bulk_commit();
+    }
     GT_MARK(13);
   }
   GT_FINI
+  if (tid == 0) bulk_wait<0>();   // o's stores complete before the CTA exits
 
   if (ok && owner && p.S_T) {
 #pragma unroll
@@ -838,6 +850,21 @@ bool encode_gen_map(CUtensorMap *m, const void *base, bool bf16, const FwdParams
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The output o [B][T][H][64] fp32 as a 4-D map for the TMA stores: boxes of 32 columns x 32
+// tokens (128 bytes per row) with the 128-byte swizzle.
+bool encode_out_map(CUtensorMap *m, void *base, const FwdParams &p) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = gen_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)p.H, (cuuint64_t)p.T, (cuuint64_t)p.B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kD * 4, (cuuint64_t)p.H * kD * 4,
+                                 (cuuint64_t)p.T * p.H * kD * 4};
+  const cuuint32_t box[4] = {32, 1, 32, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool forward_tc_general_supported(const FwdParams &p, gdr_dtype dtype) {
@@ -853,7 +880,7 @@ cudaError_t launch_forward_tc_general(const FwdParams &p, cudaStream_t stream) {
   if (!encode_gen_map(&maps.q, p.q, true, p) || !encode_gen_map(&maps.k, p.k, true, p) ||
       !encode_gen_map(&maps.v, p.v, true, p) || (e1 && !encode_gen_map(&maps.e1, p.e1, true, p)) ||
       (e2 && !encode_gen_map(&maps.e2, p.e2, true, p)) ||
-      !encode_gen_map(&maps.lw, p.log_w, false, p))
+      !encode_gen_map(&maps.lw, p.log_w, false, p) || !encode_out_map(&maps.o, p.o, p))
     return cudaErrorInvalidValue;
   void (*kern)(FwdParams, const GenMaps) = nullptr;
   switch (p.form) {
