@@ -149,6 +149,7 @@ struct PrepMisc {             // byte offsets inside PrepSmem::MISC
   static constexpr uint32_t SLOT = 80;      // uint32_t     TMEM base
   static constexpr uint32_t ABORT = 84;     // int          a bounded wait ran out
   static constexpr uint32_t EXACT = 88;     // int [2]      the buffer's chunk takes the exact path
+  static constexpr uint32_t QREADY = 96;    // uint64_t [2] Muir: back -> front: the q tile activated
   static constexpr uint32_t CNT = 128;      // uint32_t [16] issued / completed counts (drain)
   static constexpr uint32_t TBAR = 192;     // uint64_t [2] timing build: MMA1 / MMA2 group timing
 };
@@ -286,6 +287,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
   uint64_t *wfull = reinterpret_cast<uint64_t *>(misc + PrepMisc::WFULL);
   uint64_t *lfull = reinterpret_cast<uint64_t *>(misc + PrepMisc::LFULL);
   uint64_t *ready = reinterpret_cast<uint64_t *>(misc + PrepMisc::READY);
+  uint64_t *qready = reinterpret_cast<uint64_t *>(misc + PrepMisc::QREADY);
   uint64_t *bar1 = reinterpret_cast<uint64_t *>(misc + PrepMisc::BAR1);
   uint64_t *bar2 = reinterpret_cast<uint64_t *>(misc + PrepMisc::BAR2);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(misc + PrepMisc::SLOT);
@@ -326,6 +328,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
       mbar_init(bfull + i, 1);
       mbar_init(wfull + i, 1);
       mbar_init(ready + i, 1);
+      mbar_init(qready + i, 1);
       mbar_init(bar1 + i, 1);
       sexact[i] = 0;
     }
@@ -368,34 +371,16 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
       uint8_t *rec = rec_of(item);
       float *a1s = sA1 + (j & 3) * kDK;
       GDR_PREP_PHASE(0);
-      // Muir: this thread's 4 tokens x 8 channels of z_q and 8 static gains, loaded now so
-      // that their latency overlaps the waits and the scan
-      uint4 zq_raw[4];
-      float gs8[8];
-      if constexpr (kMuir) {
-        const int bh = bh_of(item), hh = bh % H;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int tt = c_of(item) * kC + 4 * tb + i;
-          zq_raw[i] = tt < T ? ld16(gzq + (((size_t)(bh / H) * T + tt) * H + hh) * kDK + j0)
-                             : make_uint4(0u, 0u, 0u, 0u);
-        }
-        if (p.gamma_stat) {
-          const float4 a = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0));
-          const float4 c = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0 + 4));
-          gs8[0] = a.x; gs8[1] = a.y; gs8[2] = a.z; gs8[3] = a.w;
-          gs8[4] = c.x; gs8[5] = c.y; gs8[6] = c.z; gs8[7] = c.w;
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) gs8[e] = 1.f;
-        }
-      }
+      // Muir: the head's a_log, loaded now so that its latency overlaps the waits
+      const float a_log = kMuir ? __ldg(p.a_log + bh_of(item) % H) : 0.f;
 
-      // chunk j's log w, tiles and write gate have landed
+      // chunk j's log w, tiles and write gate have landed (Muir: and the back group has
+      // activated its q tile)
       if (poller) sexact[bi] = 0;
       if (!group_wait<FrontSync>(lfull, j & 1, sabort, poller)) break;
       if (!group_wait<FrontSync>(bfull + bi, (j >> 1) & 1, sabort, poller)) break;
       if (wg_front && !group_wait<FrontSync>(wfull + bi, (j >> 1) & 1, sabort, poller)) break;
+      if (kMuir && !group_wait<FrontSync>(qready + bi, (j >> 1) & 1, sabort, poller)) break;
       if (poller) {
         cnt[kLDone] = j + 1;
         cnt[kBDone0 + bi] += 1;
@@ -409,7 +394,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
       if constexpr (kMuir) {
         // log alpha = -exp(a_log[h]) softplus(z_f); tokens past T keep the state (log alpha
         // = 0), as the zero-filled log w of the plain path does
-        const float rate = __expf(p.a_log[bh_of(item) % H]);
+        const float rate = __expf(a_log);
         const int tpad = T - c_of(item) * kC;
         const __nv_bfloat16 *zl = reinterpret_cast<const __nv_bfloat16 *>(smem + SL::SLW);
 #pragma unroll
@@ -533,25 +518,17 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
             }
             unpack8(*reinterpret_cast<const uint4 *>(buf + oq), q8);
             if constexpr (kMuir) {
-              // k = l2norm(silu(k)), q^ = gamma_stat 2 sigmoid(z_q) l2norm(silu(q)), b = 2 sigmoid(z_b)
-              float zq8[8];
-              unpack8(zq_raw[i], zq8);
+              // k = l2norm(silu(k)), b = 2 sigmoid(z_b); the q tile already holds q^ (the
+              // back group's activate_q)
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 k8[e] = silu_f(k8[e]);
-                q8[e] = silu_f(q8[e]);
                 b8[e] = 2.f * sigmoid_f(b8[e]);
               }
-              const float nk = inv_norm16(k8), nq = inv_norm16(q8);
+              const float nk = inv_norm16(k8);
 #pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                k8[e] *= nk;
-                q8[e] *= nq * gs8[e] * 2.f * sigmoid_f(zq8[e]);
-              }
-              if (g == 0) {
-                sNRM[bi * 2 * kC + t] = nq;
-                sNRM[bi * 2 * kC + kC + t] = nk;
-              }
+              for (int e = 0; e < 8; ++e) k8[e] *= nk;
+              if (g == 0) sNRM[bi * 2 * kC + kC + t] = nk;
             }
             float av[8], aq[8], bl[8], kt[8], qp[8];
 #pragma unroll
@@ -635,7 +612,56 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
   } else {
     // =========================================================== back group
     const bool poller = gt == 0;
-    for (int j = 0; j < nloc; ++j) {
+    // Muir: q^ = gamma_stat 2 sigmoid(z_q) l2norm(silu(q)) in place in chunk jq's q tile,
+    // once its tiles have landed; then the front group may form Q f from it.  The back
+    // group does this for chunk j + 2 after its own chunk j, in time it would otherwise
+    // spend waiting for the front group.  Returns false when the CTA aborts.
+    auto activate_q = [&](int jq) -> bool {
+      const int bq = jq & 1;
+      if (!group_wait<BackSync>(bfull + bq, (jq >> 1) & 1, sabort, poller)) return false;
+      const int g = gt & 15, tb = gt >> 4, j0 = 8 * g;
+      const int it = item_of(jq), bh = bh_of(it), hh = bh % H, t0 = c_of(it) * kC;
+      uint4 zq_raw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int tt = t0 + 4 * tb + i;
+        zq_raw[i] = tt < T ? ld16(gzq + (((size_t)(bh / H) * T + tt) * H + hh) * kDK + j0)
+                           : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float gs8[8];
+      if (p.gamma_stat) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0));
+        const float4 c = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0 + 4));
+        gs8[0] = a.x; gs8[1] = a.y; gs8[2] = a.z; gs8[3] = a.w;
+        gs8[4] = c.x; gs8[5] = c.y; gs8[6] = c.z; gs8[7] = c.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) gs8[e] = 1.f;
+      }
+      uint8_t *qb = smem + bq * SL::BUF;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 4 * tb + i;
+        const uint32_t oq = SL::A_LM + sw128_offset(kC + t, j0, 2 * kC * 128);
+        float q8[8], zq8[8];
+        unpack8(*reinterpret_cast<const uint4 *>(qb + oq), q8);
+        unpack8(zq_raw[i], zq8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q8[e] = silu_f(q8[e]);
+        const float nq = inv_norm16(q8);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q8[e] *= nq * gs8[e] * 2.f * sigmoid_f(zq8[e]);
+        st_smem16(qb, oq, pack8(q8));
+        if (g == 0) sNRM[bq * 2 * kC + t] = nq;
+      }
+      BackSync::sync();
+      if (poller) mbar_arrive(qready + bq);
+      return true;
+    };
+    bool live = true;
+    if constexpr (kMuir)
+      for (int jq = 0; jq < 2 && jq < nloc && live; ++jq) live = activate_q(jq);
+    for (int j = 0; j < nloc && live; ++j) {
       const int item = item_of(j), c = c_of(item), bh = bh_of(item), h = bh % H, b = bh / H;
       const int t0 = c * kC, n = min(kC, T - t0), bi = j & 1;
       uint8_t *buf = smem + bi * SL::BUF;
@@ -817,6 +843,8 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
       BackSync::sync();          // U / Y read before the next MMA2 overwrites them
       if (flags && gt == 0) publish(flags + (size_t)bh * nch + c);
       GDR_PREP_PHASE(13);
+      if constexpr (kMuir)
+        if (j + 2 < nloc && !activate_q(j + 2)) break;
     }
   }
 
