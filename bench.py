@@ -382,6 +382,9 @@ def bench_other_workloads(ctx, args, gdr):
         ws = gdr.new_workspace(gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"],
                                                               d["log_w"], d["e1"], d["e2"],
                                                               w.chunk, args.algo), ctx.dev)
+        kernel = gdr.gdr_forward_kernel_name(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
+                                             d["e2"], chunk=w.chunk, algo=args.algo,
+                                             workspace_bytes=ws.numel())
 
         def call():
             return gdr.gdr_forward_chunked(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
@@ -405,7 +408,8 @@ def bench_other_workloads(ctx, args, gdr):
         gbs = nbytes / (ms * 1e-3) / 1e9
         nbytes_wg = fwd_algorithmic_bytes(w, with_write_gate=True)
         out.append({"workload": name, "form": w.form, "dtype": w.dtype, "B": w.B, "H": w.H,
-                    "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "ms_per_call": ms,
+                    "T": w.T, "dk": w.dk, "dv": w.dv, "chunk": w.chunk, "kernel": kernel,
+                    "ms_per_call": ms,
                     "tokens_per_s": w.tokens * ctx.world / (ms * 1e-3),
                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": ctx.peaks["hbm_gbs"],
                                  "unit": "GB/s", "frac": gbs / ctx.peaks["hbm_gbs"],

@@ -86,16 +86,24 @@ typedef enum {
 
 /* Kernel selection for gdr_forward_chunked. */
 typedef enum {
-  GDR_ALGO_AUTO = 0,   /* tensor-core kernel where it applies, else the fp32 kernel        */
+  GDR_ALGO_AUTO = 0,   /* tensor-core kernel where it applies, else the token-recurrent
+                          kernel (measured faster than the fp32 chunkwise kernel on every
+                          fp32 shape tried, from B=1, H=2, T=256 to B=8, H=32, T=2048)      */
   GDR_ALGO_FP32 = 1,   /* fp32 CUDA-core kernel: every product in fp32 (all forms, all dtypes) */
-  GDR_ALGO_TC = 2      /* tcgen05/TMEM kernels: bf16 operands, fp32 accumulate and state.
+  GDR_ALGO_TC = 2,     /* tcgen05/TMEM kernels: bf16 operands, fp32 accumulate and state.
                           They apply to bf16 inputs with chunk >= 64 for
                             GDN2, dk = dv = 128: two kernels with a per-chunk record
                                  workspace, or one kernel with the status word only;
                             GLA, dk = dv = 128: the two kernels (GDR_ERR_WORKSPACE
-                                 without the record workspace; AUTO then takes fp32);
+                                 without the record workspace; AUTO then takes the
+                                 token-recurrent kernel);
                             every form, dk = dv = 64: one kernel, status word only;
                           GDR_ERR_UNSUPPORTED elsewhere.                                  */
+  GDR_ALGO_RECURRENT = 3  /* the recurrence token by token (fp32 state in registers, one warp
+                          per value column; all forms, dtypes and sizes; no workspace).  No
+                          chunk parallelism: its time grows with T at a fixed cost per token,
+                          which for few heads and short sequences is far below the chunkwise
+                          kernels' cost per chunk.  The chunk length is ignored.        */
 } gdr_algo;
 
 /*
@@ -132,6 +140,17 @@ typedef struct {
 gdr_status gdr_forward_workspace_size(const gdr_fwd_args *args, size_t *bytes);
 
 /*
+ * Which kernel gdr_forward_chunked runs for these arguments, workspace included (host-only:
+ * no CUDA call and no pointer dereferenced; the same checks, so a call it rejects returns the
+ * same status).  *name is a
+ * static string: "none" (no work), "copy_state" (T = 0: S_T = S0), "tc_two_stream" (every
+ * form at d = 64 on tcgen05), "tc_split" (prep and chain kernels with per-chunk records),
+ * "tc_single" (one tensor-core kernel), "fp32" (the fp32 chunkwise kernel) or "recurrent"
+ * (the token-recurrent kernel).
+ */
+gdr_status gdr_forward_kernel_name(const gdr_fwd_args *args, const char **name);
+
+/*
  * Chunkwise-parallel forward over whole sequences: for every (b, h) runs the
  * recurrence over t = 1..T from S0 and writes every o_t and, if S_T != NULL, the
  * final state.  Chunkwise algorithm: "Muir ...", section 2.2 (effective write,
@@ -164,11 +183,11 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *args, void *stream);
  *   - GDN2, bf16, dk = dv = 128, algo AUTO or TC: the single-kernel tensor-core
  *     forward (not the faster two-kernel one, whose records do not fit);
  *   - GLA, bf16, dk = dv = 128: algo TC returns GDR_ERR_WORKSPACE; algo AUTO runs
- *     the fp32 kernel;
+ *     the token-recurrent kernel;
  *   - every form at bf16, dk = dv = 64, algo AUTO or TC: the two-stream
  *     tensor-core kernel, as gdr_forward_chunked;
- *   - everything else (algo FP32, fp32 inputs, other sizes): the fp32 kernel, as
- *     gdr_forward_chunked.
+ *   - everything else: algo FP32 the fp32 chunkwise kernel, algo AUTO or RECURRENT
+ *     (fp32 inputs, other sizes) the token-recurrent kernel, as gdr_forward_chunked.
  * The results are those of the kernel named, within the same error bars.
  *
  *   - Arguments are checked on the host, as gdr_forward_chunked checks them, before

@@ -167,7 +167,7 @@ gdr_status forward_plan(const gdr_fwd_args *a, const void *workspace, size_t wor
   if (!form_ok(a->form) || !dtype_ok(a->dtype)) return GDR_ERR_INVALID_ARG;
   if (a->B < 0 || a->H < 0 || a->T < 0) return GDR_ERR_INVALID_ARG;
   if (!dim_ok(a->dk) || !dim_ok(a->dv) || !chunk_ok(a->chunk)) return GDR_ERR_UNSUPPORTED;
-  if (a->algo < GDR_ALGO_AUTO || a->algo > GDR_ALGO_TC) return GDR_ERR_INVALID_ARG;
+  if (a->algo < GDR_ALGO_AUTO || a->algo > GDR_ALGO_RECURRENT) return GDR_ERR_INVALID_ARG;
   const size_t tokens = (size_t)a->B * a->T * a->H;
   gdr_status st = check_token_ptrs(a->form, tokens, a->q, a->k, a->v, a->log_w, a->e1, a->e2,
                                    a->o);
@@ -183,6 +183,11 @@ gdr_status forward_plan(const gdr_fwd_args *a, const void *workspace, size_t wor
     return GDR_OK;
   }
   const FwdParams p = fwd_params(a);
+  if (a->algo == GDR_ALGO_RECURRENT) {
+    if (!forward_recur_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
+    *path = FwdPath::kRecur;   // needs no workspace
+    return GDR_OK;
+  }
   if (uses_tc_general(a, p)) {   // two-stream forms, d = 64: one fused kernel, status word only
     if (workspace_bytes < kStatusBytes) return GDR_ERR_WORKSPACE;
     *path = FwdPath::kTcGeneral;
@@ -203,6 +208,12 @@ gdr_status forward_plan(const gdr_fwd_args *a, const void *workspace, size_t wor
       return GDR_OK;
     }
     if (a->algo == GDR_ALGO_TC) return GDR_ERR_WORKSPACE;
+  }
+  // AUTO without a tensor-core path: the token recurrence, which ran faster than the fp32
+  // chunkwise kernel on every shape measured (that kernel stays behind GDR_ALGO_FP32)
+  if (a->algo == GDR_ALGO_AUTO && forward_recur_supported(a->dk, a->dv)) {
+    *path = FwdPath::kRecur;
+    return GDR_OK;
   }
   if (!forward_fp32_supported(a->dk, a->dv)) return GDR_ERR_UNSUPPORTED;
   *path = FwdPath::kFp32;     // needs no workspace (a status word is used when given)
@@ -253,6 +264,24 @@ gdr_status gdr_state_init(float *S, int B, int H, int dk, int dv, const float *s
   return cuda_status(cudaMemsetAsync(S, 0, n * sizeof(float), st));
 }
 
+gdr_status gdr_forward_kernel_name(const gdr_fwd_args *a, const char **name) {
+  if (!name) return GDR_ERR_INVALID_ARG;
+  gdr::FwdPath path;
+  const gdr_status st = gdr::forward_plan(a, a ? a->workspace : nullptr, a ? a->workspace_bytes : 0,
+                                          &path);
+  if (st != GDR_OK) return st;
+  switch (path) {
+    case gdr::FwdPath::kNone: *name = "none"; break;
+    case gdr::FwdPath::kCopyState: *name = "copy_state"; break;
+    case gdr::FwdPath::kTcGeneral: *name = "tc_two_stream"; break;
+    case gdr::FwdPath::kTcSplit: *name = "tc_split"; break;
+    case gdr::FwdPath::kTcSingle: *name = "tc_single"; break;
+    case gdr::FwdPath::kRecur: *name = "recurrent"; break;
+    default: *name = "fp32"; break;
+  }
+  return GDR_OK;
+}
+
 gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
   gdr::FwdPath path;
   const gdr_status st = gdr::forward_plan(a, a ? a->workspace : nullptr, a ? a->workspace_bytes : 0,
@@ -267,12 +296,14 @@ gdr_status gdr_forward_chunked(const gdr_fwd_args *a, void *stream) {
     default:
       break;
   }
-  if (path != gdr::FwdPath::kFp32 && !a->workspace) return GDR_ERR_WORKSPACE;
+  if (path != gdr::FwdPath::kFp32 && path != gdr::FwdPath::kRecur && !a->workspace)
+    return GDR_ERR_WORKSPACE;
   const gdr::FwdParams p = fwd_params(a);
   switch (path) {
     case gdr::FwdPath::kTcGeneral: return cuda_status(gdr::launch_forward_tc_general(p, s));
     case gdr::FwdPath::kTcSplit: return cuda_status(gdr::launch_forward_tc_split(p, a->workspace, s));
     case gdr::FwdPath::kTcSingle: return cuda_status(gdr::launch_forward_tc(p, s));
+    case gdr::FwdPath::kRecur: return cuda_status(gdr::launch_forward_recur(p, a->dtype, s));
     default: return cuda_status(gdr::launch_forward_fp32(p, a->dtype, s));
   }
 }

@@ -122,6 +122,8 @@ cudaError_t fill_f32(float *p, size_t n, float x, cudaStream_t stream);
 cudaError_t launch_decode(const gdr_step_args &a, cudaStream_t stream);
 cudaError_t launch_forward_fp32(const FwdParams &p, gdr_dtype dtype, cudaStream_t stream);
 bool forward_fp32_supported(int dk, int dv);
+cudaError_t launch_forward_recur(const FwdParams &p, gdr_dtype dtype, cudaStream_t stream);
+bool forward_recur_supported(int dk, int dv);
 cudaError_t launch_forward_tc(const FwdParams &p, cudaStream_t stream);
 bool forward_tc_supported(const FwdParams &p, gdr_dtype dtype);
 // Tensor-core path for the two-stream forms (general, RWKV-7), d_k = d_v = 64: one
@@ -137,7 +139,7 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
 constexpr size_t kStatusBytes = 256;
 
 // Which kernel gdr_forward_chunked runs for given arguments and workspace size.
-enum class FwdPath { kNone, kCopyState, kTcGeneral, kTcSplit, kTcSingle, kFp32 };
+enum class FwdPath { kNone, kCopyState, kTcGeneral, kTcSplit, kTcSingle, kFp32, kRecur };
 // Host validation and selection (no CUDA call): every check gdr_forward_chunked makes on
 // its arguments and on a workspace at `workspace` (alignment; may be null) of
 // `workspace_bytes` bytes, except that a null workspace on a path that needs one is

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_PKG, "libgdr.so")
 
 FORMS = {"general": 0, "gdn2": 1, "rwkv7": 2, "gla": 3}
 DTYPES = {"f32": 0, "bf16": 1}
-ALGOS = {"auto": 0, "fp32": 1, "tc": 2}
+ALGOS = {"auto": 0, "fp32": 1, "tc": 2, "recurrent": 3}
 STATUS = {0: "GDR_OK", 1: "GDR_ERR_INVALID_ARG", 2: "GDR_ERR_UNSUPPORTED",
           3: "GDR_ERR_MISALIGNED", 4: "GDR_ERR_CUDA", 5: "GDR_ERR_DEVICE_CHECK",
           6: "GDR_ERR_TIMEOUT", 7: "GDR_ERR_WORKSPACE"}
@@ -81,6 +81,8 @@ def _declare(lib):
     lib.gdr_forward_chunked.argtypes = [ctypes.POINTER(gdr_fwd_args), _vp]
     lib.gdr_forward_workspace_size.argtypes = [ctypes.POINTER(gdr_fwd_args),
                                                ctypes.POINTER(ctypes.c_size_t)]
+    lib.gdr_forward_kernel_name.argtypes = [ctypes.POINTER(gdr_fwd_args),
+                                            ctypes.POINTER(ctypes.c_char_p)]
     lib.gdr_backward_chunked.argtypes = [ctypes.POINTER(gdr_bwd_args), _vp]
     lib.gdr_backward_workspace_size.argtypes = [ctypes.POINTER(gdr_bwd_args),
                                                 ctypes.POINTER(ctypes.c_size_t)]
@@ -94,7 +96,7 @@ def _declare(lib):
     lib.gdr_read_status.argtypes = [_vp, _vp, ctypes.POINTER(_c_int)]
     lib.gdr_status_string.restype = ctypes.c_char_p
     lib.gdr_status_string.argtypes = [_c_int]
-    for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size",
+    for fn in ("gdr_forward_chunked", "gdr_forward_workspace_size", "gdr_forward_kernel_name",
                "gdr_backward_chunked", "gdr_backward_workspace_size",
                "gdr_muir_forward", "gdr_muir_workspace_size", "gdr_mlstm_forward",
                "gdr_state_compose",
@@ -173,7 +175,7 @@ def _e_shapes(form, lead, dk, dv):
     return None, None
 
 
-def _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, workspace):
+def _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, workspace, o_ptr=None):
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dname, tdt = _dtype_of(q)
@@ -188,14 +190,16 @@ def _fwd_struct(form, q, k, v, log_w, e1, e2, S0, o, S_T, chunk, algo, workspace
         _need(e2, "e2", tdt, s2)
     if S0 is not None:
         _need(S0, "S0", torch.float32, (B, H, dk, dv))
-    _need(o, "o", torch.float32, (B, T, H, dv))
+    if o_ptr is None:
+        _need(o, "o", torch.float32, (B, T, H, dv))
     if S_T is not None:
         _need(S_T, "S_T", torch.float32, (B, H, dk, dv))
     a = gdr_fwd_args()
     a.form, a.dtype, a.algo = FORMS[form], DTYPES[dname], ALGOS[algo]
     a.B, a.H, a.T, a.dk, a.dv, a.chunk = B, H, T, dk, dv, chunk
     a.q, a.k, a.v, a.log_w = _ptr(q), _ptr(k), _ptr(v), _ptr(log_w)
-    a.e1, a.e2, a.S0, a.o, a.S_T = _ptr(e1), _ptr(e2), _ptr(S0), _ptr(o), _ptr(S_T)
+    a.e1, a.e2, a.S0, a.S_T = _ptr(e1), _ptr(e2), _ptr(S0), _ptr(S_T)
+    a.o = _ptr(o) if o_ptr is None else o_ptr
     if workspace is not None:
         a.workspace = _ptr(_workspace(workspace))
         a.workspace_bytes = workspace.numel() * workspace.element_size()
@@ -212,6 +216,23 @@ def gdr_forward_workspace_size(form, q, k, v, log_w, e1=None, e2=None, chunk=64,
     _check("gdr_forward_workspace_size",
            _load().gdr_forward_workspace_size(ctypes.byref(a), ctypes.byref(n)))
     return int(n.value)
+
+
+def gdr_forward_kernel_name(form, q, k, v, log_w, e1=None, e2=None, S0=None, *, chunk=64,
+                            algo="auto", workspace_bytes=None):
+    """The kernel ``gdr_forward_chunked`` runs for these inputs (a host-only query): with
+    ``workspace_bytes`` None, the workspace it allocates by default."""
+    B, T, H, dk = q.shape
+    if workspace_bytes is None:
+        workspace_bytes = gdr_forward_workspace_size(form, q, k, v, log_w, e1, e2, chunk, algo)
+    # o and the workspace: the query checks only that they are given and aligned
+    a = _fwd_struct(form, q, k, v, log_w, e1, e2, S0, None, None, chunk, algo, None,
+                    o_ptr=ctypes.c_void_p(256))
+    a.workspace = ctypes.c_void_p(256)
+    a.workspace_bytes = int(workspace_bytes)
+    name = ctypes.c_char_p()
+    _check("gdr_forward_kernel_name", _load().gdr_forward_kernel_name(ctypes.byref(a), ctypes.byref(name)))
+    return name.value.decode()
 
 
 def new_workspace(nbytes, device):

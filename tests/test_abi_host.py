@@ -67,6 +67,50 @@ def test_forward_rejects_bad_arguments_on_host(lib, kw, code):
     assert lib.gdr_forward_chunked(ctypes.byref(a), None) == code
 
 
+def _kernel_name(lib, a):
+    name = ctypes.c_char_p()
+    rc = lib.gdr_forward_kernel_name(ctypes.byref(a), ctypes.byref(name))
+    return rc, (name.value.decode() if rc == 0 else None)
+
+
+def _tc_split_bytes(lib, a):
+    n = ctypes.c_size_t(0)
+    assert lib.gdr_forward_workspace_size(ctypes.byref(a), ctypes.byref(n)) == 0
+    return n.value
+
+
+def test_forward_kernel_selection(lib):
+    """The host-side plan of gdr_forward_chunked, as the name query reports it (no GPU)."""
+    ws = ctypes.c_void_p(0x100000)
+    # GDN-2 bf16 d = 128: two kernels with the record workspace, one kernel with the status
+    # word only; fp32 inputs take the token recurrence under AUTO and the chunkwise fp32
+    # kernel under FP32
+    big = _args(dk=128, dv=128, T=4096, H=16, B=4)
+    need = _tc_split_bytes(lib, big)
+    assert need > 4096
+    assert _kernel_name(lib, _args(dk=128, dv=128, T=4096, H=16, B=4, workspace=ws,
+                                   workspace_bytes=need)) == (0, "tc_split")
+    assert _kernel_name(lib, _args(dk=128, dv=128, T=4096, H=16, B=4, workspace=ws,
+                                   workspace_bytes=256)) == (0, "tc_single")
+    assert _kernel_name(lib, _args(dk=128, dv=128, dtype=0, workspace=ws,
+                                   workspace_bytes=256)) == (0, "recurrent")
+    assert _kernel_name(lib, _args(dtype=0, algo=1)) == (0, "fp32")
+    assert _kernel_name(lib, _args(dtype=0, algo=3)) == (0, "recurrent")
+    # every form at bf16, d = 64: the two-stream tensor-core kernel (status word only)
+    assert _kernel_name(lib, _args(workspace=ws, workspace_bytes=256)) == (0, "tc_two_stream")
+    # bf16 at d = 64 without the status word: GDR_ERR_WORKSPACE, as the forward itself
+    assert _kernel_name(lib, _args())[0] == 7
+    # no tokens: S_T = S0; no sequences: nothing
+    assert _kernel_name(lib, _args(T=0, S_T=ctypes.c_void_p(0x20000))) == (0, "copy_state")
+    assert _kernel_name(lib, _args(B=0)) == (0, "none")
+    # the same host checks as the forward
+    assert _kernel_name(lib, _args(dk=48))[0] == 2
+    assert _kernel_name(lib, _args(algo=7))[0] == 1
+    name = ctypes.c_char_p()
+    assert lib.gdr_forward_kernel_name(ctypes.byref(_args()), None) == 1
+    assert lib.gdr_forward_kernel_name(None, ctypes.byref(name)) == 1
+
+
 def test_forward_zero_batch_is_a_noop(lib):
     a = _args(B=0, q=None, k=None, v=None, log_w=None, e1=None, o=None)
     assert lib.gdr_forward_chunked(ctypes.byref(a), None) == 0

@@ -42,8 +42,10 @@ def _case(form, d, seed=9):
 # (form, d, algo, the allocating call's workspace that selects the same kernel):
 #   GDN-2 d = 128: the single-kernel tensor-core forward (status word only, 256 bytes)
 #   RWKV-7 d = 64: the two-stream tensor-core kernel
-#   GLA d = 128 with algo auto: the fp32 kernel (the tensor-core path needs records)
-CASES = [("gdn2", 128, "tc", 256), ("rwkv7", 64, "auto", 256), ("gla", 128, "auto", 256)]
+#   GLA d = 128 with algo auto: the token-recurrent kernel (the tensor-core path needs records)
+#   GLA d = 128 with algo fp32: the fp32 chunkwise kernel
+CASES = [("gdn2", 128, "tc", 256), ("rwkv7", 64, "auto", 256), ("gla", 128, "auto", 256),
+         ("gla", 128, "fp32", 256)]
 
 
 @pytest.mark.parametrize("form,d,algo,ws", CASES)
