@@ -353,16 +353,15 @@ def bench_forward(ctx, args, gdr):
         raise RuntimeError(f"device status after the timed steps: {status}")
     ms_total = ctx.max_over_ranks(t0.elapsed_time(t1))
     ms_kernel = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    # launches per call: the tensor-core path with a full workspace runs a prep and a
-    # chain kernel; every other path is one kernel
-    full_ws = ws.numel() >= gdr.gdr_forward_workspace_size(w.form, d["q"], d["k"], d["v"],
-                                                            d["log_w"], d["e1"], d["e2"],
-                                                            w.chunk, "tc") > 256
-    per_call = 2 if (args.algo in ("auto", "tc") and full_ws and w.form == "gdn2"
-                     and w.dtype == "bf16" and w.dk == w.dv == 128 and w.chunk in (64, 128)) else 1
+    # launches per call: the two-kernel tensor-core path runs a prep and a chain kernel;
+    # every other path is one kernel
+    kernel = gdr.gdr_forward_kernel_name(w.form, d["q"], d["k"], d["v"], d["log_w"], d["e1"],
+                                         d["e2"], chunk=w.chunk, algo=args.algo,
+                                         workspace_bytes=ws.numel())
+    per_call = 2 if kernel == "tc_split" else 1
     res = {"w": w, "ms_per_step": ms_total / args.steps, "ms_kernel": ms_kernel,
            "clocks": clk.summary(), "launches": args.steps * per_call,
-           "launches_per_call": per_call}
+           "launches_per_call": per_call, "kernel": kernel}
     if args.only == "all":
         res["e2e"] = bench_e2e(ctx, args, gdr, w, inp, names, ws)
     return res
@@ -771,6 +770,7 @@ def main():
                        "l2": f"inputs larger than L2 ({nbytes / 2**20:.0f} MiB per step > 126 MiB)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": ctx.peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / ctx.peaks["hbm_gbs"],
+                         "kernel_path": fwd["kernel"],
                          "traffic": (FWD_TC_TRAFFIC_PER_CHUNK * w.B * w.H * -(-w.T // 64)
                                      if fwd["launches_per_call"] == 2 else None),
                          "peak_source": ctx.peaks["source"],
