@@ -890,26 +890,31 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 //          D[c&1] += [M; *] V~             (M = 128, K = C; rows C..2C-1 are discarded)
 //   S <- Diag(pi_n) S + DS                 (fp32, all warps)
 //   O = rows 0..C-1 of D[c&1]              (read while MMA3 of chunk c + 1 runs)
-// Warp 0 issues the MMAs (lane 0, from converged code); warp 2 refills the record
-// ring (three records for NV = 64, two for NV = 128, the size shared memory allows) as
-// soon as MMA4 has released a buffer.  NV = 128 runs 512 threads, 32 columns each.
+// Warp 0 issues the MMAs (lane 0, from converged code); warp 1 refills the record
+// ring (three records for NV = 32 and 64, two for NV = 128, the size shared memory
+// allows) as soon as MMA4 has released a buffer.  Threads: 32 value columns each (NV = 32
+// runs 128 threads, 128 runs 512).  NV = 32 (few long sequences: twice the chains, half
+// the vector work per step) keeps S0's bf16 copy and V~ in the 64-byte swizzle, whose atom
+// is the slice's 32 columns, and fetches the whole 64-column block of U that holds them.
 template <int NV>
 struct ChainSmem {
-  // per buffer: QY | KT | MM | U slice (C x NV) | pi.  The U slice sits directly after
-  // M, so [M; U slice] is a valid 128-row K-major operand whose lower half only
-  // feeds accumulator rows that are discarded.
-  static constexpr int NBUF = NV == 64 ? 3 : 2;                // records in the ring
-  static constexpr int NT = NV == 64 ? 256 : 512;               // threads: 32 columns each
-  static constexpr uint32_t TMEM_COLS = NV == 64 ? 256 : 512;   // D x 2 and DS, NV columns each
+  // per buffer: QY | KT | MM | U block(s) (C x UB) | pi.  The U block sits directly after
+  // M, so [M; U] is a valid 128-row K-major operand whose lower half only feeds
+  // accumulator rows that are discarded.
+  static constexpr int UB = NV == 32 ? 64 : NV;                // U columns fetched
+  static constexpr int NBUF = NV == 128 ? 2 : 3;               // records in the ring
+  static constexpr int NT = 4 * NV;                            // threads: 32 columns each
+  static constexpr uint32_t TMEM_COLS = NV == 32 ? 128 : 4 * NV;   // D x 2 and DS, NV columns each
   static constexpr uint32_t B_U = Rec::FRONT;
-  static constexpr uint32_t B_PI = B_U + kC * NV * 2;
+  static constexpr uint32_t B_PI = B_U + kC * UB * 2;
   static constexpr uint32_t BUF = ((B_PI + kDK * 4 + 1023) / 1024) * 1024;
   static constexpr uint32_t S0B = NBUF * BUF;                 // bf16 S0   DK x NV
   static constexpr uint32_t VT = S0B + kDK * NV * 2;          // bf16 V~   C x NV
   static constexpr uint32_t MISC = VT + kC * NV * 2;          // barriers, TMEM slot, flags
   static constexpr uint32_t ALLOC = MISC + 128 + 1024;
-  static constexpr uint32_t TX = Rec::FRONT + kC * NV * 2 + kDK * 4;  // bytes per record fetch
-  static_assert(NV == 64 || NV == 128, "one or both 64-column blocks of U per CTA");
+  static constexpr uint32_t TX = Rec::FRONT + kC * UB * 2 + kDK * 4;  // bytes per record fetch
+  static_assert(NV == 32 || NV == 64 || NV == 128, "a half, one or both 64-column blocks of U");
+  static_assert(VT % 1024 == 0 && S0B % 1024 == 0, "swizzled operand tiles aligned");
   static_assert(B_U == Rec::MM + kC * kC * 2,
                 "[M; first 64 columns of U] must form one 128-row operand");
   static_assert(ALLOC <= 227 * 1024, "shared memory");
@@ -937,7 +942,8 @@ __device__ __forceinline__ void fetch_record(uint8_t *smem, uint64_t *full, uint
   ++fiss[buf];
   mbar_arrive_expect_tx(full + buf, SL::TX);
   bulk_g2s(dst, src, Rec::FRONT, full + buf);
-  bulk_g2s(dst + SL::B_U, src + Rec::U + slice * (kC * 128), kC * NV * 2, full + buf);
+  const int ublk = NV == 32 ? slice >> 1 : slice;      // the 64-column block(s) of U
+  bulk_g2s(dst + SL::B_U, src + Rec::U + ublk * (kC * 128), kC * SL::UB * 2, full + buf);
   bulk_g2s(dst + SL::B_PI, src + Rec::PI, kDK * 4, full + buf);
 }
 
@@ -981,6 +987,13 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
   using SL = ChainSmem<NV>;
   constexpr int NBUF = SL::NBUF, NT = SL::NT;
   constexpr int HALF = 32;      // value columns per thread: NT / 128 column groups of 32
+  // bf16 S0 copy and V~ (MN-major B operands of N = NV): byte offsets and descriptors
+  auto s0_off = [](int row, int col) -> uint32_t {
+    return NV == 32 ? sw64_offset(row, col) : sw128_offset(row, col, kDK * 128);
+  };
+  auto vt_off = [](int row, int col) -> uint32_t {
+    return NV == 32 ? sw64_offset(row, col) : sw128_offset(row, col, kC * 128);
+  };
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
@@ -1040,7 +1053,7 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
   }
 #pragma unroll
   for (int i = 0; i < HALF; i += 8)
-    st_smem16(smem, SL::S0B + sw128_offset(jrow, hf * HALF + i, kDK * 128), pack8(st + i));
+    st_smem16(smem, SL::S0B + s0_off(jrow, hf * HALF + i), pack8(st + i));
   fence_proxy_async_smem();
   tc_fence_before();
   ChainSync<NT>::sync();
@@ -1071,7 +1084,8 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
 #pragma unroll
     for (int s = 0; s < kDK / 16; ++s) {
       const uint64_t a = sdesc_sw128(bb + Rec::QY + (s >> 2) * Rec::QY_STRIDE + (s & 3) * 32, 16, 1024);
-      const uint64_t bs = sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
+      const uint64_t bs = NV == 32 ? sdesc_sw64(sb + SL::S0B + s * 1024, kDK * 64, 512)
+                                   : sdesc_sw128(sb + SL::S0B + s * 2048, kDK * 128, 1024);
       mma_bf16_warp(tmem + NV * (c & 1), a, bs, id, s > 0);
     }
     mma_commit_warp(bar3);
@@ -1112,10 +1126,11 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
 #pragma unroll
       for (int i = 0; i < HALF; i += 8) {
         float u8[8];
-        unpack8(*reinterpret_cast<const uint4 *>(bsm + SL::B_U + sw128_offset(t, hf * HALF + i, kC * 128)), u8);
+        const int ucol = (NV == 32 ? (slice & 1) * 32 : hf * HALF) + i;   // column in the U block
+        unpack8(*reinterpret_cast<const uint4 *>(bsm + SL::B_U + sw128_offset(t, ucol, kC * 128)), u8);
 #pragma unroll
         for (int e = 0; e < 8; ++e) u8[e] = (t < n) ? u8[e] - d[i + e] : 0.f;
-        st_smem16(smem, SL::VT + sw128_offset(t, hf * HALF + i, kC * 128), pack8(u8));
+        st_smem16(smem, SL::VT + vt_off(t, hf * HALF + i), pack8(u8));
       }
     }
     fence_proxy_async_smem();
@@ -1132,7 +1147,8 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
 #pragma unroll
       for (int s = 0; s < kC / 16; ++s) {
         const uint64_t ak = sdesc_sw128(bb + Rec::KT + s * 2048, kC * 128, 1024);
-        const uint64_t bv = sdesc_sw128(sb + SL::VT + s * 2048, kC * 128, 1024);
+        const uint64_t bv = NV == 32 ? sdesc_sw64(sb + SL::VT + s * 1024, kC * 64, 512)
+                                     : sdesc_sw128(sb + SL::VT + s * 2048, kC * 128, 1024);
         const uint64_t am = sdesc_sw128(bb + Rec::MM + s * 32, 16, 1024);
         mma_bf16_warp(tDS, ak, bv, ids, s > 0);
         mma_bf16_warp(tD, am, bv, ido, 1);
@@ -1162,7 +1178,7 @@ __device__ __forceinline__ void chain_body(const FwdParams &p, const uint8_t *re
       for (int i = 0; i < HALF; ++i) st[i] = pn * st[i] + d[i];
 #pragma unroll
       for (int i = 0; i < HALF; i += 8)
-        st_smem16(smem, SL::S0B + sw128_offset(jrow, hf * HALF + i, kDK * 128), pack8(st + i));
+        st_smem16(smem, SL::S0B + s0_off(jrow, hf * HALF + i), pack8(st + i));
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -1271,6 +1287,32 @@ bool encode_input_map(CUtensorMap *m, const void *base, CUtensorMapDataType type
   return tma::encode_input_map(m, base, type, elem, box0, kC, swizzle, p.H, p.T, p.B);
 }
 
+// The one-launch path with value slices of NV columns (tc_fused_kernel): one CTA per SM,
+// the first B H (d_v / NV) running the chains.  *launched stays false when the kernel
+// cannot keep one CTA resident per SM (the caller then takes the two launches).
+template <int NV>
+cudaError_t launch_fused(const FwdParams &p, uint8_t *records, const PrepMaps &maps, int sms,
+                         int items, cudaStream_t stream, bool *launched) {
+  *launched = false;
+  auto fused = p.muir ? tc_fused_kernel<true, NV> : tc_fused_kernel<false, NV>;
+  const int smem = (int)(PrepSmem::ALLOC > ChainSmem<NV>::ALLOC ? PrepSmem::ALLOC : ChainSmem<NV>::ALLOC);
+  cudaError_t e = cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused, kPrepThreads, smem)) != cudaSuccess)
+    return e;
+  if (per_sm < 1) return cudaSuccess;
+  uint32_t *flags = reinterpret_cast<uint32_t *>(records + (size_t)items * Rec::BYTES);
+  if ((e = cudaMemsetAsync(flags, 0, (size_t)items * 4, stream)) != cudaSuccess) return e;
+  FwdParams pp = p;
+  PrepMaps mm = maps;
+  int nchain = (p.dv / NV) * p.H * p.B;
+  void *args[] = {&pp, &records, &mm, &flags, &nchain};
+  *launched = true;
+  return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(fused), dim3(sms), dim3(kPrepThreads),
+                                     args, (size_t)smem, stream);
+}
+
 }  // namespace
 
 cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStream_t stream) {
@@ -1305,24 +1347,17 @@ cudaError_t launch_forward_tc_split(const FwdParams &p, void *workspace, cudaStr
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int nch = num_chunks(p.T);
   const int items = p.B * p.H * nch;
-  int nchain = (p.dv / NV) * p.H * p.B;
-  if (nchain * 3 <= sms && nch >= kFusedMinChunks) {
-    // few long sequences: chains and prep in one cooperative launch (tc_fused_kernel)
-    auto fused = p.muir ? tc_fused_kernel<true, NV> : tc_fused_kernel<false, NV>;
-    const int smem = (int)(PrepSmem::ALLOC > ChainSmem<NV>::ALLOC ? PrepSmem::ALLOC : ChainSmem<NV>::ALLOC);
-    if ((e = cudaFuncSetAttribute(fused, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-      return e;
-    int per_sm = 0;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fused, kPrepThreads, smem)) != cudaSuccess)
-      return e;
-    if (per_sm >= 1) {
-      uint32_t *flags = reinterpret_cast<uint32_t *>(records + (size_t)items * Rec::BYTES);
-      if ((e = cudaMemsetAsync(flags, 0, (size_t)items * 4, stream)) != cudaSuccess) return e;
-      FwdParams pp = p;
-      void *args[] = {&pp, &records, &maps, &flags, &nchain};
-      return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(fused), dim3(sms),
-                                         dim3(kPrepThreads), args, (size_t)smem, stream);
-    }
+  if (nch >= kFusedMinChunks) {
+    // few long sequences: chains and prep in one cooperative launch (tc_fused_kernel), with
+    // 32-column value slices while their chains take at most half the SMs, else 64-column
+    // slices while theirs take at most a third
+    const int bh = p.B * p.H;
+    bool launched = false;
+    if (bh * (p.dv / 32) * 2 <= sms)
+      e = launch_fused<32>(p, records, maps, sms, items, stream, &launched);
+    else if (bh * (p.dv / NV) * 3 <= sms)
+      e = launch_fused<NV>(p, records, maps, sms, items, stream, &launched);
+    if (e != cudaSuccess || launched) return e;
   }
   prep<<<min(items, sms), kPrepThreads, PrepSmem::ALLOC, stream>>>(p, records, maps);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -282,6 +282,20 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// The same for a 64-byte-swizzled operand (layout type 4): one 32-column atom per row.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (4ull << 61);
+}
+
+// Byte offset of element (row, col < 32) in a bf16 tile stored row-major in 64-byte
+// swizzled atoms (512-byte aligned): 64 bytes per row, 16-byte chunks XOR-permuted by
+// (row >> 1) & 3.  As an MN-major operand (row = K index, col = M/N index) its stride
+// byte offset is 512 (eight rows).
+__host__ __device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t col) {
+  return row * 64u + ((((col >> 3) ^ ((row >> 1) & 3u))) << 4) + (col & 7u) * 2u;
+}
+
 // Byte offset of element (row, col) in a bf16 tile stored row-major in 128-byte
 // swizzled atoms: each row holds 64 columns per atom (128 B), 16-byte chunks are
 // XOR-permuted by (row & 7), and 64-column blocks are `block_stride` bytes apart.

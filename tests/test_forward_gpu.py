@@ -169,13 +169,14 @@ def test_tc_full_size_gdn2(path):
     check_parity(S, S_ref, (0, 1), TOL["bf16"], f"tc-{path} gdn2_bf16 S_T")
 
 
-@pytest.mark.parametrize("form", ["gdn2", "gla"])
-def test_tc_long_sequences_one_launch(form):
-    """Few long sequences (here 2 heads x 41 chunks): prep and chain CTAs share one
+@pytest.mark.parametrize("form,H", [("gdn2", 2), ("gla", 2), ("gdn2", 20)])
+def test_tc_long_sequences_one_launch(form, H):
+    """Few long sequences (here 2 or 20 heads x 41 chunks): prep and chain CTAs share one
     cooperative launch, the chain CTAs fetching each record once a prep CTA has published
-    it.  Against the oracle, with a ragged tail and an initial state; bit-identical on a
-    second call."""
-    w = small(form, "bf16", dk=128, dv=128, T=64 * 40 + 17, B=1, H=2, chunk=64)
+    it.  Two heads run 32-column value slices (8 chains), twenty heads 64-column slices
+    (40 chains: 32-column ones would take more than half the SMs).  Against the oracle,
+    with a ragged tail and an initial state; bit-identical on a second call."""
+    w = small(form, "bf16", dk=128, dv=128, T=64 * 40 + 17, B=1, H=H, chunk=64)
     inp = synth.forward_inputs(w)
     inp["S0"] = synth.round_f32(np.random.default_rng(12).normal(0, 0.5, (w.B, w.H, 128, 128)))
     o, S = gpu_forward(w, inp, algo="tc")
