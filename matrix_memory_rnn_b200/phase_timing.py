@@ -185,7 +185,7 @@ def measure_muir(batch=4, calls=3):
         gdr._lib = saved
     nch = (w.T + 63) // 64
     return {"w": w, "calls": calls, "threads": list(threads), "cycles": list(cycles),
-            "prep_chunks": w.B * w.H * nch * calls, "chain_chunks": w.B * w.H * (w.dv // 64) * nch * calls}
+            "prep_chunks": w.B * w.H * nch * calls, "chain_chunks": threads[0] * nch}
 
 
 def measure(batch=1, calls=3, lib=None, preset="gdn2_bf16"):
@@ -234,8 +234,10 @@ def measure(batch=1, calls=3, lib=None, preset="gdn2_bf16"):
         os.environ.pop("GDR_TIMING_MMA", None)
     out["union"] = union
     nch = (w.T + 63) // 64
-    out.update({"prep_chunks": w.B * w.H * nch * calls,    # each recorder sees every chunk
-                "chain_chunks": w.B * w.H * (w.dv // 64) * nch * calls,
+    # each prep recorder sees every chunk; each chain CTA's recorder the chunks of its sequence
+    # (the chain CTAs per call depend on the value-slice width the launch chose)
+    out.update({"prep_chunks": w.B * w.H * nch * calls,
+                "chain_chunks": out["threads"][0] * nch,
                 "mma_cycles": list(mma_cycles), "mma_groups": list(mma_groups)})
     return out
 
@@ -343,7 +345,9 @@ def measure_mlstm(batch=4, calls=3):
 
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
-    ap.add_argument("--batch", type=int, default=4, help="B of the GDN-2 bf16 workload (H=16, T=4096)")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="B of the workload (default: 4 for the H=16, T=4096 shapes, the preset's own B "
+                         "for --preset gdn2_long)")
     ap.add_argument("--calls", type=int, default=3, help="timed forward calls after one warm-up call")
     ap.add_argument("--peak-tflops", type=float, default=None,
                     help="bf16 dense peak of the whole GPU (default: MEASURED_PEAKS.json's, else 1590)")
@@ -358,10 +362,12 @@ def main(argv=None) -> int:
     ap.add_argument("--mlstm", action="store_true",
                     help="the mLSTM cell's tensor-core kernel instead of the forward")
     args = ap.parse_args(argv)
+    batch = args.batch if args.batch is not None else (
+        synth.PRESETS[args.preset].B if args.preset == "gdn2_long" and not (args.muir or args.mlstm) else 4)
 
     if args.mlstm:
-        per = measure_mlstm(args.batch, args.calls)
-        print(f"mlstm_tc_kernel, bf16, B={args.batch}, H=16, T=4096, d=128: cycles per chunk")
+        per = measure_mlstm(batch, args.calls)
+        print(f"mlstm_tc_kernel, bf16, B={batch}, H=16, T=4096, d=128: cycles per chunk")
         for r, (who, phases) in enumerate(MLSTM_PHASES.items()):
             print(f"\n{who}")
             for i, label in phases:
@@ -376,8 +382,8 @@ def main(argv=None) -> int:
             print(f"  {label:55s} {per[i]:9.0f}")
         print(f"  {'sum':55s} {sum(per[i] for i, _ in GENERAL_PHASES):9.0f}")
         return 0
-    m = (measure_muir(args.batch, args.calls) if args.muir
-         else measure(args.batch, args.calls, preset=args.preset))
+    m = (measure_muir(batch, args.calls) if args.muir
+         else measure(batch, args.calls, preset=args.preset))
     w = m["w"]
     print(f"{'Muir mixer (fused) on ' if args.muir else ''}GDN-2 bf16, B={w.B}, H={w.H}, T={w.T}, d=128, C=64; {args.calls} calls; "
           f"recording threads: prep {m['threads'][1]}, chain {m['threads'][0]}")
