@@ -893,9 +893,10 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 // Warp 0 issues the MMAs (lane 0, from converged code); warp 1 refills the record
 // ring (three records for NV = 32 and 64, two for NV = 128, the size shared memory
 // allows) as soon as MMA4 has released a buffer.  Threads: 32 value columns each (NV = 32
-// runs 128 threads, 128 runs 512).  NV = 32 (few long sequences: twice the chains, half
-// the vector work per step) keeps S0's bf16 copy and V~ in the 64-byte swizzle, whose atom
-// is the slice's 32 columns, and fetches the whole 64-column block of U that holds them.
+// runs 128 threads, 128 runs 512).  NV = 32 (few long sequences: twice the chains, each
+// CTA with half the threads and N = 32 products) keeps S0's bf16 copy and V~ in the
+// 64-byte swizzle, whose atom is the slice's 32 columns, and fetches the whole 64-column
+// block of U that holds them.
 template <int NV>
 struct ChainSmem {
   // per buffer: QY | KT | MM | U block(s) (C x UB) | pi.  The U block sits directly after
