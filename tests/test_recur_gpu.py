@@ -52,3 +52,17 @@ def test_small_rwkv7_fp32_workload_full_size():
     o_ref, S_ref = oracle_forward(w, inp)
     check_parity(o, o_ref, (0, 2), TOL_FP32_KERNEL, "rwkv7_f32 auto o")
     check_parity(S, S_ref, (0, 1), TOL_FP32_KERNEL, "rwkv7_f32 auto S")
+
+
+@pytest.mark.parametrize("form", FORMS)
+def test_recurrent_long_d128(form):
+    """d_k = d_v = 128 over 1001 tokens (125 staging blocks and a one-token tail), fp32 inputs
+    through algo auto, from a nonzero state: the per-step rounding of the fp32 state stays
+    at the fp32 bar over the whole sequence."""
+    w = small(form, "f32", dk=128, dv=128, T=1001, B=1, H=3, chunk=64, seed=77)
+    inp = synth.forward_inputs(w)
+    inp["S0"] = synth.round_f32(np.random.default_rng(5).normal(0.0, 0.5, (w.B, w.H, 128, 128)))
+    o, S = gpu_forward(w, inp, algo="auto")
+    o_ref, S_ref = oracle_forward(w, inp)
+    check_parity(o, o_ref, (0, 2), TOL_FP32_KERNEL, f"recurrent long {form} o")
+    check_parity(S, S_ref, (0, 1), TOL_FP32_KERNEL, f"recurrent long {form} S")
