@@ -615,20 +615,26 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
     // Muir: q^ = gamma_stat 2 sigmoid(z_q) l2norm(silu(q)) in place in chunk jq's q tile,
     // once its tiles have landed; then the front group may form Q f from it.  The back
     // group does this for chunk j + 2 after its own chunk j, in time it would otherwise
-    // spend waiting for the front group.  Returns false when the CTA aborts.
-    auto activate_q = [&](int jq) -> bool {
-      const int bq = jq & 1;
-      if (!group_wait<BackSync>(bfull + bq, (jq >> 1) & 1, sabort, poller)) return false;
+    // spend waiting for the front group.  Its z_q rows are read from global memory by
+    // prefetch_q as soon as the chunk's tiles are requested, so that their latency
+    // overlaps the U/Y readout instead of following the wait for the tiles.  Returns
+    // false when the CTA aborts.
+    uint4 zq_raw[4];
+    auto prefetch_q = [&](int jq) {
       const int g = gt & 15, tb = gt >> 4, j0 = 8 * g;
       const int it = item_of(jq), bh = bh_of(it), hh = bh % H, t0 = c_of(it) * kC;
-      uint4 zq_raw[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int tt = t0 + 4 * tb + i;
         zq_raw[i] = tt < T ? ld16(gzq + (((size_t)(bh / H) * T + tt) * H + hh) * kDK + j0)
                            : make_uint4(0u, 0u, 0u, 0u);
       }
-      float gs8[8];
+    };
+    auto activate_q = [&](int jq) -> bool {
+      const int bq = jq & 1;
+      const int g = gt & 15, tb = gt >> 4, j0 = 8 * g;
+      const int it = item_of(jq), bh = bh_of(it), hh = bh % H;
+      float gs8[8];    // the head's static gain, requested before the wait for the tiles
       if (p.gamma_stat) {
         const float4 a = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0));
         const float4 c = __ldg(reinterpret_cast<const float4 *>(p.gamma_stat + hh * kDK + j0 + 4));
@@ -638,6 +644,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
 #pragma unroll
         for (int e = 0; e < 8; ++e) gs8[e] = 1.f;
       }
+      if (!group_wait<BackSync>(bfull + bq, (jq >> 1) & 1, sabort, poller)) return false;
       uint8_t *qb = smem + bq * SL::BUF;
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -660,7 +667,10 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
     };
     bool live = true;
     if constexpr (kMuir)
-      for (int jq = 0; jq < 2 && jq < nloc && live; ++jq) live = activate_q(jq);
+      for (int jq = 0; jq < 2 && jq < nloc && live; ++jq) {
+        prefetch_q(jq);
+        live = activate_q(jq);
+      }
     for (int j = 0; j < nloc && live; ++j) {
       const int item = item_of(j), c = c_of(item), bh = bh_of(item), h = bh % H, b = bh / H;
       const int t0 = c * kC, n = min(kC, T - t0), bi = j & 1;
@@ -809,6 +819,8 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
         load_tiles(buf, maps, bfull + bi, bhn / H, bhn % H, cn * kC, has_b);
         cnt[kBIss0 + bi] += 1;
       }
+      if constexpr (kMuir)
+        if (j + 2 < nloc) prefetch_q(j + 2);
 
       // ---- U and Y (x alpha_1) -> bf16 record tiles.  M = 64 accumulators: row
       //      16 qd + r in TMEM lane 32 qd + r.  Warp (qd, cpart) reads U (cpart 0) or
