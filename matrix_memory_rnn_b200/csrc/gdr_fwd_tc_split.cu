@@ -148,7 +148,7 @@ struct PrepMisc {             // byte offsets inside PrepSmem::MISC
   static constexpr uint32_t BAR2 = 72;      // uint64_t     MMA2 done
   static constexpr uint32_t SLOT = 80;      // uint32_t     TMEM base
   static constexpr uint32_t ABORT = 84;     // int          a bounded wait ran out
-  static constexpr uint32_t EXACT = 88;     // int [2]      the buffer's chunk takes the exact path
+  static constexpr uint32_t EXACT = 112;    // int [4]      chunk j takes the exact path (entry j & 3)
   static constexpr uint32_t QREADY = 96;    // uint64_t [2] Muir: back -> front: the q tile activated
   static constexpr uint32_t CNT = 128;      // uint32_t [16] issued / completed counts (drain)
   static constexpr uint32_t TBAR = 192;     // uint64_t [2] timing build: MMA1 / MMA2 group timing
@@ -331,6 +331,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
       mbar_init(qready + i, 1);
       mbar_init(bar1 + i, 1);
       sexact[i] = 0;
+      sexact[i + 2] = 0;
     }
     mbar_init(lfull, 1);
     mbar_init(bar2, 1);
@@ -374,16 +375,17 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
       // Muir: the head's a_log, loaded now so that its latency overlaps the waits
       const float a_log = kMuir ? __ldg(p.a_log + bh_of(item) % H) : 0.f;
 
-      // chunk j's log w, tiles and write gate have landed (Muir: and the back group has
-      // activated its q tile)
-      if (poller) sexact[bi] = 0;
+      // chunk j's log w, tiles and write gate have landed.  Muir: the scan (softplus of
+      // z_f) needs only the log-w staging, so the tiles and the back group's activation of
+      // the q tile are waited for after it, while it runs.  The exact-path flag and a1s
+      // are per chunk (entry j & 3): the back group is done with chunk j - 4's by now.
+      if (poller) sexact[j & 3] = 0;
       if (!group_wait<FrontSync>(lfull, j & 1, sabort, poller)) break;
-      if (!group_wait<FrontSync>(bfull + bi, (j >> 1) & 1, sabort, poller)) break;
+      if (!kMuir && !group_wait<FrontSync>(bfull + bi, (j >> 1) & 1, sabort, poller)) break;
       if (wg_front && !group_wait<FrontSync>(wfull + bi, (j >> 1) & 1, sabort, poller)) break;
-      if (kMuir && !group_wait<FrontSync>(qready + bi, (j >> 1) & 1, sabort, poller)) break;
       if (poller) {
         cnt[kLDone] = j + 1;
-        cnt[kBDone0 + bi] += 1;
+        if (!kMuir) cnt[kBDone0 + bi] += 1;
         if (wg_front) cnt[kWDone0 + bi] += 1;
       }
       GDR_PREP_PHASE(1);
@@ -477,7 +479,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
           ed[e] = __expf(dn[e]);
           over |= dn[e] < -kMaxChunkDecay;
         }
-        if (over) sexact[bi] = 1;
+        if (over) sexact[j & 3] = 1;
         if (tb == 0) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -487,7 +489,12 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
         }
       }
       FrontSync::sync();
-      const bool exact = sexact[bi] != 0;
+      if constexpr (kMuir) {
+        if (!group_wait<FrontSync>(bfull + bi, (j >> 1) & 1, sabort, poller)) break;
+        if (!group_wait<FrontSync>(qready + bi, (j >> 1) & 1, sabort, poller)) break;
+        if (poller) cnt[kBDone0 + bi] += 1;
+      }
+      const bool exact = sexact[j & 3] != 0;
       GDR_PREP_PHASE(2);
 
       // ---- operand tiles, in place: k -> K g, b -> K^ f, q -> Q f; Q_pi, K~ to the
@@ -703,7 +710,7 @@ __device__ __forceinline__ void prep_body(const FwdParams &p, uint8_t *records, 
       if (!group_wait<BackSync>(bar1 + bi, (j >> 1) & 1, sabort, poller)) break;
       if (poller) cnt[kM1Done0 + bi] += 1;
       tc_fence_after();
-      const bool exact = sexact[bi] != 0;
+      const bool exact = sexact[j & 3] != 0;
       GDR_PREP_PHASE(9);
 
       // ---- L (fp32, strictly lower; over the dead K g tile) and M (bf16 -> record)
