@@ -93,10 +93,10 @@ def fwd_flops(w) -> int:
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum from one ncu capture of the
 # current kernels on a half-size case, scaled by the units processed).  Forward: prep +
 # chain, per (b, h, 64-token chunk) of the GDN-2 bf16 d = 128 tensor-core path (B = 2, 2048
-# chunks: prep 235.0 MB read + 107.1 MB written, chain 152.1 MB read + 37.0 MB written);
+# chunks: prep 235.0 MB read + 109.9 MB written, chain 152.1 MB read + 38.7 MB written);
 # decode: per (b, h) step of the d = 128 persistent kernel.  Must be re-measured when those
 # kernels change.
-FWD_TC_TRAFFIC_PER_CHUNK = (234995968 + 107078400 + 152093952 + 36988416) / 2048
+FWD_TC_TRAFFIC_PER_CHUNK = (235030528 + 109881344 + 152095488 + 38657536) / 2048
 DEC_TRAFFIC_PER_HEAD = (137.9e6 + 81.0e6) / (64 * 32)
 
 
